@@ -1,0 +1,303 @@
+"""fp64 CPU oracle for the causal delta rule (DeltaNet, Gated DeltaNet, KDA).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product path (the CUDA library and its Python binding) never imports, links
+or calls anything here, and this package imports nothing from the product.
+
+Contents
+--------
+``delta_rule``            sequential recurrence in fp64 (C, ``dn_oracle.c``),
+                          error form or transition-then-write form.
+``additive``              additive (Hebbian) linear attention (C).
+``brute_force``           explicit expansion with d_k x d_k products, T <= 16.
+``chunked``               fp64 restatement of the chunkwise (UT transform)
+                          equations, used only to check the chunk algebra
+                          against the sequential recurrence.
+``wy_transition``         the WY form of one chunk's product of transitions.
+
+Every function takes and returns numpy arrays.  Layouts: tokens
+``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
+``[B, H, T, d_k]``, states ``[B, H, d_k, d_v]`` (row i = key channel).
+The gate argument ``g`` is the log-decay; the decay is ``exp(g)``.
+
+Pins: see ``tests/test_oracle_pins.py``.  Parity status of each function is
+listed there; the delta-rule columns of the 64x64 associative-recall table in
+"Linear attention and Gated DeltaNet" (ch. 28, "The state is an associative
+memory") are parity unpinned (the page does not state beta), every other
+function here is pinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+GATE_NONE, GATE_SCALAR, GATE_PER_KEY = 0, 1, 2
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        L = ctypes.c_long
+        for name in ("dno_delta_error_form", "dno_delta_transition_form"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, dp, dp, dp,
+                           L, L, L, L, L, ctypes.c_double, ctypes.c_int]
+        lib.dno_additive.restype = ctypes.c_int
+        lib.dno_additive.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, L,
+                                     ctypes.c_double, ctypes.c_int]
+        lib.dno_max_threads.restype = ctypes.c_int
+        lib.dno_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    """Threads the C oracle uses when ``nthreads=0`` (OpenMP default)."""
+    return int(_load().dno_max_threads())
+
+
+def _f64(x):
+    if x is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    return a
+
+
+def _ptr(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def gate_kind(g, k) -> int:
+    """Infer the gate from the shape of ``g``: None, [B,H,T] or [B,H,T,d_k]."""
+    if g is None:
+        return GATE_NONE
+    g = np.asarray(g)
+    if g.shape == np.asarray(k).shape[:-1]:
+        return GATE_SCALAR
+    if g.shape == np.asarray(k).shape:
+        return GATE_PER_KEY
+    raise ValueError(f"gate shape {g.shape} matches neither [B,H,T] nor [B,H,T,d_k]")
+
+
+def delta_rule(q, k, v, beta, g=None, S0=None, scale=1.0, form="error",
+               nthreads=0):
+    """Run the delta rule token by token in fp64; return ``(o, S_T)``.
+
+    ``form="error"``: forget, predict, correct, write, read ("Linear attention
+    and Gated DeltaNet", ch. 28, "Gated DeltaNet" and "The recurrent form";
+    KDA per "A walk through of the DeltaNet family", its KDA update).
+    ``form="transition"``: ``S = (I - beta k k^T) Diag(alpha) S + beta k v^T``
+    with an explicit d_k x d_k matrix (D2L 12.5, "One rule, two readings",
+    matrix form; "Gating: the modern cell").
+    """
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    gate = gate_kind(g, k)
+    g = _f64(g)
+    S0 = _f64(S0)
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape[:3] == (B, H, T) and beta.shape == (B, H, T)
+    if S0 is not None:
+        assert S0.shape == (B, H, dk, dv)
+    o = np.empty((B, H, T, dv), np.float64)
+    ST = np.empty((B, H, dk, dv), np.float64)
+    fn = {"error": _load().dno_delta_error_form,
+          "transition": _load().dno_delta_transition_form}[form]
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), gate, _ptr(S0),
+            _ptr(o), _ptr(ST), B, H, T, dk, dv, float(scale), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return o, ST
+
+
+def additive(q, k, v, S0=None, scale=1.0, nthreads=0):
+    """Additive linear attention ``S += k v^T``, ``o = S^T (scale q)`` in fp64
+    ("Linear attention and Gated DeltaNet", ch. 28, "Removing the softmax")."""
+    q, k, v, S0 = _f64(q), _f64(k), _f64(v), _f64(S0)
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    o = np.empty((B, H, T, dv), np.float64)
+    ST = np.empty((B, H, dk, dv), np.float64)
+    rc = _load().dno_additive(_ptr(q), _ptr(k), _ptr(v), _ptr(S0), _ptr(o),
+                              _ptr(ST), B, H, T, dk, dv, float(scale),
+                              int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return o, ST
+
+
+# ---------------------------------------------------------------------------
+# numpy restatements (fp64), written from the displayed equations
+# ---------------------------------------------------------------------------
+
+def _decay_vectors(g, k):
+    """Per-token, per-key-channel log-decay ``[B,H,T,d_k]``: zeros without a
+    gate, the scalar broadcast over channels for Gated DeltaNet, itself for
+    KDA.  With identical channels the per-key formulas below are exactly the
+    scalar ones."""
+    k = np.asarray(k)
+    gate = gate_kind(g, k)
+    if gate == GATE_NONE:
+        return np.zeros(k.shape, np.float64)
+    g = np.asarray(g, np.float64)
+    if gate == GATE_SCALAR:
+        return np.broadcast_to(g[..., None], k.shape).astype(np.float64)
+    return g.copy()
+
+
+def transition_matrix(k_t, beta_t, logdecay_t):
+    """``M_t = (I - beta_t k_t k_t^T) Diag(exp(logdecay_t))`` (d_k x d_k): the
+    per-token transition of the delta rule, forget first (D2L 12.5, "Gating:
+    the modern cell"; KDA order per "A walk through of the DeltaNet family")."""
+    k_t = np.asarray(k_t, np.float64)
+    dk = k_t.shape[0]
+    return (np.eye(dk) - beta_t * np.outer(k_t, k_t)) * np.exp(logdecay_t)[None, :]
+
+
+def brute_force(q, k, v, beta, g=None, S0=None, scale=1.0):
+    """Explicit expansion, no recursion on S (T <= 16):
+
+        S_t = (M_t ... M_1) S_0 + sum_{j<=t} (M_t ... M_{j+1}) beta_j k_j v_j^T
+        o_t = S_t^T (scale q_t)
+
+    Every product is formed afresh from the transition matrices."""
+    q, k, v, beta = (np.asarray(x, np.float64) for x in (q, k, v, beta))
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    if T > 16:
+        raise ValueError("brute force expansion is for T <= 16")
+    lg = _decay_vectors(g, k)
+    S0 = np.zeros((B, H, dk, dv)) if S0 is None else np.asarray(S0, np.float64)
+    o = np.empty((B, H, T, dv))
+    ST = np.empty((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            Ms = [transition_matrix(k[b, h, t], beta[b, h, t], lg[b, h, t]) for t in range(T)]
+
+            def prod(hi, lo):  # M_hi ... M_lo  (1-based, inclusive); identity if lo > hi
+                P = np.eye(dk)
+                for s in range(lo, hi + 1):
+                    P = Ms[s - 1] @ P
+                return P
+
+            for t in range(1, T + 1):
+                S = prod(t, 1) @ S0[b, h]
+                for j in range(1, t + 1):
+                    S = S + prod(t, j + 1) @ (beta[b, h, j - 1] * np.outer(k[b, h, j - 1], v[b, h, j - 1]))
+                o[b, h, t - 1] = S.T @ (scale * q[b, h, t - 1])
+                if t == T:
+                    ST[b, h] = S
+            if T == 0:
+                ST[b, h] = S0[b, h]
+    return o, ST
+
+
+def _strict_lower(m):
+    """Entries strictly below the diagonal (the chunk system's coupling)."""
+    return np.tril(m, -1)
+
+
+def _lower(m):
+    """Entries on and below the diagonal (causal mask, diagonal kept)."""
+    return np.tril(m, 0)
+
+
+def _solve_unit_lower(L, rhs):
+    """Solve ``L X = rhs`` for unit lower-triangular L (a library routine)."""
+    from scipy.linalg import solve_triangular
+    return solve_triangular(L, rhs, lower=True, unit_diagonal=True)
+
+
+def chunked(q, k, v, beta, g=None, S0=None, scale=1.0, chunk=64):
+    """Chunkwise form in fp64, from the displayed equations of "Linear
+    attention and Gated DeltaNet" (ch. 28, "The chunked form: recurrence as
+    matrix multiplication"), extended to a per-key decay.
+
+    The sequence is zero-padded to a multiple of ``chunk`` (q, k, v rows zero,
+    beta = 0 and log-decay 0, i.e. identity steps) and split into chunks.
+    Inside a chunk, with Gamma_i = sum_{m<=i} g_m (per key channel),
+    kd_ij = sum_c k_ic k_jc exp(Gamma_ic - Gamma_jc) and
+    qd_ij = sum_c q_ic k_jc exp(Gamma_ic - Gamma_jc) for j <= i:
+
+        (I + strict_tril(beta_i kd_ij)) U = beta V - beta (K * e^Gamma) S_0
+        O     = (Q * e^Gamma) S_0 + tril(qd) U
+        S_end = Diag(e^Gamma_C) S_0 + (K * e^(Gamma_C - Gamma))^T U
+
+    With one decay shared by every channel these are the page's equations
+    with D_ij = exp(G_i - G_j).  ``scale`` multiplies q before anything else.
+    """
+    q, k, v, beta = (np.asarray(x, np.float64) for x in (q, k, v, beta))
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    lg = _decay_vectors(g, k)
+    q = q * scale
+    C = int(chunk)
+    pad = (-T) % C
+    if pad:
+        q = np.concatenate([q, np.zeros((B, H, pad, dk))], axis=2)
+        k = np.concatenate([k, np.zeros((B, H, pad, dk))], axis=2)
+        v = np.concatenate([v, np.zeros((B, H, pad, dv))], axis=2)
+        beta = np.concatenate([beta, np.zeros((B, H, pad))], axis=2)
+        lg = np.concatenate([lg, np.zeros((B, H, pad, dk))], axis=2)
+    n = (T + pad) // C
+    S_all = np.zeros((B, H, dk, dv)) if S0 is None else np.array(S0, np.float64)
+    out = np.zeros((B, H, T + pad, dv))
+    for b in range(B):
+        for h in range(H):
+            S = S_all[b, h].copy()
+            for c in range(n):
+                sl = slice(c * C, (c + 1) * C)
+                Qc, Kc, Vc = q[b, h, sl], k[b, h, sl], v[b, h, sl]
+                bc = beta[b, h, sl]
+                Gam = np.cumsum(lg[b, h, sl], axis=0)            # [C, dk], inclusive
+                # pairwise decayed products, j <= i only (upper part is masked)
+                diff = Gam[:, None, :] - Gam[None, :, :]          # [i, j, c]
+                causal = np.tril(np.ones((C, C), bool))
+                Dp = np.where(causal[..., None], np.exp(np.where(causal[..., None], diff, 0.0)), 0.0)
+                kd = np.einsum("ic,jc,ijc->ij", Kc, Kc, Dp)
+                qd = np.einsum("ic,jc,ijc->ij", Qc, Kc, Dp)
+                system = np.eye(C) + _strict_lower(bc[:, None] * kd)
+                rhs = bc[:, None] * Vc - bc[:, None] * ((Kc * np.exp(Gam)) @ S)
+                U = _solve_unit_lower(system, rhs)
+                out[b, h, sl] = (Qc * np.exp(Gam)) @ S + _lower(qd) @ U
+                tail = np.exp(Gam[-1][None, :] - Gam)             # [C, dk]
+                S = np.exp(Gam[-1])[:, None] * S + (Kc * tail).T @ U
+            S_all[b, h] = S
+    return out[:, :, :T], S_all
+
+
+def wy_transition(k, beta, g=None):
+    """Product of one chunk's transitions ``M_C ... M_1`` in WY form:
+
+        Diag(e^Gamma_C) - (K * e^(Gamma_C - Gamma))^T W,
+        W = (I + strict_tril(beta_i kd_ij))^{-1} (beta * K * e^Gamma)
+
+    for a single chunk: ``k [C, d_k]``, ``beta [C]``, ``g`` None, ``[C]`` or
+    ``[C, d_k]`` (D2L 12.5, "Training it: the WY trick"; ch. 28's chunk
+    system, whose S_0-dependent part this is)."""
+    k = np.asarray(k, np.float64)
+    beta = np.asarray(beta, np.float64)
+    C, dk = k.shape
+    lg = _decay_vectors(None if g is None else np.asarray(g)[None, None],
+                        k[None, None])[0, 0]
+    Gam = np.cumsum(lg, axis=0)
+    kd = np.zeros((C, C))
+    for i in range(C):
+        for j in range(i + 1):
+            kd[i, j] = np.sum(k[i] * k[j] * np.exp(Gam[i] - Gam[j]))
+    system = np.eye(C) + _strict_lower(beta[:, None] * kd)
+    W = _solve_unit_lower(system, beta[:, None] * k * np.exp(Gam))
+    return np.diag(np.exp(Gam[-1])) - (k * np.exp(Gam[-1][None, :] - Gam)).T @ W

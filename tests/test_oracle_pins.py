@@ -1,0 +1,366 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test names the passage it follows.  Parity status per oracle function:
+
+* ``delta_rule`` (error form)       pinned: worked example, exact recall,
+  overwrite recall, reflection parity, closed forms, brute force.
+* ``delta_rule`` (transition form)  pinned: agrees with the error form, and
+  both with the brute-force expansion.
+* ``additive``                      pinned: associative-recall table (additive
+  column), overwrite recall at R = 1.
+* ``brute_force``                   pinned: worked example, closed forms.
+* ``chunked``                       pinned: equals the recurrence at T = 37 for
+  chunk sizes 1, 5, 8, 16, 64 with S0 != 0, for all three gates; a planted
+  wrong triangle is caught.
+* ``wy_transition``                 pinned: equals the explicit product of the
+  chunk's transition matrices.
+* delta-rule columns of the associative-recall table: parity unpinned (the page
+  does not state beta); computed here as context only.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def rand_problem(rng, B, H, T, dk, dv, gate, s0=True, beta_range=(0.05, 1.0)):
+    q = rng.standard_normal((B, H, T, dk))
+    k = rng.standard_normal((B, H, T, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, H, T, dv))
+    beta = rng.uniform(*beta_range, size=(B, H, T))
+    g = None
+    if gate == "scalar":
+        g = -rng.uniform(0.0, 0.7, size=(B, H, T))
+    elif gate == "per_key":
+        g = -rng.uniform(0.0, 0.7, size=(B, H, T, dk))
+    S0 = rng.standard_normal((B, H, dk, dv)) * 0.5 if s0 else None
+    return q, k, v, beta, g, S0
+
+
+def rel(a, b):
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-300))
+
+
+# --- ch. 28, "Correct: the delta rule": the worked example ---------------------
+
+def _worked(d):
+    w = gold("worked_example.json")
+    k = np.zeros(d); k[: 2] = w["k"]
+    q = np.zeros(d); q[: 2] = w["q"]
+    v = np.zeros(d); v[: 2] = w["v"]
+    betas = [s["beta"] for s in w["steps"]]
+    T = len(betas)
+    shp = (1, 1, T, d)
+    Q = np.broadcast_to(q, shp).copy()
+    K = np.broadcast_to(k, shp).copy()
+    V = np.broadcast_to(v, shp).copy()
+    beta = np.array(betas).reshape(1, 1, T)
+    return w, Q, K, V, beta
+
+
+@pytest.mark.parametrize("d", [2, 64])
+def test_worked_example_exact(d):
+    w, Q, K, V, beta = _worked(d)
+    for form in ("error", "transition"):
+        o, S = oracle.delta_rule(Q, K, V, beta, form=form)
+        # after both steps: row 0 of the state is exactly v
+        assert S[0, 0, 0, :2].tolist() == w["steps"][-1]["state_row0"]
+        assert np.all(S[0, 0, 1:] == 0) and np.all(S[0, 0, 0, 2:] == 0)
+        for t, st in enumerate(w["steps"]):
+            assert o[0, 0, t, :2].tolist() == st["output"], (form, t)
+            assert np.all(o[0, 0, t, 2:] == 0)
+    # the state after the first step alone
+    o1, S1 = oracle.delta_rule(Q[:, :, :1], K[:, :, :1], V[:, :, :1], beta[:, :, :1])
+    assert S1[0, 0, 0, :2].tolist() == w["steps"][0]["state_row0"]
+    ob, Sb = oracle.brute_force(Q, K, V, beta)
+    assert ob[0, 0, :, :2].tolist() == [s["output"] for s in w["steps"]]
+
+
+# --- ch. 28, "Correct: the delta rule": beta = 1 and a unit key replace the value
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_exact_single_key_recall(gate):
+    rng = np.random.default_rng(11)
+    dk, dv, T = 16, 12, 9
+    q, k, v, beta, g, S0 = rand_problem(rng, 1, 1, T, dk, dv, gate)
+    # keys exactly unit in fp64: basis vectors and a 3-4-5 rational vector
+    ks = np.zeros((T, dk))
+    for t in range(T):
+        if t % 2 == 0:
+            ks[t, t % dk] = 1.0
+        else:
+            ks[t, t % dk] = 0.6
+            ks[t, (t + 3) % dk] = 0.8
+    k[0, 0] = ks
+    beta[:] = 1.0
+    # read with q = k: o_t = S_t^T k_t must equal v_t
+    o, _ = oracle.delta_rule(k, k, v, beta, g, S0)
+    assert rel(o, v) <= 1e-12
+
+
+# --- D2L 12.5, "Overwriting, measured" ------------------------------------------
+
+def overwrite_recall(rule, R, trials=100, seed=0, d=64, n_keys=8):
+    rng = np.random.default_rng(seed + 1000 * R)
+    correct = 0
+    for _ in range(trials):
+        Qm, _ = np.linalg.qr(rng.standard_normal((d, d)))
+        keys = Qm[:, :n_keys].T                       # 8 orthonormal keys
+        vals = rng.standard_normal((n_keys, R, d))
+        order = rng.permutation([(i, r) for i in range(n_keys) for r in range(R)])
+        # R re-bindings per key, in a shuffled order; the value index r is just a label
+        seq_k = np.stack([keys[i] for i, r in order])[None, None]
+        seq_v = np.stack([vals[i, r] for i, r in order])[None, None]
+        latest = {}
+        for i, r in order:
+            latest[i] = r
+        T = seq_k.shape[2]
+        if rule == "delta":
+            _, S = oracle.delta_rule(seq_k, seq_k, seq_v, np.ones((1, 1, T)))
+        else:
+            _, S = oracle.additive(seq_k, seq_k, seq_v)
+        S = S[0, 0]
+        for i in range(n_keys):
+            read = S.T @ keys[i]
+            cos = vals[i] @ read / (np.linalg.norm(vals[i], axis=1) * max(np.linalg.norm(read), 1e-300))
+            correct += int(np.argmax(cos) == latest[i])
+    return correct / (trials * n_keys)
+
+
+def test_overwrite_recall_table():
+    w = gold("overwrite_recall.json")
+    prev = None
+    for R, want_delta in zip(w["writes_per_key"], w["delta"]):
+        assert overwrite_recall("delta", R) == want_delta == 1.0
+        add = overwrite_recall("additive", R)
+        if R == 1:
+            assert add == 1.0
+        else:
+            assert add < prev
+            assert abs(add - 1.0 / R) <= 0.15
+        prev = add
+
+
+# --- D2L 12.5, "One rule, two readings": error form == transition form -----------
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_error_and_transition_forms_agree(gate):
+    rng = np.random.default_rng(3)
+    q, k, v, beta, g, S0 = rand_problem(rng, 2, 3, 64, 16, 8, gate)
+    o1, S1 = oracle.delta_rule(q, k, v, beta, g, S0, scale=0.7, form="error")
+    o2, S2 = oracle.delta_rule(q, k, v, beta, g, S0, scale=0.7, form="transition")
+    assert rel(o2, o1) <= 1e-12 and rel(S2, S1) <= 1e-12
+
+
+def test_forms_agree_at_page_size():
+    # the slide's case: d_k = d_v = 64, T = 512, unit keys, beta = sigmoid(N(0,1))
+    rng = np.random.default_rng(0)
+    T, d = 512, 64
+    Q = rng.standard_normal((1, 1, T, d))
+    K = rng.standard_normal((1, 1, T, d))
+    K /= np.maximum(np.linalg.norm(K, axis=-1, keepdims=True), 1e-12)
+    V = rng.standard_normal((1, 1, T, d))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((1, 1, T))))
+    y1, _ = oracle.delta_rule(Q, K, V, beta, form="error")
+    y2, _ = oracle.delta_rule(Q, K, V, beta, form="transition")
+    # the page reports 1.38e-06 in fp32 and asserts < 1e-5; fp64 is far tighter
+    assert np.abs(y1 - y2).max() / np.abs(y1).max() < 1e-12
+
+
+# --- explicit expansion on T <= 16 ----------------------------------------------
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_brute_force_matches_recurrence(gate):
+    rng = np.random.default_rng(5)
+    q, k, v, beta, g, S0 = rand_problem(rng, 1, 2, 13, 8, 6, gate)
+    ob, Sb = oracle.brute_force(q, k, v, beta, g, S0, scale=1.3)
+    o, S = oracle.delta_rule(q, k, v, beta, g, S0, scale=1.3)
+    assert rel(o, ob) <= 1e-12 and rel(S, Sb) <= 1e-12
+
+
+# --- special cases with closed forms --------------------------------------------
+
+def test_zero_gate_equals_deltanet_exactly():
+    rng = np.random.default_rng(6)
+    q, k, v, beta, _, S0 = rand_problem(rng, 2, 2, 40, 16, 16, "none")
+    o0, S0_ = oracle.delta_rule(q, k, v, beta, None, S0)
+    o1, S1 = oracle.delta_rule(q, k, v, beta, np.zeros(beta.shape), S0)
+    assert np.array_equal(o0, o1) and np.array_equal(S0_, S1)
+
+
+def test_per_key_with_shared_channels_equals_scalar_gate():
+    rng = np.random.default_rng(7)
+    q, k, v, beta, g, S0 = rand_problem(rng, 2, 2, 40, 16, 16, "scalar")
+    gk = np.repeat(g[..., None], 16, axis=-1)
+    o1, S1 = oracle.delta_rule(q, k, v, beta, g, S0)
+    o2, S2 = oracle.delta_rule(q, k, v, beta, gk, S0)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_beta_zero_is_pure_decay(gate):
+    # beta = 0: o_t = (Diag(e^{Gamma_t}) S0)^T (scale q_t) with Gamma_t the inclusive cumsum
+    rng = np.random.default_rng(8)
+    q, k, v, beta, g, S0 = rand_problem(rng, 1, 2, 20, 8, 8, gate)
+    beta[:] = 0.0
+    o, S = oracle.delta_rule(q, k, v, beta, g, S0, scale=0.5)
+    if g is None:
+        lg = np.zeros(k.shape)
+    elif g.ndim == 3:
+        lg = np.repeat(g[..., None], 8, axis=-1)
+    else:
+        lg = g
+    Gam = np.cumsum(lg, axis=2)
+    want = np.einsum("bhtc,bhcj,bhtc->bhtj", np.exp(Gam), S0, 0.5 * q)
+    assert rel(o, want) <= 1e-12
+    assert rel(S, np.exp(Gam[:, :, -1])[..., None] * S0) <= 1e-12
+
+
+def test_first_token_from_zero_state():
+    # S0 = 0, T = 1: o = beta (scale q . k) v
+    rng = np.random.default_rng(9)
+    q, k, v, beta, g, _ = rand_problem(rng, 3, 2, 1, 16, 8, "scalar", s0=False)
+    o, S = oracle.delta_rule(q, k, v, beta, g, None, scale=0.25)
+    want = beta[..., None] * np.sum(0.25 * q * k, -1)[..., None] * v
+    assert rel(o, want) <= 1e-13
+    assert rel(S, np.einsum("bhc,bhj->bhcj", k[:, :, 0], beta[:, :, 0, None] * v[:, :, 0])) <= 1e-13
+
+
+# --- D2L 12.5, "The reflection hiding in the delta rule" -------------------------
+
+def test_reflection_eigenvalues():
+    w = gold("reflection.json")
+    rng = np.random.default_rng(10)
+    k = rng.standard_normal(16)
+    k /= np.linalg.norm(k)
+    for row in w["eigen"]:
+        M = oracle.transition_matrix(k, row["beta"], np.zeros(16))
+        ev = np.sort(np.linalg.eigvalsh((M + M.T) / 2))
+        assert abs(ev[0] - row["along_k"]) < 1e-12 or abs(ev[-1] - row["along_k"]) < 1e-12
+        others = ev[1:] if abs(ev[0] - row["along_k"]) < 1e-12 else ev[:-1]
+        assert np.allclose(others, row["elsewhere"], atol=1e-12)
+
+
+@pytest.mark.parametrize("T", [8, 24, 64])
+def test_reflection_parity_exact(T):
+    # k = e_1, S0 = e_1 e_1^T, v = 0, beta_t = 2 x_t: o_t[0] = (-1)^(x_1 + ... + x_t)
+    w = gold("reflection.json")
+    rng = np.random.default_rng(T)
+    d = 8
+    x = rng.integers(0, 2, size=T)
+    e1 = np.zeros(d); e1[0] = 1.0
+    K = np.broadcast_to(e1, (1, 1, T, d)).copy()
+    V = np.zeros((1, 1, T, d))
+    S0 = np.zeros((1, 1, d, d)); S0[0, 0, 0, 0] = 1.0
+    beta = (2.0 * x).reshape(1, 1, T)
+    o, _ = oracle.delta_rule(K, K, V, beta, None, S0)
+    want = (-1.0) ** np.cumsum(x)
+    acc = float(np.mean(np.sign(o[0, 0, :, 0]) == want))
+    assert np.array_equal(o[0, 0, :, 0], want)
+    assert acc == w["parity_accuracy_beta2"][str(T)]
+
+
+# --- ch. 28, "The state is an associative memory": additive column ---------------
+
+def test_associative_recall_additive_column():
+    w = gold("associative_recall_64.json")
+    d = w["key_dim"]
+    rng = np.random.default_rng(12)
+    for n, page in zip(w["pairs"], w["additive_error_all"]):
+        errs = []
+        for _ in range(40):
+            K = rng.standard_normal((n, d)); K /= np.linalg.norm(K, axis=1, keepdims=True)
+            V = rng.standard_normal((n, d))
+            _, S = oracle.additive(K[None, None], K[None, None], V[None, None])
+            Rd = K @ S[0, 0]
+            errs.append(np.mean(np.linalg.norm(Rd - V, axis=1) / np.linalg.norm(V, axis=1)))
+        got = float(np.mean(errs))
+        assert abs(got - page) <= 0.10 * page, (n, got, page)
+        # and the closed form of the interference: sqrt((n - 1) / d)
+        assert abs(got - np.sqrt((n - 1) / d)) <= 0.05 * np.sqrt((n - 1) / d)
+
+
+# --- ch. 28, "The chunked form": chunked == recurrent, T = 37, S0 != 0 ------------
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+@pytest.mark.parametrize("chunk", [1, 5, 8, 16, 64])
+def test_chunked_matches_recurrence(gate, chunk):
+    rng = np.random.default_rng(13)
+    q, k, v, beta, g, S0 = rand_problem(rng, 1, 2, 37, 16, 12, gate)
+    o, S = oracle.delta_rule(q, k, v, beta, g, S0, scale=0.8)
+    oc, Sc = oracle.chunked(q, k, v, beta, g, S0, scale=0.8, chunk=chunk)
+    assert rel(oc, o) <= 1e-12 and rel(Sc, S) <= 1e-12
+
+
+def test_planted_wrong_triangle_is_caught(monkeypatch):
+    # ch. 28's note: keeping the wrong triangle of the system passes chunk size 1
+    rng = np.random.default_rng(14)
+    q, k, v, beta, g, S0 = rand_problem(rng, 1, 1, 37, 16, 12, "scalar")
+    o, S = oracle.delta_rule(q, k, v, beta, g, S0)
+    monkeypatch.setattr(oracle, "_strict_lower", lambda m: np.tril(m.T, -1))   # transposed coupling
+    oc1, _ = oracle.chunked(q, k, v, beta, g, S0, chunk=1)
+    oc5, _ = oracle.chunked(q, k, v, beta, g, S0, chunk=5)
+    assert rel(oc1, o) <= 1e-12          # chunk size 1 cannot see the mistake
+    assert rel(oc5, o) > 1e-3            # a non-divisor chunk size does
+
+
+# --- D2L 12.5, "Training it: the WY trick" ---------------------------------------
+
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_wy_transition_equals_explicit_product(gate):
+    rng = np.random.default_rng(15)
+    C, dk = 10, 12
+    _, k, _, beta, g, _ = rand_problem(rng, 1, 1, C, dk, 4, gate)
+    k, beta = k[0, 0], beta[0, 0]
+    gg = None if g is None else g[0, 0]
+    if gg is None:
+        lg = np.zeros((C, dk))
+    elif gg.ndim == 1:
+        lg = np.repeat(gg[:, None], dk, axis=1)
+    else:
+        lg = gg
+    P = np.eye(dk)
+    for t in range(C):
+        P = oracle.transition_matrix(k[t], beta[t], lg[t]) @ P
+    assert rel(oracle.wy_transition(k, beta, gg), P) <= 1e-12
+
+
+# --- resumability: the state is the checkpoint ------------------------------------
+
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_resume_is_exact(gate):
+    rng = np.random.default_rng(16)
+    q, k, v, beta, g, S0 = rand_problem(rng, 2, 2, 50, 16, 16, gate)
+    o, S = oracle.delta_rule(q, k, v, beta, g, S0)
+    sl1, sl2 = slice(0, 23), slice(23, 50)
+    gp = (lambda s: None) if g is None else (lambda s: g[:, :, s])
+    o1, S1 = oracle.delta_rule(q[:, :, sl1], k[:, :, sl1], v[:, :, sl1], beta[:, :, sl1], gp(sl1), S0)
+    o2, S2 = oracle.delta_rule(q[:, :, sl2], k[:, :, sl2], v[:, :, sl2], beta[:, :, sl2], gp(sl2), S1)
+    assert np.array_equal(np.concatenate([o1, o2], axis=2), o) and np.array_equal(S2, S)
+
+
+def test_delta_columns_context_only():
+    """Delta columns of the 64x64 recall table: parity unpinned (beta not
+    stated).  Computed at beta = 1 as context; only sanity-checked: delta's
+    error on the last 8 pairs stays below the additive error."""
+    d, n = 64, 64
+    rng = np.random.default_rng(17)
+    K = rng.standard_normal((n, d)); K /= np.linalg.norm(K, axis=1, keepdims=True)
+    V = rng.standard_normal((n, d))
+    _, S = oracle.delta_rule(K[None, None], K[None, None], V[None, None], np.ones((1, 1, n)))
+    _, Sa = oracle.additive(K[None, None], K[None, None], V[None, None])
+    last = slice(n - 8, n)
+    e_delta = np.mean(np.linalg.norm(K[last] @ S[0, 0] - V[last], axis=1) / np.linalg.norm(V[last], axis=1))
+    e_add = np.mean(np.linalg.norm(K[last] @ Sa[0, 0] - V[last], axis=1) / np.linalg.norm(V[last], axis=1))
+    assert e_delta < e_add
