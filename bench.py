@@ -1,0 +1,460 @@
+#!/usr/bin/env python3
+"""Benchmark of the delta-rule layer: chunked prefill + decode step on B200.
+
+One step = the whole hot path over one batch of synthetic inputs resident in
+HBM:
+  * chunked prefill of a Gated DeltaNet batch: B=4 sequences, H=16 heads,
+    T=4096 tokens, d_k=d_v=128, bf16 q/k/v, fp32 beta/g, chunk 64, returning o
+    and the final fp32 state (dn_chunk_fwd);
+  * one recurrent decode step of a serving batch: B=256 sequences, H=32 heads,
+    d_k=d_v=128, fp32 state resident in HBM and updated in place, one bf16
+    token per sequence (dn_decode_step; token sets cycle through a bank of 16).
+
+value = (prefill tokens + decode tokens) per second = (4*4096 + 256) / step
+time, summed over ranks (each rank runs its own copy of the workload: the
+heads and sequences are independent, so there is no data-path collective).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--path auto|simt|tc] [--no-cpu-baseline] [--no-e2e]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "delta-rule layer prefill tokens/s + decode tokens/s, % of tensor/HBM roofline"
+C = 64
+
+
+def prefill_flops(B, H, T, dk, dv, chunk=C):
+    """Counted FLOPs of the chunked form (each matmul 2mnk, each triangular solve
+    C^2 n, full C x C products): 5 C^2 d_k + 3 C^2 d_v + 6 C d_k d_v per chunk."""
+    n_chunks = B * H * ((T + chunk - 1) // chunk)
+    return n_chunks * (5 * chunk * chunk * dk + 3 * chunk * chunk * dv + 6 * chunk * dk * dv)
+
+
+def prefill_bytes(B, H, T, dk, dv, esz=2, gate_per_key=False, s0=False, st=True):
+    """Algorithmic HBM bytes: q, k, v and o once in their dtype, beta and g fp32
+    once, S0 / S_T fp32 once when present."""
+    tok = B * H * T
+    g = 4 * (dk if gate_per_key else 1)
+    b = tok * (esz * (2 * dk + 2 * dv) + 4 + g)
+    b += (B * H * dk * dv * 4) * (int(s0) + int(st))
+    return b
+
+
+def decode_bytes(B, H, dk, dv, esz=2):
+    """State read + written once (fp32) plus the token vectors and o."""
+    return B * H * (2 * dk * dv * 4 + esz * (2 * dk + 2 * dv) + 8)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def traffic_for(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    has not changed since it was captured (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        ent = tab[kernel_key]
+        src = os.path.join(ROOT, ent["source"])
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != ent["source_sha256"]:
+                return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons, polled through NVML from a
+    background thread for the whole timed region (nvidia-smi as a fallback).
+    The reasons reported are the union over samples."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_id):
+        self.device_id = device_id
+        self.samples = []
+        self._stop = None
+
+    def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            if isinstance(self.device_id, str):
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.device_id)
+            else:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(self.device_id))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            getr = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), getr(h)))
+                    except Exception:
+                        pass
+                    self._stop.wait(0.002)
+            self._thread = threading.Thread(target=poll, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+            self.max_mhz = None
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "source": "nvml"}
+        reasons = sorted({name for _, r in self.samples for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(prefill_heads=64, decode_heads=8192, seed_offset=0):
+    """Time the fp64 oracle on a bounded sample of the same workload and scale
+    to the whole step: returns (tokens/s, seconds per full step, description)."""
+    import numpy as np
+    import oracle
+    from delta_rule_recurrent_02_b200 import workloads as W
+    cfg = W.GDN_PREFILL
+    inp = W.gen_prefill(1, prefill_heads, cfg.T, cfg.dk, cfg.dv, dtype=cfg.dtype, gate=cfg.gate,
+                        seed=cfg.seed + seed_offset, q_norm=True, g_shift=cfg.g_shift)
+    f = lambda t: None if t is None else t.double().numpy()
+    args = [f(inp[n]) for n in ("q", "k", "v", "beta", "g")]
+    t0 = time.perf_counter()
+    oracle.delta_rule(*args, None, scale=cfg.scale)
+    tp = time.perf_counter() - t0
+    dc = W.DECODE
+    dinp = W.gen_decode(dc, B=1, H=decode_heads, bank=1)
+    dargs = [f(dinp[n][0])[:, :, None] for n in ("q", "k", "v")]
+    db = f(dinp["beta"][0])[:, :, None]
+    dg = f(dinp["g"][0])[:, :, None]
+    S = f(dinp["S"])
+    t0 = time.perf_counter()
+    oracle.delta_rule(dargs[0], dargs[1], dargs[2], db, dg, S, scale=dc.scale)
+    td = time.perf_counter() - t0
+    full_p = tp * (cfg.B * cfg.H) / prefill_heads
+    full_d = td * (dc.B * dc.H) / decode_heads
+    tokens = cfg.B * cfg.T + dc.B
+    desc = (f"{prefill_heads} of {cfg.B * cfg.H} prefill heads (T={cfg.T}) in {tp:.2f} s and "
+            f"{decode_heads} of {dc.B * dc.H} decode heads in {td:.3f} s, scaled by head count to "
+            f"one full step ({full_p + full_d:.1f} s)")
+    return tokens / (full_p + full_d), full_p + full_d, desc, (tokens, full_p, full_d)
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle timed as it stands on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    vals = []
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        v, secs, desc, _ = oracle_sample_rate(prefill_heads=16, decode_heads=2048, seed_offset=s)
+        if s >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    tokens = 4 * 4096 + 256
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tokens / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config():
+    return {"workload": "gated_deltanet_prefill_B4_H16_T4096_d128_bf16_chunk64 + "
+                        "decode_step_B256_H32_d128_bf16_fp32state",
+            "prefill": {"B": 4, "H": 16, "T": 4096, "d_k": 128, "d_v": 128, "chunk": 64,
+                        "gate": "scalar", "tokens_per_step": 4 * 4096},
+            "decode": {"B": 256, "H": 32, "d_k": 128, "d_v": 128, "gate": "scalar",
+                       "tokens_per_step": 256, "token_bank": 16},
+            "l2": "no flush: every step streams > 1.3 GB (prefill inputs 274 MB, decode state "
+                  "1.07 GB read+write), more than the 126 MB L2",
+            "parallelism": "independent replicas, one per GPU"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import delta_rule_recurrent_02_b200 as dn
+    from delta_rule_recurrent_02_b200 import workloads as W
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dn.load_library()
+    peaks = load_peaks()
+
+    # ---- inputs (seeded per rank), resident in HBM --------------------------
+    pc = W.GDN_PREFILL
+    pin = W.gen_prefill(pc.B, pc.H, pc.T, pc.dk, pc.dv, dtype=pc.dtype, gate=pc.gate,
+                        seed=pc.seed + 1000 * rank, q_norm=True, g_shift=pc.g_shift)
+    dc = W.DECODE
+    din = W.gen_decode(dc)
+    P = {k: (None if v is None else v.to(dev)) for k, v in pin.items()}
+    D = {k: (None if v is None else v.to(dev)) for k, v in din.items()}
+    o_p = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
+    o_d = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
+    S_dec = D["S"]
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o_p, S_T, chunk=pc.chunk,
+                        scale=pc.scale, path=args.path, stream=stream)
+
+    def decode(s):
+        j = s % dc.bank
+        dn.dn_decode_step(D["q"][j], D["k"][j], D["v"][j], D["beta"][j], D["g"][j], S_dec, o_d,
+                          scale=dc.scale, stream=stream)
+
+    for s in range(args.warmup):
+        prefill()
+        decode(s)
+    dn.dn_device_status(stream)
+    barrier(world)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(_smi_id(torch, dev, local))
+    with sampler:
+        barrier(world)
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            prefill()
+            ev[s][1].record(stream)
+            decode(args.warmup + s)
+            ev[s][2].record(stream)
+        t_end.record(stream)
+        barrier(world)
+    dn.dn_device_status(stream)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    dec_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    pre_ms = max_over_ranks(pre_ms, world)
+    dec_ms = max_over_ranks(dec_ms, world)
+    ms_per_step = total_ms / args.steps
+    tokens_step = pc.B * pc.T + dc.B
+    value = world * tokens_step / (ms_per_step * 1e-3)
+    clocks = sampler.summary()
+
+    # ---- roofline per kernel ---------------------------------------------------
+    pf = prefill_flops(pc.B, pc.H, pc.T, pc.dk, pc.dv)
+    pb = prefill_bytes(pc.B, pc.H, pc.T, pc.dk, pc.dv)
+    db = decode_bytes(dc.B, dc.H, dc.dk, dc.dv)
+    used_tc = args.path == "tc" or (args.path == "auto" and _tc_active(dn, P, o_p, S_T, pc, stream))
+    pre_kernel = "chunk_tc" if used_tc else "chunk_simt"
+    pre_tflops = pf / (pre_ms * 1e-3) / 1e12
+    pre_gbs = pb / (pre_ms * 1e-3) / 1e9
+    dec_gbs = db / (dec_ms * 1e-3) / 1e9
+    tensor_floor = pf / (peaks["bf16_tflops"] * 1e12)
+    hbm_floor = pb / (peaks["hbm_gbs"] * 1e9)
+    pre_roof = {"kernel": pre_kernel, "bound": "hbm" if hbm_floor >= tensor_floor else "tensor",
+                "achieved": pre_gbs if hbm_floor >= tensor_floor else pre_tflops,
+                "peak": peaks["hbm_gbs"] if hbm_floor >= tensor_floor else peaks["bf16_tflops"],
+                "unit": "GB/s" if hbm_floor >= tensor_floor else "TFLOP/s",
+                "traffic": traffic_for(pre_kernel), "algorithmic_bytes": pb, "counted_flops": pf,
+                "tensor_tflops": pre_tflops, "tensor_frac": pre_tflops / peaks["bf16_tflops"],
+                "tensor_frac_sustained": pre_tflops / peaks["bf16_tflops_sustained"],
+                "hbm_gbs": pre_gbs, "hbm_frac": pre_gbs / peaks["hbm_gbs"],
+                "ms_per_launch": pre_ms, "peaks": peaks["source"]}
+    pre_roof["frac"] = pre_roof["achieved"] / pre_roof["peak"]
+    dec_roof = {"kernel": "decode_step", "bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"], "traffic": traffic_for("decode_step"),
+                "algorithmic_bytes": db, "ms_per_launch": dec_ms, "peaks": peaks["source"]}
+    dominant = pre_roof if pre_ms >= dec_ms else dec_roof
+    roofline = {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roofline["kernel"] = dominant["kernel"]
+
+    # ---- end to end through the C ABI with host buffers -------------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_step)
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if used_tc else "f32",
+            "data": "synthetic", "config": workload_config(),
+            "prefill": {"tokens_per_s": world * pc.B * pc.T / (pre_ms * 1e-3), "roofline": pre_roof},
+            "decode": {"tokens_per_s": world * dc.B / (dec_ms * 1e-3), "roofline": dec_roof},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]
+        v = statistics.median(r[0] for r in reps)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle.max_threads(),
+                                "kind": "oracle",
+                                "sample": f"median of {len(reps)} repetitions; each: " + reps[0][2]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _smi_id(torch, dev, local):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return local
+
+
+def _tc_active(dn, P, o_p, S_T, pc, stream):
+    lib = dn.load_library()
+    # the same request on the tensor-core path: DN_OK means the automatic choice uses it
+    import ctypes
+    st = lib.dn_chunk_fwd_ex(P["q"].data_ptr(), P["k"].data_ptr(), P["v"].data_ptr(), P["beta"].data_ptr(),
+                             P["g"].data_ptr(), None, o_p.data_ptr(), S_T.data_ptr(), pc.B, pc.T, pc.H,
+                             pc.dk, pc.dv, pc.chunk, pc.scale, 1, 1, 2, ctypes.c_void_p(stream.cuda_stream))
+    return st == 0
+
+
+def run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_step):
+    """Same step through the C ABI with pinned HOST buffers: per step, copy the
+    prefill inputs and the decode token set host->device, run both calls, copy
+    o, S_T and the decode output device->host.  The decode state stays
+    resident (it is the layer's memory, like weights)."""
+    hp = {k: (None if v is None else v.pin_memory()) for k, v in pin.items()}
+    hd = {k: (None if v is None else v.pin_memory()) for k, v in din.items() if k != "S"}
+    P = {k: torch.empty_like(v, device=dev) for k, v in hp.items() if v is not None}
+    Dt = {k: torch.empty_like(v[0], device=dev) for k, v in hd.items() if v is not None}
+    S_dec = din["S"].to(dev)
+    o_p = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
+    o_d = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
+    h_o = torch.empty(o_p.shape, dtype=o_p.dtype).pin_memory()
+    h_S = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    h_od = torch.empty(o_d.shape, dtype=o_d.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in hp.values() if v is not None) + \
+        sum(v[0].numel() * v.element_size() for v in hd.values() if v is not None)
+    d2h = sum(t.numel() * t.element_size() for t in (h_o, h_S, h_od))
+
+    def step(s):
+        for k, v in hp.items():
+            if v is not None:
+                P[k].copy_(v, non_blocking=True)
+        j = s % dc.bank
+        for k, v in hd.items():
+            if v is not None:
+                Dt[k].copy_(v[j], non_blocking=True)
+        dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o_p, S_T, chunk=pc.chunk,
+                        scale=pc.scale, path=args.path, stream=stream)
+        dn.dn_decode_step(Dt["q"], Dt["k"], Dt["v"], Dt["beta"], Dt["g"], S_dec, o_d, scale=dc.scale,
+                          stream=stream)
+        h_o.copy_(o_p, non_blocking=True)
+        h_S.copy_(S_T, non_blocking=True)
+        h_od.copy_(o_d, non_blocking=True)
+
+    for s in range(args.warmup):
+        step(s)
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(args.steps):
+        step(s)
+    b.record(stream)
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
+    return {"value": world * tokens_step / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

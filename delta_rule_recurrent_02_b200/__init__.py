@@ -1,1 +1,182 @@
-"""B200 (sm_100a) causal delta-rule layer: chunked prefill and decode step."""
+"""B200 (sm_100a) causal delta-rule layer: chunked prefill and decode step.
+
+A thin Python binding over the C ABI of ``include/dn.h`` (``libdn.so``, built
+in-tree by ``delta_rule_recurrent_02_b200/build.py``).  The binding only
+marshals arguments: torch tensors supply device pointers and streams, and
+every arithmetic step runs in the library's CUDA kernels.  There is no CPU
+path: if the library is missing, or a tensor is not on a CUDA device, the
+call raises.
+
+Functions with the ABI's names take preallocated outputs:
+
+    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=64, scale=1.0, ...)
+    dn_decode_step(q, k, v, beta, g, S, o, scale=1.0, ...)
+    dn_device_status(stream=None)
+
+and two conveniences allocate the outputs with torch:
+
+    o, S_T = chunk_fwd(q, k, v, beta, g=None, S0=None, chunk=64, scale=1.0)
+    o      = decode_step(q, k, v, beta, S, g=None, scale=1.0)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_decode_step",
+           "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
+           "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
+
+DN_OK, DN_ERR_INVALID, DN_ERR_UNSUPPORTED, DN_ERR_CUDA, DN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+_DTYPES = {"f32": 0, "bf16": 1}
+_GATES = {"none": 0, "scalar": 1, "per_key": 2}
+_PATHS = {"auto": 0, "simt": 1, "tc": 2}
+
+ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_decode_step", "dn_device_status",
+               "dn_status_str", "dn_last_error", "dn_version")
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class DNError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} [status {status}]")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libdn.so")
+
+
+def load_library():
+    """Load ``libdn.so`` and declare the ABI's signatures.  Raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m delta_rule_recurrent_02_b200.build` "
+                           "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    vp, fp, I, F = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.dn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, vp]
+    lib.dn_chunk_fwd.restype = I
+    lib.dn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, I, vp]
+    lib.dn_chunk_fwd_ex.restype = I
+    lib.dn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp]
+    lib.dn_decode_step.restype = I
+    lib.dn_device_status.argtypes = [vp]
+    lib.dn_device_status.restype = I
+    lib.dn_status_str.argtypes = [I]
+    lib.dn_status_str.restype = ctypes.c_char_p
+    lib.dn_last_error.argtypes = []
+    lib.dn_last_error.restype = ctypes.c_char_p
+    lib.dn_version.argtypes = []
+    lib.dn_version.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(lib, status: int):
+    if status != DN_OK:
+        msg = (lib.dn_last_error() or b"").decode() or lib.dn_status_str(status).decode()
+        raise DNError(status, msg)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("dn: tensors must be CUDA tensors (the library takes device pointers)")
+    if not t.is_contiguous():
+        raise ValueError("dn: tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return _DTYPES["f32"]
+    if t.dtype == torch.bfloat16:
+        return _DTYPES["bf16"]
+    raise ValueError(f"dn: unsupported token dtype {t.dtype}")
+
+
+def _gate_code(gate, g, lead_shape) -> int:
+    if gate is not None:
+        return _GATES[gate]
+    if g is None:
+        return _GATES["none"]
+    return _GATES["scalar"] if tuple(g.shape) == tuple(lead_shape) else _GATES["per_key"]
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _f32(t):
+    import torch
+    if t is not None and t.dtype != torch.float32:
+        raise ValueError("dn: beta, g and states must be float32")
+    return t
+
+
+def dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, *, chunk: int = 64, scale: float = 1.0,
+                 gate: str | None = None, path: str = "auto", stream=None) -> None:
+    """Chunked prefill through ``dn_chunk_fwd_ex``; writes ``o`` and ``S_T``."""
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    for t in (beta, g, S0, S_T):
+        _f32(t)
+    st = lib.dn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o),
+                             _ptr(S_T), B, T, H, dk, dv, int(chunk), float(scale), _dtype_code(q),
+                             _gate_code(gate, g, (B, H, T)), _PATHS[path], _stream(stream))
+    _check(lib, st)
+
+
+def dn_decode_step(q, k, v, beta, g, S, o, *, scale: float = 1.0, gate: str | None = None,
+                   stream=None) -> None:
+    """One decode step through ``dn_decode_step``; updates ``S`` in place, writes ``o``."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for t in (beta, g, S):
+        _f32(t)
+    st = lib.dn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S), _ptr(o),
+                            B, H, dk, dv, float(scale), _dtype_code(q),
+                            _gate_code(gate, g, (B, H)), _stream(stream))
+    _check(lib, st)
+
+
+def dn_device_status(stream=None) -> None:
+    """Synchronise the stream and raise DNError(DN_ERR_TIMEOUT) if a kernel gave up."""
+    lib = load_library()
+    _check(lib, lib.dn_device_status(_stream(stream)))
+
+
+def chunk_fwd(q, k, v, beta, g=None, S0=None, *, chunk: int = 64, scale: float = 1.0,
+              gate: str | None = None, path: str = "auto", want_state: bool = True, stream=None):
+    """Allocate ``o`` (dtype of q) and ``S_T`` (fp32), run the prefill, return both."""
+    import torch
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
+    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=chunk, scale=scale, gate=gate, path=path,
+                 stream=stream)
+    return o, S_T
+
+
+def decode_step(q, k, v, beta, S, g=None, *, scale: float = 1.0, gate: str | None = None,
+                stream=None):
+    """Allocate ``o``, run one decode step (S updated in place), return ``o``."""
+    import torch
+    B, H, _ = q.shape
+    o = torch.empty((B, H, v.shape[-1]), dtype=q.dtype, device=q.device)
+    dn_decode_step(q, k, v, beta, g, S, o, scale=scale, gate=gate, stream=stream)
+    return o

@@ -1,0 +1,339 @@
+// chunk_simt.cu -- chunked delta-rule prefill on the CUDA cores, fp32 math.
+//
+// The chunkwise form of "Linear attention and Gated DeltaNet" (ch. 28, "The
+// chunked form: recurrence as matrix multiplication"), with the per-key
+// decay of KDA folded in.  Inside a chunk of Cc <= 64 tokens, with
+// Gamma_i = sum_{m<=i} g_m (per key channel; one value for a scalar gate,
+// zero without a gate):
+//
+//   A_ij  = beta_i sum_c k_ic k_jc e^(Gamma_ic - Gamma_jc)        j <  i
+//   P_ij  =        sum_c q_ic k_jc e^(Gamma_ic - Gamma_jc)        j <= i
+//   (I + A) U = diag(beta) (V - (K * e^Gamma) S)                    (UT transform)
+//   O     = (Q * e^Gamma) S + P U
+//   S    <- Diag(e^Gamma_last) S + (K * e^(Gamma_last - Gamma))^T U
+//
+// which is the page's system with its right-hand side factored as
+// beta * (V - e^G (K S_0)).  A partial last chunk just uses Cc < chunk rows,
+// which equals zero padding with g = 0 and beta = 0.
+//
+// This is the fp32 path (fp32 or bf16 storage, fp32 arithmetic, any chunk
+// size 1..64).  One CTA owns one (b, h) and a 32-wide slice of the value
+// dimension: columns of S evolve independently given K, beta and g, so the
+// slices need no communication.  The state slice stays in shared memory for
+// the whole sequence; the only HBM traffic is the token tiles, o, and S0/S_T.
+#include "dn_common.cuh"
+#include "dn_kernels.h"
+
+namespace dn {
+
+namespace {
+
+constexpr int kNT = 256;     // threads per CTA
+constexpr int kDVT = 32;     // value columns per CTA
+constexpr int kCmax = 64;    // largest chunk
+constexpr int kVS = kDVT + 1;
+constexpr int kCS = kCmax + 1;
+
+template <int DK, int GATE>
+struct SimtSmem {
+    static constexpr int KS = DK + 1;
+    static constexpr int kK = 0;                              // K      [Cmax][KS]
+    static constexpr int kQ = kK + kCmax * KS;                // Q      [Cmax][KS]
+    static constexpr int kG = kQ + kCmax * KS;                // Gamma  [Cmax][KS] or [Cmax]
+    static constexpr int kGn = (GATE == kGatePerKey) ? kCmax * KS : kCmax;
+    static constexpr int kKx = kG + kGn;                      // scaled K (per-key only)
+    static constexpr int kKxn = (GATE == kGatePerKey) ? kCmax * KS : 0;
+    static constexpr int kV = kKx + kKxn;                     // V -> R -> U [Cmax][VS]
+    static constexpr int kA = kV + kCmax * kVS;               // A      [Cmax][CS]
+    static constexpr int kP = kA + kCmax * kCS;               // P      [Cmax][CS]
+    static constexpr int kS = kP + kCmax * kCS;               // S      [DK][VS]
+    static constexpr int kB = kS + DK * kVS;                  // beta   [Cmax]
+    static constexpr int kE = kB + kCmax;                     // e^G_i  [Cmax]
+    static constexpr int kT = kE + kCmax;                     // e^(G_last - G_i) [Cmax]
+    static constexpr int kTotal = kT + kCmax;
+    static constexpr size_t bytes = sizeof(float) * kTotal;
+};
+
+}  // namespace
+
+template <int DK, int GATE, typename Tin>
+__global__ void __launch_bounds__(kNT)
+chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                  const Tin* __restrict__ v, const float* __restrict__ beta,
+                  const float* __restrict__ g, const float* S0,
+                  Tin* __restrict__ o, float* S_T, int T, int DV, int chunk,
+                  float scale) {
+    using L = SimtSmem<DK, GATE>;
+    constexpr int KS = L::KS;
+    extern __shared__ float sm[];
+    float* Ks = sm + L::kK;
+    float* Qs = sm + L::kQ;
+    float* Gm = sm + L::kG;
+    float* Kx = sm + L::kKx;
+    float* Vs = sm + L::kV;
+    float* Am = sm + L::kA;
+    float* Pm = sm + L::kP;
+    float* Ss = sm + L::kS;
+    float* bs = sm + L::kB;
+    float* eG = sm + L::kE;
+    float* eT = sm + L::kT;
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int ntiles = DV / kDVT;
+    const int64_t bh = blockIdx.x / ntiles;
+    const int col0 = (blockIdx.x % ntiles) * kDVT;
+    const int64_t tok0 = bh * (int64_t)T;
+
+    // state slice S[:, col0 : col0 + 32]
+    for (int x = tid; x < DK * kDVT; x += kNT) {
+        const int i = x / kDVT, j = x % kDVT;
+        Ss[i * kVS + j] = S0 ? S0[(bh * DK + i) * DV + col0 + j] : 0.f;
+    }
+
+    // Token tiles of the next chunk are prefetched into registers while the
+    // current chunk is computed, so HBM latency is off the critical path.
+    constexpr int NVK = kCmax * DK / 4 / kNT;      // float4-groups of K (or Q, or g) per thread
+    constexpr int NVV = kCmax * kDVT / 4 / kNT;    // float4-groups of the V slice per thread
+    float4 pk[NVK], pq[NVK], pg[GATE == kGatePerKey ? NVK : 1], pv[NVV];
+    float pb = 0.f, ps = 0.f;
+    auto prefetch = [&](int c0) {
+        const int Cc = min(chunk, T - c0);
+        const int64_t t0 = tok0 + c0;
+#pragma unroll
+        for (int u = 0; u < NVK; ++u) {
+            const int x = tid + u * kNT;             // group index: row x / (DK/4), col 4 * (x % (DK/4))
+            if (x < Cc * DK / 4) {
+                const int64_t off = (t0 + x / (DK / 4)) * DK + 4 * (x % (DK / 4));
+                pk[u] = ld4(k + off);
+                pq[u] = ld4(q + off);
+                if (GATE == kGatePerKey) pg[u] = *reinterpret_cast<const float4*>(g + off);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < NVV; ++u) {
+            const int x = tid + u * kNT;
+            if (x < Cc * kDVT / 4)
+                pv[u] = ld4(v + (t0 + x / (kDVT / 4)) * DV + col0 + 4 * (x % (kDVT / 4)));
+        }
+        if (tid < Cc) {
+            pb = beta[t0 + tid];
+            if (GATE == kGateScalar) ps = g[t0 + tid];
+        }
+    };
+    if (T > 0) prefetch(0);
+
+    for (int c0 = 0; c0 < T; c0 += chunk) {
+        const int Cc = min(chunk, T - c0);
+        __syncthreads();   // previous chunk fully consumed
+        // ---- the chunk's tiles: registers -> shared memory -----------------
+#pragma unroll
+        for (int u = 0; u < NVK; ++u) {
+            const int x = tid + u * kNT;
+            if (x < Cc * DK / 4) {
+                const int i = x / (DK / 4), c = 4 * (x % (DK / 4));
+                float* kd = Ks + i * KS + c;
+                float* qd = Qs + i * KS + c;
+                kd[0] = pk[u].x; kd[1] = pk[u].y; kd[2] = pk[u].z; kd[3] = pk[u].w;
+                qd[0] = scale * pq[u].x; qd[1] = scale * pq[u].y; qd[2] = scale * pq[u].z; qd[3] = scale * pq[u].w;
+                if (GATE == kGatePerKey) {
+                    float* gd = Gm + i * KS + c;
+                    gd[0] = pg[u].x; gd[1] = pg[u].y; gd[2] = pg[u].z; gd[3] = pg[u].w;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < NVV; ++u) {
+            const int x = tid + u * kNT;
+            if (x < Cc * kDVT / 4) {
+                float* vd = Vs + (x / (kDVT / 4)) * kVS + 4 * (x % (kDVT / 4));
+                vd[0] = pv[u].x; vd[1] = pv[u].y; vd[2] = pv[u].z; vd[3] = pv[u].w;
+            }
+        }
+        if (tid < Cc) {
+            bs[tid] = pb;
+            if (GATE == kGateScalar) Gm[tid] = ps;
+        }
+        __syncthreads();
+        if (c0 + chunk < T) prefetch(c0 + chunk);
+        // ---- cumulative log-decay (inclusive) ---------------------------
+        if (GATE == kGateScalar) {
+            if (warp == 0) {
+                float a0 = lane < Cc ? Gm[lane] : 0.f;
+                float a1 = lane + 32 < Cc ? Gm[lane + 32] : 0.f;
+#pragma unroll
+                for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, a0, o2);
+                    const float y1 = __shfl_up_sync(0xffffffffu, a1, o2);
+                    if (lane >= o2) { a0 += y0; a1 += y1; }
+                }
+                a1 += __shfl_sync(0xffffffffu, a0, 31);
+                if (lane < Cc) Gm[lane] = a0;
+                if (lane + 32 < Cc) Gm[lane + 32] = a1;
+                __syncwarp();
+                const float Glast = Gm[Cc - 1];
+                for (int i = lane; i < Cc; i += 32) {
+                    eG[i] = expf(Gm[i]);
+                    eT[i] = expf(Glast - Gm[i]);
+                }
+            }
+        } else if (GATE == kGatePerKey) {
+            for (int c = tid; c < DK; c += kNT) {
+                float acc = 0.f;
+                for (int i = 0; i < Cc; ++i) {
+                    acc += Gm[i * KS + c];
+                    Gm[i * KS + c] = acc;
+                }
+            }
+        } else {
+            for (int i = tid; i < Cc; i += kNT) { eG[i] = 1.f; eT[i] = 1.f; }
+        }
+        __syncthreads();
+        // ---- pairwise decayed products: A (strict lower) and P (lower) ---
+        for (int p = tid; p < Cc * Cc; p += kNT) {
+            const int i = p / Cc, j = p % Cc;
+            float kd = 0.f, qd = 0.f;
+            if (j <= i) {
+                const float* ki = Ks + i * KS;
+                const float* qi = Qs + i * KS;
+                const float* kj = Ks + j * KS;
+                if (GATE == kGatePerKey) {
+                    const float* gi = Gm + i * KS;
+                    const float* gj = Gm + j * KS;
+#pragma unroll 4
+                    for (int c = 0; c < DK; ++c) {
+                        const float w = kj[c] * expf(gi[c] - gj[c]);
+                        kd += ki[c] * w;
+                        qd += qi[c] * w;
+                    }
+                } else {
+#pragma unroll 8
+                    for (int c = 0; c < DK; ++c) {
+                        kd += ki[c] * kj[c];
+                        qd += qi[c] * kj[c];
+                    }
+                    if (GATE == kGateScalar) {
+                        const float d = expf(Gm[i] - Gm[j]);
+                        kd *= d;
+                        qd *= d;
+                    }
+                }
+            }
+            Am[i * kCS + j] = (j < i) ? bs[i] * kd : 0.f;
+            Pm[i * kCS + j] = qd;
+        }
+        if (GATE == kGatePerKey) {
+            __syncthreads();   // P used the raw q; now Q <- Q * e^Gamma, Kx <- K * e^Gamma
+            for (int x = tid; x < Cc * DK; x += kNT) {
+                const int i = x / DK, c = x % DK;
+                const float e = expf(Gm[i * KS + c]);
+                Qs[i * KS + c] *= e;
+                Kx[i * KS + c] = Ks[i * KS + c] * e;
+            }
+        }
+        __syncthreads();
+        // ---- right-hand side: beta * (V - (K * e^Gamma) S) ---------------
+        {
+            const int j = lane;
+            for (int i = warp; i < Cc; i += kNT / 32) {
+                const float* kr = (GATE == kGatePerKey) ? (Kx + i * KS) : (Ks + i * KS);
+                float acc = 0.f;
+#pragma unroll 8
+                for (int c = 0; c < DK; ++c) acc += kr[c] * Ss[c * kVS + j];
+                if (GATE != kGatePerKey) acc *= eG[i];
+                Vs[i * kVS + j] = bs[i] * (Vs[i * kVS + j] - acc);
+            }
+        }
+        __syncthreads();
+        // ---- forward substitution (I + A) U = rhs, 4 columns per warp ----
+        {
+            const int j = warp * 4 + (lane >> 3);
+            const int part = lane & 7;
+            for (int i = 1; i < Cc; ++i) {
+                float acc = 0.f;
+                for (int m = part; m < i; m += 8) acc += Am[i * kCS + m] * Vs[m * kVS + j];
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                if (part == 0) Vs[i * kVS + j] -= acc;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        // ---- output: O = (Q * e^Gamma) S + P U ---------------------------
+        {
+            const int j = lane;
+            for (int i = warp; i < Cc; i += kNT / 32) {
+                const float* qr = Qs + i * KS;
+                float acc = 0.f;
+#pragma unroll 8
+                for (int c = 0; c < DK; ++c) acc += qr[c] * Ss[c * kVS + j];
+                if (GATE != kGatePerKey) acc *= eG[i];
+                const float* pr = Pm + i * kCS;
+                for (int m = 0; m <= i; ++m) acc += pr[m] * Vs[m * kVS + j];
+                st_elem(o + (tok0 + c0 + i) * DV + col0 + j, acc);
+            }
+        }
+        if (GATE == kGatePerKey) {
+            __syncthreads();   // Kx <- K * e^(Gamma_last - Gamma)
+            for (int x = tid; x < Cc * DK; x += kNT) {
+                const int i = x / DK, c = x % DK;
+                Kx[i * KS + c] = Ks[i * KS + c] * expf(Gm[(Cc - 1) * KS + c] - Gm[i * KS + c]);
+            }
+        }
+        __syncthreads();
+        // ---- state: S <- Diag(e^Gamma_last) S + (K * e^(Gamma_last - Gamma))^T U
+        {
+            const int j = lane;
+            for (int c = warp; c < DK; c += kNT / 32) {
+                float acc = 0.f;
+                if (GATE == kGatePerKey) {
+                    for (int i = 0; i < Cc; ++i) acc += Kx[i * KS + c] * Vs[i * kVS + j];
+                    Ss[c * kVS + j] = expf(Gm[(Cc - 1) * KS + c]) * Ss[c * kVS + j] + acc;
+                } else {
+                    for (int i = 0; i < Cc; ++i) acc += Ks[i * KS + c] * eT[i] * Vs[i * kVS + j];
+                    const float dec = (GATE == kGateScalar) ? expf(Gm[Cc - 1]) : 1.f;
+                    Ss[c * kVS + j] = dec * Ss[c * kVS + j] + acc;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (S_T) {
+        for (int x = tid; x < DK * kDVT; x += kNT) {
+            const int i = x / kDVT, j = x % kDVT;
+            S_T[(bh * DK + i) * DV + col0 + j] = Ss[i * kVS + j];
+        }
+    }
+}
+
+template <int DK, int GATE, typename Tin>
+static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t st) {
+    using L = SimtSmem<DK, GATE>;
+    auto kern = chunk_simt_kernel<DK, GATE, Tin>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = a.B * a.H * (a.dv / kDVT);
+    kern<<<(unsigned)grid, kNT, L::bytes, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+        a.beta, a.g, a.S0, static_cast<Tin*>(a.o), a.S_T, (int)a.T, a.dv, a.chunk, a.scale);
+    return cudaGetLastError();
+}
+
+template <int DK, typename Tin>
+static cudaError_t launch_simt_gate(const ChunkArgs& a, cudaStream_t st) {
+    switch (a.gate) {
+        case kGateNone: return launch_simt_t<DK, kGateNone, Tin>(a, st);
+        case kGateScalar: return launch_simt_t<DK, kGateScalar, Tin>(a, st);
+        default: return launch_simt_t<DK, kGatePerKey, Tin>(a, st);
+    }
+}
+
+cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t st) {
+    if (a.B * a.H == 0) return cudaSuccess;
+    if (a.dk == 128)
+        return a.bf16 ? launch_simt_gate<128, __nv_bfloat16>(a, st) : launch_simt_gate<128, float>(a, st);
+    return a.bf16 ? launch_simt_gate<64, __nv_bfloat16>(a, st) : launch_simt_gate<64, float>(a, st);
+}
+
+}  // namespace dn

@@ -1,0 +1,143 @@
+// decode_step.cu -- one recurrent step of the delta rule per (sequence, head).
+//
+// "Linear attention and Gated DeltaNet" (ch. 28), "The recurrent form": for
+// each head, decay the d_k x d_v fp32 state, predict p = S~^T k, write
+// S = S~ + k (beta (v - p))^T and read o = S^T (scale q); for KDA the decay
+// scales row i (key channel i) by exp(g_i) ("A walk through of the DeltaNet
+// family", the KDA recurrence).  The page calls the step memory-bound on the
+// state; the kernel therefore streams each state exactly once in and once
+// out of HBM and does everything else on chip.
+//
+// One CTA owns one head.  Thread (rs, cg) holds rows rs, rs + RS, ... and the
+// four columns 4cg .. 4cg+3 of S in registers (a warp covers one full 512-byte
+// row per 128-bit access, so every load and store is coalesced).  The two
+// reductions over rows (p = S~^T k and S~^T q') go through shared memory;
+// the output uses o = S~^T q' + (q'.k) delta, which needs S~ only, so the
+// state is read once and written once.
+#include "dn_common.cuh"
+#include "dn_kernels.h"
+
+namespace dn {
+
+template <int DK, int DV, typename Tin, int GATE>
+__global__ void __launch_bounds__(2 * DV)
+decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                   const Tin* __restrict__ v, const float* __restrict__ beta,
+                   const float* __restrict__ g, float* __restrict__ S,
+                   Tin* __restrict__ o, float scale) {
+    constexpr int NT = 2 * DV;     // threads
+    constexpr int TPR = DV / 4;    // threads per state row
+    constexpr int RS = NT / TPR;   // row sets (8)
+    constexpr int RPT = DK / RS;   // rows per thread
+    const int64_t head = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int cg = tid % TPR;
+    const int rs = tid / TPR;
+
+    __shared__ float ks[DK], qs[DK], as[DK];
+    __shared__ float4 red_p[RS][TPR], red_q[RS][TPR];
+    __shared__ float qk_s;
+
+    float* Sh = S + head * (DK * DV);
+    float4 s[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m)
+        s[m] = ld_stream_f4(Sh + (rs + RS * m) * DV + cg * 4);
+
+    for (int i = tid; i < DK; i += NT) {
+        ks[i] = ld_elem(k + head * DK + i);
+        qs[i] = scale * ld_elem(q + head * DK + i);
+        if (GATE == kGatePerKey) as[i] = expf(g[head * DK + i]);
+    }
+    const float4 vv = ld4(v + head * DV + cg * 4);
+    const float b = beta[head];
+    const float a = (GATE == kGateScalar) ? expf(g[head]) : 1.0f;
+    __syncthreads();
+
+    if (tid < 32) {
+        float x = 0.f;
+        for (int i = tid; i < DK; i += 32) x += qs[i] * ks[i];
+        x = warp_sum(x);
+        if (tid == 0) qk_s = x;
+    }
+
+    float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = p4;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int r = rs + RS * m;
+        const float d = (GATE == kGatePerKey) ? as[r] : a;
+        if (GATE != kGateNone) {
+            s[m].x *= d; s[m].y *= d; s[m].z *= d; s[m].w *= d;
+        }
+        const float kr = ks[r], qr = qs[r];
+        p4.x += kr * s[m].x; p4.y += kr * s[m].y; p4.z += kr * s[m].z; p4.w += kr * s[m].w;
+        q4.x += qr * s[m].x; q4.y += qr * s[m].y; q4.z += qr * s[m].z; q4.w += qr * s[m].w;
+    }
+    red_p[rs][cg] = p4;
+    red_q[rs][cg] = q4;
+    __syncthreads();
+
+    float4 pred = make_float4(0.f, 0.f, 0.f, 0.f), qsum = pred;
+#pragma unroll
+    for (int r = 0; r < RS; ++r) {
+        const float4 x = red_p[r][cg], y = red_q[r][cg];
+        pred.x += x.x; pred.y += x.y; pred.z += x.z; pred.w += x.w;
+        qsum.x += y.x; qsum.y += y.y; qsum.z += y.z; qsum.w += y.w;
+    }
+    float4 dl;
+    dl.x = b * (vv.x - pred.x); dl.y = b * (vv.y - pred.y);
+    dl.z = b * (vv.z - pred.z); dl.w = b * (vv.w - pred.w);
+
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int r = rs + RS * m;
+        const float kr = ks[r];
+        float4 x = s[m];
+        x.x += kr * dl.x; x.y += kr * dl.y; x.z += kr * dl.z; x.w += kr * dl.w;
+        st_stream_f4(Sh + r * DV + cg * 4, x);
+    }
+    if (rs == 0) {
+        const float qk = qk_s;
+        float4 ov;
+        ov.x = qsum.x + qk * dl.x; ov.y = qsum.y + qk * dl.y;
+        ov.z = qsum.z + qk * dl.z; ov.w = qsum.w + qk * dl.w;
+        st4(o + head * DV + cg * 4, ov);
+    }
+}
+
+template <int DK, int DV, typename Tin>
+static cudaError_t launch_decode_gate(const DecodeArgs& a, cudaStream_t st) {
+    const unsigned grid = (unsigned)(a.B * a.H);
+    const Tin* q = static_cast<const Tin*>(a.q);
+    const Tin* k = static_cast<const Tin*>(a.k);
+    const Tin* v = static_cast<const Tin*>(a.v);
+    Tin* o = static_cast<Tin*>(a.o);
+    switch (a.gate) {
+        case kGateNone:
+            decode_step_kernel<DK, DV, Tin, kGateNone><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            break;
+        case kGateScalar:
+            decode_step_kernel<DK, DV, Tin, kGateScalar><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            break;
+        default:
+            decode_step_kernel<DK, DV, Tin, kGatePerKey><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            break;
+    }
+    return cudaGetLastError();
+}
+
+template <int DK, int DV>
+static cudaError_t launch_decode_dims(const DecodeArgs& a, cudaStream_t st) {
+    return a.bf16 ? launch_decode_gate<DK, DV, __nv_bfloat16>(a, st)
+                  : launch_decode_gate<DK, DV, float>(a, st);
+}
+
+cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st) {
+    if (a.B * a.H == 0) return cudaSuccess;
+    if (a.dk == 128 && a.dv == 128) return launch_decode_dims<128, 128>(a, st);
+    if (a.dk == 128 && a.dv == 64) return launch_decode_dims<128, 64>(a, st);
+    if (a.dk == 64 && a.dv == 128) return launch_decode_dims<64, 128>(a, st);
+    return launch_decode_dims<64, 64>(a, st);
+}
+
+}  // namespace dn

@@ -1,0 +1,225 @@
+// dn_api.cu -- the C ABI: argument validation, kernel choice, launch, status.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/dn.h"
+#include "dn_kernels.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_last_error[0] = '\0';
+    return DN_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(DN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Device status word: kernels with bounded waits OR a code into it when they
+// give up.  One per device (a module-scope __device__ variable exists once per
+// device context).
+__device__ unsigned int g_device_status;
+
+unsigned int* status_word(cudaError_t* err) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_device_status);
+    return static_cast<unsigned int*>(p);
+}
+
+struct Range {
+    uintptr_t lo, hi;   // [lo, hi)
+    bool valid() const { return lo != 0 && hi > lo; }
+};
+
+Range rng(const void* p, int64_t bytes) {
+    Range r;
+    r.lo = reinterpret_cast<uintptr_t>(p);
+    r.hi = r.lo + (uintptr_t)(bytes > 0 ? bytes : 0);
+    return r;
+}
+
+bool overlap(Range a, Range b) {
+    if (!a.valid() || !b.valid()) return false;
+    return a.lo < b.hi && b.lo < a.hi;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+}  // namespace
+
+extern "C" {
+
+int dn_version(void) { return (1 << 16) | 0; }
+
+const char* dn_status_str(int status) {
+    switch (status) {
+        case DN_OK: return "DN_OK";
+        case DN_ERR_INVALID: return "DN_ERR_INVALID: invalid argument";
+        case DN_ERR_UNSUPPORTED: return "DN_ERR_UNSUPPORTED: request outside the supported set";
+        case DN_ERR_CUDA: return "DN_ERR_CUDA: CUDA call or kernel launch failed";
+        case DN_ERR_TIMEOUT: return "DN_ERR_TIMEOUT: a bounded device wait gave up";
+        default: return "unknown dn_status";
+    }
+}
+
+const char* dn_last_error(void) { return g_last_error; }
+
+int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+                    const float* g, const float* S0, void* o, float* S_T,
+                    int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                    dn_dtype dtype, dn_gate gate, dn_path path, void* cuda_stream) {
+    if (B < 0 || T < 0 || H < 0) return fail(DN_ERR_INVALID, "B, T, H must be >= 0 (got %d, %d, %d)", B, T, H);
+    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
+    if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
+        return fail(DN_ERR_INVALID, "unknown gate %d", (int)gate);
+    if (path != DN_PATH_AUTO && path != DN_PATH_SIMT && path != DN_PATH_TC)
+        return fail(DN_ERR_INVALID, "unknown path %d", (int)path);
+    if (d_k <= 0 || d_v <= 0) return fail(DN_ERR_INVALID, "d_k, d_v must be > 0");
+    if (chunk <= 0) return fail(DN_ERR_INVALID, "chunk must be > 0 (got %d)", chunk);
+    if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return fail(DN_ERR_INVALID, "scale is not finite");
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(DN_ERR_UNSUPPORTED, "d_k, d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
+    const int64_t ntok = (int64_t)B * H * T;
+    const int64_t esz = dtype == DN_BF16 ? 2 : 4;
+    const bool empty_tokens = ntok == 0;
+    if (!empty_tokens && (!q || !k || !v || !beta || !o))
+        return fail(DN_ERR_INVALID, "q, k, v, beta and o are required");
+    if (gate == DN_GATE_NONE && g) return fail(DN_ERR_INVALID, "g must be NULL when gate is DN_GATE_NONE");
+    if (gate != DN_GATE_NONE && !g && !empty_tokens) return fail(DN_ERR_INVALID, "g is required for this gate");
+    const void* p16[] = {q, k, v, o, S0, S_T};
+    const char* n16[] = {"q", "k", "v", "o", "S0", "S_T"};
+    for (int i = 0; i < 6; ++i)
+        if (p16[i] && !aligned(p16[i], 16)) return fail(DN_ERR_INVALID, "%s is not 16-byte aligned", n16[i]);
+    if ((beta && !aligned(beta, 4)) || (g && !aligned(g, 4)))
+        return fail(DN_ERR_INVALID, "beta and g must be 4-byte aligned");
+    if (gate == DN_GATE_PER_KEY && g && !aligned(g, 16))
+        return fail(DN_ERR_INVALID, "a per-key g must be 16-byte aligned");
+    const int64_t gcount = gate == DN_GATE_PER_KEY ? ntok * d_k : ntok;
+    const int64_t sbytes = (int64_t)B * H * d_k * d_v * 4;
+    Range rq = rng(q, ntok * d_k * esz), rk = rng(k, ntok * d_k * esz), rv = rng(v, ntok * d_v * esz);
+    Range rb = rng(beta, ntok * 4), rg = rng(g, gcount * 4), rs0 = rng(S0, sbytes);
+    Range ro = rng(o, ntok * d_v * esz), rst = rng(S_T, sbytes);
+    Range ins[] = {rq, rk, rv, rb, rg, rs0};
+    for (Range r : ins)
+        if (overlap(ro, r) || overlap(ro, rst)) return fail(DN_ERR_INVALID, "o overlaps another argument");
+    Range ins2[] = {rq, rk, rv, rb, rg};
+    for (Range r : ins2)
+        if (overlap(rst, r)) return fail(DN_ERR_INVALID, "S_T overlaps an input other than S0");
+    if (S_T && S0 && (void*)S_T != (const void*)S0 && overlap(rst, rs0))
+        return fail(DN_ERR_INVALID, "S_T partly overlaps S0");
+
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    if ((int64_t)B * H == 0) return ok();
+
+    dn::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk; a.scale = scale;
+    a.bf16 = dtype == DN_BF16; a.gate = (int)gate;
+    cudaError_t e;
+    a.status = status_word(&e);
+    if (e != cudaSuccess) return cuda_fail(e, "status word");
+
+    if (T == 0) {   // nothing to read: the final state is the initial one
+        if (!S_T) return ok();
+        if (S0 && (const void*)S0 != (void*)S_T) e = cudaMemcpyAsync(S_T, S0, sbytes, cudaMemcpyDeviceToDevice, st);
+        else if (!S0) e = cudaMemsetAsync(S_T, 0, sbytes, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "T = 0 state copy");
+    }
+
+    bool use_tc = false;
+    if (path == DN_PATH_TC) {
+        if (!dn::tc_supports(a))
+            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128");
+        use_tc = true;
+    } else if (path == DN_PATH_AUTO) {
+        use_tc = dn::tc_supports(a);
+    }
+    if (!use_tc && chunk > 64) return fail(DN_ERR_UNSUPPORTED, "chunk must be <= 64 (got %d)", chunk);
+    e = use_tc ? dn::launch_chunk_tc(a, st) : dn::launch_chunk_simt(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core chunk kernel" : "SIMT chunk kernel");
+    return ok();
+}
+
+int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
+                 const float* g, const float* S0, void* o, float* S_T,
+                 int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                 dn_dtype dtype, dn_gate gate, void* cuda_stream) {
+    return dn_chunk_fwd_ex(q, k, v, beta, g, S0, o, S_T, B, T, H, d_k, d_v, chunk, scale,
+                           dtype, gate, DN_PATH_AUTO, cuda_stream);
+}
+
+int dn_decode_step(const void* q, const void* k, const void* v, const float* beta,
+                   const float* g, float* S, void* o, int B, int H, int d_k, int d_v,
+                   float scale, dn_dtype dtype, dn_gate gate, void* cuda_stream) {
+    if (B < 0 || H < 0) return fail(DN_ERR_INVALID, "B, H must be >= 0 (got %d, %d)", B, H);
+    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
+    if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
+        return fail(DN_ERR_INVALID, "unknown gate %d", (int)gate);
+    if (d_k <= 0 || d_v <= 0) return fail(DN_ERR_INVALID, "d_k, d_v must be > 0");
+    if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return fail(DN_ERR_INVALID, "scale is not finite");
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(DN_ERR_UNSUPPORTED, "d_k, d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
+    const int64_t nh = (int64_t)B * H;
+    if (nh == 0) return ok();
+    if (!q || !k || !v || !beta || !S || !o) return fail(DN_ERR_INVALID, "q, k, v, beta, S and o are required");
+    if (gate == DN_GATE_NONE && g) return fail(DN_ERR_INVALID, "g must be NULL when gate is DN_GATE_NONE");
+    if (gate != DN_GATE_NONE && !g) return fail(DN_ERR_INVALID, "g is required for this gate");
+    const void* p16[] = {q, k, v, o, S};
+    const char* n16[] = {"q", "k", "v", "o", "S"};
+    for (int i = 0; i < 5; ++i)
+        if (!aligned(p16[i], 16)) return fail(DN_ERR_INVALID, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(beta, 4) || (g && !aligned(g, 4))) return fail(DN_ERR_INVALID, "beta and g must be 4-byte aligned");
+    if (gate == DN_GATE_PER_KEY && !aligned(g, 16)) return fail(DN_ERR_INVALID, "a per-key g must be 16-byte aligned");
+    const int64_t esz = dtype == DN_BF16 ? 2 : 4;
+    Range rq = rng(q, nh * d_k * esz), rk = rng(k, nh * d_k * esz), rv = rng(v, nh * d_v * esz);
+    Range rb = rng(beta, nh * 4), rg = rng(g, (gate == DN_GATE_PER_KEY ? nh * d_k : nh) * 4);
+    Range rs = rng(S, nh * d_k * d_v * 4), ro = rng(o, nh * d_v * esz);
+    Range others[] = {rq, rk, rv, rb, rg, rs};
+    for (Range r : others)
+        if (overlap(ro, r)) return fail(DN_ERR_INVALID, "o overlaps another argument");
+    Range ins[] = {rq, rk, rv, rb, rg};
+    for (Range r : ins)
+        if (overlap(rs, r)) return fail(DN_ERR_INVALID, "S overlaps an input");
+
+    dn::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S = S; a.o = o;
+    a.B = B; a.H = H; a.dk = d_k; a.dv = d_v; a.scale = scale;
+    a.bf16 = dtype == DN_BF16; a.gate = (int)gate;
+    cudaError_t e = dn::launch_decode_step(a, static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
+    return ok();
+}
+
+int dn_device_status(void* cuda_stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "read status word");
+    if (word != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+        return fail(DN_ERR_TIMEOUT, "a kernel gave up on a bounded wait (status 0x%x)", word);
+    }
+    return ok();
+}
+
+}  // extern "C"

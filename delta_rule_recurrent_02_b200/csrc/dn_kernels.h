@@ -1,0 +1,41 @@
+// dn_kernels.h -- launchers behind the C ABI (private to the library).
+// Arguments arrive already validated by dn_api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dn {
+
+struct ChunkArgs {
+    const void* q; const void* k; const void* v;
+    const float* beta; const float* g; const float* S0;
+    void* o; float* S_T;
+    int64_t B, T, H;
+    int dk, dv, chunk;
+    float scale;
+    bool bf16;
+    int gate;                 // Gate
+    unsigned int* status;     // device status word of the current device
+};
+
+struct DecodeArgs {
+    const void* q; const void* k; const void* v;
+    const float* beta; const float* g;
+    float* S; void* o;
+    int64_t B, H;
+    int dk, dv;
+    float scale;
+    bool bf16;
+    int gate;
+};
+
+cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t st);
+
+// Tensor-core (tcgen05) chunk kernel.  tc_supports() says whether the request
+// is inside the kernel's coverage (bf16, chunk 64, d_k = d_v = 128).
+bool tc_supports(const ChunkArgs& a);
+cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st);
+
+}  // namespace dn

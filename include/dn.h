@@ -1,0 +1,151 @@
+/*
+ * dn.h -- C ABI of the B200 (sm_100a) causal delta-rule layer.
+ *
+ * The layer keeps, per sequence b and head h, a state S of d_k x d_v fp32
+ * values (row i = key channel, column j = value channel) and for every token
+ * t runs
+ *
+ *     forget   S~  = decay_t(S)          (none | exp(g_t) S | Diag(exp(g_t)) S)
+ *     predict  p   = S~^T k_t
+ *     correct  e   = beta_t (v_t - p)
+ *     write    S   = S~ + k_t e^T
+ *     read     o_t = S^T (scale q_t)     (after the write)
+ *
+ * i.e. S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ * with alpha_t = exp(g_t) (decay first; for a scalar alpha this is
+ * alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T).  Sources: "Linear attention and Gated DeltaNet"
+ * (inference.shantanugoel.com, ch. 28), sections "Correct: the delta rule",
+ * "Gated DeltaNet" and "The recurrent form" (the contract: q, k [B,H,T,Dk]
+ * already L2-normalised, v [B,H,T,Dv], g and beta [B,H,T], optional initial
+ * state [B,H,Dk,Dv], returning o and the final state); section "The chunked
+ * form" (same contract and result, computed chunk by chunk); D2L 12.5
+ * "DeltaNet", slides "One rule, two readings" and "Gating: the modern cell";
+ * and "A walk through of the DeltaNet family of linear attention variants"
+ * (selinyilmaz.dev), its KDA update with a per-key-channel decay.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no state between calls except a
+ *     per-device status word read by dn_device_status().
+ *   - Every layout is dense row-major (C order) with the shapes given.
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Inputs must stay valid until the work ends.
+ *   - The return value is a dn_status.  Nothing throws or aborts across the
+ *     ABI.  On DN_ERR_INVALID / DN_ERR_UNSUPPORTED nothing was launched and
+ *     no output was touched; dn_last_error() gives the reason.
+ *   - beta is not clamped (values in (0, 2) give the negative-eigenvalue
+ *     transitions of D2L 12.5, "The reflection hiding in the delta rule").
+ *     g is the log-decay (alpha = exp(g)); g <= 0 is expected but not
+ *     enforced.  k is not normalised by the library.
+ *   - Pointers to q, k, v, o, S0, S_T and S must be 16-byte aligned, as must a
+ *     per-key g; beta and a scalar g 4-byte aligned.
+ */
+#ifndef DN_H
+#define DN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DN_API __attribute__((visibility("default")))
+#else
+#define DN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DN_OK = 0,
+    DN_ERR_INVALID = 1,      /* null required pointer, bad size, misalignment, aliasing */
+    DN_ERR_UNSUPPORTED = 2,  /* valid request this library does not implement */
+    DN_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed */
+    DN_ERR_TIMEOUT = 4       /* a bounded device wait gave up (see dn_device_status) */
+} dn_status;
+
+typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;   /* storage type of q, k, v and o */
+
+typedef enum {
+    DN_GATE_NONE = 0,     /* DeltaNet: alpha = 1, g must be NULL            */
+    DN_GATE_SCALAR = 1,   /* Gated DeltaNet: g [B,H,T] (decode: [B,H])       */
+    DN_GATE_PER_KEY = 2   /* KDA: g [B,H,T,d_k] (decode: [B,H,d_k])          */
+} dn_gate;
+
+typedef enum {
+    DN_PATH_AUTO = 0,     /* tensor-core path when it supports the request, else SIMT */
+    DN_PATH_SIMT = 1,     /* fp32 CUDA-core chunk kernel: any chunk 1..64          */
+    DN_PATH_TC = 2        /* tcgen05 chunk kernel: bf16, chunk 64, d_k = d_v = 128 */
+} dn_path;
+
+/*
+ * dn_chunk_fwd -- chunked prefill ("The chunked form", ch. 28).
+ *
+ *   q     [B,H,T,d_k]  dtype   queries (multiplied by `scale` inside)
+ *   k     [B,H,T,d_k]  dtype   keys
+ *   v     [B,H,T,d_v]  dtype   values
+ *   beta  [B,H,T]      fp32    write strengths
+ *   g     NULL | [B,H,T] | [B,H,T,d_k]  fp32 log-decay, per `gate`
+ *   S0    NULL (zero state) | [B,H,d_k,d_v] fp32, read only
+ *   o     [B,H,T,d_v]  dtype   output, o_t read after token t's write
+ *   S_T   NULL (not written) | [B,H,d_k,d_v] fp32 final state; may equal S0
+ *         exactly (in-place continuation), must not partly overlap it
+ *   chunk tokens per chunk; the result does not depend on it beyond rounding
+ *         (the last chunk may be partial: it equals zero padding with g = 0,
+ *         beta = 0).  SIMT path: 1..64; tensor-core path: 64.
+ *   d_k, d_v in {64, 128}.  B, H, T >= 0 (T = 0 writes S_T = S0 or zeros).
+ *
+ * o must not overlap any input.  Returns DN_ERR_UNSUPPORTED for a d or chunk
+ * outside the ranges above (or a DN_PATH_TC request the tensor-core kernel
+ * does not cover).
+ */
+DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
+                 const float* beta, const float* g, const float* S0,
+                 void* o, float* S_T,
+                 int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                 dn_dtype dtype, dn_gate gate, void* cuda_stream);
+
+/* dn_chunk_fwd with an explicit kernel choice (for tests and benchmarks). */
+DN_API int dn_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                    const float* beta, const float* g, const float* S0,
+                    void* o, float* S_T,
+                    int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                    dn_dtype dtype, dn_gate gate, dn_path path, void* cuda_stream);
+
+/*
+ * dn_decode_step -- one recurrent step ("The recurrent form", ch. 28; KDA's
+ * recurrence in "A walk through of the DeltaNet family").
+ *
+ *   q, k  [B,H,d_k] dtype;  v [B,H,d_v] dtype;  beta [B,H] fp32
+ *   g     NULL | [B,H] | [B,H,d_k] fp32 per `gate`
+ *   S     [B,H,d_k,d_v] fp32, updated in place
+ *   o     [B,H,d_v] dtype, must not overlap any other argument
+ *   d_k, d_v in {64, 128}; B, H >= 0.
+ */
+DN_API int dn_decode_step(const void* q, const void* k, const void* v,
+                   const float* beta, const float* g, float* S, void* o,
+                   int B, int H, int d_k, int d_v, float scale,
+                   dn_dtype dtype, dn_gate gate, void* cuda_stream);
+
+/*
+ * dn_device_status -- synchronise `cuda_stream`, then read and clear the
+ * status word of the current device.  Returns DN_ERR_TIMEOUT if a kernel of
+ * this library launched since the previous call gave up on a bounded wait
+ * (its outputs are then unspecified), DN_ERR_CUDA if the synchronisation
+ * failed, else DN_OK.
+ */
+DN_API int dn_device_status(void* cuda_stream);
+
+/* Static description of a status code. */
+DN_API const char* dn_status_str(int status);
+
+/* Reason for the last non-DN_OK return on the calling thread ("" if none). */
+DN_API const char* dn_last_error(void);
+
+/* ABI version, (major << 16) | minor. */
+DN_API int dn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DN_H */

@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point ``include/dn.h`` declares, and rejects bad arguments before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import delta_rule_recurrent_02_b200 as dn
+from delta_rule_recurrent_02_b200 import build as dn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dn_build.build()
+    return dn.load_library()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "dn.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"DN_API\s+[\w\s\*]+?\b(dn_\w+)\s*\(", text)))
+
+
+def test_header_declares_abi():
+    assert declared_symbols() == sorted(dn.ABI_SYMBOLS)
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dn_version() >> 16 == 1
+    for code in range(5):
+        assert lib.dn_status_str(code).startswith(b"DN_")
+    assert lib.dn_status_str(99) == b"unknown dn_status"
+
+
+# Fake, never dereferenced addresses: validation must fail before any CUDA call.
+A = 0x10000000
+STEP = 0x01000000
+
+
+def chunk_call(lib, **over):
+    args = dict(q=A, k=A + STEP, v=A + 2 * STEP, beta=A + 3 * STEP, g=A + 4 * STEP, S0=None,
+                o=A + 5 * STEP, S_T=A + 6 * STEP, B=1, T=8, H=1, dk=64, dv=64, chunk=8,
+                scale=1.0, dtype=0, gate=1, path=0)
+    args.update(over)
+    return lib.dn_chunk_fwd_ex(args["q"], args["k"], args["v"], args["beta"], args["g"], args["S0"],
+                               args["o"], args["S_T"], args["B"], args["T"], args["H"], args["dk"],
+                               args["dv"], args["chunk"], args["scale"], args["dtype"], args["gate"],
+                               args["path"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=-1), dn.DN_ERR_INVALID),
+    (dict(T=-3), dn.DN_ERR_INVALID),
+    (dict(q=None), dn.DN_ERR_INVALID),
+    (dict(o=None), dn.DN_ERR_INVALID),
+    (dict(g=None), dn.DN_ERR_INVALID),                       # scalar gate needs g
+    (dict(gate=0), dn.DN_ERR_INVALID),                       # no gate but g given
+    (dict(gate=7), dn.DN_ERR_INVALID),
+    (dict(dtype=5), dn.DN_ERR_INVALID),
+    (dict(path=9), dn.DN_ERR_INVALID),
+    (dict(chunk=0), dn.DN_ERR_INVALID),
+    (dict(scale=float("nan")), dn.DN_ERR_INVALID),
+    (dict(q=A + 8), dn.DN_ERR_INVALID),                       # not 16-byte aligned
+    (dict(beta=A + 3 * STEP + 2), dn.DN_ERR_INVALID),         # not 4-byte aligned
+    (dict(gate=2, g=A + 4 * STEP + 4), dn.DN_ERR_INVALID),    # per-key g not 16-byte aligned
+    (dict(o=A + 64), dn.DN_ERR_INVALID),                      # o overlaps q
+    (dict(S_T=A + 2 * STEP), dn.DN_ERR_INVALID),              # S_T overlaps v
+    (dict(S0=A + 7 * STEP, S_T=A + 7 * STEP + 256), dn.DN_ERR_INVALID),  # partial overlap
+    (dict(dk=96), dn.DN_ERR_UNSUPPORTED),
+    (dict(dv=256), dn.DN_ERR_UNSUPPORTED),
+])
+def test_chunk_fwd_rejects(lib, over, code):
+    assert chunk_call(lib, **over) == code
+    assert lib.dn_last_error() != b""
+
+
+def test_chunk_fwd_empty_batch_is_ok_without_device(lib):
+    assert chunk_call(lib, B=0) == dn.DN_OK
+    assert chunk_call(lib, H=0, q=None, k=None, v=None, beta=None, g=None, o=None) == dn.DN_OK
+
+
+def decode_call(lib, **over):
+    args = dict(q=A, k=A + STEP, v=A + 2 * STEP, beta=A + 3 * STEP, g=A + 4 * STEP,
+                S=A + 5 * STEP, o=A + 6 * STEP, B=2, H=3, dk=128, dv=128, scale=1.0, dtype=1, gate=1)
+    args.update(over)
+    return lib.dn_decode_step(args["q"], args["k"], args["v"], args["beta"], args["g"], args["S"],
+                              args["o"], args["B"], args["H"], args["dk"], args["dv"], args["scale"],
+                              args["dtype"], args["gate"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=-2), dn.DN_ERR_INVALID),
+    (dict(S=None), dn.DN_ERR_INVALID),
+    (dict(g=None), dn.DN_ERR_INVALID),
+    (dict(o=A + 5 * STEP + 4096), dn.DN_ERR_INVALID),         # o inside S
+    (dict(S=A + 32), dn.DN_ERR_INVALID),                      # S overlaps q
+    (dict(k=A + STEP + 4), dn.DN_ERR_INVALID),
+    (dict(dk=32), dn.DN_ERR_UNSUPPORTED),
+])
+def test_decode_rejects(lib, over, code):
+    assert decode_call(lib, **over) == code
+
+
+def test_decode_empty_is_ok(lib):
+    assert decode_call(lib, B=0) == dn.DN_OK
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 1, 8, 64)
+    with pytest.raises(ValueError):
+        dn.dn_chunk_fwd(q, q, q, torch.zeros(1, 1, 8), None, None, torch.zeros(1, 1, 8, 64), None)

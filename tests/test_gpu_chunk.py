@@ -1,0 +1,205 @@
+"""Chunked prefill on the GPU against the fp64 oracle ("Linear attention and
+Gated DeltaNet", ch. 28, "The chunked form": same contract and result as the
+recurrent form; its test plan: chunk sizes 1, 5, 8 and 64 on 37 tokens with a
+non-zero initial state, because a chunk size of 1 hides a wrong triangle)."""
+import numpy as np
+import pytest
+import torch
+
+import delta_rule_recurrent_02_b200 as dn
+import oracle
+from delta_rule_recurrent_02_b200 import workloads as W
+from _util import TOL, assert_close, f64, oracle_prefill, pick, to_dev
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["simt"]
+
+
+def run(d, scale, chunk=64, path="simt", gate=None):
+    return dn.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], chunk=chunk,
+                        scale=scale, path=path, gate=gate)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+@pytest.mark.parametrize("chunk", [1, 5, 8, 16, 64])
+@pytest.mark.parametrize("d", [64, 128])
+def test_chunk_t37_nonzero_state(cuda_device, dtype, gate, chunk, d):
+    inp = W.gen_prefill(2, 3, 37, d, d, dtype=dtype, gate=gate, seed=100 + chunk, s0_std=0.5,
+                        g_shift=0.5)
+    sc = d ** -0.5
+    o, S = run(to_dev(inp), sc, chunk=chunk, path="simt")
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(o, ro, dtype, "o")
+    assert_close(S, rS, dtype, "S_T")
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 517])
+@pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
+def test_chunk_ragged_lengths(cuda_device, path, T, gate):
+    inp = W.gen_prefill(2, 2, T, 128, 128, dtype="bf16", gate=gate, seed=T, s0_std=0.1)
+    sc = 128 ** -0.5
+    o, S = run(to_dev(inp), sc, path=path)
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(S, rS, "bf16", "S_T")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_worked_example(cuda_device, path):
+    # ch. 28 worked example, embedded at d = 128 (and 64 for SIMT): exact
+    dims = [128] if path == "tc" else [64, 128]
+    dts = [torch.bfloat16] if path == "tc" else [torch.float32, torch.bfloat16]
+    for d in dims:
+        for td in dts:
+            q = torch.zeros(1, 1, 2, d, dtype=td, device="cuda"); q[0, 0, :, 0] = 1
+            v = torch.zeros(1, 1, 2, d, dtype=td, device="cuda"); v[0, 0, :, 0] = 2; v[0, 0, :, 1] = 4
+            beta = torch.tensor([[[0.5, 1.0]]], device="cuda")
+            o, S = dn.chunk_fwd(q, q, v, beta, None, None, path=path)
+            assert o[0, 0, 0, :2].float().tolist() == [1.0, 2.0]
+            assert o[0, 0, 1, :2].float().tolist() == [2.0, 4.0]
+            assert torch.count_nonzero(o[0, 0, :, 2:]) == 0
+            assert S[0, 0, 0, :2].tolist() == [2.0, 4.0] and torch.count_nonzero(S) == 2
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T", [8, 24, 64, 200])
+def test_chunk_reflection_parity_exact(cuda_device, path, T):
+    # D2L 12.5, "The reflection hiding in the delta rule": k = e_1, S0 = e_1 e_1^T,
+    # v = 0, beta_t = 2 x_t, q = e_1: o_t[0] = (-1)^(x_1 + ... + x_t), exactly.
+    d = 128
+    gen = torch.Generator().manual_seed(T)
+    x = torch.randint(0, 2, (T,), generator=gen)
+    td = torch.bfloat16
+    k = torch.zeros(1, 1, T, d, dtype=td); k[..., 0] = 1
+    v = torch.zeros(1, 1, T, d, dtype=td)
+    S0 = torch.zeros(1, 1, d, d); S0[0, 0, 0, 0] = 1
+    beta = (2.0 * x).float().reshape(1, 1, T)
+    o, S = dn.chunk_fwd(k.cuda(), k.cuda(), v.cuda(), beta.cuda(), None, S0.cuda(), path=path)
+    want = (-1.0) ** torch.cumsum(x, 0).double()
+    assert torch.equal(o[0, 0, :, 0].double().cpu(), want)
+    assert torch.count_nonzero(o[0, 0, :, 1:]) == 0
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_chunk_beta_zero_pure_decay(cuda_device, path, gate):
+    # beta = 0: o_t = (Diag(e^Gamma_t) S0)^T (scale q_t), S_T = Diag(e^Gamma_T) S0.
+    # A mild decay (g ~ -softplus(N(0,1) - 1)) keeps e^Gamma_T inside the fp32 range.
+    inp = W.gen_prefill(1, 2, 100, 128, 128, dtype="bf16", gate=gate, seed=7, s0_std=0.1, g_shift=-1.0)
+    inp["beta"].zero_()
+    sc = 128 ** -0.5
+    o, S = run(to_dev(inp), sc, path=path)
+    g = f64(inp["g"])
+    lg = np.repeat(g[..., None], 128, -1) if g.ndim == 3 else g
+    Gam = np.cumsum(lg, axis=2)
+    want_o = np.einsum("bhtc,bhcj,bhtc->bhtj", np.exp(Gam), f64(inp["S0"]), sc * f64(inp["q"]))
+    assert_close(o, want_o, "bf16", "o")
+    assert_close(S, np.exp(Gam[:, :, -1])[..., None] * f64(inp["S0"]), "f32", "S_T")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_resume_through_state(cuda_device, path):
+    inp = W.gen_prefill(2, 4, 300, 128, 128, dtype="bf16", gate="scalar", seed=9, s0_std=0.1)
+    d = to_dev(inp)
+    sc = 128 ** -0.5
+    o, S = run(d, sc, path=path)
+    cut = 128
+    first = {n: (None if t is None or n == "S0" else t[:, :, :cut].contiguous()) for n, t in d.items()}
+    first["S0"] = d["S0"]
+    second = {n: (None if t is None or n == "S0" else t[:, :, cut:].contiguous()) for n, t in d.items()}
+    o1, S1 = run(first, sc, path=path)
+    second["S0"] = S1
+    o2, S2 = run(second, sc, path=path)
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(torch.cat([o1, o2], dim=2), ro, "bf16", "o (resumed)")
+    assert_close(S2, rS, "bf16", "S_T (resumed)")
+    # in-place continuation: S_T may be the same buffer as S0
+    S_inplace = S1.clone()
+    dn.dn_chunk_fwd(second["q"], second["k"], second["v"], second["beta"], second["g"], S_inplace,
+                    torch.empty_like(o2), S_inplace, scale=sc, path=path)
+    assert_close(S_inplace, rS, "bf16", "S_T (in place)")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_overwrites_poisoned_outputs(cuda_device, path):
+    inp = W.gen_prefill(2, 3, 130, 128, 128, dtype="bf16", gate="scalar", seed=11)
+    d = to_dev(inp)
+    o = torch.full((2, 3, 130, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    S = torch.full((2, 3, 128, 128), float("nan"), device="cuda")
+    dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], None, o, S, scale=0.1, path=path)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+
+
+def test_chunk_empty_inputs(cuda_device):
+    # T = 0: no output rows; S_T = S0 (or zeros).  B = 0: nothing at all.
+    S0 = torch.randn(2, 3, 64, 64, device="cuda")
+    z = lambda *s, dt=torch.float32: torch.zeros(*s, dtype=dt, device="cuda")
+    S_T = torch.full_like(S0, float("nan"))
+    dn.dn_chunk_fwd(z(2, 3, 0, 64), z(2, 3, 0, 64), z(2, 3, 0, 64), z(2, 3, 0), None, S0,
+                    z(2, 3, 0, 64), S_T, chunk=16)
+    assert torch.equal(S_T, S0)
+    dn.dn_chunk_fwd(z(2, 3, 0, 64), z(2, 3, 0, 64), z(2, 3, 0, 64), z(2, 3, 0), None, None,
+                    z(2, 3, 0, 64), S_T, chunk=16)
+    assert torch.count_nonzero(S_T) == 0
+    o, S = dn.chunk_fwd(z(0, 3, 5, 64), z(0, 3, 5, 64), z(0, 3, 5, 64), z(0, 3, 5), None, None)
+    assert o.shape == (0, 3, 5, 64)
+
+
+def test_chunk_errors_on_device(cuda_device):
+    q = torch.zeros(1, 1, 8, 64, device="cuda")
+    beta = torch.zeros(1, 1, 8, device="cuda")
+    with pytest.raises(dn.DNError) as ei:
+        dn.chunk_fwd(q, q, q, beta, None, None, chunk=65, path="simt")
+    assert ei.value.status == dn.DN_ERR_UNSUPPORTED
+    with pytest.raises(dn.DNError) as ei:
+        dn.chunk_fwd(q, q, q, beta, None, None, path="tc")   # fp32 is not on the tensor-core path
+    assert ei.value.status == dn.DN_ERR_UNSUPPORTED
+    with pytest.raises(dn.DNError) as ei:
+        dn.chunk_fwd(q, q, q, beta, None, None, gate="scalar")   # gate without g
+    assert ei.value.status == dn.DN_ERR_INVALID
+
+
+# --- the five workloads at full size -----------------------------------------
+
+def test_deltanet_small_full(cuda_device):
+    cfg = W.DELTANET_SMALL
+    inp = W.gen_prefill_config(cfg)
+    o, S = run(to_dev(inp), cfg.scale, chunk=cfg.chunk, path="simt")
+    ro, rS = oracle_prefill(inp, cfg.scale)
+    assert_close(o, ro, "f32", "o")
+    assert_close(S, rS, "f32", "S_T")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_gated_deltanet_full(cuda_device, path):
+    cfg = W.GDN_PREFILL
+    inp = W.gen_prefill_config(cfg)
+    o, S = run(to_dev(inp), cfg.scale, chunk=cfg.chunk, path=path)
+    ro, rS = oracle_prefill(inp, cfg.scale)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(S, rS, "bf16", "S_T")
+
+
+def _sampled(cfg, path, n_heads, seed):
+    inp = W.gen_prefill_config(cfg)
+    o, S = run(to_dev(inp), cfg.scale, chunk=cfg.chunk, path=path)
+    gen = torch.Generator().manual_seed(seed)
+    flat = torch.randperm(cfg.B * cfg.H, generator=gen)[:n_heads].tolist()
+    bh = [(f // cfg.H, f % cfg.H) for f in flat]
+    ro, rS = oracle_prefill(inp, cfg.scale, bh=bh)
+    assert_close(pick(o.cpu(), bh), ro, "bf16", "o (sampled heads)")
+    assert_close(pick(S.cpu(), bh), rS, "bf16", "S_T (sampled heads)")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_gated_deltanet_long_sampled(cuda_device, path):
+    _sampled(W.GDN_LONG, path, n_heads=4, seed=1)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_kda_sampled(cuda_device, path):
+    _sampled(W.KDA_PREFILL, path, n_heads=8, seed=2)
