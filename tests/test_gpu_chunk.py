@@ -13,7 +13,14 @@ from _util import TOL, assert_close, f64, oracle_prefill, pick, to_dev
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["simt"]
+PATHS = ["simt", "tc"]
+# the tensor-core path covers bf16, chunk 64, d_k = d_v = 128 and the none / scalar gates
+TC_GATES = ("none", "scalar")
+
+
+def skip_unsupported(path, gate):
+    if path == "tc" and gate not in TC_GATES:
+        pytest.skip("per-key gate runs on the SIMT path")
 
 
 def run(d, scale, chunk=64, path="simt", gate=None):
@@ -39,6 +46,7 @@ def test_chunk_t37_nonzero_state(cuda_device, dtype, gate, chunk, d):
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 517])
 @pytest.mark.parametrize("gate", ["none", "scalar", "per_key"])
 def test_chunk_ragged_lengths(cuda_device, path, T, gate):
+    skip_unsupported(path, gate)
     inp = W.gen_prefill(2, 2, T, 128, 128, dtype="bf16", gate=gate, seed=T, s0_std=0.1)
     sc = 128 ** -0.5
     o, S = run(to_dev(inp), sc, path=path)
@@ -86,6 +94,7 @@ def test_chunk_reflection_parity_exact(cuda_device, path, T):
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("gate", ["scalar", "per_key"])
 def test_chunk_beta_zero_pure_decay(cuda_device, path, gate):
+    skip_unsupported(path, gate)
     # beta = 0: o_t = (Diag(e^Gamma_t) S0)^T (scale q_t), S_T = Diag(e^Gamma_T) S0.
     # A mild decay (g ~ -softplus(N(0,1) - 1)) keeps e^Gamma_T inside the fp32 range.
     inp = W.gen_prefill(1, 2, 100, 128, 128, dtype="bf16", gate=gate, seed=7, s0_std=0.1, g_shift=-1.0)
@@ -200,6 +209,5 @@ def test_gated_deltanet_long_sampled(cuda_device, path):
     _sampled(W.GDN_LONG, path, n_heads=4, seed=1)
 
 
-@pytest.mark.parametrize("path", PATHS)
-def test_kda_sampled(cuda_device, path):
-    _sampled(W.KDA_PREFILL, path, n_heads=8, seed=2)
+def test_kda_sampled(cuda_device):
+    _sampled(W.KDA_PREFILL, "auto", n_heads=8, seed=2)
