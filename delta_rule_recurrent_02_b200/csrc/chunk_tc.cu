@@ -8,33 +8,34 @@
 //   A   = strict_tril(beta_i k_i.k_j D_ij),     T = (I + A)^-1      (UT transform)
 //   W   = T diag(beta e^G) K,                   u = T diag(beta) V
 //   U   = u - W S                                (values actually written)
-//   O   = scale (e^G * Q) S + P U,              P = scale tril(Q K^T * D)
+//   O   = Qh S + P U,   Qh = scale e^G * Q,     P = scale tril(Q K^T * D)
 //   S  <- e^(G_last) S + (K * e^(G_last - G))^T U
 //
-// Every product is issued as tcgen05.mma (bf16 operands in shared memory,
-// fp32 accumulators in TMEM) with M = 128 by computing the transposed
-// products: the d_v (or d_k) dimension is the MMA's M, the chunk is its N.
+// Every product runs as tcgen05.mma with M = 128 by computing the transposed
+// products (the d_v or d_k dimension is the MMA's M, the chunk is its N):
 //
-//   gram   [K;Q] K^T          M=128 (64 key rows, 64 query rows) N=64  K=d_k
-//   W^T  = K^T (T diag(beta e^G))^T                      M=d_k  N=64   K=64
-//   u^T  = V^T (T diag(beta))^T                          M=d_v  N=64   K=64
-//   U^T  = u^T - S^T W^T                                 M=d_v  N=64   K=d_k
-//   O1^T = S^T Q^T                                       M=d_v  N=64   K=d_k
-//   dS^T = U^T (K * e^(G_last - G))                      M=d_v  N=d_k  K=64
-//   O2^T = U^T P^T                                       M=d_v  N=64   K=64
+//   gram   [K;Q] K^T       A = K,Q tiles (smem)    B = K tile            -> TMEM G
+//   W^T  = K^T Tw^T        A = K tile (MN-major)   B = T diag(beta e^G)  -> TMEM W
+//   u^T  = V^T Tb^T        A = V tile (MN-major)   B = T diag(beta)      -> TMEM U
+//   U^T += -S^T W^T        A = S^T (TMEM, bf16)    B = W^T (smem)        -> TMEM U
+//   O^T  = S^T Qh^T        A = S^T (TMEM, bf16)    B = Qh (smem)         -> TMEM O
+//   S^T += U^T K~          A = U^T (TMEM, bf16)    B = K~ (smem)         -> TMEM S
+//   O^T += U^T P^T         A = U^T (TMEM, bf16)    B = P (smem)          -> TMEM O
 //
-// The fp32 state lives in registers (thread = one value column j, one half of
-// the key channels) and a bf16 copy S^T in shared memory feeds the MMAs; the
-// 64 x 64 unit-lower system is inverted in fp32 on the CUDA cores (blocked:
-// 16 x 16 diagonal inverses by forward substitution, then the off-diagonal
-// blocks by block products).  q, k and v tiles arrive by TMA (128-byte
-// swizzle) into a double-buffered stage, prefetched two chunks ahead.
+// The CTA owns one (b, h) and runs two pipelines that overlap:
+//   * the chunk-parallel "prework" of chunk c+1 (gram -> masks -> 64 x 64
+//     unit-lower inverse on the CUDA cores -> W, u, Qh, K~, P), and
+//   * the sequential state chain of chunk c (U, S, O), whose state stays in
+//     TMEM (fp32 accumulator, pre-scaled by the next chunk's decay) with a
+//     bf16 copy in TMEM that feeds the next products directly.
+// Warp roles: 0 TMA + gate precompute, 1 prework MMA issue, 2 TMEM allocation,
+// 3 state-chain MMA issue, 4-11 prework, 12-15 state chain and output.  Stages of q, k, v tiles arrive
+// by TMA (128-byte swizzle) two chunks ahead.
 //
-// One CTA owns one (b, h) for the whole sequence.  A partial last chunk is
-// handled by treating rows >= Cc as beta = 0, g = 0 (rows past the tensor's
-// end are zero-filled by TMA; rows of the next head are masked out), which
-// equals zero padding.  Every wait on an mbarrier is bounded; on a timeout
-// the kernel records it in the status word, drains its own copies and exits.
+// A partial last chunk treats rows >= Cc as beta = 0, g = 0 (rows past the
+// tensor's end are zero-filled by TMA; rows of the next head are masked),
+// which equals zero padding.  Every wait is bounded: on a timeout the kernel
+// records it in the status word, lets its own copies land and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -51,28 +52,125 @@ namespace {
 
 constexpr int kC = 64;          // chunk
 constexpr int kD = 128;         // d_k = d_v
-constexpr int kNT = 256;        // 8 warps: two warpgroups
-// TMEM columns (fp32, 128 lanes)
-constexpr uint32_t TM_G = 0, TM_W = 64, TM_U = 128, TM_O1 = 192, TM_O2 = 256, TM_S = 320;
+constexpr int kNT = 512;        // 16 warps
+constexpr int kPreWarp0 = 4;    // prework warps 4..11
+constexpr int kPreThreads = 256;
+constexpr int kChainWarp0 = 12; // chain warps 12..15
+constexpr int kChainThreads = 128;
+
+// TMEM columns (32-bit, 128 lanes)
+constexpr uint32_t TM_SACC = 0;     // S^T fp32 [dv lanes][dk cols], pre-scaled by the coming chunk's decay
+constexpr uint32_t TM_ST = 128;     // S^T bf16 pairs [dv][dk/2]
+constexpr uint32_t TM_UT = 192;     // U^T bf16 pairs [dv][C/2]
+constexpr uint32_t TM_U = 224;      // U^T fp32 accumulator [dv][C]
+constexpr uint32_t TM_O = 288;      // O^T fp32 accumulator [dv][C]
+constexpr uint32_t TM_G = 352;      // gram: lanes 0-63 K K^T, 64-127 Q K^T
+constexpr uint32_t TM_W = 416;      // W^T fp32 [dk][C]
 constexpr uint32_t TM_COLS = 512;
+
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;          // 2 stages x 32 KiB: [d-block][K rows 0-63 | Q rows 64-127][128 B]
 constexpr uint32_t SZ_KQ = 32768;
 constexpr uint32_t OFF_V = 65536;       // 2 stages x 16 KiB: [d-block][64 rows][128 B]
 constexpr uint32_t SZ_V = 16384;
-constexpr uint32_t OFF_ST = 98304;      // S^T bf16, K-major A: [c-block][128 rows j][128 B]   32 KiB
-constexpr uint32_t OFF_UT = 131072;     // U^T bf16, K-major A: [128 rows][128 B]; fp32 A during the solve
-constexpr uint32_t OFF_WT = 147456;     // W^T bf16, MN-major B: [128 rows c][128 B]; fp32 T during the solve
-constexpr uint32_t OFF_KT = 163840;     // K * e^(G_last - G), MN-major B: [c-block][64 rows][128 B]
-constexpr uint32_t OFF_TW = 180224;     // T diag(beta e^G), K-major B [64 rows i][128 B]
-constexpr uint32_t OFF_TB = 188416;     // T diag(beta)
-constexpr uint32_t OFF_PM = 196608;     // P, K-major B [64 rows i][128 B]
-constexpr uint32_t OFF_MISC = 204800;   // gates, barriers, TMEM slot, flags
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 2048 + 1024;
-constexpr uint32_t STAGE_TX = 6 * 8192; // six 64 x 64 bf16 boxes per stage
+constexpr uint32_t OFF_QH = 98304;      // Qh, K-major B [N=i][K=c]: [c-block][64 rows][128 B]
+constexpr uint32_t OFF_WT = 114688;     // W^T, MN-major B [K=c rows][N=i]: [128 rows][128 B]
+constexpr uint32_t OFF_KT = 131072;     // 2 x K~, MN-major B [K=j rows][N=c]: [c-block][64 rows][128 B]
+constexpr uint32_t OFF_PM = 163840;     // 2 x P, K-major B [N=i][K=j]: [64 rows][128 B]
+constexpr uint32_t OFF_A = 180224;      // fp32 64 x 68: A, then M = D^-1 A; later Tw (8 KiB) + Tb (8 KiB) bf16
+constexpr uint32_t OFF_T = 197632;      // fp32 64 x 68: T = (I + A)^-1
+constexpr uint32_t OFF_GATE = 215040;   // 4 gate slots
+constexpr uint32_t GATE_FLOATS = 384;
+constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr uint32_t STAGE_TX = 6 * 8192;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
-__device__ __forceinline__ int aidx(int i, int j) { return i * 64 + (j ^ (i & 31)); }
+// gate slot layout (floats)
+constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320;
+
+// barrier indices
+enum {
+    B_FULL0 = 0, B_FULL1, B_FREE0, B_FREE1,              // TMA stages
+    B_GATE0, B_GATE1, B_GATE2, B_GATE3,                  // gate slots
+    B_GRAM, B_WU, B_WSQS, B_KUPU,                        // MMA completions
+    B_TW, B_READY, B_KP0, B_KP1, B_GFREE,                // prework -> MMA
+    B_UT, B_UFREE, B_ST, B_OFREE,                        // chain -> MMA
+    B_COUNT
+};
+
+// fp32 64 x 64 matrix, rows padded to 68 floats: 16-byte aligned rows, and
+// rows r and r + 1 start 4 banks apart (conflict-free row, column and 16 x 16
+// block accesses)
+constexpr int kFS = 68;
+__device__ __forceinline__ int fidx(int i, int j) { return i * kFS + j; }
+
+// acc[e] += sum_m X[xr + ii][xc + m] * Y[yr + m][yc + j0 + e] over a 16 x 16
+// block pair; lane -> (ii = lane / 2, j0 = 8 (lane % 2)).
+__device__ __forceinline__ void blk16(const float* X, int xr, int xc, const float* Y, int yr, int yc,
+                                      float (&acc)[8], int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    float xrow[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(X + fidx(xr + ii, xc + 4 * q));
+        xrow[4 * q + 0] = v.x; xrow[4 * q + 1] = v.y; xrow[4 * q + 2] = v.z; xrow[4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const float4 a = *reinterpret_cast<const float4*>(Y + fidx(yr + m, yc + j0));
+        const float4 b = *reinterpret_cast<const float4*>(Y + fidx(yr + m, yc + j0 + 4));
+        acc[0] += xrow[m] * a.x; acc[1] += xrow[m] * a.y; acc[2] += xrow[m] * a.z; acc[3] += xrow[m] * a.w;
+        acc[4] += xrow[m] * b.x; acc[5] += xrow[m] * b.y; acc[6] += xrow[m] * b.z; acc[7] += xrow[m] * b.w;
+    }
+}
+
+__device__ __forceinline__ void blk16_store(float* Z, int zr, int zc, const float (&acc)[8], float sign, int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    *reinterpret_cast<float4*>(Z + fidx(zr + ii, zc + j0)) =
+        make_float4(sign * acc[0], sign * acc[1], sign * acc[2], sign * acc[3]);
+    *reinterpret_cast<float4*>(Z + fidx(zr + ii, zc + j0 + 4)) =
+        make_float4(sign * acc[4], sign * acc[5], sign * acc[6], sign * acc[7]);
+}
+
+__device__ __forceinline__ void zero8(float (&a)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[e] = 0.f;
+}
+
+// e^(G_i - G_j) = 2^(G2_i - G2_j) with G2 = G log2(e), for j <= i (the
+// exponent is <= 0 for g <= 0; very old positions underflow to 0).
+__device__ __forceinline__ float decay2(float g2i, float g2j) { return exp2f(g2i - g2j); }
+
+// Scale 8 bf16 values (one 16-byte chunk) by f and store them at dst.
+__device__ __forceinline__ void scale_chunk(uint32_t src, uint32_t dst, float f) {
+    const uint4 w = ld_shared_v4(src);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+    st_shared_v4(dst, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+}
+
+struct Ctl {
+    uint32_t bar0;                 // address of barrier 0
+    volatile int* abort;
+    __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
+    // bounded wait; gives up early once another role has aborted
+    __device__ bool wait(int i, uint32_t parity) const {
+        const uint32_t b = bar(i);
+        if (mbar_try_wait(b, parity)) return true;
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+            if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitNs) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+};
 
 }  // namespace
 
@@ -82,121 +180,72 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ beta,
                 const float* __restrict__ g, const float* S0, __nv_bfloat16* __restrict__ o,
                 float* S_T, int T, float scale, unsigned int* status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base, derived from the __shared__ array itself so that
+    // every access below compiles to a shared-memory (not generic) instruction
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
-    float* bs = reinterpret_cast<float*>(sm + OFF_MISC);   // beta (0 past the chunk's end)
-    float* Gs = bs + 64;                                      // inclusive cumulative log-decay
-    float* eGs = Gs + 64;                                     // e^G_i
-    float* eTs = eGs + 64;                                    // e^(G_last - G_i)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_MISC + 1024);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 1024 + 64);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 1024 + 72);
-    float* Am = reinterpret_cast<float*>(sm + OFF_UT);
-    float* Tm = reinterpret_cast<float*>(sm + OFF_WT);
+    float* gates = reinterpret_cast<float*>(sm + OFF_GATE);
+    float* Am = reinterpret_cast<float*>(sm + OFF_A);
+    float* Tm = reinterpret_cast<float*>(sm + OFF_T);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 8 * B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + 8 * B_COUNT + 8);
+    Ctl ctl{sb + OFF_BAR, abort_flag};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wg = warp >> 2;                              // warpgroup: which half of the columns
-    const int row = ((warp & 3) << 5) + lane;              // TMEM lane of this thread
-    const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
     const int64_t bh = blockIdx.x;
-    const int nchunks = (T + kC - 1) / kC;
-    const uint32_t bar_full[2] = {smem_u32(&bars[0]), smem_u32(&bars[1])};
-    const uint32_t bar_mma = smem_u32(&bars[2]);
+    const int n = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        mbar_init(bar_full[0], 1);
-        mbar_init(bar_full[1], 1);
-        mbar_init(bar_mma, 1);
+        const uint32_t counts[B_COUNT] = {1, 1, kPreThreads, kPreThreads, 1, 1, 1, 1, 1, 1, 1, 1,
+                                          kPreThreads, kPreThreads, kPreThreads, kPreThreads, kPreThreads,
+                                          kChainThreads, kChainThreads, kChainThreads, kChainThreads};
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(ctl.bar(i), counts[i]);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
     }
-    if (warp == 0) {
+    if (warp == 2) {
         tmem_alloc(smem_u32(tmem_slot), TM_COLS);
         tmem_relinquish();
     }
-
-    // State: this thread holds S[c][j] for j = row, c = 64 wg + n.
-    float Sreg[64];
-    {
-        const float* src = S0 ? S0 + (bh * kD + wg * 64) * kD + row : nullptr;
-#pragma unroll
-        for (int n = 0; n < 64; ++n) Sreg[n] = src ? src[(int64_t)n * kD] : 0.f;
-        const uint32_t st = sb + OFF_ST + wg * 16384;
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8)
-            st_shared_v4(st + sw128_off(row, q8),
-                         pack_bf16x2(Sreg[8 * q8 + 0], Sreg[8 * q8 + 1]), pack_bf16x2(Sreg[8 * q8 + 2], Sreg[8 * q8 + 3]),
-                         pack_bf16x2(Sreg[8 * q8 + 4], Sreg[8 * q8 + 5]), pack_bf16x2(Sreg[8 * q8 + 6], Sreg[8 * q8 + 7]));
-    }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto issue = [&](int cc) {
-        const int s = cc & 1;
-        const int y = (int)(bh * T + (int64_t)cc * kC);
-        const uint32_t kq = sb + OFF_KQ + s * SZ_KQ, vv = sb + OFF_V + s * SZ_V;
-        mbar_arrive_expect_tx(bar_full[s], STAGE_TX);
-        tma_load_2d(kq + 0, &tm_k, 0, y, bar_full[s]);
-        tma_load_2d(kq + 16384, &tm_k, 64, y, bar_full[s]);
-        tma_load_2d(kq + 8192, &tm_q, 0, y, bar_full[s]);
-        tma_load_2d(kq + 24576, &tm_q, 64, y, bar_full[s]);
-        tma_load_2d(vv + 0, &tm_v, 0, y, bar_full[s]);
-        tma_load_2d(vv + 8192, &tm_v, 64, y, bar_full[s]);
-    };
-    int issued = 0;      // chunks whose loads were issued (leader only)
-    if (tid == 0) {
-        issue(0);
-        issued = 1;
-        if (nchunks > 1) { issue(1); issued = 2; }
-    }
-
-    // gate values of the next chunk, prefetched by warp 0
-    float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
-    auto fetch_gates = [&](int cc) {
-        const int64_t t0 = bh * T + (int64_t)cc * kC;
-        const int Cn = min(kC, T - cc * kC);
-        nb0 = lane < Cn ? beta[t0 + lane] : 0.f;
-        nb1 = lane + 32 < Cn ? beta[t0 + lane + 32] : 0.f;
-        if (GATE == kGateScalar) {
-            ng0 = lane < Cn ? g[t0 + lane] : 0.f;
-            ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
+    if (warp == 0) {
+        // ================= producer: gates + TMA ================================
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
         }
-    };
-    if (warp == 0) fetch_gates(0);
-
-    uint32_t mma_phase = 0;
-    bool good = true;
-    auto wait_mma = [&]() {
-        good &= mbar_wait_bounded(bar_mma, mma_phase, kWaitNs);
-        mma_phase ^= 1u;
-        tc_fence_after();
-    };
-    // barrier that also spreads a timeout to every thread; returns true to stop
-    auto sync_check = [&]() -> bool {
-        if (!good) *abort_flag = 1;
-        __syncthreads();
-        return *abort_flag != 0;
-    };
-
-    int c = 0;
-    for (; c < nchunks; ++c) {
-        const int s = c & 1;
-        const int c0 = c * kC;
-        const int Cc = min(kC, T - c0);
-        const uint32_t KQ = sb + OFF_KQ + s * SZ_KQ;
-        const uint32_t VS = sb + OFF_V + s * SZ_V;
-
-        // ---- gates of this chunk (warp 0) ----------------------------------
-        if (warp == 0) {
-            float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
-            if (c + 1 < nchunks) fetch_gates(c + 1);
+        int issued = 0;
+        // beta / g of the next chunk, loaded one chunk ahead
+        float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
+        auto fetch = [&](int cc) {
+            const int64_t t0 = bh * T + (int64_t)cc * kC;
+            const int Cn = min(kC, T - cc * kC);
+            nb0 = lane < Cn ? beta[t0 + lane] : 0.f;
+            nb1 = lane + 32 < Cn ? beta[t0 + lane + 32] : 0.f;
+            if (GATE == kGateScalar) {
+                ng0 = lane < Cn ? g[t0 + lane] : 0.f;
+                ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
+            }
+        };
+        fetch(0);
+        for (int cc = 0; cc < n; ++cc) {
+            const int s = cc & 1;
+            if (cc >= 2) {
+                bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - 2) >> 1) & 1u) : true;
+                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+            }
+            // gates of chunk cc into slot cc % 4
+            float* gs = gates + (cc & 3) * GATE_FLOATS;
+            const int64_t t0 = bh * T + (int64_t)cc * kC;
+            const float b0 = nb0, b1 = nb1;
+            float a0 = ng0, a1 = ng1;
+            if (cc + 1 < n) fetch(cc + 1);
 #pragma unroll
             for (int o2 = 1; o2 < 32; o2 <<= 1) {
                 const float y0 = __shfl_up_sync(0xffffffffu, a0, o2);
@@ -205,276 +254,393 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             a1 += __shfl_sync(0xffffffffu, a0, 31);
             const float Glast = __shfl_sync(0xffffffffu, a1, 31);
-            bs[lane] = b0; bs[lane + 32] = b1;
-            Gs[lane] = a0; Gs[lane + 32] = a1;
-            eGs[lane] = expf(a0); eGs[lane + 32] = expf(a1);
-            eTs[lane] = expf(Glast - a0); eTs[lane + 32] = expf(Glast - a1);
-        }
-        // ---- gram: [K;Q] K^T -------------------------------------------------
-        // every thread observes the stage's TMA completion (it reads the K tile below)
-        good &= mbar_wait_bounded(bar_full[s], (uint32_t)(c >> 1) & 1u, kWaitNs);
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(tmem + TM_G, sw128_desc(a, 16, 1024), sw128_desc(a, 16, 1024),
-                         idesc_bf16(128, 64, 0, 0), kk > 0);
+            const float L2E = 1.4426950408889634f;
+            gs[G_BETA + lane] = b0; gs[G_BETA + lane + 32] = b1;
+            gs[G_G2 + lane] = a0 * L2E; gs[G_G2 + lane + 32] = a1 * L2E;
+            const float e0 = expf(a0), e1 = expf(a1);
+            gs[G_EG + lane] = e0; gs[G_EG + lane + 32] = e1;
+            gs[G_BEG + lane] = b0 * e0; gs[G_BEG + lane + 32] = b1 * e1;
+            gs[G_ET + lane] = expf(Glast - a0); gs[G_ET + lane + 32] = expf(Glast - a1);
+            if (lane == 0) gs[G_GAMMA] = expf(Glast);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+                const int y = (int)t0;
+                const uint32_t kq = sb + OFF_KQ + s * SZ_KQ, vv = sb + OFF_V + s * SZ_V;
+                const uint32_t fb = ctl.bar(B_FULL0 + s);
+                mbar_arrive_expect_tx(fb, STAGE_TX);
+                tma_load_2d(kq + 0, &tm_k, 0, y, fb);
+                tma_load_2d(kq + 16384, &tm_k, 64, y, fb);
+                tma_load_2d(kq + 8192, &tm_q, 0, y, fb);
+                tma_load_2d(kq + 24576, &tm_q, 64, y, fb);
+                tma_load_2d(vv + 0, &tm_v, 0, y, fb);
+                tma_load_2d(vv + 8192, &tm_v, 64, y, fb);
             }
-            mma_commit(bar_mma);
+            issued = cc + 1;
         }
-        if (sync_check()) break;
-        wait_mma();
-        {
-            float r[32];
-            tmem_ld32(tmem + lane_off + TM_G + wg * 32, r);
-            tmem_wait_ld();
-            const int jb = wg * 32;
-            if (row < 64) {                     // K K^T rows -> A (fp32)
-                const int i = row;
-                const float bi = bs[i], Gi = Gs[i];
+        if (*abort_flag && lane == 0) {
+            // let every load this CTA issued land before its shared memory is released
+            for (int cc = max(0, issued - 2); cc < issued; ++cc)
+                mbar_wait_bounded(ctl.bar(B_FULL0 + (cc & 1)), (uint32_t)(cc >> 1) & 1u, kWaitNs);
+        }
+    } else if (warp == 1 || warp == 3) {
+        // ================= MMA issue: warp 1 lane 0 the prework products (gram, W, u),
+        // warp 3 lane 0 the state-chain products; each commits its own MMAs =====
+        if (lane == 0) {
+            const uint32_t I_GRAM = idesc_bf16(128, 64, 0, 0);
+            const uint32_t I_MNK = idesc_bf16(128, 64, 1, 0);       // A MN-major, B K-major
+            const uint32_t I_WS = idesc_bf16(128, 64, 0, 1, 1);     // -A, B MN-major
+            const uint32_t I_KK = idesc_bf16(128, 64, 0, 0);
+            const uint32_t I_KU = idesc_bf16(128, 128, 0, 1);
+            bool ok = true;
+            if (warp == 1) {
+                for (int c = 0; ok && c < n; ++c) {
+                    const uint32_t par = (uint32_t)c & 1u;
+                    // [K;Q] K^T once the stage has landed and the previous gram was read
+                    ok = ctl.wait(B_FULL0 + (c & 1), (uint32_t)(c >> 1) & 1u) && (c == 0 || ctl.wait(B_GFREE, par ^ 1u));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t kq = sb + OFF_KQ + (c & 1) * SZ_KQ, vv = sb + OFF_V + (c & 1) * SZ_V;
 #pragma unroll
-                for (int n = 0; n < 32; ++n) {
-                    const int j = jb + n;
-                    float a = 0.f;
-                    if (j < i && i < Cc) a = bi * r[n] * expf(Gi - Gs[j]);
-                    Am[aidx(i, j)] = a;
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t a = kq + (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_bf16(tmem + TM_G, sw128_desc(a, 16, 1024), sw128_desc(a, 16, 1024), I_GRAM, kk > 0);
+                    }
+                    mma_commit(ctl.bar(B_GRAM));
+                    // W^T = K^T Tw^T and u^T = V^T Tb^T once T is ready and U was read
+                    ok = ctl.wait(B_TW, par) && (c == 0 || ctl.wait(B_UFREE, par ^ 1u));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + TM_W, sw128_desc(kq + kk * 2048, 16384, 1024),
+                                 sw128_desc(sb + OFF_A + kk * 32, 16, 1024), I_MNK, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + TM_U, sw128_desc(vv + kk * 2048, 8192, 1024),
+                                 sw128_desc(sb + OFF_A + 8192 + kk * 32, 16, 1024), I_MNK, kk > 0);
+                    mma_commit(ctl.bar(B_WU));
                 }
-            } else {                            // Q K^T rows -> P (bf16)
-                const int i = row - 64;
-                const float Gi = Gs[i];
-                float p[32];
+            } else {
+                for (int c = 0; ok && c < n; ++c) {
+                    const uint32_t par = (uint32_t)c & 1u;
+                    // U^T += -S^T W^T ; O^T = S^T Qh^T
+                    ok = ctl.wait(B_READY, par) && ctl.wait(B_ST, par) && (c == 0 || ctl.wait(B_OFREE, par ^ 1u));
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int n = 0; n < 32; ++n) {
-                    const int j = jb + n;
-                    p[n] = (j <= i && i < Cc) ? scale * r[n] * expf(Gi - Gs[j]) : 0.f;
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + TM_U, tmem + TM_ST + kk * 8,
+                                    sw128_desc(sb + OFF_WT + kk * 2048, 8192, 1024), I_WS, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_ST + kk * 8,
+                                    sw128_desc(sb + OFF_QH + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), I_KK,
+                                    kk > 0);
+                    mma_commit(ctl.bar(B_WSQS));
+                    // S^T += U^T K~ ; O^T += U^T P^T
+                    ok = ctl.wait(B_UT, par) && ctl.wait(B_KP0 + (c & 1), (uint32_t)(c >> 1) & 1u);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t kt = sb + OFF_KT + (c & 1) * 16384, pm = sb + OFF_PM + (c & 1) * 8192;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + TM_SACC, tmem + TM_UT + kk * 8, sw128_desc(kt + kk * 2048, 8192, 1024),
+                                    I_KU, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tmem + TM_O, tmem + TM_UT + kk * 8, sw128_desc(pm + kk * 32, 16, 1024), I_KK, 1);
+                    mma_commit(ctl.bar(B_KUPU));
                 }
-                const uint32_t pm = sb + OFF_PM;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    st_shared_v4(pm + sw128_off(i, wg * 4 + q4),
-                                 pack_bf16x2(p[8 * q4 + 0], p[8 * q4 + 1]), pack_bf16x2(p[8 * q4 + 2], p[8 * q4 + 3]),
-                                 pack_bf16x2(p[8 * q4 + 4], p[8 * q4 + 5]), pack_bf16x2(p[8 * q4 + 6], p[8 * q4 + 7]));
             }
+            if (!ok) *abort_flag = 1;
         }
-        // K * e^(G_last - G) into the MN-major B tile (same swizzled layout as the TMA tile)
+    } else if (warp >= kPreWarp0 && warp < kChainWarp0) {
+        // ================= prework (256 threads) ================================
+        const int pt = tid - kPreWarp0 * 32;       // 0..255
+        const int pw = warp - kPreWarp0;           // 0..7
+        const int q = warp & 3;                    // TMEM lane quarter
+        const int h = pw >> 2;                     // column half
+        const int r = (q << 5) + lane;             // TMEM lane (row)
+        const uint32_t lane_off = (uint32_t)(q << 5) << 16;
+        for (int c = 0; c < n; ++c) {
+            const int s = c & 1;
+            const uint32_t par = (uint32_t)c & 1u;
+            const int Cc = min(kC, T - c * kC);
+            const float* gs = gates + (c & 3) * GATE_FLOATS;
+            const uint32_t kq = sb + OFF_KQ + s * SZ_KQ;
+            bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) && ctl.wait(B_GRAM, par) &&
+                      ctl.wait(B_FULL0 + s, (uint32_t)(c >> 1) & 1u);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(1, kPreThreads, !ok)) break;
+            tc_fence_after();
+            // ---- gram rows: A = strict_tril(beta_i (K K^T)_ij D_ij) (fp32, for the solve)
+            //      and P = scale tril((Q K^T)_ij D_ij) (bf16 B tile), rows i < Cc --------
+            {
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_G + h * 32, v);
+                tmem_wait_ld();
+                const float* g2p = gs + G_G2 + h * 32;
+                if (r < 64) {
+                    const int i = r;
+                    const float bi = i < Cc ? gs[G_BETA + i] : 0.f;
+                    const float g2i = gs[G_G2 + i];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int x = tid + u * kNT;            // 0..1023
-            const int blk = x >> 9, t = (x >> 3) & 63, ch = x & 7;
-            const uint4 w = ld_shared_v4(KQ + blk * 16384 + sw128_off(t, ch));
-            const float f = t < Cc ? eTs[t] : 0.f;
-            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-            float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-            float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-            st_shared_v4(sb + OFF_KT + blk * 8192 + sw128_off(t, ch),
-                         pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                         pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
-        }
-        // zero T
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 gj = *reinterpret_cast<const float4*>(g2p + 4 * q4);
+                        const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+                        float a[4];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) Tm[tid + u * kNT] = 0.f;
-        tc_fence_before();
-        if (sync_check()) break;
-
-        // ---- T = (I + A)^-1, blocked ----------------------------------------
-        if (warp < 4 && lane < 16) {            // 16 x 16 diagonal inverses
-            const int k0 = warp * 16, jj = lane;
-            float x[16];
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = h * 32 + q4 * 4 + e;
+                            a[e] = j < i ? bi * v[q4 * 4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                        }
+                        *reinterpret_cast<float4*>(Am + fidx(i, h * 32 + q4 * 4)) = make_float4(a[0], a[1], a[2], a[3]);
+                    }
+                } else {
+                    const int i = r - 64;
+                    const float si = i < Cc ? scale : 0.f;
+                    const float g2i = gs[G_G2 + i];
+                    const uint32_t pm = sb + OFF_PM + (c & 1) * 8192;
 #pragma unroll
-            for (int ii = 0; ii < 16; ++ii) {
-                float acc = (ii == jj) ? 1.f : 0.f;
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 ga = *reinterpret_cast<const float4*>(g2p + 8 * q4);
+                        const float4 gb = *reinterpret_cast<const float4*>(g2p + 8 * q4 + 4);
+                        const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                        float p[8];
 #pragma unroll
-                for (int m = 0; m < ii; ++m) acc -= Am[aidx(k0 + ii, k0 + m)] * x[m];
-                x[ii] = acc;
-            }
-#pragma unroll
-            for (int ii = 0; ii < 16; ++ii) Tm[(k0 + ii) * 64 + k0 + jj] = x[ii];
-        }
-        __syncthreads();
-        {
-            const int ii = tid >> 4, jj = tid & 15;
-            // T_kl = -D_k sum_{m=l}^{k-1} A_km T_ml, by block diagonals d = k - l
-#pragma unroll
-            for (int d = 1; d <= 3; ++d) {
-                float X[3];
-#pragma unroll
-                for (int b = 0; b < 4 - d; ++b) {
-                    const int l = b, k = b + d;
-                    float acc = 0.f;
-                    for (int mb = l; mb < k; ++mb)
-#pragma unroll
-                        for (int m = 0; m < 16; ++m)
-                            acc += Am[aidx(16 * k + ii, 16 * mb + m)] * Tm[(16 * mb + m) * 64 + 16 * l + jj];
-                    X[b] = acc;
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = h * 32 + q4 * 8 + e;
+                            p[e] = j <= i ? si * v[q4 * 8 + e] * decay2(g2i, gjv[e]) : 0.f;
+                        }
+                        st_shared_v4(pm + sw128_off(i, h * 4 + q4), pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
+                                     pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+                    }
                 }
-                __syncthreads();
+            }
+            // ---- K~ = K * e^(G_last - G) (rows >= Cc zero) into this chunk's buffer --------
 #pragma unroll
-                for (int b = 0; b < 4 - d; ++b) Tm[(16 * (b + d) + ii) * 64 + 16 * b + jj] = X[b];
-                __syncthreads();
+            for (int u = 0; u < 4; ++u) {
+                const int x = pt + u * kPreThreads;        // 0..1023
+                const int blk = x >> 9, t = (x >> 3) & 63, ch = x & 7;
+                const float f = t < Cc ? gs[G_ET + t] : 0.f;
+                scale_chunk(kq + blk * 16384 + sw128_off(t, ch),
+                            sb + OFF_KT + (c & 1) * 16384 + blk * 8192 + sw128_off(t, ch), f);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_KP0 + (c & 1)));
+            mbar_arrive(ctl.bar(B_GFREE));
+            named_bar_sync(1, kPreThreads);
+            // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T -------------
+            if (pw < 4 && lane < 16) {
+                const int k0 = pw * 16, jj = lane;
+                float x[16];
 #pragma unroll
-                for (int b = 0; b < 4 - d; ++b) {
-                    const int l = b, k = b + d;
-                    float acc = 0.f;
+                for (int ii = 0; ii < 16; ++ii) {
+                    float p0 = (ii == jj) ? 1.f : 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc += Tm[(16 * k + ii) * 64 + 16 * k + m] * Tm[(16 * k + m) * 64 + 16 * l + jj];
-                    X[b] = -acc;
+                    for (int m = 0; m + 3 < ii; m += 4) {
+                        const float4 av = *reinterpret_cast<const float4*>(Am + fidx(k0 + ii, k0 + m));
+                        p0 -= av.x * x[m]; p1 -= av.y * x[m + 1]; p2 -= av.z * x[m + 2]; p3 -= av.w * x[m + 3];
+                    }
+#pragma unroll
+                    for (int m = ii & ~3; m < ii; ++m) p0 -= Am[fidx(k0 + ii, k0 + m)] * x[m];
+                    x[ii] = (p0 + p1) + (p2 + p3);
                 }
-                __syncthreads();
 #pragma unroll
-                for (int b = 0; b < 4 - d; ++b) Tm[(16 * (b + d) + ii) * 64 + 16 * b + jj] = X[b];
-                __syncthreads();
+                for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
             }
-        }
-        // T diag(beta e^G) and T diag(beta) as bf16 K-major B tiles
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int x = tid + u * kNT;            // 0..511
-            const int i = x >> 3, ch = x & 7;
-            float tw[8], tb[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int j = ch * 8 + e;
-                const float t = Tm[i * 64 + j];
-                tb[e] = t * bs[j];
-                tw[e] = tb[e] * eGs[j];
+            named_bar_sync(1, kPreThreads);
+            // ---- M_kl = D_k A_kl (k > l), in place of A_kl ----------------------------
+            if (pw < 6) {
+                const int kb[6] = {1, 2, 3, 2, 3, 3}, lb[6] = {0, 0, 0, 1, 1, 2};
+                const int k = kb[pw], l = lb[pw];
+                float acc[8];
+                zero8(acc);
+                blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
+                __syncwarp();
+                blk16_store(Am, 16 * k, 16 * l, acc, 1.f, lane);
             }
-            st_shared_v4(sb + OFF_TW + sw128_off(i, ch), pack_bf16x2(tw[0], tw[1]), pack_bf16x2(tw[2], tw[3]),
-                         pack_bf16x2(tw[4], tw[5]), pack_bf16x2(tw[6], tw[7]));
-            st_shared_v4(sb + OFF_TB + sw128_off(i, ch), pack_bf16x2(tb[0], tb[1]), pack_bf16x2(tb[2], tb[3]),
-                         pack_bf16x2(tb[4], tb[5]), pack_bf16x2(tb[6], tb[7]));
-        }
-        fence_async_smem();
-        if (sync_check()) break;
-
-        // ---- W^T = K^T Tw^T, u^T = V^T Tb^T ------------------------------------
-        if (tid == 0) {
+            named_bar_sync(1, kPreThreads);
+            // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds ----------------------
+            {
+                float acc[8];
+                zero8(acc);
+                if (pw == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store(Tm, 16, 0, acc, -1.f, lane); }
+                if (pw == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store(Tm, 32, 16, acc, -1.f, lane); }
+                if (pw == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store(Tm, 48, 32, acc, -1.f, lane); }
+                if (pw == 3) blk16(Am, 32, 0, Tm, 0, 0, acc, lane);
+                if (pw == 4) blk16(Am, 48, 16, Tm, 16, 16, acc, lane);
+                if (pw == 5) blk16(Am, 48, 0, Tm, 0, 0, acc, lane);
+                named_bar_sync(1, kPreThreads);
+                if (pw == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store(Tm, 32, 0, acc, -1.f, lane); }
+                if (pw == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store(Tm, 48, 16, acc, -1.f, lane); }
+                if (pw == 5) blk16(Am, 48, 16, Tm, 16, 0, acc, lane);
+                named_bar_sync(1, kPreThreads);
+                if (pw == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store(Tm, 48, 0, acc, -1.f, lane); }
+                named_bar_sync(1, kPreThreads);
+            }
+            // ---- Tw = T diag(beta e^G), Tb = T diag(beta): bf16 K-major B tiles --------
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int x = pt + u * kPreThreads;        // 0..511
+                const int i = x >> 3, ch = x & 7;
+                const bool zero_blk = (ch >> 1) > (i >> 4);  // above the block diagonal: T is 0
+                const float4 t0 = *reinterpret_cast<const float4*>(Tm + fidx(i, ch * 8));
+                const float4 t1 = *reinterpret_cast<const float4*>(Tm + fidx(i, ch * 8 + 4));
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                const float4 b0 = *reinterpret_cast<const float4*>(gs + G_BETA + ch * 8);
+                const float4 b1 = *reinterpret_cast<const float4*>(gs + G_BETA + ch * 8 + 4);
+                const float4 w0 = *reinterpret_cast<const float4*>(gs + G_BEG + ch * 8);
+                const float4 w1 = *reinterpret_cast<const float4*>(gs + G_BEG + ch * 8 + 4);
+                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                const float bw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float tw[8], tb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float t = zero_blk ? 0.f : tv[e];
+                    tb[e] = t * bb[e];
+                    tw[e] = t * bw[e];
+                }
+                st_shared_v4(sb + OFF_A + sw128_off(i, ch), pack_bf16x2(tw[0], tw[1]), pack_bf16x2(tw[2], tw[3]),
+                             pack_bf16x2(tw[4], tw[5]), pack_bf16x2(tw[6], tw[7]));
+                st_shared_v4(sb + OFF_A + 8192 + sw128_off(i, ch), pack_bf16x2(tb[0], tb[1]),
+                             pack_bf16x2(tb[2], tb[3]), pack_bf16x2(tb[4], tb[5]), pack_bf16x2(tb[6], tb[7]));
+            }
+            fence_async_smem();
+            mbar_arrive(ctl.bar(B_TW));
+            // ---- Qh, then W^T (TMEM) -> smem, once the previous chunk's products read them ---
+            ok = c == 0 || ctl.wait(B_WSQS, par ^ 1u);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(1, kPreThreads, !ok)) break;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int x = pt + u * kPreThreads;        // 0..1023
+                const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                scale_chunk(kq + blk * 16384 + 8192 + sw128_off(i, ch), sb + OFF_QH + blk * 8192 + sw128_off(i, ch), f);
+            }
+            ok = ctl.wait(B_WU, par);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(1, kPreThreads, !ok)) break;
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_W, sw128_desc(KQ + kk * 2048, 16384, 1024),
-                         sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), idesc_bf16(128, 64, 1, 0), kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_U, sw128_desc(VS + kk * 2048, 8192, 1024),
-                         sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), idesc_bf16(128, 64, 1, 0), kk > 0);
-            mma_commit(bar_mma);
-        }
-        wait_mma();
-        {
-            float r[32];
-            tmem_ld32(tmem + lane_off + TM_W + wg * 32, r);
-            tmem_wait_ld();
-            const uint32_t wt = sb + OFF_WT;       // row = key channel c = row, columns i
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                st_shared_v4(wt + sw128_off(row, wg * 4 + q4),
-                             pack_bf16x2(r[8 * q4 + 0], r[8 * q4 + 1]), pack_bf16x2(r[8 * q4 + 2], r[8 * q4 + 3]),
-                             pack_bf16x2(r[8 * q4 + 4], r[8 * q4 + 5]), pack_bf16x2(r[8 * q4 + 6], r[8 * q4 + 7]));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (sync_check()) break;
-
-        // ---- U^T = u^T - S^T W^T, O1^T = S^T Q^T -------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_ST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                         sw128_desc(sb + OFF_WT + kk * 2048, 8192, 1024), idesc_bf16(128, 64, 0, 1, 1), 1);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16(tmem + TM_O1, sw128_desc(sb + OFF_ST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                         sw128_desc(KQ + 8192 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                         idesc_bf16(128, 64, 0, 0), kk > 0);
-            mma_commit(bar_mma);
-        }
-        wait_mma();
-        {
-            float r[32];
-            tmem_ld32(tmem + lane_off + TM_U + wg * 32, r);
-            tmem_wait_ld();
-            const uint32_t ut = sb + OFF_UT;       // row = value channel j, columns = token i
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                st_shared_v4(ut + sw128_off(row, wg * 4 + q4),
-                             pack_bf16x2(r[8 * q4 + 0], r[8 * q4 + 1]), pack_bf16x2(r[8 * q4 + 2], r[8 * q4 + 3]),
-                             pack_bf16x2(r[8 * q4 + 4], r[8 * q4 + 5]), pack_bf16x2(r[8 * q4 + 6], r[8 * q4 + 7]));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        if (sync_check()) break;
-
-        // ---- dS^T = U^T K~, O2^T = U^T P^T -------------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_S, sw128_desc(sb + OFF_UT + kk * 32, 16, 1024),
-                         sw128_desc(sb + OFF_KT + kk * 2048, 8192, 1024), idesc_bf16(128, 128, 0, 1), kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_O2, sw128_desc(sb + OFF_UT + kk * 32, 16, 1024),
-                         sw128_desc(sb + OFF_PM + kk * 32, 16, 1024), idesc_bf16(128, 64, 0, 0), kk > 0);
-            mma_commit(bar_mma);
-        }
-        wait_mma();
-        if (tid == 0 && good && c + 2 < nchunks) {   // stage s is free again
-            issue(c + 2);
-            issued = c + 3;
-        }
-        {
-            // state update S <- e^(G_last) S + dS and its bf16 copy S^T
-            const float gamma = eGs[63];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float r[32];
-                tmem_ld32(tmem + lane_off + TM_S + wg * 64 + h * 32, r);
+            {
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_W + h * 32, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int n = 0; n < 32; ++n) Sreg[h * 32 + n] = gamma * Sreg[h * 32 + n] + r[n];
+                for (int q4 = 0; q4 < 4; ++q4)
+                    st_shared_v4(sb + OFF_WT + sw128_off(r, h * 4 + q4),
+                                 pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                                 pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
             }
-            const uint32_t st = sb + OFF_ST + wg * 16384;
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
-                st_shared_v4(st + sw128_off(row, q8),
-                             pack_bf16x2(Sreg[8 * q8 + 0], Sreg[8 * q8 + 1]), pack_bf16x2(Sreg[8 * q8 + 2], Sreg[8 * q8 + 3]),
-                             pack_bf16x2(Sreg[8 * q8 + 4], Sreg[8 * q8 + 5]), pack_bf16x2(Sreg[8 * q8 + 6], Sreg[8 * q8 + 7]));
-            // output o[i][j] = scale e^G_i O1 + O2 for this thread's j = row, i = 32 wg + n
-            float r1[32], r2[32];
-            tmem_ld32(tmem + lane_off + TM_O1 + wg * 32, r1);
-            tmem_ld32(tmem + lane_off + TM_O2 + wg * 32, r2);
-            tmem_wait_ld();
-            __nv_bfloat16* ob = o + (bh * T + c0) * kD + row;
-#pragma unroll
-            for (int n = 0; n < 32; ++n) {
-                const int i = wg * 32 + n;
-                if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(scale * eGs[i] * r1[n] + r2[n]);
-            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_READY));
+            mbar_arrive(ctl.bar(B_FREE0 + s));
         }
-        fence_async_smem();
-        tc_fence_before();
-        if (sync_check()) break;
+    } else if (warp >= kChainWarp0) {
+        // ================= state chain and output (128 threads) =================
+        const int j = ((warp & 3) << 5) + lane;      // value channel = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+        bool ok = ctl.wait(B_GATE0, 0);
+        if (!ok) *abort_flag = 1;
+        ok = !named_bar_any(2, kChainThreads, !ok);
+        if (ok) {
+            // S0 -> TMEM: fp32 pre-scaled by chunk 0's decay, and its bf16 copy
+            const float gamma0 = gates[G_GAMMA];
+#pragma unroll 1
+            for (int pc = 0; pc < 4; ++pc) {
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = S0 ? S0[(bh * kD + pc * 32 + e) * kD + j] : 0.f;
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= gamma0;
+                tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_ST));
+        }
+        for (int c = 0; ok && c < n; ++c) {
+            const uint32_t par = (uint32_t)c & 1u;
+            const int Cc = min(kC, T - c * kC);
+            // ---- U^T -> bf16 pairs in TMEM ------------------------------------------
+            ok = ctl.wait(B_WSQS, par);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_U + hh * 32, v);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st16(tmem + lane_off + TM_UT + hh * 16, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_UT));
+            mbar_arrive(ctl.bar(B_UFREE));
+            // ---- state: S_{c+1} = gamma_c S_c + dS (already summed in TMEM) ---------------
+            ok = ctl.wait(B_KUPU, par) && (c + 1 >= n || ctl.wait(B_GATE0 + ((c + 1) & 3), (uint32_t)((c + 1) >> 2) & 1u));
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            tc_fence_after();
+            const bool last = c + 1 == n;
+            const float gnext = last ? 1.f : gates[((c + 1) & 3) * GATE_FLOATS + G_GAMMA];
+#pragma unroll 1
+            for (int pc = 0; pc < 4; ++pc) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_SACC + pc * 32, v);
+                tmem_wait_ld();
+                if (last) {
+                    if (S_T) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) S_T[(bh * kD + pc * 32 + e) * kD + j] = v[e];
+                    }
+                } else {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                    tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= gnext;
+                    tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_ST));
+            // ---- output rows of this chunk -----------------------------------------------
+            __nv_bfloat16* ob = o + (bh * T + (int64_t)c * kC) * kD + j;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_O + hh * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = hh * 32 + e;
+                    if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_OFREE));
+        }
+        if (!ok) *abort_flag = 1;
     }
 
-    const bool aborted = *abort_flag != 0;
-    if (aborted) {
-        if (tid == 0) {
-            // let every load this CTA issued land before the CTA's shared memory is released
-            for (int cc = c; cc < issued; ++cc)
-                mbar_wait_bounded(bar_full[cc & 1], (uint32_t)(cc >> 1) & 1u, kWaitNs);
-            atomicOr(status, 1u);
-        }
-    } else if (S_T) {
-        float* dst = S_T + (bh * kD + wg * 64) * kD + row;
-#pragma unroll
-        for (int n = 0; n < 64; ++n) dst[(int64_t)n * kD] = Sreg[n];
-    }
-    tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (*abort_flag && tid == 0) atomicOr(status, 1u);
+    if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }
