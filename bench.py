@@ -260,11 +260,15 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+                    help="launch one kernel of the step a few times without timing (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_case:
+        return run_profile_case(args)
 
     import torch
     import delta_rule_recurrent_02_b200 as dn
@@ -384,6 +388,36 @@ def main():
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_profile_case(args):
+    """Launch the prefill (or the decode step) of the benchmark workload
+    args.warmup + args.steps times, with no timing: a small, fixed program for
+    ncu captures (one kernel per launch, inputs resident on the device)."""
+    import torch
+    import delta_rule_recurrent_02_b200 as dn
+    from delta_rule_recurrent_02_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    if args.profile_case == "prefill":
+        pc = W.GDN_PREFILL
+        P = {k: (None if v is None else v.to(dev)) for k, v in W.gen_prefill_config(pc).items()}
+        o = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
+        S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o, S_T, chunk=pc.chunk,
+                            scale=pc.scale, path=args.path)
+    else:
+        dc = W.DECODE
+        D = {k: (None if v is None else v.to(dev)) for k, v in W.gen_decode(dc).items()}
+        o = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
+        for s in range(args.warmup + args.steps):
+            j = s % dc.bank
+            dn.dn_decode_step(D["q"][j], D["k"][j], D["v"][j], D["beta"][j], D["g"][j], D["S"], o,
+                              scale=dc.scale)
+    dn.dn_device_status()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": args.profile_case, "launches": args.warmup + args.steps}))
     return 0
 
 

@@ -93,7 +93,7 @@ constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMM
 enum {
     B_FULL0 = 0, B_FULL1, B_FREE0, B_FREE1,              // TMA stages
     B_GATE0, B_GATE1, B_GATE2, B_GATE3,                  // gate slots
-    B_GRAM, B_WU, B_WSQS, B_KUPU,                        // MMA completions
+    B_GRAM, B_WU, B_WS, B_WSQS, B_KUPU,                  // MMA completions
     B_TW, B_READY, B_KP0, B_KP1, B_GFREE,                // prework -> MMA
     B_UT, B_UFREE, B_ST, B_OFREE,                        // chain -> MMA
     B_COUNT
@@ -197,7 +197,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int n = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        const uint32_t counts[B_COUNT] = {1, 1, kPreThreads, kPreThreads, 1, 1, 1, 1, 1, 1, 1, 1,
+        const uint32_t counts[B_COUNT] = {1, 1, kPreThreads, kPreThreads, 1, 1, 1, 1, 1, 1, 1, 1, 1,
                                           kPreThreads, kPreThreads, kPreThreads, kPreThreads, kPreThreads,
                                           kChainThreads, kChainThreads, kChainThreads, kChainThreads};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(ctl.bar(i), counts[i]);
@@ -324,14 +324,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             } else {
                 for (int c = 0; ok && c < n; ++c) {
                     const uint32_t par = (uint32_t)c & 1u;
-                    // U^T += -S^T W^T ; O^T = S^T Qh^T
-                    ok = ctl.wait(B_READY, par) && ctl.wait(B_ST, par) && (c == 0 || ctl.wait(B_OFREE, par ^ 1u));
+                    // U^T += -S^T W^T (the chain's critical product), then O^T = S^T Qh^T
+                    // once the previous output has been read
+                    ok = ctl.wait(B_READY, par) && ctl.wait(B_ST, par);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ts(tmem + TM_U, tmem + TM_ST + kk * 8,
                                     sw128_desc(sb + OFF_WT + kk * 2048, 8192, 1024), I_WS, 1);
+                    mma_commit(ctl.bar(B_WS));
+                    ok = c == 0 || ctl.wait(B_OFREE, par ^ 1u);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ts(tmem + TM_O, tmem + TM_ST + kk * 8,
@@ -418,18 +423,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            // ---- K~ = K * e^(G_last - G) (rows >= Cc zero) into this chunk's buffer --------
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int x = pt + u * kPreThreads;        // 0..1023
-                const int blk = x >> 9, t = (x >> 3) & 63, ch = x & 7;
-                const float f = t < Cc ? gs[G_ET + t] : 0.f;
-                scale_chunk(kq + blk * 16384 + sw128_off(t, ch),
-                            sb + OFF_KT + (c & 1) * 16384 + blk * 8192 + sw128_off(t, ch), f);
-            }
-            fence_async_smem();
             tc_fence_before();
-            mbar_arrive(ctl.bar(B_KP0 + (c & 1)));
             mbar_arrive(ctl.bar(B_GFREE));
             named_bar_sync(1, kPreThreads);
             // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T -------------
@@ -510,6 +504,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_async_smem();
             mbar_arrive(ctl.bar(B_TW));
+            // ---- K~ = K * e^(G_last - G) (rows >= Cc zero) into this chunk's buffer --------
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int x = pt + u * kPreThreads;        // 0..1023
+                const int blk = x >> 9, t = (x >> 3) & 63, ch = x & 7;
+                const float f = t < Cc ? gs[G_ET + t] : 0.f;
+                scale_chunk(kq + blk * 16384 + sw128_off(t, ch),
+                            sb + OFF_KT + (c & 1) * 16384 + blk * 8192 + sw128_off(t, ch), f);
+            }
+            fence_async_smem();
+            mbar_arrive(ctl.bar(B_KP0 + (c & 1)));
             // ---- Qh, then W^T (TMEM) -> smem, once the previous chunk's products read them ---
             ok = c == 0 || ctl.wait(B_WSQS, par ^ 1u);
             if (!ok) *abort_flag = 1;
@@ -571,7 +576,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t par = (uint32_t)c & 1u;
             const int Cc = min(kC, T - c * kC);
             // ---- U^T -> bf16 pairs in TMEM ------------------------------------------
-            ok = ctl.wait(B_WSQS, par);
+            ok = ctl.wait(B_WS, par);
             if (!ok) *abort_flag = 1;
             if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
             tc_fence_after();
