@@ -155,14 +155,21 @@ def dist_setup():
     return world, rank, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The largest value of x over all ranks (a timing, so the slowest rank wins)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step, ms_per_step, world):
+    """Whole-job units per second: every rank processes its own units per step
+    (weak scaling) and the step time is the slowest rank's."""
+    return world * units_per_rank_step / (ms_per_step * 1e-3)
 
 
 def barrier(world):
@@ -332,7 +339,7 @@ def main():
     dec_ms = max_over_ranks(dec_ms, world)
     ms_per_step = total_ms / args.steps
     tokens_step = pc.B * pc.T + dc.B
-    value = world * tokens_step / (ms_per_step * 1e-3)
+    value = job_throughput(tokens_step, ms_per_step, world)
     clocks = sampler.summary()
 
     # ---- roofline per kernel ---------------------------------------------------

@@ -30,7 +30,7 @@ __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_decode
 DN_OK, DN_ERR_INVALID, DN_ERR_UNSUPPORTED, DN_ERR_CUDA, DN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 _DTYPES = {"f32": 0, "bf16": 1}
 _GATES = {"none": 0, "scalar": 1, "per_key": 2}
-_PATHS = {"auto": 0, "simt": 1, "tc": 2}
+_PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_decode_step", "dn_device_status",
                "dn_status_str", "dn_last_error", "dn_version")

@@ -66,6 +66,7 @@ constexpr uint32_t TM_U = 224;      // U^T fp32 accumulator [dv][C]
 constexpr uint32_t TM_O = 288;      // O^T fp32 accumulator [dv][C]
 constexpr uint32_t TM_G = 352;      // gram: lanes 0-63 K K^T, 64-127 Q K^T
 constexpr uint32_t TM_W = 416;      // W^T fp32 [dk][C]
+constexpr uint32_t TM_UK = 480;     // (U * e^(G_last - G))^T bf16 pairs [dv][C/2]
 constexpr uint32_t TM_COLS = 512;
 
 // shared memory (bytes from a 1024-aligned base)
@@ -73,11 +74,13 @@ constexpr uint32_t OFF_KQ = 0;          // 2 stages x 32 KiB: [d-block][K rows 0
 constexpr uint32_t SZ_KQ = 32768;
 constexpr uint32_t OFF_V = 65536;       // 2 stages x 16 KiB: [d-block][64 rows][128 B]
 constexpr uint32_t SZ_V = 16384;
-constexpr uint32_t OFF_QH = 98304;      // Qh, K-major B [N=i][K=c]: [c-block][64 rows][128 B]
+constexpr uint32_t OFF_QH = 98304;      // Qh (even chunks), K-major B [N=i][K=c]: [c-block][64 rows][128 B]
+constexpr uint32_t OFF_QH1 = 147456;    // Qh (odd chunks)
 constexpr uint32_t OFF_WT = 114688;     // W^T, MN-major B [K=c rows][N=i]: [128 rows][128 B]
-constexpr uint32_t OFF_KT = 131072;     // 2 x K~, MN-major B [K=j rows][N=c]: [c-block][64 rows][128 B]
+constexpr uint32_t OFF_TW = 131072;     // T diag(beta e^G), K-major B [N=i][K=j]: [64 rows][128 B]
+constexpr uint32_t OFF_TB = 139264;     // T diag(beta), same layout
 constexpr uint32_t OFF_PM = 163840;     // 2 x P, K-major B [N=i][K=j]: [64 rows][128 B]
-constexpr uint32_t OFF_A = 180224;      // fp32 64 x 68: A, then M = D^-1 A; later Tw (8 KiB) + Tb (8 KiB) bf16
+constexpr uint32_t OFF_A = 180224;      // fp32 64 x 68: A, then M = D^-1 A
 constexpr uint32_t OFF_T = 197632;      // fp32 64 x 68: T = (I + A)^-1
 constexpr uint32_t OFF_GATE = 215040;   // 4 gate slots
 constexpr uint32_t GATE_FLOATS = 384;
@@ -133,6 +136,27 @@ __device__ __forceinline__ void blk16_store(float* Z, int zr, int zc, const floa
         make_float4(sign * acc[4], sign * acc[5], sign * acc[6], sign * acc[7]);
 }
 
+// Store -acc as T block rows (fp32) and as the bf16 B tiles T diag(beta e^G)
+// and T diag(beta): lane (ii, j0) owns 8 consecutive columns = one 16-byte chunk.
+__device__ __forceinline__ void blk16_store_t(float* Tm, uint32_t tw, uint32_t tb, const float* gs, int zr, int zc,
+                                              const float (&acc)[8], int lane, int g_beta, int g_beg) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    float t[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = -acc[e];
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0)) = make_float4(t[0], t[1], t[2], t[3]);
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0 + 4)) = make_float4(t[4], t[5], t[6], t[7]);
+    const float4 b0 = *reinterpret_cast<const float4*>(gs + g_beta + zc + j0);
+    const float4 b1 = *reinterpret_cast<const float4*>(gs + g_beta + zc + j0 + 4);
+    const float4 w0 = *reinterpret_cast<const float4*>(gs + g_beg + zc + j0);
+    const float4 w1 = *reinterpret_cast<const float4*>(gs + g_beg + zc + j0 + 4);
+    const int row = zr + ii, ch = (zc + j0) >> 3;
+    st_shared_v4(tw + sw128_off(row, ch), pack_bf16x2(t[0] * w0.x, t[1] * w0.y), pack_bf16x2(t[2] * w0.z, t[3] * w0.w),
+                 pack_bf16x2(t[4] * w1.x, t[5] * w1.y), pack_bf16x2(t[6] * w1.z, t[7] * w1.w));
+    st_shared_v4(tb + sw128_off(row, ch), pack_bf16x2(t[0] * b0.x, t[1] * b0.y), pack_bf16x2(t[2] * b0.z, t[3] * b0.w),
+                 pack_bf16x2(t[4] * b1.x, t[5] * b1.y), pack_bf16x2(t[6] * b1.z, t[7] * b1.w));
+}
+
 __device__ __forceinline__ void zero8(float (&a)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = 0.f;
@@ -179,7 +203,7 @@ __global__ void __launch_bounds__(kNT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ beta,
                 const float* __restrict__ g, const float* S0, __nv_bfloat16* __restrict__ o,
-                float* S_T, int T, float scale, unsigned int* status) {
+                float* S_T, int T, float scale, unsigned int* status, int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
@@ -197,7 +221,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int n = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        const uint32_t counts[B_COUNT] = {1, 1, kPreThreads, kPreThreads, 1, 1, 1, 1, 1, 1, 1, 1, 1,
+        const uint32_t counts[B_COUNT] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1,
                                           kPreThreads, kPreThreads, kPreThreads, kPreThreads, kPreThreads,
                                           kChainThreads, kChainThreads, kChainThreads, kChainThreads};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(ctl.bar(i), counts[i]);
@@ -236,10 +260,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fetch(0);
         for (int cc = 0; cc < n; ++cc) {
             const int s = cc & 1;
-            if (cc >= 2) {
-                bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - 2) >> 1) & 1u) : true;
-                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
-            }
             // gates of chunk cc into slot cc % 4
             float* gs = gates + (cc & 3) * GATE_FLOATS;
             const int64_t t0 = bh * T + (int64_t)cc * kC;
@@ -263,8 +283,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             gs[G_ET + lane] = expf(Glast - a0); gs[G_ET + lane + 32] = expf(Glast - a1);
             if (lane == 0) gs[G_GAMMA] = expf(Glast);
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            // the stage is free once the state product of chunk cc - 2 is done
+            if (cc >= 2) {
+                bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - 2) >> 1) & 1u) : true;
+                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+            }
+            if (lane == 0 && !(test_flags & 1)) {
                 const int y = (int)t0;
                 const uint32_t kq = sb + OFF_KQ + s * SZ_KQ, vv = sb + OFF_V + s * SZ_V;
                 const uint32_t fb = ctl.bar(B_FULL0 + s);
@@ -276,7 +301,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_load_2d(vv + 0, &tm_v, 0, y, fb);
                 tma_load_2d(vv + 8192, &tm_v, 64, y, fb);
             }
-            issued = cc + 1;
+            if (!(test_flags & 1)) issued = cc + 1;
         }
         if (*abort_flag && lane == 0) {
             // let every load this CTA issued land before its shared memory is released
@@ -314,11 +339,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(tmem + TM_W, sw128_desc(kq + kk * 2048, 16384, 1024),
-                                 sw128_desc(sb + OFF_A + kk * 32, 16, 1024), I_MNK, kk > 0);
+                                 sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), I_MNK, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(tmem + TM_U, sw128_desc(vv + kk * 2048, 8192, 1024),
-                                 sw128_desc(sb + OFF_A + 8192 + kk * 32, 16, 1024), I_MNK, kk > 0);
+                                 sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), I_MNK, kk > 0);
                     mma_commit(ctl.bar(B_WU));
                 }
             } else {
@@ -340,22 +365,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ts(tmem + TM_O, tmem + TM_ST + kk * 8,
-                                    sw128_desc(sb + OFF_QH + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), I_KK,
-                                    kk > 0);
+                                    sw128_desc((c & 1 ? sb + OFF_QH1 : sb + OFF_QH) + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                               16, 1024), I_KK, kk > 0);
                     mma_commit(ctl.bar(B_WSQS));
                     // S^T += U^T K~ ; O^T += U^T P^T
                     ok = ctl.wait(B_UT, par) && ctl.wait(B_KP0 + (c & 1), (uint32_t)(c >> 1) & 1u);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t kt = sb + OFF_KT + (c & 1) * 16384, pm = sb + OFF_PM + (c & 1) * 8192;
+                    const uint32_t kq = sb + OFF_KQ + (c & 1) * SZ_KQ, pm = sb + OFF_PM + (c & 1) * 8192;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ts(tmem + TM_SACC, tmem + TM_UT + kk * 8, sw128_desc(kt + kk * 2048, 8192, 1024),
+                        mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(kq + kk * 2048, 16384, 1024),
                                     I_KU, 1);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ts(tmem + TM_O, tmem + TM_UT + kk * 8, sw128_desc(pm + kk * 32, 16, 1024), I_KK, 1);
                     mma_commit(ctl.bar(B_KUPU));
+                    mma_commit(ctl.bar(B_FREE0 + (c & 1)));   // the stage's last reader is done
                 }
             }
             if (!ok) *abort_flag = 1;
@@ -368,6 +394,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int h = pw >> 2;                     // column half
         const int r = (q << 5) + lane;             // TMEM lane (row)
         const uint32_t lane_off = (uint32_t)(q << 5) << 16;
+        // the blocks of T above the block diagonal are zero for every chunk
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st_shared_v4(sb + OFF_TW + (uint32_t)(pt + u * kPreThreads) * 16, 0u, 0u, 0u, 0u);
         for (int c = 0; c < n; ++c) {
             const int s = c & 1;
             const uint32_t par = (uint32_t)c & 1u;
@@ -423,7 +452,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
+            fence_async_smem();
             tc_fence_before();
+            mbar_arrive(ctl.bar(B_KP0 + (c & 1)));
             mbar_arrive(ctl.bar(B_GFREE));
             named_bar_sync(1, kPreThreads);
             // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T -------------
@@ -455,78 +486,60 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
                 __syncwarp();
                 blk16_store(Am, 16 * k, 16 * l, acc, 1.f, lane);
+            } else {
+                // warps 6, 7: diagonal blocks D_k of T -> bf16 Tw / Tb chunks
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int x = (pw - 6) * 32 + lane + u * 64;     // 0..127
+                    const int blk = x >> 5, i = 16 * blk + ((x >> 1) & 15), j0 = 16 * blk + 8 * (x & 1);
+                    const float4 t0 = *reinterpret_cast<const float4*>(Tm + fidx(i, j0));
+                    const float4 t1 = *reinterpret_cast<const float4*>(Tm + fidx(i, j0 + 4));
+                    const float4 b0 = *reinterpret_cast<const float4*>(gs + G_BETA + j0);
+                    const float4 b1 = *reinterpret_cast<const float4*>(gs + G_BETA + j0 + 4);
+                    const float4 w0 = *reinterpret_cast<const float4*>(gs + G_BEG + j0);
+                    const float4 w1 = *reinterpret_cast<const float4*>(gs + G_BEG + j0 + 4);
+                    st_shared_v4(sb + OFF_TW + sw128_off(i, j0 >> 3), pack_bf16x2(t0.x * w0.x, t0.y * w0.y),
+                                 pack_bf16x2(t0.z * w0.z, t0.w * w0.w), pack_bf16x2(t1.x * w1.x, t1.y * w1.y),
+                                 pack_bf16x2(t1.z * w1.z, t1.w * w1.w));
+                    st_shared_v4(sb + OFF_TB + sw128_off(i, j0 >> 3), pack_bf16x2(t0.x * b0.x, t0.y * b0.y),
+                                 pack_bf16x2(t0.z * b0.z, t0.w * b0.w), pack_bf16x2(t1.x * b1.x, t1.y * b1.y),
+                                 pack_bf16x2(t1.z * b1.z, t1.w * b1.w));
+                }
             }
             named_bar_sync(1, kPreThreads);
             // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds ----------------------
             {
                 float acc[8];
                 zero8(acc);
-                if (pw == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store(Tm, 16, 0, acc, -1.f, lane); }
-                if (pw == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store(Tm, 32, 16, acc, -1.f, lane); }
-                if (pw == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store(Tm, 48, 32, acc, -1.f, lane); }
+                const uint32_t tw = sb + OFF_TW, tb = sb + OFF_TB;
+                if (pw == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 16, 0, acc, lane, G_BETA, G_BEG); }
+                if (pw == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store_t(Tm, tw, tb, gs, 32, 16, acc, lane, G_BETA, G_BEG); }
+                if (pw == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 32, acc, lane, G_BETA, G_BEG); }
                 if (pw == 3) blk16(Am, 32, 0, Tm, 0, 0, acc, lane);
                 if (pw == 4) blk16(Am, 48, 16, Tm, 16, 16, acc, lane);
                 if (pw == 5) blk16(Am, 48, 0, Tm, 0, 0, acc, lane);
                 named_bar_sync(1, kPreThreads);
-                if (pw == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store(Tm, 32, 0, acc, -1.f, lane); }
-                if (pw == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store(Tm, 48, 16, acc, -1.f, lane); }
+                if (pw == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 32, 0, acc, lane, G_BETA, G_BEG); }
+                if (pw == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 16, acc, lane, G_BETA, G_BEG); }
                 if (pw == 5) blk16(Am, 48, 16, Tm, 16, 0, acc, lane);
                 named_bar_sync(1, kPreThreads);
-                if (pw == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store(Tm, 48, 0, acc, -1.f, lane); }
-                named_bar_sync(1, kPreThreads);
-            }
-            // ---- Tw = T diag(beta e^G), Tb = T diag(beta): bf16 K-major B tiles --------
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int x = pt + u * kPreThreads;        // 0..511
-                const int i = x >> 3, ch = x & 7;
-                const bool zero_blk = (ch >> 1) > (i >> 4);  // above the block diagonal: T is 0
-                const float4 t0 = *reinterpret_cast<const float4*>(Tm + fidx(i, ch * 8));
-                const float4 t1 = *reinterpret_cast<const float4*>(Tm + fidx(i, ch * 8 + 4));
-                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                const float4 b0 = *reinterpret_cast<const float4*>(gs + G_BETA + ch * 8);
-                const float4 b1 = *reinterpret_cast<const float4*>(gs + G_BETA + ch * 8 + 4);
-                const float4 w0 = *reinterpret_cast<const float4*>(gs + G_BEG + ch * 8);
-                const float4 w1 = *reinterpret_cast<const float4*>(gs + G_BEG + ch * 8 + 4);
-                const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                const float bw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                float tw[8], tb[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float t = zero_blk ? 0.f : tv[e];
-                    tb[e] = t * bb[e];
-                    tw[e] = t * bw[e];
-                }
-                st_shared_v4(sb + OFF_A + sw128_off(i, ch), pack_bf16x2(tw[0], tw[1]), pack_bf16x2(tw[2], tw[3]),
-                             pack_bf16x2(tw[4], tw[5]), pack_bf16x2(tw[6], tw[7]));
-                st_shared_v4(sb + OFF_A + 8192 + sw128_off(i, ch), pack_bf16x2(tb[0], tb[1]),
-                             pack_bf16x2(tb[2], tb[3]), pack_bf16x2(tb[4], tb[5]), pack_bf16x2(tb[6], tb[7]));
+                if (pw == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 0, acc, lane, G_BETA, G_BEG); }
             }
             fence_async_smem();
             mbar_arrive(ctl.bar(B_TW));
-            // ---- K~ = K * e^(G_last - G) (rows >= Cc zero) into this chunk's buffer --------
+            // ---- Qh into this chunk's buffer (the previous user, two chunks back, is done) ----
+            {
+                const uint32_t qh = (c & 1) ? sb + OFF_QH1 : sb + OFF_QH;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int x = pt + u * kPreThreads;        // 0..1023
-                const int blk = x >> 9, t = (x >> 3) & 63, ch = x & 7;
-                const float f = t < Cc ? gs[G_ET + t] : 0.f;
-                scale_chunk(kq + blk * 16384 + sw128_off(t, ch),
-                            sb + OFF_KT + (c & 1) * 16384 + blk * 8192 + sw128_off(t, ch), f);
+                for (int u = 0; u < 4; ++u) {
+                    const int x = pt + u * kPreThreads;        // 0..1023
+                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                    scale_chunk(kq + blk * 16384 + 8192 + sw128_off(i, ch), qh + blk * 8192 + sw128_off(i, ch), f);
+                }
             }
-            fence_async_smem();
-            mbar_arrive(ctl.bar(B_KP0 + (c & 1)));
-            // ---- Qh, then W^T (TMEM) -> smem, once the previous chunk's products read them ---
-            ok = c == 0 || ctl.wait(B_WSQS, par ^ 1u);
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(1, kPreThreads, !ok)) break;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int x = pt + u * kPreThreads;        // 0..1023
-                const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
-                const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
-                scale_chunk(kq + blk * 16384 + 8192 + sw128_off(i, ch), sb + OFF_QH + blk * 8192 + sw128_off(i, ch), f);
-            }
-            ok = ctl.wait(B_WU, par);
+            // ---- W^T (TMEM) -> smem once W is computed and the previous chunk's product read it
+            ok = ctl.wait(B_WU, par) && (c == 0 || ctl.wait(B_WS, par ^ 1u));
             if (!ok) *abort_flag = 1;
             if (named_bar_any(1, kPreThreads, !ok)) break;
             tc_fence_after();
@@ -543,7 +556,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(ctl.bar(B_READY));
-            mbar_arrive(ctl.bar(B_FREE0 + s));
         }
     } else if (warp >= kChainWarp0) {
         // ================= state chain and output (128 threads) =================
@@ -580,6 +592,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!ok) *abort_flag = 1;
             if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
             tc_fence_after();
+            const float* gsc = gates + (c & 3) * GATE_FLOATS;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float v[32];
@@ -589,6 +602,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 tmem_st16(tmem + lane_off + TM_UT + hh * 16, pk);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + hh * 32 + 4 * q4);
+                    pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
+                    pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
+                }
+                tmem_st16(tmem + lane_off + TM_UK + hh * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -692,14 +712,14 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(a.B * a.H), kNT, SMEM_BYTES, st>>>(tq, tk, tv, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
-                                                          a.scale, a.status);
+                                                          a.scale, a.status, a.test_flags);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 bool tc_supports(const ChunkArgs& a) {
-    return a.bf16 && a.chunk == kC && a.dk == kD && a.dv == kD && a.gate != kGatePerKey && a.T >= 1 &&
+    return a.bf16 && a.chunk == kC && a.dk == kD && a.dv == kD && a.gate != kGatePerKey &&
            a.B * a.H * a.T < (int64_t(1) << 31);
 }
 

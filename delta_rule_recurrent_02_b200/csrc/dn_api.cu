@@ -88,7 +88,7 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
     if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
     if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
         return fail(DN_ERR_INVALID, "unknown gate %d", (int)gate);
-    if (path != DN_PATH_AUTO && path != DN_PATH_SIMT && path != DN_PATH_TC)
+    if (path != DN_PATH_AUTO && path != DN_PATH_SIMT && path != DN_PATH_TC && path != DN_PATH_TC_STALL_TEST)
         return fail(DN_ERR_INVALID, "unknown path %d", (int)path);
     if (d_k <= 0 || d_v <= 0) return fail(DN_ERR_INVALID, "d_k, d_v must be > 0");
     if (chunk <= 0) return fail(DN_ERR_INVALID, "chunk must be > 0 (got %d)", chunk);
@@ -131,6 +131,19 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk; a.scale = scale;
     a.bf16 = dtype == DN_BF16; a.gate = (int)gate;
+    a.test_flags = path == DN_PATH_TC_STALL_TEST ? 1 : 0;
+
+    // kernel choice first: an unsupported request touches no device state
+    bool use_tc = false;
+    if (path == DN_PATH_TC || path == DN_PATH_TC_STALL_TEST) {
+        if (!dn::tc_supports(a))
+            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128 and no per-key gate");
+        use_tc = true;
+    } else if (path == DN_PATH_AUTO) {
+        use_tc = dn::tc_supports(a);
+    }
+    if (!use_tc && chunk > 64) return fail(DN_ERR_UNSUPPORTED, "chunk must be <= 64 (got %d)", chunk);
+
     cudaError_t e;
     a.status = status_word(&e);
     if (e != cudaSuccess) return cuda_fail(e, "status word");
@@ -142,15 +155,6 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
         return e == cudaSuccess ? ok() : cuda_fail(e, "T = 0 state copy");
     }
 
-    bool use_tc = false;
-    if (path == DN_PATH_TC) {
-        if (!dn::tc_supports(a))
-            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128");
-        use_tc = true;
-    } else if (path == DN_PATH_AUTO) {
-        use_tc = dn::tc_supports(a);
-    }
-    if (!use_tc && chunk > 64) return fail(DN_ERR_UNSUPPORTED, "chunk must be <= 64 (got %d)", chunk);
     e = use_tc ? dn::launch_chunk_tc(a, st) : dn::launch_chunk_simt(a, st);
     if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core chunk kernel" : "SIMT chunk kernel");
     return ok();

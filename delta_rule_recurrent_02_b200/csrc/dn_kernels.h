@@ -17,6 +17,7 @@ struct ChunkArgs {
     bool bf16;
     int gate;                 // Gate
     unsigned int* status;     // device status word of the current device
+    int test_flags;           // 1: withhold the tensor-core kernel's input loads (failure-path self-test)
 };
 
 struct DecodeArgs {

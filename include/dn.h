@@ -74,7 +74,12 @@ typedef enum {
 typedef enum {
     DN_PATH_AUTO = 0,     /* tensor-core path when it supports the request, else SIMT */
     DN_PATH_SIMT = 1,     /* fp32 CUDA-core chunk kernel: any chunk 1..64          */
-    DN_PATH_TC = 2        /* tcgen05 chunk kernel: bf16, chunk 64, d_k = d_v = 128 */
+    DN_PATH_TC = 2,       /* tcgen05 chunk kernel: bf16, chunk 64, d_k = d_v = 128 */
+    /* Self-test of the failure path: the tensor-core kernel runs with its input
+     * loads withheld, so every bounded wait inside it expires (about one second);
+     * nothing is written to o or S_T, dn_device_status() then returns
+     * DN_ERR_TIMEOUT, and the CUDA context stays usable. */
+    DN_PATH_TC_STALL_TEST = 3
 } dn_path;
 
 /*

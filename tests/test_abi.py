@@ -77,6 +77,8 @@ def chunk_call(lib, **over):
     (dict(S0=A + 7 * STEP, S_T=A + 7 * STEP + 256), dn.DN_ERR_INVALID),  # partial overlap
     (dict(dk=96), dn.DN_ERR_UNSUPPORTED),
     (dict(dv=256), dn.DN_ERR_UNSUPPORTED),
+    (dict(path=2), dn.DN_ERR_UNSUPPORTED),                    # tensor-core path needs bf16, d = 128
+    (dict(path=3), dn.DN_ERR_UNSUPPORTED),                    # so does its self-test
 ])
 def test_chunk_fwd_rejects(lib, over, code):
     assert chunk_call(lib, **over) == code
