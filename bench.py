@@ -300,10 +300,11 @@ def main():
     o_d = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
     S_dec = D["S"]
     stream = torch.cuda.current_stream()
+    ws = prefill_workspace(dn, torch, pc, args.path, dev)
 
     def prefill():
         dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o_p, S_T, chunk=pc.chunk,
-                        scale=pc.scale, path=args.path, stream=stream)
+                        scale=pc.scale, path=args.path, workspace=ws, stream=stream)
 
     def decode(s):
         j = s % dc.bank
@@ -346,8 +347,8 @@ def main():
     pf = prefill_flops(pc.B, pc.H, pc.T, pc.dk, pc.dv)
     pb = prefill_bytes(pc.B, pc.H, pc.T, pc.dk, pc.dv)
     db = decode_bytes(dc.B, dc.H, dc.dk, dc.dv)
-    used_tc = args.path == "tc" or (args.path == "auto" and _tc_active(dn, P, o_p, S_T, pc, stream))
-    pre_kernel = "chunk_tc" if used_tc else "chunk_simt"
+    used_tc = ws is not None          # only the tensor-core path takes a workspace
+    pre_kernel = "chunk_wy+chunk_tc" if used_tc else "chunk_simt"
     pre_tflops = pf / (pre_ms * 1e-3) / 1e12
     pre_gbs = pb / (pre_ms * 1e-3) / 1e9
     dec_gbs = db / (dec_ms * 1e-3) / 1e9
@@ -381,7 +382,8 @@ def main():
             "data": "synthetic", "config": workload_config(),
             "prefill": {"tokens_per_s": world * pc.B * pc.T / (pre_ms * 1e-3), "roofline": pre_roof},
             "decode": {"tokens_per_s": world * dc.B / (dec_ms * 1e-3), "roofline": dec_roof},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks}
+            "roofline": roofline, "e2e": e2e, "gpu_launches": (3 if used_tc else 2) * args.steps,
+            "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]
@@ -411,9 +413,10 @@ def run_profile_case(args):
         P = {k: (None if v is None else v.to(dev)) for k, v in W.gen_prefill_config(pc).items()}
         o = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
         S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
+        ws = prefill_workspace(dn, torch, pc, args.path, dev)
         for _ in range(args.warmup + args.steps):
             dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o, S_T, chunk=pc.chunk,
-                            scale=pc.scale, path=args.path)
+                            scale=pc.scale, path=args.path, workspace=ws)
     else:
         dc = W.DECODE
         D = {k: (None if v is None else v.to(dev)) for k, v in W.gen_decode(dc).items()}
@@ -436,14 +439,11 @@ def _smi_id(torch, dev, local):
         return local
 
 
-def _tc_active(dn, P, o_p, S_T, pc, stream):
-    lib = dn.load_library()
-    # the same request on the tensor-core path: DN_OK means the automatic choice uses it
-    import ctypes
-    st = lib.dn_chunk_fwd_ex(P["q"].data_ptr(), P["k"].data_ptr(), P["v"].data_ptr(), P["beta"].data_ptr(),
-                             P["g"].data_ptr(), None, o_p.data_ptr(), S_T.data_ptr(), pc.B, pc.T, pc.H,
-                             pc.dk, pc.dv, pc.chunk, pc.scale, 1, 1, 2, ctypes.c_void_p(stream.cuda_stream))
-    return st == 0
+def prefill_workspace(dn, torch, pc, path, dev):
+    """The prefill's workspace, allocated once like a caller that reuses it (None if the path needs none)."""
+    nbytes = dn.dn_chunk_fwd_workspace_size(pc.B, pc.T, pc.H, pc.dk, pc.dv, chunk=pc.chunk, dtype=pc.dtype,
+                                            gate=pc.gate, path=path)
+    return torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
 
 
 def run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_step):
@@ -459,6 +459,7 @@ def run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_ste
     o_p = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
     o_d = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
+    ws = prefill_workspace(dn, torch, pc, args.path, dev)
     h_o = torch.empty(o_p.shape, dtype=o_p.dtype).pin_memory()
     h_S = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
     h_od = torch.empty(o_d.shape, dtype=o_d.dtype).pin_memory()
@@ -475,7 +476,7 @@ def run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_ste
             if v is not None:
                 Dt[k].copy_(v[j], non_blocking=True)
         dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o_p, S_T, chunk=pc.chunk,
-                        scale=pc.scale, path=args.path, stream=stream)
+                        scale=pc.scale, path=args.path, workspace=ws, stream=stream)
         dn.dn_decode_step(Dt["q"], Dt["k"], Dt["v"], Dt["beta"], Dt["g"], S_dec, o_d, scale=dc.scale,
                           stream=stream)
         h_o.copy_(o_p, non_blocking=True)

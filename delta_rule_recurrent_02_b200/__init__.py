@@ -9,11 +9,12 @@ call raises.
 
 Functions with the ABI's names take preallocated outputs:
 
-    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=64, scale=1.0, ...)
+    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=64, scale=1.0, workspace=None, ...)
+    dn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, chunk=64, dtype="bf16", gate="scalar", path="auto")
     dn_decode_step(q, k, v, beta, g, S, o, scale=1.0, ...)
     dn_device_status(stream=None)
 
-and two conveniences allocate the outputs with torch:
+and two conveniences allocate the outputs (and the prefill's workspace) with torch:
 
     o, S_T = chunk_fwd(q, k, v, beta, g=None, S0=None, chunk=64, scale=1.0)
     o      = decode_step(q, k, v, beta, S, g=None, scale=1.0)
@@ -23,7 +24,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_decode_step",
+__all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
+           "dn_decode_step",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
 
@@ -32,8 +34,8 @@ _DTYPES = {"f32": 0, "bf16": 1}
 _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
-ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_decode_step", "dn_device_status",
-               "dn_status_str", "dn_last_error", "dn_version")
+ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_decode_step",
+               "dn_device_status", "dn_status_str", "dn_last_error", "dn_version")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -59,11 +61,13 @@ def load_library():
         raise RuntimeError(f"{path} is missing: build it with `python -m delta_rule_recurrent_02_b200.build` "
                            "(there is no fallback implementation)")
     lib = ctypes.CDLL(path)
-    vp, fp, I, F = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    vp, fp, I, F, Z = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.dn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, vp]
     lib.dn_chunk_fwd.restype = I
-    lib.dn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, I, vp]
+    lib.dn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, I, vp, Z, vp]
     lib.dn_chunk_fwd_ex.restype = I
+    lib.dn_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I, ctypes.POINTER(Z)]
+    lib.dn_chunk_fwd_workspace_size.restype = I
     lib.dn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp]
     lib.dn_decode_step.restype = I
     lib.dn_device_status.argtypes = [vp]
@@ -125,17 +129,33 @@ def _f32(t):
     return t
 
 
+def dn_chunk_fwd_workspace_size(B: int, T: int, H: int, d_k: int, d_v: int, *, chunk: int = 64,
+                                dtype: str = "bf16", gate: str = "scalar", path: str = "auto") -> int:
+    """Bytes of workspace ``dn_chunk_fwd`` needs for this request (0 if none)."""
+    lib = load_library()
+    out = ctypes.c_size_t(0)
+    _check(lib, lib.dn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, int(chunk), _DTYPES[dtype], _GATES[gate],
+                                                _PATHS[path], ctypes.byref(out)))
+    return out.value
+
+
 def dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, *, chunk: int = 64, scale: float = 1.0,
-                 gate: str | None = None, path: str = "auto", stream=None) -> None:
-    """Chunked prefill through ``dn_chunk_fwd_ex``; writes ``o`` and ``S_T``."""
+                 gate: str | None = None, path: str = "auto", workspace=None, stream=None) -> None:
+    """Chunked prefill through ``dn_chunk_fwd_ex``; writes ``o`` and ``S_T``.
+
+    ``workspace`` is a CUDA tensor of at least ``dn_chunk_fwd_workspace_size``
+    bytes, or None (the library then allocates one stream-ordered for the call).
+    """
     lib = load_library()
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     for t in (beta, g, S0, S_T):
         _f32(t)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.dn_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o),
                              _ptr(S_T), B, T, H, dk, dv, int(chunk), float(scale), _dtype_code(q),
-                             _gate_code(gate, g, (B, H, T)), _PATHS[path], _stream(stream))
+                             _gate_code(gate, g, (B, H, T)), _PATHS[path], _ptr(workspace), ws_bytes,
+                             _stream(stream))
     _check(lib, st)
 
 
@@ -161,14 +181,19 @@ def dn_device_status(stream=None) -> None:
 
 def chunk_fwd(q, k, v, beta, g=None, S0=None, *, chunk: int = 64, scale: float = 1.0,
               gate: str | None = None, path: str = "auto", want_state: bool = True, stream=None):
-    """Allocate ``o`` (dtype of q) and ``S_T`` (fp32), run the prefill, return both."""
+    """Allocate ``o`` (dtype of q), ``S_T`` (fp32) and the workspace, run the prefill, return (o, S_T)."""
     import torch
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
     S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
-    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=chunk, scale=scale, gate=gate, path=path,
-                 stream=stream)
+    gcode = _gate_code(gate, g, (B, H, T))
+    gname = {v2: k2 for k2, v2 in _GATES.items()}[gcode]
+    dname = {v2: k2 for k2, v2 in _DTYPES.items()}[_dtype_code(q)]
+    nbytes = dn_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk=chunk, dtype=dname, gate=gname, path=path)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=chunk, scale=scale, gate=gname, path=path,
+                 workspace=ws, stream=stream)
     return o, S_T
 
 

@@ -1,0 +1,115 @@
+// chunk_tc_common.cuh -- pieces shared by the two tensor-core chunk kernels:
+// chunk_wy.cu (the UT/WY transform of every chunk, in parallel) and
+// chunk_tc.cu (the sequential state pass and the output).
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "dn_common.cuh"
+#include "dn_kernels.h"
+#include "sm100.cuh"
+
+namespace dn {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int kC = 64;                      // chunk
+constexpr int kD = 128;                     // d_k = d_v
+constexpr uint64_t kWaitNs = 1000000000ull; // every mbarrier wait gives up after 1 s
+
+// One chunk's W^T or u^T in the workspace: bf16, [128 rows (d_k or d_v)][64 columns (position)].
+constexpr size_t kWsTileBytes = (size_t)kD * kC * 2;
+
+// Gate slot of one chunk (floats).
+constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320;
+constexpr uint32_t GATE_FLOATS = 384;
+
+// Gates of one chunk from beta and g at positions lane and lane + 32 (zero past
+// the chunk's end, which makes those positions identity steps).  G is the
+// inclusive prefix sum of g inside the chunk ("Linear attention and Gated
+// DeltaNet", ch. 28, the chunked form: cumulative log-decay); the slot gets
+// beta, G log2(e), e^G, e^(G_last - G), beta e^G and e^(G_last).  One warp.
+__device__ __forceinline__ void chunk_gates(float* gs, float b0, float b1, float a0, float a1, int lane) {
+#pragma unroll
+    for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const float y0 = __shfl_up_sync(0xffffffffu, a0, o2);
+        const float y1 = __shfl_up_sync(0xffffffffu, a1, o2);
+        if (lane >= o2) { a0 += y0; a1 += y1; }
+    }
+    a1 += __shfl_sync(0xffffffffu, a0, 31);
+    const float Glast = __shfl_sync(0xffffffffu, a1, 31);
+    const float L2E = 1.4426950408889634f;
+    gs[G_BETA + lane] = b0; gs[G_BETA + lane + 32] = b1;
+    gs[G_G2 + lane] = a0 * L2E; gs[G_G2 + lane + 32] = a1 * L2E;
+    const float e0 = expf(a0), e1 = expf(a1);
+    gs[G_EG + lane] = e0; gs[G_EG + lane + 32] = e1;
+    gs[G_BEG + lane] = b0 * e0; gs[G_BEG + lane + 32] = b1 * e1;
+    gs[G_ET + lane] = expf(Glast - a0); gs[G_ET + lane + 32] = expf(Glast - a1);
+    if (lane == 0) gs[G_GAMMA] = expf(Glast);
+}
+
+// e^(G_i - G_j) = 2^(G2_i - G2_j) with G2 = G log2(e), for j <= i (the
+// exponent is <= 0 for g <= 0; very old positions underflow to 0).
+__device__ __forceinline__ float decay2(float g2i, float g2j) { return exp2f(g2i - g2j); }
+
+// Bounded mbarrier waits for a CTA whose roles share an abort flag in shared memory.
+struct Ctl {
+    uint32_t bar0;                 // address of barrier 0
+    volatile int* abort;
+    __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
+    // gives up after kWaitNs, or early once another role has aborted
+    __device__ bool wait(int i, uint32_t parity) const {
+        const uint32_t b = bar(i);
+        if (mbar_try_wait(b, parity)) return true;
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+            if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitNs) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+};
+
+// ---- host side ---------------------------------------------------------------
+
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill past the end.
+inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+// The UT/WY transform of every chunk into the workspace halves w_ws and u_ws
+// (chunk_wy.cu); tk, tv map k and v as [B H T][128] with 64 x 64 boxes.
+cudaError_t launch_chunk_wy(const ChunkArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                            __nv_bfloat16* w_ws, __nv_bfloat16* u_ws, cudaStream_t st);
+
+}  // namespace dn

@@ -61,11 +61,46 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
+// Size / enum / path checks shared by dn_chunk_fwd_ex and dn_chunk_fwd_workspace_size.
+// Fills the non-pointer fields of *a and the kernel choice.
+int plan_chunk(int B, int T, int H, int d_k, int d_v, int chunk, dn_dtype dtype, dn_gate gate, dn_path path,
+               dn::ChunkArgs* a, bool* use_tc) {
+    if (B < 0 || T < 0 || H < 0) return fail(DN_ERR_INVALID, "B, T, H must be >= 0 (got %d, %d, %d)", B, T, H);
+    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
+    if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
+        return fail(DN_ERR_INVALID, "unknown gate %d", (int)gate);
+    if (path != DN_PATH_AUTO && path != DN_PATH_SIMT && path != DN_PATH_TC && path != DN_PATH_TC_STALL_TEST)
+        return fail(DN_ERR_INVALID, "unknown path %d", (int)path);
+    if (d_k <= 0 || d_v <= 0) return fail(DN_ERR_INVALID, "d_k, d_v must be > 0");
+    if (chunk <= 0) return fail(DN_ERR_INVALID, "chunk must be > 0 (got %d)", chunk);
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(DN_ERR_UNSUPPORTED, "d_k, d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
+    *a = dn::ChunkArgs{};
+    a->B = B; a->T = T; a->H = H; a->dk = d_k; a->dv = d_v; a->chunk = chunk;
+    a->bf16 = dtype == DN_BF16; a->gate = (int)gate;
+    a->test_flags = path == DN_PATH_TC_STALL_TEST ? 1 : 0;
+    // kernel choice before any CUDA call: an unsupported request touches no device state
+    *use_tc = false;
+    if (path == DN_PATH_TC || path == DN_PATH_TC_STALL_TEST) {
+        if (!dn::tc_supports(*a))
+            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128 and no per-key gate");
+        *use_tc = true;
+    } else if (path == DN_PATH_AUTO) {
+        *use_tc = dn::tc_supports(*a);
+    }
+    if (!*use_tc && chunk > 64) return fail(DN_ERR_UNSUPPORTED, "chunk must be <= 64 (got %d)", chunk);
+    return DN_OK;
+}
+
+size_t workspace_needed(const dn::ChunkArgs& a, bool use_tc) {
+    return use_tc && (int64_t)a.B * a.H * a.T > 0 ? dn::tc_workspace_bytes(a) : 0;
+}
+
 }  // namespace
 
 extern "C" {
 
-int dn_version(void) { return (1 << 16) | 0; }
+int dn_version(void) { return (2 << 16) | 0; }
 
 const char* dn_status_str(int status) {
     switch (status) {
@@ -80,21 +115,27 @@ const char* dn_status_str(int status) {
 
 const char* dn_last_error(void) { return g_last_error; }
 
+int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk, dn_dtype dtype, dn_gate gate,
+                                dn_path path, size_t* bytes) {
+    if (!bytes) return fail(DN_ERR_INVALID, "bytes must not be NULL");
+    dn::ChunkArgs a;
+    bool use_tc;
+    const int st = plan_chunk(B, T, H, d_k, d_v, chunk, dtype, gate, path, &a, &use_tc);
+    if (st != DN_OK) return st;
+    *bytes = workspace_needed(a, use_tc);
+    return ok();
+}
+
 int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
                     const float* g, const float* S0, void* o, float* S_T,
                     int B, int T, int H, int d_k, int d_v, int chunk, float scale,
-                    dn_dtype dtype, dn_gate gate, dn_path path, void* cuda_stream) {
-    if (B < 0 || T < 0 || H < 0) return fail(DN_ERR_INVALID, "B, T, H must be >= 0 (got %d, %d, %d)", B, T, H);
-    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
-    if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
-        return fail(DN_ERR_INVALID, "unknown gate %d", (int)gate);
-    if (path != DN_PATH_AUTO && path != DN_PATH_SIMT && path != DN_PATH_TC && path != DN_PATH_TC_STALL_TEST)
-        return fail(DN_ERR_INVALID, "unknown path %d", (int)path);
-    if (d_k <= 0 || d_v <= 0) return fail(DN_ERR_INVALID, "d_k, d_v must be > 0");
-    if (chunk <= 0) return fail(DN_ERR_INVALID, "chunk must be > 0 (got %d)", chunk);
+                    dn_dtype dtype, dn_gate gate, dn_path path, void* workspace, size_t workspace_bytes,
+                    void* cuda_stream) {
+    dn::ChunkArgs a;
+    bool use_tc;
+    const int pst = plan_chunk(B, T, H, d_k, d_v, chunk, dtype, gate, path, &a, &use_tc);
+    if (pst != DN_OK) return pst;
     if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return fail(DN_ERR_INVALID, "scale is not finite");
-    if (!supported_d(d_k) || !supported_d(d_v))
-        return fail(DN_ERR_UNSUPPORTED, "d_k, d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
     const int64_t ntok = (int64_t)B * H * T;
     const int64_t esz = dtype == DN_BF16 ? 2 : 4;
     const bool empty_tokens = ntok == 0;
@@ -123,26 +164,22 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
         if (overlap(rst, r)) return fail(DN_ERR_INVALID, "S_T overlaps an input other than S0");
     if (S_T && S0 && (void*)S_T != (const void*)S0 && overlap(rst, rs0))
         return fail(DN_ERR_INVALID, "S_T partly overlaps S0");
+    const size_t need = workspace_needed(a, use_tc);
+    if (workspace && need > 0) {
+        if (workspace_bytes < need)
+            return fail(DN_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
+        if (!aligned(workspace, 256)) return fail(DN_ERR_INVALID, "workspace is not 256-byte aligned");
+        Range rw = rng(workspace, (int64_t)need);
+        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst};
+        for (Range r : all)
+            if (overlap(rw, r)) return fail(DN_ERR_INVALID, "workspace overlaps another argument");
+    }
 
     cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
     if ((int64_t)B * H == 0) return ok();
 
-    dn::ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T;
-    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk; a.scale = scale;
-    a.bf16 = dtype == DN_BF16; a.gate = (int)gate;
-    a.test_flags = path == DN_PATH_TC_STALL_TEST ? 1 : 0;
-
-    // kernel choice first: an unsupported request touches no device state
-    bool use_tc = false;
-    if (path == DN_PATH_TC || path == DN_PATH_TC_STALL_TEST) {
-        if (!dn::tc_supports(a))
-            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128 and no per-key gate");
-        use_tc = true;
-    } else if (path == DN_PATH_AUTO) {
-        use_tc = dn::tc_supports(a);
-    }
-    if (!use_tc && chunk > 64) return fail(DN_ERR_UNSUPPORTED, "chunk must be <= 64 (got %d)", chunk);
+    a.scale = scale;
 
     cudaError_t e;
     a.status = status_word(&e);
@@ -155,9 +192,24 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
         return e == cudaSuccess ? ok() : cuda_fail(e, "T = 0 state copy");
     }
 
-    e = use_tc ? dn::launch_chunk_tc(a, st) : dn::launch_chunk_simt(a, st);
-    if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core chunk kernel" : "SIMT chunk kernel");
-    return ok();
+    if (!use_tc) {
+        e = dn::launch_chunk_simt(a, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "SIMT chunk kernel");
+    }
+    // the tensor-core path keeps W^T and u^T of every chunk in a workspace: the
+    // caller's, else a stream-ordered allocation released on the same stream
+    void* own = nullptr;
+    if (!workspace) {
+        e = cudaMallocAsync(&own, need, st);
+        if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    }
+    a.ws = workspace ? workspace : own;
+    e = dn::launch_chunk_tc(a, st);
+    if (own) {
+        const cudaError_t ef = cudaFreeAsync(own, st);
+        if (e == cudaSuccess) e = ef;
+    }
+    return e == cudaSuccess ? ok() : cuda_fail(e, "tensor-core chunk kernels");
 }
 
 int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
@@ -165,7 +217,7 @@ int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
                  int B, int T, int H, int d_k, int d_v, int chunk, float scale,
                  dn_dtype dtype, dn_gate gate, void* cuda_stream) {
     return dn_chunk_fwd_ex(q, k, v, beta, g, S0, o, S_T, B, T, H, d_k, d_v, chunk, scale,
-                           dtype, gate, DN_PATH_AUTO, cuda_stream);
+                           dtype, gate, DN_PATH_AUTO, nullptr, 0, cuda_stream);
 }
 
 int dn_decode_step(const void* q, const void* k, const void* v, const float* beta,

@@ -17,7 +17,8 @@ struct ChunkArgs {
     bool bf16;
     int gate;                 // Gate
     unsigned int* status;     // device status word of the current device
-    int test_flags;           // 1: withhold the tensor-core kernel's input loads (failure-path self-test)
+    int test_flags;           // 1: withhold the tensor-core kernels' input loads (failure-path self-test)
+    void* ws;                 // tensor-core path: workspace of tc_workspace_bytes(), 256-byte aligned
 };
 
 struct DecodeArgs {
@@ -34,9 +35,12 @@ struct DecodeArgs {
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t st);
 
-// Tensor-core (tcgen05) chunk kernel.  tc_supports() says whether the request
-// is inside the kernel's coverage (bf16, chunk 64, d_k = d_v = 128).
+// Tensor-core (tcgen05) chunk path: the per-chunk UT/WY transform (chunk_wy.cu)
+// then the state pass (chunk_tc.cu).  tc_supports() says whether the request
+// is inside its coverage (bf16, chunk 64, d_k = d_v = 128, no per-key gate);
+// tc_workspace_bytes() is the size of a.ws it needs (W^T and u^T of every chunk).
 bool tc_supports(const ChunkArgs& a);
+size_t tc_workspace_bytes(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st);
 
 }  // namespace dn

@@ -24,9 +24,12 @@
  * (selinyilmaz.dev), its KDA update with a per-key-channel decay.
  *
  * Conventions for every entry point
- *   - All tensor pointers are DEVICE pointers owned by the caller; the library
- *     allocates no device memory and keeps no state between calls except a
- *     per-device status word read by dn_device_status().
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library keeps no state between calls except a per-device status word
+ *     read by dn_device_status(), and allocates no device memory except the
+ *     tensor-core prefill's workspace when the caller passes none (a
+ *     stream-ordered cudaMallocAsync / cudaFreeAsync pair on the call's
+ *     stream; see dn_chunk_fwd_workspace_size).
  *   - Every layout is dense row-major (C order) with the shapes given.
  *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the
  *     legacy default stream).  Inputs must stay valid until the work ends.
@@ -43,6 +46,7 @@
 #ifndef DN_H
 #define DN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -74,9 +78,9 @@ typedef enum {
 typedef enum {
     DN_PATH_AUTO = 0,     /* tensor-core path when it supports the request, else SIMT */
     DN_PATH_SIMT = 1,     /* fp32 CUDA-core chunk kernel: any chunk 1..64          */
-    DN_PATH_TC = 2,       /* tcgen05 chunk kernel: bf16, chunk 64, d_k = d_v = 128 */
-    /* Self-test of the failure path: the tensor-core kernel runs with its input
-     * loads withheld, so every bounded wait inside it expires (about one second);
+    DN_PATH_TC = 2,       /* tcgen05 chunk kernels: bf16, chunk 64, d_k = d_v = 128, no per-key gate */
+    /* Self-test of the failure path: the tensor-core kernels run with their input
+     * loads withheld, so every bounded wait inside them expires (about two seconds);
      * nothing is written to o or S_T, dn_device_status() then returns
      * DN_ERR_TIMEOUT, and the CUDA context stays usable. */
     DN_PATH_TC_STALL_TEST = 3
@@ -100,8 +104,10 @@ typedef enum {
  *   d_k, d_v in {64, 128}.  B, H, T >= 0 (T = 0 writes S_T = S0 or zeros).
  *
  * o must not overlap any input.  Returns DN_ERR_UNSUPPORTED for a d or chunk
- * outside the ranges above (or a DN_PATH_TC request the tensor-core kernel
- * does not cover).
+ * outside the ranges above (or a DN_PATH_TC request the tensor-core kernels
+ * do not cover).  The kernels are chosen as by DN_PATH_AUTO; a workspace the
+ * tensor-core path needs is allocated and freed stream-ordered on
+ * `cuda_stream` (pass one to dn_chunk_fwd_ex to avoid that).
  */
 DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
                  const float* beta, const float* g, const float* S0,
@@ -109,12 +115,35 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
                  int B, int T, int H, int d_k, int d_v, int chunk, float scale,
                  dn_dtype dtype, dn_gate gate, void* cuda_stream);
 
-/* dn_chunk_fwd with an explicit kernel choice (for tests and benchmarks). */
+/*
+ * dn_chunk_fwd_workspace_size -- bytes of device workspace that dn_chunk_fwd_ex
+ * uses for this request on `path` (0 when the chosen kernels need none).  The
+ * tensor-core path computes W = T diag(beta e^G) K and u = T diag(beta) V of
+ * every chunk ("Training it: the WY trick", D2L 12.5) in a kernel that runs
+ * over all chunks at once, then streams them into the sequential state pass:
+ * 32 KiB per (b, h, chunk), i.e. B * H * ceil(T / 64) * 32768 bytes.  Sizes
+ * are checked as in dn_chunk_fwd_ex; *bytes is written on DN_OK only.
+ */
+DN_API int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk,
+                                       dn_dtype dtype, dn_gate gate, dn_path path, size_t* bytes);
+
+/*
+ * dn_chunk_fwd with an explicit kernel choice and workspace.
+ *   workspace        NULL: when the kernels need one, the call allocates it
+ *                    stream-ordered on `cuda_stream` and frees it there;
+ *                    otherwise a device buffer of at least
+ *                    dn_chunk_fwd_workspace_size() bytes, 256-byte aligned,
+ *                    overlapping no argument.  Its contents are scratch
+ *                    (overwritten; nothing needs initialising) and it must not
+ *                    be used by other work until this call's work has ended.
+ *   workspace_bytes  its size (ignored when workspace is NULL).
+ */
 DN_API int dn_chunk_fwd_ex(const void* q, const void* k, const void* v,
                     const float* beta, const float* g, const float* S0,
                     void* o, float* S_T,
                     int B, int T, int H, int d_k, int d_v, int chunk, float scale,
-                    dn_dtype dtype, dn_gate gate, dn_path path, void* cuda_stream);
+                    dn_dtype dtype, dn_gate gate, dn_path path,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
  * dn_decode_step -- one recurrent step ("The recurrent form", ch. 28; KDA's

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dn_version() >> 16 == 1
+    assert lib.dn_version() >> 16 == 2
     for code in range(5):
         assert lib.dn_status_str(code).startswith(b"DN_")
     assert lib.dn_status_str(99) == b"unknown dn_status"
@@ -49,12 +49,17 @@ STEP = 0x01000000
 def chunk_call(lib, **over):
     args = dict(q=A, k=A + STEP, v=A + 2 * STEP, beta=A + 3 * STEP, g=A + 4 * STEP, S0=None,
                 o=A + 5 * STEP, S_T=A + 6 * STEP, B=1, T=8, H=1, dk=64, dv=64, chunk=8,
-                scale=1.0, dtype=0, gate=1, path=0)
+                scale=1.0, dtype=0, gate=1, path=0, ws=None, ws_bytes=0)
     args.update(over)
     return lib.dn_chunk_fwd_ex(args["q"], args["k"], args["v"], args["beta"], args["g"], args["S0"],
                                args["o"], args["S_T"], args["B"], args["T"], args["H"], args["dk"],
                                args["dv"], args["chunk"], args["scale"], args["dtype"], args["gate"],
-                               args["path"], None)
+                               args["path"], args["ws"], args["ws_bytes"], None)
+
+
+# a request the tensor-core path covers (bf16, chunk 64, d_k = d_v = 128)
+TC = dict(dtype=1, dk=128, dv=128, chunk=64, path=2)
+WS = A + 8 * STEP
 
 
 @pytest.mark.parametrize("over,code", [
@@ -79,10 +84,35 @@ def chunk_call(lib, **over):
     (dict(dv=256), dn.DN_ERR_UNSUPPORTED),
     (dict(path=2), dn.DN_ERR_UNSUPPORTED),                    # tensor-core path needs bf16, d = 128
     (dict(path=3), dn.DN_ERR_UNSUPPORTED),                    # so does its self-test
+    (dict(TC, ws=WS, ws_bytes=32767), dn.DN_ERR_INVALID),     # workspace smaller than one chunk's W, u
+    (dict(TC, ws=WS + 128, ws_bytes=1 << 20), dn.DN_ERR_INVALID),   # not 256-byte aligned
+    (dict(TC, ws=A + 256, ws_bytes=1 << 20), dn.DN_ERR_INVALID),    # overlaps q
+    (dict(TC, ws=A + 6 * STEP, ws_bytes=1 << 20), dn.DN_ERR_INVALID),  # overlaps S_T
 ])
 def test_chunk_fwd_rejects(lib, over, code):
     assert chunk_call(lib, **over) == code
     assert lib.dn_last_error() != b""
+
+
+def ws_size(lib, B=2, T=130, H=3, dk=128, dv=128, chunk=64, dtype=1, gate=1, path=0):
+    out = ctypes.c_size_t(12345)
+    st = lib.dn_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, dtype, gate, path, ctypes.byref(out))
+    return st, out.value
+
+
+def test_workspace_size():
+    lib = dn.load_library()
+    # W^T and u^T, bf16 128 x 64 each, per (b, h, chunk): ceil(130 / 64) = 3 chunks
+    assert ws_size(lib) == (dn.DN_OK, 2 * 3 * 3 * 2 * 128 * 64 * 2)
+    assert ws_size(lib, path=2) == (dn.DN_OK, 2 * 3 * 3 * 32768)
+    assert ws_size(lib, T=0) == (dn.DN_OK, 0)
+    assert ws_size(lib, path=1) == (dn.DN_OK, 0)             # SIMT needs none
+    assert ws_size(lib, dtype=0) == (dn.DN_OK, 0)            # fp32 runs on SIMT under auto
+    assert ws_size(lib, gate=2) == (dn.DN_OK, 0)             # so does the per-key gate
+    assert ws_size(lib, dtype=0, path=2)[0] == dn.DN_ERR_UNSUPPORTED
+    assert ws_size(lib, B=-1) == (dn.DN_ERR_INVALID, 12345)  # not written on failure
+    assert lib.dn_chunk_fwd_workspace_size(1, 8, 1, 128, 128, 64, 1, 1, 0, None) == dn.DN_ERR_INVALID
+    assert dn.dn_chunk_fwd_workspace_size(1, 64, 1, 128, 128) == 32768
 
 
 def test_chunk_fwd_empty_batch_is_ok_without_device(lib):

@@ -143,6 +143,35 @@ def test_chunk_overwrites_poisoned_outputs(cuda_device, path):
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
 
 
+def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
+    # the tensor-core path keeps W^T and u^T of every chunk in a workspace: a
+    # caller's buffer (poisoned with NaN first: it is scratch, nothing is read
+    # before it is written) and the library's own stream-ordered allocation
+    # give bit-identical results, which match the oracle
+    inp = W.gen_prefill(2, 3, 200, 128, 128, dtype="bf16", gate="scalar", seed=12, s0_std=0.2)
+    d = to_dev(inp)
+    sc = 128 ** -0.5
+    nbytes = dn.dn_chunk_fwd_workspace_size(2, 200, 3, 128, 128, path="tc")
+    assert nbytes == 2 * 3 * 4 * 32768
+    ws = torch.full((nbytes // 2,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    outs = []
+    for w in (ws, None):
+        o = torch.empty((2, 3, 200, 128), dtype=torch.bfloat16, device="cuda")
+        S = torch.empty((2, 3, 128, 128), device="cuda")
+        dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o, S, scale=sc, path="tc",
+                        workspace=w)
+        outs.append((o, S))
+    dn.dn_device_status()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(outs[0][0], ro, "bf16", "o")
+    assert_close(outs[0][1], rS, "bf16", "S_T")
+    with pytest.raises(dn.DNError) as ei:
+        dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], outs[0][0], outs[0][1], scale=sc,
+                        path="tc", workspace=ws[: nbytes // 4])
+    assert ei.value.status == dn.DN_ERR_INVALID
+
+
 def test_chunk_empty_inputs(cuda_device):
     # T = 0: no output rows; S_T = S0 (or zeros).  B = 0: nothing at all.
     S0 = torch.randn(2, 3, 64, 64, device="cuda")
