@@ -34,8 +34,8 @@ _DTYPES = {"f32": 0, "bf16": 1}
 _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
-ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_decode_step",
-               "dn_device_status", "dn_status_str", "dn_last_error", "dn_version")
+ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
+               "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None

@@ -98,6 +98,10 @@ size_t workspace_needed(const dn::ChunkArgs& a, bool use_tc) {
 
 }  // namespace
 
+namespace dn {
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace dn
+
 extern "C" {
 
 int dn_version(void) { return (2 << 16) | 0; }

@@ -43,4 +43,7 @@ bool tc_supports(const ChunkArgs& a);
 size_t tc_workspace_bytes(const ChunkArgs& a);
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st);
 
+// Record `msg` as the calling thread's dn_last_error() and return `code`.
+int report_error(int code, const char* msg);
+
 }  // namespace dn

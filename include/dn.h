@@ -146,6 +146,38 @@ DN_API int dn_chunk_fwd_ex(const void* q, const void* k, const void* v,
                     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * dn_chunk_fwd_noalloc -- dn_chunk_fwd for callers that cannot allocate device
+ * memory (a process that reserved the device's memory for its own pools, a
+ * framework whose allocator must see every byte, or a latency-critical loop
+ * that cannot afford an allocation or its implicit synchronisation).  The
+ * pages have no counterpart: it is a deployment variant of dn_chunk_fwd.
+ *
+ * Same arguments, kernel choice and results as dn_chunk_fwd.  The tensor-core
+ * path's scratch workspace (dn_chunk_fwd_workspace_size bytes) comes from a
+ * fixed area of DN_NOALLOC_SCRATCH_BYTES compiled into the library; no call
+ * allocates or frees memory.
+ *   - The area exists once per device, created when the library's code is
+ *     loaded there, and is held until the process exits.
+ *   - The first call on a device looks up the area's address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - A request needing more scratch than the area returns DN_ERR_UNSUPPORTED
+ *     (dn_last_error() gives both sizes) before any device work.
+ *   - Every call on a device shares the area and it keeps the last call's
+ *     contents.  Nothing in it needs clearing (each call writes every byte it
+ *     reads), but calls whose GPU work overlaps (other streams, other host
+ *     threads) race on it: order them on one stream, or use dn_chunk_fwd_ex
+ *     with separate workspaces.
+ */
+#define DN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)   /* 64 MiB: 2048 (b, h, chunk) tiles */
+
+DN_API int dn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                const float* beta, const float* g, const float* S0,
+                                void* o, float* S_T,
+                                int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                                dn_dtype dtype, dn_gate gate, void* cuda_stream);
+
+/*
  * dn_decode_step -- one recurrent step ("The recurrent form", ch. 28; KDA's
  * recurrence in "A walk through of the DeltaNet family").
  *
