@@ -20,8 +20,25 @@ constexpr int kC = 64;                      // chunk
 constexpr int kD = 128;                     // d_k = d_v
 constexpr uint64_t kWaitNs = 1000000000ull; // every mbarrier wait gives up after 1 s
 
-// One chunk's W^T or u^T in the workspace: bf16, [128 rows (d_k or d_v)][64 columns (position)].
-constexpr size_t kWsTileBytes = (size_t)kD * kC * 2;
+// Workspace per (b, h, chunk), written by chunk_wy.cu and read by chunk_tc.cu,
+// four bf16 arrays one after another:
+//   -W   [tiles * 64 rows (position)][128 (d_k)]
+//   u^T  [tiles * 128 rows (d_v)][64 (position)]
+//   P    [tiles * 64 rows (i)][64 (j)]
+//   Qh   [tiles * 64 rows (position)][128 (d_k)]
+constexpr size_t kWsWBytes = (size_t)kC * kD * 2;
+constexpr size_t kWsUBytes = (size_t)kD * kC * 2;
+constexpr size_t kWsPBytes = (size_t)kC * kC * 2;
+constexpr size_t kWsQBytes = (size_t)kC * kD * 2;
+constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes + kWsQBytes;
+
+// Tensor maps of the tensor-core path (128-byte swizzle, 64-column boxes):
+// q, k, v as [B H T][128] with 64-row boxes; the workspace's -W and Qh as
+// [tiles 64][128] with 64-row boxes, u^T as [tiles 128][64] with 128-row
+// boxes, P as [tiles 64][64] with 64-row boxes.
+struct TcMaps {
+    CUtensorMap q, k, v, w, u, p, qh;
+};
 
 // Gate slot of one chunk (floats).
 constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320;
@@ -52,8 +69,10 @@ __device__ __forceinline__ void chunk_gates(float* gs, float b0, float b1, float
 }
 
 // e^(G_i - G_j) = 2^(G2_i - G2_j) with G2 = G log2(e), for j <= i (the
-// exponent is <= 0 for g <= 0; very old positions underflow to 0).
-__device__ __forceinline__ float decay2(float g2i, float g2j) { return exp2f(g2i - g2j); }
+// exponent is <= 0 for g <= 0; very old positions underflow to 0).  The SFU's
+// 2^x is accurate to about 2^-22 relative, far inside the bf16 rounding of
+// the tiles these factors enter.
+__device__ __forceinline__ float decay2(float g2i, float g2j) { return ex2_approx(g2i - g2j); }
 
 // Bounded mbarrier waits for a CTA whose roles share an abort flag in shared memory.
 struct Ctl {
@@ -107,9 +126,7 @@ inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t 
 
 }  // namespace tc
 
-// The UT/WY transform of every chunk into the workspace halves w_ws and u_ws
-// (chunk_wy.cu); tk, tv map k and v as [B H T][128] with 64 x 64 boxes.
-cudaError_t launch_chunk_wy(const ChunkArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                            __nv_bfloat16* w_ws, __nv_bfloat16* u_ws, cudaStream_t st);
+// The state-independent part of every chunk into the workspace (chunk_wy.cu).
+cudaError_t launch_chunk_wy(const ChunkArgs& a, const tc::TcMaps& m, cudaStream_t st);
 
 }  // namespace dn

@@ -1,5 +1,6 @@
-// chunk_wy.cu -- the UT/WY transform of every chunk, in parallel over
-// (b, h, chunk), on the sm_100a tensor cores and CUDA cores.
+// chunk_wy.cu -- everything of the chunked delta rule that does not depend on
+// the state, in parallel over (b, h, chunk), on the sm_100a tensor cores and
+// CUDA cores.
 //
 // Same mathematics as "Linear attention and Gated DeltaNet" (ch. 28, "The
 // chunked form") and D2L 12.5 ("Training it: the WY trick"): inside a chunk
@@ -8,26 +9,30 @@
 //
 //   A = strict_tril(beta_i k_i.k_j D_ij),   T = (I + A)^-1   (unit lower)
 //   W = T diag(beta e^G) K,                 u = T diag(beta) V
+//   P = scale tril(q_i.k_j D_ij)            (the intra-chunk attention)
+//   Qh = scale e^G Q                        (the queries seen from the chunk start)
 //
-// Nothing here depends on the state, so every chunk is an independent CTA (two
-// fit on an SM).  W^T and u^T leave as bf16 [128][64] tiles of the workspace,
-// which the state-pass kernel (chunk_tc.cu) streams back with TMA.  One CTA:
+// Every chunk is an independent CTA (three fit on an SM).  The state pass
+// (chunk_tc.cu) streams the results back with TMA from the workspace, as bf16
+// tiles: -W [64 rows][128] (row-major, negated so that S^T (-W)^T = -(W S)^T),
+// u^T [128][64], P [64][64] and Qh [64][128].  One CTA:
 //
-//   TMA       K (loaded twice, stacked, so that the gram has M = 128) and V
-//   tcgen05   [K;K] K^T -> TMEM (bf16 -> fp32)
-//   CUDA core masks and decay -> A (fp32, shared memory)
+//   TMA       K and Q tiles, stacked per 64-column block as [K rows | Q rows]
+//   tcgen05   [K;Q] K^T -> TMEM (bf16 -> fp32): K K^T for A, Q K^T for P
+//   CUDA core masks and decay -> A (fp32, shared memory) and P (bf16); Qh in place
+//   TMA       P and Qh out, then V over the Q rows, while the rest runs
 //   CUDA core T = (I + A)^-1: the 16 x 16 diagonal blocks D_k = (I + A_kk)^-1
 //             by forward substitution, M_kl = D_k A_kl, then
 //             T_kl = -sum_{m=l}^{k-1} M_km T_ml in three rounds (fp32);
-//             T diag(beta e^G) and T diag(beta) as bf16 operand tiles
+//             then T diag(beta e^G) and T diag(beta) as bf16 operand tiles
 //   tcgen05   W^T = K^T (T diag(beta e^G))^T, u^T = V^T (T diag(beta))^T -> TMEM
-//   epilogue  TMEM -> bf16 -> workspace
+//   epilogue  TMEM -> bf16 tiles in shared memory -> TMA stores to the workspace
 //
-// A partial last chunk has beta = 0 and g = 0 past its end: those rows of A,
-// and those columns of W^T and u^T, are zero (equal to zero padding).  Rows
-// past the end of the tensor are zero-filled by TMA; rows of the next head
-// are multiplied by those zeros.  Every wait is bounded; on a timeout the CTA
-// records it in the status word and exits.
+// A partial last chunk has beta = 0 and g = 0 past its end: those rows of A
+// and P, and those columns of W^T and u^T, are zero (equal to zero padding).
+// Rows past the end of the tensor are zero-filled by TMA; rows of the next
+// head are multiplied by those zeros.  Every wait is bounded; on a timeout the
+// CTA records it in the status word and exits.
 #include "chunk_tc_common.cuh"
 #include "dn_kernels.h"
 
@@ -41,19 +46,19 @@ namespace {
 constexpr int kNT = 256;        // 8 warps
 
 // TMEM columns (32-bit, 128 lanes)
-constexpr uint32_t TM_G = 0;    // gram [K;K] K^T (lanes 64-127 repeat lanes 0-63)
+constexpr uint32_t TM_G = 0;    // gram [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T
 constexpr uint32_t TM_W = 0;    // W^T fp32 [dk][C], after the gram has been read
 constexpr uint32_t TM_U = 64;   // u^T fp32 [dv][C]
 constexpr uint32_t TM_COLS = 128;
 
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_K = 0;           // [d-block][K rows | K rows again][128 B] = 32 KiB
-constexpr uint32_t OFF_TW = 8192;       // T diag(beta e^G) in d-block 0's copy, once the gram is done
-constexpr uint32_t OFF_TB = 24576;      // T diag(beta) in d-block 1's copy
-constexpr uint32_t OFF_V = 32768;       // [d-block][64 rows][128 B] = 16 KiB
-constexpr uint32_t OFF_A = 49152;       // fp32 64 x 68: A, then M = D^-1 A
-constexpr uint32_t OFF_T = 66560;       // fp32 64 x 68: T = (I + A)^-1
-constexpr uint32_t OFF_GATE = 83968;    // one gate slot
+constexpr uint32_t OFF_KV = 0;          // [d-block][K rows 0-63 | Q (Qh) rows, then V rows][128 B] = 32 KiB;
+                                        // last, the -W and u^T output tiles
+constexpr uint32_t OFF_A = 32768;       // fp32 64 x 68: A, then M = D^-1 A; then the bf16 tiles
+constexpr uint32_t OFF_TW = OFF_A;      //   T diag(beta e^G), K-major B [N=i][K=j]: [64 rows][128 B]
+constexpr uint32_t OFF_TB = OFF_A + 8192;   // T diag(beta), same layout
+constexpr uint32_t OFF_T = 50176;       // fp32 64 x 68: T = (I + A)^-1; first the P output tile
+constexpr uint32_t OFF_GATE = 67584;    // one gate slot
 constexpr uint32_t OFF_BAR = OFF_GATE + GATE_FLOATS * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 enum { B_FULL = 0, B_MMA = 1 };
@@ -90,31 +95,21 @@ __device__ __forceinline__ void blk16_store(float* Z, int zr, int zc, const floa
     *reinterpret_cast<float4*>(Z + fidx(zr + ii, zc + j0 + 4)) = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
-// Eight consecutive entries t[0..7] of T at (row, col0..col0+7) -> one
-// 16-byte chunk of each bf16 operand tile, T diag(beta e^G) and T diag(beta).
-__device__ __forceinline__ void store_t_tiles(uint32_t tw, uint32_t tb, const float* gs, int row, int col0,
-                                              const float (&t)[8]) {
-    const float4 b0 = *reinterpret_cast<const float4*>(gs + G_BETA + col0);
-    const float4 b1 = *reinterpret_cast<const float4*>(gs + G_BETA + col0 + 4);
-    const float4 w0 = *reinterpret_cast<const float4*>(gs + G_BEG + col0);
-    const float4 w1 = *reinterpret_cast<const float4*>(gs + G_BEG + col0 + 4);
-    const uint32_t off = sw128_off(row, col0 >> 3);
-    st_shared_v4(tw + off, pack_bf16x2(t[0] * w0.x, t[1] * w0.y), pack_bf16x2(t[2] * w0.z, t[3] * w0.w),
-                 pack_bf16x2(t[4] * w1.x, t[5] * w1.y), pack_bf16x2(t[6] * w1.z, t[7] * w1.w));
-    st_shared_v4(tb + off, pack_bf16x2(t[0] * b0.x, t[1] * b0.y), pack_bf16x2(t[2] * b0.z, t[3] * b0.w),
-                 pack_bf16x2(t[4] * b1.x, t[5] * b1.y), pack_bf16x2(t[6] * b1.z, t[7] * b1.w));
+// T_zr,zc = -acc (fp32).
+__device__ __forceinline__ void blk16_store_neg(float* Tm, int zr, int zc, const float (&acc)[8], int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0 + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
 }
 
-// T_zr,zc = -acc: into T (fp32) and into the two bf16 operand tiles.
-__device__ __forceinline__ void blk16_store_t(float* Tm, uint32_t tw, uint32_t tb, const float* gs, int zr, int zc,
-                                              const float (&acc)[8], int lane) {
-    const int ii = lane >> 1, j0 = (lane & 1) * 8;
-    float t[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) t[e] = -acc[e];
-    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0)) = make_float4(t[0], t[1], t[2], t[3]);
-    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0 + 4)) = make_float4(t[4], t[5], t[6], t[7]);
-    store_t_tiles(tw, tb, gs, zr + ii, zc + j0, t);
+// Scale 8 bf16 values (one 16-byte chunk) by f and store them at dst.
+__device__ __forceinline__ void scale_chunk(uint32_t src, uint32_t dst, float f) {
+    const uint4 w = ld_shared_v4(src);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+    st_shared_v4(dst, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
 }
 
 __device__ __forceinline__ void zero8(float (&a)[8]) {
@@ -125,10 +120,13 @@ __device__ __forceinline__ void zero8(float (&a)[8]) {
 }  // namespace
 
 template <int GATE>
-__global__ void __launch_bounds__(kNT, 2)
-chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const float* __restrict__ beta, const float* __restrict__ g, __nv_bfloat16* __restrict__ w_out,
-                __nv_bfloat16* __restrict__ u_out, int T, int n, unsigned int* status, int test_flags) {
+__global__ void __launch_bounds__(kNT, 3)
+chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_p,
+                const __grid_constant__ CUtensorMap tm_qh, const float* __restrict__ beta,
+                const float* __restrict__ g, int T, int n, float scale,
+                unsigned int* status, int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
@@ -148,6 +146,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int Cc = min(kC, T - c * kC);
     const int64_t t0 = bh * T + (int64_t)c * kC;
     const bool load = !(test_flags & 1);
+    int loads = 0;                                   // load groups issued (thread 0)
 
     if (tid == 0) {
         mbar_init(ctl.bar(B_FULL), 1);
@@ -165,17 +164,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
 
     if (tid == 0 && load) {
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
         const uint32_t fb = ctl.bar(B_FULL);
         const int y = (int)t0;
-        mbar_arrive_expect_tx(fb, 6 * 8192);
-        tma_load_2d(sb + OFF_K + 0, &tm_k, 0, y, fb);
-        tma_load_2d(sb + OFF_K + 16384, &tm_k, 64, y, fb);
-        tma_load_2d(sb + OFF_K + 8192, &tm_k, 0, y, fb);
-        tma_load_2d(sb + OFF_K + 24576, &tm_k, 64, y, fb);
-        tma_load_2d(sb + OFF_V + 0, &tm_v, 0, y, fb);
-        tma_load_2d(sb + OFF_V + 8192, &tm_v, 64, y, fb);
+        mbar_arrive_expect_tx(fb, 4 * 8192);
+        tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, y, fb);
+        tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, y, fb);
+        tma_load_2d(sb + OFF_KV + 8192, &tm_q, 0, y, fb);
+        tma_load_2d(sb + OFF_KV + 24576, &tm_q, 64, y, fb);
+        loads = 1;
     }
     if (warp == 2) {
         const float b0 = lane < Cc ? beta[t0 + lane] : 0.f;
@@ -189,14 +185,14 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     bool ok = true;
     if (tid == 0) {
-        // [K;K] K^T once K has landed
+        // [K;Q] K^T once the tiles have landed
         ok = ctl.wait(B_FULL, 0);
         if (ok) {
             tc_fence_after();
             const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = sb + OFF_K + (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint32_t a = sb + OFF_KV + (kk >> 2) * 16384 + (kk & 3) * 32;
                 mma_bf16(tmem + TM_G, sw128_desc(a, 16, 1024), sw128_desc(a, 16, 1024), idesc, kk > 0);
             }
             mma_commit(ctl.bar(B_MMA));
@@ -207,40 +203,83 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
 
-    // ---- A = strict_tril(beta_i (K K^T)_ij D_ij): lane r holds row r mod 64; the two
-    //      copies of a row split its columns, the two warps of a lane quarter again ----
+    // ---- A = strict_tril(beta_i (K K^T)_ij D_ij) from TMEM lanes 0-63 (warps 0, 1, 4, 5)
+    //      and P = scale tril((Q K^T)_ij D_ij) from lanes 64-127 (warps 2, 3, 6, 7), 32
+    //      columns per thread --------------------------------------------------------------
     {
         const int q = warp & 3;
-        const int r = (q << 5) + lane;
-        const int i = r & 63;
-        const int j0 = ((r >> 6) << 5) + ((warp >> 2) << 4);
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
-        tmem_wait_ld();
-        const float bi = gs[G_BETA + i];              // zero past the chunk's end
+        const int i = ((q & 1) << 5) + lane;
+        const int j0 = (warp >> 2) << 5;
         const float g2i = gs[G_G2 + i];
+        if (q < 2) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
+            tmem_wait_ld();
+            const float bi = gs[G_BETA + i];          // zero past the chunk's end
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 gj = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 4 * q4);
-            const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
-            float a[4];
+            for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 gj = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 4 * q4);
+                const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+                float a[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = j0 + 4 * q4 + e;
-                a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j0 + 4 * q4 + e;
+                    a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                }
+                *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
             }
-            *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
-        }
-        // the K copy is free now: zero the operand tiles (their blocks above the
-        // block diagonal stay zero)
+        } else if (q == 2 && j0 == 32) {
+            // rows 0-31 x columns 32-63 lie above the diagonal
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const uint32_t off = (uint32_t)(tid + u * kNT) * 16;    // 512 chunks of 16 B per tile
-            st_shared_v4(sb + OFF_TW + off, 0u, 0u, 0u, 0u);
-            st_shared_v4(sb + OFF_TB + off, 0u, 0u, 0u, 0u);
+            for (int q4 = 0; q4 < 4; ++q4) st_shared_v4(sb + OFF_T + sw128_off(i, 4 + q4), 0u, 0u, 0u, 0u);
+        } else {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
+            tmem_wait_ld();
+            const float si = i < Cc ? scale : 0.f;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
+                const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
+                const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                float pv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = j0 + 8 * q4 + e;
+                    pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                }
+                st_shared_v4(sb + OFF_T + sw128_off(i, (j0 >> 3) + q4), pack_bf16x2(pv[0], pv[1]),
+                             pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+            }
+        }
+        // Qh = scale e^G Q in place over the Q rows (the gram has read them)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int x = tid + u * kNT;                   // 0..1023: (d-block, row, 16-byte chunk)
+            const int blk = x >> 9, r = (x >> 3) & 63, ch = x & 7;
+            const uint32_t a = sb + OFF_KV + blk * 16384 + 8192 + sw128_off(r, ch);
+            scale_chunk(a, a, r < Cc ? scale * gs[G_EG + r] : 0.f);
         }
     }
+    fence_async_smem();
     tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        // P and Qh out; then V over the Q rows, and T's buffer is reused, once the copies have read them
+        const int y = (int)(tile * kC);
+        tma_store_2d(&tm_p, 0, y, sb + OFF_T);
+        tma_store_2d(&tm_qh, 0, y, sb + OFF_KV + 8192);
+        tma_store_2d(&tm_qh, 64, y, sb + OFF_KV + 24576);
+        bulk_commit_group();
+        bulk_wait_read_all();
+        if (load) {
+            const uint32_t fb = ctl.bar(B_FULL);
+            mbar_arrive_expect_tx(fb, 2 * 8192);
+            tma_load_2d(sb + OFF_KV + 8192, &tm_v, 0, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 24576, &tm_v, 64, (int)t0, fb);
+            loads = 2;
+        }
+    }
     __syncthreads();
 
     // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
@@ -263,7 +302,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
     }
     __syncthreads();
-    // ---- M_kl = D_k A_kl (k > l), in place of A_kl; warps 6, 7: D_k -> operand tiles ----
+    // ---- M_kl = D_k A_kl (k > l), in place of A_kl -------------------------------------
     if (warp < 6) {
         // (k, l) = (1,0) (2,0) (3,0) (2,1) (3,1) (3,2) for warps 0..5
         const int k = (0x332321 >> (4 * warp)) & 15, l = (0x211000 >> (4 * warp)) & 15;
@@ -272,73 +311,113 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
         __syncwarp();
         blk16_store(Am, 16 * k, 16 * l, acc, lane);
-    } else {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int x = (warp - 6) * 32 + lane + u * 64;     // 0..127
-            const int blk = x >> 5, i = 16 * blk + ((x >> 1) & 15), j0 = 16 * blk + 8 * (x & 1);
-            const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, j0));
-            const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, j0 + 4));
-            const float t[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-            store_t_tiles(sb + OFF_TW, sb + OFF_TB, gs, i, j0, t);
-        }
     }
     __syncthreads();
     // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds ------------------------------
     {
         float acc[8];
         zero8(acc);
-        const uint32_t tw = sb + OFF_TW, tb = sb + OFF_TB;
-        if (warp == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 16, 0, acc, lane); }
-        if (warp == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store_t(Tm, tw, tb, gs, 32, 16, acc, lane); }
-        if (warp == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 32, acc, lane); }
+        if (warp == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store_neg(Tm, 16, 0, acc, lane); }
+        if (warp == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store_neg(Tm, 32, 16, acc, lane); }
+        if (warp == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store_neg(Tm, 48, 32, acc, lane); }
         if (warp == 3) blk16(Am, 32, 0, Tm, 0, 0, acc, lane);
         if (warp == 4) blk16(Am, 48, 16, Tm, 16, 16, acc, lane);
         if (warp == 5) blk16(Am, 48, 0, Tm, 0, 0, acc, lane);
         __syncthreads();
-        if (warp == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 32, 0, acc, lane); }
-        if (warp == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 16, acc, lane); }
+        if (warp == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store_neg(Tm, 32, 0, acc, lane); }
+        if (warp == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store_neg(Tm, 48, 16, acc, lane); }
         if (warp == 5) blk16(Am, 48, 16, Tm, 16, 0, acc, lane);
         __syncthreads();
-        if (warp == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store_t(Tm, tw, tb, gs, 48, 0, acc, lane); }
+        if (warp == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store_neg(Tm, 48, 0, acc, lane); }
+    }
+    __syncthreads();
+    // ---- T diag(beta e^G) and T diag(beta) as bf16 operand tiles, over A (zero above
+    //      the block diagonal, where T was never written) ----------------------------------
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int x = tid + u * kNT;                   // 0..511: (row, 8-column chunk)
+        const int i = x >> 3, ch = x & 7;
+        uint32_t w4[4] = {0u, 0u, 0u, 0u}, b4[4] = {0u, 0u, 0u, 0u};
+        if ((ch >> 1) <= (i >> 4)) {
+            const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
+            const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
+            const float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
+            const float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
+            const float4 c0 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch);
+            const float4 c1 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch + 4);
+            w4[0] = pack_bf16x2(t0v.x * e0.x, t0v.y * e0.y); w4[1] = pack_bf16x2(t0v.z * e0.z, t0v.w * e0.w);
+            w4[2] = pack_bf16x2(t1v.x * e1.x, t1v.y * e1.y); w4[3] = pack_bf16x2(t1v.z * e1.z, t1v.w * e1.w);
+            b4[0] = pack_bf16x2(t0v.x * c0.x, t0v.y * c0.y); b4[1] = pack_bf16x2(t0v.z * c0.z, t0v.w * c0.w);
+            b4[2] = pack_bf16x2(t1v.x * c1.x, t1v.y * c1.y); b4[3] = pack_bf16x2(t1v.z * c1.z, t1v.w * c1.w);
+        }
+        st_shared_v4(sb + OFF_TW + sw128_off(i, ch), w4[0], w4[1], w4[2], w4[3]);
+        st_shared_v4(sb + OFF_TB + sw128_off(i, ch), b4[0], b4[1], b4[2], b4[3]);
     }
     fence_async_smem();
     __syncthreads();
 
-    // ---- W^T = K^T Tw^T, u^T = V^T Tb^T ------------------------------------------------
+    // ---- W^T = K^T Tw^T, u^T = V^T Tb^T once V is in ------------------------------------
     if (tid == 0) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64, 1, 0);    // A MN-major, B K-major
+        ok = ctl.wait(B_FULL, 1);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, 64, 1, 0);    // A MN-major, B K-major
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_K + kk * 2048, 16384, 1024),
-                     sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), idesc, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_KV + kk * 2048, 16384, 1024),
+                         sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), idesc, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_V + kk * 2048, 8192, 1024),
-                     sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), idesc, kk > 0);
-        mma_commit(ctl.bar(B_MMA));
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_KV + 8192 + kk * 2048, 16384, 1024),
+                         sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), idesc, kk > 0);
+            mma_commit(ctl.bar(B_MMA));
+        }
     }
-    ok = ctl.wait(B_MMA, 1);
+    ok = ok && ctl.wait(B_MMA, 1);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    // ---- TMEM -> bf16 rows of the workspace: warps 0-3 W^T, 4-7 u^T ------------------
-    {
-        const int q = warp & 3;
-        const int r = (q << 5) + lane;
-        const bool is_u = warp >= 4;
-        __nv_bfloat16* out = (is_u ? u_out : w_out) + (tile * kD + r) * kC;
+    // ---- TMEM -> bf16 tiles over K and V (read by now), then TMA stores.  Warps 0-3:
+    //      -W, row-major [64 rows][128] as two [64][128 B] column blocks (lane r is
+    //      column r: element stores); warps 4-7: u^T [128][128 B] (lane r is row r) ------
+    if (warp < 4) {
+        const int r = (warp << 5) + lane;              // d_k channel
+        const uint32_t base = sb + OFF_KV + (uint32_t)(r >> 6) * 8192 + (uint32_t)(r & 7) * 2;
+        const int ch = (r & 63) >> 3;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float v[32];
-            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + (is_u ? TM_U : TM_W) + hh * 32, v);
+            tmem_ld32(tmem + ((uint32_t)(warp << 5) << 16) + TM_W + hh * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = hh * 32 + e;
+                st_shared_b16(base + (uint32_t)(i * 128 + ((ch ^ (i & 7)) << 4)), __float2bfloat16_rn(-v[e]));
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = (q << 5) + lane;
+        const uint32_t dst = sb + OFF_KV + 16384;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_U + hh * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
-                st_global_v4(out + hh * 32 + q4 * 8, pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
+                st_shared_v4(dst + sw128_off(r, hh * 4 + q4), pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
                              pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]), pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
                              pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
         }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_2d(&tm_w, 0, (int)(tile * kC), sb + OFF_KV);
+        tma_store_2d(&tm_w, 64, (int)(tile * kC), sb + OFF_KV + 8192);
+        tma_store_2d(&tm_u, 0, (int)(tile * kD), sb + OFF_KV + 16384);
+        bulk_commit_group();
+        bulk_wait_read_all();        // the writes complete before the next kernel on the stream starts
     }
 
 done:
@@ -346,7 +425,8 @@ done:
     __syncthreads();
     if (*abort_flag && tid == 0) {
         // let the loads land before the shared memory is released
-        if (load) mbar_wait_bounded(ctl.bar(B_FULL), 0, kWaitNs);
+        if (loads > 0) mbar_wait_bounded(ctl.bar(B_FULL), (uint32_t)(loads - 1), kWaitNs);
+        bulk_wait_all();
         atomicOr(status, 1u);
     }
     if (warp == 1) {
@@ -360,23 +440,20 @@ done:
 namespace {
 
 template <int GATE>
-cudaError_t launch_wy_gate(const ChunkArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                           __nv_bfloat16* w_ws, __nv_bfloat16* u_ws, int n, cudaStream_t st) {
+cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStream_t st) {
     auto kern = chunk_wy_kernel<GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(tk, tv, a.beta, a.g, w_ws, u_ws, (int)a.T, n,
-                                                              a.status, a.test_flags);
+    kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(m.q, m.k, m.v, m.w, m.u, m.p, m.qh, a.beta, a.g,
+                                                              (int)a.T, n, a.scale, a.status, a.test_flags);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_wy(const ChunkArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                            __nv_bfloat16* w_ws, __nv_bfloat16* u_ws, cudaStream_t st) {
+cudaError_t launch_chunk_wy(const ChunkArgs& a, const TcMaps& m, cudaStream_t st) {
     const int n = (int)((a.T + kC - 1) / kC);
-    return a.gate == kGateScalar ? launch_wy_gate<kGateScalar>(a, tk, tv, w_ws, u_ws, n, st)
-                                 : launch_wy_gate<kGateNone>(a, tk, tv, w_ws, u_ws, n, st);
+    return a.gate == kGateScalar ? launch_wy_gate<kGateScalar>(a, m, n, st) : launch_wy_gate<kGateNone>(a, m, n, st);
 }
 
 }  // namespace dn
