@@ -1,11 +1,11 @@
 // chunk_tc.cu -- the sequential state pass of the chunked delta rule on the
-// sm_100a tensor cores, fed by the per-chunk -W, u, P and Qh of chunk_wy.cu.
+// sm_100a tensor cores, fed by the per-chunk -W, u and P of chunk_wy.cu.
 //
 // Same mathematics as the chunkwise form of "Linear attention and Gated
 // DeltaNet" (ch. 28, "The chunked form: recurrence as matrix multiplication";
 // D2L 12.5, "Training it: the WY trick"): with W = T diag(beta e^G) K,
-// u = T diag(beta) V, P = scale tril(Q K^T * D) and Qh = scale e^G Q of each
-// chunk computed,
+// u = T diag(beta) V and P = scale tril(Q K^T * D) of each chunk computed, and
+// Qh = scale e^G Q,
 //
 //   U   = u - W S                                (values actually written)
 //   O   = Qh S + P U
@@ -27,9 +27,10 @@
 // drains while the next one runs.  The U and state epilogues run in two
 // halves with a barrier each, so that the tensor pipe starts on the first half
 // of a contraction while the second is converted.  Warp roles: 0 TMA + gates,
-// 2 TMEM allocation, 3 MMA issue, 4-7 output rows, 8-15 U and the state (two
-// warps per TMEM lane quarter).  Stages of k, Qh, -W, u^T and P tiles arrive
-// by TMA (128-byte swizzle) three chunks ahead.
+// 2 TMEM allocation, 3 MMA issue, 4-7 Qh (in place over the q tile) and the
+// output rows, 8-15 U and the state (two warps per TMEM lane quarter).  Stages
+// of k, q, -W, u^T and P tiles arrive by TMA (128-byte swizzle) three chunks
+// ahead.
 //
 // A partial last chunk has beta = 0, g = 0 past its end (rows past the
 // tensor's end are zero-filled by TMA; rows of the next head are masked),
@@ -46,7 +47,7 @@ using namespace tc;
 namespace {
 
 constexpr int kNT = 512;          // 16 warps
-constexpr int kSideWarp0 = 4;     // output warps 4..7
+constexpr int kSideWarp0 = 4;     // Qh / output warps 4..7
 constexpr int kSideThreads = 128;
 constexpr int kChainWarp0 = 8;    // state warps 8..15
 constexpr int kChainThreads = 256;
@@ -65,7 +66,7 @@ constexpr uint32_t TM_COLS = 512;
 constexpr int kStages = 3;
 constexpr uint32_t SZ_STAGE = 73728;    // one chunk's tiles:
 constexpr uint32_t ST_K = 0;            //   K [d-block][64 rows][128 B]                        16 KiB
-constexpr uint32_t ST_B = 16384;        //   [d-block][Qh rows 0-63 | -W rows 64-127][128 B]    32 KiB
+constexpr uint32_t ST_B = 16384;        //   [d-block][q -> Qh rows 0-63 | -W rows 64-127][128 B] 32 KiB
 constexpr uint32_t ST_UT = 49152;       //   u^T [128 rows (dv)][128 B (C)]                      16 KiB
 constexpr uint32_t ST_P = 65536;        //   P [64 rows (i)][128 B (j)]                           8 KiB
 constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
@@ -79,7 +80,7 @@ enum {
     B_FULL0 = 0, B_FREE0 = 3,                            // TMA stages (3 each)
     B_GATE0 = 6,                                         // gate slots (4)
     B_WS = 10, B_KU, B_PU0, B_PU1,                       // MMA completions
-    B_OFREE0, B_OFREE1,                                  // output warps -> MMA
+    B_READY0, B_READY1, B_READY2, B_OFREE0, B_OFREE1,    // Qh / output warps -> MMA (Qh per stage)
     B_UTA, B_UTB, B_STA, B_STB,                          // state warps -> MMA (first / second half)
     B_COUNT
 };
@@ -89,11 +90,11 @@ static_assert(OFF_BAR + 8 * B_COUNT + 16 <= OFF_BAR + 256, "barrier area");
 
 template <int GATE>
 __global__ void __launch_bounds__(kNT, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_qh,
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
                 const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ beta,
                 const float* __restrict__ g, const float* S0, __nv_bfloat16* __restrict__ o, float* S_T, int T,
-                unsigned int* status, int test_flags) {
+                float scale, unsigned int* status, int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
@@ -110,7 +111,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads : i >= B_OFREE0 ? kSideThreads : 1);
+            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads : i >= B_READY0 ? kSideThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -127,7 +128,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ================= producer: gates + TMA ================================
         if (lane == 0) {
             prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_qh);
+            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_w);
             prefetch_tmap(&tm_u);
             prefetch_tmap(&tm_p);
@@ -166,8 +167,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 mbar_arrive_expect_tx(fb, STAGE_TX);
                 tma_load_2d(st + ST_K + 0, &tm_k, 0, y, fb);
                 tma_load_2d(st + ST_K + 8192, &tm_k, 64, y, fb);
-                tma_load_2d(st + ST_B + 0, &tm_qh, 0, (int)(tile * kC), fb);
-                tma_load_2d(st + ST_B + 16384, &tm_qh, 64, (int)(tile * kC), fb);
+                tma_load_2d(st + ST_B + 0, &tm_q, 0, y, fb);
+                tma_load_2d(st + ST_B + 16384, &tm_q, 64, y, fb);
                 tma_load_2d(st + ST_B + 8192, &tm_w, 0, (int)(tile * kC), fb);
                 tma_load_2d(st + ST_B + 24576, &tm_w, 64, (int)(tile * kC), fb);
                 tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
@@ -196,6 +197,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 // chunk c - 2 is out, the first half of d_k as soon as the state's first half
                 // is written, then the second
                 ok = ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u) &&
+                     ctl.wait(B_READY0 + s, (uint32_t)(c / kStages) & 1u) &&
                      (c < 2 || ctl.wait(B_OFREE0 + (c & 1), (uint32_t)((c - 2) >> 1) & 1u)) && ctl.wait(B_STA, par);
                 if (!ok) break;
                 tc_fence_after();
@@ -239,30 +241,61 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (!ok) *abort_flag = 1;
         }
     } else if (warp >= kSideWarp0 && warp < kChainWarp0) {
-        // ================= output rows (128 threads) =================================
+        // ================= Qh of each chunk, output rows of the previous one (128 threads)
+        const int sid = tid - kSideWarp0 * 32;     // 0..127
         const int q = warp & 3;                    // TMEM lane quarter
         const int j = (q << 5) + lane;             // value channel = TMEM lane
-        for (int c = 0; c < n; ++c) {
-            const int Cc = min(kC, T - c * kC);
-            bool ok = ctl.wait(B_PU0 + (c & 1), (uint32_t)(c >> 1) & 1u);
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(1, kSideThreads, !ok)) break;
-            tc_fence_after();
-            __nv_bfloat16* ob = o + (bh * T + (int64_t)c * kC) * kD + j;
-            const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (c & 1) * 128;
+        for (int c = 0; c <= n; ++c) {
+            if (c < n) {
+                // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
+                const int s = c % kStages;
+                const int Cc = min(kC, T - c * kC);
+                const float* gs = gates + (c & 3) * GATE_FLOATS;
+                const uint32_t st = sb + s * SZ_STAGE;
+                bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) &&
+                          ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
+                if (!ok) *abort_flag = 1;
+                if (named_bar_any(1, kSideThreads, !ok)) break;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[32];
-                tmem_ld32(oc + hh * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = hh * 32 + e;
-                    if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                for (int u = 0; u < 8; ++u) {
+                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
+                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                    const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
+                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                    const uint4 w = ld_shared_v4(a);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                 }
+                fence_async_smem();
+                mbar_arrive(ctl.bar(B_READY0 + s));
             }
-            tc_fence_before();
-            mbar_arrive(ctl.bar(B_OFREE0 + (c & 1)));
+            if (c >= 1) {
+                // ---- output rows of chunk c - 1 --------------------------------------------
+                const int cp = c - 1;
+                const int Cc = min(kC, T - cp * kC);
+                bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
+                if (!ok) *abort_flag = 1;
+                if (named_bar_any(1, kSideThreads, !ok)) break;
+                tc_fence_after();
+                __nv_bfloat16* ob = o + (bh * T + (int64_t)cp * kC) * kD + j;
+                const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp & 1) * 128;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tmem_ld32(oc + hh * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = hh * 32 + e;
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
+            }
         }
     } else if (warp >= kChainWarp0) {
         // ================= U and the state (256 threads) ===========================
@@ -388,25 +421,23 @@ template <int GATE>
 cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     const uint64_t rows = (uint64_t)(a.B * a.H * a.T);
     const uint64_t tiles = (uint64_t)(a.B * a.H * ((a.T + kC - 1) / kC));
-    uint8_t* ws = static_cast<uint8_t*>(a.ws);
-    const uint8_t* w_ws = ws;
-    const uint8_t* u_ws = w_ws + tiles * kWsWBytes;
-    const uint8_t* p_ws = u_ws + tiles * kWsUBytes;
-    const uint8_t* q_ws = p_ws + tiles * kWsPBytes;
+    uint8_t* w_ws = static_cast<uint8_t*>(a.ws);
+    uint8_t* u_ws = w_ws + tiles * kWsWBytes;
+    uint8_t* p_ws = u_ws + tiles * kWsUBytes;
     TcMaps m;
     if (!make_tmap(&m.q, a.q, kD, rows, 64) || !make_tmap(&m.k, a.k, kD, rows, 64) ||
         !make_tmap(&m.v, a.v, kD, rows, 64) || !make_tmap(&m.w, w_ws, kD, tiles * kC, 64) ||
-        !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64) ||
-        !make_tmap(&m.qh, q_ws, kD, tiles * kC, 64))
+        !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64))
         return cudaErrorInvalidValue;
+    m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
     cudaError_t e = launch_chunk_wy(a, m, st);
     if (e != cudaSuccess) return e;
     auto kern = chunk_tc_kernel<GATE>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(a.B * a.H), kNT, SMEM_BYTES, st>>>(m.k, m.qh, m.w, m.u, m.p, a.beta, a.g, a.S0,
+    kern<<<(unsigned)(a.B * a.H), kNT, SMEM_BYTES, st>>>(m.k, m.q, m.w, m.u, m.p, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
-                                                          a.status, a.test_flags);
+                                                          a.scale, a.status, a.test_flags);
     return cudaGetLastError();
 }
 

@@ -21,23 +21,22 @@ constexpr int kD = 128;                     // d_k = d_v
 constexpr uint64_t kWaitNs = 1000000000ull; // every mbarrier wait gives up after 1 s
 
 // Workspace per (b, h, chunk), written by chunk_wy.cu and read by chunk_tc.cu,
-// four bf16 arrays one after another:
+// three bf16 arrays one after another:
 //   -W   [tiles * 64 rows (position)][128 (d_k)]
 //   u^T  [tiles * 128 rows (d_v)][64 (position)]
 //   P    [tiles * 64 rows (i)][64 (j)]
-//   Qh   [tiles * 64 rows (position)][128 (d_k)]
 constexpr size_t kWsWBytes = (size_t)kC * kD * 2;
 constexpr size_t kWsUBytes = (size_t)kD * kC * 2;
 constexpr size_t kWsPBytes = (size_t)kC * kC * 2;
-constexpr size_t kWsQBytes = (size_t)kC * kD * 2;
-constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes + kWsQBytes;
+constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes;
 
 // Tensor maps of the tensor-core path (128-byte swizzle, 64-column boxes):
-// q, k, v as [B H T][128] with 64-row boxes; the workspace's -W and Qh as
-// [tiles 64][128] with 64-row boxes, u^T as [tiles 128][64] with 128-row
-// boxes, P as [tiles 64][64] with 64-row boxes.
+// q, k, v as [B H T][128] with 64-row boxes; the workspace's -W as [tiles 64][128]
+// with 64-row boxes, u^T as [tiles 128][64] with 128-row boxes, P as
+// [tiles 64][64] with 64-row boxes.
 struct TcMaps {
-    CUtensorMap q, k, v, w, u, p, qh;
+    CUtensorMap q, k, v, w, u, p;
+    __nv_bfloat16* p_ws;     // the workspace's P array (written with plain stores)
 };
 
 // Gate slot of one chunk (floats).

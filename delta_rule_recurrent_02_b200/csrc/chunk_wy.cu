@@ -10,21 +10,21 @@
 //   A = strict_tril(beta_i k_i.k_j D_ij),   T = (I + A)^-1   (unit lower)
 //   W = T diag(beta e^G) K,                 u = T diag(beta) V
 //   P = scale tril(q_i.k_j D_ij)            (the intra-chunk attention)
-//   Qh = scale e^G Q                        (the queries seen from the chunk start)
 //
-// Every chunk is an independent CTA (three fit on an SM).  The state pass
+// Every chunk is an independent CTA (four fit on an SM).  The state pass
 // (chunk_tc.cu) streams the results back with TMA from the workspace, as bf16
 // tiles: -W [64 rows][128] (row-major, negated so that S^T (-W)^T = -(W S)^T),
-// u^T [128][64], P [64][64] and Qh [64][128].  One CTA:
+// u^T [128][64] and P [64][64].  One CTA:
 //
 //   TMA       K and Q tiles, stacked per 64-column block as [K rows | Q rows]
 //   tcgen05   [K;Q] K^T -> TMEM (bf16 -> fp32): K K^T for A, Q K^T for P
-//   CUDA core masks and decay -> A (fp32, shared memory) and P (bf16); Qh in place
-//   TMA       P and Qh out, then V over the Q rows, while the rest runs
-//   CUDA core T = (I + A)^-1: the 16 x 16 diagonal blocks D_k = (I + A_kk)^-1
-//             by forward substitution, M_kl = D_k A_kl, then
-//             T_kl = -sum_{m=l}^{k-1} M_km T_ml in three rounds (fp32);
+//   CUDA core masks and decay -> A (fp32, shared memory); P (bf16) straight to
+//             the workspace
+//   CUDA core T = (I + A)^-1 over the tiles' space: the 16 x 16 diagonal blocks
+//             D_k = (I + A_kk)^-1 by forward substitution, M_kl = D_k A_kl,
+//             then T_kl = -sum_{m=l}^{k-1} M_km T_ml in three rounds (fp32);
 //             then T diag(beta e^G) and T diag(beta) as bf16 operand tiles
+//   TMA       K and V again (from L2) over T
 //   tcgen05   W^T = K^T (T diag(beta e^G))^T, u^T = V^T (T diag(beta))^T -> TMEM
 //   epilogue  TMEM -> bf16 tiles in shared memory -> TMA stores to the workspace
 //
@@ -52,13 +52,14 @@ constexpr uint32_t TM_U = 64;   // u^T fp32 [dv][C]
 constexpr uint32_t TM_COLS = 128;
 
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KV = 0;          // [d-block][K rows 0-63 | Q (Qh) rows, then V rows][128 B] = 32 KiB;
-                                        // last, the -W and u^T output tiles
+constexpr uint32_t OFF_KV = 0;          // [d-block][K rows 0-63 | Q rows][128 B] = 32 KiB for the gram;
+                                        // T during the solve; [d-block][K | V] for W and u; last,
+                                        // the -W and u^T output tiles
+constexpr uint32_t OFF_T = 0;           // fp32 64 x 68: T = (I + A)^-1
 constexpr uint32_t OFF_A = 32768;       // fp32 64 x 68: A, then M = D^-1 A; then the bf16 tiles
 constexpr uint32_t OFF_TW = OFF_A;      //   T diag(beta e^G), K-major B [N=i][K=j]: [64 rows][128 B]
 constexpr uint32_t OFF_TB = OFF_A + 8192;   // T diag(beta), same layout
-constexpr uint32_t OFF_T = 50176;       // fp32 64 x 68: T = (I + A)^-1; first the P output tile
-constexpr uint32_t OFF_GATE = 67584;    // one gate slot
+constexpr uint32_t OFF_GATE = 50176;    // one gate slot
 constexpr uint32_t OFF_BAR = OFF_GATE + GATE_FLOATS * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 enum { B_FULL = 0, B_MMA = 1 };
@@ -102,16 +103,6 @@ __device__ __forceinline__ void blk16_store_neg(float* Tm, int zr, int zc, const
     *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0 + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
 }
 
-// Scale 8 bf16 values (one 16-byte chunk) by f and store them at dst.
-__device__ __forceinline__ void scale_chunk(uint32_t src, uint32_t dst, float f) {
-    const uint4 w = ld_shared_v4(src);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-    st_shared_v4(dst, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
-}
-
 __device__ __forceinline__ void zero8(float (&a)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = 0.f;
@@ -120,11 +111,11 @@ __device__ __forceinline__ void zero8(float (&a)[8]) {
 }  // namespace
 
 template <int GATE>
-__global__ void __launch_bounds__(kNT, 3)
+__global__ void __launch_bounds__(kNT, 4)
 chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
-                const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_p,
-                const __grid_constant__ CUtensorMap tm_qh, const float* __restrict__ beta,
+                const __grid_constant__ CUtensorMap tm_u, __nv_bfloat16* __restrict__ p_out,
+                const float* __restrict__ beta,
                 const float* __restrict__ g, int T, int n, float scale,
                 unsigned int* status, int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -211,7 +202,12 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int i = ((q & 1) << 5) + lane;
         const int j0 = (warp >> 2) << 5;
         const float g2i = gs[G_G2 + i];
-        if (q < 2) {
+        if (q == 0 && j0 == 32) {
+            // A rows 0-31 x columns 32-63 lie above the diagonal
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+                *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if (q < 2) {
             float v[32];
             tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
             tmem_wait_ld();
@@ -228,58 +224,36 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
             }
-        } else if (q == 2 && j0 == 32) {
-            // rows 0-31 x columns 32-63 lie above the diagonal
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) st_shared_v4(sb + OFF_T + sw128_off(i, 4 + q4), 0u, 0u, 0u, 0u);
         } else {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
-            tmem_wait_ld();
-            const float si = i < Cc ? scale : 0.f;
+            // P row i, columns j0 .. j0 + 31 -> workspace (row-major [64][64])
+            __nv_bfloat16* prow = p_out + (tile * kC + i) * kC + j0;
+            if (q == 2 && j0 == 32) {
+                // rows 0-31 x columns 32-63 lie above the diagonal
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
-                const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
-                const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                float pv[8];
+                for (int q4 = 0; q4 < 4; ++q4) st_global_v4(prow + 8 * q4, 0u, 0u, 0u, 0u);
+            } else {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
+                tmem_wait_ld();
+                const float si = i < Cc ? scale : 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = j0 + 8 * q4 + e;
-                    pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
+                    const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
+                    const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    float pv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = j0 + 8 * q4 + e;
+                        pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                    }
+                    st_global_v4(prow + 8 * q4, pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
+                                 pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
                 }
-                st_shared_v4(sb + OFF_T + sw128_off(i, (j0 >> 3) + q4), pack_bf16x2(pv[0], pv[1]),
-                             pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
             }
         }
-        // Qh = scale e^G Q in place over the Q rows (the gram has read them)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int x = tid + u * kNT;                   // 0..1023: (d-block, row, 16-byte chunk)
-            const int blk = x >> 9, r = (x >> 3) & 63, ch = x & 7;
-            const uint32_t a = sb + OFF_KV + blk * 16384 + 8192 + sw128_off(r, ch);
-            scale_chunk(a, a, r < Cc ? scale * gs[G_EG + r] : 0.f);
-        }
     }
-    fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        // P and Qh out; then V over the Q rows, and T's buffer is reused, once the copies have read them
-        const int y = (int)(tile * kC);
-        tma_store_2d(&tm_p, 0, y, sb + OFF_T);
-        tma_store_2d(&tm_qh, 0, y, sb + OFF_KV + 8192);
-        tma_store_2d(&tm_qh, 64, y, sb + OFF_KV + 24576);
-        bulk_commit_group();
-        bulk_wait_read_all();
-        if (load) {
-            const uint32_t fb = ctl.bar(B_FULL);
-            mbar_arrive_expect_tx(fb, 2 * 8192);
-            tma_load_2d(sb + OFF_KV + 8192, &tm_v, 0, (int)t0, fb);
-            tma_load_2d(sb + OFF_KV + 24576, &tm_v, 64, (int)t0, fb);
-            loads = 2;
-        }
-    }
     __syncthreads();
 
     // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
@@ -313,22 +287,31 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         blk16_store(Am, 16 * k, 16 * l, acc, lane);
     }
     __syncthreads();
-    // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds ------------------------------
+    // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds; one block product per warp
+    //      and round, (k, m, l) from the tables below (4 bits each) ----------------------
     {
+        // round 1, warps 0-5: T_10, T_21, T_32 complete; T_20, T_31, T_30 start (m = l)
+        // round 2, warps 3-5: T_20, T_31 complete (m = l + 1); T_30 continues (m = 1)
+        // round 3, warp 5:    T_30 completes (m = 2)
         float acc[8];
         zero8(acc);
-        if (warp == 0) { blk16(Am, 16, 0, Tm, 0, 0, acc, lane); blk16_store_neg(Tm, 16, 0, acc, lane); }
-        if (warp == 1) { blk16(Am, 32, 16, Tm, 16, 16, acc, lane); blk16_store_neg(Tm, 32, 16, acc, lane); }
-        if (warp == 2) { blk16(Am, 48, 32, Tm, 32, 32, acc, lane); blk16_store_neg(Tm, 48, 32, acc, lane); }
-        if (warp == 3) blk16(Am, 32, 0, Tm, 0, 0, acc, lane);
-        if (warp == 4) blk16(Am, 48, 16, Tm, 16, 16, acc, lane);
-        if (warp == 5) blk16(Am, 48, 0, Tm, 0, 0, acc, lane);
+        if (warp < 6) {
+            const int k = (0x332321 >> (4 * warp)) & 15, l = (0x010210 >> (4 * warp)) & 15;
+            blk16(Am, 16 * k, 16 * l, Tm, 16 * l, 16 * l, acc, lane);
+            if (warp < 3) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
         __syncthreads();
-        if (warp == 3) { blk16(Am, 32, 16, Tm, 16, 0, acc, lane); blk16_store_neg(Tm, 32, 0, acc, lane); }
-        if (warp == 4) { blk16(Am, 48, 32, Tm, 32, 16, acc, lane); blk16_store_neg(Tm, 48, 16, acc, lane); }
-        if (warp == 5) blk16(Am, 48, 16, Tm, 16, 0, acc, lane);
+        if (warp >= 3 && warp < 6) {
+            const int k = (0x332 >> (4 * (warp - 3))) & 15, m = (0x121 >> (4 * (warp - 3))) & 15;
+            const int l = (0x010 >> (4 * (warp - 3))) & 15;
+            blk16(Am, 16 * k, 16 * m, Tm, 16 * m, 16 * l, acc, lane);
+            if (warp < 5) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
         __syncthreads();
-        if (warp == 5) { blk16(Am, 48, 32, Tm, 32, 0, acc, lane); blk16_store_neg(Tm, 48, 0, acc, lane); }
+        if (warp == 5) {
+            blk16(Am, 48, 32, Tm, 32, 0, acc, lane);
+            blk16_store_neg(Tm, 48, 0, acc, lane);
+        }
     }
     __syncthreads();
     // ---- T diag(beta e^G) and T diag(beta) as bf16 operand tiles, over A (zero above
@@ -356,8 +339,17 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     fence_async_smem();
     __syncthreads();
 
-    // ---- W^T = K^T Tw^T, u^T = V^T Tb^T once V is in ------------------------------------
+    // ---- K and V (L2-resident by now) over T, then W^T = K^T Tw^T, u^T = V^T Tb^T -------
     if (tid == 0) {
+        if (load) {
+            const uint32_t fb = ctl.bar(B_FULL);
+            mbar_arrive_expect_tx(fb, 4 * 8192);
+            tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 8192, &tm_v, 0, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 24576, &tm_v, 64, (int)t0, fb);
+            loads = 2;
+        }
         ok = ctl.wait(B_FULL, 1);
         if (ok) {
             tc_fence_after();
@@ -444,7 +436,7 @@ cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStrea
     auto kern = chunk_wy_kernel<GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(m.q, m.k, m.v, m.w, m.u, m.p, m.qh, a.beta, a.g,
+    kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(m.q, m.k, m.v, m.w, m.u, m.p_ws, a.beta, a.g,
                                                               (int)a.T, n, a.scale, a.status, a.test_flags);
     return cudaGetLastError();
 }

@@ -118,11 +118,11 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
 /*
  * dn_chunk_fwd_workspace_size -- bytes of device workspace that dn_chunk_fwd_ex
  * uses for this request on `path` (0 when the chosen kernels need none).  The
- * tensor-core path computes W = T diag(beta e^G) K, u = T diag(beta) V, the
- * intra-chunk attention P and the decayed queries of every chunk ("Training it:
- * the WY trick", D2L 12.5; "The chunked form", ch. 28) in a kernel that runs
- * over all chunks at once, then streams them into the sequential state pass:
- * 56 KiB per (b, h, chunk), i.e. B * H * ceil(T / 64) * 57344 bytes.  Sizes are checked
+ * tensor-core path computes W = T diag(beta e^G) K, u = T diag(beta) V and the
+ * intra-chunk attention P of every chunk ("Training it: the WY trick", D2L
+ * 12.5; "The chunked form", ch. 28) in a kernel that runs over all chunks at
+ * once, then streams them into the sequential state pass: 40 KiB per
+ * (b, h, chunk), i.e. B * H * ceil(T / 64) * 40960 bytes.  Sizes are checked
  * as in dn_chunk_fwd_ex; *bytes is written on DN_OK only.
  */
 DN_API int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk,
@@ -170,7 +170,7 @@ DN_API int dn_chunk_fwd_ex(const void* q, const void* k, const void* v,
  *     threads) race on it: order them on one stream, or use dn_chunk_fwd_ex
  *     with separate workspaces.
  */
-#define DN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)   /* 64 MiB: 1170 (b, h, chunk) tiles */
+#define DN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)   /* 64 MiB: 1638 (b, h, chunk) tiles */
 
 DN_API int dn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                 const float* beta, const float* g, const float* S0,

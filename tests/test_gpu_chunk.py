@@ -144,7 +144,7 @@ def test_chunk_overwrites_poisoned_outputs(cuda_device, path):
 
 
 def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
-    # the tensor-core path keeps -W, u^T, P and Qh of every chunk in a workspace: a
+    # the tensor-core path keeps -W, u^T and P of every chunk in a workspace: a
     # caller's buffer (poisoned with NaN first: it is scratch, nothing is read
     # before it is written) and the library's own stream-ordered allocation
     # give bit-identical results, which match the oracle
@@ -152,7 +152,7 @@ def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
     d = to_dev(inp)
     sc = 128 ** -0.5
     nbytes = dn.dn_chunk_fwd_workspace_size(2, 200, 3, 128, 128, path="tc")
-    assert nbytes == 2 * 3 * 4 * 57344
+    assert nbytes == 2 * 3 * 4 * 40960
     ws = torch.full((nbytes // 2,), float("nan"), dtype=torch.bfloat16, device="cuda")
     outs = []
     for w in (ws, None):
