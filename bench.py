@@ -70,18 +70,26 @@ def load_peaks():
                 "source": "fallback"}
 
 
+def sources_sha256(paths):
+    """sha256 over the concatenated contents of the given repo-relative files."""
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_for(kernel_key):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    has not changed since it was captured (else None)."""
+    """DRAM bytes per launch (per call, for a path of several kernels) from a
+    committed ncu summary, if none of the sources has changed since it was
+    captured (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             tab = json.load(f)
         ent = tab[kernel_key]
-        src = os.path.join(ROOT, ent["source"])
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != ent["source_sha256"]:
-                return None
+        if sources_sha256(ent["sources"]) != ent["sources_sha256"]:
+            return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:
         return None
