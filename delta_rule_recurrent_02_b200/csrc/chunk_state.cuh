@@ -1,0 +1,449 @@
+// chunk_state.cuh -- the sequential state pass of the chunked delta rule on the
+// sm_100a tensor cores, fed by the per-chunk -W, u and P of chunk_wy.cu.
+//
+// Same mathematics as the chunkwise form of "Linear attention and Gated
+// DeltaNet" (ch. 28, "The chunked form: recurrence as matrix multiplication";
+// D2L 12.5, "Training it: the WY trick"): with W = T diag(beta e^G) K,
+// u = T diag(beta) V and P = scale tril(Q K^T * D) of each chunk computed, and
+// Qh = scale e^G Q,
+//
+//   U   = u - W S                                (values actually written)
+//   O   = Qh S + P U
+//   S  <- e^(G_last) S + (K * e^(G_last - G))^T U
+//
+// Every product runs as tcgen05.mma with M = 128 in transposed form (d_v is
+// the MMA's M).  A tcgen05.mma costs the tensor pipe about the same time for
+// any N up to 128, so the two products of the state share one MMA of N = 128:
+//
+//   [O^T | U^T] = S^T [Qh ; -W]^T   A = S^T (TMEM, bf16)  B = [Qh rows | -W rows] (smem)
+//   U^T        += u^T               (epilogue)
+//   S^T        += U~^T K            A = U~^T (TMEM, bf16) B = K tile (smem)
+//   O^T        += U^T P^T           A = U^T (TMEM, bf16)  B = P (smem)
+//
+// with U~ = U * e^(G_last - G) (the decay of K folded into U's rows).  The CTA
+// owns one (b, h); its state stays in TMEM (fp32 accumulator, pre-scaled by
+// the next chunk's decay, plus a bf16 copy that feeds the next products), and
+// [O | U] alternates between two TMEM buffers so that the output of one chunk
+// drains while the next one runs.  The U and state epilogues run in two
+// halves with a barrier each, so that the tensor pipe starts on the first half
+// of a contraction while the second is converted.  Warp roles: 0 TMA + gates,
+// 2 TMEM allocation, 3 MMA issue, 4-7 Qh (in place over the q tile) and the
+// output rows, 8-15 U and the state (two warps per TMEM lane quarter).  Stages
+// of k, q, -W, u^T and P tiles arrive by TMA (128-byte swizzle) three chunks
+// ahead.
+//
+// A partial last chunk has beta = 0, g = 0 past its end (rows past the
+// tensor's end are zero-filled by TMA; rows of the next head are masked),
+// which equals zero padding.  Every wait is bounded: on a timeout the kernel
+// records it in the status word, lets its own copies land and exits.
+#pragma once
+
+#include "chunk_tc_common.cuh"
+
+namespace dn {
+namespace state {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int kNT = 512;          // 16 warps
+constexpr int kSideWarp0 = 4;     // Qh / output warps 4..7
+constexpr int kSideThreads = 128;
+constexpr int kChainWarp0 = 8;    // state warps 8..15
+constexpr int kChainThreads = 256;
+static_assert(kSideThreads == (kChainWarp0 - kSideWarp0) * 32 && kChainThreads == kNT - kChainWarp0 * 32,
+              "named-barrier thread counts must match the warps of each role");
+// named barriers: 1 Qh / output warps, 2 state warps, kCtaBar all kNT threads
+constexpr uint32_t kCtaBar = 3;
+
+// TMEM columns (32-bit, 128 lanes)
+constexpr uint32_t TM_SACC = 0;     // S^T fp32 [dv lanes][dk cols], pre-scaled by the coming chunk's decay
+constexpr uint32_t TM_OU = 128;     // 2 x [O^T | U^T] fp32, [dv][C | C], by chunk parity
+constexpr uint32_t TM_ST = 384;     // S^T bf16 pairs [dv][dk/2]
+constexpr uint32_t TM_UT = 448;     // U^T bf16 pairs [dv][C/2]
+constexpr uint32_t TM_UK = 480;     // U~^T bf16 pairs [dv][C/2]
+constexpr uint32_t TM_COLS = 512;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr int kStages = 3;
+constexpr uint32_t SZ_STAGE = 73728;    // one chunk's tiles:
+constexpr uint32_t ST_K = 0;            //   K [d-block][64 rows][128 B]                        16 KiB
+constexpr uint32_t ST_B = 16384;        //   [d-block][q -> Qh rows 0-63 | -W rows 64-127][128 B] 32 KiB
+constexpr uint32_t ST_UT = 49152;       //   u^T [128 rows (dv)][128 B (C)]                      16 KiB
+constexpr uint32_t ST_P = 65536;        //   P [64 rows (i)][128 B (j)]                           8 KiB
+constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
+constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
+constexpr uint32_t STATE_BYTES = OFF_BAR + 256;   // from a 1024-aligned base
+constexpr uint32_t STAGE_TX = SZ_STAGE;
+
+// barrier indices; where a waiter could otherwise see a barrier two phases on,
+// there is one per chunk parity
+enum {
+    B_FULL0 = 0, B_FREE0 = 3,                            // TMA stages (3 each)
+    B_GATE0 = 6,                                         // gate slots (4)
+    B_WS = 10, B_KU, B_PU0, B_PU1,                       // MMA completions
+    B_READY0, B_READY1, B_READY2, B_OFREE0, B_OFREE1,    // Qh / output warps -> MMA (Qh per stage)
+    B_UTA, B_UTB, B_STA, B_STB,                          // state warps -> MMA (first / second half)
+    B_COUNT
+};
+static_assert(OFF_BAR + 8 * B_COUNT + 16 <= OFF_BAR + 256, "barrier area");
+
+struct Args {
+    const CUtensorMap* tm_k;
+    const CUtensorMap* tm_q;
+    const CUtensorMap* tm_w;
+    const CUtensorMap* tm_u;
+    const CUtensorMap* tm_p;
+    const unsigned int* flags;
+    const float* beta;
+    const float* g;
+    const float* S0;
+    __nv_bfloat16* o;
+    float* S_T;
+    int T;
+    float scale;
+    unsigned int* status;
+    int test_flags;
+};
+
+// The state pass of head `head`, run by threads 0 .. kNT - 1 of a CTA whose
+// shared memory starts (1024-aligned) at sm.
+template <int GATE>
+__device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head) {
+    const CUtensorMap& tm_k = *ar.tm_k;
+    const CUtensorMap& tm_q = *ar.tm_q;
+    const CUtensorMap& tm_w = *ar.tm_w;
+    const CUtensorMap& tm_u = *ar.tm_u;
+    const CUtensorMap& tm_p = *ar.tm_p;
+    const unsigned int* __restrict__ flags = ar.flags;
+    const float* __restrict__ beta = ar.beta;
+    const float* __restrict__ g = ar.g;
+    const float* S0 = ar.S0;
+    __nv_bfloat16* __restrict__ o = ar.o;
+    float* S_T = ar.S_T;
+    const int T = ar.T;
+    const float scale = ar.scale;
+    unsigned int* status = ar.status;
+    const int test_flags = ar.test_flags;
+    const uint32_t sb = smem_u32(sm);
+    float* gates = reinterpret_cast<float*>(sm + OFF_GATE);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 8 * B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + 8 * B_COUNT + 8);
+    Ctl ctl{sb + OFF_BAR, abort_flag};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t bh = head;
+    const int n = (T + kC - 1) / kC;
+
+    if (tid == 0) {
+        for (int i = 0; i < B_COUNT; ++i)
+            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads : i >= B_READY0 ? kSideThreads : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_slot), TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    named_bar_sync(kCtaBar, kNT);
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= producer: gates + TMA ================================
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_w);
+            prefetch_tmap(&tm_u);
+            prefetch_tmap(&tm_p);
+        }
+        int issued = 0;
+        // beta / g of the next chunk, loaded one chunk ahead
+        float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
+        auto fetch = [&](int cc) {
+            const int64_t t0 = bh * T + (int64_t)cc * kC;
+            const int Cn = min(kC, T - cc * kC);
+            nb0 = lane < Cn ? beta[t0 + lane] : 0.f;
+            nb1 = lane + 32 < Cn ? beta[t0 + lane + 32] : 0.f;
+            if (GATE == kGateScalar) {
+                ng0 = lane < Cn ? g[t0 + lane] : 0.f;
+                ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
+            }
+        };
+        fetch(0);
+        for (int cc = 0; cc < n; ++cc) {
+            const int s = cc % kStages;
+            const float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
+            if (cc + 1 < n) fetch(cc + 1);
+            chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            // the stage is free once the products of chunk cc - 3 are done
+            if (cc >= kStages) {
+                bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - kStages) / kStages) & 1u) : true;
+                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+            }
+            if (!(test_flags & 1)) {
+                // this chunk's workspace tiles are written (by another CTA, possibly right now)
+                bool ok = lane == 0 ? wait_flag(flags + bh * n + cc, abort_flag) : true;
+                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
+            }
+            if (lane == 0 && !(test_flags & 1)) {
+                fence_async_global();
+                const int y = (int)(bh * T + (int64_t)cc * kC);
+                const int64_t tile = bh * n + cc;
+                const uint32_t st = sb + s * SZ_STAGE;
+                const uint32_t fb = ctl.bar(B_FULL0 + s);
+                mbar_arrive_expect_tx(fb, STAGE_TX);
+                tma_load_2d(st + ST_K + 0, &tm_k, 0, y, fb);
+                tma_load_2d(st + ST_K + 8192, &tm_k, 64, y, fb);
+                tma_load_2d(st + ST_B + 0, &tm_q, 0, y, fb);
+                tma_load_2d(st + ST_B + 16384, &tm_q, 64, y, fb);
+                tma_load_2d(st + ST_B + 8192, &tm_w, 0, (int)(tile * kC), fb);
+                tma_load_2d(st + ST_B + 24576, &tm_w, 64, (int)(tile * kC), fb);
+                tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
+                tma_load_2d(st + ST_P, &tm_p, 0, (int)(tile * kC), fb);
+            }
+            if (!(test_flags & 1)) issued = cc + 1;
+        }
+        if (*abort_flag && lane == 0) {
+            // let every load this CTA issued land before its shared memory is released
+            for (int cc = max(0, issued - kStages); cc < issued; ++cc)
+                mbar_wait_bounded(ctl.bar(B_FULL0 + cc % kStages), (uint32_t)(cc / kStages) & 1u, kWaitNs);
+        }
+    } else if (warp == 3) {
+        // ================= MMA issue (one thread) ====================================
+        if (lane == 0) {
+            const uint32_t I_SW = idesc_bf16(128, 128, 0, 0);       // [O|U] = S^T [Qh;-W]^T
+            const uint32_t I_KU = idesc_bf16(128, 128, 0, 1);       // B MN-major
+            const uint32_t I_PU = idesc_bf16(128, 64, 0, 0);
+            bool ok = true;
+            for (int c = 0; ok && c < n; ++c) {
+                const uint32_t par = (uint32_t)c & 1u;
+                const int s = c % kStages;
+                const uint32_t st = sb + s * SZ_STAGE;
+                const uint32_t ou = tmem + TM_OU + (c & 1) * 128;
+                // [O|U]^T = S^T [Qh;-W]^T: once the tiles are in and this buffer's output of
+                // chunk c - 2 is out, the first half of d_k as soon as the state's first half
+                // is written, then the second
+                ok = ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u) &&
+                     ctl.wait(B_READY0 + s, (uint32_t)(c / kStages) & 1u) &&
+                     (c < 2 || ctl.wait(B_OFREE0 + (c & 1), (uint32_t)((c - 2) >> 1) & 1u)) && ctl.wait(B_STA, par);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
+                                sw128_desc(st + ST_B + (kk & 3) * 32, 16, 1024), I_SW, kk > 0);
+                ok = ctl.wait(B_STB, par);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
+                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
+                                sw128_desc(st + ST_B + 16384 + (kk & 3) * 32, 16, 1024), I_SW, 1);
+                mma_commit(ctl.bar(B_WS));
+                // S^T += U~^T K and O^T += U^T P^T, positions 0-31 then 32-63
+                ok = ctl.wait(B_UTA, par);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk)
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
+                                I_KU, 1);
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk)
+                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
+                ok = ctl.wait(B_UTB, par);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 2; kk < 4; ++kk)
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
+                                I_KU, 1);
+                mma_commit(ctl.bar(B_KU));
+#pragma unroll
+                for (int kk = 2; kk < 4; ++kk)
+                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
+                mma_commit(ctl.bar(B_PU0 + (c & 1)));
+                mma_commit(ctl.bar(B_FREE0 + s));        // the stage's last reader is done
+            }
+            if (!ok) *abort_flag = 1;
+        }
+    } else if (warp >= kSideWarp0 && warp < kChainWarp0) {
+        // ================= Qh of each chunk, output rows of the previous one (128 threads)
+        const int sid = tid - kSideWarp0 * 32;     // 0..127
+        const int q = warp & 3;                    // TMEM lane quarter
+        const int j = (q << 5) + lane;             // value channel = TMEM lane
+        for (int c = 0; c <= n; ++c) {
+            if (c < n) {
+                // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
+                const int s = c % kStages;
+                const int Cc = min(kC, T - c * kC);
+                const float* gs = gates + (c & 3) * GATE_FLOATS;
+                const uint32_t st = sb + s * SZ_STAGE;
+                bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) &&
+                          ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
+                if (!ok) *abort_flag = 1;
+                if (named_bar_any(1, kSideThreads, !ok)) break;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
+                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                    const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
+                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                    const uint4 w = ld_shared_v4(a);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                }
+                fence_async_smem();
+                mbar_arrive(ctl.bar(B_READY0 + s));
+            }
+            if (c >= 1) {
+                // ---- output rows of chunk c - 1 --------------------------------------------
+                const int cp = c - 1;
+                const int Cc = min(kC, T - cp * kC);
+                bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
+                if (!ok) *abort_flag = 1;
+                if (named_bar_any(1, kSideThreads, !ok)) break;
+                tc_fence_after();
+                __nv_bfloat16* ob = o + (bh * T + (int64_t)cp * kC) * kD + j;
+                const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp & 1) * 128;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tmem_ld32(oc + hh * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = hh * 32 + e;
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
+            }
+        }
+    } else if (warp >= kChainWarp0) {
+        // ================= U and the state (256 threads) ===========================
+        const int q = warp & 3;
+        const int hc = (warp - kChainWarp0) >> 2;    // which half of each pass
+        const int j = (q << 5) + lane;               // value channel = TMEM lane
+        const uint32_t lane_off = (uint32_t)(q << 5) << 16;
+        bool ok = ctl.wait(B_GATE0, 0);
+        if (!ok) *abort_flag = 1;
+        ok = !named_bar_any(2, kChainThreads, !ok);
+        if (ok) {
+            // S0 -> TMEM: fp32 pre-scaled by chunk 0's decay, and its bf16 copy
+            const float gamma0 = gates[G_GAMMA];
+#pragma unroll 1
+            for (int p = 0; p < 2; ++p) {
+                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = S0 ? S0[(bh * kD + pc * 32 + e) * kD + j] : 0.f;
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= gamma0;
+                tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
+            }
+        }
+        for (int c = 0; ok && c < n; ++c) {
+            const uint32_t par = (uint32_t)c & 1u;
+            const uint32_t st = sb + (c % kStages) * SZ_STAGE;
+            // ---- U = u - W S -> bf16 pairs in TMEM, plain and decayed (U~), in two passes
+            //      over positions 0-31 and 32-63 ------------------------------------------
+            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            tc_fence_after();
+            const float* gsc = gates + (c & 3) * GATE_FLOATS;
+#pragma unroll 1
+            for (int p = 0; p < 2; ++p) {
+                const int i0 = 32 * p + 16 * hc;         // positions i0 .. i0 + 15
+                float v[16];
+                tmem_ld16(tmem + lane_off + TM_OU + (c & 1) * 128 + 64 + i0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const uint4 w = ld_shared_v4(st + ST_UT + sw128_off(j, (i0 >> 3) + ch));
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        v[8 * ch + 2 * e] += f.x;
+                        v[8 * ch + 2 * e + 1] += f.y;
+                    }
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st8(tmem + lane_off + TM_UT + (i0 >> 1), pk);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
+                    pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
+                    pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
+                }
+                tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
+            }
+            // ---- state: S_{c+1} = gamma_c S_c + dS (already summed in TMEM), in two passes
+            //      over d_k 0-63 and 64-127 ---------------------------------------------------
+            ok = ctl.wait(B_KU, par) && (c + 1 >= n || ctl.wait(B_GATE0 + ((c + 1) & 3), (uint32_t)((c + 1) >> 2) & 1u));
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            tc_fence_after();
+            const bool last = c + 1 == n;
+            const float gnext = last ? 1.f : gates[((c + 1) & 3) * GATE_FLOATS + G_GAMMA];
+#pragma unroll 1
+            for (int p = 0; p < 2; ++p) {
+                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
+                float v[32];
+                tmem_ld32(tmem + lane_off + TM_SACC + pc * 32, v);
+                tmem_wait_ld();
+                if (last) {
+                    if (S_T) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) S_T[(bh * kD + pc * 32 + e) * kD + j] = v[e];
+                    }
+                } else {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                    tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= gnext;
+                    tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
+            }
+        }
+        if (!ok) *abort_flag = 1;
+    }
+
+    named_bar_sync(kCtaBar, kNT);
+    if (*abort_flag && tid == 0) atomicOr(status, 1u);
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+}  // namespace state
+}  // namespace dn

@@ -1,42 +1,18 @@
-// chunk_tc.cu -- the sequential state pass of the chunked delta rule on the
-// sm_100a tensor cores, fed by the per-chunk -W, u and P of chunk_wy.cu.
+// chunk_tc.cu -- the tensor-core prefill: the per-chunk WY transform
+// (chunk_wy.cuh) and the sequential state pass (chunk_state.cuh).
 //
-// Same mathematics as the chunkwise form of "Linear attention and Gated
-// DeltaNet" (ch. 28, "The chunked form: recurrence as matrix multiplication";
-// D2L 12.5, "Training it: the WY trick"): with W = T diag(beta e^G) K,
-// u = T diag(beta) V and P = scale tril(Q K^T * D) of each chunk computed, and
-// Qh = scale e^G Q,
-//
-//   U   = u - W S                                (values actually written)
-//   O   = Qh S + P U
-//   S  <- e^(G_last) S + (K * e^(G_last - G))^T U
-//
-// Every product runs as tcgen05.mma with M = 128 in transposed form (d_v is
-// the MMA's M).  A tcgen05.mma costs the tensor pipe about the same time for
-// any N up to 128, so the two products of the state share one MMA of N = 128:
-//
-//   [O^T | U^T] = S^T [Qh ; -W]^T   A = S^T (TMEM, bf16)  B = [Qh rows | -W rows] (smem)
-//   U^T        += u^T               (epilogue)
-//   S^T        += U~^T K            A = U~^T (TMEM, bf16) B = K tile (smem)
-//   O^T        += U^T P^T           A = U^T (TMEM, bf16)  B = P (smem)
-//
-// with U~ = U * e^(G_last - G) (the decay of K folded into U's rows).  The CTA
-// owns one (b, h); its state stays in TMEM (fp32 accumulator, pre-scaled by
-// the next chunk's decay, plus a bf16 copy that feeds the next products), and
-// [O | U] alternates between two TMEM buffers so that the output of one chunk
-// drains while the next one runs.  The U and state epilogues run in two
-// halves with a barrier each, so that the tensor pipe starts on the first half
-// of a contraction while the second is converted.  Warp roles: 0 TMA + gates,
-// 2 TMEM allocation, 3 MMA issue, 4-7 Qh (in place over the q tile) and the
-// output rows, 8-15 U and the state (two warps per TMEM lane quarter).  Stages
-// of k, q, -W, u^T and P tiles arrive by TMA (128-byte swizzle) three chunks
-// ahead.
-//
-// A partial last chunk has beta = 0, g = 0 past its end (rows past the
-// tensor's end are zero-filled by TMA; rows of the next head are masked),
-// which equals zero padding.  Every wait is bounded: on a timeout the kernel
-// records it in the status word, lets its own copies land and exits.
-#include "chunk_tc_common.cuh"
+// Two ways to run them, both with a ready flag per workspace tile:
+//   * one cooperative launch (chunk_fused_kernel), one CTA per SM: CTAs
+//     0 .. B H - 1 run the state pass of one head each, the others run four
+//     groups of 8 warps that take the WY tiles chunk by chunk (chunk 0 of every
+//     head first).  A cooperative launch guarantees that every CTA is resident,
+//     so the state pass may wait for tiles that other CTAs are writing; the WY
+//     work overlaps the latency-bound state pass and its tiles are read while
+//     still in L2.  Used while B H leaves a quarter of the SMs to the WY groups.
+//   * otherwise two launches on the stream: chunk_wy_kernel over all tiles,
+//     then chunk_state_kernel (whose flags are then all set).
+#include "chunk_state.cuh"
+#include "chunk_wy.cuh"
 #include "dn_kernels.h"
 
 namespace dn {
@@ -44,372 +20,78 @@ namespace dn {
 using namespace sm100;
 using namespace tc;
 
-namespace {
-
-constexpr int kNT = 512;          // 16 warps
-constexpr int kSideWarp0 = 4;     // Qh / output warps 4..7
-constexpr int kSideThreads = 128;
-constexpr int kChainWarp0 = 8;    // state warps 8..15
-constexpr int kChainThreads = 256;
-static_assert(kSideThreads == (kChainWarp0 - kSideWarp0) * 32 && kChainThreads == kNT - kChainWarp0 * 32,
-              "named-barrier thread counts must match the warps of each role");
-
-// TMEM columns (32-bit, 128 lanes)
-constexpr uint32_t TM_SACC = 0;     // S^T fp32 [dv lanes][dk cols], pre-scaled by the coming chunk's decay
-constexpr uint32_t TM_OU = 128;     // 2 x [O^T | U^T] fp32, [dv][C | C], by chunk parity
-constexpr uint32_t TM_ST = 384;     // S^T bf16 pairs [dv][dk/2]
-constexpr uint32_t TM_UT = 448;     // U^T bf16 pairs [dv][C/2]
-constexpr uint32_t TM_UK = 480;     // U~^T bf16 pairs [dv][C/2]
-constexpr uint32_t TM_COLS = 512;
-
-// shared memory (bytes from a 1024-aligned base)
-constexpr int kStages = 3;
-constexpr uint32_t SZ_STAGE = 73728;    // one chunk's tiles:
-constexpr uint32_t ST_K = 0;            //   K [d-block][64 rows][128 B]                        16 KiB
-constexpr uint32_t ST_B = 16384;        //   [d-block][q -> Qh rows 0-63 | -W rows 64-127][128 B] 32 KiB
-constexpr uint32_t ST_UT = 49152;       //   u^T [128 rows (dv)][128 B (C)]                      16 KiB
-constexpr uint32_t ST_P = 65536;        //   P [64 rows (i)][128 B (j)]                           8 KiB
-constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
-constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t STAGE_TX = SZ_STAGE;
-
-// barrier indices; where a waiter could otherwise see a barrier two phases on,
-// there is one per chunk parity
-enum {
-    B_FULL0 = 0, B_FREE0 = 3,                            // TMA stages (3 each)
-    B_GATE0 = 6,                                         // gate slots (4)
-    B_WS = 10, B_KU, B_PU0, B_PU1,                       // MMA completions
-    B_READY0, B_READY1, B_READY2, B_OFREE0, B_OFREE1,    // Qh / output warps -> MMA (Qh per stage)
-    B_UTA, B_UTB, B_STA, B_STB,                          // state warps -> MMA (first / second half)
-    B_COUNT
-};
-static_assert(OFF_BAR + 8 * B_COUNT + 16 <= OFF_BAR + 256, "barrier area");
-
-}  // namespace
-
 template <int GATE>
-__global__ void __launch_bounds__(kNT, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
-                const __grid_constant__ CUtensorMap tm_p, const float* __restrict__ beta,
-                const float* __restrict__ g, const float* S0, __nv_bfloat16* __restrict__ o, float* S_T, int T,
-                float scale, unsigned int* status, int test_flags) {
+__global__ void __launch_bounds__(state::kNT, 1)
+chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_p, const unsigned int* __restrict__ flags,
+                   const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
+                   __nv_bfloat16* __restrict__ o, float* S_T, int T, float scale, unsigned int* status,
+                   int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const uint32_t sb = smem_u32(sm);
-    float* gates = reinterpret_cast<float*>(sm + OFF_GATE);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 8 * B_COUNT);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + 8 * B_COUNT + 8);
-    Ctl ctl{sb + OFF_BAR, abort_flag};
+    const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags};
+    state::state_pass<GATE>(sm, ar, blockIdx.x);
+}
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t bh = blockIdx.x;
-    const int n = (T + kC - 1) / kC;
+namespace {
+constexpr int kFusedThreads = 4 * wy::kNT;          // 32 warps: 4 WY groups, or the state pass + 16 idle warps
+static_assert(state::kNT <= kFusedThreads, "fused CTA size");
+constexpr uint32_t kFusedBytes = (state::STATE_BYTES > 4 * wy::GROUP_BYTES ? state::STATE_BYTES : 4 * wy::GROUP_BYTES) + 1024;
+}  // namespace
 
-    if (tid == 0) {
-        for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads : i >= B_READY0 ? kSideThreads : 1);
-        *abort_flag = 0;
+template <int GATE>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_p,
+                   __nv_bfloat16* __restrict__ p_out, unsigned int* __restrict__ flags, int BH,
+                   const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
+                   __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale, unsigned int* status,
+                   int test_flags) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if ((int)blockIdx.x < BH) {
+        // ---- state pass of head blockIdx.x (warps 0-15) --------------------------------
+        if (warp >= state::kNT / 32) return;
+        const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
+                             test_flags};
+        state::state_pass<GATE>(sm, ar, blockIdx.x);
+        return;
+    }
+    // ---- four WY groups, each taking every G-th tile in chunk-major order -----------------
+    const int grp = warp >> 3;                       // 0..3
+    const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(sm + 4 * wy::GROUP_BYTES - 16);
+    wy::Group x = wy::make_group(sm + grp * wy::GROUP_BYTES, 0u, 1u + (uint32_t)grp, tid - grp * wy::kNT);
+    if (x.tid == 0) {
+        wy::init_group(x);
         fence_mbar_init();
     }
-    if (warp == 2) {
-        tmem_alloc(smem_u32(tmem_slot), TM_COLS);
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), 4 * wy::TM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ================= producer: gates + TMA ================================
-        if (lane == 0) {
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_w);
-            prefetch_tmap(&tm_u);
-            prefetch_tmap(&tm_p);
-        }
-        int issued = 0;
-        // beta / g of the next chunk, loaded one chunk ahead
-        float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
-        auto fetch = [&](int cc) {
-            const int64_t t0 = bh * T + (int64_t)cc * kC;
-            const int Cn = min(kC, T - cc * kC);
-            nb0 = lane < Cn ? beta[t0 + lane] : 0.f;
-            nb1 = lane + 32 < Cn ? beta[t0 + lane + 32] : 0.f;
-            if (GATE == kGateScalar) {
-                ng0 = lane < Cn ? g[t0 + lane] : 0.f;
-                ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
-            }
-        };
-        fetch(0);
-        for (int cc = 0; cc < n; ++cc) {
-            const int s = cc % kStages;
-            const float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
-            if (cc + 1 < n) fetch(cc + 1);
-            chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
-            // the stage is free once the products of chunk cc - 3 are done
-            if (cc >= kStages) {
-                bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - kStages) / kStages) & 1u) : true;
-                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
-            }
-            if (lane == 0 && !(test_flags & 1)) {
-                const int y = (int)(bh * T + (int64_t)cc * kC);
-                const int64_t tile = bh * n + cc;
-                const uint32_t st = sb + s * SZ_STAGE;
-                const uint32_t fb = ctl.bar(B_FULL0 + s);
-                mbar_arrive_expect_tx(fb, STAGE_TX);
-                tma_load_2d(st + ST_K + 0, &tm_k, 0, y, fb);
-                tma_load_2d(st + ST_K + 8192, &tm_k, 64, y, fb);
-                tma_load_2d(st + ST_B + 0, &tm_q, 0, y, fb);
-                tma_load_2d(st + ST_B + 16384, &tm_q, 64, y, fb);
-                tma_load_2d(st + ST_B + 8192, &tm_w, 0, (int)(tile * kC), fb);
-                tma_load_2d(st + ST_B + 24576, &tm_w, 64, (int)(tile * kC), fb);
-                tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
-                tma_load_2d(st + ST_P, &tm_p, 0, (int)(tile * kC), fb);
-            }
-            if (!(test_flags & 1)) issued = cc + 1;
-        }
-        if (*abort_flag && lane == 0) {
-            // let every load this CTA issued land before its shared memory is released
-            for (int cc = max(0, issued - kStages); cc < issued; ++cc)
-                mbar_wait_bounded(ctl.bar(B_FULL0 + cc % kStages), (uint32_t)(cc / kStages) & 1u, kWaitNs);
-        }
-    } else if (warp == 3) {
-        // ================= MMA issue (one thread) ====================================
-        if (lane == 0) {
-            const uint32_t I_SW = idesc_bf16(128, 128, 0, 0);       // [O|U] = S^T [Qh;-W]^T
-            const uint32_t I_KU = idesc_bf16(128, 128, 0, 1);       // B MN-major
-            const uint32_t I_PU = idesc_bf16(128, 64, 0, 0);
-            bool ok = true;
-            for (int c = 0; ok && c < n; ++c) {
-                const uint32_t par = (uint32_t)c & 1u;
-                const int s = c % kStages;
-                const uint32_t st = sb + s * SZ_STAGE;
-                const uint32_t ou = tmem + TM_OU + (c & 1) * 128;
-                // [O|U]^T = S^T [Qh;-W]^T: once the tiles are in and this buffer's output of
-                // chunk c - 2 is out, the first half of d_k as soon as the state's first half
-                // is written, then the second
-                ok = ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u) &&
-                     ctl.wait(B_READY0 + s, (uint32_t)(c / kStages) & 1u) &&
-                     (c < 2 || ctl.wait(B_OFREE0 + (c & 1), (uint32_t)((c - 2) >> 1) & 1u)) && ctl.wait(B_STA, par);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
-                                sw128_desc(st + ST_B + (kk & 3) * 32, 16, 1024), I_SW, kk > 0);
-                ok = ctl.wait(B_STB, par);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 4; kk < 8; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
-                                sw128_desc(st + ST_B + 16384 + (kk & 3) * 32, 16, 1024), I_SW, 1);
-                mma_commit(ctl.bar(B_WS));
-                // S^T += U~^T K and O^T += U^T P^T, positions 0-31 then 32-63
-                ok = ctl.wait(B_UTA, par);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
-                                I_KU, 1);
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
-                ok = ctl.wait(B_UTB, par);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 2; kk < 4; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
-                                I_KU, 1);
-                mma_commit(ctl.bar(B_KU));
-#pragma unroll
-                for (int kk = 2; kk < 4; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
-                mma_commit(ctl.bar(B_PU0 + (c & 1)));
-                mma_commit(ctl.bar(B_FREE0 + s));        // the stage's last reader is done
-            }
-            if (!ok) *abort_flag = 1;
-        }
-    } else if (warp >= kSideWarp0 && warp < kChainWarp0) {
-        // ================= Qh of each chunk, output rows of the previous one (128 threads)
-        const int sid = tid - kSideWarp0 * 32;     // 0..127
-        const int q = warp & 3;                    // TMEM lane quarter
-        const int j = (q << 5) + lane;             // value channel = TMEM lane
-        for (int c = 0; c <= n; ++c) {
-            if (c < n) {
-                // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
-                const int s = c % kStages;
-                const int Cc = min(kC, T - c * kC);
-                const float* gs = gates + (c & 3) * GATE_FLOATS;
-                const uint32_t st = sb + s * SZ_STAGE;
-                bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) &&
-                          ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
-                if (!ok) *abort_flag = 1;
-                if (named_bar_any(1, kSideThreads, !ok)) break;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
-                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
-                    const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
-                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
-                    const uint4 w = ld_shared_v4(a);
-                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
-                }
-                fence_async_smem();
-                mbar_arrive(ctl.bar(B_READY0 + s));
-            }
-            if (c >= 1) {
-                // ---- output rows of chunk c - 1 --------------------------------------------
-                const int cp = c - 1;
-                const int Cc = min(kC, T - cp * kC);
-                bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
-                if (!ok) *abort_flag = 1;
-                if (named_bar_any(1, kSideThreads, !ok)) break;
-                tc_fence_after();
-                __nv_bfloat16* ob = o + (bh * T + (int64_t)cp * kC) * kD + j;
-                const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp & 1) * 128;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    tmem_ld32(oc + hh * 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = hh * 32 + e;
-                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
-            }
-        }
-    } else if (warp >= kChainWarp0) {
-        // ================= U and the state (256 threads) ===========================
-        const int q = warp & 3;
-        const int hc = (warp - kChainWarp0) >> 2;    // which half of each pass
-        const int j = (q << 5) + lane;               // value channel = TMEM lane
-        const uint32_t lane_off = (uint32_t)(q << 5) << 16;
-        bool ok = ctl.wait(B_GATE0, 0);
-        if (!ok) *abort_flag = 1;
-        ok = !named_bar_any(2, kChainThreads, !ok);
-        if (ok) {
-            // S0 -> TMEM: fp32 pre-scaled by chunk 0's decay, and its bf16 copy
-            const float gamma0 = gates[G_GAMMA];
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
-                float v[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = S0 ? S0[(bh * kD + pc * 32 + e) * kD + j] : 0.f;
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= gamma0;
-                tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
-            }
-        }
-        for (int c = 0; ok && c < n; ++c) {
-            const uint32_t par = (uint32_t)c & 1u;
-            const uint32_t st = sb + (c % kStages) * SZ_STAGE;
-            // ---- U = u - W S -> bf16 pairs in TMEM, plain and decayed (U~), in two passes
-            //      over positions 0-31 and 32-63 ------------------------------------------
-            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
-            tc_fence_after();
-            const float* gsc = gates + (c & 3) * GATE_FLOATS;
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const int i0 = 32 * p + 16 * hc;         // positions i0 .. i0 + 15
-                float v[16];
-                tmem_ld16(tmem + lane_off + TM_OU + (c & 1) * 128 + 64 + i0, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    const uint4 w = ld_shared_v4(st + ST_UT + sw128_off(j, (i0 >> 3) + ch));
-                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(h2[e]);
-                        v[8 * ch + 2 * e] += f.x;
-                        v[8 * ch + 2 * e + 1] += f.y;
-                    }
-                }
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                tmem_st8(tmem + lane_off + TM_UT + (i0 >> 1), pk);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
-                    pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
-                    pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
-                }
-                tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
-            }
-            // ---- state: S_{c+1} = gamma_c S_c + dS (already summed in TMEM), in two passes
-            //      over d_k 0-63 and 64-127 ---------------------------------------------------
-            ok = ctl.wait(B_KU, par) && (c + 1 >= n || ctl.wait(B_GATE0 + ((c + 1) & 3), (uint32_t)((c + 1) >> 2) & 1u));
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
-            tc_fence_after();
-            const bool last = c + 1 == n;
-            const float gnext = last ? 1.f : gates[((c + 1) & 3) * GATE_FLOATS + G_GAMMA];
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
-                float v[32];
-                tmem_ld32(tmem + lane_off + TM_SACC + pc * 32, v);
-                tmem_wait_ld();
-                if (last) {
-                    if (S_T) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) S_T[(bh * kD + pc * 32 + e) * kD + j] = v[e];
-                    }
-                } else {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                    tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= gnext;
-                    tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
-            }
-        }
-        if (!ok) *abort_flag = 1;
+    x.tmem = *tmem_slot + (uint32_t)grp * wy::TM_COLS;
+    const wy::Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags};
+    const int64_t tiles = (int64_t)BH * n;
+    const int64_t G = (int64_t)(gridDim.x - BH) * 4;
+    bool ok = true;
+    for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles; t += G) {
+        const int c = (int)(t / BH);
+        ok = wy::wy_tile<GATE>(x, ar, c, t - (int64_t)c * BH);
     }
-
+    tc_fence_before();
     __syncthreads();
-    if (*abort_flag && tid == 0) atomicOr(status, 1u);
-    if (warp == 2) {
+    if (!ok && x.tid == 0) atomicOr(status, 1u);
+    if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, TM_COLS);
+        tmem_dealloc(*tmem_slot, 4 * wy::TM_COLS);
     }
 }
 
@@ -417,10 +99,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 namespace {
 
+// The single-launch prefill needs one resident CTA per SM and leaves at least
+// a quarter of them (and 16) to the WY groups.
+bool fused_fits(int64_t BH, int num_sms) {
+    return BH + 16 <= num_sms && BH * 4 <= (int64_t)num_sms * 3;
+}
+
 template <int GATE>
 cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     const uint64_t rows = (uint64_t)(a.B * a.H * a.T);
-    const uint64_t tiles = (uint64_t)(a.B * a.H * ((a.T + kC - 1) / kC));
+    const int n = (int)((a.T + kC - 1) / kC);
+    const uint64_t tiles = (uint64_t)(a.B * a.H) * (uint64_t)n;
     uint8_t* w_ws = static_cast<uint8_t*>(a.ws);
     uint8_t* u_ws = w_ws + tiles * kWsWBytes;
     uint8_t* p_ws = u_ws + tiles * kWsUBytes;
@@ -430,14 +119,50 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64))
         return cudaErrorInvalidValue;
     m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
-    cudaError_t e = launch_chunk_wy(a, m, st);
+    m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles));
+    cudaError_t e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
     if (e != cudaSuccess) return e;
-    auto kern = chunk_tc_kernel<GATE>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+
+    int dev = 0, num_sms = 0, coop = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(a.B * a.H), kNT, SMEM_BYTES, st>>>(m.k, m.q, m.w, m.u, m.p, a.beta, a.g, a.S0,
-                                                          static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
-                                                          a.scale, a.status, a.test_flags);
+    const int64_t BH = a.B * a.H;
+    if (coop && fused_fits(BH, num_sms)) {
+        auto kern = chunk_fused_kernel<GATE>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedBytes);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedThreads, kFusedBytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm >= 1) {
+            int bh_i = (int)BH, T_i = (int)a.T, n_i = n;
+            float scale = a.scale;
+            int test_flags = a.test_flags;
+            __nv_bfloat16* p_out = m.p_ws;
+            unsigned int* flags = m.flags;
+            const float* beta = a.beta;
+            const float* g = a.g;
+            const float* S0 = a.S0;
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+            float* S_T = a.S_T;
+            unsigned int* status = a.status;
+            void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
+                            &T_i, &n_i, &scale, &status, &test_flags};
+            return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
+                                               dim3(kFusedThreads), args, kFusedBytes, st);
+        }
+    }
+    e = launch_chunk_wy(a, m, st);
+    if (e != cudaSuccess) return e;
+    auto kern = chunk_state_kernel<GATE>;
+    const uint32_t bytes = state::STATE_BYTES + 1024;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, m.flags, a.beta, a.g, a.S0,
+                                                  static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
+                                                  a.status, a.test_flags);
     return cudaGetLastError();
 }
 
@@ -451,7 +176,7 @@ bool tc_supports(const ChunkArgs& a) {
 
 size_t tc_workspace_bytes(const ChunkArgs& a) {
     const int64_t n = (a.T + kC - 1) / kC;
-    return (size_t)(a.B * a.H * n) * kWsTileBytes;
+    return ws_total_bytes((uint64_t)(a.B * a.H * n));
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {

@@ -29,6 +29,10 @@ constexpr size_t kWsWBytes = (size_t)kC * kD * 2;
 constexpr size_t kWsUBytes = (size_t)kD * kC * 2;
 constexpr size_t kWsPBytes = (size_t)kC * kC * 2;
 constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes;
+// ...then one 32-bit ready flag per tile, set (release) once the tile is
+// written and awaited (acquire) before the state pass loads it.
+inline size_t ws_flags_offset(uint64_t tiles) { return (size_t)tiles * kWsTileBytes; }
+inline size_t ws_total_bytes(uint64_t tiles) { return ws_flags_offset(tiles) + ((tiles * 4 + 255) / 256) * 256; }
 
 // Tensor maps of the tensor-core path (128-byte swizzle, 64-column boxes):
 // q, k, v as [B H T][128] with 64-row boxes; the workspace's -W as [tiles 64][128]
@@ -37,6 +41,7 @@ constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes;
 struct TcMaps {
     CUtensorMap q, k, v, w, u, p;
     __nv_bfloat16* p_ws;     // the workspace's P array (written with plain stores)
+    unsigned int* flags;     // the workspace's ready flags, zeroed before each prefill
 };
 
 // Gate slot of one chunk (floats).
@@ -72,6 +77,21 @@ __device__ __forceinline__ void chunk_gates(float* gs, float b0, float b1, float
 // 2^x is accurate to about 2^-22 relative, far inside the bf16 rounding of
 // the tiles these factors enter.
 __device__ __forceinline__ float decay2(float g2i, float g2j) { return ex2_approx(g2i - g2j); }
+
+// Wait (bounded) for a ready flag set with release semantics by another CTA.
+__device__ __forceinline__ bool wait_flag(const unsigned int* f, volatile int* abort) {
+    if (ld_acquire_gpu(f)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(f)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
 
 // Bounded mbarrier waits for a CTA whose roles share an abort flag in shared memory.
 struct Ctl {

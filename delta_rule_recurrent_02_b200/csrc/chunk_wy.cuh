@@ -1,0 +1,464 @@
+// chunk_wy.cuh -- the state-independent part of one chunk of the chunked delta
+// rule (the "WY transform" of "Linear attention and Gated DeltaNet", ch. 28,
+// "The chunked form", and D2L 12.5, "Training it: the WY trick"), as a device
+// function run by a group of 8 warps: a whole CTA in chunk_wy.cu, or one of
+// four groups of a CTA in the single-launch prefill of chunk_tc.cu.
+//
+// Inside a chunk of C = 64 tokens, with G_i the inclusive cumulative
+// log-decay and D_ij = e^(G_i - G_j),
+//
+//   A = strict_tril(beta_i k_i.k_j D_ij),   T = (I + A)^-1   (unit lower)
+//   W = T diag(beta e^G) K,                 u = T diag(beta) V
+//   P = scale tril(q_i.k_j D_ij)            (the intra-chunk attention)
+//
+// written to the workspace as bf16 tiles: -W [64 rows][128] (row-major,
+// negated so that S^T (-W)^T = -(W S)^T), u^T [128][64] and P [64][64], then
+// the tile's ready flag (release).  Steps of one tile:
+//
+//   TMA       K and Q tiles, stacked per 64-column block as [K rows | Q rows]
+//   tcgen05   [K;Q] K^T -> TMEM (bf16 -> fp32): K K^T for A, Q K^T for P
+//   CUDA core masks and decay -> A (fp32, shared memory); P (bf16) straight to
+//             the workspace
+//   CUDA core T = (I + A)^-1 over the tiles' space: the 16 x 16 diagonal blocks
+//             D_k = (I + A_kk)^-1 by forward substitution, M_kl = D_k A_kl,
+//             then T_kl = -sum_{m=l}^{k-1} M_km T_ml in three rounds (fp32);
+//             then T diag(beta e^G) and T diag(beta) as bf16 operand tiles
+//   TMA       K and V again (from L2) over T
+//   tcgen05   W^T = K^T (T diag(beta e^G))^T, u^T = V^T (T diag(beta))^T -> TMEM
+//   epilogue  TMEM -> bf16 tiles in shared memory -> TMA stores to the workspace
+//
+// A partial last chunk has beta = 0 and g = 0 past its end: those rows of A
+// and P, and those columns of W^T and u^T, are zero (equal to zero padding).
+// Rows past the end of the tensor are zero-filled by TMA; rows of the next
+// head are multiplied by those zeros.  Every wait is bounded; on a timeout the
+// group stops.
+#pragma once
+
+#include "chunk_tc_common.cuh"
+
+namespace dn {
+namespace wy {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int kNT = 256;        // 8 warps per group
+
+// TMEM columns (32-bit, 128 lanes)
+constexpr uint32_t TM_G = 0;    // gram [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T
+constexpr uint32_t TM_W = 0;    // W^T fp32 [dk][C], after the gram has been read
+constexpr uint32_t TM_U = 64;   // u^T fp32 [dv][C]
+constexpr uint32_t TM_COLS = 128;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_KV = 0;          // [d-block][K rows 0-63 | Q rows][128 B] = 32 KiB for the gram;
+                                        // T during the solve; [d-block][K | V] for W and u; last,
+                                        // the -W and u^T output tiles
+constexpr uint32_t OFF_T = 0;           // fp32 64 x 68: T = (I + A)^-1
+constexpr uint32_t OFF_A = 32768;       // fp32 64 x 68: A, then M = D^-1 A; then the bf16 tiles
+constexpr uint32_t OFF_TW = OFF_A;      //   T diag(beta e^G), K-major B [N=i][K=j]: [64 rows][128 B]
+constexpr uint32_t OFF_TB = OFF_A + 8192;   // T diag(beta), same layout
+constexpr uint32_t OFF_GATE = 50176;    // one gate slot
+constexpr uint32_t OFF_BAR = OFF_GATE + GATE_FLOATS * 4;
+constexpr uint32_t GROUP_BYTES = 52224;  // one group's shared memory, a multiple of 1024
+static_assert(OFF_BAR + 64 <= GROUP_BYTES, "group layout");
+enum { B_FULL = 0, B_MMA = 1 };
+
+// fp32 64 x 64 matrix, rows padded to 68 floats: 16-byte aligned rows, and
+// rows r and r + 1 start 4 banks apart (conflict-free row, column and 16 x 16
+// block accesses)
+constexpr int kFS = 68;
+__device__ __forceinline__ int fidx(int i, int j) { return i * kFS + j; }
+
+// acc[e] += sum_m X[xr + ii][xc + m] * Y[yr + m][yc + j0 + e] over a 16 x 16
+// block pair; lane -> (ii = lane / 2, j0 = 8 (lane % 2)).
+__device__ __forceinline__ void blk16(const float* X, int xr, int xc, const float* Y, int yr, int yc,
+                                      float (&acc)[8], int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    float xrow[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(X + fidx(xr + ii, xc + 4 * q));
+        xrow[4 * q + 0] = v.x; xrow[4 * q + 1] = v.y; xrow[4 * q + 2] = v.z; xrow[4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const float4 a = *reinterpret_cast<const float4*>(Y + fidx(yr + m, yc + j0));
+        const float4 b = *reinterpret_cast<const float4*>(Y + fidx(yr + m, yc + j0 + 4));
+        acc[0] += xrow[m] * a.x; acc[1] += xrow[m] * a.y; acc[2] += xrow[m] * a.z; acc[3] += xrow[m] * a.w;
+        acc[4] += xrow[m] * b.x; acc[5] += xrow[m] * b.y; acc[6] += xrow[m] * b.z; acc[7] += xrow[m] * b.w;
+    }
+}
+
+__device__ __forceinline__ void blk16_store(float* Z, int zr, int zc, const float (&acc)[8], int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    *reinterpret_cast<float4*>(Z + fidx(zr + ii, zc + j0)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(Z + fidx(zr + ii, zc + j0 + 4)) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// T_zr,zc = -acc (fp32).
+__device__ __forceinline__ void blk16_store_neg(float* Tm, int zr, int zc, const float (&acc)[8], int lane) {
+    const int ii = lane >> 1, j0 = (lane & 1) * 8;
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    *reinterpret_cast<float4*>(Tm + fidx(zr + ii, zc + j0 + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+}
+
+__device__ __forceinline__ void zero8(float (&a)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[e] = 0.f;
+}
+
+
+// One group of kNT threads and its resources.  Each mbarrier completes two
+// phases per tile (parities 0 then 1), so a group can run tile after tile.
+struct Group {
+    uint8_t* sm;             // 1024-aligned shared memory of GROUP_BYTES
+    uint32_t sb;             // its shared-space address
+    uint32_t tmem;           // first of the group's TM_COLS TMEM columns
+    uint32_t bar;            // named barrier of the group's kNT threads
+    int tid, warp, lane;     // within the group
+    Ctl ctl;
+};
+
+__device__ __forceinline__ Group make_group(uint8_t* sm, uint32_t tmem, uint32_t bar, int tid) {
+    Group x;
+    x.sm = sm;
+    x.sb = smem_u32(sm);
+    x.tmem = tmem;
+    x.bar = bar;
+    x.tid = tid;
+    x.warp = tid >> 5;
+    x.lane = tid & 31;
+    x.ctl = Ctl{x.sb + OFF_BAR, reinterpret_cast<volatile int*>(sm + OFF_BAR + 20)};
+    return x;
+}
+
+// Barriers and the abort flag of a group (one thread, before the group's first tile).
+__device__ __forceinline__ void init_group(const Group& x) {
+    mbar_init(x.ctl.bar(B_FULL), 1);
+    mbar_init(x.ctl.bar(B_MMA), 1);
+    *x.ctl.abort = 0;
+}
+
+struct Args {
+    const CUtensorMap* tm_q;
+    const CUtensorMap* tm_k;
+    const CUtensorMap* tm_v;
+    const CUtensorMap* tm_w;
+    const CUtensorMap* tm_u;
+    __nv_bfloat16* p_out;
+    unsigned int* flags;
+    const float* beta;
+    const float* g;
+    int T, n;
+    float scale;
+    int test_flags;
+};
+
+// Chunk c of head bh.  Returns false (the group's abort flag set) if a wait gave up.
+template <int GATE>
+__device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh) {
+    const uint32_t sb = x.sb;
+    float* gs = reinterpret_cast<float*>(x.sm + OFF_GATE);
+    float* Am = reinterpret_cast<float*>(x.sm + OFF_A);
+    float* Tm = reinterpret_cast<float*>(x.sm + OFF_T);
+    const Ctl& ctl = x.ctl;
+    volatile int* abort_flag = ctl.abort;
+    const uint32_t tmem = x.tmem;
+    const int tid = x.tid, warp = x.warp, lane = x.lane;
+    const int T = ar.T, n = ar.n;
+    const float scale = ar.scale;
+    const float* __restrict__ beta = ar.beta;
+    const float* __restrict__ g = ar.g;
+    __nv_bfloat16* __restrict__ p_out = ar.p_out;
+    unsigned int* flags = ar.flags;
+    const CUtensorMap& tm_q = *ar.tm_q;
+    const CUtensorMap& tm_k = *ar.tm_k;
+    const CUtensorMap& tm_v = *ar.tm_v;
+    const CUtensorMap& tm_w = *ar.tm_w;
+    const CUtensorMap& tm_u = *ar.tm_u;
+    const int64_t tile = bh * n + c;
+    const int Cc = min(kC, T - c * kC);
+    const int64_t t0 = bh * T + (int64_t)c * kC;
+    const bool load = !(ar.test_flags & 1);
+    int loads = 0;                                   // load groups issued (thread 0)
+
+    if (tid == 0 && load) {
+        const uint32_t fb = ctl.bar(B_FULL);
+        const int y = (int)t0;
+        mbar_arrive_expect_tx(fb, 4 * 8192);
+        tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, y, fb);
+        tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, y, fb);
+        tma_load_2d(sb + OFF_KV + 8192, &tm_q, 0, y, fb);
+        tma_load_2d(sb + OFF_KV + 24576, &tm_q, 64, y, fb);
+        loads = 1;
+    }
+    if (warp == 2) {
+        const float b0 = lane < Cc ? beta[t0 + lane] : 0.f;
+        const float b1 = lane + 32 < Cc ? beta[t0 + lane + 32] : 0.f;
+        float a0 = 0.f, a1 = 0.f;
+        if (GATE == kGateScalar) {
+            a0 = lane < Cc ? g[t0 + lane] : 0.f;
+            a1 = lane + 32 < Cc ? g[t0 + lane + 32] : 0.f;
+        }
+        chunk_gates(gs, b0, b1, a0, a1, lane);
+    }
+    bool ok = true;
+    if (tid == 0) {
+        // [K;Q] K^T once the tiles have landed
+        ok = ctl.wait(B_FULL, 0);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a = sb + OFF_KV + (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16(tmem + TM_G, sw128_desc(a, 16, 1024), sw128_desc(a, 16, 1024), idesc, kk > 0);
+            }
+            mma_commit(ctl.bar(B_MMA));
+        }
+    }
+    named_bar_sync(x.bar, kNT);                       // gates visible
+    ok = ok && ctl.wait(B_MMA, 0);
+    if (named_bar_any(x.bar, kNT, !ok)) goto done;
+    tc_fence_after();
+
+    // ---- A = strict_tril(beta_i (K K^T)_ij D_ij) from TMEM lanes 0-63 (warps 0, 1, 4, 5)
+    //      and P = scale tril((Q K^T)_ij D_ij) from lanes 64-127 (warps 2, 3, 6, 7), 32
+    //      columns per thread --------------------------------------------------------------
+    {
+        const int q = warp & 3;
+        const int i = ((q & 1) << 5) + lane;
+        const int j0 = (warp >> 2) << 5;
+        const float g2i = gs[G_G2 + i];
+        if (q == 0 && j0 == 32) {
+            // A rows 0-31 x columns 32-63 lie above the diagonal
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+                *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if (q < 2) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
+            tmem_wait_ld();
+            const float bi = gs[G_BETA + i];          // zero past the chunk's end
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 gj = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 4 * q4);
+                const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+                float a[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j0 + 4 * q4 + e;
+                    a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                }
+                *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
+            }
+        } else {
+            // P row i, columns j0 .. j0 + 31 -> workspace (row-major [64][64])
+            __nv_bfloat16* prow = p_out + (tile * kC + i) * kC + j0;
+            if (q == 2 && j0 == 32) {
+                // rows 0-31 x columns 32-63 lie above the diagonal
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) st_global_v4(prow + 8 * q4, 0u, 0u, 0u, 0u);
+            } else {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
+                tmem_wait_ld();
+                const float si = i < Cc ? scale : 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
+                    const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
+                    const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    float pv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = j0 + 8 * q4 + e;
+                        pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                    }
+                    st_global_v4(prow + 8 * q4, pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
+                                 pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    named_bar_sync(x.bar, kNT);
+
+    // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
+    if (warp < 4 && lane < 16) {
+        const int k0 = warp * 16, jj = lane;
+        float x[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+            float p0 = (ii == jj) ? 1.f : 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+            for (int m = 0; m + 3 < ii; m += 4) {
+                const float4 av = *reinterpret_cast<const float4*>(Am + fidx(k0 + ii, k0 + m));
+                p0 -= av.x * x[m]; p1 -= av.y * x[m + 1]; p2 -= av.z * x[m + 2]; p3 -= av.w * x[m + 3];
+            }
+#pragma unroll
+            for (int m = ii & ~3; m < ii; ++m) p0 -= Am[fidx(k0 + ii, k0 + m)] * x[m];
+            x[ii] = (p0 + p1) + (p2 + p3);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
+    }
+    named_bar_sync(x.bar, kNT);
+    // ---- M_kl = D_k A_kl (k > l), in place of A_kl -------------------------------------
+    if (warp < 6) {
+        // (k, l) = (1,0) (2,0) (3,0) (2,1) (3,1) (3,2) for warps 0..5
+        const int k = (0x332321 >> (4 * warp)) & 15, l = (0x211000 >> (4 * warp)) & 15;
+        float acc[8];
+        zero8(acc);
+        blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
+        __syncwarp();
+        blk16_store(Am, 16 * k, 16 * l, acc, lane);
+    }
+    named_bar_sync(x.bar, kNT);
+    // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds; one block product per warp
+    //      and round, (k, m, l) from the tables below (4 bits each) ----------------------
+    {
+        // round 1, warps 0-5: T_10, T_21, T_32 complete; T_20, T_31, T_30 start (m = l)
+        // round 2, warps 3-5: T_20, T_31 complete (m = l + 1); T_30 continues (m = 1)
+        // round 3, warp 5:    T_30 completes (m = 2)
+        float acc[8];
+        zero8(acc);
+        if (warp < 6) {
+            const int k = (0x332321 >> (4 * warp)) & 15, l = (0x010210 >> (4 * warp)) & 15;
+            blk16(Am, 16 * k, 16 * l, Tm, 16 * l, 16 * l, acc, lane);
+            if (warp < 3) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
+        named_bar_sync(x.bar, kNT);
+        if (warp >= 3 && warp < 6) {
+            const int k = (0x332 >> (4 * (warp - 3))) & 15, m = (0x121 >> (4 * (warp - 3))) & 15;
+            const int l = (0x010 >> (4 * (warp - 3))) & 15;
+            blk16(Am, 16 * k, 16 * m, Tm, 16 * m, 16 * l, acc, lane);
+            if (warp < 5) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
+        named_bar_sync(x.bar, kNT);
+        if (warp == 5) {
+            blk16(Am, 48, 32, Tm, 32, 0, acc, lane);
+            blk16_store_neg(Tm, 48, 0, acc, lane);
+        }
+    }
+    named_bar_sync(x.bar, kNT);
+    // ---- T diag(beta e^G) and T diag(beta) as bf16 operand tiles, over A (zero above
+    //      the block diagonal, where T was never written) ----------------------------------
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int x = tid + u * kNT;                   // 0..511: (row, 8-column chunk)
+        const int i = x >> 3, ch = x & 7;
+        uint32_t w4[4] = {0u, 0u, 0u, 0u}, b4[4] = {0u, 0u, 0u, 0u};
+        if ((ch >> 1) <= (i >> 4)) {
+            const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
+            const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
+            const float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
+            const float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
+            const float4 c0 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch);
+            const float4 c1 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch + 4);
+            w4[0] = pack_bf16x2(t0v.x * e0.x, t0v.y * e0.y); w4[1] = pack_bf16x2(t0v.z * e0.z, t0v.w * e0.w);
+            w4[2] = pack_bf16x2(t1v.x * e1.x, t1v.y * e1.y); w4[3] = pack_bf16x2(t1v.z * e1.z, t1v.w * e1.w);
+            b4[0] = pack_bf16x2(t0v.x * c0.x, t0v.y * c0.y); b4[1] = pack_bf16x2(t0v.z * c0.z, t0v.w * c0.w);
+            b4[2] = pack_bf16x2(t1v.x * c1.x, t1v.y * c1.y); b4[3] = pack_bf16x2(t1v.z * c1.z, t1v.w * c1.w);
+        }
+        st_shared_v4(sb + OFF_TW + sw128_off(i, ch), w4[0], w4[1], w4[2], w4[3]);
+        st_shared_v4(sb + OFF_TB + sw128_off(i, ch), b4[0], b4[1], b4[2], b4[3]);
+    }
+    fence_async_smem();
+    named_bar_sync(x.bar, kNT);
+
+    // ---- K and V (L2-resident by now) over T, then W^T = K^T Tw^T, u^T = V^T Tb^T -------
+    if (tid == 0) {
+        if (load) {
+            const uint32_t fb = ctl.bar(B_FULL);
+            mbar_arrive_expect_tx(fb, 4 * 8192);
+            tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 8192, &tm_v, 0, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 24576, &tm_v, 64, (int)t0, fb);
+            loads = 2;
+        }
+        ok = ctl.wait(B_FULL, 1);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, 64, 1, 0);    // A MN-major, B K-major
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_KV + kk * 2048, 16384, 1024),
+                         sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), idesc, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_KV + 8192 + kk * 2048, 16384, 1024),
+                         sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), idesc, kk > 0);
+            mma_commit(ctl.bar(B_MMA));
+        }
+    }
+    ok = ok && ctl.wait(B_MMA, 1);
+    if (named_bar_any(x.bar, kNT, !ok)) goto done;
+    tc_fence_after();
+    // ---- TMEM -> bf16 tiles over K and V (read by now), then TMA stores.  Warps 0-3:
+    //      -W, row-major [64 rows][128] as two [64][128 B] column blocks (lane r is
+    //      column r: element stores); warps 4-7: u^T [128][128 B] (lane r is row r) ------
+    if (warp < 4) {
+        const int r = (warp << 5) + lane;              // d_k channel
+        const uint32_t base = sb + OFF_KV + (uint32_t)(r >> 6) * 8192 + (uint32_t)(r & 7) * 2;
+        const int ch = (r & 63) >> 3;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp << 5) << 16) + TM_W + hh * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = hh * 32 + e;
+                st_shared_b16(base + (uint32_t)(i * 128 + ((ch ^ (i & 7)) << 4)), __float2bfloat16_rn(-v[e]));
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = (q << 5) + lane;
+        const uint32_t dst = sb + OFF_KV + 16384;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_U + hh * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                st_shared_v4(dst + sw128_off(r, hh * 4 + q4), pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
+                             pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]), pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                             pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+        }
+    }
+    fence_async_smem();
+    named_bar_sync(x.bar, kNT);
+    if (tid == 0) {
+        tma_store_2d(&tm_w, 0, (int)(tile * kC), sb + OFF_KV);
+        tma_store_2d(&tm_w, 64, (int)(tile * kC), sb + OFF_KV + 8192);
+        tma_store_2d(&tm_u, 0, (int)(tile * kD), sb + OFF_KV + 16384);
+        bulk_commit_group();
+        // publish the tile: its stores complete, then its ready flag (release)
+        bulk_wait_all();
+        fence_async_global();
+        __threadfence();
+        st_release_gpu(flags + tile, 1u);
+    }
+    tc_fence_before();
+    named_bar_sync(x.bar, kNT);
+    return true;
+
+done:
+    tc_fence_before();
+    named_bar_sync(x.bar, kNT);
+    if (tid == 0) {
+        // let the loads land before the shared memory is reused or released
+        if (loads > 0) mbar_wait_bounded(ctl.bar(B_FULL), (uint32_t)(loads - 1), kWaitNs);
+        bulk_wait_all();
+    }
+    *abort_flag = 1;
+    return false;
+}
+
+}  // namespace wy
+}  // namespace dn

@@ -91,6 +91,21 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Orders this thread's global-memory accesses through the generic proxy with
+// those through the async proxy (TMA): after a bulk store completes, before
+// publishing it; after observing a publication, before a bulk load of it.
+__device__ __forceinline__ void fence_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void st_release_gpu(unsigned int* p, unsigned int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Writes by threads to shared memory, made visible to the async proxy
 // (tensor cores, TMA) before a barrier.
 __device__ __forceinline__ void fence_async_smem() {

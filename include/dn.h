@@ -121,8 +121,9 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
  * tensor-core path computes W = T diag(beta e^G) K, u = T diag(beta) V and the
  * intra-chunk attention P of every chunk ("Training it: the WY trick", D2L
  * 12.5; "The chunked form", ch. 28) in a kernel that runs over all chunks at
- * once, then streams them into the sequential state pass: 40 KiB per
- * (b, h, chunk), i.e. B * H * ceil(T / 64) * 40960 bytes.  Sizes are checked
+ * once, then streams them into the sequential state pass: 40 KiB and a 4-byte
+ * ready flag per (b, h, chunk), i.e. with n = B * H * ceil(T / 64) chunks,
+ * n * 40960 + (4 n rounded up to a multiple of 256) bytes.  Sizes are checked
  * as in dn_chunk_fwd_ex; *bytes is written on DN_OK only.
  */
 DN_API int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk,

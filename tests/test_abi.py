@@ -84,7 +84,7 @@ WS = A + 8 * STEP
     (dict(dv=256), dn.DN_ERR_UNSUPPORTED),
     (dict(path=2), dn.DN_ERR_UNSUPPORTED),                    # tensor-core path needs bf16, d = 128
     (dict(path=3), dn.DN_ERR_UNSUPPORTED),                    # so does its self-test
-    (dict(TC, ws=WS, ws_bytes=40959), dn.DN_ERR_INVALID),     # workspace smaller than one chunk's tiles
+    (dict(TC, ws=WS, ws_bytes=40960 + 255), dn.DN_ERR_INVALID),     # workspace smaller than one chunk's tiles
     (dict(TC, ws=WS + 128, ws_bytes=1 << 20), dn.DN_ERR_INVALID),   # not 256-byte aligned
     (dict(TC, ws=A + 256, ws_bytes=1 << 20), dn.DN_ERR_INVALID),    # overlaps q
     (dict(TC, ws=A + 6 * STEP, ws_bytes=1 << 20), dn.DN_ERR_INVALID),  # overlaps S_T
@@ -102,10 +102,11 @@ def ws_size(lib, B=2, T=130, H=3, dk=128, dv=128, chunk=64, dtype=1, gate=1, pat
 
 def test_workspace_size():
     lib = dn.load_library()
-    # -W and u^T (bf16, 64 x 128 each) and P (bf16, 64 x 64) per (b, h, chunk):
-    # ceil(130 / 64) = 3 chunks
-    assert ws_size(lib) == (dn.DN_OK, 2 * 3 * 3 * (2 * 64 * 128 + 64 * 64) * 2)
-    assert ws_size(lib, path=2) == (dn.DN_OK, 2 * 3 * 3 * 40960)
+    # -W and u^T (bf16, 64 x 128 each) and P (bf16, 64 x 64) per (b, h, chunk), then
+    # a 4-byte ready flag per chunk rounded up to 256 bytes: ceil(130 / 64) = 3 chunks
+    tiles = 2 * 3 * 3
+    assert ws_size(lib) == (dn.DN_OK, tiles * (2 * 64 * 128 + 64 * 64) * 2 + 256)
+    assert ws_size(lib, path=2) == (dn.DN_OK, tiles * 40960 + 256)
     assert ws_size(lib, T=0) == (dn.DN_OK, 0)
     assert ws_size(lib, path=1) == (dn.DN_OK, 0)             # SIMT needs none
     assert ws_size(lib, dtype=0) == (dn.DN_OK, 0)            # fp32 runs on SIMT under auto
@@ -113,7 +114,7 @@ def test_workspace_size():
     assert ws_size(lib, dtype=0, path=2)[0] == dn.DN_ERR_UNSUPPORTED
     assert ws_size(lib, B=-1) == (dn.DN_ERR_INVALID, 12345)  # not written on failure
     assert lib.dn_chunk_fwd_workspace_size(1, 8, 1, 128, 128, 64, 1, 1, 0, None) == dn.DN_ERR_INVALID
-    assert dn.dn_chunk_fwd_workspace_size(1, 64, 1, 128, 128) == 40960
+    assert dn.dn_chunk_fwd_workspace_size(1, 64, 1, 128, 128) == 40960 + 256
 
 
 def test_chunk_fwd_empty_batch_is_ok_without_device(lib):

@@ -54,7 +54,7 @@ def test_noalloc_matches_dn_chunk_fwd_on_two_calls(cuda_device):
 
 
 def test_noalloc_rejects_requests_above_its_scratch_area():
-    # 32 heads x 1024 chunks x 40 KiB = 1.25 GiB of scratch, above the fixed
+    # 32 heads x 1024 chunks x (40 KiB + a 4-byte flag) = 1.25 GiB of scratch, above the fixed
     # 64 MiB: refused before any device work (the fake addresses are never used)
     lib, f = noalloc_fn()
     A, STEP = 0x10000000, 0x40000000
@@ -62,4 +62,4 @@ def test_noalloc_rejects_requests_above_its_scratch_area():
            1, 65536, 32, 128, 128, 64, 1.0, 1, 1, None)
     assert st == dn.DN_ERR_UNSUPPORTED
     msg = lib.dn_last_error().decode()
-    assert str(32 * 1024 * 40960) in msg and str(64 << 20) in msg
+    assert str(32 * 1024 * (40960 + 4)) in msg and str(64 << 20) in msg
