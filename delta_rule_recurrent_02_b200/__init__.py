@@ -25,7 +25,7 @@ import ctypes
 import os
 
 __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
-           "dn_decode_step",
+           "dn_decode_step", "dn_kernel_launches",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
 
@@ -35,7 +35,8 @@ _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
-               "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version")
+               "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version",
+               "dn_kernel_launches")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -78,8 +79,16 @@ def load_library():
     lib.dn_last_error.restype = ctypes.c_char_p
     lib.dn_version.argtypes = []
     lib.dn_version.restype = I
+    lib.dn_kernel_launches.argtypes = []
+    lib.dn_kernel_launches.restype = ctypes.c_ulonglong
     _lib = lib
     return lib
+
+
+def dn_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far (all threads
+    and devices); the difference of two reads counts a region's launches."""
+    return int(load_library().dn_kernel_launches())
 
 
 def _check(lib, status: int):

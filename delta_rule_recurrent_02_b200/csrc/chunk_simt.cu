@@ -317,7 +317,7 @@ static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t st) {
     kern<<<(unsigned)grid, kNT, L::bytes, st>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         a.beta, a.g, a.S0, static_cast<Tin*>(a.o), a.S_T, (int)a.T, a.dv, a.chunk, a.scale);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
 }
 
 template <int DK, typename Tin>

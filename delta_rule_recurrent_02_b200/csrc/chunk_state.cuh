@@ -23,8 +23,8 @@
 // with U~ = U * e^(G_last - G) (the decay of K folded into U's rows).  The CTA
 // owns one (b, h); its state stays in TMEM (fp32 accumulator, pre-scaled by
 // the next chunk's decay, plus a bf16 copy that feeds the next products), and
-// [O | U] alternates between two TMEM buffers so that the output of one chunk
-// drains while the next one runs.  The U and state epilogues run in two
+// [O | U] alternates between two TMEM buffers (one when the SM also hosts a WY
+// group) so that the output of one chunk drains while the next one runs.  The U and state epilogues run in two
 // halves with a barrier each, so that the tensor pipe starts on the first half
 // of a contraction while the second is converted.  Warp roles: 0 TMA + gates,
 // 2 TMEM allocation, 3 MMA issue, 4-7 Qh (in place over the q tile) and the
@@ -58,22 +58,31 @@ constexpr uint32_t kCtaBar = 3;
 
 // TMEM columns (32-bit, 128 lanes)
 constexpr uint32_t TM_SACC = 0;     // S^T fp32 [dv lanes][dk cols], pre-scaled by the coming chunk's decay
-constexpr uint32_t TM_OU = 128;     // 2 x [O^T | U^T] fp32, [dv][C | C], by chunk parity
-constexpr uint32_t TM_ST = 384;     // S^T bf16 pairs [dv][dk/2]
-constexpr uint32_t TM_UT = 448;     // U^T bf16 pairs [dv][C/2]
-constexpr uint32_t TM_UK = 480;     // U~^T bf16 pairs [dv][C/2]
-constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_OU = 128;     // kOuBufs x [O^T | U^T] fp32, [dv][C | C], by chunk
+constexpr uint32_t TM_COLS = 512;   // allocated (a hosted WY group uses the columns past Layout::kCols)
 
 // shared memory (bytes from a 1024-aligned base)
-constexpr int kStages = 3;
 constexpr uint32_t SZ_STAGE = 73728;    // one chunk's tiles:
 constexpr uint32_t ST_K = 0;            //   K [d-block][64 rows][128 B]                        16 KiB
 constexpr uint32_t ST_B = 16384;        //   [d-block][q -> Qh rows 0-63 | -W rows 64-127][128 B] 32 KiB
 constexpr uint32_t ST_UT = 49152;       //   u^T [128 rows (dv)][128 B (C)]                      16 KiB
 constexpr uint32_t ST_P = 65536;        //   P [64 rows (i)][128 B (j)]                           8 KiB
-constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
-constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
-constexpr uint32_t STATE_BYTES = OFF_BAR + 256;   // from a 1024-aligned base
+
+// Two layouts: alone on its SM (three stages, two [O|U] buffers, all 512 TMEM
+// columns), or hosting a WY group (two stages, one [O|U] buffer, 384 columns;
+// the group gets the other 128 and the shared memory past STATE_BYTES).
+template <bool HOSTED>
+struct Layout {
+    static constexpr int kStages = HOSTED ? 2 : 3;
+    static constexpr int kOuBufs = HOSTED ? 1 : 2;
+    static constexpr uint32_t TM_ST = TM_OU + 128 * kOuBufs;   // S^T bf16 pairs [dv][dk/2]
+    static constexpr uint32_t TM_UT = TM_ST + 64;               // U^T bf16 pairs [dv][C/2]
+    static constexpr uint32_t TM_UK = TM_UT + 32;               // U~^T bf16 pairs [dv][C/2]
+    static constexpr uint32_t kCols = TM_UK + 32;
+    static constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
+    static constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
+    static constexpr uint32_t STATE_BYTES = OFF_BAR + 256;
+};
 constexpr uint32_t STAGE_TX = SZ_STAGE;
 
 // barrier indices; where a waiter could otherwise see a barrier two phases on,
@@ -86,7 +95,7 @@ enum {
     B_UTA, B_UTB, B_STA, B_STB,                          // state warps -> MMA (first / second half)
     B_COUNT
 };
-static_assert(OFF_BAR + 8 * B_COUNT + 16 <= OFF_BAR + 256, "barrier area");
+static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
 
 struct Args {
     const CUtensorMap* tm_k;
@@ -94,7 +103,7 @@ struct Args {
     const CUtensorMap* tm_w;
     const CUtensorMap* tm_u;
     const CUtensorMap* tm_p;
-    const unsigned int* flags;
+    const unsigned int* flags;      // ready flags of the workspace tiles; null: all written already
     const float* beta;
     const float* g;
     const float* S0;
@@ -107,9 +116,14 @@ struct Args {
 };
 
 // The state pass of head `head`, run by threads 0 .. kNT - 1 of a CTA whose
-// shared memory starts (1024-aligned) at sm.
-template <int GATE>
-__device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head) {
+// shared memory starts (1024-aligned) at sm.  HOSTED: the caller allocated the
+// TMEM (base tmem_given) and shares the SM with a WY group.
+template <int GATE, bool HOSTED>
+__device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head, uint32_t tmem_given) {
+    using L = Layout<HOSTED>;
+    constexpr int kStages = L::kStages;
+    constexpr uint32_t OFF_GATE = L::OFF_GATE, OFF_BAR = L::OFF_BAR;
+    constexpr uint32_t TM_ST = L::TM_ST, TM_UT = L::TM_UT, TM_UK = L::TM_UK;
     const CUtensorMap& tm_k = *ar.tm_k;
     const CUtensorMap& tm_q = *ar.tm_q;
     const CUtensorMap& tm_w = *ar.tm_w;
@@ -141,14 +155,14 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 2) {
+    if (!HOSTED && warp == 2) {
         tmem_alloc(smem_u32(tmem_slot), TM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     named_bar_sync(kCtaBar, kNT);
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = HOSTED ? tmem_given : *tmem_slot;
 
     if (warp == 0) {
         // ================= producer: gates + TMA ================================
@@ -185,7 +199,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - kStages) / kStages) & 1u) : true;
                 if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
             }
-            if (!(test_flags & 1)) {
+            if (!(test_flags & 1) && flags) {
                 // this chunk's workspace tiles are written (by another CTA, possibly right now)
                 bool ok = lane == 0 ? wait_flag(flags + bh * n + cc, abort_flag) : true;
                 if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
@@ -224,13 +238,15 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 const uint32_t par = (uint32_t)c & 1u;
                 const int s = c % kStages;
                 const uint32_t st = sb + s * SZ_STAGE;
-                const uint32_t ou = tmem + TM_OU + (c & 1) * 128;
+                const uint32_t ou = tmem + TM_OU + (c % L::kOuBufs) * 128;
                 // [O|U]^T = S^T [Qh;-W]^T: once the tiles are in and this buffer's output of
                 // chunk c - 2 is out, the first half of d_k as soon as the state's first half
                 // is written, then the second
                 ok = ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u) &&
                      ctl.wait(B_READY0 + s, (uint32_t)(c / kStages) & 1u) &&
-                     (c < 2 || ctl.wait(B_OFREE0 + (c & 1), (uint32_t)((c - 2) >> 1) & 1u)) && ctl.wait(B_STA, par);
+                     (c < L::kOuBufs || ctl.wait(B_OFREE0 + ((c - L::kOuBufs) & 1),
+                                                 (uint32_t)((c - L::kOuBufs) >> 1) & 1u)) &&
+                     ctl.wait(B_STA, par);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
@@ -313,7 +329,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 if (named_bar_any(1, kSideThreads, !ok)) break;
                 tc_fence_after();
                 __nv_bfloat16* ob = o + (bh * T + (int64_t)cp * kC) * kD + j;
-                const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp & 1) * 128;
+                const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -373,7 +389,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             for (int p = 0; p < 2; ++p) {
                 const int i0 = 32 * p + 16 * hc;         // positions i0 .. i0 + 15
                 float v[16];
-                tmem_ld16(tmem + lane_off + TM_OU + (c & 1) * 128 + 64 + i0, v);
+                tmem_ld16(tmem + lane_off + TM_OU + (c % L::kOuBufs) * 128 + 64 + i0, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) {
@@ -439,7 +455,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 
     named_bar_sync(kCtaBar, kNT);
     if (*abort_flag && tid == 0) atomicOr(status, 1u);
-    if (warp == 2) {
+    if (!HOSTED && warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }

@@ -8,7 +8,9 @@
 //     head first).  A cooperative launch guarantees that every CTA is resident,
 //     so the state pass may wait for tiles that other CTAs are writing; the WY
 //     work overlaps the latency-bound state pass and its tiles are read while
-//     still in L2.  Used while B H leaves a quarter of the SMs to the WY groups.
+//     still in L2.  With many heads the WY work is the longer of the two, and
+//     each state-pass CTA also hosts a WY group (HOSTED: two stages, one [O|U]
+//     buffer).  Used while B H leaves a quarter of the SMs to the WY groups.
 //   * otherwise two launches on the stream: chunk_wy_kernel over all tiles,
 //     then chunk_state_kernel (whose flags are then all set).
 #include "chunk_state.cuh"
@@ -33,16 +35,23 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags};
-    state::state_pass<GATE>(sm, ar, blockIdx.x);
+    state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
 }
 
 namespace {
-constexpr int kFusedThreads = 4 * wy::kNT;          // 32 warps: 4 WY groups, or the state pass + 16 idle warps
-static_assert(state::kNT <= kFusedThreads, "fused CTA size");
-constexpr uint32_t kFusedBytes = (state::STATE_BYTES > 4 * wy::GROUP_BYTES ? state::STATE_BYTES : 4 * wy::GROUP_BYTES) + 1024;
+constexpr int kFusedThreads = 4 * wy::kNT;          // 32 warps: 4 WY groups, or the state pass + up to 16 more
+static_assert(state::kNT + wy::kNT <= kFusedThreads, "fused CTA size");
+constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+// a hosted WY group's shared memory starts past the hosted state pass's
+constexpr uint32_t kHostedWyOff = align1k(state::Layout<true>::STATE_BYTES);
+constexpr uint32_t cmax(uint32_t a, uint32_t b) { return a > b ? a : b; }
+constexpr uint32_t kFusedBytes =
+    cmax(cmax(state::Layout<false>::STATE_BYTES, 4 * wy::GROUP_BYTES), kHostedWyOff + wy::GROUP_BYTES) + 1024;
+static_assert(state::Layout<true>::kCols + wy::TM_COLS <= state::TM_COLS, "hosted TMEM split");
+constexpr uint32_t kHostBar = 6;                    // named barrier of the hosting CTA's state pass + WY group
 }  // namespace
 
-template <int GATE>
+template <int GATE, bool HOSTED>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
@@ -54,12 +63,52 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags};
+    const int64_t tiles = (int64_t)BH * n;
+    const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     if ((int)blockIdx.x < BH) {
-        // ---- state pass of head blockIdx.x (warps 0-15) --------------------------------
-        if (warp >= state::kNT / 32) return;
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags};
-        state::state_pass<GATE>(sm, ar, blockIdx.x);
+        if (!HOSTED) {
+            // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
+            if (warp >= state::kNT / 32) return;
+            state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
+            return;
+        }
+        // ---- state pass (warps 0-15) and one WY group (warps 16-23) ------------------------
+        constexpr int kHostThreads = state::kNT + wy::kNT;
+        if (tid >= kHostThreads) return;
+        uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kHostedWyOff + wy::GROUP_BYTES - 16);
+        wy::Group x = wy::make_group(sm + kHostedWyOff, 0u, 4u, tid - state::kNT);
+        if (tid == state::kNT) {
+            wy::init_group(x);
+            fence_mbar_init();
+        }
+        if (warp == 2) {
+            tmem_alloc(smem_u32(tslot), state::TM_COLS);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        named_bar_sync(kHostBar, kHostThreads);
+        tc_fence_after();
+        const uint32_t tbase = *tslot;
+        if (tid < state::kNT) {
+            state::state_pass<GATE, true>(sm, ar, blockIdx.x, tbase);
+        } else {
+            x.tmem = tbase + state::Layout<true>::kCols;
+            bool ok = true;
+            for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles; t += G) {
+                const int c = (int)(t / BH);
+                ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH);
+            }
+            if (!ok && x.tid == 0) atomicOr(status, 1u);
+        }
+        tc_fence_before();
+        named_bar_sync(kHostBar, kHostThreads);
+        if (warp == 2) {
+            tc_fence_after();
+            tmem_dealloc(tbase, state::TM_COLS);
+        }
         return;
     }
     // ---- four WY groups, each taking every G-th tile in chunk-major order -----------------
@@ -78,13 +127,10 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     x.tmem = *tmem_slot + (uint32_t)grp * wy::TM_COLS;
-    const wy::Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags};
-    const int64_t tiles = (int64_t)BH * n;
-    const int64_t G = (int64_t)(gridDim.x - BH) * 4;
     bool ok = true;
     for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles; t += G) {
         const int c = (int)(t / BH);
-        ok = wy::wy_tile<GATE>(x, ar, c, t - (int64_t)c * BH);
+        ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH);
     }
     tc_fence_before();
     __syncthreads();
@@ -120,17 +166,17 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles));
-    cudaError_t e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
-    if (e != cudaSuccess) return e;
 
     int dev = 0, num_sms = 0, coop = 0;
-    e = cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
     const int64_t BH = a.B * a.H;
     if (coop && fused_fits(BH, num_sms)) {
-        auto kern = chunk_fused_kernel<GATE>;
+        // with many heads the dedicated WY groups get scarce: the state-pass CTAs
+        // host one each (measured: at 64 heads of 148 SMs hosting is not yet a gain)
+        auto kern = BH * 2 > (int64_t)num_sms + 12 ? chunk_fused_kernel<GATE, true> : chunk_fused_kernel<GATE, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedBytes);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
@@ -150,20 +196,24 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             unsigned int* status = a.status;
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
                             &T_i, &n_i, &scale, &status, &test_flags};
-            return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
-                                               dim3(kFusedThreads), args, kFusedBytes, st);
+            // the flags are cleared on the same stream right before the launch
+            e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
+            if (e != cudaSuccess) return e;
+            return counted(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
+                                                       dim3(kFusedThreads), args, kFusedBytes, st));
         }
     }
     e = launch_chunk_wy(a, m, st);
     if (e != cudaSuccess) return e;
     auto kern = chunk_state_kernel<GATE>;
-    const uint32_t bytes = state::STATE_BYTES + 1024;
+    const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, m.flags, a.beta, a.g, a.S0,
+    // the WY kernel has finished before this launch starts: no flags to wait for
+    kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
                                                   a.status, a.test_flags);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
 }
 
 }  // namespace

@@ -65,7 +65,7 @@ cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStrea
     kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(m.q, m.k, m.v, m.w, m.u, m.p_ws, m.flags,
                                                               (int)(a.B * a.H), a.beta, a.g, (int)a.T, n, a.scale,
                                                               a.status, a.test_flags);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
 }
 
 }  // namespace

@@ -123,7 +123,7 @@ static cudaError_t launch_decode_gate(const DecodeArgs& a, cudaStream_t st) {
             decode_step_kernel<DK, DV, Tin, kGatePerKey><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
             break;
     }
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
 }
 
 template <int DK, int DV>

@@ -1,5 +1,6 @@
 // dn_api.cu -- the C ABI: argument validation, kernel choice, launch, status.
 #include <cuda_runtime.h>
+#include <atomic>
 #include <stdarg.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -100,11 +101,16 @@ size_t workspace_needed(const dn::ChunkArgs& a, bool use_tc) {
 
 namespace dn {
 int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 }  // namespace dn
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 0; }
+int dn_version(void) { return (2 << 16) | 1; }
+
+unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 
 const char* dn_status_str(int status) {
     switch (status) {

@@ -46,4 +46,12 @@ cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st);
 // Record `msg` as the calling thread's dn_last_error() and return `code`.
 int report_error(int code, const char* msg);
 
+// Count one kernel launch of this library (read by dn_kernel_launches()).
+void count_launch();
+// `e` is the result of one kernel launch: count it if it succeeded.
+inline cudaError_t counted(cudaError_t e) {
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
 }  // namespace dn

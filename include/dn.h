@@ -212,6 +212,15 @@ DN_API const char* dn_last_error(void);
 /* ABI version, (major << 16) | minor. */
 DN_API int dn_version(void);
 
+/*
+ * dn_kernel_launches -- number of CUDA kernels this library has launched in
+ * this process, over all threads and devices (monotonic; counted when the
+ * launch call succeeds, not when the kernel ends).  Memsets and copies on the
+ * caller's stream are not kernels of this library and are not counted.  The
+ * difference of two reads brackets the kernels a region of calls issued.
+ */
+DN_API unsigned long long dn_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -90,8 +90,10 @@ WS = A + 8 * STEP
     (dict(TC, ws=A + 6 * STEP, ws_bytes=1 << 20), dn.DN_ERR_INVALID),  # overlaps S_T
 ])
 def test_chunk_fwd_rejects(lib, over, code):
+    before = lib.dn_kernel_launches()
     assert chunk_call(lib, **over) == code
     assert lib.dn_last_error() != b""
+    assert lib.dn_kernel_launches() == before        # refused before any launch
 
 
 def ws_size(lib, B=2, T=130, H=3, dk=128, dv=128, chunk=64, dtype=1, gate=1, path=0):

@@ -172,6 +172,36 @@ def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
     assert ei.value.status == dn.DN_ERR_INVALID
 
 
+@pytest.mark.parametrize("B,H,T", [(3, 32, 200), (4, 32, 130)])
+def test_tc_many_heads(cuda_device, B, H, T):
+    # 96 heads: the single launch in which each state-pass CTA also hosts a WY
+    # group; 128 heads: the two launches (WY kernel, then state pass)
+    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate="scalar", seed=B * H + T, s0_std=0.2)
+    sc = 128 ** -0.5
+    o, S = run(to_dev(inp), sc, path="tc")
+    dn.dn_device_status()
+    bh = [(0, 0), (1, 7), (B - 1, H - 1), (B // 2, H // 2)]
+    ro, rS = oracle_prefill(inp, sc, bh=bh)
+    assert_close(pick(o, bh), ro, "bf16", "o")
+    assert_close(pick(S, bh), rS, "bf16", "S_T")
+
+
+@pytest.mark.parametrize("B,H,T,path,kernels", [
+    (4, 16, 4096, "tc", 1),      # the cooperative launch: WY groups beside the state pass
+    (3, 32, 200, "tc", 1),       # the same, each state-pass CTA hosting a WY group
+    (4, 32, 130, "tc", 2),       # too many heads for one launch: WY kernel, then state pass
+    (2, 3, 200, "simt", 1),
+])
+def test_chunk_kernel_launch_count(cuda_device, B, H, T, path, kernels):
+    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate="scalar", seed=5, s0_std=0.2)
+    d = to_dev(inp)
+    torch.cuda.synchronize()
+    before = dn.dn_kernel_launches()
+    run(d, 0.1, path=path)
+    assert dn.dn_kernel_launches() - before == kernels
+    dn.dn_device_status()
+
+
 def test_chunk_empty_inputs(cuda_device):
     # T = 0: no output rows; S_T = S0 (or zeros).  B = 0: nothing at all.
     S0 = torch.randn(2, 3, 64, 64, device="cuda")
