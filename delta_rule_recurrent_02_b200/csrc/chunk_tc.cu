@@ -97,10 +97,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         } else {
             x.tmem = tbase + state::Layout<true>::kCols;
             bool ok = true;
+            int64_t pending = -1;
             for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles; t += G) {
                 const int c = (int)(t / BH);
-                ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH);
+                ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
             }
+            if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
             if (!ok && x.tid == 0) atomicOr(status, 1u);
         }
         tc_fence_before();
@@ -128,10 +130,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     x.tmem = *tmem_slot + (uint32_t)grp * wy::TM_COLS;
     bool ok = true;
+    int64_t pending = -1;
     for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles; t += G) {
         const int c = (int)(t / BH);
-        ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH);
+        ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
     }
+    if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
     tc_fence_before();
     __syncthreads();
     if (!ok && x.tid == 0) atomicOr(status, 1u);

@@ -41,7 +41,9 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // chunk-major order: chunk 0 of every head first
     const int c = (int)(blockIdx.x / (unsigned)BH);
     const int64_t bh = blockIdx.x - (int64_t)c * BH;
-    const bool ok = wy_tile<GATE>(x, ar, c, bh);
+    int64_t pending = -1;
+    const bool ok = wy_tile<GATE>(x, ar, c, bh, pending);
+    if (ok && tid == kStoreTid) publish_pending(ar, pending);
     tc_fence_before();
     __syncthreads();
     if (!ok && tid == 0) atomicOr(status, 1u);

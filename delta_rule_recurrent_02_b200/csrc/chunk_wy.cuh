@@ -17,15 +17,23 @@
 //
 //   TMA       K and Q tiles, stacked per 64-column block as [K rows | Q rows]
 //   tcgen05   [K;Q] K^T -> TMEM (bf16 -> fp32): K K^T for A, Q K^T for P
+//   TMA       V, into the dead K/Q space beside T (it lands during the solve)
 //   CUDA core masks and decay -> A (fp32, shared memory); P (bf16) straight to
 //             the workspace
-//   CUDA core T = (I + A)^-1 over the tiles' space: the 16 x 16 diagonal blocks
+//   CUDA core T = (I + A)^-1 at the start of that space: the 16 x 16 diagonal blocks
 //             D_k = (I + A_kk)^-1 by forward substitution, M_kl = D_k A_kl,
 //             then T_kl = -sum_{m=l}^{k-1} M_km T_ml in three rounds (fp32);
 //             then T diag(beta e^G) and T diag(beta) as bf16 operand tiles
-//   TMA       K and V again (from L2) over T
+//   TMA       K again (from L2) over T
 //   tcgen05   W^T = K^T (T diag(beta e^G))^T, u^T = V^T (T diag(beta))^T -> TMEM
 //   epilogue  TMEM -> bf16 tiles in shared memory -> TMA stores to the workspace
+//
+// The ready flag of a tile is raised once its stores are complete, and by a
+// thread with time to spare: the output stores are issued by kStoreTid (warp 6),
+// which raises the flag during the group's next tile, in the A/P epilogue where
+// warp 6 has only zeros to write (after the group's last tile, the caller
+// raises it with publish_pending()).  The gpu-scope release costs about a
+// thousand cycles under load; there it is off the group's critical path.
 //
 // A partial last chunk has beta = 0 and g = 0 past its end: those rows of A
 // and P, and those columns of W^T and u^T, are zero (equal to zero padding).
@@ -43,6 +51,7 @@ using namespace sm100;
 using namespace tc;
 
 constexpr int kNT = 256;        // 8 warps per group
+constexpr int kStoreTid = 192;  // issues the output stores and raises the ready flags
 
 // TMEM columns (32-bit, 128 lanes)
 constexpr uint32_t TM_G = 0;    // gram [K;Q] K^T: lanes 0-63 K K^T, 64-127 Q K^T
@@ -50,18 +59,25 @@ constexpr uint32_t TM_W = 0;    // W^T fp32 [dk][C], after the gram has been rea
 constexpr uint32_t TM_U = 64;   // u^T fp32 [dv][C]
 constexpr uint32_t TM_COLS = 128;
 
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KV = 0;          // [d-block][K rows 0-63 | Q rows][128 B] = 32 KiB for the gram;
-                                        // T during the solve; [d-block][K | V] for W and u; last,
-                                        // the -W and u^T output tiles
+// shared memory (bytes from a 1024-aligned base), in the order of use:
+//   [0, 32K)      the gram's [K0 | Q0 | K1 | Q1] (d-block b's 64 x 64 bf16 K and Q tiles)
+//   [0, 17K)      T (fp32, padded rows), while V = [V0 | V1] lands in [17K, 33K)
+//   [0, 16K)      K = [K0 | K1] again, beside V, for W and u
+//   [0, 32K)      the -W and u^T output tiles
+//   [33K, 50K)    A, then M = D^-1 A; then the bf16 Tw, Tb operand tiles
+constexpr uint32_t OFF_KV = 0;
 constexpr uint32_t OFF_T = 0;           // fp32 64 x 68: T = (I + A)^-1
-constexpr uint32_t OFF_A = 32768;       // fp32 64 x 68: A, then M = D^-1 A; then the bf16 tiles
+constexpr uint32_t OFF_V = 17408;       // V tiles, loaded once the gram has read K and Q
+constexpr uint32_t OFF_A = 33792;       // fp32 64 x 68: A, then M = D^-1 A; then the bf16 tiles
 constexpr uint32_t OFF_TW = OFF_A;      //   T diag(beta e^G), K-major B [N=i][K=j]: [64 rows][128 B]
 constexpr uint32_t OFF_TB = OFF_A + 8192;   // T diag(beta), same layout
-constexpr uint32_t OFF_GATE = 50176;    // one gate slot
+constexpr uint32_t OFF_GATE = OFF_A + 17408;   // one gate slot
 constexpr uint32_t OFF_BAR = OFF_GATE + GATE_FLOATS * 4;
-constexpr uint32_t GROUP_BYTES = 52224;  // one group's shared memory, a multiple of 1024
-static_assert(OFF_BAR + 64 <= GROUP_BYTES, "group layout");
+constexpr uint32_t GROUP_BYTES = 53248;  // one group's shared memory, a multiple of 1024
+// (the last 16 bytes of a group stay free: a CTA keeps its TMEM address there)
+static_assert(OFF_BAR + 64 <= GROUP_BYTES - 16, "group layout");
+static_assert(OFF_T + 64 * 68 * 4 <= OFF_V && OFF_V + 16384 <= OFF_A, "T, V and A overlap");
+static_assert(OFF_V % 1024 == 0 && OFF_A % 1024 == 0 && OFF_TB % 1024 == 0, "128-byte swizzle atoms");
 enum { B_FULL = 0, B_MMA = 1 };
 
 // fp32 64 x 64 matrix, rows padded to 68 floats: 16-byte aligned rows, and
@@ -155,9 +171,25 @@ struct Args {
     int test_flags;
 };
 
-// Chunk c of head bh.  Returns false (the group's abort flag set) if a wait gave up.
+// Thread kStoreTid of a group: raise the ready flag of the group's previous
+// tile, if one is pending, once its stores (issued by this thread) are
+// complete.  The proxy fence orders those async-proxy writes before the
+// release; the other threads' writes of the tile (P) precede it through the
+// group barriers.  A reader that acquires the flag and fences its async proxy
+// reads the tiles.
+__device__ __forceinline__ void publish_pending(const Args& ar, int64_t& pending) {
+    if (pending < 0) return;
+    bulk_wait_all();
+    fence_async_global();
+    st_release_gpu(ar.flags + pending, 1u);
+    pending = -1;
+}
+
+// Chunk c of head bh.  `pending` (thread kStoreTid's copy counts) is the
+// group's tile whose flag is still to be raised, or -1; on return it is this
+// tile.  Returns false (the group's abort flag set) if a wait gave up.
 template <int GATE>
-__device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh) {
+__device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh, int64_t& pending) {
     const uint32_t sb = x.sb;
     float* gs = reinterpret_cast<float*>(x.sm + OFF_GATE);
     float* Am = reinterpret_cast<float*>(x.sm + OFF_A);
@@ -171,7 +203,6 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     const float* __restrict__ beta = ar.beta;
     const float* __restrict__ g = ar.g;
     __nv_bfloat16* __restrict__ p_out = ar.p_out;
-    unsigned int* flags = ar.flags;
     const CUtensorMap& tm_q = *ar.tm_q;
     const CUtensorMap& tm_k = *ar.tm_k;
     const CUtensorMap& tm_v = *ar.tm_v;
@@ -222,6 +253,15 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     ok = ok && ctl.wait(B_MMA, 0);
     if (named_bar_any(x.bar, kNT, !ok)) goto done;
     tc_fence_after();
+    if (tid == 0 && load) {
+        // V into the second half of the K/Q space, which the gram has read; the
+        // phase also counts the K tiles issued after the solve
+        const uint32_t fb = ctl.bar(B_FULL);
+        mbar_arrive_expect_tx(fb, 4 * 8192);
+        tma_load_2d(sb + OFF_V + 0, &tm_v, 0, (int)t0, fb);
+        tma_load_2d(sb + OFF_V + 8192, &tm_v, 64, (int)t0, fb);
+        loads = 2;
+    }
 
     // ---- A = strict_tril(beta_i (K K^T)_ij D_ij) from TMEM lanes 0-63 (warps 0, 1, 4, 5)
     //      and P = scale tril((Q K^T)_ij D_ij) from lanes 64-127 (warps 2, 3, 6, 7), 32
@@ -257,7 +297,11 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             // P row i, columns j0 .. j0 + 31 -> workspace (row-major [64][64])
             __nv_bfloat16* prow = p_out + (tile * kC + i) * kC + j0;
             if (q == 2 && j0 == 32) {
-                // rows 0-31 x columns 32-63 lie above the diagonal
+                // warp 6: the previous tile's ready flag, then zeros: rows 0-31 x
+                // columns 32-63 lie above the diagonal
+                static_assert(kStoreTid == 6 * 32, "the flag is raised by warp 6");
+                if (tid == kStoreTid) publish_pending(ar, pending);
+                __syncwarp();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) st_global_v4(prow + 8 * q4, 0u, 0u, 0u, 0u);
             } else {
@@ -368,16 +412,12 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     fence_async_smem();
     named_bar_sync(x.bar, kNT);
 
-    // ---- K and V (L2-resident by now) over T, then W^T = K^T Tw^T, u^T = V^T Tb^T -------
+    // ---- K (L2-resident by now) over T, then W^T = K^T Tw^T, u^T = V^T Tb^T -------------
     if (tid == 0) {
         if (load) {
-            const uint32_t fb = ctl.bar(B_FULL);
-            mbar_arrive_expect_tx(fb, 4 * 8192);
+            const uint32_t fb = ctl.bar(B_FULL);     // the phase V opened
             tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, (int)t0, fb);
-            tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, (int)t0, fb);
-            tma_load_2d(sb + OFF_KV + 8192, &tm_v, 0, (int)t0, fb);
-            tma_load_2d(sb + OFF_KV + 24576, &tm_v, 64, (int)t0, fb);
-            loads = 2;
+            tma_load_2d(sb + OFF_KV + 8192, &tm_k, 64, (int)t0, fb);
         }
         ok = ctl.wait(B_FULL, 1);
         if (ok) {
@@ -385,11 +425,11 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             const uint32_t idesc = idesc_bf16(128, 64, 1, 0);    // A MN-major, B K-major
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_KV + kk * 2048, 16384, 1024),
+                mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_KV + kk * 2048, 8192, 1024),
                          sw128_desc(sb + OFF_TW + kk * 32, 16, 1024), idesc, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_KV + 8192 + kk * 2048, 16384, 1024),
+                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_V + kk * 2048, 8192, 1024),
                          sw128_desc(sb + OFF_TB + kk * 32, 16, 1024), idesc, kk > 0);
             mma_commit(ctl.bar(B_MMA));
         }
@@ -433,16 +473,15 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     }
     fence_async_smem();
     named_bar_sync(x.bar, kNT);
-    if (tid == 0) {
+    if (tid == kStoreTid) {
         tma_store_2d(&tm_w, 0, (int)(tile * kC), sb + OFF_KV);
         tma_store_2d(&tm_w, 64, (int)(tile * kC), sb + OFF_KV + 8192);
         tma_store_2d(&tm_u, 0, (int)(tile * kD), sb + OFF_KV + 16384);
         bulk_commit_group();
-        // publish the tile: its stores complete, then its ready flag (release)
-        bulk_wait_all();
-        fence_async_global();
-        __threadfence();
-        st_release_gpu(flags + tile, 1u);
+        // the staging tiles are read: the space is free for the next tile's loads;
+        // the flag waits until the stores are complete
+        bulk_wait_read_all();
+        pending = tile;
     }
     tc_fence_before();
     named_bar_sync(x.bar, kNT);
@@ -454,6 +493,9 @@ done:
     if (tid == 0) {
         // let the loads land before the shared memory is reused or released
         if (loads > 0) mbar_wait_bounded(ctl.bar(B_FULL), (uint32_t)(loads - 1), kWaitNs);
+    }
+    if (tid == kStoreTid) {
+        publish_pending(ar, pending);
         bulk_wait_all();
     }
     *abort_flag = 1;
