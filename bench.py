@@ -250,6 +250,60 @@ def run_reference(args):
     return 0
 
 
+def measure_prefill_configs(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
+    """Each prefill workload of the method alone (small DeltaNet, long Gated
+    DeltaNet, KDA): median of `calls` CUDA-event-timed calls after `warm`, with
+    the path the library picks, against the counted FLOPs and algorithmic
+    bytes.  The bench-size Gated DeltaNet prefill is the step's own."""
+    out = {}
+    for cfg in (W.DELTANET_SMALL, W.GDN_LONG, W.KDA_PREFILL):
+        inp = W.gen_prefill_config(cfg)
+        d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+        o = torch.empty((cfg.B, cfg.H, cfg.T, cfg.dv), dtype=W.torch_dtype(cfg.dtype), device=dev)
+        S_T = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+        nws = dn.dn_chunk_fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, chunk=cfg.chunk,
+                                             dtype=cfg.dtype, gate=cfg.gate)
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+
+        def call():
+            dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o, S_T, chunk=cfg.chunk,
+                            scale=cfg.scale, workspace=ws, stream=stream)
+
+        for _ in range(warm):
+            call()
+        k0 = dn.dn_kernel_launches()
+        call()
+        launches = dn.dn_kernel_launches() - k0
+        ts = []
+        for _ in range(calls):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        dn.dn_device_status(stream)
+        ms = statistics.median(ts)
+        esz = 2 if cfg.dtype == "bf16" else 4
+        fl = prefill_flops(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.chunk)
+        by = prefill_bytes(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, esz=esz, gate_per_key=cfg.gate == "per_key",
+                           s0=cfg.s0_std is not None)
+        tf = fl / (ms * 1e-3) / 1e12
+        gb = by / (ms * 1e-3) / 1e9
+        out[cfg.name] = {"ms_per_call": ms, "tokens_per_s": cfg.B * cfg.T / (ms * 1e-3),
+                         "path": "tensor cores" if nws else "simt (fp32 CUDA cores)",
+                         "kernel_launches_per_call": launches,
+                         "counted_flops": fl, "algorithmic_bytes": by,
+                         "tensor_tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
+                         "hbm_gbs": gb, "hbm_frac": gb / peaks["hbm_gbs"],
+                         "traffic": traffic_for("chunk_simt_kda") if cfg is W.KDA_PREFILL and not nws else None,
+                         "timing": f"median of {calls} calls after {warm}, CUDA events"}
+        del d, o, S_T, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def workload_config():
     return {"workload": "gated_deltanet_prefill_B4_H16_T4096_d128_bf16_chunk64 + "
                         "decode_step_B256_H32_d128_bf16_fp32state",
@@ -275,7 +329,9 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other prefill workloads (small DeltaNet, long GDN, KDA)")
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "kda"], default=None,
                     help="launch one kernel of the step a few times without timing (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -397,6 +453,8 @@ def main():
             "decode": {"tokens_per_s": world * dc.B / (dec_ms * 1e-3), "roofline": dec_roof},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clocks}
+    if world == 1 and not args.no_configs:
+        line["other_prefill_workloads"] = measure_prefill_configs(dn, torch, W, peaks, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]
@@ -421,8 +479,8 @@ def run_profile_case(args):
     import delta_rule_recurrent_02_b200 as dn
     from delta_rule_recurrent_02_b200 import workloads as W
     dev = torch.device("cuda", 0)
-    if args.profile_case == "prefill":
-        pc = W.GDN_PREFILL
+    if args.profile_case in ("prefill", "kda"):
+        pc = W.GDN_PREFILL if args.profile_case == "prefill" else W.KDA_PREFILL
         P = {k: (None if v is None else v.to(dev)) for k, v in W.gen_prefill_config(pc).items()}
         o = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
         S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)

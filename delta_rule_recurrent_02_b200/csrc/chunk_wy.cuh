@@ -30,10 +30,10 @@
 //
 // The ready flag of a tile is raised once its stores are complete, and by a
 // thread with time to spare: the output stores are issued by kStoreTid (warp 6),
-// which raises the flag during the group's next tile, in the A/P epilogue where
-// warp 6 has only zeros to write (after the group's last tile, the caller
-// raises it with publish_pending()).  The gpu-scope release costs about a
-// thousand cycles under load; there it is off the group's critical path.
+// which raises the flag during the group's next tile, while warps 0-5 form the
+// M blocks and warp 6 has nothing else to do (after the group's last tile, the
+// caller raises it with publish_pending()).  The gpu-scope release costs about
+// 1.5k cycles under load; there it is off the group's critical path.
 //
 // A partial last chunk has beta = 0 and g = 0 past its end: those rows of A
 // and P, and those columns of W^T and u^T, are zero (equal to zero padding).
@@ -299,9 +299,6 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             if (q == 2 && j0 == 32) {
                 // warp 6: the previous tile's ready flag, then zeros: rows 0-31 x
                 // columns 32-63 lie above the diagonal
-                static_assert(kStoreTid == 6 * 32, "the flag is raised by warp 6");
-                if (tid == kStoreTid) publish_pending(ar, pending);
-                __syncwarp();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) st_global_v4(prow + 8 * q4, 0u, 0u, 0u, 0u);
             } else {
@@ -358,6 +355,8 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
         __syncwarp();
         blk16_store(Am, 16 * k, 16 * l, acc, lane);
+    } else if (tid == kStoreTid) {
+        publish_pending(ar, pending);                 // the previous tile's ready flag
     }
     named_bar_sync(x.bar, kNT);
     // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds; one block product per warp
