@@ -297,7 +297,8 @@ def measure_prefill_configs(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
                          "counted_flops": fl, "algorithmic_bytes": by,
                          "tensor_tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
                          "hbm_gbs": gb, "hbm_frac": gb / peaks["hbm_gbs"],
-                         "traffic": traffic_for("chunk_simt_kda") if cfg is W.KDA_PREFILL and not nws else None,
+                         "traffic": (traffic_for("kda_tc" if nws else "chunk_simt_kda")
+                                     if cfg is W.KDA_PREFILL else None),
                          "timing": f"median of {calls} calls after {warm}, CUDA events"}
         del d, o, S_T, ws
         torch.cuda.empty_cache()

@@ -98,8 +98,8 @@ enum {
 static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
 
 struct Args {
-    const CUtensorMap* tm_k;
-    const CUtensorMap* tm_q;
+    const CUtensorMap* tm_k;        // k; per-key gate: the workspace's K~
+    const CUtensorMap* tm_q;        // q; per-key gate: the workspace's Qh
     const CUtensorMap* tm_w;
     const CUtensorMap* tm_u;
     const CUtensorMap* tm_p;
@@ -113,7 +113,11 @@ struct Args {
     float scale;
     unsigned int* status;
     int test_flags;
+    const float* gam;               // per-key gate: the workspace's e^Gamma_last per tile and channel
 };
+
+// Gate slot with the per-key gate: e^Gamma_last of each key channel.
+constexpr int G_KGAM = 0;
 
 // The state pass of head `head`, run by threads 0 .. kNT - 1 of a CTA whose
 // shared memory starts (1024-aligned) at sm.  HOSTED: the caller allocated the
@@ -174,6 +178,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             prefetch_tmap(&tm_p);
         }
         int issued = 0;
+        constexpr bool KDA = GATE == kGatePerKey;
         // beta / g of the next chunk, loaded one chunk ahead
         float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
         auto fetch = [&](int cc) {
@@ -186,14 +191,16 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
             }
         };
-        fetch(0);
+        if (!KDA) fetch(0);
         for (int cc = 0; cc < n; ++cc) {
             const int s = cc % kStages;
-            const float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
-            if (cc + 1 < n) fetch(cc + 1);
-            chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            if (!KDA) {
+                const float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
+                if (cc + 1 < n) fetch(cc + 1);
+                chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            }
             // the stage is free once the products of chunk cc - 3 are done
             if (cc >= kStages) {
                 bool ok = lane == 0 ? ctl.wait(B_FREE0 + s, (uint32_t)((cc - kStages) / kStages) & 1u) : true;
@@ -204,10 +211,20 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 bool ok = lane == 0 ? wait_flag(flags + bh * n + cc, abort_flag) : true;
                 if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
             }
+            if (KDA) {
+                // the chunk's decays per key channel, from the workspace, into slot cc % 4:
+                // its previous reader (chunk cc - 4) is done once chunk cc - 3's products are
+                const float4 gv = test_flags & 1 ? make_float4(1.f, 1.f, 1.f, 1.f)
+                                                 : reinterpret_cast<const float4*>(ar.gam + (bh * n + cc) * kD)[lane];
+                reinterpret_cast<float4*>(gates + (cc & 3) * GATE_FLOATS + G_KGAM)[lane] = gv;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
+            }
             if (lane == 0 && !(test_flags & 1)) {
                 fence_async_global();
-                const int y = (int)(bh * T + (int64_t)cc * kC);
                 const int64_t tile = bh * n + cc;
+                // q and k rows of the chunk; with the per-key gate, Qh and K~ rows of the tile
+                const int y = KDA ? (int)(tile * kC) : (int)(bh * T + (int64_t)cc * kC);
                 const uint32_t st = sb + s * SZ_STAGE;
                 const uint32_t fb = ctl.bar(B_FULL0 + s);
                 mbar_arrive_expect_tx(fb, STAGE_TX);
@@ -304,8 +321,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                           ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
+                // (with the per-key gate the workspace holds Qh already)
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < (GATE == kGatePerKey ? 0 : 8); ++u) {
                     const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
                     const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
                     const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
@@ -356,7 +374,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
         ok = !named_bar_any(2, kChainThreads, !ok);
         if (ok) {
             // S0 -> TMEM: fp32 pre-scaled by chunk 0's decay, and its bf16 copy
-            const float gamma0 = gates[G_GAMMA];
+            const float gamma0 = GATE == kGatePerKey ? 0.f : gates[G_GAMMA];
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
                 const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
@@ -368,7 +386,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= gamma0;
+                for (int e = 0; e < 32; ++e)
+                    v[e] *= GATE == kGatePerKey ? gates[G_KGAM + pc * 32 + e] : gamma0;
                 tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
                 tmem_wait_st();
                 tc_fence_before();
@@ -406,11 +425,14 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                 for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 tmem_st8(tmem + lane_off + TM_UT + (i0 >> 1), pk);
+                if (GATE != kGatePerKey) {
+                    // U~ = U (.) e^(G_last - G) by rows; with the per-key gate K~ carries the decay
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
-                    pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
-                    pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
+                        pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
+                        pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
+                    }
                 }
                 tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
                 tmem_wait_st();
@@ -424,7 +446,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
             tc_fence_after();
             const bool last = c + 1 == n;
-            const float gnext = last ? 1.f : gates[((c + 1) & 3) * GATE_FLOATS + G_GAMMA];
+            const float* gsn = gates + ((c + 1) & 3) * GATE_FLOATS;
+            const float gnext = last || GATE == kGatePerKey ? 1.f : gsn[G_GAMMA];
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
                 const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
@@ -442,7 +465,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                     for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                     tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= gnext;
+                    for (int e = 0; e < 32; ++e) v[e] *= GATE == kGatePerKey ? gsn[G_KGAM + pc * 32 + e] : gnext;
                     tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
                     tmem_wait_st();
                 }

@@ -29,12 +29,13 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_p, const unsigned int* __restrict__ flags,
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, float scale, unsigned int* status,
-                   int test_flags) {
+                   int test_flags, const float* __restrict__ gam) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags};
+    const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
+                         gam};
     state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
 }
 
@@ -68,7 +69,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags};
+                             test_flags, nullptr};
         if (!HOSTED) {
             // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
             if (warp >= state::kNT / 32) return;
@@ -216,7 +217,42 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     // the WY kernel has finished before this launch starts: no flags to wait for
     kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
-                                                  a.status, a.test_flags);
+                                                  a.status, a.test_flags, nullptr);
+    return counted(cudaGetLastError());
+}
+
+// Per-key gate (KDA): the WY kernel for it (chunk_wy_kda.cu) over all tiles,
+// then the state pass, which reads Qh, K~ and the decays from the workspace.
+cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
+    const uint64_t rows = (uint64_t)(a.B * a.H * a.T);
+    const int n = (int)((a.T + kC - 1) / kC);
+    const uint64_t tiles = (uint64_t)(a.B * a.H) * (uint64_t)n;
+    uint8_t* w_ws = static_cast<uint8_t*>(a.ws);
+    uint8_t* u_ws = w_ws + tiles * kWsWBytes;
+    uint8_t* p_ws = u_ws + tiles * kWsUBytes;
+    uint8_t* kt_ws = p_ws + tiles * kWsPBytes;
+    uint8_t* qh_ws = kt_ws + tiles * kWsKtBytes;
+    uint8_t* gam_ws = qh_ws + tiles * kWsQhBytes;
+    TcMaps m;
+    if (!make_tmap(&m.q, a.q, kD, rows, 64) || !make_tmap(&m.k, a.k, kD, rows, 64) ||
+        !make_tmap(&m.v, a.v, kD, rows, 64) || !make_tmap(&m.w, w_ws, kD, tiles * kC, 64) ||
+        !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64) ||
+        !make_tmap(&m.kt, kt_ws, kD, tiles * kC, 64) || !make_tmap(&m.qh, qh_ws, kD, tiles * kC, 64))
+        return cudaErrorInvalidValue;
+    m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
+    m.kt_ws = reinterpret_cast<__nv_bfloat16*>(kt_ws);
+    m.qh_ws = reinterpret_cast<__nv_bfloat16*>(qh_ws);
+    m.gam_ws = reinterpret_cast<float*>(gam_ws);
+    m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles, true));
+    cudaError_t e = launch_chunk_wy_kda(a, m, st);
+    if (e != cudaSuccess) return e;
+    auto kern = chunk_state_kernel<kGatePerKey>;
+    const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(a.B * a.H), state::kNT, bytes, st>>>(m.kt, m.qh, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
+                                                          static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
+                                                          a.scale, a.status, a.test_flags, m.gam_ws);
     return counted(cudaGetLastError());
 }
 
@@ -224,17 +260,18 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
 
 bool tc_supports(const ChunkArgs& a) {
     const int64_t n = (a.T + kC - 1) / kC;
-    return a.bf16 && a.chunk == kC && a.dk == kD && a.dv == kD && a.gate != kGatePerKey &&
+    return a.bf16 && a.chunk == kC && a.dk == kD && a.dv == kD &&
            a.B * a.H * a.T < (int64_t(1) << 31) && a.B * a.H * n * kD < (int64_t(1) << 31);
 }
 
 size_t tc_workspace_bytes(const ChunkArgs& a) {
     const int64_t n = (a.T + kC - 1) / kC;
-    return ws_total_bytes((uint64_t)(a.B * a.H * n));
+    return ws_total_bytes((uint64_t)(a.B * a.H * n), a.gate == kGatePerKey);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
     if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+    if (a.gate == kGatePerKey) return launch_tc_kda(a, st);
     return a.gate == kGateScalar ? launch_tc_gate<kGateScalar>(a, st) : launch_tc_gate<kGateNone>(a, st);
 }
 

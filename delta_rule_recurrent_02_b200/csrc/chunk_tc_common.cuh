@@ -29,10 +29,24 @@ constexpr size_t kWsWBytes = (size_t)kC * kD * 2;
 constexpr size_t kWsUBytes = (size_t)kD * kC * 2;
 constexpr size_t kWsPBytes = (size_t)kC * kC * 2;
 constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes;
+// With the per-key gate (KDA) three more arrays follow, which the state pass
+// reads in place of q and k and of the scalar decays:
+//   K~   [tiles * 64 rows][128]  k (.) e^(Gamma_last - Gamma)      (bf16)
+//   Qh   [tiles * 64 rows][128]  scale q (.) e^Gamma               (bf16)
+//   gam  [tiles][128]            e^(Gamma_last), per key channel  (fp32)
+constexpr size_t kWsKtBytes = (size_t)kC * kD * 2;
+constexpr size_t kWsQhBytes = (size_t)kC * kD * 2;
+constexpr size_t kWsGamBytes = (size_t)kD * 4;
+constexpr size_t kWsKdaTileBytes = kWsTileBytes + kWsKtBytes + kWsQhBytes + kWsGamBytes;
+static_assert(kWsKdaTileBytes % 256 == 0, "flags stay 256-byte aligned");
 // ...then one 32-bit ready flag per tile, set (release) once the tile is
 // written and awaited (acquire) before the state pass loads it.
-inline size_t ws_flags_offset(uint64_t tiles) { return (size_t)tiles * kWsTileBytes; }
-inline size_t ws_total_bytes(uint64_t tiles) { return ws_flags_offset(tiles) + ((tiles * 4 + 255) / 256) * 256; }
+inline size_t ws_flags_offset(uint64_t tiles, bool kda = false) {
+    return (size_t)tiles * (kda ? kWsKdaTileBytes : kWsTileBytes);
+}
+inline size_t ws_total_bytes(uint64_t tiles, bool kda = false) {
+    return ws_flags_offset(tiles, kda) + ((tiles * 4 + 255) / 256) * 256;
+}
 
 // Tensor maps of the tensor-core path (128-byte swizzle, 64-column boxes):
 // q, k, v as [B H T][128] with 64-row boxes; the workspace's -W as [tiles 64][128]
@@ -42,6 +56,12 @@ struct TcMaps {
     CUtensorMap q, k, v, w, u, p;
     __nv_bfloat16* p_ws;     // the workspace's P array (written with plain stores)
     unsigned int* flags;     // the workspace's ready flags, zeroed before each prefill
+    // per-key gate only: the workspace's K~ and Qh as [tiles 64][128] with 64-row
+    // boxes, and its gam array
+    CUtensorMap kt, qh;
+    __nv_bfloat16* kt_ws;
+    __nv_bfloat16* qh_ws;
+    float* gam_ws;
 };
 
 // Gate slot of one chunk (floats).
@@ -145,7 +165,9 @@ inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t 
 
 }  // namespace tc
 
-// The state-independent part of every chunk into the workspace (chunk_wy.cu).
+// The state-independent part of every chunk into the workspace (chunk_wy.cu;
+// chunk_wy_kda.cu for the per-key gate).
 cudaError_t launch_chunk_wy(const ChunkArgs& a, const tc::TcMaps& m, cudaStream_t st);
+cudaError_t launch_chunk_wy_kda(const ChunkArgs& a, const tc::TcMaps& m, cudaStream_t st);
 
 }  // namespace dn

@@ -171,6 +171,78 @@ struct Args {
     int test_flags;
 };
 
+// T = (I + A)^-1 for the unit-lower 64 x 64 system of one chunk, in fp32 on
+// CUDA cores, by a group of 8 warps (named barrier `bar`, kNT threads).  Am
+// holds A (strictly lower; its blocks on and above the diagonal are never
+// read) and is overwritten by M; Tm receives T on and below the block
+// diagonal.  The 16 x 16 diagonal blocks D_k = (I + A_kk)^-1 come from forward
+// substitution, then M_kl = D_k A_kl and T_kl = -sum_{m=l}^{k-1} M_km T_ml in
+// three rounds (block forward substitution).  idle() is run by warps 6 and 7
+// while the others form M.  Ends with a group barrier.
+template <class Idle>
+__device__ __forceinline__ void wy_solve(float* Am, float* Tm, int warp, int lane, uint32_t bar, Idle idle) {
+    // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
+    if (warp < 4 && lane < 16) {
+        const int k0 = warp * 16, jj = lane;
+        float x[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+            float p0 = (ii == jj) ? 1.f : 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+            for (int m = 0; m + 3 < ii; m += 4) {
+                const float4 av = *reinterpret_cast<const float4*>(Am + fidx(k0 + ii, k0 + m));
+                p0 -= av.x * x[m]; p1 -= av.y * x[m + 1]; p2 -= av.z * x[m + 2]; p3 -= av.w * x[m + 3];
+            }
+#pragma unroll
+            for (int m = ii & ~3; m < ii; ++m) p0 -= Am[fidx(k0 + ii, k0 + m)] * x[m];
+            x[ii] = (p0 + p1) + (p2 + p3);
+        }
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
+    }
+    named_bar_sync(bar, kNT);
+    // ---- M_kl = D_k A_kl (k > l), in place of A_kl -------------------------------------
+    if (warp < 6) {
+        // (k, l) = (1,0) (2,0) (3,0) (2,1) (3,1) (3,2) for warps 0..5
+        const int k = (0x332321 >> (4 * warp)) & 15, l = (0x211000 >> (4 * warp)) & 15;
+        float acc[8];
+        zero8(acc);
+        blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
+        __syncwarp();
+        blk16_store(Am, 16 * k, 16 * l, acc, lane);
+    } else {
+        idle();                                       // warps 6 and 7 have nothing else to do
+    }
+    named_bar_sync(bar, kNT);
+    // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds; one block product per warp
+    //      and round, (k, m, l) from the tables below (4 bits each) ----------------------
+    {
+        // round 1, warps 0-5: T_10, T_21, T_32 complete; T_20, T_31, T_30 start (m = l)
+        // round 2, warps 3-5: T_20, T_31 complete (m = l + 1); T_30 continues (m = 1)
+        // round 3, warp 5:    T_30 completes (m = 2)
+        float acc[8];
+        zero8(acc);
+        if (warp < 6) {
+            const int k = (0x332321 >> (4 * warp)) & 15, l = (0x010210 >> (4 * warp)) & 15;
+            blk16(Am, 16 * k, 16 * l, Tm, 16 * l, 16 * l, acc, lane);
+            if (warp < 3) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
+        named_bar_sync(bar, kNT);
+        if (warp >= 3 && warp < 6) {
+            const int k = (0x332 >> (4 * (warp - 3))) & 15, m = (0x121 >> (4 * (warp - 3))) & 15;
+            const int l = (0x010 >> (4 * (warp - 3))) & 15;
+            blk16(Am, 16 * k, 16 * m, Tm, 16 * m, 16 * l, acc, lane);
+            if (warp < 5) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
+        }
+        named_bar_sync(bar, kNT);
+        if (warp == 5) {
+            blk16(Am, 48, 32, Tm, 32, 0, acc, lane);
+            blk16_store_neg(Tm, 48, 0, acc, lane);
+        }
+    }
+    named_bar_sync(bar, kNT);
+}
+
 // Thread kStoreTid of a group: raise the ready flag of the group's previous
 // tile, if one is pending, once its stores (issued by this thread) are
 // complete.  The proxy fence orders those async-proxy writes before the
@@ -326,66 +398,10 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     tc_fence_before();
     named_bar_sync(x.bar, kNT);
 
-    // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
-    if (warp < 4 && lane < 16) {
-        const int k0 = warp * 16, jj = lane;
-        float x[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-            float p0 = (ii == jj) ? 1.f : 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-            for (int m = 0; m + 3 < ii; m += 4) {
-                const float4 av = *reinterpret_cast<const float4*>(Am + fidx(k0 + ii, k0 + m));
-                p0 -= av.x * x[m]; p1 -= av.y * x[m + 1]; p2 -= av.z * x[m + 2]; p3 -= av.w * x[m + 3];
-            }
-#pragma unroll
-            for (int m = ii & ~3; m < ii; ++m) p0 -= Am[fidx(k0 + ii, k0 + m)] * x[m];
-            x[ii] = (p0 + p1) + (p2 + p3);
-        }
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
-    }
-    named_bar_sync(x.bar, kNT);
-    // ---- M_kl = D_k A_kl (k > l), in place of A_kl -------------------------------------
-    if (warp < 6) {
-        // (k, l) = (1,0) (2,0) (3,0) (2,1) (3,1) (3,2) for warps 0..5
-        const int k = (0x332321 >> (4 * warp)) & 15, l = (0x211000 >> (4 * warp)) & 15;
-        float acc[8];
-        zero8(acc);
-        blk16(Tm, 16 * k, 16 * k, Am, 16 * k, 16 * l, acc, lane);
-        __syncwarp();
-        blk16_store(Am, 16 * k, 16 * l, acc, lane);
-    } else if (tid == kStoreTid) {
-        publish_pending(ar, pending);                 // the previous tile's ready flag
-    }
-    named_bar_sync(x.bar, kNT);
-    // ---- T_kl = -sum_{m=l}^{k-1} M_km T_ml, three rounds; one block product per warp
-    //      and round, (k, m, l) from the tables below (4 bits each) ----------------------
-    {
-        // round 1, warps 0-5: T_10, T_21, T_32 complete; T_20, T_31, T_30 start (m = l)
-        // round 2, warps 3-5: T_20, T_31 complete (m = l + 1); T_30 continues (m = 1)
-        // round 3, warp 5:    T_30 completes (m = 2)
-        float acc[8];
-        zero8(acc);
-        if (warp < 6) {
-            const int k = (0x332321 >> (4 * warp)) & 15, l = (0x010210 >> (4 * warp)) & 15;
-            blk16(Am, 16 * k, 16 * l, Tm, 16 * l, 16 * l, acc, lane);
-            if (warp < 3) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
-        }
-        named_bar_sync(x.bar, kNT);
-        if (warp >= 3 && warp < 6) {
-            const int k = (0x332 >> (4 * (warp - 3))) & 15, m = (0x121 >> (4 * (warp - 3))) & 15;
-            const int l = (0x010 >> (4 * (warp - 3))) & 15;
-            blk16(Am, 16 * k, 16 * m, Tm, 16 * m, 16 * l, acc, lane);
-            if (warp < 5) blk16_store_neg(Tm, 16 * k, 16 * l, acc, lane);
-        }
-        named_bar_sync(x.bar, kNT);
-        if (warp == 5) {
-            blk16(Am, 48, 32, Tm, 32, 0, acc, lane);
-            blk16_store_neg(Tm, 48, 0, acc, lane);
-        }
-    }
-    named_bar_sync(x.bar, kNT);
+    // ---- T = (I + A)^-1; warp 6 raises the previous tile's ready flag meanwhile --------
+    wy_solve(Am, Tm, warp, lane, x.bar, [&] {
+        if (tid == kStoreTid) publish_pending(ar, pending);
+    });
     // ---- T diag(beta e^G) and T diag(beta) as bf16 operand tiles, over A (zero above
     //      the block diagonal, where T was never written) ----------------------------------
 #pragma unroll

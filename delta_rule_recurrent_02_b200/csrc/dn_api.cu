@@ -84,7 +84,7 @@ int plan_chunk(int B, int T, int H, int d_k, int d_v, int chunk, dn_dtype dtype,
     *use_tc = false;
     if (path == DN_PATH_TC || path == DN_PATH_TC_STALL_TEST) {
         if (!dn::tc_supports(*a))
-            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64, d_k = d_v = 128 and no per-key gate");
+            return fail(DN_ERR_UNSUPPORTED, "tensor-core path needs bf16, chunk 64 and d_k = d_v = 128");
         *use_tc = true;
     } else if (path == DN_PATH_AUTO) {
         *use_tc = dn::tc_supports(*a);
@@ -108,7 +108,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 1; }
+int dn_version(void) { return (2 << 16) | 2; }
 
 unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 

@@ -37,7 +37,7 @@ cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t st);
 
 // Tensor-core (tcgen05) chunk path: the per-chunk UT/WY transform (chunk_wy.cu)
 // then the state pass (chunk_tc.cu).  tc_supports() says whether the request
-// is inside its coverage (bf16, chunk 64, d_k = d_v = 128, no per-key gate);
+// is inside its coverage (bf16, chunk 64, d_k = d_v = 128, any gate);
 // tc_workspace_bytes() is the size of a.ws it needs (W^T and u^T of every chunk).
 bool tc_supports(const ChunkArgs& a);
 size_t tc_workspace_bytes(const ChunkArgs& a);

@@ -78,7 +78,7 @@ typedef enum {
 typedef enum {
     DN_PATH_AUTO = 0,     /* tensor-core path when it supports the request, else SIMT */
     DN_PATH_SIMT = 1,     /* fp32 CUDA-core chunk kernel: any chunk 1..64          */
-    DN_PATH_TC = 2,       /* tcgen05 chunk kernels: bf16, chunk 64, d_k = d_v = 128, no per-key gate */
+    DN_PATH_TC = 2,       /* tcgen05 chunk kernels: bf16, chunk 64, d_k = d_v = 128, any gate */
     /* Self-test of the failure path: the tensor-core kernels run with their input
      * loads withheld, so every bounded wait inside them expires (about two seconds);
      * nothing is written to o or S_T, dn_device_status() then returns
@@ -123,8 +123,15 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
  * 12.5; "The chunked form", ch. 28) in a kernel that runs over all chunks at
  * once, then streams them into the sequential state pass: 40 KiB and a 4-byte
  * ready flag per (b, h, chunk), i.e. with n = B * H * ceil(T / 64) chunks,
- * n * 40960 + (4 n rounded up to a multiple of 256) bytes.  Sizes are checked
- * as in dn_chunk_fwd_ex; *bytes is written on DN_OK only.
+ * n * 40960 + (4 n rounded up to a multiple of 256) bytes.  With the per-key
+ * gate (KDA: "A walk through of the DeltaNet family of linear attention
+ * variants") each chunk also keeps q and k with their decays applied and the
+ * chunk's decay per key channel: 72.5 KiB per chunk, n * 74240 + (4 n rounded
+ * up to a multiple of 256) bytes.  Its gram splits the decays around one
+ * reference position per 16-token block, so the tensor-core result is exact up
+ * to rounding while no key channel decays by more than e^-80 over 8
+ * consecutive tokens (the SIMT path has no such bound).  Sizes are checked as
+ * in dn_chunk_fwd_ex; *bytes is written on DN_OK only.
  */
 DN_API int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk,
                                        dn_dtype dtype, dn_gate gate, dn_path path, size_t* bytes);
@@ -209,7 +216,7 @@ DN_API const char* dn_status_str(int status);
 /* Reason for the last non-DN_OK return on the calling thread ("" if none). */
 DN_API const char* dn_last_error(void);
 
-/* ABI version, (major << 16) | minor. */
+/* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path. */
 DN_API int dn_version(void);
 
 /*

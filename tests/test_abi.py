@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dn_version() >> 16 == 2
+    assert lib.dn_version() >> 16 == 2 and lib.dn_version() & 0xffff >= 2
     for code in range(5):
         assert lib.dn_status_str(code).startswith(b"DN_")
     assert lib.dn_status_str(99) == b"unknown dn_status"
@@ -109,10 +109,13 @@ def test_workspace_size():
     tiles = 2 * 3 * 3
     assert ws_size(lib) == (dn.DN_OK, tiles * (2 * 64 * 128 + 64 * 64) * 2 + 256)
     assert ws_size(lib, path=2) == (dn.DN_OK, tiles * 40960 + 256)
+    # per-key gate: also K~ and Qh (bf16, 64 x 128 each) and e^Gamma_last (fp32, 128) per chunk
+    assert ws_size(lib, gate=2, path=2) == (dn.DN_OK, tiles * (40960 + 2 * 16384 + 512) + 256)
+    assert ws_size(lib, gate=2, path=1) == (dn.DN_OK, 0)
     assert ws_size(lib, T=0) == (dn.DN_OK, 0)
     assert ws_size(lib, path=1) == (dn.DN_OK, 0)             # SIMT needs none
     assert ws_size(lib, dtype=0) == (dn.DN_OK, 0)            # fp32 runs on SIMT under auto
-    assert ws_size(lib, gate=2) == (dn.DN_OK, 0)             # so does the per-key gate
+    assert ws_size(lib, gate=2) == ws_size(lib, gate=2, path=2)   # the per-key gate runs on tensor cores
     assert ws_size(lib, dtype=0, path=2)[0] == dn.DN_ERR_UNSUPPORTED
     assert ws_size(lib, B=-1) == (dn.DN_ERR_INVALID, 12345)  # not written on failure
     assert lib.dn_chunk_fwd_workspace_size(1, 8, 1, 128, 128, 64, 1, 1, 0, None) == dn.DN_ERR_INVALID

@@ -14,13 +14,13 @@ from _util import TOL, assert_close, f64, oracle_prefill, pick, to_dev
 pytestmark = pytest.mark.gpu
 
 PATHS = ["simt", "tc"]
-# the tensor-core path covers bf16, chunk 64, d_k = d_v = 128 and the none / scalar gates
-TC_GATES = ("none", "scalar")
+# the tensor-core path covers bf16, chunk 64, d_k = d_v = 128 and every gate
+TC_GATES = ("none", "scalar", "per_key")
 
 
 def skip_unsupported(path, gate):
     if path == "tc" and gate not in TC_GATES:
-        pytest.skip("per-key gate runs on the SIMT path")
+        pytest.skip(f"{gate} gate runs on the SIMT path")
 
 
 def run(d, scale, chunk=64, path="simt", gate=None):
@@ -192,8 +192,11 @@ def test_tc_many_heads(cuda_device, B, H, T):
     (4, 32, 130, "tc", 2),       # too many heads for one launch: WY kernel, then state pass
     (2, 3, 200, "simt", 1),
 ])
-def test_chunk_kernel_launch_count(cuda_device, B, H, T, path, kernels):
-    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate="scalar", seed=5, s0_std=0.2)
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_chunk_kernel_launch_count(cuda_device, B, H, T, path, kernels, gate):
+    if gate == "per_key" and path == "tc":
+        kernels = 2              # per-key gate: its WY kernel, then the state pass
+    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate=gate, seed=5, s0_std=0.2)
     d = to_dev(inp)
     torch.cuda.synchronize()
     before = dn.dn_kernel_launches()
@@ -268,5 +271,33 @@ def test_gated_deltanet_long_sampled(cuda_device, path):
     _sampled(W.GDN_LONG, path, n_heads=4, seed=1)
 
 
-def test_kda_sampled(cuda_device):
-    _sampled(W.KDA_PREFILL, "auto", n_heads=8, seed=2)
+@pytest.mark.parametrize("path", PATHS)
+def test_kda_sampled(cuda_device, path):
+    _sampled(W.KDA_PREFILL, path, n_heads=8, seed=2)
+
+
+@pytest.mark.parametrize("g_shift", [-1.0, 8.0])
+def test_kda_tc_weak_and_strong_decay(cuda_device, g_shift):
+    # per-key gate on tensor cores: g = -softplus(N(0,1) + shift) per channel; shift 8
+    # decays each channel by about e^-64 over 8 tokens, near the e^-80 bound of the
+    # gram's split around each 16-token block's middle; shift -1 barely decays
+    inp = W.gen_prefill(2, 3, 200, 128, 128, dtype="bf16", gate="per_key", seed=31, s0_std=0.2,
+                        g_shift=g_shift)
+    sc = 128 ** -0.5
+    o, S = run(to_dev(inp), sc, path="tc")
+    dn.dn_device_status()
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(S, rS, "bf16", "S_T")
+
+
+def test_kda_tc_matches_simt_path(cuda_device):
+    # the two kernels share no code: the tensor-core and fp32 paths agree to bf16 rounding
+    inp = W.gen_prefill(1, 4, 333, 128, 128, dtype="bf16", gate="per_key", seed=7, s0_std=0.3, g_shift=3.0)
+    sc = 128 ** -0.5
+    d = to_dev(inp)
+    o1, S1 = run(d, sc, path="tc")
+    o2, S2 = run(d, sc, path="simt")
+    dn.dn_device_status()
+    assert_close(o1, f64(o2), "bf16", "o (tc vs simt)")
+    assert_close(S1, f64(S2), "bf16", "S_T (tc vs simt)")
