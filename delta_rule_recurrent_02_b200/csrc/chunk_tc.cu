@@ -13,8 +13,13 @@
 //     buffer).  Used while B H leaves a quarter of the SMs to the WY groups.
 //   * otherwise two launches on the stream: chunk_wy_kernel over all tiles,
 //     then chunk_state_kernel (whose flags are then all set).
+// The per-key gate (KDA) works the same way with its own WY tile
+// (chunk_wy_kda.cuh, 88 KiB): chunk_fused_kda_kernel has CTAs of 16 warps, the
+// state pass of one head or two KDA WY groups; else chunk_wy_kda_kernel and
+// chunk_state_kernel<per-key>.
 #include "chunk_state.cuh"
 #include "chunk_wy.cuh"
+#include "chunk_wy_kda.cuh"
 #include "dn_kernels.h"
 
 namespace dn {
@@ -148,6 +153,68 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 // ---- host side ---------------------------------------------------------------
 
+constexpr int kFusedKdaThreads = 2 * kda::kNT;     // 16 warps: two KDA WY groups, or the state pass
+static_assert(state::kNT == kFusedKdaThreads, "fused KDA CTA size");
+constexpr uint32_t kFusedKdaBytes =
+    (state::Layout<false>::STATE_BYTES > 2 * kda::GROUP_BYTES ? state::Layout<false>::STATE_BYTES
+                                                               : 2 * kda::GROUP_BYTES) + 1024;
+
+// The per-key-gate prefill in one cooperative launch: CTAs 0 .. BH - 1 run the
+// state pass of one head each (reading Qh, K~ and the decays from the
+// workspace); the others run two KDA WY groups over the tiles, chunk-major.
+__global__ void __launch_bounds__(kFusedKdaThreads, 1)
+chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                       const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_p,
+                       const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_qh,
+                       __nv_bfloat16* p_out, __nv_bfloat16* kt_out, __nv_bfloat16* qh_out, float* gam,
+                       unsigned int* flags, int BH, const float* __restrict__ beta, const float* __restrict__ g,
+                       const float* S0, __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale,
+                       unsigned int* status, int test_flags) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    if ((int)blockIdx.x < BH) {
+        const state::Args ar{&tm_kt, &tm_qh, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
+                             test_flags, gam};
+        state::state_pass<kGatePerKey, false>(sm, ar, blockIdx.x, 0u);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int grp = warp >> 3;                       // 0, 1
+    const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(sm + 2 * kda::GROUP_BYTES - 16);
+    kda::Group x = kda::make_group(sm + grp * kda::GROUP_BYTES, 0u, 1u + (uint32_t)grp, tid - grp * kda::kNT);
+    if (x.tid == 0) {
+        kda::init_group(x);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), 2 * kda::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    x.tmem = *tmem_slot + (uint32_t)grp * kda::TM_COLS;
+    const kda::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam, flags, beta, g,
+                       T, n, scale, test_flags};
+    const int64_t tiles = (int64_t)BH * n;
+    const int64_t G = (int64_t)(gridDim.x - BH) * 2;      // WY groups in the grid
+    bool ok = true;
+    int64_t pending = -1;
+    for (int64_t t = (int64_t)(blockIdx.x - BH) * 2 + grp; ok && t < tiles; t += G) {
+        const int c = (int)(t / BH);
+        ok = kda::kda_tile(x, wa, c, t - (int64_t)c * BH, pending);
+    }
+    if (ok && x.tid == kda::kStoreTid) kda::publish_pending(wa, pending);
+    tc_fence_before();
+    __syncthreads();
+    if (!ok && x.tid == 0) atomicOr(status, 1u);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(*tmem_slot, 2 * kda::TM_COLS);
+    }
+}
+
 namespace {
 
 // The single-launch prefill needs one resident CTA per SM and leaves at least
@@ -244,7 +311,45 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     m.qh_ws = reinterpret_cast<__nv_bfloat16*>(qh_ws);
     m.gam_ws = reinterpret_cast<float*>(gam_ws);
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles, true));
-    cudaError_t e = launch_chunk_wy_kda(a, m, st);
+
+    int dev = 0, num_sms = 0, coop = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t BH = a.B * a.H;
+    if (coop && fused_fits(BH, num_sms)) {
+        auto kern = chunk_fused_kda_kernel;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedKdaBytes);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedKdaThreads, kFusedKdaBytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm >= 1) {
+            int bh_i = (int)BH, T_i = (int)a.T, n_i = n;
+            float scale = a.scale;
+            int test_flags = a.test_flags;
+            __nv_bfloat16* p_out = m.p_ws;
+            __nv_bfloat16* kt_out = m.kt_ws;
+            __nv_bfloat16* qh_out = m.qh_ws;
+            float* gam = m.gam_ws;
+            unsigned int* flags = m.flags;
+            const float* beta = a.beta;
+            const float* g = a.g;
+            const float* S0 = a.S0;
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+            float* S_T = a.S_T;
+            unsigned int* status = a.status;
+            void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &m.kt, &m.qh, &p_out, &kt_out, &qh_out, &gam,
+                            &flags, &bh_i, &beta, &g, &S0, &o, &S_T, &T_i, &n_i, &scale, &status, &test_flags};
+            // the flags are cleared on the same stream right before the launch
+            e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
+            if (e != cudaSuccess) return e;
+            return counted(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
+                                                       dim3(kFusedKdaThreads), args, kFusedKdaBytes, st));
+        }
+    }
+    e = launch_chunk_wy_kda(a, m, st);
     if (e != cudaSuccess) return e;
     auto kern = chunk_state_kernel<kGatePerKey>;
     const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;

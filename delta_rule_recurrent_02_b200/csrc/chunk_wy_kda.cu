@@ -1,445 +1,67 @@
-// chunk_wy_kda.cu -- the state-independent part of one chunk for the per-key
-// gate (KDA: "A walk through of the DeltaNet family of linear attention
-// variants", its KDA update: each key channel forgets at its own rate), on
-// tensor cores.  One CTA of 8 warps per (b, h, chunk), two CTAs per SM.
-//
-// Chunk algebra ("Linear attention and Gated DeltaNet", ch. 28, "The chunked
-// form", with the decay promoted to one value per key channel).  With Gamma_i
-// the inclusive prefix sum of g over the chunk, per channel:
-//
-//   A_ij = beta_i sum_d k_id k_jd e^(Gamma_id - Gamma_jd)          (j < i)
-//   P_ij = scale  sum_d q_id k_jd e^(Gamma_id - Gamma_jd)          (j <= i)
-//   T = (I + A)^-1,  W = T diag(beta) (K (.) e^Gamma),  u = T diag(beta) V
-//
-// and the state pass needs Qh = scale Q (.) e^Gamma, K~ = K (.) e^(Gamma_last -
-// Gamma) and gam = e^Gamma_last.
-//
-// The decays cannot leave the sum over d as row and column factors of one
-// product: Gamma falls by about 3 per position and channel, and e^-Gamma_j
-// overflows long before the end of a chunk.  So the gram is split by the
-// 16-row block I of i, and block I uses its own reference position
-// m_I = 16 I + 8:
-//
-//   e^(Gamma_i - Gamma_j) = e^(Gamma_i - Gamma_mI) e^(Gamma_mI - Gamma_j)
-//
-// For j < 16 I both factors are at most e^(decay over 8 positions); inside
-// the block likewise.  Block I is one tcgen05 product of [K^;Q^] (rows scaled
-// by e^(Gamma_i - Gamma_m(i))) with the first 16 (I + 1) rows of K scaled by
-// e^(Gamma_mI - Gamma_j): four products of N = 16, 32, 48, 64 into TMEM, of
-// which row i reads its own block's.  The exponent is capped at 80 (e^80 is
-// far inside bf16 and fp32): the results are exact up to rounding while no
-// channel decays by more than e^-80 over 8 consecutive positions.
-//
-// Steps, one 64-channel d-block at a time for the gram:
-//   TMA       K and Q, stacked per d-block as [K rows | Q rows]
-//   CUDA core g -> Gamma (log2 units) by a prefix sum over positions
-//   CUDA core scaled operands: [K^;Q^] in place, the four B tiles, K (.) e^Gamma
-//             for W; Qh, K~ and gam straight to the workspace
-//   tcgen05   D_I += [K^;Q^] B_I^T  (I = 0..3)
-// then, as for the scalar gate (chunk_wy.cuh):
-//   CUDA core A and P from the D_I; T = (I + A)^-1; T diag(beta) as bf16
-//   TMA       V over the dead K/Q tiles
-//   tcgen05   W^T = (K (.) e^Gamma)^T (T diag(beta))^T, u^T = V^T (T diag(beta))^T
-//   epilogue  -W and u^T by TMA stores, as for the scalar gate
-//
-// Every wait is bounded; on a timeout the CTA sets the status word and stops.
-#include "chunk_wy.cuh"
+// chunk_wy_kda.cu -- the state-independent part of every chunk with the
+// per-key gate (see chunk_wy_kda.cuh), one CTA per (b, h, chunk), two CTAs per
+// SM.  Used when the prefill runs as two launches (chunk_tc.cu).
+#include "chunk_wy_kda.cuh"
 #include "dn_kernels.h"
 
 namespace dn {
-namespace kda {
 
 using namespace sm100;
 using namespace tc;
-using wy::fidx;
-using wy::kNT;
 
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [K0 | Q0 | K1 | Q1] -> [K^0 | Q^0 | K^1 | Q^1]; then V = [V0 | V1];
-                                        // last, the -W and u^T output tiles
-constexpr uint32_t OFF_KW = 32768;      // K (.) e^Gamma = [Kw0 | Kw1] (the A operand of W^T)
-constexpr uint32_t OFF_G = 49152;       // Gamma log2(e) of the current d-block, fp32 [64][68];
-                                        // after the gram A (fp32 64 x 68), then T diag(beta) (bf16)
-constexpr uint32_t OFF_T = OFF_G + 64 * 68 * 4;   // T (fp32 64 x 68), after the gram
-constexpr uint32_t OFF_B = 67584;       // the current d-block's B tiles: K rows 0 .. 16 (I + 1) - 1
-                                        // scaled by e^(Gamma_mI - Gamma_j), I = 0..3
-constexpr uint32_t OFF_GATE = OFF_B + 20480;      // beta [64], then the prefix-sum segment totals [4][64]
-constexpr uint32_t OFF_BAR = OFF_GATE + 256 + 1024;
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
-static_assert(OFF_T + 64 * 68 * 4 <= OFF_GATE, "T stays inside the dead B tiles");
-static_assert(OFF_G + 64 * 68 * 4 <= OFF_B && OFF_B % 1024 == 0, "layout");
-static_assert(2 * SMEM_BYTES <= 232448, "two CTAs per SM");
-
-// B tile I: 16 (I + 1) rows of 128 bytes (64 channels), 128-byte swizzle
-__host__ __device__ constexpr uint32_t b_off(int I) { return 1024u * (uint32_t)(I * (I + 1)); }
-// TMEM: D_I at column d_col(I), 16 (I + 1) wide; W^T and u^T at 0 and 64 after the gram
-__host__ __device__ constexpr uint32_t d_col(int I) { return 8u * (uint32_t)(I * (I + 1)); }
-constexpr uint32_t TM_W = 0, TM_U = 64;
-constexpr uint32_t TM_COLS = 256;
-static_assert(b_off(3) + 8192 == 20480 && d_col(3) + 64 <= TM_COLS, "B tiles and D columns");
-
-constexpr float kCap2 = 80.f * 1.4426950408889634f;   // exponent cap, log2 units
-
-enum { B_FULL = 0, B_MMA = 1 };
-
-__device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    const float4 b = *reinterpret_cast<const float4*>(p + 4);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-
-__device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h[e]);
-        x[2 * e] = f.x;
-        x[2 * e + 1] = f.y;
-    }
-}
-
-// x (.) f as 8 bf16 (one 16-byte chunk)
-__device__ __forceinline__ uint4 scaled8(const float (&x)[8], const float (&f)[8]) {
-    return make_uint4(pack_bf16x2(x[0] * f[0], x[1] * f[1]), pack_bf16x2(x[2] * f[2], x[3] * f[3]),
-                      pack_bf16x2(x[4] * f[4], x[5] * f[5]), pack_bf16x2(x[6] * f[6], x[7] * f[7]));
-}
-
-__device__ __forceinline__ void st_shared_u4(uint32_t a, const uint4& v) { st_shared_v4(a, v.x, v.y, v.z, v.w); }
-
-__global__ void __launch_bounds__(kNT, 2)
+__global__ void __launch_bounds__(kda::kNT, 2)
 chunk_wy_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_u, __nv_bfloat16* __restrict__ p_out,
                     __nv_bfloat16* __restrict__ kt_out, __nv_bfloat16* __restrict__ qh_out,
-                    float* __restrict__ gam_out, int BH, const float* __restrict__ beta,
-                    const float* __restrict__ g, int T, int n, float scale, unsigned int* status, int test_flags) {
+                    float* __restrict__ gam_out, unsigned int* __restrict__ flags, int BH,
+                    const float* __restrict__ beta, const float* __restrict__ g, int T, int n, float scale,
+                    unsigned int* status, int test_flags) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const uint32_t sb = smem_u32(sm);
-    float* bs = reinterpret_cast<float*>(sm + OFF_GATE);              // beta of the chunk
-    float* segt = reinterpret_cast<float*>(sm + OFF_GATE + 256);      // prefix-sum segment totals
-    float* Gm = reinterpret_cast<float*>(sm + OFF_G);                 // Gamma log2(e), [64][68]
-    float* Am = reinterpret_cast<float*>(sm + OFF_G);
-    float* Tm = reinterpret_cast<float*>(sm + OFF_T);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_BAR + 20);
-    const Ctl ctl{sb + OFF_BAR, abort_flag};
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr uint32_t kBar = 1;
-
-    // chunk-major order: chunk 0 of every head first
-    const int c = (int)(blockIdx.x / (unsigned)BH);
-    const int64_t bh = blockIdx.x - (int64_t)c * BH;
-    const int64_t tile = bh * n + c;
-    const int Cc = min(kC, T - c * kC);
-    const int64_t t0 = bh * T + (int64_t)c * kC;
-    const bool load = !(test_flags & 1);
-    int loads = 0;                                   // load phases issued (thread 0)
-
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kda::GROUP_BYTES - 16);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    kda::Group x = kda::make_group(sm, 0u, 1u, tid);
     if (tid == 0) {
-        mbar_init(ctl.bar(B_FULL), 1);
-        mbar_init(ctl.bar(B_MMA), 1);
-        *abort_flag = 0;
+        kda::init_group(x);
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), TM_COLS);
+        tmem_alloc(smem_u32(tmem_slot), kda::TM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    bool ok = true;
-
-    if (tid == 0 && load) {
-        const uint32_t fb = ctl.bar(B_FULL);
-        mbar_arrive_expect_tx(fb, 4 * 8192);
-        tma_load_2d(sb + OFF_KQ + 0, &tm_k, 0, (int)t0, fb);
-        tma_load_2d(sb + OFF_KQ + 16384, &tm_k, 64, (int)t0, fb);
-        tma_load_2d(sb + OFF_KQ + 8192, &tm_q, 0, (int)t0, fb);
-        tma_load_2d(sb + OFF_KQ + 24576, &tm_q, 64, (int)t0, fb);
-        loads = 1;
-    }
-    if (warp == 0) {
-        bs[lane] = lane < Cc ? beta[t0 + lane] : 0.f;
-        bs[lane + 32] = lane + 32 < Cc ? beta[t0 + lane + 32] : 0.f;
-    }
-
-    for (int b = 0; b < 2; ++b) {
-        // ---- Gamma of channels 64 b .. 64 b + 63: thread (segment of 16 positions, channel)
-        {
-            const int ch = tid & 63, seg = tid >> 6;
-            float acc[16];
-            float run = 0.f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int i = 16 * seg + r;
-                run += i < Cc ? g[(t0 + i) * kD + 64 * b + ch] : 0.f;   // zero past the end: identity steps
-                acc[r] = run;
-            }
-            segt[seg * 64 + ch] = run;
-            named_bar_sync(kBar, kNT);
-            float off = 0.f;
-            for (int s2 = 0; s2 < seg; ++s2) off += segt[s2 * 64 + ch];
-            const float L2E = 1.4426950408889634f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Gm[fidx(16 * seg + r, ch)] = (acc[r] + off) * L2E;
-        }
-        // the K/Q tiles have landed (first d-block); the previous d-block's products
-        // have read the B tiles (second)
-        ok = b == 0 ? ctl.wait(B_FULL, 0) : ctl.wait(B_MMA, 0);
-        if (named_bar_any(kBar, kNT, !ok)) goto done;
-        tc_fence_after();
-
-        // ---- scaled operands: (row i, 8-channel chunk gq) per item, two per thread ------
-#pragma unroll 1
-        for (int u = 0; u < 2; ++u) {
-            const int x = tid + u * kNT;
-            const int i = x >> 3, gq = x & 7, blk = i >> 4;
-            float gi[8], gm[8], gc[8], kv[8], qv[8], f[8];
-            load8(Gm + fidx(i, 8 * gq), gi);
-            load8(Gm + fidx(16 * blk + 8, 8 * gq), gm);
-            load8(Gm + fidx(63, 8 * gq), gc);
-            const uint32_t ka = sb + OFF_KQ + b * 16384 + sw128_off(i, gq);
-            unpack8(ld_shared_v4(ka), kv);
-            unpack8(ld_shared_v4(ka + 8192), qv);
-            const int64_t grow = (tile * kC + i) * kD + 64 * b + 8 * gq;   // workspace element
-            // K (.) e^Gamma for W, and Qh = scale Q (.) e^Gamma
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(gi[e]);
-            st_shared_u4(sb + OFF_KW + b * 8192 + sw128_off(i, gq), scaled8(kv, f));
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= scale;
-            const uint4 qh = scaled8(qv, f);
-            st_global_v4(qh_out + grow, qh.x, qh.y, qh.z, qh.w);
-            // K~ = K (.) e^(Gamma_last - Gamma)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(gc[e] - gi[e]);
-            const uint4 kt = scaled8(kv, f);
-            st_global_v4(kt_out + grow, kt.x, kt.y, kt.z, kt.w);
-            if (i == 63) {
-                float4* gp = reinterpret_cast<float4*>(gam_out + tile * kD + 64 * b + 8 * gq);
-                gp[0] = make_float4(ex2_approx(gc[0]), ex2_approx(gc[1]), ex2_approx(gc[2]), ex2_approx(gc[3]));
-                gp[1] = make_float4(ex2_approx(gc[4]), ex2_approx(gc[5]), ex2_approx(gc[6]), ex2_approx(gc[7]));
-            }
-            // B tiles of the blocks I >= blk: K (.) e^(Gamma_mI - Gamma)
-#pragma unroll 1
-            for (int I = blk; I < 4; ++I) {
-                float gr[8];
-                load8(Gm + fidx(16 * I + 8, 8 * gq), gr);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = ex2_approx(fminf(gr[e] - gi[e], kCap2));
-                st_shared_u4(sb + OFF_B + b_off(I) + sw128_off(i, gq), scaled8(kv, f));
-            }
-            // [K^;Q^] in place: rows scaled by e^(Gamma_i - Gamma_m(i))
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(fminf(gi[e] - gm[e], kCap2));
-            st_shared_u4(ka, scaled8(kv, f));
-            st_shared_u4(ka + 8192, scaled8(qv, f));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        named_bar_sync(kBar, kNT);
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int I = 0; I < 4; ++I) {
-                const uint32_t idesc = idesc_bf16(128, 16 * (I + 1), 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + d_col(I), sw128_desc(sb + OFF_KQ + b * 16384 + kk * 32, 16, 1024),
-                             sw128_desc(sb + OFF_B + b_off(I) + kk * 32, 16, 1024), idesc, (b | kk) > 0);
-            }
-            mma_commit(ctl.bar(B_MMA));
-        }
-    }
-    ok = ctl.wait(B_MMA, 1);
-    if (named_bar_any(kBar, kNT, !ok)) goto done;
-    tc_fence_after();
-    if (tid == 0 && load) {
-        // V over the K/Q tiles, which the gram has read
-        const uint32_t fb = ctl.bar(B_FULL);
-        mbar_arrive_expect_tx(fb, 2 * 8192);
-        tma_load_2d(sb + OFF_KQ + 0, &tm_v, 0, (int)t0, fb);
-        tma_load_2d(sb + OFF_KQ + 8192, &tm_v, 64, (int)t0, fb);
-        loads = 2;
-    }
-
-    // ---- A (lanes 0-63) and P (lanes 64-127) from the D_I: row i reads D of its own
-    //      block; warps 0-3 take columns 0-31, warps 4-7 columns 32-63 ------------------
-    {
-        const int q = warp & 3, h = warp >> 2;
-        const int i = ((q & 1) << 5) + lane;          // row within A or P
-        const int blo = (q & 1) * 2;                  // blocks of the warp's lanes: blo, blo + 1
-        const uint32_t lane_base = tmem + ((uint32_t)(q << 5) << 16);
-        const int j0 = 32 * h;
-        if (q < 2) {
-            if (!(q == 0 && h == 1)) {                // rows 0-31 x columns 32-63: above the diagonal
-                float vlo[32], vhi[32];
-                tmem_ld32(lane_base + d_col(blo) + j0, vlo);
-                tmem_ld32(lane_base + d_col(blo + 1) + j0, vhi);
-                tmem_wait_ld();
-                const float bi = bs[i];
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    float a[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = j0 + 4 * q4 + e;
-                        const float v = lane < 16 ? vlo[4 * q4 + e] : vhi[4 * q4 + e];
-                        a[e] = j < i ? bi * v : 0.f;
-                    }
-                    *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
-                }
-            }
-        } else {
-            __nv_bfloat16* prow = p_out + (tile * kC + i) * kC + j0;
-            if (q == 2 && h == 1) {
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) st_global_v4(prow + 8 * q4, 0u, 0u, 0u, 0u);
-            } else {
-                float vlo[32], vhi[32];
-                tmem_ld32(lane_base + d_col(blo) + j0, vlo);
-                tmem_ld32(lane_base + d_col(blo + 1) + j0, vhi);
-                tmem_wait_ld();
-                const float si = i < Cc ? scale : 0.f;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float pv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = j0 + 8 * q4 + e;
-                        const float v = lane < 16 ? vlo[8 * q4 + e] : vhi[8 * q4 + e];
-                        pv[e] = j <= i ? si * v : 0.f;
-                    }
-                    st_global_v4(prow + 8 * q4, pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
-                                 pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    named_bar_sync(kBar, kNT);
-
-    // ---- T = (I + A)^-1 -------------------------------------------------------------
-    wy::wy_solve(Am, Tm, warp, lane, kBar, [] {});
-
-    // ---- T diag(beta) as a bf16 operand tile over A (zero above the block diagonal) ---
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int x = tid + u * kNT;
-        const int i = x >> 3, ch = x & 7;
-        uint32_t b4[4] = {0u, 0u, 0u, 0u};
-        if ((ch >> 1) <= (i >> 4)) {
-            const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
-            const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
-            const float4 c0 = *reinterpret_cast<const float4*>(bs + 8 * ch);
-            const float4 c1 = *reinterpret_cast<const float4*>(bs + 8 * ch + 4);
-            b4[0] = pack_bf16x2(t0v.x * c0.x, t0v.y * c0.y); b4[1] = pack_bf16x2(t0v.z * c0.z, t0v.w * c0.w);
-            b4[2] = pack_bf16x2(t1v.x * c1.x, t1v.y * c1.y); b4[3] = pack_bf16x2(t1v.z * c1.z, t1v.w * c1.w);
-        }
-        st_shared_v4(sb + OFF_G + sw128_off(i, ch), b4[0], b4[1], b4[2], b4[3]);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    named_bar_sync(kBar, kNT);
-
-    // ---- W^T = Kw^T Tb^T, u^T = V^T Tb^T ----------------------------------------------
-    if (tid == 0) {
-        ok = ctl.wait(B_FULL, 1);
-        if (ok) {
-            tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, 64, 1, 0);    // A MN-major, B K-major
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_W, sw128_desc(sb + OFF_KW + kk * 2048, 8192, 1024),
-                         sw128_desc(sb + OFF_G + kk * 32, 16, 1024), idesc, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tmem + TM_U, sw128_desc(sb + OFF_KQ + kk * 2048, 8192, 1024),
-                         sw128_desc(sb + OFF_G + kk * 32, 16, 1024), idesc, kk > 0);
-            mma_commit(ctl.bar(B_MMA));
-        }
-    }
-    // third completion of B_MMA: parity 0 again (every thread has passed the first)
-    ok = ok && ctl.wait(B_MMA, 0);
-    if (named_bar_any(kBar, kNT, !ok)) goto done;
-    tc_fence_after();
-
-    // ---- -W row-major [64][128] (warps 0-3) and u^T [128][64] (warps 4-7) over V ------
-    if (warp < 4) {
-        const int r = (warp << 5) + lane;              // d_k channel
-        const uint32_t base = sb + OFF_KQ + (uint32_t)(r >> 6) * 8192 + (uint32_t)(r & 7) * 2;
-        const int ch = (r & 63) >> 3;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp << 5) << 16) + TM_W + hh * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = hh * 32 + e;
-                st_shared_b16(base + (uint32_t)(i * 128 + ((ch ^ (i & 7)) << 4)), __float2bfloat16_rn(-v[e]));
-            }
-        }
-    } else {
-        const int q = warp & 3;
-        const int r = (q << 5) + lane;
-        const uint32_t dst = sb + OFF_KQ + 16384;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_U + hh * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                st_shared_v4(dst + sw128_off(r, hh * 4 + q4), pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
-                             pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]), pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
-                             pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
-        }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    named_bar_sync(kBar, kNT);
-    if (tid == 0) {
-        tma_store_2d(&tm_w, 0, (int)(tile * kC), sb + OFF_KQ);
-        tma_store_2d(&tm_w, 64, (int)(tile * kC), sb + OFF_KQ + 8192);
-        tma_store_2d(&tm_u, 0, (int)(tile * kD), sb + OFF_KQ + 16384);
-        bulk_commit_group();
-        bulk_wait_read_all();
-    }
-
-done:
+    x.tmem = *tmem_slot;
+    const kda::Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam_out, flags, beta, g,
+                       T, n, scale, test_flags};
+    // chunk-major order: chunk 0 of every head first
+    const int c = (int)(blockIdx.x / (unsigned)BH);
+    const int64_t bh = blockIdx.x - (int64_t)c * BH;
+    int64_t pending = -1;
+    const bool ok = kda::kda_tile(x, ar, c, bh, pending);
+    if (ok && tid == kda::kStoreTid) kda::publish_pending(ar, pending);
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-        if (*abort_flag) {
-            // let the loads land before the shared memory is released
-            if (loads > 0) mbar_wait_bounded(ctl.bar(B_FULL), (uint32_t)(loads - 1), kWaitNs);
-            atomicOr(status, 1u);
-        }
-        bulk_wait_all();
-    }
+    if (!ok && tid == 0) atomicOr(status, 1u);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TM_COLS);
+        tmem_dealloc(x.tmem, kda::TM_COLS);
     }
 }
 
-}  // namespace kda
-
 // ---- host side ---------------------------------------------------------------
 
-cudaError_t launch_chunk_wy_kda(const ChunkArgs& a, const tc::TcMaps& m, cudaStream_t st) {
-    const int n = (int)((a.T + tc::kC - 1) / tc::kC);
-    auto kern = kda::chunk_wy_kda_kernel;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kda::SMEM_BYTES);
+cudaError_t launch_chunk_wy_kda(const ChunkArgs& a, const TcMaps& m, cudaStream_t st) {
+    const int n = (int)((a.T + kC - 1) / kC);
+    constexpr uint32_t kBytes = kda::GROUP_BYTES + 1024;
+    auto kern = chunk_wy_kda_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBytes);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(a.B * a.H * n), kda::kNT, kda::SMEM_BYTES, st>>>(
-        m.q, m.k, m.v, m.w, m.u, m.p_ws, m.kt_ws, m.qh_ws, m.gam_ws, (int)(a.B * a.H), a.beta, a.g, (int)a.T, n,
-        a.scale, a.status, a.test_flags);
+    kern<<<(unsigned)(a.B * a.H * n), kda::kNT, kBytes, st>>>(
+        m.q, m.k, m.v, m.w, m.u, m.p_ws, m.kt_ws, m.qh_ws, m.gam_ws, m.flags, (int)(a.B * a.H), a.beta, a.g,
+        (int)a.T, n, a.scale, a.status, a.test_flags);
     return counted(cudaGetLastError());
 }
 

@@ -173,10 +173,11 @@ def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
 
 
 @pytest.mark.parametrize("B,H,T", [(3, 32, 200), (4, 32, 130)])
-def test_tc_many_heads(cuda_device, B, H, T):
-    # 96 heads: the single launch in which each state-pass CTA also hosts a WY
-    # group; 128 heads: the two launches (WY kernel, then state pass)
-    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate="scalar", seed=B * H + T, s0_std=0.2)
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_tc_many_heads(cuda_device, B, H, T, gate):
+    # 96 heads: the single launch (scalar gate: each state-pass CTA also hosts a
+    # WY group); 128 heads: the two launches (WY kernel, then state pass)
+    inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate=gate, seed=B * H + T, s0_std=0.2)
     sc = 128 ** -0.5
     o, S = run(to_dev(inp), sc, path="tc")
     dn.dn_device_status()
@@ -194,8 +195,6 @@ def test_tc_many_heads(cuda_device, B, H, T):
 ])
 @pytest.mark.parametrize("gate", ["scalar", "per_key"])
 def test_chunk_kernel_launch_count(cuda_device, B, H, T, path, kernels, gate):
-    if gate == "per_key" and path == "tc":
-        kernels = 2              # per-key gate: its WY kernel, then the state pass
     inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate=gate, seed=5, s0_std=0.2)
     d = to_dev(inp)
     torch.cuda.synchronize()

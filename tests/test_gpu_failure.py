@@ -12,8 +12,9 @@ from _util import assert_close, oracle_prefill, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_device):
-    inp = W.gen_prefill(1, 2, 130, 128, 128, dtype="bf16", gate="scalar", seed=31, s0_std=0.1)
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_bounded_wait_timeout_is_reported_and_context_survives(cuda_device, gate):
+    inp = W.gen_prefill(1, 2, 130, 128, 128, dtype="bf16", gate=gate, seed=31, s0_std=0.1)
     d = to_dev(inp)
     sc = 128 ** -0.5
     dn.dn_device_status()                      # clean start
