@@ -69,9 +69,11 @@ constexpr uint32_t OFF_G = 49152;       // Gamma log2(e) of the current d-block,
 constexpr uint32_t OFF_T = OFF_G + 64 * 68 * 4;   // T (fp32 64 x 68), after the gram
 constexpr uint32_t OFF_B = 67584;       // the current d-block's B tiles: K rows 0 .. 16 (I + 1) - 1
                                         // scaled by e^(Gamma_mI - Gamma_j), I = 0..3
-constexpr uint32_t OFF_GATE = OFF_B + 20480;      // beta [64], then the prefix-sum segment totals [4][64]
-constexpr uint32_t OFF_BAR = OFF_GATE + 256 + 1024;
-constexpr uint32_t GROUP_BYTES = 90112;     // one group's shared memory, a multiple of 1024
+constexpr uint32_t OFF_GATE = OFF_B + 20480;      // beta [64]
+constexpr uint32_t OFF_TAB = OFF_GATE + 256;      // per d-block factor tables [18][64] fp32 (below); the
+                                                  // prefix-sum segment totals [4][64] before them
+constexpr uint32_t OFF_BAR = OFF_TAB + 18 * 64 * 4;
+constexpr uint32_t GROUP_BYTES = 93184;     // one group's shared memory, a multiple of 1024
 // (the last 16 bytes of a group stay free: a CTA keeps its TMEM address there)
 static_assert(OFF_BAR + 64 <= GROUP_BYTES - 16, "group layout");
 static_assert(OFF_T + 64 * 68 * 4 <= OFF_GATE, "T stays inside the dead B tiles");
@@ -87,6 +89,15 @@ constexpr uint32_t TM_COLS = 256;
 static_assert(b_off(3) + 8192 == 20480 && d_col(3) + 64 <= TM_COLS, "B tiles and D columns");
 
 constexpr float kCap2 = 80.f * 1.4426950408889634f;   // exponent cap, log2 units
+
+// Factor tables of one d-block, by 16-row block b (m_b = 16 b + 8) and channel:
+//   TAB_EM + b      e^Gamma_mb
+//   TAB_FC + b      e^(Gamma_last - Gamma_mb)
+//   TAB_R + p(I,b)  e^(Gamma_mI - Gamma_mb), I >= b, p(I, b) = I (I + 1) / 2 + b
+// so that every factor of row i (block b) is e1 = e^(Gamma_i - Gamma_mb) or
+// r1 = e^(Gamma_mb - Gamma_i) times one table entry: two exponentials per element.
+constexpr int TAB_EM = 0, TAB_FC = 4, TAB_R = 8, TAB_ROWS = 18;
+__host__ __device__ constexpr int tab_pair(int I, int b) { return I * (I + 1) / 2 + b; }
 
 constexpr int kStoreTid = wy::kStoreTid;   // issues the output stores and raises the ready flags
 // B_FULL completes twice per tile (K and Q; V); B_MMA three times (the gram's
@@ -191,7 +202,8 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
     uint8_t* sm = x.sm;
     const uint32_t sb = x.sb;
     float* bs = reinterpret_cast<float*>(sm + OFF_GATE);              // beta of the chunk
-    float* segt = reinterpret_cast<float*>(sm + OFF_GATE + 256);      // prefix-sum segment totals
+    float* segt = reinterpret_cast<float*>(sm + OFF_TAB);             // prefix-sum segment totals
+    float* tab = reinterpret_cast<float*>(sm + OFF_TAB);              // factor tables
     float* Gm = reinterpret_cast<float*>(sm + OFF_G);                 // Gamma log2(e), [64][68]
     float* Am = reinterpret_cast<float*>(sm + OFF_G);
     float* Tm = reinterpret_cast<float*>(sm + OFF_T);
@@ -233,18 +245,30 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
         bs[lane + 32] = lane + 32 < Cc ? beta[t0 + lane + 32] : 0.f;
     }
 
+    // g of thread (segment of 16 positions, channel), one d-block ahead: the second
+    // d-block's loads are under way while the first is processed
+    const int gch = tid & 63, gseg = tid >> 6;
+    float gv[16];
+    auto load_g = [&](int bb) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int i = 16 * gseg + r;
+            gv[r] = i < Cc ? g[(t0 + i) * kD + 64 * bb + gch] : 0.f;   // zero past the end: identity steps
+        }
+    };
+    load_g(0);
     for (int b = 0; b < 2; ++b) {
-        // ---- Gamma of channels 64 b .. 64 b + 63: thread (segment of 16 positions, channel)
+        // ---- Gamma of channels 64 b .. 64 b + 63 --------------------------------------
         {
-            const int ch = tid & 63, seg = tid >> 6;
+            const int ch = gch, seg = gseg;
             float acc[16];
             float run = 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                const int i = 16 * seg + r;
-                run += i < Cc ? g[(t0 + i) * kD + 64 * b + ch] : 0.f;   // zero past the end: identity steps
+                run += gv[r];
                 acc[r] = run;
             }
+            if (b == 0) load_g(1);
             segt[seg * 64 + ch] = run;
             named_bar_sync(kBar, kNT);
             float off = 0.f;
@@ -258,52 +282,72 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
         ok = b == 0 ? ctl.wait(B_FULL, 0) : wait_mma(x);
         if (named_bar_any(kBar, kNT, !ok)) goto done;
         tc_fence_after();
+        // ---- factor tables (over the segment totals, read by now) ----------------------
+        for (int idx = tid; idx < TAB_ROWS * 64; idx += kNT) {
+            const int tr = idx >> 6, ch = idx & 63;
+            float v;
+            if (tr < TAB_FC) {
+                v = ex2_approx(Gm[fidx(16 * tr + 8, ch)]);
+            } else if (tr < TAB_R) {
+                v = ex2_approx(Gm[fidx(63, ch)] - Gm[fidx(16 * (tr - TAB_FC) + 8, ch)]);
+            } else {
+                const int p = tr - TAB_R;                       // (I, b) in the order of tab_pair
+                const int I = (int)((0x3333222110ull >> (4 * p)) & 15), bb = (int)((0x3210210100ull >> (4 * p)) & 15);
+                v = ex2_approx(Gm[fidx(16 * I + 8, ch)] - Gm[fidx(16 * bb + 8, ch)]);
+            }
+            tab[idx] = v;
+        }
+        named_bar_sync(kBar, kNT);
 
         // ---- scaled operands: (row i, 8-channel chunk gq) per item, two per thread ------
 #pragma unroll 1
         for (int u = 0; u < 2; ++u) {
             const int x = tid + u * kNT;
             const int i = x >> 3, gq = x & 7, blk = i >> 4;
-            float gi[8], gm[8], gc[8], kv[8], qv[8], f[8];
+            float gi[8], gm[8], kv[8], qv[8], e1[8], r1[8], f[8], t8[8];
             load8(Gm + fidx(i, 8 * gq), gi);
             load8(Gm + fidx(16 * blk + 8, 8 * gq), gm);
-            load8(Gm + fidx(63, 8 * gq), gc);
             const uint32_t ka = sb + OFF_KQ + b * 16384 + sw128_off(i, gq);
             unpack8(ld_shared_v4(ka), kv);
             unpack8(ld_shared_v4(ka + 8192), qv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                e1[e] = ex2_approx(fminf(gi[e] - gm[e], kCap2));
+                r1[e] = ex2_approx(fminf(gm[e] - gi[e], kCap2));
+            }
+            const float* trow = tab + 8 * gq;
             const int64_t grow = (tile * kC + i) * kD + 64 * b + 8 * gq;   // workspace element
             // K (.) e^Gamma for W, and Qh = scale Q (.) e^Gamma
+            load8(trow + (TAB_EM + blk) * 64, t8);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(gi[e]);
+            for (int e = 0; e < 8; ++e) f[e] = e1[e] * t8[e];
             st_shared_u4(sb + OFF_KW + b * 8192 + sw128_off(i, gq), scaled8(kv, f));
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] *= scale;
             const uint4 qh = scaled8(qv, f);
             st_global_v4(qh_out + grow, qh.x, qh.y, qh.z, qh.w);
             // K~ = K (.) e^(Gamma_last - Gamma)
+            load8(trow + (TAB_FC + blk) * 64, t8);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(gc[e] - gi[e]);
+            for (int e = 0; e < 8; ++e) f[e] = r1[e] * t8[e];
             const uint4 kt = scaled8(kv, f);
             st_global_v4(kt_out + grow, kt.x, kt.y, kt.z, kt.w);
             if (i == 63) {
                 float4* gp = reinterpret_cast<float4*>(gam_out + tile * kD + 64 * b + 8 * gq);
-                gp[0] = make_float4(ex2_approx(gc[0]), ex2_approx(gc[1]), ex2_approx(gc[2]), ex2_approx(gc[3]));
-                gp[1] = make_float4(ex2_approx(gc[4]), ex2_approx(gc[5]), ex2_approx(gc[6]), ex2_approx(gc[7]));
+                gp[0] = make_float4(ex2_approx(gi[0]), ex2_approx(gi[1]), ex2_approx(gi[2]), ex2_approx(gi[3]));
+                gp[1] = make_float4(ex2_approx(gi[4]), ex2_approx(gi[5]), ex2_approx(gi[6]), ex2_approx(gi[7]));
             }
             // B tiles of the blocks I >= blk: K (.) e^(Gamma_mI - Gamma)
 #pragma unroll 1
             for (int I = blk; I < 4; ++I) {
-                float gr[8];
-                load8(Gm + fidx(16 * I + 8, 8 * gq), gr);
+                load8(trow + (TAB_R + tab_pair(I, blk)) * 64, t8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = ex2_approx(fminf(gr[e] - gi[e], kCap2));
+                for (int e = 0; e < 8; ++e) f[e] = r1[e] * t8[e];
                 st_shared_u4(sb + OFF_B + b_off(I) + sw128_off(i, gq), scaled8(kv, f));
             }
             // [K^;Q^] in place: rows scaled by e^(Gamma_i - Gamma_m(i))
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ex2_approx(fminf(gi[e] - gm[e], kCap2));
-            st_shared_u4(ka, scaled8(kv, f));
-            st_shared_u4(ka + 8192, scaled8(qv, f));
+            st_shared_u4(ka, scaled8(kv, e1));
+            st_shared_u4(ka + 8192, scaled8(qv, e1));
         }
         fence_async_smem();
         tc_fence_before();
