@@ -69,8 +69,11 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags};
     const int64_t tiles = (int64_t)BH * n;
+    // the tile counter follows the ready flags: each group's first tile is its index,
+    // the later ones come from tickets, in order (chunk-major), to whichever group is free
+    const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
+                      flags + tiles};
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
@@ -104,9 +107,10 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             x.tmem = tbase + state::Layout<true>::kCols;
             bool ok = true;
             int64_t pending = -1;
-            for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles; t += G) {
+            for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles;) {
                 const int c = (int)(t / BH);
                 ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
+                if (ok) t = G + (int64_t)wy::next_ticket(x);
             }
             if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
             if (!ok && x.tid == 0) atomicOr(status, 1u);
@@ -137,9 +141,10 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     x.tmem = *tmem_slot + (uint32_t)grp * wy::TM_COLS;
     bool ok = true;
     int64_t pending = -1;
-    for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles; t += G) {
+    for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles;) {
         const int c = (int)(t / BH);
         ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
+        if (ok) t = G + (int64_t)wy::next_ticket(x);
     }
     if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
     tc_fence_before();
@@ -195,15 +200,17 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     __syncthreads();
     tc_fence_after();
     x.tmem = *tmem_slot + (uint32_t)grp * kda::TM_COLS;
-    const kda::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam, flags, beta, g,
-                       T, n, scale, test_flags};
     const int64_t tiles = (int64_t)BH * n;
+    // first tile by group index, then tickets from the counter after the flags
+    const kda::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam, flags, beta, g,
+                       T, n, scale, test_flags, flags + tiles};
     const int64_t G = (int64_t)(gridDim.x - BH) * 2;      // WY groups in the grid
     bool ok = true;
     int64_t pending = -1;
-    for (int64_t t = (int64_t)(blockIdx.x - BH) * 2 + grp; ok && t < tiles; t += G) {
+    for (int64_t t = (int64_t)(blockIdx.x - BH) * 2 + grp; ok && t < tiles;) {
         const int c = (int)(t / BH);
         ok = kda::kda_tile(x, wa, c, t - (int64_t)c * BH, pending);
+        if (ok) t = G + (int64_t)kda::next_ticket(x);
     }
     if (ok && x.tid == kda::kStoreTid) kda::publish_pending(wa, pending);
     tc_fence_before();
@@ -269,7 +276,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
                             &T_i, &n_i, &scale, &status, &test_flags};
             // the flags are cleared on the same stream right before the launch
-            e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
+            e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
             return counted(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
                                                        dim3(kFusedThreads), args, kFusedBytes, st));
@@ -343,7 +350,7 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &m.kt, &m.qh, &p_out, &kt_out, &qh_out, &gam,
                             &flags, &bh_i, &beta, &g, &S0, &o, &S_T, &T_i, &n_i, &scale, &status, &test_flags};
             // the flags are cleared on the same stream right before the launch
-            e = cudaMemsetAsync(m.flags, 0, tiles * 4, st);
+            e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
             return counted(cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3((unsigned)num_sms),
                                                        dim3(kFusedKdaThreads), args, kFusedKdaBytes, st));

@@ -40,12 +40,15 @@ constexpr size_t kWsGamBytes = (size_t)kD * 4;
 constexpr size_t kWsKdaTileBytes = kWsTileBytes + kWsKtBytes + kWsQhBytes + kWsGamBytes;
 static_assert(kWsKdaTileBytes % 256 == 0, "flags stay 256-byte aligned");
 // ...then one 32-bit ready flag per tile, set (release) once the tile is
-// written and awaited (acquire) before the state pass loads it.
+// written and awaited (acquire) before the state pass loads it, and one
+// 32-bit counter from which the single-launch WY groups take their tiles after
+// the first; all zeroed before each prefill.
 inline size_t ws_flags_offset(uint64_t tiles, bool kda = false) {
     return (size_t)tiles * (kda ? kWsKdaTileBytes : kWsTileBytes);
 }
+inline size_t ws_flag_words(uint64_t tiles) { return (size_t)tiles + 1; }
 inline size_t ws_total_bytes(uint64_t tiles, bool kda = false) {
-    return ws_flags_offset(tiles, kda) + ((tiles * 4 + 255) / 256) * 256;
+    return ws_flags_offset(tiles, kda) + ((ws_flag_words(tiles) * 4 + 255) / 256) * 256;
 }
 
 // Tensor maps of the tensor-core path (128-byte swizzle, 64-column boxes):

@@ -149,6 +149,11 @@ __device__ __forceinline__ Group make_group(uint8_t* sm, uint32_t tmem, uint32_t
     return x;
 }
 
+// The ticket thread 0 took during the group's last tile (after wy_tile returned true).
+__device__ __forceinline__ unsigned int next_ticket(const Group& x) {
+    return *reinterpret_cast<volatile const unsigned int*>(x.sm + OFF_BAR + 24);
+}
+
 // Barriers and the abort flag of a group (one thread, before the group's first tile).
 __device__ __forceinline__ void init_group(const Group& x) {
     mbar_init(x.ctl.bar(B_FULL), 1);
@@ -169,6 +174,7 @@ struct Args {
     int T, n;
     float scale;
     int test_flags;
+    unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
 };
 
 // T = (I + A)^-1 for the unit-lower 64 x 64 system of one chunk, in fp32 on
@@ -259,7 +265,9 @@ __device__ __forceinline__ void publish_pending(const Args& ar, int64_t& pending
 
 // Chunk c of head bh.  `pending` (thread kStoreTid's copy counts) is the
 // group's tile whose flag is still to be raised, or -1; on return it is this
-// tile.  Returns false (the group's abort flag set) if a wait gave up.
+// tile.  With a tile counter, thread 0 also takes the group's next ticket,
+// readable with next_ticket() once this returns.  Returns false (the group's
+// abort flag set) if a wait gave up.
 template <int GATE>
 __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh, int64_t& pending) {
     const uint32_t sb = x.sb;
@@ -285,6 +293,8 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     const int64_t t0 = bh * T + (int64_t)c * kC;
     const bool load = !(ar.test_flags & 1);
     int loads = 0;                                   // load groups issued (thread 0)
+    // the next ticket, taken now and used after the tile: its latency is hidden
+    const unsigned int ticket = tid == 0 && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
 
     if (tid == 0 && load) {
         const uint32_t fb = ctl.bar(B_FULL);
@@ -498,6 +508,7 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         bulk_wait_read_all();
         pending = tile;
     }
+    if (tid == 0) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
     tc_fence_before();
     named_bar_sync(x.bar, kNT);
     return true;

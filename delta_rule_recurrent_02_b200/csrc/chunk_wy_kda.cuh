@@ -176,7 +176,13 @@ struct Args {
     int T, n;
     float scale;
     int test_flags;
+    unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
 };
+
+// The ticket thread 0 took during the group's last tile (after kda_tile returned true).
+__device__ __forceinline__ unsigned int next_ticket(const Group& x) {
+    return *reinterpret_cast<volatile const unsigned int*>(x.sm + OFF_BAR + 24);
+}
 
 // Thread kStoreTid: raise the previous tile's ready flag once its stores
 // (issued by this thread) are complete; as wy::publish_pending.
@@ -197,7 +203,8 @@ __device__ __forceinline__ bool wait_mma(Group& x) {
 
 // Chunk c of head bh.  `pending` (thread kStoreTid's copy counts) is the
 // group's tile whose flag is still to be raised, or -1; on return it is this
-// tile.  Returns false (the group's abort flag set) if a wait gave up.
+// tile.  With a tile counter, thread 0 also takes the group's next ticket
+// (next_ticket()).  Returns false (the group's abort flag set) if a wait gave up.
 __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_t bh, int64_t& pending) {
     uint8_t* sm = x.sm;
     const uint32_t sb = x.sb;
@@ -230,6 +237,8 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
     const bool load = !(ar.test_flags & 1);
     int loads = 0;                                   // load phases issued (thread 0)
     bool ok = true;
+    // the group's next ticket, taken now and used after the tile: its latency is hidden
+    const unsigned int ticket = tid == 0 && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
 
     if (tid == 0 && load) {
         const uint32_t fb = ctl.bar(B_FULL);
@@ -526,6 +535,7 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
         bulk_wait_read_all();
         pending = tile;
     }
+    if (tid == 0) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
     tc_fence_before();
     named_bar_sync(kBar, kNT);
     return true;

@@ -122,12 +122,13 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
  * intra-chunk attention P of every chunk ("Training it: the WY trick", D2L
  * 12.5; "The chunked form", ch. 28) in a kernel that runs over all chunks at
  * once, then streams them into the sequential state pass: 40 KiB and a 4-byte
- * ready flag per (b, h, chunk), i.e. with n = B * H * ceil(T / 64) chunks,
- * n * 40960 + (4 n rounded up to a multiple of 256) bytes.  With the per-key
+ * ready flag per (b, h, chunk), and a 4-byte tile counter, i.e. with
+ * n = B * H * ceil(T / 64) chunks, n * 40960 + (4 (n + 1) rounded up to a
+ * multiple of 256) bytes.  With the per-key
  * gate (KDA: "A walk through of the DeltaNet family of linear attention
  * variants") each chunk also keeps q and k with their decays applied and the
- * chunk's decay per key channel: 72.5 KiB per chunk, n * 74240 + (4 n rounded
- * up to a multiple of 256) bytes.  Its gram splits the decays around one
+ * chunk's decay per key channel: 72.5 KiB per chunk, n * 74240 + (4 (n + 1)
+ * rounded up to a multiple of 256) bytes.  Its gram splits the decays around one
  * reference position per 16-token block, so the tensor-core result is exact up
  * to rounding while no key channel decays by more than e^-80 over 8
  * consecutive tokens (the SIMT path has no such bound).  Sizes are checked as

@@ -54,12 +54,15 @@ def test_noalloc_matches_dn_chunk_fwd_on_two_calls(cuda_device):
 
 
 def test_noalloc_rejects_requests_above_its_scratch_area():
-    # 32 heads x 1024 chunks x (40 KiB + a 4-byte flag) = 1.25 GiB of scratch, above the fixed
-    # 64 MiB: refused before any device work (the fake addresses are never used)
+    # 32 heads x 1024 chunks x 40 KiB, plus a 4-byte flag per chunk and a tile counter, is
+    # 1.25 GiB of scratch, above the fixed 64 MiB: refused before any device work (the fake
+    # addresses are never used)
     lib, f = noalloc_fn()
     A, STEP = 0x10000000, 0x40000000
     st = f(A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, None, A + 5 * STEP, None,
            1, 65536, 32, 128, 128, 64, 1.0, 1, 1, None)
     assert st == dn.DN_ERR_UNSUPPORTED
     msg = lib.dn_last_error().decode()
-    assert str(32 * 1024 * (40960 + 4)) in msg and str(64 << 20) in msg
+    n = 32 * 1024
+    need = n * 40960 + (4 * (n + 1) + 255) // 256 * 256
+    assert str(need) in msg and str(64 << 20) in msg
