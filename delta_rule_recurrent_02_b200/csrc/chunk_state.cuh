@@ -250,6 +250,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             const uint32_t I_SW = idesc_bf16(128, 128, 0, 0);       // [O|U] = S^T [Qh;-W]^T
             const uint32_t I_KU = idesc_bf16(128, 128, 0, 1);       // B MN-major
             const uint32_t I_PU = idesc_bf16(128, 64, 0, 0);
+            // A operand of KU: U~^T, or U^T itself with the per-key gate (K~ carries the decay)
+            const uint32_t TM_KU_A = GATE == kGatePerKey ? TM_UT : TM_UK;
             bool ok = true;
             for (int c = 0; ok && c < n; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
@@ -266,17 +268,21 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                      ctl.wait(B_STA, par);
                 if (!ok) break;
                 tc_fence_after();
+                // the stage's operand descriptors once; a step along K is a constant added to
+                // the start-address field (address / 16; the stage is 1024-byte aligned and the
+                // offsets stay inside the field)
+                const uint64_t dB = sw128_desc(st + ST_B, 16, 1024);     // [Qh | -W] rows, K-major
+                const uint64_t dK = sw128_desc(st + ST_K, 8192, 1024);   // K, MN-major
+                const uint64_t dP = sw128_desc(st + ST_P, 16, 1024);     // P, K-major
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
-                                sw128_desc(st + ST_B + (kk & 3) * 32, 16, 1024), I_SW, kk > 0);
+                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8, dB + (uint64_t)(2 * kk), I_SW, kk > 0);
                 ok = ctl.wait(B_STB, par);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 4; kk < 8; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8,
-                                sw128_desc(st + ST_B + 16384 + (kk & 3) * 32, 16, 1024), I_SW, 1);
+                    mma_bf16_ts(ou, tmem + TM_ST + kk * 8, dB + (uint64_t)(16384 / 16 + 2 * (kk & 3)), I_SW, 1);
                 mma_commit(ctl.bar(B_WS));
                 // S^T += U~^T K and O^T += U^T P^T, positions 0-31 then 32-63
                 ok = ctl.wait(B_UTA, par);
@@ -284,22 +290,20 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
-                                I_KU, 1);
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_KU_A + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
+                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, dP + (uint64_t)(2 * kk), I_PU, 1);
                 ok = ctl.wait(B_UTB, par);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 2; kk < 4; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UK + kk * 8, sw128_desc(st + ST_K + kk * 2048, 8192, 1024),
-                                I_KU, 1);
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_KU_A + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
                 mma_commit(ctl.bar(B_KU));
 #pragma unroll
                 for (int kk = 2; kk < 4; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, sw128_desc(st + ST_P + kk * 32, 16, 1024), I_PU, 1);
+                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, dP + (uint64_t)(2 * kk), I_PU, 1);
                 mma_commit(ctl.bar(B_PU0 + (c & 1)));
                 mma_commit(ctl.bar(B_FREE0 + s));        // the stage's last reader is done
             }
@@ -426,15 +430,16 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 tmem_st8(tmem + lane_off + TM_UT + (i0 >> 1), pk);
                 if (GATE != kGatePerKey) {
-                    // U~ = U (.) e^(G_last - G) by rows; with the per-key gate K~ carries the decay
+                    // U~ = U (.) e^(G_last - G) by rows; with the per-key gate K~ carries the
+                    // decay and the KU product reads U^T itself
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
                         pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
                         pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
                     }
+                    tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
                 }
-                tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
