@@ -177,19 +177,12 @@ struct Args {
     unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
 };
 
-// T = (I + A)^-1 for the unit-lower 64 x 64 system of one chunk, in fp32 on
-// CUDA cores, by a group of 8 warps (named barrier `bar`, kNT threads).  Am
-// holds A (strictly lower; its blocks on and above the diagonal are never
-// read) and is overwritten by M; Tm receives T on and below the block
-// diagonal.  The 16 x 16 diagonal blocks D_k = (I + A_kk)^-1 come from forward
-// substitution, then M_kl = D_k A_kl and T_kl = -sum_{m=l}^{k-1} M_km T_ml in
-// three rounds (block forward substitution).  idle() is run by warps 6 and 7
-// while the others form M.  Ends with a group barrier.
-template <class Idle>
-__device__ __forceinline__ void wy_solve(float* Am, float* Tm, int warp, int lane, uint32_t bar, Idle idle) {
-    // ---- 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 into T ------------------------
-    if (warp < 4 && lane < 16) {
-        const int k0 = warp * 16, jj = lane;
+// The 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 of blocks kb and kb + 1
+// into T, by forward substitution: one warp, lane -> (block kb + lane / 16,
+// column lane % 16).  A's rows of those blocks must be visible to the warp.
+__device__ __forceinline__ void wy_diag2(const float* Am, float* Tm, int kb, int lane) {
+    {
+        const int k0 = (kb + (lane >> 4)) * 16, jj = lane & 15;
         float x[16];
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
@@ -206,7 +199,18 @@ __device__ __forceinline__ void wy_solve(float* Am, float* Tm, int warp, int lan
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) Tm[fidx(k0 + ii, k0 + jj)] = x[ii];
     }
-    named_bar_sync(bar, kNT);
+}
+
+// T = (I + A)^-1 for the unit-lower 64 x 64 system of one chunk, in fp32 on
+// CUDA cores, by a group of 8 warps (named barrier `bar`, kNT threads), once
+// the diagonal inverses D_k are in Tm (wy_diag2) and the group has passed a
+// barrier.  Am holds A (strictly lower; the blocks above its diagonal blocks
+// are never read) and is overwritten by M; Tm receives T on and below the
+// block diagonal: M_kl = D_k A_kl, then T_kl = -sum_{m=l}^{k-1} M_km T_ml in
+// three rounds (block forward substitution).  idle() is run by warps 6 and 7
+// while the others form M.  Ends with a group barrier.
+template <class Idle>
+__device__ __forceinline__ void wy_solve(float* Am, float* Tm, int warp, int lane, uint32_t bar, Idle idle) {
     // ---- M_kl = D_k A_kl (k > l), in place of A_kl -------------------------------------
     if (warp < 6) {
         // (k, l) = (1,0) (2,0) (3,0) (2,1) (3,1) (3,2) for warps 0..5
@@ -354,10 +358,7 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         const int j0 = (warp >> 2) << 5;
         const float g2i = gs[G_G2 + i];
         if (q == 0 && j0 == 32) {
-            // A rows 0-31 x columns 32-63 lie above the diagonal
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-                *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(0.f, 0.f, 0.f, 0.f);
+            // A rows 0-31 x columns 32-63 lie above the diagonal: never read
         } else if (q < 2) {
             float v[32];
             tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
@@ -374,6 +375,11 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                     a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
                 }
                 *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
+            }
+            if (warp == 0 || warp == 5) {
+                // the diagonal blocks of the rows just written: 0 and 1 (warp 0), 2 and 3 (warp 5)
+                __syncwarp();
+                wy_diag2(Am, Tm, warp == 0 ? 0 : 2, lane);
             }
         } else {
             // P row i, columns j0 .. j0 + 31 -> workspace (row-major [64][64])

@@ -412,6 +412,11 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
                     }
                     *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
                 }
+                if (warp == 0 || warp == 5) {
+                    // the diagonal blocks of the rows just written: 0 and 1 (warp 0), 2 and 3 (warp 5)
+                    __syncwarp();
+                    wy::wy_diag2(Am, Tm, warp == 0 ? 0 : 2, lane);
+                }
             }
         } else {
             __nv_bfloat16* prow = p_out + (tile * kC + i) * kC + j0;
