@@ -72,9 +72,9 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int64_t tiles = (int64_t)BH * n;
     // the tile counter follows the ready flags: each group's first tile is its index,
     // the later ones come from tickets, in order (chunk-major), to whichever group is free
-    const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
-                      flags + tiles};
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
+    const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
+                      flags + tiles, BH, (int)G};
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags, nullptr};
@@ -202,9 +202,9 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     x.tmem = *tmem_slot + (uint32_t)grp * kda::TM_COLS;
     const int64_t tiles = (int64_t)BH * n;
     // first tile by group index, then tickets from the counter after the flags
-    const kda::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam, flags, beta, g,
-                       T, n, scale, test_flags, flags + tiles};
     const int64_t G = (int64_t)(gridDim.x - BH) * 2;      // WY groups in the grid
+    const kda::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam, flags, beta, g,
+                       T, n, scale, test_flags, flags + tiles, BH, (int)G};
     bool ok = true;
     int64_t pending = -1;
     for (int64_t t = (int64_t)(blockIdx.x - BH) * 2 + grp; ok && t < tiles;) {

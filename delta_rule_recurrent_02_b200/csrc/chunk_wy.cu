@@ -37,7 +37,8 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     x.tmem = *tmem_slot;
-    const Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags, nullptr};
+    const Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags, nullptr,
+                  BH, 0};
     // chunk-major order: chunk 0 of every head first
     const int c = (int)(blockIdx.x / (unsigned)BH);
     const int64_t bh = blockIdx.x - (int64_t)c * BH;

@@ -149,7 +149,7 @@ __device__ __forceinline__ Group make_group(uint8_t* sm, uint32_t tmem, uint32_t
     return x;
 }
 
-// The ticket thread 0 took during the group's last tile (after wy_tile returned true).
+// The ticket taken during the group's last tile (after wy_tile returned true).
 __device__ __forceinline__ unsigned int next_ticket(const Group& x) {
     return *reinterpret_cast<volatile const unsigned int*>(x.sm + OFF_BAR + 24);
 }
@@ -175,7 +175,29 @@ struct Args {
     float scale;
     int test_flags;
     unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
+    int BH, G;               // with a counter: heads and WY groups (a ticket x is tile G + x)
 };
+
+// Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
+// (if any) into L2, so that its loads at the group's next tile hit L2: K, Q
+// and V by tensor prefetches, beta and g of a full chunk by bulk prefetches.
+__device__ __forceinline__ void prefetch_next(const Args& ar, unsigned int ticket, bool gated) {
+    if (!ar.counter) return;
+    const int64_t tn = (int64_t)ar.G + ticket;
+    if (tn >= (int64_t)ar.BH * ar.n) return;
+    const int cn = (int)(tn / ar.BH);
+    const int64_t y = (tn - (int64_t)cn * ar.BH) * ar.T + (int64_t)cn * kC;
+    tma_prefetch_2d(ar.tm_k, 0, (int)y);
+    tma_prefetch_2d(ar.tm_k, 64, (int)y);
+    tma_prefetch_2d(ar.tm_q, 0, (int)y);
+    tma_prefetch_2d(ar.tm_q, 64, (int)y);
+    tma_prefetch_2d(ar.tm_v, 0, (int)y);
+    tma_prefetch_2d(ar.tm_v, 64, (int)y);
+    if (ar.T - cn * kC >= kC) {
+        bulk_prefetch_l2(ar.beta + y, kC * 4);
+        if (gated) bulk_prefetch_l2(ar.g + y, kC * 4);
+    }
+}
 
 // The 16 x 16 diagonal inverses D_k = (I + A_kk)^-1 of blocks kb and kb + 1
 // into T, by forward substitution: one warp, lane -> (block kb + lane / 16,
@@ -269,8 +291,9 @@ __device__ __forceinline__ void publish_pending(const Args& ar, int64_t& pending
 
 // Chunk c of head bh.  `pending` (thread kStoreTid's copy counts) is the
 // group's tile whose flag is still to be raised, or -1; on return it is this
-// tile.  With a tile counter, thread 0 also takes the group's next ticket,
-// readable with next_ticket() once this returns.  Returns false (the group's
+// tile.  With a tile counter, thread kStoreTid also takes the group's next
+// ticket, prefetches that tile's inputs into L2, and hands the ticket on
+// (next_ticket() once this returns).  Returns false (the group's
 // abort flag set) if a wait gave up.
 template <int GATE>
 __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh, int64_t& pending) {
@@ -297,8 +320,9 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     const int64_t t0 = bh * T + (int64_t)c * kC;
     const bool load = !(ar.test_flags & 1);
     int loads = 0;                                   // load groups issued (thread 0)
-    // the next ticket, taken now and used after the tile: its latency is hidden
-    const unsigned int ticket = tid == 0 && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
+    // the next ticket, taken now (by the thread that prefetches for it and hands it on)
+    // and used after the tile: its latency is hidden
+    const unsigned int ticket = tid == kStoreTid && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
 
     if (tid == 0 && load) {
         const uint32_t fb = ctl.bar(B_FULL);
@@ -416,7 +440,10 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
 
     // ---- T = (I + A)^-1; warp 6 raises the previous tile's ready flag meanwhile --------
     wy_solve(Am, Tm, warp, lane, x.bar, [&] {
-        if (tid == kStoreTid) publish_pending(ar, pending);
+        if (tid == kStoreTid) {
+            publish_pending(ar, pending);
+            prefetch_next(ar, ticket, GATE == kGateScalar);
+        }
     });
     // ---- T diag(beta e^G) and T diag(beta) as bf16 operand tiles, over A (zero above
     //      the block diagonal, where T was never written) ----------------------------------
@@ -514,7 +541,7 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         bulk_wait_read_all();
         pending = tile;
     }
-    if (tid == 0) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
+    if (tid == kStoreTid) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
     tc_fence_before();
     named_bar_sync(x.bar, kNT);
     return true;

@@ -35,7 +35,7 @@ chunk_wy_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_after();
     x.tmem = *tmem_slot;
     const kda::Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, kt_out, qh_out, gam_out, flags, beta, g,
-                       T, n, scale, test_flags, nullptr};
+                       T, n, scale, test_flags, nullptr, BH, 0};
     // chunk-major order: chunk 0 of every head first
     const int c = (int)(blockIdx.x / (unsigned)BH);
     const int64_t bh = blockIdx.x - (int64_t)c * BH;

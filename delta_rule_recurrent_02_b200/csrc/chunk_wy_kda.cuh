@@ -177,9 +177,31 @@ struct Args {
     float scale;
     int test_flags;
     unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
+    int BH, G;               // with a counter: heads and WY groups (a ticket x is tile G + x)
 };
 
-// The ticket thread 0 took during the group's last tile (after kda_tile returned true).
+// Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
+// (if any) into L2: K, Q and V by tensor prefetches, beta and the 32 KiB of g
+// of a full chunk by bulk prefetches.
+__device__ __forceinline__ void prefetch_next(const Args& ar, unsigned int ticket) {
+    if (!ar.counter) return;
+    const int64_t tn = (int64_t)ar.G + ticket;
+    if (tn >= (int64_t)ar.BH * ar.n) return;
+    const int cn = (int)(tn / ar.BH);
+    const int64_t y = (tn - (int64_t)cn * ar.BH) * ar.T + (int64_t)cn * kC;
+    tma_prefetch_2d(ar.tm_k, 0, (int)y);
+    tma_prefetch_2d(ar.tm_k, 64, (int)y);
+    tma_prefetch_2d(ar.tm_q, 0, (int)y);
+    tma_prefetch_2d(ar.tm_q, 64, (int)y);
+    tma_prefetch_2d(ar.tm_v, 0, (int)y);
+    tma_prefetch_2d(ar.tm_v, 64, (int)y);
+    if (ar.T - cn * kC >= kC) {
+        bulk_prefetch_l2(ar.beta + y, kC * 4);
+        bulk_prefetch_l2(ar.g + y * kD, kC * kD * 4);
+    }
+}
+
+// The ticket taken during the group's last tile (after kda_tile returned true).
 __device__ __forceinline__ unsigned int next_ticket(const Group& x) {
     return *reinterpret_cast<volatile const unsigned int*>(x.sm + OFF_BAR + 24);
 }
@@ -237,8 +259,9 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
     const bool load = !(ar.test_flags & 1);
     int loads = 0;                                   // load phases issued (thread 0)
     bool ok = true;
-    // the group's next ticket, taken now and used after the tile: its latency is hidden
-    const unsigned int ticket = tid == 0 && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
+    // the group's next ticket, taken now (by the thread that prefetches for it and hands
+    // it on) and used after the tile: its latency is hidden
+    const unsigned int ticket = tid == kStoreTid && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
 
     if (tid == 0 && load) {
         const uint32_t fb = ctl.bar(B_FULL);
@@ -449,7 +472,10 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
 
     // ---- T = (I + A)^-1; warp 6 raises the previous tile's ready flag meanwhile --------
     wy::wy_solve(Am, Tm, warp, lane, kBar, [&] {
-        if (tid == kStoreTid) publish_pending(ar, pending);
+        if (tid == kStoreTid) {
+            publish_pending(ar, pending);
+            prefetch_next(ar, ticket);
+        }
     });
 
     // ---- T diag(beta) as a bf16 operand tile over A (zero above the block diagonal) ---
@@ -540,7 +566,7 @@ __device__ __forceinline__ bool kda_tile(Group& x, const Args& ar, int c, int64_
         bulk_wait_read_all();
         pending = tile;
     }
-    if (tid == 0) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
+    if (tid == kStoreTid) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
     tc_fence_before();
     named_bar_sync(kBar, kNT);
     return true;

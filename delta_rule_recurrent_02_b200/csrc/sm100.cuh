@@ -74,6 +74,20 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// Prefetch one tile of a tensor map into L2 (no shared memory, nothing to wait
+// for; coordinates past the tensor's end are dropped by the bounds check).
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y) : "memory");
+}
+// Prefetch `bytes` (a multiple of 16, inside one allocation) at p into L2; a
+// p that is not 16-byte aligned is skipped (the bulk copy requires it).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    if (reinterpret_cast<uint64_t>(p) & 15u) return;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
 // Tile store shared -> global through a tensor map (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uint32_t src) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
