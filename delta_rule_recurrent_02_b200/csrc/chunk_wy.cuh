@@ -495,39 +495,33 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     ok = ok && ctl.wait(B_MMA, 1);
     if (named_bar_any(x.bar, kNT, !ok)) goto done;
     tc_fence_after();
-    // ---- TMEM -> bf16 tiles over K and V (read by now), then TMA stores.  Warps 0-3:
-    //      -W, row-major [64 rows][128] as two [64][128 B] column blocks (lane r is
-    //      column r: element stores); warps 4-7: u^T [128][128 B] (lane r is row r) ------
-    if (warp < 4) {
-        const int r = (warp << 5) + lane;              // d_k channel
+    // ---- TMEM -> bf16 -W and u^T tiles over K and V (read by now), then TMA stores -------
+    {
+        // warp w: TMEM lane quarter w % 4 (-W: d_k channels; u^T: d_v rows), positions
+        // 32 (w / 4) .. 32 (w / 4) + 31 of both
+        const int q = warp & 3, hh = warp >> 2;
+        const int r = (q << 5) + lane;
+        const uint32_t lanes = tmem + ((uint32_t)(q << 5) << 16);
+        float v[32];
+        // -W row-major [64 positions][128 d_k] as two [64][128 B] column blocks: lane r is column r
+        tmem_ld32(lanes + TM_W + hh * 32, v);
+        tmem_wait_ld();
         const uint32_t base = sb + OFF_KV + (uint32_t)(r >> 6) * 8192 + (uint32_t)(r & 7) * 2;
         const int ch = (r & 63) >> 3;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp << 5) << 16) + TM_W + hh * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = hh * 32 + e;
-                st_shared_b16(base + (uint32_t)(i * 128 + ((ch ^ (i & 7)) << 4)), __float2bfloat16_rn(-v[e]));
-            }
+        for (int e = 0; e < 32; ++e) {
+            const int i = hh * 32 + e;
+            st_shared_b16(base + (uint32_t)(i * 128 + ((ch ^ (i & 7)) << 4)), __float2bfloat16_rn(-v[e]));
         }
-    } else {
-        const int q = warp & 3;
-        const int r = (q << 5) + lane;
+        // u^T [128 d_v][64 positions]: lane r is row r
+        tmem_ld32(lanes + TM_U + hh * 32, v);
+        tmem_wait_ld();
         const uint32_t dst = sb + OFF_KV + 16384;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[32];
-            tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_U + hh * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                st_shared_v4(dst + sw128_off(r, hh * 4 + q4), pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
-                             pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]), pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
-                             pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
-        }
+        for (int q4 = 0; q4 < 4; ++q4)
+            st_shared_v4(dst + sw128_off(r, hh * 4 + q4), pack_bf16x2(v[8 * q4 + 0], v[8 * q4 + 1]),
+                         pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]), pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                         pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
     }
     fence_async_smem();
     named_bar_sync(x.bar, kNT);
