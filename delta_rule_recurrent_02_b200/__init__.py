@@ -25,6 +25,7 @@ import ctypes
 import os
 
 __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
+           "dn_chunk_fwd_snapshots",
            "dn_decode_step", "dn_kernel_launches",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
@@ -35,6 +36,7 @@ _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
+               "dn_chunk_fwd_snapshots",
                "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version",
                "dn_kernel_launches")
 
@@ -67,6 +69,9 @@ def load_library():
     lib.dn_chunk_fwd.restype = I
     lib.dn_chunk_fwd_ex.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, I, vp, Z, vp]
     lib.dn_chunk_fwd_ex.restype = I
+    lib.dn_chunk_fwd_snapshots.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, I, I, I, I, I, I, I, F, I, I, I,
+                                           vp, Z, vp]
+    lib.dn_chunk_fwd_snapshots.restype = I
     lib.dn_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I, ctypes.POINTER(Z)]
     lib.dn_chunk_fwd_workspace_size.restype = I
     lib.dn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp]
@@ -165,6 +170,25 @@ def dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, *, chunk: int = 64, scale: float 
                              _ptr(S_T), B, T, H, dk, dv, int(chunk), float(scale), _dtype_code(q),
                              _gate_code(gate, g, (B, H, T)), _PATHS[path], _ptr(workspace), ws_bytes,
                              _stream(stream))
+    _check(lib, st)
+
+
+def dn_chunk_fwd_snapshots(q, k, v, beta, g, S0, o, S_T, snaps, every: int, *, chunk: int = 64,
+                           scale: float = 1.0, gate: str | None = None, path: str = "auto", workspace=None,
+                           stream=None) -> None:
+    """``dn_chunk_fwd`` that also writes ``snaps`` [B, H, n_snap, d_k, d_v] fp32, the
+    state after every ``every`` chunks (n_snap = T // (every * chunk)), through
+    ``dn_chunk_fwd_snapshots``."""
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    for t in (beta, g, S0, S_T, snaps):
+        _f32(t)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.dn_chunk_fwd_snapshots(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o),
+                                    _ptr(S_T), _ptr(snaps), int(every), B, T, H, dk, dv, int(chunk), float(scale),
+                                    _dtype_code(q), _gate_code(gate, g, (B, H, T)), _PATHS[path],
+                                    _ptr(workspace), ws_bytes, _stream(stream))
     _check(lib, st)
 
 

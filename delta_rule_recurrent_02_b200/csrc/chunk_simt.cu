@@ -62,7 +62,7 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const float* __restrict__ beta,
                   const float* __restrict__ g, const float* S0,
                   Tin* __restrict__ o, float* S_T, int T, int DV, int chunk,
-                  float scale) {
+                  float scale, float* snaps, int snap_every, int n_snap) {
     using L = SimtSmem<DK, GATE>;
     constexpr int KS = L::KS;
     extern __shared__ float sm[];
@@ -297,6 +297,18 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 }
             }
         }
+        // ---- snapshot: the state after chunks 1 .. (s + 1) snap_every (full chunks only)
+        if (snaps) {
+            const int ci = c0 / chunk + 1;               // chunks done
+            if (ci % snap_every == 0 && ci / snap_every <= n_snap) {
+                __syncthreads();
+                const int64_t sn = bh * n_snap + ci / snap_every - 1;
+                for (int x = tid; x < DK * kDVT; x += kNT) {
+                    const int i = x / kDVT, j = x % kDVT;
+                    snaps[(sn * DK + i) * DV + col0 + j] = Ss[i * kVS + j];
+                }
+            }
+        }
     }
     __syncthreads();
     if (S_T) {
@@ -316,7 +328,8 @@ static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t st) {
     const int64_t grid = a.B * a.H * (a.dv / kDVT);
     kern<<<(unsigned)grid, kNT, L::bytes, st>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-        a.beta, a.g, a.S0, static_cast<Tin*>(a.o), a.S_T, (int)a.T, a.dv, a.chunk, a.scale);
+        a.beta, a.g, a.S0, static_cast<Tin*>(a.o), a.S_T, (int)a.T, a.dv, a.chunk, a.scale, a.snaps, a.snap_every,
+        a.n_snap);
     return counted(cudaGetLastError());
 }
 

@@ -114,6 +114,8 @@ struct Args {
     unsigned int* status;
     int test_flags;
     const float* gam;               // per-key gate: the workspace's e^Gamma_last per tile and channel
+    float* snaps;                   // null, or [heads][n_snap][d_k][d_v]: the state after every
+    int snap_every, n_snap;         //   snap_every chunks (full chunks only)
 };
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
@@ -452,6 +454,10 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             tc_fence_after();
             const bool last = c + 1 == n;
             const float* gsn = gates + ((c + 1) & 3) * GATE_FLOATS;
+            // snapshot s = (c + 1) / snap_every - 1 of the state after this chunk
+            const bool snap = ar.snaps && (c + 1) % ar.snap_every == 0 && (c + 1) / ar.snap_every <= ar.n_snap;
+            float* snap_out = snap ? ar.snaps + ((bh * ar.n_snap + (c + 1) / ar.snap_every - 1) * kD) * kD + j
+                                   : nullptr;
             const float gnext = last || GATE == kGatePerKey ? 1.f : gsn[G_GAMMA];
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
@@ -459,6 +465,10 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 float v[32];
                 tmem_ld32(tmem + lane_off + TM_SACC + pc * 32, v);
                 tmem_wait_ld();
+                if (snap) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) snap_out[(pc * 32 + e) * kD] = v[e];
+                }
                 if (last) {
                     if (S_T) {
 #pragma unroll

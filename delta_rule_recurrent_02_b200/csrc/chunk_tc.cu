@@ -34,13 +34,13 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_p, const unsigned int* __restrict__ flags,
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, float scale, unsigned int* status,
-                   int test_flags, const float* __restrict__ gam) {
+                   int test_flags, const float* __restrict__ gam, float* snaps, int snap_every, int n_snap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
-                         gam};
+                         gam, snaps, snap_every, n_snap};
     state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
 }
 
@@ -65,7 +65,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    __nv_bfloat16* __restrict__ p_out, unsigned int* __restrict__ flags, int BH,
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale, unsigned int* status,
-                   int test_flags) {
+                   int test_flags, float* snaps, int snap_every, int n_snap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -77,7 +77,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                       flags + tiles, BH, (int)G};
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, nullptr};
+                             test_flags, nullptr, snaps, snap_every, n_snap};
         if (!HOSTED) {
             // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
             if (warp >= state::kNT / 32) return;
@@ -175,12 +175,12 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        __nv_bfloat16* p_out, __nv_bfloat16* kt_out, __nv_bfloat16* qh_out, float* gam,
                        unsigned int* flags, int BH, const float* __restrict__ beta, const float* __restrict__ g,
                        const float* S0, __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale,
-                       unsigned int* status, int test_flags) {
+                       unsigned int* status, int test_flags, float* snaps, int snap_every, int n_snap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_kt, &tm_qh, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, gam};
+                             test_flags, gam, snaps, snap_every, n_snap};
         state::state_pass<kGatePerKey, false>(sm, ar, blockIdx.x, 0u);
         return;
     }
@@ -273,8 +273,10 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
             float* S_T = a.S_T;
             unsigned int* status = a.status;
+            float* snaps = a.snaps;
+            int snap_every = a.snap_every, n_snap = a.n_snap;
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
-                            &T_i, &n_i, &scale, &status, &test_flags};
+                            &T_i, &n_i, &scale, &status, &test_flags, &snaps, &snap_every, &n_snap};
             // the flags are cleared on the same stream right before the launch
             e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
@@ -291,7 +293,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     // the WY kernel has finished before this launch starts: no flags to wait for
     kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
-                                                  a.status, a.test_flags, nullptr);
+                                                  a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap);
     return counted(cudaGetLastError());
 }
 
@@ -347,8 +349,11 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
             float* S_T = a.S_T;
             unsigned int* status = a.status;
+            float* snaps = a.snaps;
+            int snap_every = a.snap_every, n_snap = a.n_snap;
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &m.kt, &m.qh, &p_out, &kt_out, &qh_out, &gam,
-                            &flags, &bh_i, &beta, &g, &S0, &o, &S_T, &T_i, &n_i, &scale, &status, &test_flags};
+                            &flags, &bh_i, &beta, &g, &S0, &o, &S_T, &T_i, &n_i, &scale, &status, &test_flags,
+                            &snaps, &snap_every, &n_snap};
             // the flags are cleared on the same stream right before the launch
             e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
@@ -364,7 +369,8 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(a.B * a.H), state::kNT, bytes, st>>>(m.kt, m.qh, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
-                                                          a.scale, a.status, a.test_flags, m.gam_ws);
+                                                          a.scale, a.status, a.test_flags, m.gam_ws, a.snaps,
+                                                          a.snap_every, a.n_snap);
     return counted(cudaGetLastError());
 }
 

@@ -108,7 +108,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 2; }
+int dn_version(void) { return (2 << 16) | 3; }
 
 unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 
@@ -136,11 +136,11 @@ int dn_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int chunk
     return ok();
 }
 
-int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+static int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* beta,
                     const float* g, const float* S0, void* o, float* S_T,
                     int B, int T, int H, int d_k, int d_v, int chunk, float scale,
                     dn_dtype dtype, dn_gate gate, dn_path path, void* workspace, size_t workspace_bytes,
-                    void* cuda_stream) {
+                    void* cuda_stream, float* snaps, int every) {
     dn::ChunkArgs a;
     bool use_tc;
     const int pst = plan_chunk(B, T, H, d_k, d_v, chunk, dtype, gate, path, &a, &use_tc);
@@ -174,13 +174,23 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
         if (overlap(rst, r)) return fail(DN_ERR_INVALID, "S_T overlaps an input other than S0");
     if (S_T && S0 && (void*)S_T != (const void*)S0 && overlap(rst, rs0))
         return fail(DN_ERR_INVALID, "S_T partly overlaps S0");
+    // snapshots: the state after every `every` chunks, at full chunk boundaries only
+    if (snaps && every < 1) return fail(DN_ERR_INVALID, "every must be >= 1 (got %d)", every);
+    const int n_snap = snaps ? (int)(T / ((int64_t)every * chunk)) : 0;
+    Range rsn = rng(n_snap > 0 ? snaps : nullptr, (int64_t)B * H * n_snap * d_k * d_v * 4);
+    if (n_snap > 0) {
+        if (!aligned(snaps, 16)) return fail(DN_ERR_INVALID, "snaps is not 16-byte aligned");
+        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst};
+        for (Range r : all)
+            if (overlap(rsn, r)) return fail(DN_ERR_INVALID, "snaps overlaps another argument");
+    }
     const size_t need = workspace_needed(a, use_tc);
     if (workspace && need > 0) {
         if (workspace_bytes < need)
             return fail(DN_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
         if (!aligned(workspace, 256)) return fail(DN_ERR_INVALID, "workspace is not 256-byte aligned");
         Range rw = rng(workspace, (int64_t)need);
-        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst};
+        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst, rsn};
         for (Range r : all)
             if (overlap(rw, r)) return fail(DN_ERR_INVALID, "workspace overlaps another argument");
     }
@@ -190,6 +200,9 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
 
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T;
     a.scale = scale;
+    a.snaps = n_snap > 0 ? snaps : nullptr;
+    a.snap_every = every;
+    a.n_snap = n_snap;
 
     cudaError_t e;
     a.status = status_word(&e);
@@ -220,6 +233,24 @@ int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* be
         if (e == cudaSuccess) e = ef;
     }
     return e == cudaSuccess ? ok() : cuda_fail(e, "tensor-core chunk kernels");
+}
+
+int dn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+                    const float* g, const float* S0, void* o, float* S_T,
+                    int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                    dn_dtype dtype, dn_gate gate, dn_path path, void* workspace, size_t workspace_bytes,
+                    void* cuda_stream) {
+    return chunk_fwd_impl(q, k, v, beta, g, S0, o, S_T, B, T, H, d_k, d_v, chunk, scale, dtype, gate, path,
+                          workspace, workspace_bytes, cuda_stream, nullptr, 0);
+}
+
+int dn_chunk_fwd_snapshots(const void* q, const void* k, const void* v, const float* beta,
+                           const float* g, const float* S0, void* o, float* S_T, float* snaps, int every,
+                           int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                           dn_dtype dtype, dn_gate gate, dn_path path, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream) {
+    return chunk_fwd_impl(q, k, v, beta, g, S0, o, S_T, B, T, H, d_k, d_v, chunk, scale, dtype, gate, path,
+                          workspace, workspace_bytes, cuda_stream, snaps, every);
 }
 
 int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,

@@ -19,6 +19,8 @@ struct ChunkArgs {
     unsigned int* status;     // device status word of the current device
     int test_flags;           // 1: withhold the tensor-core kernels' input loads (failure-path self-test)
     void* ws;                 // tensor-core path: workspace of tc_workspace_bytes(), 256-byte aligned
+    float* snaps;             // null, or [B, H, n_snap, d_k, d_v]: the state after every snap_every chunks
+    int snap_every, n_snap;
 };
 
 struct DecodeArgs {

@@ -156,6 +156,28 @@ DN_API int dn_chunk_fwd_ex(const void* q, const void* k, const void* v,
                     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * dn_chunk_fwd_snapshots -- dn_chunk_fwd_ex that also writes the state at
+ * chunk boundaries.  An engine keeps such snapshots to roll a request back
+ * after rejected speculative tokens and to cache prefixes at block boundaries
+ * ("Linear attention and Gated DeltaNet", ch. 28, "The state a request
+ * carries").
+ *   snaps  NULL (no snapshots, as dn_chunk_fwd_ex) or [B,H,n_snap,d_k,d_v]
+ *          fp32, 16-byte aligned, overlapping no other argument, with
+ *          n_snap = floor(T / (every * chunk)): snapshot s is the state after
+ *          the first (s + 1) * every * chunk tokens of each (b, h), the value
+ *          S_T would have for that prefix.  A partial last chunk has none.
+ *   every  chunks between snapshots, >= 1 (DN_ERR_INVALID otherwise).
+ * Everything else is as for dn_chunk_fwd_ex.  On the tensor-core path each
+ * snapshot costs one extra write of 64 KiB per head.
+ */
+DN_API int dn_chunk_fwd_snapshots(const void* q, const void* k, const void* v,
+                                  const float* beta, const float* g, const float* S0,
+                                  void* o, float* S_T, float* snaps, int every,
+                                  int B, int T, int H, int d_k, int d_v, int chunk, float scale,
+                                  dn_dtype dtype, dn_gate gate, dn_path path,
+                                  void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * dn_chunk_fwd_noalloc -- dn_chunk_fwd for callers that cannot allocate device
  * memory (a process that reserved the device's memory for its own pools, a
  * framework whose allocator must see every byte, or a latency-critical loop
@@ -217,7 +239,8 @@ DN_API const char* dn_status_str(int status);
 /* Reason for the last non-DN_OK return on the calling thread ("" if none). */
 DN_API const char* dn_last_error(void);
 
-/* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path. */
+/* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path;
+ * 2.3: dn_chunk_fwd_snapshots. */
 DN_API int dn_version(void);
 
 /*

@@ -158,3 +158,27 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 1, 8, 64)
     with pytest.raises(ValueError):
         dn.dn_chunk_fwd(q, q, q, torch.zeros(1, 1, 8), None, None, torch.zeros(1, 1, 8, 64), None)
+
+
+def snap_call(lib, snaps, every, **over):
+    args = dict(q=A, k=A + STEP, v=A + 2 * STEP, beta=A + 3 * STEP, g=A + 4 * STEP, S0=None,
+                o=A + 5 * STEP, S_T=A + 6 * STEP, B=1, T=128, H=1, dk=64, dv=64, chunk=16,
+                scale=1.0, dtype=0, gate=1, path=1)
+    args.update(over)
+    return lib.dn_chunk_fwd_snapshots(args["q"], args["k"], args["v"], args["beta"], args["g"], args["S0"],
+                                      args["o"], args["S_T"], snaps, every, args["B"], args["T"], args["H"],
+                                      args["dk"], args["dv"], args["chunk"], args["scale"], args["dtype"],
+                                      args["gate"], args["path"], None, 0, None)
+
+
+@pytest.mark.parametrize("snaps,every,what", [
+    (A + 9 * STEP, 0, "every"),              # every must be >= 1
+    (A + 9 * STEP + 8, 1, "aligned"),        # not 16-byte aligned
+    (A + 2 * STEP + 64, 1, "overlaps"),      # overlaps v
+    (A + 6 * STEP, 2, "overlaps"),           # overlaps S_T
+])
+def test_chunk_snapshots_rejects(lib, snaps, every, what):
+    before = lib.dn_kernel_launches()
+    assert snap_call(lib, snaps, every) == dn.DN_ERR_INVALID
+    assert what in lib.dn_last_error().decode()
+    assert lib.dn_kernel_launches() == before

@@ -300,3 +300,39 @@ def test_kda_tc_matches_simt_path(cuda_device):
     dn.dn_device_status()
     assert_close(o1, f64(o2), "bf16", "o (tc vs simt)")
     assert_close(S1, f64(S2), "bf16", "S_T (tc vs simt)")
+
+
+def _prefix(inp, t_end):
+    """The same problem cut to its first t_end tokens (S0 unchanged)."""
+    out = {}
+    for name, t in inp.items():
+        out[name] = None if t is None or name == "S0" else t[:, :, :t_end].contiguous()
+    out["S0"] = inp["S0"]
+    return out
+
+
+@pytest.mark.parametrize("path,gate,chunk", [("simt", "scalar", 16), ("simt", "per_key", 64), ("tc", "none", 64),
+                                             ("tc", "scalar", 64), ("tc", "per_key", 64)])
+@pytest.mark.parametrize("T,every", [(300, 2), (256, 1)])
+def test_chunk_state_snapshots(cuda_device, path, gate, chunk, T, every):
+    # snapshot s is the state after the first (s + 1) * every * chunk tokens, i.e. the
+    # final state of that prefix (the oracle's S_T on the cut problem); a partial last
+    # chunk has none.  With T = 256 and every = 1 the last snapshot is S_T itself.
+    inp = W.gen_prefill(2, 3, T, 128, 128, dtype="bf16", gate=gate, seed=T + every, s0_std=0.2)
+    d = to_dev(inp)
+    sc = 128 ** -0.5
+    n_snap = T // (every * chunk)
+    snaps = torch.full((2, 3, n_snap, 128, 128), float("nan"), device="cuda")
+    o = torch.empty((2, 3, T, 128), dtype=torch.bfloat16, device="cuda")
+    S = torch.empty((2, 3, 128, 128), device="cuda")
+    dn.dn_chunk_fwd_snapshots(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o, S, snaps, every,
+                              chunk=chunk, scale=sc, path=path)
+    dn.dn_device_status()
+    ro, rS = oracle_prefill(inp, sc)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(S, rS, "bf16", "S_T")
+    for s in range(n_snap):
+        _, rs = oracle_prefill(_prefix(inp, (s + 1) * every * chunk), sc)
+        assert_close(snaps[:, :, s], rs, "bf16", f"snapshot {s}")
+    if T % (every * chunk) == 0:
+        assert torch.equal(snaps[:, :, -1], S)
