@@ -15,6 +15,8 @@ Contents
                           equations, used only to check the chunk algebra
                           against the sequential recurrence.
 ``wy_transition``         the WY form of one chunk's product of transitions.
+``gdn_prologue``          steps 4 and 5 of the Gated DeltaNet layer: unit q and
+                          k, beta = sigmoid(b), g = -exp(A_log) softplus(a + dt_bias).
 
 Every function takes and returns numpy arrays.  Layouts: tokens
 ``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
@@ -301,3 +303,26 @@ def wy_transition(k, beta, g=None):
     system = np.eye(C) + _strict_lower(beta[:, None] * kd)
     W = _solve_unit_lower(system, beta[:, None] * k * np.exp(Gam))
     return np.diag(np.exp(Gam[-1])) - (k * np.exp(Gam[-1][None, :] - Gam)).T @ W
+
+
+def gdn_prologue(q, k, b, a, A_log, dt_bias, eps=1e-12):
+    """Steps 4 and 5 of the Gated DeltaNet layer ("Linear attention and Gated
+    DeltaNet", ch. 28, "The full layer"), in fp64, on raw per-token inputs:
+
+    - q and k normalised over the head dimension, x / max(||x||_2, eps): the
+      pages call l2norm without defining it and elsewhere use the
+      F.normalize contract for unit keys, which this restates;
+    - beta = sigmoid(b), the write strength in (0, 1);
+    - g = -exp(A_log[h]) * softplus(a + dt_bias[h]), the log-decay (always
+      negative), with softplus(x) = log(1 + e^x) (numpy's logaddexp(0, x)).
+
+    q, k [B,H,T,d_k]; b, a [B,H,T]; A_log, dt_bias [H].  Returns
+    ``(q_hat, k_hat, beta, g)``; ``scale`` still applies to q_hat inside the
+    rule."""
+    q, k, b, a = _f64(q), _f64(k), _f64(b), _f64(a)
+    A_log, dt_bias = _f64(A_log), _f64(dt_bias)
+    qn = q / np.maximum(np.linalg.norm(q, axis=-1, keepdims=True), eps)
+    kn = k / np.maximum(np.linalg.norm(k, axis=-1, keepdims=True), eps)
+    beta = 1.0 / (1.0 + np.exp(-b))
+    g = -np.exp(A_log)[None, :, None] * np.logaddexp(0.0, a + dt_bias[None, :, None])
+    return qn, kn, beta, g

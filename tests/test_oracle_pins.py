@@ -364,3 +364,51 @@ def test_delta_columns_context_only():
     e_delta = np.mean(np.linalg.norm(K[last] @ S[0, 0] - V[last], axis=1) / np.linalg.norm(V[last], axis=1))
     e_add = np.mean(np.linalg.norm(K[last] @ Sa[0, 0] - V[last], axis=1) / np.linalg.norm(V[last], axis=1))
     assert e_delta < e_add
+
+
+# ---- the Gated DeltaNet layer's prologue ("The full layer", steps 4 and 5) -----------
+
+def test_gdn_prologue_closed_forms():
+    """sigmoid(0) = 1/2; softplus(0) = ln 2 so g = -e^A_log ln 2 at a + dt_bias = 0;
+    softplus(x) -> x for large x and -> e^x for very negative x; exp(A_log) scales g."""
+    B, H, T, d = 1, 2, 4, 8
+    q = np.ones((B, H, T, d)); k = np.ones((B, H, T, d))
+    b = np.array([0.0, 2.0, -2.0, 40.0])[None, None].repeat(H, axis=1)
+    a = np.array([0.0, 60.0, -60.0, 1.0])[None, None].repeat(H, axis=1)
+    A_log = np.array([0.0, np.log(2.0)]); dt_bias = np.zeros(H)
+    _, _, beta, g = oracle.gdn_prologue(q, k, b, a, A_log, dt_bias)
+    assert beta[0, 0, 0] == 0.5
+    assert np.isclose(beta[0, 0, 1], 1 / (1 + np.exp(-2.0)), rtol=0, atol=1e-15)
+    assert np.isclose(beta[0, 0, 1] + beta[0, 0, 2], 1.0, rtol=0, atol=1e-15)   # sigmoid(x) + sigmoid(-x) = 1
+    assert np.isclose(g[0, 0, 0], -np.log(2.0), rtol=1e-15)
+    assert np.isclose(g[0, 1, 0], -2 * np.log(2.0), rtol=1e-15)                   # exp(A_log) = 2
+    assert np.isclose(g[0, 0, 1], -60.0, rtol=1e-15)                              # softplus(60) = 60 + e^-60
+    assert np.isclose(g[0, 0, 2], -np.exp(-60.0), rtol=1e-12)                     # softplus(-60) ~ e^-60
+    assert np.isclose(g[0, 0, 3], -np.log1p(np.e), rtol=1e-15)
+    assert (g <= 0).all()
+
+
+def test_gdn_prologue_dt_bias_shifts_a():
+    rng = np.random.default_rng(3)
+    a = rng.standard_normal((2, 3, 5)); dtb = rng.standard_normal(3); A_log = rng.standard_normal(3)
+    q = rng.standard_normal((2, 3, 5, 4)); b = rng.standard_normal((2, 3, 5))
+    g1 = oracle.gdn_prologue(q, q, b, a + dtb[None, :, None], A_log, np.zeros(3))[3]
+    g2 = oracle.gdn_prologue(q, q, b, a, A_log, dtb)[3]
+    assert np.allclose(g1, g2, rtol=1e-15, atol=0)
+
+
+def test_gdn_prologue_unit_rows():
+    """Unit norm over the head dimension, invariant to a positive scale of the row,
+    direction kept; a zero row stays zero (the max(||x||, eps) clamp)."""
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((2, 2, 6, 16)); k = rng.standard_normal((2, 2, 6, 16))
+    q[0, 0, 0] = 0.0
+    b = np.zeros((2, 2, 6)); a = np.zeros((2, 2, 6)); p = np.zeros(2)
+    qn, kn, _, _ = oracle.gdn_prologue(q, k, b, a, p, p)
+    nq = np.linalg.norm(qn, axis=-1); nk = np.linalg.norm(kn, axis=-1)
+    assert np.allclose(nk, 1.0, rtol=0, atol=1e-15)
+    assert np.allclose(nq.ravel()[1:], 1.0, rtol=0, atol=1e-15) and nq[0, 0, 0] == 0.0
+    qn2, _, _, _ = oracle.gdn_prologue(7.5 * q, k, b, a, p, p)
+    assert np.allclose(qn2, qn, rtol=0, atol=1e-15)
+    cos = np.sum(qn[0, 1, 2] * q[0, 1, 2]) / np.linalg.norm(q[0, 1, 2])
+    assert np.isclose(cos, 1.0, rtol=0, atol=1e-15)
