@@ -302,7 +302,54 @@ def measure_prefill_configs(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
                          "timing": f"median of {calls} calls after {warm}, CUDA events"}
         del d, o, S_T, ws
         torch.cuda.empty_cache()
+    out["gated_deltanet_layer_prologue_bf16_B4_H16_T4096_d128"] = measure_gdn_prologue(dn, torch, W, peaks, dev,
+                                                                                        stream, calls, warm)
     return out
+
+
+def measure_gdn_prologue(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
+    """The bench-size Gated DeltaNet prefill with the layer's prologue fused in
+    (dn_chunk_fwd_gdn: raw q and k normalised inside, beta and g from the raw b,
+    a and the per-head A_log, dt_bias), same shape and timing as above."""
+    pc = W.GDN_PREFILL
+    gen = torch.Generator().manual_seed(pc.seed)
+    B, H, T, dk, dv = pc.B, pc.H, pc.T, pc.dk, pc.dv
+    q = (torch.randn(B, H, T, dk, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    k = (torch.randn(B, H, T, dk, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, H, T, dv, generator=gen).to(torch.bfloat16).to(dev)
+    b = torch.randn(B, H, T, generator=gen).to(dev)
+    a = torch.randn(B, H, T, generator=gen).to(dev)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen)).to(dev)
+    dt_bias = torch.randn(H, generator=gen).to(dev)
+    o = torch.empty((B, H, T, dv), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(dn.dn_chunk_fwd_workspace_size(B, T, H, dk, dv, path="tc"), dtype=torch.uint8, device=dev)
+
+    def call():
+        dn.dn_chunk_fwd_gdn(q, k, v, b, a, A_log, dt_bias, None, o, S_T, scale=pc.scale, workspace=ws,
+                            stream=stream)
+
+    for _ in range(warm):
+        call()
+    ts = []
+    for _ in range(calls):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    dn.dn_device_status(stream)
+    ms = statistics.median(ts)
+    fl = prefill_flops(B, H, T, dk, dv)
+    by = prefill_bytes(B, H, T, dk, dv) + 2 * H * 4
+    tf = fl / (ms * 1e-3) / 1e12
+    gb = by / (ms * 1e-3) / 1e9
+    return {"ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3), "path": "tensor cores, layer prologue fused",
+            "counted_flops": fl, "algorithmic_bytes": by, "tensor_tflops": tf,
+            "tensor_frac": tf / peaks["bf16_tflops"], "hbm_gbs": gb, "hbm_frac": gb / peaks["hbm_gbs"],
+            "traffic": None, "timing": f"median of {calls} calls after {warm}, CUDA events"}
 
 
 def workload_config():

@@ -116,6 +116,12 @@ struct Args {
     const float* gam;               // per-key gate: the workspace's e^Gamma_last per tile and channel
     float* snaps;                   // null, or [heads][n_snap][d_k][d_v]: the state after every
     int snap_every, n_snap;         //   snap_every chunks (full chunks only)
+    // the layer's prologue inside the kernels (scalar gate): beta and g hold the raw inputs
+    // b and a, q and k are normalised per row (per-head A_log, dt_bias; H heads per batch row)
+    int prologue;
+    const float* A_log;
+    const float* dt_bias;
+    int H;
 };
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
@@ -124,7 +130,8 @@ constexpr int G_KGAM = 0;
 // The state pass of head `head`, run by threads 0 .. kNT - 1 of a CTA whose
 // shared memory starts (1024-aligned) at sm.  HOSTED: the caller allocated the
 // TMEM (base tmem_given) and shares the SM with a WY group.
-template <int GATE, bool HOSTED>
+// PRO: the layer's prologue (raw gates, unit q and k) is compiled in (scalar gate).
+template <int GATE, bool HOSTED, bool PRO = false>
 __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head, uint32_t tmem_given) {
     using L = Layout<HOSTED>;
     constexpr int kStages = L::kStages;
@@ -183,6 +190,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
         constexpr bool KDA = GATE == kGatePerKey;
         // beta / g of the next chunk, loaded one chunk ahead
         float nb0 = 0.f, nb1 = 0.f, ng0 = 0.f, ng1 = 0.f;
+        const float eA = PRO ? expf(ar.A_log[bh % ar.H]) : 0.f;
+        const float dtb = PRO ? ar.dt_bias[bh % ar.H] : 0.f;
         auto fetch = [&](int cc) {
             const int64_t t0 = bh * T + (int64_t)cc * kC;
             const int Cn = min(kC, T - cc * kC);
@@ -191,6 +200,11 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             if (GATE == kGateScalar) {
                 ng0 = lane < Cn ? g[t0 + lane] : 0.f;
                 ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
+                if (PRO) {
+                    // beta and g from the raw inputs, as the WY side computes them
+                    if (lane < Cn) gdn_raw_gates(nb0, ng0, eA, dtb);
+                    if (lane + 32 < Cn) gdn_raw_gates(nb1, ng1, eA, dtb);
+                }
             }
         };
         if (!KDA) fetch(0);
@@ -321,19 +335,31 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
                 const int s = c % kStages;
                 const int Cc = min(kC, T - c * kC);
-                const float* gs = gates + (c & 3) * GATE_FLOATS;
+                float* gs = gates + (c & 3) * GATE_FLOATS;
                 const uint32_t st = sb + s * SZ_STAGE;
                 bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) &&
                           ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
+                if (PRO) {
+                    // 1 / ||q_i|| and 1 / ||k_i|| of the chunk from the stage's tiles, two
+                    // threads per row (read by the U epilogue after this chunk's READY)
+                    const int r = sid >> 1;
+                    const float rq = inv_row_norm(st + ST_B, r, sid & 1, 16384);
+                    const float rk = inv_row_norm(st + ST_K, r, sid & 1, 8192);
+                    if ((sid & 1) == 0) {
+                        gs[G_RQ + r] = rq;
+                        gs[G_RK + r] = rk;
+                    }
+                    named_bar_sync(1, kSideThreads);
+                }
                 // (with the per-key gate the workspace holds Qh already)
 #pragma unroll
                 for (int u = 0; u < (GATE == kGatePerKey ? 0 : 8); ++u) {
                     const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
                     const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
                     const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
-                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                    const float f = i < Cc ? (PRO ? scale * gs[G_EG + i] * gs[G_RQ + i] : scale * gs[G_EG + i]) : 0.f;
                     const uint4 w = ld_shared_v4(a);
                     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
                     const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
@@ -405,7 +431,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             const uint32_t st = sb + (c % kStages) * SZ_STAGE;
             // ---- U = u - W S -> bf16 pairs in TMEM, plain and decayed (U~), in two passes
             //      over positions 0-31 and 32-63 ------------------------------------------
-            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
+            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u) &&
+                 (!PRO || ctl.wait(B_READY0 + c % kStages, (uint32_t)(c / kStages) & 1u));
             if (!ok) *abort_flag = 1;
             if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
             tc_fence_after();
@@ -436,7 +463,12 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                     // decay and the KU product reads U^T itself
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        const float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
+                        float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
+                        if (PRO) {
+                            // times 1 / ||k_i||: K^T diag(1 / ||k||) U~ is K~^T U~ with unit keys
+                            const float4 rk = *reinterpret_cast<const float4*>(gsc + G_RK + i0 + 4 * q4);
+                            et.x *= rk.x; et.y *= rk.y; et.z *= rk.z; et.w *= rk.w;
+                        }
                         pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
                         pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
                     }

@@ -27,21 +27,22 @@ namespace dn {
 using namespace sm100;
 using namespace tc;
 
-template <int GATE>
+template <int GATE, bool PRO>
 __global__ void __launch_bounds__(state::kNT, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
                    const __grid_constant__ CUtensorMap tm_p, const unsigned int* __restrict__ flags,
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, float scale, unsigned int* status,
-                   int test_flags, const float* __restrict__ gam, float* snaps, int snap_every, int n_snap) {
+                   int test_flags, const float* __restrict__ gam, float* snaps, int snap_every, int n_snap,
+                   Prologue pro) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
-                         gam, snaps, snap_every, n_snap};
-    state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
+                         gam, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H};
+    state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
 }
 
 namespace {
@@ -57,7 +58,7 @@ static_assert(state::Layout<true>::kCols + wy::TM_COLS <= state::TM_COLS, "hoste
 constexpr uint32_t kHostBar = 6;                    // named barrier of the hosting CTA's state pass + WY group
 }  // namespace
 
-template <int GATE, bool HOSTED>
+template <int GATE, bool HOSTED, bool PRO>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
@@ -65,7 +66,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    __nv_bfloat16* __restrict__ p_out, unsigned int* __restrict__ flags, int BH,
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale, unsigned int* status,
-                   int test_flags, float* snaps, int snap_every, int n_snap) {
+                   int test_flags, float* snaps, int snap_every, int n_snap, Prologue pro) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -74,14 +75,14 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // the later ones come from tickets, in order (chunk-major), to whichever group is free
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
-                      flags + tiles, BH, (int)G};
+                      flags + tiles, BH, (int)G, pro.on, pro.A_log, pro.dt_bias, pro.H};
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, nullptr, snaps, snap_every, n_snap};
+                             test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H};
         if (!HOSTED) {
             // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
             if (warp >= state::kNT / 32) return;
-            state::state_pass<GATE, false>(sm, ar, blockIdx.x, 0u);
+            state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
             return;
         }
         // ---- state pass (warps 0-15) and one WY group (warps 16-23) ------------------------
@@ -102,14 +103,14 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tc_fence_after();
         const uint32_t tbase = *tslot;
         if (tid < state::kNT) {
-            state::state_pass<GATE, true>(sm, ar, blockIdx.x, tbase);
+            state::state_pass<GATE, true, PRO>(sm, ar, blockIdx.x, tbase);
         } else {
             x.tmem = tbase + state::Layout<true>::kCols;
             bool ok = true;
             int64_t pending = -1;
             for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles;) {
                 const int c = (int)(t / BH);
-                ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
+                ok = wy::wy_tile<GATE, PRO>(x, wa, c, t - (int64_t)c * BH, pending);
                 if (ok) t = G + (int64_t)wy::next_ticket(x);
             }
             if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
@@ -143,7 +144,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int64_t pending = -1;
     for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles;) {
         const int c = (int)(t / BH);
-        ok = wy::wy_tile<GATE>(x, wa, c, t - (int64_t)c * BH, pending);
+        ok = wy::wy_tile<GATE, PRO>(x, wa, c, t - (int64_t)c * BH, pending);
         if (ok) t = G + (int64_t)wy::next_ticket(x);
     }
     if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
@@ -180,7 +181,7 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_kt, &tm_qh, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, gam, snaps, snap_every, n_snap};
+                             test_flags, gam, snaps, snap_every, n_snap, 0, nullptr, nullptr, 1};
         state::state_pass<kGatePerKey, false>(sm, ar, blockIdx.x, 0u);
         return;
     }
@@ -230,7 +231,7 @@ bool fused_fits(int64_t BH, int num_sms) {
     return BH + 16 <= num_sms && BH * 4 <= (int64_t)num_sms * 3;
 }
 
-template <int GATE>
+template <int GATE, bool PRO>
 cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     const uint64_t rows = (uint64_t)(a.B * a.H * a.T);
     const int n = (int)((a.T + kC - 1) / kC);
@@ -255,7 +256,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     if (coop && fused_fits(BH, num_sms)) {
         // with many heads the dedicated WY groups get scarce: the state-pass CTAs
         // host one each (measured: at 64 heads of 148 SMs hosting is not yet a gain)
-        auto kern = BH * 2 > (int64_t)num_sms + 12 ? chunk_fused_kernel<GATE, true> : chunk_fused_kernel<GATE, false>;
+        auto kern = BH * 2 > (int64_t)num_sms + 12 ? chunk_fused_kernel<GATE, true, PRO> : chunk_fused_kernel<GATE, false, PRO>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedBytes);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
@@ -275,8 +276,9 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             unsigned int* status = a.status;
             float* snaps = a.snaps;
             int snap_every = a.snap_every, n_snap = a.n_snap;
+            Prologue pro{a.prologue ? 1 : 0, a.A_log, a.dt_bias, (int)a.H};
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
-                            &T_i, &n_i, &scale, &status, &test_flags, &snaps, &snap_every, &n_snap};
+                            &T_i, &n_i, &scale, &status, &test_flags, &snaps, &snap_every, &n_snap, &pro};
             // the flags are cleared on the same stream right before the launch
             e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
@@ -286,14 +288,15 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     }
     e = launch_chunk_wy(a, m, st);
     if (e != cudaSuccess) return e;
-    auto kern = chunk_state_kernel<GATE>;
+    auto kern = chunk_state_kernel<GATE, PRO>;
     const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     // the WY kernel has finished before this launch starts: no flags to wait for
     kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
-                                                  a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap);
+                                                  a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap,
+                                                  Prologue{a.prologue ? 1 : 0, a.A_log, a.dt_bias, (int)a.H});
     return counted(cudaGetLastError());
 }
 
@@ -363,14 +366,14 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     }
     e = launch_chunk_wy_kda(a, m, st);
     if (e != cudaSuccess) return e;
-    auto kern = chunk_state_kernel<kGatePerKey>;
+    auto kern = chunk_state_kernel<kGatePerKey, false>;
     const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(a.B * a.H), state::kNT, bytes, st>>>(m.kt, m.qh, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
                                                           a.scale, a.status, a.test_flags, m.gam_ws, a.snaps,
-                                                          a.snap_every, a.n_snap);
+                                                          a.snap_every, a.n_snap, Prologue{0, nullptr, nullptr, 1});
     return counted(cudaGetLastError());
 }
 
@@ -390,7 +393,8 @@ size_t tc_workspace_bytes(const ChunkArgs& a) {
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
     if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
     if (a.gate == kGatePerKey) return launch_tc_kda(a, st);
-    return a.gate == kGateScalar ? launch_tc_gate<kGateScalar>(a, st) : launch_tc_gate<kGateNone>(a, st);
+    if (a.prologue) return launch_tc_gate<kGateScalar, true>(a, st);   // the layer prologue: scalar gate
+    return a.gate == kGateScalar ? launch_tc_gate<kGateScalar, false>(a, st) : launch_tc_gate<kGateNone, false>(a, st);
 }
 
 }  // namespace dn

@@ -67,9 +67,50 @@ struct TcMaps {
     float* gam_ws;
 };
 
-// Gate slot of one chunk (floats).
-constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320;
-constexpr uint32_t GATE_FLOATS = 384;
+// The Gated DeltaNet layer's prologue, fused into the prefill kernels (scalar
+// gate): when `on`, the beta and g arrays hold the raw inputs b and a, and q
+// and k are normalised per row inside the kernels.
+struct Prologue {
+    int on;
+    const float* A_log;      // [H]
+    const float* dt_bias;    // [H]
+    int H;                   // heads per batch row (head of bh: bh % H)
+};
+
+// Gate slot of one chunk (floats).  G_RQ / G_RK: 1 / ||q_i|| and 1 / ||k_i||
+// when the layer's prologue normalises q and k inside the kernels, else 1.
+constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320, G_RQ = 384, G_RK = 448;
+constexpr uint32_t GATE_FLOATS = 512;
+
+// The Gated DeltaNet layer's gates from its raw per-token inputs ("Linear
+// attention and Gated DeltaNet", ch. 28, "The full layer", step 5): beta =
+// sigmoid(b), g = -exp(A_log) softplus(a + dt_bias), softplus(x) = log(1 + e^x)
+// (x above 20 taken as x).  eA = exp(A_log) of the head.
+__device__ __forceinline__ void gdn_raw_gates(float& b, float& a, float eA, float dt_bias) {
+    b = 1.f / (1.f + expf(-b));
+    const float x = a + dt_bias;
+    a = -eA * (x > 20.f ? x : log1pf(expf(x)));
+}
+
+// 1 / max(||x||, 1e-12) for a row of d_k = 128 bf16 values in a [rows][128 B]
+// tile pair with 128-byte swizzle (blocks of 64 columns `block_bytes` apart),
+// summed by two threads: this one takes the 64 columns of block `half`; the
+// partner (lane ^ 1) the other.
+__device__ __forceinline__ float inv_row_norm(uint32_t tile, int row, int half, uint32_t block_bytes) {
+    float ss = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        const uint4 w = ld_shared_v4(tile + (uint32_t)half * block_bytes + sw128_off(row, ch));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            ss += f.x * f.x + f.y * f.y;
+        }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    return 1.f / fmaxf(sqrtf(ss), 1e-12f);
+}
 
 // Gates of one chunk from beta and g at positions lane and lane + 32 (zero past
 // the chunk's end, which makes those positions identity steps).  G is the

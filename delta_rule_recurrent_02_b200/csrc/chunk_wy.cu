@@ -11,13 +11,14 @@ using namespace sm100;
 using namespace tc;
 using namespace wy;
 
-template <int GATE>
+template <int GATE, bool PRO>
 __global__ void __launch_bounds__(kNT, 4)
 chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
                 const __grid_constant__ CUtensorMap tm_u, __nv_bfloat16* __restrict__ p_out,
                 unsigned int* __restrict__ flags, int BH, const float* __restrict__ beta,
-                const float* __restrict__ g, int T, int n, float scale, unsigned int* status, int test_flags) {
+                const float* __restrict__ g, int T, int n, float scale, unsigned int* status, int test_flags,
+                Prologue pro) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
@@ -38,12 +39,12 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     x.tmem = *tmem_slot;
     const Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags, nullptr,
-                  BH, 0};
+                  BH, 0, pro.on, pro.A_log, pro.dt_bias, pro.H};
     // chunk-major order: chunk 0 of every head first
     const int c = (int)(blockIdx.x / (unsigned)BH);
     const int64_t bh = blockIdx.x - (int64_t)c * BH;
     int64_t pending = -1;
-    const bool ok = wy_tile<GATE>(x, ar, c, bh, pending);
+    const bool ok = wy_tile<GATE, PRO>(x, ar, c, bh, pending);
     if (ok && tid == kStoreTid) publish_pending(ar, pending);
     tc_fence_before();
     __syncthreads();
@@ -60,14 +61,15 @@ namespace {
 
 constexpr uint32_t SMEM_BYTES = GROUP_BYTES + 1024;
 
-template <int GATE>
+template <int GATE, bool PRO>
 cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStream_t st) {
-    auto kern = chunk_wy_kernel<GATE>;
+    auto kern = chunk_wy_kernel<GATE, PRO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(a.B * a.H * n), kNT, SMEM_BYTES, st>>>(m.q, m.k, m.v, m.w, m.u, m.p_ws, m.flags,
                                                               (int)(a.B * a.H), a.beta, a.g, (int)a.T, n, a.scale,
-                                                              a.status, a.test_flags);
+                                                              a.status, a.test_flags,
+                                                              Prologue{a.prologue ? 1 : 0, a.A_log, a.dt_bias, (int)a.H});
     return counted(cudaGetLastError());
 }
 
@@ -75,7 +77,9 @@ cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStrea
 
 cudaError_t launch_chunk_wy(const ChunkArgs& a, const TcMaps& m, cudaStream_t st) {
     const int n = (int)((a.T + kC - 1) / kC);
-    return a.gate == kGateScalar ? launch_wy_gate<kGateScalar>(a, m, n, st) : launch_wy_gate<kGateNone>(a, m, n, st);
+    if (a.prologue) return launch_wy_gate<kGateScalar, true>(a, m, n, st);
+    return a.gate == kGateScalar ? launch_wy_gate<kGateScalar, false>(a, m, n, st)
+                                 : launch_wy_gate<kGateNone, false>(a, m, n, st);
 }
 
 }  // namespace dn

@@ -73,7 +73,7 @@ constexpr uint32_t OFF_TW = OFF_A;      //   T diag(beta e^G), K-major B [N=i][K
 constexpr uint32_t OFF_TB = OFF_A + 8192;   // T diag(beta), same layout
 constexpr uint32_t OFF_GATE = OFF_A + 17408;   // one gate slot
 constexpr uint32_t OFF_BAR = OFF_GATE + GATE_FLOATS * 4;
-constexpr uint32_t GROUP_BYTES = 53248;  // one group's shared memory, a multiple of 1024
+constexpr uint32_t GROUP_BYTES = 54272;  // one group's shared memory, a multiple of 1024
 // (the last 16 bytes of a group stay free: a CTA keeps its TMEM address there)
 static_assert(OFF_BAR + 64 <= GROUP_BYTES - 16, "group layout");
 static_assert(OFF_T + 64 * 68 * 4 <= OFF_V && OFF_V + 16384 <= OFF_A, "T, V and A overlap");
@@ -176,6 +176,12 @@ struct Args {
     int test_flags;
     unsigned int* counter;   // tile counter of the single launch (null: the caller picks every tile)
     int BH, G;               // with a counter: heads and WY groups (a ticket x is tile G + x)
+    // the layer's prologue inside the kernels: beta and g hold the raw inputs b and a,
+    // q and k are normalised per row (the per-head A_log, dt_bias; H heads per batch row)
+    int prologue;
+    const float* A_log;
+    const float* dt_bias;
+    int H;
 };
 
 // Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
@@ -295,7 +301,8 @@ __device__ __forceinline__ void publish_pending(const Args& ar, int64_t& pending
 // ticket, prefetches that tile's inputs into L2, and hands the ticket on
 // (next_ticket() once this returns).  Returns false (the group's
 // abort flag set) if a wait gave up.
-template <int GATE>
+// PRO: the layer's prologue (raw gates, unit q and k) is compiled in.
+template <int GATE, bool PRO = false>
 __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, int64_t bh, int64_t& pending) {
     const uint32_t sb = x.sb;
     float* gs = reinterpret_cast<float*>(x.sm + OFF_GATE);
@@ -335,12 +342,19 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         loads = 1;
     }
     if (warp == 2) {
-        const float b0 = lane < Cc ? beta[t0 + lane] : 0.f;
-        const float b1 = lane + 32 < Cc ? beta[t0 + lane + 32] : 0.f;
+        float b0 = lane < Cc ? beta[t0 + lane] : 0.f;
+        float b1 = lane + 32 < Cc ? beta[t0 + lane + 32] : 0.f;
         float a0 = 0.f, a1 = 0.f;
         if (GATE == kGateScalar) {
             a0 = lane < Cc ? g[t0 + lane] : 0.f;
             a1 = lane + 32 < Cc ? g[t0 + lane + 32] : 0.f;
+        }
+        if (PRO) {
+            // beta and g from the raw inputs (positions past the end stay identity steps)
+            const int h = (int)(bh % ar.H);
+            const float eA = expf(ar.A_log[h]), dtb = ar.dt_bias[h];
+            if (lane < Cc) gdn_raw_gates(b0, a0, eA, dtb);
+            if (lane + 32 < Cc) gdn_raw_gates(b1, a1, eA, dtb);
         }
         chunk_gates(gs, b0, b1, a0, a1, lane);
     }
@@ -357,6 +371,17 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                 mma_bf16(tmem + TM_G, sw128_desc(a, 16, 1024), sw128_desc(a, 16, 1024), idesc, kk > 0);
             }
             mma_commit(ctl.bar(B_MMA));
+        }
+    }
+    if (PRO) {
+        // 1 / ||k_i|| and 1 / ||q_i|| from the tiles (rows 0-63 K, 64-127 Q of each d-block),
+        // two threads per row, while the gram runs
+        if (ctl.wait(B_FULL, 0)) {
+            const int r = tid >> 1;
+            const float rn = inv_row_norm(sb + OFF_KV, r, tid & 1, 16384);
+            if ((tid & 1) == 0) gs[r < 64 ? G_RK + r : G_RQ + r - 64] = rn;
+        } else {
+            ok = false;
         }
     }
     named_bar_sync(x.bar, kNT);                       // gates visible
@@ -387,16 +412,22 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             float v[32];
             tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
             tmem_wait_ld();
-            const float bi = gs[G_BETA + i];          // zero past the chunk's end
+            const float bi = PRO ? gs[G_BETA + i] * gs[G_RK + i] : gs[G_BETA + i];   // zero past the chunk's end
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
                 const float4 gj = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 4 * q4);
                 const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+                float rkv[4] = {1.f, 1.f, 1.f, 1.f};
+                if (PRO) {
+                    const float4 rk = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 4 * q4);
+                    rkv[0] = rk.x; rkv[1] = rk.y; rkv[2] = rk.z; rkv[3] = rk.w;
+                }
                 float a[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j0 + 4 * q4 + e;
-                    a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                    const float vv = PRO ? v[4 * q4 + e] * rkv[e] : v[4 * q4 + e];
+                    a[e] = j < i ? bi * vv * decay2(g2i, gjv[e]) : 0.f;
                 }
                 *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
             }
@@ -417,17 +448,25 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
                 tmem_wait_ld();
-                const float si = i < Cc ? scale : 0.f;
+                const float si = i < Cc ? (PRO ? scale * gs[G_RQ + i] : scale) : 0.f;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
                     const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
                     const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    float rkv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                    if (PRO) {
+                        const float4 ra = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 8 * q4);
+                        const float4 rb = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 8 * q4 + 4);
+                        rkv[0] = ra.x; rkv[1] = ra.y; rkv[2] = ra.z; rkv[3] = ra.w;
+                        rkv[4] = rb.x; rkv[5] = rb.y; rkv[6] = rb.z; rkv[7] = rb.w;
+                    }
                     float pv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = j0 + 8 * q4 + e;
-                        pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                        const float vv = PRO ? v[8 * q4 + e] * rkv[e] : v[8 * q4 + e];
+                        pv[e] = j <= i ? si * vv * decay2(g2i, gjv[e]) : 0.f;
                     }
                     st_global_v4(prow + 8 * q4, pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
                                  pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
@@ -455,8 +494,15 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         if ((ch >> 1) <= (i >> 4)) {
             const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
             const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
-            const float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
-            const float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
+            float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
+            float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
+            if (PRO) {
+                // T diag(beta e^G / ||k||): W = T diag(beta e^G) K / ||k|| by rows of K
+                const float4 r0 = *reinterpret_cast<const float4*>(gs + G_RK + 8 * ch);
+                const float4 r1 = *reinterpret_cast<const float4*>(gs + G_RK + 8 * ch + 4);
+                e0.x *= r0.x; e0.y *= r0.y; e0.z *= r0.z; e0.w *= r0.w;
+                e1.x *= r1.x; e1.y *= r1.y; e1.z *= r1.z; e1.w *= r1.w;
+            }
             const float4 c0 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch);
             const float4 c1 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch + 4);
             w4[0] = pack_bf16x2(t0v.x * e0.x, t0v.y * e0.y); w4[1] = pack_bf16x2(t0v.z * e0.z, t0v.w * e0.w);

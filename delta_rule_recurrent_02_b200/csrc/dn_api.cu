@@ -108,7 +108,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 3; }
+int dn_version(void) { return (2 << 16) | 4; }
 
 unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 
@@ -140,7 +140,8 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
                     const float* g, const float* S0, void* o, float* S_T,
                     int B, int T, int H, int d_k, int d_v, int chunk, float scale,
                     dn_dtype dtype, dn_gate gate, dn_path path, void* workspace, size_t workspace_bytes,
-                    void* cuda_stream, float* snaps, int every) {
+                    void* cuda_stream, float* snaps, int every, const float* A_log = nullptr,
+                    const float* dt_bias = nullptr) {
     dn::ChunkArgs a;
     bool use_tc;
     const int pst = plan_chunk(B, T, H, d_k, d_v, chunk, dtype, gate, path, &a, &use_tc);
@@ -174,6 +175,15 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
         if (overlap(rst, r)) return fail(DN_ERR_INVALID, "S_T overlaps an input other than S0");
     if (S_T && S0 && (void*)S_T != (const void*)S0 && overlap(rst, rs0))
         return fail(DN_ERR_INVALID, "S_T partly overlaps S0");
+    // the layer prologue (dn_chunk_fwd_gdn): beta and g hold the raw b and a
+    const bool pro = A_log != nullptr || dt_bias != nullptr;
+    Range rpa = rng(A_log, (int64_t)H * 4), rpd = rng(dt_bias, (int64_t)H * 4);
+    if (pro) {
+        if (!A_log || !dt_bias) return fail(DN_ERR_INVALID, "A_log and dt_bias are both required");
+        if (!aligned(A_log, 4) || !aligned(dt_bias, 4)) return fail(DN_ERR_INVALID, "A_log and dt_bias must be 4-byte aligned");
+        if (overlap(ro, rpa) || overlap(ro, rpd) || overlap(rst, rpa) || overlap(rst, rpd))
+            return fail(DN_ERR_INVALID, "o or S_T overlaps A_log or dt_bias");
+    }
     // snapshots: the state after every `every` chunks, at full chunk boundaries only
     if (snaps && every < 1) return fail(DN_ERR_INVALID, "every must be >= 1 (got %d)", every);
     const int n_snap = snaps ? (int)(T / ((int64_t)every * chunk)) : 0;
@@ -190,7 +200,7 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
             return fail(DN_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
         if (!aligned(workspace, 256)) return fail(DN_ERR_INVALID, "workspace is not 256-byte aligned");
         Range rw = rng(workspace, (int64_t)need);
-        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst, rsn};
+        Range all[] = {rq, rk, rv, rb, rg, rs0, ro, rst, rsn, rpa, rpd};
         for (Range r : all)
             if (overlap(rw, r)) return fail(DN_ERR_INVALID, "workspace overlaps another argument");
     }
@@ -203,6 +213,9 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const flo
     a.snaps = n_snap > 0 ? snaps : nullptr;
     a.snap_every = every;
     a.n_snap = n_snap;
+    a.prologue = pro;
+    a.A_log = A_log;
+    a.dt_bias = dt_bias;
 
     cudaError_t e;
     a.status = status_word(&e);
@@ -251,6 +264,15 @@ int dn_chunk_fwd_snapshots(const void* q, const void* k, const void* v, const fl
                            void* cuda_stream) {
     return chunk_fwd_impl(q, k, v, beta, g, S0, o, S_T, B, T, H, d_k, d_v, chunk, scale, dtype, gate, path,
                           workspace, workspace_bytes, cuda_stream, snaps, every);
+}
+
+int dn_chunk_fwd_gdn(const void* q, const void* k, const void* v, const float* b, const float* a,
+                     const float* A_log, const float* dt_bias, const float* S0, void* o, float* S_T,
+                     int B, int T, int H, int d_k, int d_v, float scale,
+                     void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    if (!A_log || !dt_bias) return fail(DN_ERR_INVALID, "A_log and dt_bias are required");
+    return chunk_fwd_impl(q, k, v, b, a, S0, o, S_T, B, T, H, d_k, d_v, 64, scale, DN_BF16, DN_GATE_SCALAR,
+                          DN_PATH_TC, workspace, workspace_bytes, cuda_stream, nullptr, 0, A_log, dt_bias);
 }
 
 int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,

@@ -21,6 +21,11 @@ struct ChunkArgs {
     void* ws;                 // tensor-core path: workspace of tc_workspace_bytes(), 256-byte aligned
     float* snaps;             // null, or [B, H, n_snap, d_k, d_v]: the state after every snap_every chunks
     int snap_every, n_snap;
+    // the layer's prologue inside the kernels (tensor-core path, scalar gate): beta and g
+    // hold the raw b and a; q and k are normalised per row
+    bool prologue;
+    const float* A_log;       // [H]
+    const float* dt_bias;     // [H]
 };
 
 struct DecodeArgs {

@@ -178,6 +178,26 @@ DN_API int dn_chunk_fwd_snapshots(const void* q, const void* k, const void* v,
                                   void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * dn_chunk_fwd_gdn -- the Gated DeltaNet prefill with the layer's prologue
+ * fused into the kernels ("Linear attention and Gated DeltaNet", ch. 28, "The
+ * full layer", steps 4 and 5): the rule runs on
+ *   q / max(||q||, 1e-12), k / max(||k||, 1e-12)  (norms over d_k, per token),
+ *   beta = sigmoid(b),  g = -exp(A_log[h]) * softplus(a + dt_bias[h])
+ * (softplus(x) = log(1 + e^x)), as dn_chunk_fwd with the scalar gate on these.
+ *   q, k  [B,H,T,d_k] bf16, raw (not normalised);  v [B,H,T,d_v] bf16
+ *   b, a  [B,H,T] fp32 raw write-strength and decay inputs, 4-byte aligned
+ *   A_log, dt_bias  [H] fp32 per head, 4-byte aligned, required
+ *   S0, o, S_T, scale, workspace, workspace_bytes, cuda_stream as dn_chunk_fwd_ex
+ * Tensor-core path only: d_k = d_v = 128 (chunk 64); DN_ERR_UNSUPPORTED
+ * otherwise.  The workspace is the scalar gate's (dn_chunk_fwd_workspace_size
+ * with DN_BF16, DN_GATE_SCALAR, DN_PATH_TC).
+ */
+DN_API int dn_chunk_fwd_gdn(const void* q, const void* k, const void* v, const float* b, const float* a,
+                            const float* A_log, const float* dt_bias, const float* S0, void* o, float* S_T,
+                            int B, int T, int H, int d_k, int d_v, float scale,
+                            void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * dn_chunk_fwd_noalloc -- dn_chunk_fwd for callers that cannot allocate device
  * memory (a process that reserved the device's memory for its own pools, a
  * framework whose allocator must see every byte, or a latency-critical loop
@@ -240,7 +260,7 @@ DN_API const char* dn_status_str(int status);
 DN_API const char* dn_last_error(void);
 
 /* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path;
- * 2.3: dn_chunk_fwd_snapshots. */
+ * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn. */
 DN_API int dn_version(void);
 
 /*

@@ -182,3 +182,27 @@ def test_chunk_snapshots_rejects(lib, snaps, every, what):
     assert snap_call(lib, snaps, every) == dn.DN_ERR_INVALID
     assert what in lib.dn_last_error().decode()
     assert lib.dn_kernel_launches() == before
+
+
+def gdn_call(lib, **over):
+    args = dict(q=A, k=A + STEP, v=A + 2 * STEP, b=A + 3 * STEP, a=A + 4 * STEP, A_log=A + 10 * STEP,
+                dt_bias=A + 11 * STEP, S0=None, o=A + 5 * STEP, S_T=A + 6 * STEP, B=1, T=128, H=2, dk=128, dv=128)
+    args.update(over)
+    return lib.dn_chunk_fwd_gdn(args["q"], args["k"], args["v"], args["b"], args["a"], args["A_log"],
+                                args["dt_bias"], args["S0"], args["o"], args["S_T"], args["B"], args["T"],
+                                args["H"], args["dk"], args["dv"], 1.0, None, 0, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(A_log=None), dn.DN_ERR_INVALID),
+    (dict(dt_bias=None), dn.DN_ERR_INVALID),
+    (dict(A_log=A + 10 * STEP + 2), dn.DN_ERR_INVALID),     # not 4-byte aligned
+    (dict(dt_bias=A + 5 * STEP + 4), dn.DN_ERR_INVALID),    # inside o
+    (dict(dk=64, dv=64), dn.DN_ERR_UNSUPPORTED),            # tensor-core path only
+    (dict(a=None), dn.DN_ERR_INVALID),                      # the raw decay input is required
+])
+def test_gdn_layer_rejects(lib, over, code):
+    before = lib.dn_kernel_launches()
+    assert gdn_call(lib, **over) == code
+    assert lib.dn_last_error() != b""
+    assert lib.dn_kernel_launches() == before

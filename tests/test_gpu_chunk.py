@@ -336,3 +336,61 @@ def test_chunk_state_snapshots(cuda_device, path, gate, chunk, T, every):
         assert_close(snaps[:, :, s], rs, "bf16", f"snapshot {s}")
     if T % (every * chunk) == 0:
         assert torch.equal(snaps[:, :, -1], S)
+
+
+def _gdn_raw(B, H, T, seed, zero_rows=False):
+    """Raw layer inputs: q and k of varied norms (not normalised), b and a ~ N(0,1),
+    A_log = log U(1, 16), dt_bias ~ N(0, 0.5)."""
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, T, 128, generator=gen) * (0.2 + 3 * torch.rand(B, H, T, 1, generator=gen))
+    k = torch.randn(B, H, T, 128, generator=gen) * (0.2 + 3 * torch.rand(B, H, T, 1, generator=gen))
+    if zero_rows:
+        q[0, 0, 5] = 0.0
+        k[0, 0, 7] = 0.0
+    v = torch.randn(B, H, T, 128, generator=gen)
+    b = torch.randn(B, H, T, generator=gen)
+    a = torch.randn(B, H, T, generator=gen)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen))
+    dt_bias = 0.5 * torch.randn(H, generator=gen)
+    S0 = 0.2 * torch.randn(B, H, 128, 128, generator=gen)
+    return {"q": q.to(torch.bfloat16), "k": k.to(torch.bfloat16), "v": v.to(torch.bfloat16), "b": b, "a": a,
+            "A_log": A_log, "dt_bias": dt_bias, "S0": S0}
+
+
+def _gdn_oracle(raw, scale, bh=None):
+    qn, kn, beta, g = oracle.gdn_prologue(f64(raw["q"]), f64(raw["k"]), f64(raw["b"]), f64(raw["a"]),
+                                          f64(raw["A_log"]), f64(raw["dt_bias"]))
+    inp = {"q": torch.from_numpy(qn), "k": torch.from_numpy(kn), "v": raw["v"], "beta": torch.from_numpy(beta),
+           "g": torch.from_numpy(g), "S0": raw["S0"]}
+    return oracle_prefill(inp, scale, bh=bh)
+
+
+@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 2, 64), (3, 32, 200), (4, 32, 130)])
+def test_gdn_layer_prologue(cuda_device, B, H, T):
+    # 6 heads and 2 heads: the single launch; 96 heads: hosted WY groups; 128 heads: two launches
+    raw = _gdn_raw(B, H, T, seed=B * 100 + H + T, zero_rows=True)
+    d = to_dev(raw)
+    sc = 128 ** -0.5
+    o = torch.full((B, H, T, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    S = torch.full((B, H, 128, 128), float("nan"), device="cuda")
+    dn.dn_chunk_fwd_gdn(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], d["S0"], o, S, scale=sc)
+    dn.dn_device_status()
+    bh = None if B * H <= 8 else [(0, 0), (B - 1, H - 1), (B // 2, 5)]
+    ro, rS = _gdn_oracle(raw, sc, bh=bh)
+    assert_close(o if bh is None else pick(o, bh), ro, "bf16", "o")
+    assert_close(S if bh is None else pick(S, bh), rS, "bf16", "S_T")
+
+
+def test_gdn_layer_prologue_full_size_sampled(cuda_device):
+    B, H, T = 4, 16, 4096
+    raw = _gdn_raw(B, H, T, seed=9)
+    d = to_dev(raw)
+    sc = 128 ** -0.5
+    o = torch.empty((B, H, T, 128), dtype=torch.bfloat16, device="cuda")
+    S = torch.empty((B, H, 128, 128), device="cuda")
+    dn.dn_chunk_fwd_gdn(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], d["S0"], o, S, scale=sc)
+    dn.dn_device_status()
+    bh = [(0, 0), (3, 15), (1, 7)]
+    ro, rS = _gdn_oracle(raw, sc, bh=bh)
+    assert_close(pick(o.cpu(), bh), ro, "bf16", "o (sampled heads)")
+    assert_close(pick(S.cpu(), bh), rS, "bf16", "S_T (sampled heads)")
