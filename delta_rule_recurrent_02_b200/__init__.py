@@ -25,7 +25,7 @@ import ctypes
 import os
 
 __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
-           "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn",
+           "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
            "dn_decode_step", "dn_kernel_launches",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
@@ -36,7 +36,7 @@ _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
-               "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn",
+               "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
                "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version",
                "dn_kernel_launches")
 
@@ -74,6 +74,8 @@ def load_library():
     lib.dn_chunk_fwd_snapshots.restype = I
     lib.dn_chunk_fwd_gdn.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, I, I, I, I, I, F, vp, Z, vp]
     lib.dn_chunk_fwd_gdn.restype = I
+    lib.dn_decode_step_gdn.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, I, I, I, I, F, I, vp]
+    lib.dn_decode_step_gdn.restype = I
     lib.dn_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I, ctypes.POINTER(Z)]
     lib.dn_chunk_fwd_workspace_size.restype = I
     lib.dn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp]
@@ -208,6 +210,20 @@ def dn_chunk_fwd_gdn(q, k, v, b, a, A_log, dt_bias, S0, o, S_T, *, scale: float 
     st = lib.dn_chunk_fwd_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias), _ptr(S0),
                               _ptr(o), _ptr(S_T), B, T, H, dk, dv, float(scale), _ptr(workspace), ws_bytes,
                               _stream(stream))
+    _check(lib, st)
+
+
+def dn_decode_step_gdn(q, k, v, b, a, A_log, dt_bias, S, o, *, scale: float = 1.0, stream=None) -> None:
+    """One decode step with the Gated DeltaNet layer's prologue fused in, through
+    ``dn_decode_step_gdn``: q and k [B, H, d] raw, b and a [B, H] raw, A_log and
+    dt_bias [H]; updates S in place and writes o."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for t in (b, a, A_log, dt_bias, S):
+        _f32(t)
+    st = lib.dn_decode_step_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias), _ptr(S),
+                                _ptr(o), B, H, dk, dv, float(scale), _dtype_code(q), _stream(stream))
     _check(lib, st)
 
 

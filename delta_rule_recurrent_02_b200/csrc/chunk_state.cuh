@@ -200,19 +200,21 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             if (GATE == kGateScalar) {
                 ng0 = lane < Cn ? g[t0 + lane] : 0.f;
                 ng1 = lane + 32 < Cn ? g[t0 + lane + 32] : 0.f;
-                if (PRO) {
-                    // beta and g from the raw inputs, as the WY side computes them
-                    if (lane < Cn) gdn_raw_gates(nb0, ng0, eA, dtb);
-                    if (lane + 32 < Cn) gdn_raw_gates(nb1, ng1, eA, dtb);
-                }
             }
         };
         if (!KDA) fetch(0);
         for (int cc = 0; cc < n; ++cc) {
             const int s = cc % kStages;
             if (!KDA) {
-                const float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
+                float b0 = nb0, b1 = nb1, a0 = ng0, a1 = ng1;
                 if (cc + 1 < n) fetch(cc + 1);
+                if (PRO) {
+                    // beta and g from the raw inputs, as the WY side computes them (here, one
+                    // chunk after the loads were issued, so their latency stays hidden)
+                    const int Cn = min(kC, T - cc * kC);
+                    if (lane < Cn) gdn_raw_gates(b0, a0, eA, dtb);
+                    if (lane + 32 < Cn) gdn_raw_gates(b1, a1, eA, dtb);
+                }
                 chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));

@@ -82,16 +82,6 @@ struct Prologue {
 constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320, G_RQ = 384, G_RK = 448;
 constexpr uint32_t GATE_FLOATS = 512;
 
-// The Gated DeltaNet layer's gates from its raw per-token inputs ("Linear
-// attention and Gated DeltaNet", ch. 28, "The full layer", step 5): beta =
-// sigmoid(b), g = -exp(A_log) softplus(a + dt_bias), softplus(x) = log(1 + e^x)
-// (x above 20 taken as x).  eA = exp(A_log) of the head.
-__device__ __forceinline__ void gdn_raw_gates(float& b, float& a, float eA, float dt_bias) {
-    b = 1.f / (1.f + expf(-b));
-    const float x = a + dt_bias;
-    a = -eA * (x > 20.f ? x : log1pf(expf(x)));
-}
-
 // 1 / max(||x||, 1e-12) for a row of d_k = 128 bf16 values in a [rows][128 B]
 // tile pair with 128-byte swizzle (blocks of 64 columns `block_bytes` apart),
 // summed by two threads: this one takes the 64 columns of block `half`; the

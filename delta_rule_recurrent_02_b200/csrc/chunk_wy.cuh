@@ -385,6 +385,15 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         }
     }
     named_bar_sync(x.bar, kNT);                       // gates visible
+    if (PRO && tid < kC) {
+        // the key norms enter the gram as a column factor folded into the decay,
+        // rk_j 2^(G2_i - G2_j) = 2^(G2_i - (G2_j - log2 rk_j)): the shifted column
+        // table goes where e^(G_last - G) was (the state pass's, unused here), and
+        // T diag(beta e^G) takes rk_j by scaling beta e^G
+        const float rk = gs[G_RK + tid];
+        gs[G_ET + tid] = gs[G_G2 + tid] - log2f(rk);
+        gs[G_BEG + tid] *= rk;
+    }
     ok = ok && ctl.wait(B_MMA, 0);
     if (named_bar_any(x.bar, kNT, !ok)) goto done;
     tc_fence_after();
@@ -413,21 +422,16 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
             tmem_wait_ld();
             const float bi = PRO ? gs[G_BETA + i] * gs[G_RK + i] : gs[G_BETA + i];   // zero past the chunk's end
+            const float* g2c = gs + (PRO ? G_ET : G_G2);   // column table (with the key norms folded in)
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
-                const float4 gj = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 4 * q4);
+                const float4 gj = *reinterpret_cast<const float4*>(g2c + j0 + 4 * q4);
                 const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
-                float rkv[4] = {1.f, 1.f, 1.f, 1.f};
-                if (PRO) {
-                    const float4 rk = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 4 * q4);
-                    rkv[0] = rk.x; rkv[1] = rk.y; rkv[2] = rk.z; rkv[3] = rk.w;
-                }
                 float a[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j0 + 4 * q4 + e;
-                    const float vv = PRO ? v[4 * q4 + e] * rkv[e] : v[4 * q4 + e];
-                    a[e] = j < i ? bi * vv * decay2(g2i, gjv[e]) : 0.f;
+                    a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
                 }
                 *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
             }
@@ -449,24 +453,17 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                 tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
                 tmem_wait_ld();
                 const float si = i < Cc ? (PRO ? scale * gs[G_RQ + i] : scale) : 0.f;
+                const float* g2c = gs + (PRO ? G_ET : G_G2);   // column table (with the key norms folded in)
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 ga = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4);
-                    const float4 gb = *reinterpret_cast<const float4*>(gs + G_G2 + j0 + 8 * q4 + 4);
+                    const float4 ga = *reinterpret_cast<const float4*>(g2c + j0 + 8 * q4);
+                    const float4 gb = *reinterpret_cast<const float4*>(g2c + j0 + 8 * q4 + 4);
                     const float gjv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                    float rkv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
-                    if (PRO) {
-                        const float4 ra = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 8 * q4);
-                        const float4 rb = *reinterpret_cast<const float4*>(gs + G_RK + j0 + 8 * q4 + 4);
-                        rkv[0] = ra.x; rkv[1] = ra.y; rkv[2] = ra.z; rkv[3] = ra.w;
-                        rkv[4] = rb.x; rkv[5] = rb.y; rkv[6] = rb.z; rkv[7] = rb.w;
-                    }
                     float pv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = j0 + 8 * q4 + e;
-                        const float vv = PRO ? v[8 * q4 + e] * rkv[e] : v[8 * q4 + e];
-                        pv[e] = j <= i ? si * vv * decay2(g2i, gjv[e]) : 0.f;
+                        pv[e] = j <= i ? si * v[8 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
                     }
                     st_global_v4(prow + 8 * q4, pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
                                  pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
@@ -494,15 +491,9 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         if ((ch >> 1) <= (i >> 4)) {
             const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
             const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
-            float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
-            float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
-            if (PRO) {
-                // T diag(beta e^G / ||k||): W = T diag(beta e^G) K / ||k|| by rows of K
-                const float4 r0 = *reinterpret_cast<const float4*>(gs + G_RK + 8 * ch);
-                const float4 r1 = *reinterpret_cast<const float4*>(gs + G_RK + 8 * ch + 4);
-                e0.x *= r0.x; e0.y *= r0.y; e0.z *= r0.z; e0.w *= r0.w;
-                e1.x *= r1.x; e1.y *= r1.y; e1.z *= r1.z; e1.w *= r1.w;
-            }
+            // (with the prologue beta e^G / ||k||: W = T diag(beta e^G) K / ||k|| by rows of K)
+            const float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
+            const float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
             const float4 c0 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch);
             const float4 c1 = *reinterpret_cast<const float4*>(gs + G_BETA + 8 * ch + 4);
             w4[0] = pack_bf16x2(t0v.x * e0.x, t0v.y * e0.y); w4[1] = pack_bf16x2(t0v.z * e0.z, t0v.w * e0.w);

@@ -19,12 +19,16 @@
 
 namespace dn {
 
-template <int DK, int DV, typename Tin, int GATE>
+// PRO: the Gated DeltaNet layer's prologue ("The full layer", steps 4 and 5):
+// q and k normalised per head, beta = sigmoid(b), g = -exp(A_log) softplus(a +
+// dt_bias), from the raw b and a in `beta` and `g` (scalar gate).
+template <int DK, int DV, typename Tin, int GATE, bool PRO = false>
 __global__ void __launch_bounds__(2 * DV)
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const float* __restrict__ beta,
                    const float* __restrict__ g, float* __restrict__ S,
-                   Tin* __restrict__ o, float scale) {
+                   Tin* __restrict__ o, float scale, const float* __restrict__ A_log = nullptr,
+                   const float* __restrict__ dt_bias = nullptr, int H = 1) {
     constexpr int NT = 2 * DV;     // threads
     constexpr int TPR = DV / 4;    // threads per state row
     constexpr int RS = NT / TPR;   // row sets (8)
@@ -37,6 +41,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     __shared__ float ks[DK], qs[DK], as[DK];
     __shared__ float4 red_p[RS][TPR], red_q[RS][TPR];
     __shared__ float qk_s;
+    __shared__ float rn_s[2];
 
     float* Sh = S + head * (DK * DV);
     float4 s[RPT];
@@ -46,13 +51,39 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 
     for (int i = tid; i < DK; i += NT) {
         ks[i] = ld_elem(k + head * DK + i);
-        qs[i] = scale * ld_elem(q + head * DK + i);
+        qs[i] = (PRO ? 1.f : scale) * ld_elem(q + head * DK + i);
         if (GATE == kGatePerKey) as[i] = expf(g[head * DK + i]);
     }
     const float4 vv = ld4(v + head * DV + cg * 4);
-    const float b = beta[head];
-    const float a = (GATE == kGateScalar) ? expf(g[head]) : 1.0f;
+    float b = beta[head];
+    float a = (GATE == kGateScalar) ? g[head] : 0.f;
+    if (PRO) gdn_raw_gates(b, a, expf(A_log[head % H]), dt_bias[head % H]);
+    if (GATE == kGateScalar) a = expf(a);
+    else a = 1.0f;
     __syncthreads();
+    if (PRO) {
+        // k / max(||k||, 1e-12) and scale q / max(||q||, 1e-12)
+        if (tid < 32) {
+            float sk = 0.f, sq = 0.f;
+            for (int i = tid; i < DK; i += 32) {
+                sk += ks[i] * ks[i];
+                sq += qs[i] * qs[i];
+            }
+            sk = warp_sum(sk);
+            sq = warp_sum(sq);
+            if (tid == 0) {
+                rn_s[0] = 1.f / fmaxf(sqrtf(sk), 1e-12f);
+                rn_s[1] = scale / fmaxf(sqrtf(sq), 1e-12f);
+            }
+        }
+        __syncthreads();
+        const float rk = rn_s[0], rq = rn_s[1];
+        for (int i = tid; i < DK; i += NT) {
+            ks[i] *= rk;
+            qs[i] *= rq;
+        }
+        __syncthreads();
+    }
 
     if (tid < 32) {
         float x = 0.f;
@@ -112,6 +143,11 @@ static cudaError_t launch_decode_gate(const DecodeArgs& a, cudaStream_t st) {
     const Tin* k = static_cast<const Tin*>(a.k);
     const Tin* v = static_cast<const Tin*>(a.v);
     Tin* o = static_cast<Tin*>(a.o);
+    if (a.prologue) {
+        decode_step_kernel<DK, DV, Tin, kGateScalar, true><<<grid, 2 * DV, 0, st>>>(
+            q, k, v, a.beta, a.g, a.S, o, a.scale, a.A_log, a.dt_bias, (int)a.H);
+        return counted(cudaGetLastError());
+    }
     switch (a.gate) {
         case kGateNone:
             decode_step_kernel<DK, DV, Tin, kGateNone><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);

@@ -108,7 +108,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 4; }
+int dn_version(void) { return (2 << 16) | 5; }
 
 unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 
@@ -283,9 +283,10 @@ int dn_chunk_fwd(const void* q, const void* k, const void* v, const float* beta,
                            dtype, gate, DN_PATH_AUTO, nullptr, 0, cuda_stream);
 }
 
-int dn_decode_step(const void* q, const void* k, const void* v, const float* beta,
-                   const float* g, float* S, void* o, int B, int H, int d_k, int d_v,
-                   float scale, dn_dtype dtype, dn_gate gate, void* cuda_stream) {
+static int decode_impl(const void* q, const void* k, const void* v, const float* beta,
+                       const float* g, float* S, void* o, int B, int H, int d_k, int d_v,
+                       float scale, dn_dtype dtype, dn_gate gate, void* cuda_stream,
+                       const float* A_log = nullptr, const float* dt_bias = nullptr) {
     if (B < 0 || H < 0) return fail(DN_ERR_INVALID, "B, H must be >= 0 (got %d, %d)", B, H);
     if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
     if (gate != DN_GATE_NONE && gate != DN_GATE_SCALAR && gate != DN_GATE_PER_KEY)
@@ -315,14 +316,36 @@ int dn_decode_step(const void* q, const void* k, const void* v, const float* bet
     Range ins[] = {rq, rk, rv, rb, rg};
     for (Range r : ins)
         if (overlap(rs, r)) return fail(DN_ERR_INVALID, "S overlaps an input");
+    const bool pro = A_log != nullptr;
+    if (pro) {
+        if (!aligned(A_log, 4) || !aligned(dt_bias, 4)) return fail(DN_ERR_INVALID, "A_log and dt_bias must be 4-byte aligned");
+        Range rpa = rng(A_log, (int64_t)H * 4), rpd = rng(dt_bias, (int64_t)H * 4);
+        if (overlap(ro, rpa) || overlap(ro, rpd) || overlap(rs, rpa) || overlap(rs, rpd))
+            return fail(DN_ERR_INVALID, "o or S overlaps A_log or dt_bias");
+    }
 
     dn::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.S = S; a.o = o;
     a.B = B; a.H = H; a.dk = d_k; a.dv = d_v; a.scale = scale;
     a.bf16 = dtype == DN_BF16; a.gate = (int)gate;
+    a.prologue = pro; a.A_log = A_log; a.dt_bias = dt_bias;
     cudaError_t e = dn::launch_decode_step(a, static_cast<cudaStream_t>(cuda_stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
     return ok();
+}
+
+int dn_decode_step(const void* q, const void* k, const void* v, const float* beta,
+                   const float* g, float* S, void* o, int B, int H, int d_k, int d_v,
+                   float scale, dn_dtype dtype, dn_gate gate, void* cuda_stream) {
+    return decode_impl(q, k, v, beta, g, S, o, B, H, d_k, d_v, scale, dtype, gate, cuda_stream);
+}
+
+int dn_decode_step_gdn(const void* q, const void* k, const void* v, const float* b, const float* a,
+                       const float* A_log, const float* dt_bias, float* S, void* o, int B, int H, int d_k,
+                       int d_v, float scale, dn_dtype dtype, void* cuda_stream) {
+    if ((int64_t)B * H > 0 && (!A_log || !dt_bias)) return fail(DN_ERR_INVALID, "A_log and dt_bias are required");
+    return decode_impl(q, k, v, b, a, S, o, B, H, d_k, d_v, scale, dtype, DN_GATE_SCALAR, cuda_stream, A_log,
+                       dt_bias);
 }
 
 int dn_device_status(void* cuda_stream) {

@@ -53,4 +53,14 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// The Gated DeltaNet layer's gates from its raw per-token inputs ("Linear
+// attention and Gated DeltaNet", ch. 28, "The full layer", step 5): beta =
+// sigmoid(b), g = -exp(A_log) softplus(a + dt_bias), softplus(x) = log(1 + e^x)
+// (x above 20 taken as x).  eA = exp(A_log) of the head.
+__device__ __forceinline__ void gdn_raw_gates(float& b, float& a, float eA, float dt_bias) {
+    b = 1.f / (1.f + expf(-b));
+    const float x = a + dt_bias;
+    a = -eA * (x > 20.f ? x : log1pf(expf(x)));
+}
+
 }  // namespace dn

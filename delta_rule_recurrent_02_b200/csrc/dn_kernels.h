@@ -37,6 +37,11 @@ struct DecodeArgs {
     float scale;
     bool bf16;
     int gate;
+    // the layer's prologue (scalar gate): beta and g hold the raw b and a; q and k are
+    // normalised inside
+    bool prologue;
+    const float* A_log;       // [H]
+    const float* dt_bias;     // [H]
 };
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);

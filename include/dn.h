@@ -245,6 +245,20 @@ DN_API int dn_decode_step(const void* q, const void* k, const void* v,
                    dn_dtype dtype, dn_gate gate, void* cuda_stream);
 
 /*
+ * dn_decode_step_gdn -- dn_decode_step with the Gated DeltaNet layer's
+ * prologue ("Linear attention and Gated DeltaNet", ch. 28, "The full layer",
+ * steps 4 and 5) fused into the kernel: the step runs on
+ *   q / max(||q||, 1e-12), k / max(||k||, 1e-12),
+ *   beta = sigmoid(b), g = -exp(A_log[h]) * softplus(a + dt_bias[h])
+ * as dn_decode_step with the scalar gate on these.
+ *   q, k [B,H,d_k] raw; v [B,H,d_v]; b, a [B,H] fp32 raw; A_log, dt_bias [H]
+ *   fp32 (required, 4-byte aligned); S, o, d_k, d_v, scale, dtype as dn_decode_step.
+ */
+DN_API int dn_decode_step_gdn(const void* q, const void* k, const void* v, const float* b, const float* a,
+                              const float* A_log, const float* dt_bias, float* S, void* o,
+                              int B, int H, int d_k, int d_v, float scale, dn_dtype dtype, void* cuda_stream);
+
+/*
  * dn_device_status -- synchronise `cuda_stream`, then read and clear the
  * status word of the current device.  Returns DN_ERR_TIMEOUT if a kernel of
  * this library launched since the previous call gave up on a bounded wait
@@ -260,7 +274,7 @@ DN_API const char* dn_status_str(int status);
 DN_API const char* dn_last_error(void);
 
 /* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path;
- * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn. */
+ * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn; 2.5: dn_decode_step_gdn. */
 DN_API int dn_version(void);
 
 /*

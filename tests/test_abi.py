@@ -206,3 +206,10 @@ def test_gdn_layer_rejects(lib, over, code):
     assert gdn_call(lib, **over) == code
     assert lib.dn_last_error() != b""
     assert lib.dn_kernel_launches() == before
+
+
+def test_decode_layer_rejects_missing_params(lib):
+    A0 = 0x10000000
+    st = lib.dn_decode_step_gdn(A0, A0 + STEP, A0 + 2 * STEP, A0 + 3 * STEP, A0 + 4 * STEP, None, None,
+                                A0 + 5 * STEP, A0 + 6 * STEP, 2, 3, 128, 128, 1.0, 1, None)
+    assert st == dn.DN_ERR_INVALID and b"A_log" in lib.dn_last_error()

@@ -122,3 +122,37 @@ def test_decode_empty_and_errors(cuda_device):
     with pytest.raises(dn.DNError) as ei:
         dn.decode_step(q, q, q, torch.zeros(1, 1, device="cuda"), torch.zeros(1, 1, 96, 96, device="cuda"))
     assert ei.value.status == dn.DN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
+def test_decode_layer_prologue(cuda_device, dtype, dk, dv):
+    # dn_decode_step_gdn: raw q and k (varied norms, one zero row), raw b and a with the
+    # per-head A_log and dt_bias, against the oracle prologue then the oracle recurrence
+    B, H, steps = 3, 5, 8
+    gen = torch.Generator().manual_seed(55 + dk)
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    q = (torch.randn(steps, B, H, dk, generator=gen) * (0.2 + 3 * torch.rand(steps, B, H, 1, generator=gen))).to(td)
+    k = (torch.randn(steps, B, H, dk, generator=gen) * (0.2 + 3 * torch.rand(steps, B, H, 1, generator=gen))).to(td)
+    q[2, 1, 3] = 0
+    v = torch.randn(steps, B, H, dv, generator=gen).to(td)
+    b = torch.randn(steps, B, H, generator=gen)
+    a = torch.randn(steps, B, H, generator=gen)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen))
+    dt_bias = 0.5 * torch.randn(H, generator=gen)
+    S0 = 0.1 * torch.randn(B, H, dk, dv, generator=gen)
+    sc = dk ** -0.5
+    S = S0.cuda().clone()
+    outs = []
+    for s in range(steps):
+        o = torch.empty((B, H, dv), dtype=td, device="cuda")
+        dn.dn_decode_step_gdn(q[s].cuda(), k[s].cuda(), v[s].cuda(), b[s].cuda(), a[s].cuda(), A_log.cuda(),
+                              dt_bias.cuda(), S, o, scale=sc)
+        outs.append(o)
+    dn.dn_device_status()
+    # the prologue on [B,H,steps,...] (steps become the time axis)
+    tr = lambda t: f64(t).transpose((1, 2, 0) + tuple(range(3, t.dim())))
+    qn, kn, beta, g = oracle.gdn_prologue(tr(q), tr(k), tr(b), tr(a), f64(A_log), f64(dt_bias))
+    ro, rS = oracle.delta_rule(qn, kn, tr(v), beta, g, f64(S0), scale=sc)
+    assert_close(torch.stack(outs).permute(1, 2, 0, 3), ro, dtype, "o")
+    assert_close(S, rS, dtype, "S")
