@@ -17,6 +17,10 @@ Contents
 ``wy_transition``         the WY form of one chunk's product of transitions.
 ``gdn_prologue``          steps 4 and 5 of the Gated DeltaNet layer: unit q and
                           k, beta = sigmoid(b), g = -exp(A_log) softplus(a + dt_bias).
+``causal_conv1d``        step 2 of the layer: depthwise causal conv over time
+                          (kernel K, SiLU) with the K-1 previous inputs carried.
+``rms_norm_gated``        step 7 of the layer: RMSNorm of each head's output
+                          times a per-channel weight and SiLU (or sigmoid) of z.
 
 Every function takes and returns numpy arrays.  Layouts: tokens
 ``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
@@ -326,3 +330,57 @@ def gdn_prologue(q, k, b, a, A_log, dt_bias, eps=1e-12):
     beta = 1.0 / (1.0 + np.exp(-b))
     g = -np.exp(A_log)[None, :, None] * np.logaddexp(0.0, a + dt_bias[None, :, None])
     return qn, kn, beta, g
+
+
+def causal_conv1d(x, weight, state=None, activation=True):
+    """Step 2 of the Gated DeltaNet layer ("Linear attention and Gated
+    DeltaNet", ch. 28, "The full layer" and its ``causal_conv1d``), in fp64:
+    a depthwise causal convolution over time, one length-K filter per channel,
+    then SiLU, carrying the previous K-1 inputs as its state.
+
+    Written from its definition: with ``joined = concat(state, x)`` along time
+    (K-1 history rows, then the T new rows),
+
+        y[t, c] = sum_{j=0}^{K-1} weight[c, j] * joined[t + j, c],
+
+    so ``weight[c, K-1]`` multiplies the current input and output t sees
+    inputs t-K+1 .. t only; ``silu(y) = y / (1 + e^-y)`` when ``activation``.
+    The new state is the last K-1 rows of ``joined``.
+
+    Layout: token-major, x [B, T, C] and state [B, K-1, C] (oldest row
+    first); the page writes the same arrays channel-major.  weight [C, K].
+    A missing state is K-1 rows of zeros.  Returns ``(y, new_state)``."""
+    x, weight = _f64(x), _f64(weight)
+    B, T, C = x.shape
+    K = weight.shape[1]
+    state = np.zeros((B, K - 1, C)) if state is None else _f64(state)
+    joined = np.concatenate([state, x], axis=1)
+    y = np.zeros((B, T, C))
+    for t in range(T):
+        for j in range(K):
+            y[:, t, :] += weight[:, j][None, :] * joined[:, t + j, :]
+    if activation:
+        y = y / (1.0 + np.exp(-y))
+    return y, joined[:, T:, :].copy()
+
+
+def rms_norm_gated(x, z, weight, eps=1e-6, activation="silu"):
+    """Step 7 of the Gated DeltaNet layer ("Linear attention and Gated
+    DeltaNet", ch. 28, ``RMSNormGated``), in fp64: each row of a head's
+    read-out divided by its root mean square, times a per-channel weight and
+    a gate of z,
+
+        y = weight * x / sqrt(mean(x^2) + eps) * act(z),
+
+    act = SiLU (``z / (1 + e^-z)``) or the logistic sigmoid.  The mean runs
+    over the last axis (the head's d_v channels); weight [d_v] is shared by
+    every head.  x and z have the same shape; returns y of that shape."""
+    x, z, weight = _f64(x), _f64(z), _f64(weight)
+    normed = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    if activation == "silu":
+        gate = z / (1.0 + np.exp(-z))
+    elif activation == "sigmoid":
+        gate = 1.0 / (1.0 + np.exp(-z))
+    else:
+        raise ValueError(f"activation {activation!r}")
+    return weight * normed * gate

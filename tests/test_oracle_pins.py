@@ -412,3 +412,98 @@ def test_gdn_prologue_unit_rows():
     assert np.allclose(qn2, qn, rtol=0, atol=1e-15)
     cos = np.sum(qn[0, 1, 2] * q[0, 1, 2]) / np.linalg.norm(q[0, 1, 2])
     assert np.isclose(cos, 1.0, rtol=0, atol=1e-15)
+
+
+# ---- causal_conv1d: pinned by filters with known outputs, a library convolution and
+#      the carried-history property -----------------------------------------------------
+
+def test_causal_conv1d_identity_and_shift_filters():
+    """weight [0, .., 0, 1] passes the current input (SiLU of it with the activation);
+    weight [1, 0, .., 0] is a delay of K-1 steps that reads the carried state first."""
+    rng = np.random.default_rng(11)
+    B, T, C, K = 2, 9, 5, 4
+    x = rng.standard_normal((B, T, C)); st = rng.standard_normal((B, K - 1, C))
+    ident = np.zeros((C, K)); ident[:, K - 1] = 1.0
+    y, _ = oracle.causal_conv1d(x, ident, st, activation=False)
+    assert np.array_equal(y, x)
+    ys, _ = oracle.causal_conv1d(x, ident, st, activation=True)
+    assert np.allclose(ys, x / (1 + np.exp(-x)), rtol=1e-15, atol=0)
+    delay = np.zeros((C, K)); delay[:, 0] = 1.0
+    y, new = oracle.causal_conv1d(x, delay, st, activation=False)
+    assert np.array_equal(y[:, :K - 1], st) and np.array_equal(y[:, K - 1:], x[:, :T - K + 1])
+    assert np.array_equal(new, x[:, T - K + 1:])
+    y0, _ = oracle.causal_conv1d(x, delay, None, activation=False)      # no state: zeros
+    assert not y0[:, :K - 1].any()
+
+
+def test_causal_conv1d_matches_numpy_convolve():
+    """Each channel against numpy's full convolution of the joined sequence with the
+    reversed filter (the 'valid' part): a library routine the oracle does not use."""
+    rng = np.random.default_rng(12)
+    B, T, C, K = 2, 13, 6, 4
+    x = rng.standard_normal((B, T, C)); w = rng.standard_normal((C, K)); st = rng.standard_normal((B, K - 1, C))
+    y, _ = oracle.causal_conv1d(x, w, st, activation=False)
+    for b in range(B):
+        for c in range(C):
+            joined = np.concatenate([st[b, :, c], x[b, :, c]])
+            ref = np.convolve(joined, w[c, ::-1], mode="valid")
+            assert np.allclose(y[b, :, c], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_causal_conv1d_impulse_response_and_causality():
+    """An impulse at t0 in channel c shows the filter reversed at t0 .. t0+K-1 and
+    nothing before t0 or in other channels."""
+    B, T, C, K, t0 = 1, 12, 3, 4, 5
+    w = np.arange(1.0, C * K + 1).reshape(C, K)
+    x = np.zeros((B, T, C)); x[0, t0, 1] = 1.0
+    y, _ = oracle.causal_conv1d(x, w, None, activation=False)
+    assert not y[0, :t0].any() and not y[0, :, [0, 2]].any()
+    assert np.array_equal(y[0, t0:t0 + K, 1], w[1, ::-1])
+    assert not y[0, t0 + K:].any()
+
+
+@pytest.mark.parametrize("T1", [0, 1, 2, 5, 11])
+def test_causal_conv1d_carried_state_splits_sequences(T1):
+    """Running [0, T1) and then [T1, T) with the returned state equals one run over
+    [0, T), including splits shorter than K-1 (the state then keeps old rows)."""
+    rng = np.random.default_rng(13 + T1)
+    B, T, C, K = 2, 11, 4, 4
+    x = rng.standard_normal((B, T, C)); w = rng.standard_normal((C, K)); st = rng.standard_normal((B, K - 1, C))
+    y, s = oracle.causal_conv1d(x, w, st)
+    ya, sa = oracle.causal_conv1d(x[:, :T1], w, st)
+    yb, sb = oracle.causal_conv1d(x[:, T1:], w, sa)
+    assert np.allclose(np.concatenate([ya, yb], axis=1), y, rtol=1e-14, atol=1e-14)
+    assert np.array_equal(sb, s)
+
+
+# ---- rms_norm_gated: closed forms --------------------------------------------------------
+
+def test_rms_norm_gated_closed_forms():
+    """With eps = 0 the normed row has mean square 1 and is invariant to a positive
+    scale of x; a constant row c maps to sign(c); silu(0) = 0 closes the gate;
+    sigmoid(0) = 1/2; the weight multiplies channel by channel."""
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((3, 4, 16)); z = rng.standard_normal((3, 4, 16)); w = rng.standard_normal(16)
+    one = np.ones(16)
+    big = np.full_like(z, 60.0)          # silu(60) = 60 / (1 + e^-60)
+    n = oracle.rms_norm_gated(x, big, one, eps=0.0) / (60.0 / (1 + np.exp(-60.0)))
+    assert np.allclose(np.mean(n * n, axis=-1), 1.0, rtol=0, atol=1e-14)
+    assert np.allclose(oracle.rms_norm_gated(3.7 * x, z, w, eps=0.0), oracle.rms_norm_gated(x, z, w, eps=0.0),
+                       rtol=1e-14, atol=1e-14)
+    c = np.full((1, 16), -2.5)
+    assert np.allclose(oracle.rms_norm_gated(c, big[0, :1], one, eps=0.0), -60.0 / (1 + np.exp(-60.0)), rtol=1e-15)
+    assert not oracle.rms_norm_gated(x, np.zeros_like(z), w).any()
+    half = oracle.rms_norm_gated(x, np.zeros_like(z), one, eps=0.0, activation="sigmoid")
+    assert np.allclose(half, 0.5 * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True)), rtol=1e-14)
+    a = oracle.rms_norm_gated(x, z, w); b = oracle.rms_norm_gated(x, z, one)
+    assert np.allclose(a, b * w, rtol=1e-14, atol=1e-14)
+
+
+def test_rms_norm_gated_eps_and_zero_row():
+    """eps enters under the root with the mean square: a zero row stays zero and a row
+    of rms r is scaled by 1 / sqrt(r^2 + eps)."""
+    x = np.zeros((2, 8)); x[1] = 1e-3
+    y = oracle.rms_norm_gated(x, np.full((2, 8), 50.0), np.ones(8), eps=1e-6, activation="sigmoid")
+    assert not y[0].any()
+    expect = 1e-3 / np.sqrt(1e-6 + 1e-6) / (1 + np.exp(-50.0))
+    assert np.allclose(y[1], expect, rtol=1e-14)
