@@ -352,6 +352,69 @@ def measure_gdn_prologue(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
             "traffic": None, "timing": f"median of {calls} calls after {warm}, CUDA events"}
 
 
+def measure_layer_ops(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
+    """The layer steps on either side of the rule at the bench prefill's shape
+    (B=4, T=4096, 16 heads of 128), bf16, each against the HBM roofline:
+    the causal conv (K=4, SiLU) of q, k and v as three calls on the column
+    slices of one [B, T, 3*16*128] projection output, head-major outputs and
+    carried states; and the gated RMSNorm of o [B, 16, T, 128] (head-major)
+    with z [B, T, 16, 128] into y [B, T, 16, 128]."""
+    pc = W.GDN_PREFILL
+    B, H, T, d, K = pc.B, pc.H, pc.T, pc.dk, 4
+    C3 = 3 * H * d
+    gen = torch.Generator().manual_seed(pc.seed + 1)
+    proj = torch.randn(B, T, C3, generator=gen).to(torch.bfloat16).to(dev)
+    w = (torch.randn(C3, K, generator=gen) * 0.5).to(dev)
+    s_in = torch.randn(B, K - 1, C3, generator=gen).to(torch.bfloat16).to(dev)
+    ys = [torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    w_parts = [w[i * H * d:(i + 1) * H * d].contiguous() for i in range(3)]
+    s_parts = [s_in[:, :, i * H * d:(i + 1) * H * d].contiguous() for i in range(3)]
+    s_outs = [torch.empty_like(sp) for sp in s_parts]
+
+    def conv():
+        for i in range(3):
+            dn.dn_causal_conv1d(proj[:, :, i * H * d:(i + 1) * H * d], w_parts[i], ys[i], s_parts[i], s_outs[i],
+                                head_dim=d, stream=stream)
+
+    o = torch.randn(B, H, T, d, generator=gen).to(torch.bfloat16).to(dev)
+    z = torch.randn(B, T, H, d, generator=gen).to(torch.bfloat16).to(dev)
+    nw = torch.ones(d, device=dev)
+    y = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+
+    def norm():
+        dn.dn_rms_norm_gated(o, z, nw, y, stream=stream)
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(calls):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        dn.dn_device_status(stream)
+        return statistics.median(ts)
+
+    out = {}
+    conv_bytes = 2 * B * T * C3 * 2 + C3 * K * 4 + 2 * B * (K - 1) * C3 * 2
+    norm_bytes = 3 * B * T * H * d * 2 + d * 4
+    for name, fn, by, launches in (
+            (f"causal_conv1d_qkv_bf16_B{B}_T{T}_C{C3}_K{K}", conv, conv_bytes, 3),
+            (f"rms_norm_gated_bf16_B{B}_T{T}_H{H}_d{d}", norm, norm_bytes, 1)):
+        ms = timed(fn)
+        gb = by / (ms * 1e-3) / 1e9
+        out[name] = {"ms_per_call": ms, "algorithmic_bytes": by, "hbm_gbs": gb, "hbm_frac": gb / peaks["hbm_gbs"],
+                     "kernel_launches_per_call": launches, "bound": "hbm",
+                     "timing": f"median of {calls} calls after {warm}, CUDA events"}
+    del proj, w, s_in, ys, o, z, y
+    torch.cuda.empty_cache()
+    return out
+
+
 def workload_config():
     return {"workload": "gated_deltanet_prefill_B4_H16_T4096_d128_bf16_chunk64 + "
                         "decode_step_B256_H32_d128_bf16_fp32state",
@@ -503,6 +566,7 @@ def main():
             "clocks": clocks}
     if world == 1 and not args.no_configs:
         line["other_prefill_workloads"] = measure_prefill_configs(dn, torch, W, peaks, dev, stream)
+        line["layer_ops"] = measure_layer_ops(dn, torch, W, peaks, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]

@@ -26,7 +26,7 @@ import os
 
 __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
            "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
-           "dn_decode_step", "dn_kernel_launches",
+           "dn_decode_step", "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
 
@@ -38,7 +38,7 @@ _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
                "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
                "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version",
-               "dn_kernel_launches")
+               "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -88,6 +88,10 @@ def load_library():
     lib.dn_last_error.restype = ctypes.c_char_p
     lib.dn_version.argtypes = []
     lib.dn_version.restype = I
+    lib.dn_causal_conv1d.argtypes = [vp, I, fp, vp, vp, vp, I, I, I, I, I, I, I, vp]
+    lib.dn_causal_conv1d.restype = I
+    lib.dn_rms_norm_gated.argtypes = [vp, vp, fp, vp, I, I, I, I, F, I, I, I, vp]
+    lib.dn_rms_norm_gated.restype = I
     lib.dn_kernel_launches.argtypes = []
     lib.dn_kernel_launches.restype = ctypes.c_ulonglong
     _lib = lib
@@ -238,6 +242,42 @@ def dn_decode_step(q, k, v, beta, g, S, o, *, scale: float = 1.0, gate: str | No
     st = lib.dn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S), _ptr(o),
                             B, H, dk, dv, float(scale), _dtype_code(q),
                             _gate_code(gate, g, (B, H)), _stream(stream))
+    _check(lib, st)
+
+
+def dn_causal_conv1d(x, weight, y, state_in=None, state_out=None, *, head_dim: int | None = None,
+                     activation: bool = True, stream=None) -> None:
+    """Depthwise causal conv over time with carried history, through
+    ``dn_causal_conv1d``: x [B, T, C] (its rows may be a column slice of a wider
+    tensor: unit stride over channels, any row stride), weight [C, K] fp32,
+    states [B, K-1, C] in x's dtype, y [B, C // head_dim, T, head_dim]
+    (head_dim defaults to C: y is then [B, T, C] in effect)."""
+    lib = load_library()
+    B, T, C = x.shape
+    K = weight.shape[-1]
+    if not x.is_cuda:
+        raise ValueError("dn: tensors must be CUDA tensors (the library takes device pointers)")
+    if x.stride(2) != 1 or (T > 1 and B > 1 and x.stride(0) != T * x.stride(1)):
+        raise ValueError("dn: x needs unit channel stride and rows evenly spaced across the batch")
+    ld_x = x.stride(1) if T > 1 else (x.stride(0) if B > 1 else C)
+    _f32(weight)
+    st = lib.dn_causal_conv1d(x.data_ptr(), ld_x, _ptr(weight), _ptr(state_in), _ptr(y), _ptr(state_out),
+                              B, T, C, K, C if head_dim is None else head_dim, 1 if activation else 0,
+                              _dtype_code(x), _stream(stream))
+    _check(lib, st)
+
+
+def dn_rms_norm_gated(x, z, weight, y, *, eps: float = 1e-6, x_head_major: bool = True,
+                      activation: str = "silu", stream=None) -> None:
+    """Gated RMSNorm of each head's output row, through ``dn_rms_norm_gated``:
+    x [B, H, T, D] (x_head_major) or [B, T, H, D]; z and y [B, T, H, D];
+    weight [D] fp32; activation "silu" or "sigmoid"."""
+    lib = load_library()
+    B, T, H, D = z.shape
+    _f32(weight)
+    st = lib.dn_rms_norm_gated(_ptr(x), _ptr(z), _ptr(weight), _ptr(y), B, T, H, D, float(eps),
+                               1 if x_head_major else 0, {"silu": 1, "sigmoid": 0}[activation],
+                               _dtype_code(x), _stream(stream))
     _check(lib, st)
 
 

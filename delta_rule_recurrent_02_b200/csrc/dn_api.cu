@@ -108,7 +108,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
-int dn_version(void) { return (2 << 16) | 5; }
+int dn_version(void) { return (2 << 16) | 6; }
 
 unsigned long long dn_kernel_launches(void) { return dn::g_launches.load(std::memory_order_relaxed); }
 
@@ -346,6 +346,69 @@ int dn_decode_step_gdn(const void* q, const void* k, const void* v, const float*
     if ((int64_t)B * H > 0 && (!A_log || !dt_bias)) return fail(DN_ERR_INVALID, "A_log and dt_bias are required");
     return decode_impl(q, k, v, b, a, S, o, B, H, d_k, d_v, scale, dtype, DN_GATE_SCALAR, cuda_stream, A_log,
                        dt_bias);
+}
+
+int dn_causal_conv1d(const void* x, int ld_x, const float* weight, const void* state_in, void* y,
+                     void* state_out, int B, int T, int C, int K, int head_dim, int activation, dn_dtype dtype,
+                     void* cuda_stream) {
+    if (B < 0 || T < 0 || C < 0) return fail(DN_ERR_INVALID, "B, T, C must be >= 0 (got %d, %d, %d)", B, T, C);
+    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
+    if (K < 1 || K > 4) return fail(DN_ERR_UNSUPPORTED, "K must be 1..4 (got %d)", K);
+    if (activation != 0 && activation != 1) return fail(DN_ERR_INVALID, "activation must be 0 or 1");
+    if (B == 0 || C == 0) return ok();
+    if (ld_x < C) return fail(DN_ERR_INVALID, "ld_x (%d) must be >= C (%d)", ld_x, C);
+    if (head_dim <= 0 || C % head_dim != 0) return fail(DN_ERR_INVALID, "head_dim (%d) must divide C (%d)", head_dim, C);
+    if (B > 65535 || T > 16 * 65535) return fail(DN_ERR_UNSUPPORTED, "B <= 65535 and T <= 1048560 (got %d, %d)", B, T);
+    if (!weight || (T > 0 && (!x || !y))) return fail(DN_ERR_INVALID, "x, weight and y are required");
+    const int64_t esz = dtype == DN_BF16 ? 2 : 4;
+    const void* pe[] = {x, y, state_in, state_out};
+    for (const void* p : pe)
+        if (p && !aligned(p, (uintptr_t)esz)) return fail(DN_ERR_INVALID, "x, y and the states must be %d-byte aligned", (int)esz);
+    if (!aligned(weight, 4)) return fail(DN_ERR_INVALID, "weight must be 4-byte aligned");
+    const int64_t nst = (int64_t)B * (K - 1) * C * esz;
+    Range rx = rng(x, T > 0 ? ((int64_t)B * T - 1) * ld_x * esz + (int64_t)C * esz : 0);
+    Range rw = rng(weight, (int64_t)C * K * 4), ry = rng(y, (int64_t)B * T * C * esz);
+    Range rsi = rng(state_in, K > 1 ? nst : 0), rso = rng(state_out, K > 1 ? nst : 0);
+    if (overlap(ry, rx) || overlap(ry, rw) || overlap(ry, rsi) || overlap(ry, rso))
+        return fail(DN_ERR_INVALID, "y overlaps another argument");
+    if (overlap(rso, rx) || overlap(rso, rw)) return fail(DN_ERR_INVALID, "state_out overlaps x or weight");
+    if (overlap(rso, rsi) && !(state_out == state_in && T <= 16))
+        return fail(DN_ERR_INVALID, "state_out may be state_in itself only when T <= 16; otherwise it must not overlap it");
+    const int V = (int)(16 / esz);
+    bool vec = C % V == 0 && ld_x % V == 0 && head_dim % V == 0;
+    for (const void* p : pe)
+        if (p && !aligned(p, 16)) vec = false;
+    dn::ConvArgs a;
+    a.x = x; a.ld_x = ld_x; a.weight = weight; a.state_in = state_in; a.y = y; a.state_out = state_out;
+    a.B = B; a.T = T; a.C = C; a.K = K; a.head_dim = head_dim;
+    a.activation = activation == 1; a.bf16 = dtype == DN_BF16; a.vec = vec;
+    if (T == 0 && (!state_out || K == 1)) return ok();
+    cudaError_t e = dn::launch_causal_conv1d(a, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "causal conv kernel");
+}
+
+int dn_rms_norm_gated(const void* x, const void* z, const float* weight, void* y, int B, int T, int H, int D,
+                      float eps, int x_head_major, int activation, dn_dtype dtype, void* cuda_stream) {
+    if (B < 0 || T < 0 || H < 0) return fail(DN_ERR_INVALID, "B, T, H must be >= 0 (got %d, %d, %d)", B, T, H);
+    if (dtype != DN_F32 && dtype != DN_BF16) return fail(DN_ERR_INVALID, "unknown dtype %d", (int)dtype);
+    if (D != 64 && D != 128 && D != 256) return fail(DN_ERR_UNSUPPORTED, "D must be 64, 128 or 256 (got %d)", D);
+    if (!(eps >= 0.f) || eps > 3.0e38f) return fail(DN_ERR_INVALID, "eps must be finite and >= 0");
+    if (activation != 0 && activation != 1) return fail(DN_ERR_INVALID, "activation must be 0 or 1");
+    if (x_head_major != 0 && x_head_major != 1) return fail(DN_ERR_INVALID, "x_head_major must be 0 or 1");
+    const int64_t rows = (int64_t)B * T * H;
+    if (rows == 0) return ok();
+    if (!x || !z || !weight || !y) return fail(DN_ERR_INVALID, "x, z, weight and y are required");
+    if (!aligned(x, 16) || !aligned(z, 16) || !aligned(y, 16)) return fail(DN_ERR_INVALID, "x, z and y must be 16-byte aligned");
+    if (!aligned(weight, 4)) return fail(DN_ERR_INVALID, "weight must be 4-byte aligned");
+    const int64_t esz = dtype == DN_BF16 ? 2 : 4;
+    Range rx = rng(x, rows * D * esz), rz = rng(z, rows * D * esz), ry = rng(y, rows * D * esz);
+    Range rw = rng(weight, (int64_t)D * 4);
+    if (overlap(ry, rx) || overlap(ry, rz) || overlap(ry, rw)) return fail(DN_ERR_INVALID, "y overlaps another argument");
+    dn::NormArgs a;
+    a.x = x; a.z = z; a.weight = weight; a.y = y; a.B = B; a.T = T; a.H = H; a.D = D; a.eps = eps;
+    a.silu = activation == 1; a.x_head_major = x_head_major == 1; a.bf16 = dtype == DN_BF16;
+    cudaError_t e = dn::launch_rms_norm_gated(a, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "gated RMSNorm kernel");
 }
 
 int dn_device_status(void* cuda_stream) {

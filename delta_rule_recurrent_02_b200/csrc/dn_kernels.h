@@ -45,6 +45,37 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
+
+// The layer's causal conv over time (layer_ops.cu).
+struct ConvArgs {
+    const void* x;            // [B, T, ld_x], channels 0..C-1 of each row
+    int64_t ld_x;
+    const float* weight;      // [C, K]
+    const void* state_in;     // [B, K-1, C] or null (zeros)
+    void* y;                  // [B, C / head_dim, T, head_dim]
+    void* state_out;          // [B, K-1, C] or null
+    int64_t B;
+    int T, C, K, head_dim;
+    bool activation;          // SiLU
+    bool bf16;
+    bool vec;                 // 16-byte accesses (alignment checked by the caller)
+};
+cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st);
+
+// The layer's gated RMSNorm of each head's output row (layer_ops.cu).
+struct NormArgs {
+    const void* x;            // [B, H, T, D] (x_head_major) or [B, T, H, D]
+    const void* z;            // [B, T, H, D]
+    const float* weight;      // [D]
+    void* y;                  // [B, T, H, D]
+    int64_t B, T, H;
+    int D;                    // 64, 128 or 256
+    float eps;
+    bool silu;                // else the logistic sigmoid
+    bool x_head_major;
+    bool bf16;
+};
+cudaError_t launch_rms_norm_gated(const NormArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_simt(const ChunkArgs& a, cudaStream_t st);
 
 // Tensor-core (tcgen05) chunk path: the per-chunk UT/WY transform (chunk_wy.cu)

@@ -1,0 +1,315 @@
+// layer_ops.cu -- the two Gated DeltaNet layer steps on either side of the rule
+// ("Linear attention and Gated DeltaNet", ch. 28, "The full layer"):
+//
+//   step 2, the short causal convolution over time (one length-K filter per
+//   channel, then SiLU) with the previous K-1 inputs carried as its state;
+//   step 7, the gated RMSNorm of each head's output row.
+//
+// Both are streaming work bound by HBM: 16-byte vector loads across channels
+// (coalesced), fp32 arithmetic, one rounding at the store.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "dn_kernels.h"
+
+namespace dn {
+namespace {
+
+// ---- element access: V consecutive channels as one 16-byte (or scalar) access --------
+
+template <typename T, int V>
+struct Vec;
+template <>
+struct Vec<float, 4> {
+    using raw = float4;
+    __device__ static void to_f(const raw& r, float* f) { f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w; }
+    __device__ static raw from_f(const float* f) { return make_float4(f[0], f[1], f[2], f[3]); }
+};
+template <>
+struct Vec<float, 1> {
+    using raw = float;
+    __device__ static void to_f(const raw& r, float* f) { f[0] = r; }
+    __device__ static raw from_f(const float* f) { return f[0]; }
+};
+template <>
+struct Vec<__nv_bfloat16, 8> {
+    using raw = uint4;
+    __device__ static void to_f(const raw& r, float* f) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 p = __bfloat1622float2(h[e]);
+            f[2 * e] = p.x;
+            f[2 * e + 1] = p.y;
+        }
+    }
+    __device__ static raw from_f(const float* f) {
+        raw r;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+        return r;
+    }
+};
+template <>
+struct Vec<__nv_bfloat16, 1> {
+    using raw = __nv_bfloat16;
+    __device__ static void to_f(const raw& r, float* f) { f[0] = __bfloat162float(r); }
+    __device__ static raw from_f(const float* f) { return __float2bfloat16_rn(f[0]); }
+};
+template <>
+struct Vec<__nv_bfloat16, 2> {
+    using raw = __nv_bfloat162;
+    __device__ static void to_f(const raw& r, float* f) {
+        const float2 p = __bfloat1622float2(r);
+        f[0] = p.x;
+        f[1] = p.y;
+    }
+    __device__ static raw from_f(const float* f) { return __floats2bfloat162_rn(f[0], f[1]); }
+};
+template <>
+struct Vec<__nv_bfloat16, 4> {
+    using raw = uint2;
+    __device__ static void to_f(const raw& r, float* f) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float2 p = __bfloat1622float2(h[e]);
+            f[2 * e] = p.x;
+            f[2 * e + 1] = p.y;
+        }
+    }
+    __device__ static raw from_f(const float* f) {
+        raw r;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&r);
+        h[0] = __floats2bfloat162_rn(f[0], f[1]);
+        h[1] = __floats2bfloat162_rn(f[2], f[3]);
+        return r;
+    }
+};
+template <>
+struct Vec<float, 2> {
+    using raw = float2;
+    __device__ static void to_f(const raw& r, float* f) { f[0] = r.x; f[1] = r.y; }
+    __device__ static raw from_f(const float* f) { return make_float2(f[0], f[1]); }
+};
+
+__device__ __forceinline__ float silu(float x) { return x / (1.f + expf(-x)); }
+__device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+
+// ---- causal conv ----------------------------------------------------------------------
+//
+// Thread = V consecutive channels of one sequence over kConvRows consecutive tokens.
+// Its rows, plus the K-1 before them (from x, or from the carried state before token 0),
+// are loaded up front so that every load of the tile is in flight at once; the filter
+// then slides over them in registers.  The block whose tile holds the last token also
+// writes the new state (the last K-1 inputs of history-then-x).
+
+constexpr int kConvRows = 16;
+constexpr int kConvThreads = 128;
+
+template <typename Tin, int V, int K, bool ACT>
+__global__ void __launch_bounds__(kConvThreads)
+causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __restrict__ w, const Tin* s_in,
+                     Tin* __restrict__ y, Tin* s_out, int T, int C, int hd) {
+    using VT = Vec<Tin, V>;
+    using raw = typename VT::raw;
+    const int cv = blockIdx.x * kConvThreads + threadIdx.x;
+    const int c0 = cv * V;
+    if (c0 >= C) return;
+    const int64_t b = blockIdx.z;
+    const int t0 = blockIdx.y * kConvRows;
+
+    float wf[K][V];
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+#pragma unroll
+        for (int j = 0; j < K; ++j) wf[j][v] = w[(int64_t)(c0 + v) * K + j];
+
+    // input row t of this thread's channels: x for t >= 0, the carried state before
+    const Tin* xb = x + b * T * ld_x + c0;
+    const Tin* sb = s_in ? s_in + b * (K - 1) * (int64_t)C + c0 : nullptr;
+    auto load_row = [&](int t, float* f) {
+        if (t >= 0) {
+            VT::to_f(*reinterpret_cast<const raw*>(xb + (int64_t)t * ld_x), f);
+        } else if (sb) {
+            VT::to_f(*reinterpret_cast<const raw*>(sb + (int64_t)(t + K - 1) * C), f);
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) f[v] = 0.f;
+        }
+    };
+
+    raw rows[K - 1 + kConvRows];
+#pragma unroll
+    for (int i = 0; i < K - 1 + kConvRows; ++i) {
+        const int t = t0 - (K - 1) + i;
+        if (t < 0) {
+            float f[V];
+            load_row(t, f);
+            rows[i] = VT::from_f(f);
+        } else if (t < T) {
+            rows[i] = *reinterpret_cast<const raw*>(xb + (int64_t)t * ld_x);
+        }
+    }
+    // rows before token 0 were rounded back to Tin above; they are Tin values already
+    // (the state has x's dtype), so the round trip is exact
+
+    const int nh = C / hd;
+    const int head = c0 / hd, jj = c0 - head * hd;
+    Tin* yb = y + ((b * nh + head) * (int64_t)T) * hd + jj;
+#pragma unroll
+    for (int i = 0; i < kConvRows; ++i) {
+        const int t = t0 + i;
+        if (t < T) {
+            float acc[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = 0.f;
+#pragma unroll
+            for (int j = 0; j < K; ++j) {
+                float f[V];
+                VT::to_f(rows[i + j], f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(wf[j][v], f[v], acc[v]);
+            }
+            if (ACT) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = silu(acc[v]);
+            }
+            *reinterpret_cast<raw*>(yb + (int64_t)t * hd) = VT::from_f(acc);
+        }
+    }
+
+    if (s_out && K > 1 && t0 + kConvRows >= T) {
+        // new state row j = input row T-K+1+j; read all of them before the first write
+        // (s_out may be s_in itself when the whole sequence is this one tile)
+        float sv[K > 1 ? K - 1 : 1][V];
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) load_row(T - (K - 1) + j, sv[j]);
+        Tin* so = s_out + b * (K - 1) * (int64_t)C + c0;
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) *reinterpret_cast<raw*>(so + (int64_t)j * C) = VT::from_f(sv[j]);
+    }
+}
+
+template <typename Tin, int V, int K>
+cudaError_t launch_conv_k(const ConvArgs& a, cudaStream_t st) {
+    const int n_cv = a.C / V;
+    const int tiles = a.T > 0 ? (a.T + kConvRows - 1) / kConvRows : 1;
+    const dim3 grid((unsigned)((n_cv + kConvThreads - 1) / kConvThreads), (unsigned)tiles, (unsigned)a.B);
+    const Tin* x = static_cast<const Tin*>(a.x);
+    const Tin* s_in = static_cast<const Tin*>(a.state_in);
+    Tin* y = static_cast<Tin*>(a.y);
+    Tin* s_out = static_cast<Tin*>(a.state_out);
+    if (a.activation)
+        causal_conv1d_kernel<Tin, V, K, true><<<grid, kConvThreads, 0, st>>>(x, a.ld_x, a.weight, s_in, y, s_out,
+                                                                             a.T, a.C, a.head_dim);
+    else
+        causal_conv1d_kernel<Tin, V, K, false><<<grid, kConvThreads, 0, st>>>(x, a.ld_x, a.weight, s_in, y, s_out,
+                                                                              a.T, a.C, a.head_dim);
+    return counted(cudaGetLastError());
+}
+
+template <typename Tin, int V>
+cudaError_t launch_conv_v(const ConvArgs& a, cudaStream_t st) {
+    switch (a.K) {
+        case 1: return launch_conv_k<Tin, V, 1>(a, st);
+        case 2: return launch_conv_k<Tin, V, 2>(a, st);
+        case 3: return launch_conv_k<Tin, V, 3>(a, st);
+        default: return launch_conv_k<Tin, V, 4>(a, st);
+    }
+}
+
+// ---- gated RMSNorm ------------------------------------------------------------------------
+//
+// One warp per output row (b, t, h) of D channels, D / 32 consecutive channels per lane.
+// x is read head-major [B, H, T, D] (the layout the rule writes o in) or token-major
+// [B, T, H, D]; z and y are token-major, the layout the output projection reads.
+
+constexpr int kNormWarps = 8;
+
+template <typename Tin, int D, bool SILU, bool X_HEAD_MAJOR>
+__global__ void __launch_bounds__(kNormWarps * 32)
+rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, const float* __restrict__ w,
+                      Tin* __restrict__ y, int64_t rows, int T, int H, float eps) {
+    constexpr int E = D / 32;                                  // channels per lane
+    constexpr int VW = E < 16 / (int)sizeof(Tin) ? E : 16 / (int)sizeof(Tin);   // per access
+    constexpr int NV = E / VW;
+    static_assert(E * 32 == D && NV * VW == E, "D / 32 channels per lane in whole accesses");
+    using VT = Vec<Tin, VW>;
+    using raw = typename VT::raw;
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    // r = (b T + t) H + h
+    int64_t xr = r;
+    if (X_HEAD_MAJOR) {
+        const int64_t h = r % H, bt = r / H;
+        const int64_t t = bt % T, b = bt / T;
+        xr = (b * H + h) * T + t;
+    }
+    float xf[E], zf[E];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + lane * E + u * VW), xf + u * VW);
+        VT::to_f(*reinterpret_cast<const raw*>(z + r * D + lane * E + u * VW), zf + u * VW);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(xf[e], xf[e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = 1.f / sqrtf(ss / (float)D + eps);
+    float out[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float gate = SILU ? silu(zf[e]) : sigmoid(zf[e]);
+        out[e] = w[lane * E + e] * (xf[e] * inv) * gate;
+    }
+#pragma unroll
+    for (int u = 0; u < NV; ++u) *reinterpret_cast<raw*>(y + r * D + lane * E + u * VW) = VT::from_f(out + u * VW);
+}
+
+template <typename Tin, int D>
+cudaError_t launch_norm_d(const NormArgs& a, cudaStream_t st) {
+    const int64_t rows = a.B * a.T * a.H;
+    const dim3 grid((unsigned)((rows + kNormWarps - 1) / kNormWarps));
+    const Tin* x = static_cast<const Tin*>(a.x);
+    const Tin* z = static_cast<const Tin*>(a.z);
+    Tin* y = static_cast<Tin*>(a.y);
+    const int T = (int)a.T, H = (int)a.H;
+    if (a.silu) {
+        if (a.x_head_major)
+            rms_norm_gated_kernel<Tin, D, true, true><<<grid, kNormWarps * 32, 0, st>>>(x, z, a.weight, y, rows, T, H, a.eps);
+        else
+            rms_norm_gated_kernel<Tin, D, true, false><<<grid, kNormWarps * 32, 0, st>>>(x, z, a.weight, y, rows, T, H, a.eps);
+    } else {
+        if (a.x_head_major)
+            rms_norm_gated_kernel<Tin, D, false, true><<<grid, kNormWarps * 32, 0, st>>>(x, z, a.weight, y, rows, T, H, a.eps);
+        else
+            rms_norm_gated_kernel<Tin, D, false, false><<<grid, kNormWarps * 32, 0, st>>>(x, z, a.weight, y, rows, T, H, a.eps);
+    }
+    return counted(cudaGetLastError());
+}
+
+template <typename Tin>
+cudaError_t launch_norm_t(const NormArgs& a, cudaStream_t st) {
+    switch (a.D) {
+        case 64: return launch_norm_d<Tin, 64>(a, st);
+        case 128: return launch_norm_d<Tin, 128>(a, st);
+        default: return launch_norm_d<Tin, 256>(a, st);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st) {
+    if (a.bf16) return a.vec ? launch_conv_v<__nv_bfloat16, 8>(a, st) : launch_conv_v<__nv_bfloat16, 1>(a, st);
+    return a.vec ? launch_conv_v<float, 4>(a, st) : launch_conv_v<float, 1>(a, st);
+}
+
+cudaError_t launch_rms_norm_gated(const NormArgs& a, cudaStream_t st) {
+    return a.bf16 ? launch_norm_t<__nv_bfloat16>(a, st) : launch_norm_t<float>(a, st);
+}
+
+}  // namespace dn

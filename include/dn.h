@@ -259,6 +259,57 @@ DN_API int dn_decode_step_gdn(const void* q, const void* k, const void* v, const
                               int B, int H, int d_k, int d_v, float scale, dn_dtype dtype, void* cuda_stream);
 
 /*
+ * dn_causal_conv1d -- step 2 of the Gated DeltaNet layer ("Linear attention
+ * and Gated DeltaNet", ch. 28, "The full layer", causal_conv1d): a depthwise
+ * causal convolution over time, one length-K filter per channel, then SiLU,
+ * carrying the previous K-1 inputs as its state.  With joined = the K-1 state
+ * rows followed by the T rows of x,
+ *   y[t][c] = act( sum_{j<K} weight[c][j] * joined[t + j][c] ),
+ * so weight[c][K-1] multiplies the current input; the new state is the last
+ * K-1 rows of joined.  fp32 arithmetic, one rounding at each store.
+ *
+ *   x          [B, T, ld_x] dtype, token-major; channels 0..C-1 of each row
+ *              are used (ld_x >= C: x may be a column slice of a wider
+ *              projection output, e.g. the q, k or v part)
+ *   weight     [C, K] fp32
+ *   state_in   [B, K-1, C] dtype, oldest row first, or NULL (zeros)
+ *   y          [B, C / head_dim, T, head_dim] dtype: head-major, the layout
+ *              dn_chunk_fwd and dn_decode_step read (head_dim = C gives
+ *              [B, T, C])
+ *   state_out  [B, K-1, C] dtype, or NULL.  It may be state_in itself when
+ *              T <= 16 (a decode step); otherwise it must not overlap it.
+ *   1 <= K <= 4; head_dim divides C; activation 1 = SiLU, 0 = none.  With
+ *   T = 0 only the state moves (x and y may be NULL).
+ *   Returns DN_ERR_INVALID on bad sizes, overlaps (y with any input, state_out
+ *   with x, weight or y) or misalignment (x, y and the states 2-byte (bf16) or
+ *   4-byte (f32) aligned, weight 4-byte); the kernel uses 16-byte accesses
+ *   when every pointer, ld_x, C and head_dim allow them.
+ */
+DN_API int dn_causal_conv1d(const void* x, int ld_x, const float* weight, const void* state_in,
+                            void* y, void* state_out, int B, int T, int C, int K, int head_dim,
+                            int activation, dn_dtype dtype, void* cuda_stream);
+
+/*
+ * dn_rms_norm_gated -- step 7 of the Gated DeltaNet layer ("Linear attention
+ * and Gated DeltaNet", ch. 28, RMSNormGated): each head's output row divided
+ * by its root mean square, times a per-channel weight and a gate of z,
+ *   y = weight * x / sqrt(mean(x^2) + eps) * act(z),  act = SiLU or sigmoid,
+ * in fp32 with one rounding at the store.
+ *
+ *   x       [B, H, T, D] dtype if x_head_major (the layout dn_chunk_fwd writes
+ *           o in; a decode step's o [B, H, D] is either layout with T = 1),
+ *           else [B, T, H, D]
+ *   z       [B, T, H, D] dtype;  y [B, T, H, D] dtype (token-major, the
+ *           output projection's layout), must not overlap x, z or weight
+ *   weight  [D] fp32, shared by every head
+ *   D in {64, 128, 256}; eps >= 0 and finite; activation 1 = SiLU, 0 = sigmoid.
+ *   x, z, y 16-byte aligned, weight 4-byte.
+ */
+DN_API int dn_rms_norm_gated(const void* x, const void* z, const float* weight, void* y,
+                             int B, int T, int H, int D, float eps, int x_head_major,
+                             int activation, dn_dtype dtype, void* cuda_stream);
+
+/*
  * dn_device_status -- synchronise `cuda_stream`, then read and clear the
  * status word of the current device.  Returns DN_ERR_TIMEOUT if a kernel of
  * this library launched since the previous call gave up on a bounded wait
@@ -274,7 +325,8 @@ DN_API const char* dn_status_str(int status);
 DN_API const char* dn_last_error(void);
 
 /* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path;
- * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn; 2.5: dn_decode_step_gdn. */
+ * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn; 2.5: dn_decode_step_gdn;
+ * 2.6: dn_causal_conv1d, dn_rms_norm_gated. */
 DN_API int dn_version(void);
 
 /*

@@ -213,3 +213,76 @@ def test_decode_layer_rejects_missing_params(lib):
     st = lib.dn_decode_step_gdn(A0, A0 + STEP, A0 + 2 * STEP, A0 + 3 * STEP, A0 + 4 * STEP, None, None,
                                 A0 + 5 * STEP, A0 + 6 * STEP, 2, 3, 128, 128, 1.0, 1, None)
     assert st == dn.DN_ERR_INVALID and b"A_log" in lib.dn_last_error()
+
+
+def conv_call(lib, **over):
+    args = dict(x=A, ld_x=256, w=A + STEP, s_in=None, y=A + 2 * STEP, s_out=None, B=2, T=40, C=256, K=4,
+                hd=128, act=1, dtype=1)
+    args.update(over)
+    return lib.dn_causal_conv1d(args["x"], args["ld_x"], args["w"], args["s_in"], args["y"], args["s_out"],
+                                args["B"], args["T"], args["C"], args["K"], args["hd"], args["act"], args["dtype"],
+                                None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(K=5), dn.DN_ERR_UNSUPPORTED),
+    (dict(K=0), dn.DN_ERR_UNSUPPORTED),
+    (dict(T=-1), dn.DN_ERR_INVALID),
+    (dict(dtype=7), dn.DN_ERR_INVALID),
+    (dict(act=2), dn.DN_ERR_INVALID),
+    (dict(ld_x=100), dn.DN_ERR_INVALID),                  # ld_x < C
+    (dict(hd=100), dn.DN_ERR_INVALID),                    # does not divide C
+    (dict(hd=0), dn.DN_ERR_INVALID),
+    (dict(w=None), dn.DN_ERR_INVALID),
+    (dict(y=None), dn.DN_ERR_INVALID),
+    (dict(x=None), dn.DN_ERR_INVALID),
+    (dict(x=A + 1), dn.DN_ERR_INVALID),                   # bf16 needs 2-byte alignment
+    (dict(w=A + STEP + 2), dn.DN_ERR_INVALID),
+    (dict(y=A + 100), dn.DN_ERR_INVALID),                 # y overlaps x
+    (dict(s_out=A + 64), dn.DN_ERR_INVALID),              # state_out overlaps x
+    (dict(s_in=A + 3 * STEP, s_out=A + 3 * STEP), dn.DN_ERR_INVALID),        # in place needs T <= 16
+    (dict(s_in=A + 3 * STEP, s_out=A + 3 * STEP + 512), dn.DN_ERR_INVALID),  # partial overlap
+    (dict(T=16 * 65535 + 1), dn.DN_ERR_UNSUPPORTED),
+])
+def test_causal_conv1d_rejects(lib, over, code):
+    assert conv_call(lib, **over) == code, lib.dn_last_error()
+
+
+def test_causal_conv1d_empty_is_ok(lib):
+    assert conv_call(lib, B=0) == dn.DN_OK
+    assert conv_call(lib, C=0, ld_x=0, hd=1) == dn.DN_OK
+    assert conv_call(lib, T=0, x=None) == dn.DN_OK           # no state out: nothing to do
+    assert conv_call(lib, K=1, T=0, s_out=A + 3 * STEP) == dn.DN_OK
+
+
+def norm_call(lib, **over):
+    args = dict(x=A, z=A + STEP, w=A + 2 * STEP, y=A + 3 * STEP, B=2, T=10, H=4, D=128, eps=1e-6, hm=1, act=1,
+                dtype=1)
+    args.update(over)
+    return lib.dn_rms_norm_gated(args["x"], args["z"], args["w"], args["y"], args["B"], args["T"], args["H"],
+                                 args["D"], args["eps"], args["hm"], args["act"], args["dtype"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(D=96), dn.DN_ERR_UNSUPPORTED),
+    (dict(D=512), dn.DN_ERR_UNSUPPORTED),
+    (dict(B=-1), dn.DN_ERR_INVALID),
+    (dict(eps=-1.0), dn.DN_ERR_INVALID),
+    (dict(eps=float("nan")), dn.DN_ERR_INVALID),
+    (dict(eps=float("inf")), dn.DN_ERR_INVALID),
+    (dict(hm=2), dn.DN_ERR_INVALID),
+    (dict(act=3), dn.DN_ERR_INVALID),
+    (dict(dtype=5), dn.DN_ERR_INVALID),
+    (dict(z=None), dn.DN_ERR_INVALID),
+    (dict(x=A + 8), dn.DN_ERR_INVALID),                   # 16-byte alignment
+    (dict(w=A + 2 * STEP + 2), dn.DN_ERR_INVALID),
+    (dict(y=A + STEP + 4096), dn.DN_ERR_INVALID),         # y overlaps z
+    (dict(y=A), dn.DN_ERR_INVALID),                       # y is x: not in place
+])
+def test_rms_norm_gated_rejects(lib, over, code):
+    assert norm_call(lib, **over) == code, lib.dn_last_error()
+
+
+def test_rms_norm_gated_empty_is_ok(lib):
+    assert norm_call(lib, T=0) == dn.DN_OK
+    assert norm_call(lib, H=0, x=None, z=None, y=None) == dn.DN_OK
