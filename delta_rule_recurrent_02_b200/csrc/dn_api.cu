@@ -374,10 +374,10 @@ int dn_causal_conv1d(const void* x, int ld_x, const float* weight, const void* s
     if (overlap(rso, rx) || overlap(rso, rw)) return fail(DN_ERR_INVALID, "state_out overlaps x or weight");
     if (overlap(rso, rsi) && !(state_out == state_in && T <= 16))
         return fail(DN_ERR_INVALID, "state_out may be state_in itself only when T <= 16; otherwise it must not overlap it");
-    const int V = (int)(16 / esz);
+    const int V = (int)(8 / esz);     // channels per 8-byte access
     bool vec = C % V == 0 && ld_x % V == 0 && head_dim % V == 0;
     for (const void* p : pe)
-        if (p && !aligned(p, 16)) vec = false;
+        if (p && !aligned(p, 8)) vec = false;
     dn::ConvArgs a;
     a.x = x; a.ld_x = ld_x; a.weight = weight; a.state_in = state_in; a.y = y; a.state_out = state_out;
     a.B = B; a.T = T; a.C = C; a.K = K; a.head_dim = head_dim;

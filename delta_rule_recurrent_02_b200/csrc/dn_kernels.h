@@ -58,7 +58,7 @@ struct ConvArgs {
     int T, C, K, head_dim;
     bool activation;          // SiLU
     bool bf16;
-    bool vec;                 // 16-byte accesses (alignment checked by the caller)
+    bool vec;                 // 8-byte accesses (alignment checked by the caller)
 };
 cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st);
 

@@ -5,8 +5,8 @@
 //   channel, then SiLU) with the previous K-1 inputs carried as its state;
 //   step 7, the gated RMSNorm of each head's output row.
 //
-// Both are streaming work bound by HBM: 16-byte vector loads across channels
-// (coalesced), fp32 arithmetic, one rounding at the store.
+// Both are streaming work bound by HBM: vector loads across channels (coalesced),
+// fp32 arithmetic, one rounding at the store.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -15,7 +15,7 @@
 namespace dn {
 namespace {
 
-// ---- element access: V consecutive channels as one 16-byte (or scalar) access --------
+// ---- element access: V consecutive channels as one vector (or scalar) access ----------
 
 template <typename T, int V>
 struct Vec;
@@ -94,16 +94,19 @@ struct Vec<float, 2> {
     __device__ static raw from_f(const float* f) { return make_float2(f[0], f[1]); }
 };
 
-__device__ __forceinline__ float silu(float x) { return x / (1.f + expf(-x)); }
-__device__ __forceinline__ float sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+// SiLU and the logistic sigmoid through the fast exp and a correctly rounded reciprocal:
+// for very negative x the exp overflows to inf and the reciprocal gives 0, the right limit
+__device__ __forceinline__ float sigmoid(float x) { return __frcp_rn(1.f + __expf(-x)); }
+__device__ __forceinline__ float silu(float x) { return x * sigmoid(x); }
 
 // ---- causal conv ----------------------------------------------------------------------
 //
 // Thread = V consecutive channels of one sequence over kConvRows consecutive tokens.
-// Its rows, plus the K-1 before them (from x, or from the carried state before token 0),
-// are loaded up front so that every load of the tile is in flight at once; the filter
-// then slides over them in registers.  The block whose tile holds the last token also
-// writes the new state (the last K-1 inputs of history-then-x).
+// The block's filters are staged once in shared memory, tap-major, from coalesced
+// reads.  A thread's rows, plus the K-1 before them (from x, or from the carried state
+// before token 0), are loaded up front so that every load of the tile is in flight at
+// once; the filter then slides over them in registers.  The block whose tile holds the
+// last token also writes the new state (the last K-1 inputs of history-then-x).
 
 constexpr int kConvRows = 16;
 constexpr int kConvThreads = 128;
@@ -114,17 +117,36 @@ causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __res
                      Tin* __restrict__ y, Tin* s_out, int T, int C, int hd) {
     using VT = Vec<Tin, V>;
     using raw = typename VT::raw;
-    const int cv = blockIdx.x * kConvThreads + threadIdx.x;
-    const int c0 = cv * V;
+    constexpr int kCh = kConvThreads * V;       // channels of the block
+    constexpr int kRow = kCh + 4;               // padded tap row: 16-byte aligned, banks shifted
+    __shared__ __align__(16) float ws[K][kRow];
+    const int cb0 = blockIdx.x * kCh;
+    const int nch = min(kCh, C - cb0);
+    for (int e = threadIdx.x; e < nch * K; e += kConvThreads) {
+        const int ch = e / K;
+        ws[e - ch * K][ch] = w[(int64_t)cb0 * K + e];
+    }
+    __syncthreads();
+    const int cl = threadIdx.x * V;
+    const int c0 = cb0 + cl;
     if (c0 >= C) return;
     const int64_t b = blockIdx.z;
     const int t0 = blockIdx.y * kConvRows;
 
     float wf[K][V];
 #pragma unroll
-    for (int v = 0; v < V; ++v)
+    for (int j = 0; j < K; ++j) {
+        if constexpr (V % 4 == 0) {
 #pragma unroll
-        for (int j = 0; j < K; ++j) wf[j][v] = w[(int64_t)(c0 + v) * K + j];
+            for (int v = 0; v < V; v += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(&ws[j][cl + v]);
+                wf[j][v] = f.x; wf[j][v + 1] = f.y; wf[j][v + 2] = f.z; wf[j][v + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) wf[j][v] = ws[j][cl + v];
+        }
+    }
 
     // input row t of this thread's channels: x for t >= 0, the carried state before
     const Tin* xb = x + b * T * ld_x + c0;
@@ -158,25 +180,32 @@ causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __res
     const int nh = C / hd;
     const int head = c0 / hd, jj = c0 - head * hd;
     Tin* yb = y + ((b * nh + head) * (int64_t)T) * hd + jj;
+    // sliding window of the K input rows behind output t, as floats: each row is
+    // converted once
+    float win[K][V];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) VT::to_f(rows[j], win[j]);
 #pragma unroll
     for (int i = 0; i < kConvRows; ++i) {
         const int t = t0 + i;
         if (t < T) {
+            VT::to_f(rows[i + K - 1], win[K - 1]);
             float acc[V];
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[v] = 0.f;
 #pragma unroll
-            for (int j = 0; j < K; ++j) {
-                float f[V];
-                VT::to_f(rows[i + j], f);
+            for (int j = 0; j < K; ++j)
 #pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = fmaf(wf[j][v], f[v], acc[v]);
-            }
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(wf[j][v], win[j][v], acc[v]);
             if (ACT) {
 #pragma unroll
                 for (int v = 0; v < V; ++v) acc[v] = silu(acc[v]);
             }
             *reinterpret_cast<raw*>(yb + (int64_t)t * hd) = VT::from_f(acc);
+#pragma unroll
+            for (int j = 0; j < K - 1; ++j)
+#pragma unroll
+                for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
         }
     }
 
@@ -223,10 +252,14 @@ cudaError_t launch_conv_v(const ConvArgs& a, cudaStream_t st) {
 // ---- gated RMSNorm ------------------------------------------------------------------------
 //
 // One warp per output row (b, t, h) of D channels, D / 32 consecutive channels per lane.
-// x is read head-major [B, H, T, D] (the layout the rule writes o in) or token-major
-// [B, T, H, D]; z and y are token-major, the layout the output projection reads.
+// A warp may take kNormRows rows, loading all of them before reducing any; one row per
+// warp measured faster on B200 than four (four halve the resident warps for a small
+// gain in loads in flight).  x is read head-major [B, H, T, D] (the layout the rule
+// writes o in) or token-major [B, T, H, D]; z and y are token-major, the layout the
+// output projection reads.
 
 constexpr int kNormWarps = 8;
+constexpr int kNormRows = 1;
 
 template <typename Tin, int D, bool SILU, bool X_HEAD_MAJOR>
 __global__ void __launch_bounds__(kNormWarps * 32)
@@ -239,41 +272,57 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
     using VT = Vec<Tin, VW>;
     using raw = typename VT::raw;
     const int lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5);
-    if (r >= rows) return;
-    // r = (b T + t) H + h
-    int64_t xr = r;
-    if (X_HEAD_MAJOR) {
-        const int64_t h = r % H, bt = r / H;
-        const int64_t t = bt % T, b = bt / T;
-        xr = (b * H + h) * T + t;
-    }
-    float xf[E], zf[E];
+    const int64_t r0 = ((int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5)) * kNormRows;
+    if (r0 >= rows) return;
+    float wl[E];
 #pragma unroll
-    for (int u = 0; u < NV; ++u) {
-        VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + lane * E + u * VW), xf + u * VW);
-        VT::to_f(*reinterpret_cast<const raw*>(z + r * D + lane * E + u * VW), zf + u * VW);
-    }
-    float ss = 0.f;
+    for (int e = 0; e < E; ++e) wl[e] = w[lane * E + e];
+    float xf[kNormRows][E], zf[kNormRows][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) ss = fmaf(xf[e], xf[e], ss);
+    for (int u = 0; u < kNormRows; ++u) {
+        const int64_t r = r0 + u;                  // r = (b T + t) H + h
+        if (r < rows) {
+            int64_t xr = r;
+            if (X_HEAD_MAJOR) {
+                const int64_t h = r % H, bt = r / H;
+                const int64_t t = bt % T, b = bt / T;
+                xr = (b * H + h) * T + t;
+            }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = 1.f / sqrtf(ss / (float)D + eps);
-    float out[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const float gate = SILU ? silu(zf[e]) : sigmoid(zf[e]);
-        out[e] = w[lane * E + e] * (xf[e] * inv) * gate;
+            for (int a = 0; a < NV; ++a) {
+                VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + lane * E + a * VW), xf[u] + a * VW);
+                VT::to_f(*reinterpret_cast<const raw*>(z + r * D + lane * E + a * VW), zf[u] + a * VW);
+            }
+        }
     }
 #pragma unroll
-    for (int u = 0; u < NV; ++u) *reinterpret_cast<raw*>(y + r * D + lane * E + u * VW) = VT::from_f(out + u * VW);
+    for (int u = 0; u < kNormRows; ++u) {
+        const int64_t r = r0 + u;
+        if (r < rows) {
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) ss = fmaf(xf[u][e], xf[u][e], ss);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = 1.f / sqrtf(ss / (float)D + eps);
+            float out[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float gate = SILU ? silu(zf[u][e]) : sigmoid(zf[u][e]);
+                out[e] = wl[e] * (xf[u][e] * inv) * gate;
+            }
+#pragma unroll
+            for (int a = 0; a < NV; ++a)
+                *reinterpret_cast<raw*>(y + r * D + lane * E + a * VW) = VT::from_f(out + a * VW);
+        }
+    }
 }
 
 template <typename Tin, int D>
 cudaError_t launch_norm_d(const NormArgs& a, cudaStream_t st) {
     const int64_t rows = a.B * a.T * a.H;
-    const dim3 grid((unsigned)((rows + kNormWarps - 1) / kNormWarps));
+    const int64_t per_block = (int64_t)kNormWarps * kNormRows;
+    const dim3 grid((unsigned)((rows + per_block - 1) / per_block));
     const Tin* x = static_cast<const Tin*>(a.x);
     const Tin* z = static_cast<const Tin*>(a.z);
     Tin* y = static_cast<Tin*>(a.y);
@@ -303,9 +352,10 @@ cudaError_t launch_norm_t(const NormArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+// 8-byte accesses where the layout allows (a.vec): 4 bf16 or 2 fp32 channels per thread
 cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st) {
-    if (a.bf16) return a.vec ? launch_conv_v<__nv_bfloat16, 8>(a, st) : launch_conv_v<__nv_bfloat16, 1>(a, st);
-    return a.vec ? launch_conv_v<float, 4>(a, st) : launch_conv_v<float, 1>(a, st);
+    if (a.bf16) return a.vec ? launch_conv_v<__nv_bfloat16, 4>(a, st) : launch_conv_v<__nv_bfloat16, 1>(a, st);
+    return a.vec ? launch_conv_v<float, 2>(a, st) : launch_conv_v<float, 1>(a, st);
 }
 
 cudaError_t launch_rms_norm_gated(const NormArgs& a, cudaStream_t st) {

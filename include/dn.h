@@ -282,7 +282,7 @@ DN_API int dn_decode_step_gdn(const void* q, const void* k, const void* v, const
  *   T = 0 only the state moves (x and y may be NULL).
  *   Returns DN_ERR_INVALID on bad sizes, overlaps (y with any input, state_out
  *   with x, weight or y) or misalignment (x, y and the states 2-byte (bf16) or
- *   4-byte (f32) aligned, weight 4-byte); the kernel uses 16-byte accesses
+ *   4-byte (f32) aligned, weight 4-byte); the kernel uses 8-byte accesses
  *   when every pointer, ld_x, C and head_dim allow them.
  */
 DN_API int dn_causal_conv1d(const void* x, int ld_x, const float* weight, const void* state_in,
