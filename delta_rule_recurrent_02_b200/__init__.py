@@ -11,8 +11,14 @@ Functions with the ABI's names take preallocated outputs:
 
     dn_chunk_fwd(q, k, v, beta, g, S0, o, S_T, chunk=64, scale=1.0, workspace=None, ...)
     dn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, chunk=64, dtype="bf16", gate="scalar", path="auto")
+    dn_chunk_fwd_snapshots(q, k, v, beta, g, S0, o, S_T, snaps, every, ...)
+    dn_chunk_fwd_gdn(q, k, v, b, a, A_log, dt_bias, S0, o, S_T, scale=1.0, ...)   # layer prologue fused in
     dn_decode_step(q, k, v, beta, g, S, o, scale=1.0, ...)
+    dn_decode_step_gdn(q, k, v, b, a, A_log, dt_bias, S, o, scale=1.0, ...)
+    dn_causal_conv1d(x, weight, y, state_in=None, state_out=None, head_dim=None, activation=True)
+    dn_rms_norm_gated(x, z, weight, y, eps=1e-6, x_head_major=True, activation="silu")
     dn_device_status(stream=None)
+    dn_kernel_launches()
 
 and two conveniences allocate the outputs (and the prefill's workspace) with torch:
 
