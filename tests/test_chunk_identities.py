@@ -14,7 +14,9 @@ state:
   - Q-hat rows carry r_q, and the rows of U~ carry r_k;
 - a fold that keeps r_k out of the state pass: u' = diag(r_k) u,
   W' = diag(r_k) W and P' = P diag(1/r_k), so that U' = u' - W'S = diag(r_k) U,
-  K^T U~' = K-hat^T U~ and P'U' = PU.
+  K^T U~' = K-hat^T U~ and P'U' = PU;
+- the full fold, which also moves r_q to the output rows: P'' = scale tril(QK^T * D),
+  with no norm factor at all, Q-hat without r_q, and O = diag(r_q)(Q-hat S + P''U').
 
 The chunk equations are those of the chunked form on the same page (A, T,
 W, u, P; U = u - WS; O = Q-hat S + PU; S <- e^(G_last) S + K~^T U)."""
@@ -26,7 +28,8 @@ import oracle
 
 def chunk_pass(q, k, v, beta, g, S0, scale, C, fold, drop_rk_on_u=False):
     """One (b, h) through chunks of C with the prologue's factors placed as the
-    kernels place them (fold=False) or folded into u, W and P (fold=True).
+    kernels place them (fold=False), with r_k folded into u, W and P
+    (fold=True), or with r_q moved to the output rows as well (fold="all").
     drop_rk_on_u plants a mistake: the rows of U~ lose their r_k."""
     T = k.shape[0]
     rq = 1.0 / np.maximum(np.linalg.norm(q, axis=1), 1e-12)
@@ -51,11 +54,18 @@ def chunk_pass(q, k, v, beta, g, S0, scale, C, fold, drop_rk_on_u=False):
             o[sl] = Qh @ S + P @ U
             row = decay if drop_rk_on_u else decay * r_k
             S = np.exp(G[-1]) * S + K.T @ (row[:, None] * U)
-        else:
+        elif fold is True:
             u2, W2 = r_k[:, None] * u, r_k[:, None] * W
             P2 = P / r_k[None, :]
             U2 = u2 - W2 @ S
             o[sl] = Qh @ S + P2 @ U2
+            S = np.exp(G[-1]) * S + K.T @ (decay[:, None] * U2)
+        else:
+            u2, W2 = r_k[:, None] * u, r_k[:, None] * W
+            P3 = scale * np.tril((Q @ K.T) * D)                 # the plain path's P
+            Qh3 = (scale * np.exp(G))[:, None] * Q                # the plain path's Q-hat
+            U2 = u2 - W2 @ S
+            o[sl] = r_q[:, None] * (Qh3 @ S + P3 @ U2)
             S = np.exp(G[-1]) * S + K.T @ (decay[:, None] * U2)
     return o, S
 
@@ -70,7 +80,7 @@ def layer_case(T, seed, dk=16, dv=12):
     return q, k, v, beta[0, 0], g[0, 0], S0, qn, kn
 
 
-@pytest.mark.parametrize("fold", [False, True])
+@pytest.mark.parametrize("fold", [False, True, "all"])
 @pytest.mark.parametrize("T,C", [(37, 8), (64, 16), (50, 64)])
 def test_prologue_factor_placement_matches_recurrence(fold, T, C):
     q, k, v, beta, g, S0, qn, kn = layer_case(T, 100 + T + C)
@@ -90,3 +100,21 @@ def test_factor_placement_catches_a_dropped_factor():
     o, S = chunk_pass(q, k, v, beta, g, S0, 1.0, 8, fold=False, drop_rk_on_u=True)
     assert np.abs(S - S_ref[0, 0]).max() > 1e-3 * np.abs(S_ref).max()
     assert np.abs(o - o_ref[0, 0]).max() > 1e-3 * np.abs(o_ref).max()
+
+
+def test_full_fold_with_zero_rows():
+    """A zero key row gets r_k = 1e12 and a zero query row r_q = 1e12 (the
+    max(||x||, 1e-12) clamp).  The fold then scales u and W rows by 1e12, and
+    still matches the recurrence, whose unit key and query are zero there."""
+    q, k, v, beta, g, S0, qn, kn = layer_case(30, 11)
+    q[3] = 0.0; k[5] = 0.0; k[17] = 0.0
+    qn, kn, _, _ = oracle.gdn_prologue(q[None, None], k[None, None], np.zeros((1, 1, 30)), np.zeros((1, 1, 30)),
+                                       np.zeros(1), np.zeros(1))
+    scale = q.shape[1] ** -0.5
+    o_ref, S_ref = oracle.delta_rule(qn, kn, v[None, None], beta[None, None], g[None, None], S0[None, None],
+                                     scale=scale)
+    o, S = chunk_pass(q, k, v, beta, g, S0, scale, 8, "all")
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    assert np.allclose(o, o_ref[0, 0], rtol=0, atol=1e-9 * np.abs(o_ref).max())
+    assert np.allclose(S, S_ref[0, 0], rtol=0, atol=1e-9 * np.abs(S_ref).max())
+    assert not o[3].any() or np.abs(o[3]).max() <= 1e-9 * np.abs(o_ref).max()
