@@ -21,6 +21,8 @@ Contents
                           (kernel K, SiLU) with the K-1 previous inputs carried.
 ``rms_norm_gated``        step 7 of the layer: RMSNorm of each head's output
                           times a per-channel weight and SiLU (or sigmoid) of z.
+``generalized_delta_rule`` RWKV-7's form: per-channel decay, removal key and
+                          rate, and a separate write key.
 
 Every function takes and returns numpy arrays.  Layouts: tokens
 ``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
@@ -309,14 +311,17 @@ def wy_transition(k, beta, g=None):
     return np.diag(np.exp(Gam[-1])) - (k * np.exp(Gam[-1][None, :] - Gam)).T @ W
 
 
-def gdn_prologue(q, k, b, a, A_log, dt_bias, eps=1e-12):
+def gdn_prologue(q, k, b, a, A_log, dt_bias, eps=1e-12, allow_neg_eigval=False):
     """Steps 4 and 5 of the Gated DeltaNet layer ("Linear attention and Gated
     DeltaNet", ch. 28, "The full layer"), in fp64, on raw per-token inputs:
 
     - q and k normalised over the head dimension, x / max(||x||_2, eps): the
       pages call l2norm without defining it and elsewhere use the
       F.normalize contract for unit keys, which this restates;
-    - beta = sigmoid(b), the write strength in (0, 1);
+    - beta = sigmoid(b), the write strength in (0, 1); with allow_neg_eigval,
+      beta = 2 sigmoid(b) in (0, 2), so that I - beta k k^T can have a negative
+      eigenvalue along k ("DeltaNet: Memory That Edits", "The reflection
+      hiding in the delta rule");
     - g = -exp(A_log[h]) * softplus(a + dt_bias[h]), the log-decay (always
       negative), with softplus(x) = log(1 + e^x) (numpy's logaddexp(0, x)).
 
@@ -327,7 +332,7 @@ def gdn_prologue(q, k, b, a, A_log, dt_bias, eps=1e-12):
     A_log, dt_bias = _f64(A_log), _f64(dt_bias)
     qn = q / np.maximum(np.linalg.norm(q, axis=-1, keepdims=True), eps)
     kn = k / np.maximum(np.linalg.norm(k, axis=-1, keepdims=True), eps)
-    beta = 1.0 / (1.0 + np.exp(-b))
+    beta = (2.0 if allow_neg_eigval else 1.0) / (1.0 + np.exp(-b))
     g = -np.exp(A_log)[None, :, None] * np.logaddexp(0.0, a + dt_bias[None, :, None])
     return qn, kn, beta, g
 
@@ -384,3 +389,32 @@ def rms_norm_gated(x, z, weight, eps=1e-6, activation="silu"):
     else:
         raise ValueError(f"activation {activation!r}")
     return weight * normed * gate
+
+
+def generalized_delta_rule(q, w, kappa, a, k_write, v, S0=None, scale=1.0):
+    """The generalised delta rule of RWKV-7 ("DeltaNet: Memory That Edits",
+    "The generalized delta rule"), token by token in fp64:
+
+        S_t = (diag(w_t) - (a_t * kappa_t) kappa_t^T) S_{t-1} + k_write_t v_t^T,
+        o_t = S_t^T (scale q_t),
+
+    with a per-channel decay w_t, a removal key kappa_t, a per-channel removal
+    rate a_t and a write key k_write_t that need not equal kappa_t.  The page
+    writes the state in the d_k x d_v orientation used here; the read-out
+    through q follows the rest of the family (o = S^T q).  Tying them,
+    w = 1, kappa = k, a = beta, k_write = beta k, gives DeltaNet.
+
+    q, w, kappa, a, k_write [B,H,T,d_k]; v [B,H,T,d_v]; S0 [B,H,d_k,d_v] or
+    None.  Returns ``(o, S_T)``."""
+    q, w, kappa, a, k_write, v = (_f64(x) for x in (q, w, kappa, a, k_write, v))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    S = np.zeros((B, H, dk, dv)) if S0 is None else _f64(S0).copy()
+    o = np.zeros((B, H, T, dv))
+    for t in range(T):
+        removed = np.einsum("bhk,bhkv->bhv", kappa[:, :, t], S)             # kappa^T S
+        S = (w[:, :, t, :, None] * S
+             - (a[:, :, t] * kappa[:, :, t])[..., None] * removed[:, :, None, :]
+             + k_write[:, :, t, :, None] * v[:, :, t, None, :])
+        o[:, :, t] = scale * np.einsum("bhkv,bhk->bhv", S, q[:, :, t])
+    return o, S

@@ -507,3 +507,105 @@ def test_rms_norm_gated_eps_and_zero_row():
     assert not y[0].any()
     expect = 1e-3 / np.sqrt(1e-6 + 1e-6) / (1 + np.exp(-50.0))
     assert np.allclose(y[1], expect, rtol=1e-14)
+
+
+# ---- generalized_delta_rule: pinned by the ties the page states, a brute-force
+#      expansion and the reflection eigenvalues -----------------------------------------------
+
+def _gdr_inputs(B, H, T, dk, dv, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, T, dk))
+    k = rng.standard_normal((B, H, T, dk)); k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, H, T, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((B, H, T))))
+    S0 = 0.1 * rng.standard_normal((B, H, dk, dv))
+    return rng, q, k, v, beta, S0
+
+
+def test_generalized_rule_tied_is_deltanet():
+    """w = 1, kappa = k, a = beta, k_write = beta k: DeltaNet (the page's tie)."""
+    rng, q, k, v, beta, S0 = _gdr_inputs(2, 2, 13, 8, 6, 21)
+    bk = np.broadcast_to(beta[..., None], k.shape)
+    o, S = oracle.generalized_delta_rule(q, np.ones_like(k), k, bk, bk * k, v, S0, scale=0.5)
+    o_ref, S_ref = oracle.delta_rule(q, k, v, beta, None, S0, scale=0.5)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12) and np.allclose(S, S_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_generalized_rule_with_decay_is_gated_rule(gate):
+    """alpha (I - beta k k^T) with a scalar alpha, and (I - beta k k^T) Diag(alpha)
+    with a per-key alpha, are diag(w) - (a * kappa) kappa^T with w = alpha,
+    kappa = alpha * k, a = beta / alpha, k_write = beta k."""
+    rng, q, k, v, beta, S0 = _gdr_inputs(1, 2, 11, 8, 5, 22)
+    if gate == "scalar":
+        g = -rng.random((1, 2, 11)); alpha = np.broadcast_to(np.exp(g)[..., None], k.shape)
+    else:
+        g = -rng.random((1, 2, 11, 8)); alpha = np.exp(g)
+    kappa = alpha * k
+    a = beta[..., None] / alpha
+    o, S = oracle.generalized_delta_rule(q, alpha, kappa, a, beta[..., None] * k, v, S0)
+    o_ref, S_ref = oracle.delta_rule(q, k, v, beta, g, S0)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12) and np.allclose(S, S_ref, rtol=0, atol=1e-12)
+
+
+def test_generalized_rule_brute_force():
+    """Explicit products of the d_k x d_k transitions M_t = diag(w_t) - (a_t * kappa_t) kappa_t^T:
+    S_t = M_t ... M_1 S0 + sum_s M_t ... M_{s+1} k_write_s v_s^T, with removal and write keys
+    unrelated."""
+    rng = np.random.default_rng(23)
+    T, dk, dv = 6, 5, 4
+    q, w, kap, a, kw = (rng.standard_normal((1, 1, T, dk)) for _ in range(5))
+    w = 0.5 + 0.5 * np.abs(w)
+    v = rng.standard_normal((1, 1, T, dv)); S0 = rng.standard_normal((1, 1, dk, dv))
+    o, S = oracle.generalized_delta_rule(q, w, kap, a, kw, v, S0, scale=0.7)
+    M = [np.diag(w[0, 0, t]) - np.outer(a[0, 0, t] * kap[0, 0, t], kap[0, 0, t]) for t in range(T)]
+    for t in range(T):
+        St = S0[0, 0].copy()
+        for s in range(t + 1):
+            St = M[s] @ St
+        for s in range(t + 1):
+            P = np.eye(dk)
+            for r in range(s + 1, t + 1):
+                P = M[r] @ P
+            St = St + P @ np.outer(kw[0, 0, s], v[0, 0, s])
+        assert np.allclose(o[0, 0, t], 0.7 * St.T @ q[0, 0, t], rtol=0, atol=1e-12 * max(1, np.abs(St).max()))
+    assert np.allclose(S[0, 0], St, rtol=0, atol=1e-12 * np.abs(St).max())
+
+
+def test_generalized_rule_no_removal_is_decayed_sum():
+    """a = 0: no removal; the state is the decayed sum of the writes (a closed form)."""
+    rng = np.random.default_rng(24)
+    T, dk, dv = 9, 4, 3
+    w = np.exp(-rng.random((1, 1, T, dk))); kw = rng.standard_normal((1, 1, T, dk))
+    v = rng.standard_normal((1, 1, T, dv)); q = rng.standard_normal((1, 1, T, dk))
+    _, S = oracle.generalized_delta_rule(q, w, rng.standard_normal((1, 1, T, dk)), np.zeros((1, 1, T, dk)), kw, v)
+    ref = sum(np.prod(w[0, 0, s + 1:], axis=0)[:, None] * np.outer(kw[0, 0, s], v[0, 0, s]) for s in range(T))
+    assert np.allclose(S[0, 0], ref, rtol=1e-13, atol=1e-14)
+
+
+def test_generalized_rule_reflection_eigenvalues():
+    """With w = 1, a unit kappa and a = beta, the transition is I - beta kappa kappa^T:
+    eigenvalue 1 - beta along kappa and 1 elsewhere; the page prints -1 along k at beta = 2.
+    The step applied to S = kappa e_1^T shows it (S^T kappa scales by 1 - beta)."""
+    fix = gold("reflection.json")
+    dk = 6
+    kap = np.zeros(dk); kap[2] = 1.0
+    for row in fix["eigen"]:
+        b = row["beta"]
+        S0 = np.zeros((1, 1, dk, 1)); S0[0, 0, :, 0] = kap + np.eye(dk)[4]     # along kappa and orthogonal
+        one = np.ones((1, 1, 1, dk))
+        _, S = oracle.generalized_delta_rule(np.zeros((1, 1, 1, dk)), one, kap[None, None, None], b * one,
+                                             np.zeros((1, 1, 1, dk)), np.zeros((1, 1, 1, 1)), S0)
+        assert np.isclose(S[0, 0, 2, 0], row["along_k"], rtol=0, atol=1e-15)
+        assert np.isclose(S[0, 0, 4, 0], row["elsewhere"], rtol=0, atol=1e-15)
+
+
+def test_prologue_two_sigma_gate():
+    """allow_neg_eigval doubles the gate: beta = 2 sigmoid(b) in (0, 2), beta(0) = 1."""
+    b = np.array([0.0, 3.0, -3.0, 40.0, -40.0])[None, None]
+    z = np.zeros((1, 1, 5, 4)); p = np.zeros(1)
+    _, _, beta2, _ = oracle.gdn_prologue(z + 1, z + 1, b, b, p, p, allow_neg_eigval=True)
+    _, _, beta1, _ = oracle.gdn_prologue(z + 1, z + 1, b, b, p, p)
+    assert beta2[0, 0, 0] == 1.0
+    assert np.allclose(beta2, 2 * beta1, rtol=1e-15, atol=0)
+    assert ((beta2 > 0) & (beta2 <= 2)).all() and np.isclose(beta2[0, 0, 1] + beta2[0, 0, 2], 2.0, rtol=1e-15)
