@@ -23,6 +23,8 @@ Contents
                           times a per-channel weight and SiLU (or sigmoid) of z.
 ``generalized_delta_rule`` RWKV-7's form: per-channel decay, removal key and
                           rate, and a separate write key.
+``varlen_delta_rule``     sequences packed along time (cu_seqlens), each with
+                          its own initial and final state.
 
 Every function takes and returns numpy arrays.  Layouts: tokens
 ``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
@@ -418,3 +420,37 @@ def generalized_delta_rule(q, w, kappa, a, k_write, v, S0=None, scale=1.0):
              + k_write[:, :, t, :, None] * v[:, :, t, None, :])
         o[:, :, t] = scale * np.einsum("bhkv,bhk->bhv", S, q[:, :, t])
     return o, S
+
+
+def varlen_delta_rule(q, k, v, beta, g, cu_seqlens, S0=None, scale=1.0):
+    """Variable-length packing ("Linear attention and Gated DeltaNet", ch. 28,
+    "The state a request carries": every request carries its own fixed-size
+    state): N sequences packed along time, sequence n holding tokens
+    cu_seqlens[n] .. cu_seqlens[n+1]-1, each run by ``delta_rule`` from its own
+    initial state and yielding its own final state.
+
+    q, k [1,H,T_total,d_k]; v [1,H,T_total,d_v]; beta and a scalar g
+    [1,H,T_total], a per-key g [1,H,T_total,d_k], or None; cu_seqlens [N+1]
+    non-decreasing from 0 to T_total; S0 [N,H,d_k,d_v] or None.  Returns
+    ``(o [1,H,T_total,d_v], S_T [N,H,d_k,d_v])``."""
+    cu = [int(c) for c in cu_seqlens]
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    g = _f64(g)
+    _, H, T, dk = k.shape
+    dv = v.shape[-1]
+    if cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must rise from 0 to T_total")
+    N = len(cu) - 1
+    o = np.zeros((1, H, T, dv))
+    ST = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        s0 = None if S0 is None else _f64(S0)[n:n + 1]
+        if b == a:
+            ST[n] = 0.0 if s0 is None else s0[0]
+            continue
+        gn = None if g is None else g[:, :, a:b]
+        o[:, :, a:b], st = delta_rule(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], beta[:, :, a:b], gn, s0,
+                                      scale=scale)
+        ST[n] = st[0]
+    return o, ST

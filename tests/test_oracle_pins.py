@@ -609,3 +609,55 @@ def test_prologue_two_sigma_gate():
     assert beta2[0, 0, 0] == 1.0
     assert np.allclose(beta2, 2 * beta1, rtol=1e-15, atol=0)
     assert ((beta2 > 0) & (beta2 <= 2)).all() and np.isclose(beta2[0, 0, 1] + beta2[0, 0, 2], 2.0, rtol=1e-15)
+
+
+# ---- varlen_delta_rule: pinned by the zero-padding equivalence and by isolation -----------
+
+@pytest.mark.parametrize("gate", [None, "scalar", "per_key"])
+def test_varlen_equals_padded_batch(gate):
+    """Packing equals a padded batch in which every position past a sequence's end is an
+    identity step (beta = 0, g = 0): the padding reading of a partial chunk, applied to
+    whole sequences.  Includes an empty sequence."""
+    rng = np.random.default_rng(31)
+    lens = [5, 0, 11, 1, 7]
+    N, H, dk, dv, Tm = len(lens), 2, 6, 4, max(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    Tt = int(cu[-1])
+    q = rng.standard_normal((1, H, Tt, dk)); k = rng.standard_normal((1, H, Tt, dk))
+    v = rng.standard_normal((1, H, Tt, dv)); beta = 1 / (1 + np.exp(-rng.standard_normal((1, H, Tt))))
+    g = None if gate is None else -rng.random((1, H, Tt) if gate == "scalar" else (1, H, Tt, dk))
+    S0 = 0.1 * rng.standard_normal((N, H, dk, dv))
+    o, ST = oracle.varlen_delta_rule(q, k, v, beta, g, cu, S0, scale=0.3)
+    pad = lambda x, tail: np.zeros((N, H, Tm) + tail)
+    qp, kp, vp, bp = pad(q, (dk,)), pad(k, (dk,)), pad(v, (dv,)), pad(beta, ())
+    gp = None if g is None else pad(g, g.shape[3:])
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        qp[n, :, :b - a], kp[n, :, :b - a], vp[n, :, :b - a], bp[n, :, :b - a] = (
+            q[0, :, a:b], k[0, :, a:b], v[0, :, a:b], beta[0, :, a:b])
+        if g is not None:
+            gp[n, :, :b - a] = g[0, :, a:b]
+    op, STp = oracle.delta_rule(qp, kp, vp, bp, gp, S0, scale=0.3)
+    assert np.allclose(ST, STp, rtol=0, atol=1e-13)
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        assert np.allclose(o[0, :, a:b], op[n, :, :b - a], rtol=0, atol=1e-13)
+    assert np.array_equal(ST[1], S0[1])                 # the empty sequence keeps its state
+
+
+def test_varlen_sequences_are_isolated():
+    """Changing one sequence's tokens or initial state changes nothing in the others."""
+    rng = np.random.default_rng(32)
+    cu = [0, 4, 9, 16]
+    H, dk, dv, Tt = 1, 5, 3, 16
+    q, k = rng.standard_normal((1, H, Tt, dk)), rng.standard_normal((1, H, Tt, dk))
+    v, beta = rng.standard_normal((1, H, Tt, dv)), 1 / (1 + np.exp(-rng.standard_normal((1, H, Tt))))
+    S0 = rng.standard_normal((3, H, dk, dv))
+    o1, S1 = oracle.varlen_delta_rule(q, k, v, beta, None, cu, S0)
+    v2, S02 = v.copy(), S0.copy()
+    v2[:, :, 4:9] += 1.0; S02[1] += 1.0
+    o2, S2 = oracle.varlen_delta_rule(q, k, v2, beta, None, cu, S02)
+    assert np.array_equal(o1[:, :, :4], o2[:, :, :4]) and np.array_equal(o1[:, :, 9:], o2[:, :, 9:])
+    assert np.array_equal(S1[[0, 2]], S2[[0, 2]]) and not np.allclose(S1[1], S2[1])
+    with pytest.raises(ValueError):
+        oracle.varlen_delta_rule(q, k, v, beta, None, [0, 9, 4, 16], S0)
