@@ -25,6 +25,8 @@ Contents
                           rate, and a separate write key.
 ``varlen_delta_rule``     sequences packed along time (cu_seqlens), each with
                           its own initial and final state.
+``gva_delta_rule``        grouped value heads: H_v / H_k value heads share each
+                          key head's q and k.
 
 Every function takes and returns numpy arrays.  Layouts: tokens
 ``[B, H, T, d]``, beta and a scalar gate ``[B, H, T]``, a per-key gate
@@ -454,3 +456,21 @@ def varlen_delta_rule(q, k, v, beta, g, cu_seqlens, S0=None, scale=1.0):
                                       scale=scale)
         ST[n] = st[0]
     return o, ST
+
+
+def gva_delta_rule(q, k, v, beta, g=None, S0=None, scale=1.0):
+    """Grouped value heads ("Linear attention and Gated DeltaNet", ch. 28, "The
+    full layer", step 3): more value heads than key heads, each key head shared
+    by H_v / H_k consecutive value heads, so that value head h reads q and k of
+    key head h // (H_v / H_k) (the layer's repeat_interleave of q and k over the
+    head axis).  beta, g and the state belong to the value heads.
+
+    q, k [B,H_k,T,d_k]; v [B,H_v,T,d_v]; beta [B,H_v,T]; g None, [B,H_v,T] or
+    [B,H_v,T,d_k]; S0 [B,H_v,d_k,d_v] or None.  Returns ``(o [B,H_v,T,d_v],
+    S_T [B,H_v,d_k,d_v])``."""
+    q, k = _f64(q), _f64(k)
+    Hk, Hv = k.shape[1], v.shape[1]
+    if Hv % Hk != 0:
+        raise ValueError("the value heads must be a multiple of the key heads")
+    r = Hv // Hk
+    return delta_rule(np.repeat(q, r, axis=1), np.repeat(k, r, axis=1), v, beta, g, S0, scale=scale)

@@ -661,3 +661,49 @@ def test_varlen_sequences_are_isolated():
     assert np.array_equal(S1[[0, 2]], S2[[0, 2]]) and not np.allclose(S1[1], S2[1])
     with pytest.raises(ValueError):
         oracle.varlen_delta_rule(q, k, v, beta, None, [0, 9, 4, 16], S0)
+
+
+# ---- gva_delta_rule: pinned by per-head runs, linearity in v and the 1:1 case -------------
+
+def test_gva_value_heads_read_their_key_head():
+    """Value head h of a 2-key-head, 6-value-head layer equals a plain one-head run on
+    key head h // 3, as the page's repeat_interleave pairs them (not h % 2)."""
+    rng = np.random.default_rng(41)
+    B, Hk, Hv, T, dk, dv = 2, 2, 6, 9, 5, 4
+    q, k = rng.standard_normal((B, Hk, T, dk)), rng.standard_normal((B, Hk, T, dk))
+    v = rng.standard_normal((B, Hv, T, dv)); beta = 1 / (1 + np.exp(-rng.standard_normal((B, Hv, T))))
+    g = -rng.random((B, Hv, T))
+    o, ST = oracle.gva_delta_rule(q, k, v, beta, g, scale=0.4)
+    for h in range(Hv):
+        oh, sh = oracle.delta_rule(q[:, h // 3:h // 3 + 1], k[:, h // 3:h // 3 + 1], v[:, h:h + 1],
+                                   beta[:, h:h + 1], g[:, h:h + 1], scale=0.4)
+        assert np.array_equal(o[:, h:h + 1], oh) and np.array_equal(ST[:, h:h + 1], sh)
+        if h % Hk != h // 3:
+            wrong, _ = oracle.delta_rule(q[:, h % 2:h % 2 + 1], k[:, h % 2:h % 2 + 1], v[:, h:h + 1],
+                                         beta[:, h:h + 1], g[:, h:h + 1], scale=0.4)
+            assert not np.allclose(o[:, h:h + 1], wrong)
+
+
+def test_gva_is_linear_in_v_across_shared_heads():
+    """Two value heads sharing a key head, with the same beta and g: the rule is linear
+    in (v, S0), so their outputs add up to the output for v1 + v2."""
+    rng = np.random.default_rng(42)
+    B, T, dk, dv = 1, 12, 6, 3
+    q, k = rng.standard_normal((B, 1, T, dk)), rng.standard_normal((B, 1, T, dk))
+    v = rng.standard_normal((B, 2, T, dv))
+    b1 = 1 / (1 + np.exp(-rng.standard_normal((B, 1, T)))); beta = np.repeat(b1, 2, axis=1)
+    g1 = -rng.random((B, 1, T)); g = np.repeat(g1, 2, axis=1)
+    o, _ = oracle.gva_delta_rule(q, k, v, beta, g)
+    osum, _ = oracle.gva_delta_rule(q, k, v.sum(axis=1, keepdims=True), b1, g1)
+    assert np.allclose(o.sum(axis=1, keepdims=True), osum, rtol=1e-12, atol=1e-12)
+
+
+def test_gva_one_to_one_is_the_plain_rule():
+    rng = np.random.default_rng(43)
+    q, k, v = (rng.standard_normal((1, 3, 7, 4)) for _ in range(3))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((1, 3, 7))))
+    a, _ = oracle.gva_delta_rule(q, k, v, beta)
+    b, _ = oracle.delta_rule(q, k, v, beta)
+    assert np.array_equal(a, b)
+    with pytest.raises(ValueError):
+        oracle.gva_delta_rule(q[:, :2], k[:, :2], v, beta)
