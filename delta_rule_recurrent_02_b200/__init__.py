@@ -251,6 +251,43 @@ def dn_decode_step(q, k, v, beta, g, S, o, *, scale: float = 1.0, gate: str | No
     _check(lib, st)
 
 
+def _conv_check(x, weight, y, state_in, state_out, head_dim):
+    """Shapes and dtypes of a dn_causal_conv1d call (the C ABI cannot see them)."""
+    if x.dim() != 3 or weight.dim() != 2:
+        raise ValueError("dn: x must be [B, T, C] and weight [C, K]")
+    B, T, C = x.shape
+    K = weight.shape[1]
+    hd = C if head_dim is None else int(head_dim)
+    if weight.shape[0] != C:
+        raise ValueError(f"dn: weight has {weight.shape[0]} channels, x has {C}")
+    if hd <= 0 or C % hd:
+        raise ValueError(f"dn: head_dim {hd} must divide C = {C}")
+    if y.numel() != B * T * C or (y.dim() == 4 and tuple(y.shape) != (B, C // hd, T, hd)):
+        raise ValueError(f"dn: y must be [B, C // head_dim, T, head_dim] = {(B, C // hd, T, hd)}")
+    for name, t in (("state_in", state_in), ("state_out", state_out)):
+        if t is not None and tuple(t.shape) != (B, K - 1, C):
+            raise ValueError(f"dn: {name} must be [B, K - 1, C] = {(B, K - 1, C)}, got {tuple(t.shape)}")
+    for t in (y, state_in, state_out):
+        if t is not None and t.dtype != x.dtype:
+            raise ValueError("dn: y and the states must have x's dtype")
+
+
+def _norm_check(x, z, weight, y, x_head_major):
+    """Shapes and dtypes of a dn_rms_norm_gated call."""
+    if z.dim() != 4:
+        raise ValueError("dn: z must be [B, T, H, D]")
+    B, T, H, D = z.shape
+    want_x = (B, H, T, D) if x_head_major else (B, T, H, D)
+    if tuple(x.shape) != want_x:
+        raise ValueError(f"dn: x must be {want_x}, got {tuple(x.shape)}")
+    if tuple(y.shape) != (B, T, H, D):
+        raise ValueError(f"dn: y must be [B, T, H, D] = {(B, T, H, D)}")
+    if tuple(weight.shape) != (D,):
+        raise ValueError(f"dn: weight must be [D] = ({D},)")
+    if x.dtype != z.dtype or y.dtype != z.dtype:
+        raise ValueError("dn: x, z and y must share one dtype")
+
+
 def dn_causal_conv1d(x, weight, y, state_in=None, state_out=None, *, head_dim: int | None = None,
                      activation: bool = True, stream=None) -> None:
     """Depthwise causal conv over time with carried history, through
@@ -258,6 +295,7 @@ def dn_causal_conv1d(x, weight, y, state_in=None, state_out=None, *, head_dim: i
     tensor: unit stride over channels, any row stride), weight [C, K] fp32,
     states [B, K-1, C] in x's dtype, y [B, C // head_dim, T, head_dim]
     (head_dim defaults to C: y is then [B, T, C] in effect)."""
+    _conv_check(x, weight, y, state_in, state_out, head_dim)
     lib = load_library()
     B, T, C = x.shape
     K = weight.shape[-1]
@@ -278,6 +316,7 @@ def dn_rms_norm_gated(x, z, weight, y, *, eps: float = 1e-6, x_head_major: bool 
     """Gated RMSNorm of each head's output row, through ``dn_rms_norm_gated``:
     x [B, H, T, D] (x_head_major) or [B, T, H, D]; z and y [B, T, H, D];
     weight [D] fp32; activation "silu" or "sigmoid"."""
+    _norm_check(x, z, weight, y, x_head_major)
     lib = load_library()
     B, T, H, D = z.shape
     _f32(weight)

@@ -286,3 +286,50 @@ def test_rms_norm_gated_rejects(lib, over, code):
 def test_rms_norm_gated_empty_is_ok(lib):
     assert norm_call(lib, T=0) == dn.DN_OK
     assert norm_call(lib, H=0, x=None, z=None, y=None) == dn.DN_OK
+
+
+def test_layer_op_bindings_check_shapes_before_any_device_call():
+    """The C ABI sees only pointers and sizes, so the binding checks that the tensors
+    agree: a mismatch raises before the library is called.  (CPU tensors that pass the
+    checks are then refused as not on a CUDA device.)"""
+    import torch
+    bf = torch.bfloat16
+    x = torch.zeros(2, 10, 64, dtype=bf)
+    w = torch.zeros(64, 4)
+    s = torch.zeros(2, 3, 64, dtype=bf)
+    y = torch.zeros(2, 2, 10, 32, dtype=bf)
+    bad = [
+        dict(w=torch.zeros(32, 4)),                      # channels disagree
+        dict(y=torch.zeros(2, 2, 10, 31, dtype=bf)),     # wrong output size
+        dict(y=torch.zeros(2, 10, 2, 32, dtype=bf)),     # token-major given for head-major
+        dict(s_in=torch.zeros(2, 2, 64, dtype=bf)),      # K - 1 rows
+        dict(s_out=torch.zeros(2, 3, 64)),               # dtype
+        dict(hd=24),                                     # does not divide C
+    ]
+    for over in bad:
+        a = dict(x=x, w=w, y=y, s_in=s, s_out=s, hd=32)
+        a.update(over)
+        with pytest.raises(ValueError, match=r"^dn: (?!tensors must be CUDA)"):
+            dn.dn_causal_conv1d(a["x"], a["w"], a["y"], a["s_in"], a["s_out"], head_dim=a["hd"])
+    with pytest.raises(ValueError, match="CUDA"):
+        dn.dn_causal_conv1d(x, w, y, s, s, head_dim=32)
+
+    o = torch.zeros(2, 4, 10, 128, dtype=bf)             # head-major [B, H, T, D]
+    z = torch.zeros(2, 10, 4, 128, dtype=bf)
+    yn = torch.zeros(2, 10, 4, 128, dtype=bf)
+    nw = torch.zeros(128)
+    bad = [
+        dict(x=z.clone()),                               # token-major given as head-major
+        dict(y=torch.zeros(2, 4, 10, 128, dtype=bf)),
+        dict(w=torch.zeros(64)),
+        dict(x=torch.zeros(2, 4, 10, 128)),              # dtype
+    ]
+    for over in bad:
+        a = dict(x=o, z=z, w=nw, y=yn)
+        a.update(over)
+        with pytest.raises(ValueError, match=r"^dn: (?!tensors must be CUDA)"):
+            dn.dn_rms_norm_gated(a["x"], a["z"], a["w"], a["y"])
+    with pytest.raises(ValueError, match="CUDA"):
+        dn.dn_rms_norm_gated(o, z, nw, yn)
+    with pytest.raises(ValueError, match="CUDA"):
+        dn.dn_rms_norm_gated(z, z, nw, yn, x_head_major=False)
