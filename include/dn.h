@@ -39,7 +39,8 @@
  *   - beta is not clamped (values in (0, 2) give the negative-eigenvalue
  *     transitions of D2L 12.5, "The reflection hiding in the delta rule").
  *     g is the log-decay (alpha = exp(g)); g <= 0 is expected but not
- *     enforced.  k is not normalised by the library.
+ *     enforced.  k is not normalised by the library, except by the *_gdn
+ *     entry points, which take raw q and k and normalise both.
  *   - Pointers to q, k, v, o, S0, S_T and S must be 16-byte aligned, as must a
  *     per-key g; beta and a scalar g 4-byte aligned.
  */
