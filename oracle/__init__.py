@@ -23,6 +23,7 @@ Contents
                           times a per-channel weight and SiLU (or sigmoid) of z.
 ``generalized_delta_rule`` RWKV-7's form: per-channel decay, removal key and
                           rate, and a separate write key.
+``chunked_generalized``   its chunkwise form (derived; checks the chunk algebra).
 ``varlen_delta_rule``     sequences packed along time (cu_seqlens), each with
                           its own initial and final state.
 ``gva_delta_rule``        grouped value heads: H_v / H_k value heads share each
@@ -474,3 +475,52 @@ def gva_delta_rule(q, k, v, beta, g=None, S0=None, scale=1.0):
         raise ValueError("the value heads must be a multiple of the key heads")
     r = Hv // Hk
     return delta_rule(np.repeat(q, r, axis=1), np.repeat(k, r, axis=1), v, beta, g, S0, scale=scale)
+
+
+def chunked_generalized(q, w, kappa, a, k_write, v, S0=None, scale=1.0, chunk=64):
+    """Chunkwise form of ``generalized_delta_rule`` in fp64, derived here from
+    the recurrence (the page gives only the recurrence): used only to check
+    the chunk algebra a chunked kernel would use against the token-by-token
+    rule.  Within a chunk, with l_s = a_s * kappa_s (left removal vector),
+    r_s = kappa_s (right), G_t = sum_{s<=t} log w_s per channel (chunk-local,
+    G_0 = 0) and U_s = r_s^T S_{s-1} (the removed content):
+
+        (I + M) U = R S_0 + N V,
+        M_sj = r_s^T e^(G_{s-1} - G_j) l_j,  N_sj = r_s^T e^(G_{s-1} - G_j) kw_j   (j < s),
+        R_s  = r_s^T e^(G_{s-1}),
+        S_C  = e^(G_C) S_0 + sum_s e^(G_C - G_s) (kw_s v_s^T - l_s U_s),
+        o_t  = scale (q_t^T e^(G_t) S_0 + sum_{s<=t} q_t^T e^(G_t - G_s) (kw_s v_s^T - l_s U_s)).
+
+    Explicit pairwise decays and a library triangular solve; w must be
+    positive.  Same arguments and result as ``generalized_delta_rule``."""
+    q, w, kappa, a, kw, v = (_f64(x) for x in (q, w, kappa, a, k_write, v))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    S = np.zeros((B, H, dk, dv)) if S0 is None else _f64(S0).copy()
+    o = np.zeros((B, H, T, dv))
+    for b in range(B):
+        for h in range(H):
+            St = S[b, h]
+            for c0 in range(0, T, chunk):
+                sl = slice(c0, min(c0 + chunk, T))
+                Q, L, Rv, Kw, V = q[b, h, sl], a[b, h, sl] * kappa[b, h, sl], kappa[b, h, sl], kw[b, h, sl], v[b, h, sl]
+                G = np.cumsum(np.log(w[b, h, sl]), axis=0)                 # G_1 .. G_C
+                n = G.shape[0]
+                Gp = np.vstack([np.zeros((1, dk)), G[:-1]])                # G_{s-1}
+                M = np.zeros((n, n)); N = np.zeros((n, n))
+                for s_ in range(n):
+                    for j in range(s_):
+                        dec = np.exp(Gp[s_] - G[j])
+                        M[s_, j] = np.sum(Rv[s_] * dec * L[j])
+                        N[s_, j] = np.sum(Rv[s_] * dec * Kw[j])
+                R = Rv * np.exp(Gp)
+                U = _solve_unit_lower(np.eye(n) + M, R @ St + N @ V)
+                W = Kw[:, :, None] * V[:, None, :] - L[:, :, None] * U[:, None, :]     # per s: kw v^T - l U
+                for t in range(n):
+                    dec = np.exp(G[t][None, :] - G[:t + 1])                  # e^(G_t - G_s), s <= t
+                    St_t = np.exp(G[t])[:, None] * St + np.einsum("sk,skv->kv", dec, W[:t + 1])
+                    o[b, h, c0 + t] = scale * St_t.T @ Q[t]
+                dec = np.exp(G[-1][None, :] - G)
+                St = np.exp(G[-1])[:, None] * St + np.einsum("sk,skv->kv", dec, W)
+            S[b, h] = St
+    return o, S

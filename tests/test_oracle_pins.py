@@ -707,3 +707,20 @@ def test_gva_one_to_one_is_the_plain_rule():
     assert np.array_equal(a, b)
     with pytest.raises(ValueError):
         oracle.gva_delta_rule(q[:, :2], k[:, :2], v, beta)
+
+
+@pytest.mark.parametrize("C", [1, 5, 16, 64])
+def test_chunked_generalized_equals_recurrence(C):
+    """The derived chunk algebra of the generalised rule equals the token-by-token rule
+    (T = 37, a ragged last chunk, S0 != 0, unrelated removal and write keys)."""
+    rng = np.random.default_rng(50 + C)
+    B, H, T, dk, dv = 1, 2, 37, 6, 5
+    q, kap, kw = (rng.standard_normal((B, H, T, dk)) for _ in range(3))
+    kap /= np.linalg.norm(kap, axis=-1, keepdims=True)
+    a = rng.random((B, H, T, dk)); w = np.exp(-0.3 * rng.random((B, H, T, dk)))
+    v = rng.standard_normal((B, H, T, dv)); S0 = rng.standard_normal((B, H, dk, dv))
+    o_ref, S_ref = oracle.generalized_delta_rule(q, w, kap, a, kw, v, S0, scale=0.6)
+    o, S = oracle.chunked_generalized(q, w, kap, a, kw, v, S0, scale=0.6, chunk=C)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-11 * np.abs(o_ref).max())
+    assert np.allclose(S, S_ref, rtol=0, atol=1e-11 * np.abs(S_ref).max())
+
