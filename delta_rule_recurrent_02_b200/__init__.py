@@ -13,8 +13,15 @@ Functions with the ABI's names take preallocated outputs:
     dn_chunk_fwd_workspace_size(B, T, H, d_k, d_v, chunk=64, dtype="bf16", gate="scalar", path="auto")
     dn_chunk_fwd_snapshots(q, k, v, beta, g, S0, o, S_T, snaps, every, ...)
     dn_chunk_fwd_gdn(q, k, v, b, a, A_log, dt_bias, S0, o, S_T, scale=1.0, ...)   # layer prologue fused in
+    dn_chunk_fwd_gdn_ex(..., chunk=64, path="auto", allow_neg_eigval=False, ...)  # either path; beta = 2 sigmoid(b)
+    dn_chunk_fwd_gva(q, k, v, beta, g, S0, o, S_T, scale=1.0, ...)   # H_k key heads, H value heads
+    dn_chunk_fwd_varlen(q, k, v, beta, g, S0, o, S_T, cu_seqlens, scale=1.0, ...)   # packed sequences
+    dn_chunk_fwd_varlen_workspace_size(N, T, H, d_k, d_v, dtype="bf16", gate="scalar")
+    dn_chunk_fwd_general(q, w_log, kappa, a, k, v, S0, o, S_T, chunk=32, scale=1.0)   # RWKV-7's rule
     dn_decode_step(q, k, v, beta, g, S, o, scale=1.0, ...)
+    dn_decode_step_gva(q, k, v, beta, g, S, o, scale=1.0, ...)
     dn_decode_step_gdn(q, k, v, b, a, A_log, dt_bias, S, o, scale=1.0, ...)
+    dn_decode_step_gdn_ex(..., allow_neg_eigval=False, ...)
     dn_causal_conv1d(x, weight, y, state_in=None, state_out=None, head_dim=None, activation=True)
     dn_rms_norm_gated(x, z, weight, y, eps=1e-6, x_head_major=True, activation="silu")
     dn_device_status(stream=None)
@@ -31,20 +38,24 @@ import ctypes
 import os
 
 __all__ = ["DNError", "load_library", "library_path", "dn_chunk_fwd", "dn_chunk_fwd_workspace_size",
-           "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
-           "dn_decode_step", "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated",
+           "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn", "dn_chunk_fwd_gva",
+           "dn_decode_step_gva", "dn_chunk_fwd_gdn_ex", "dn_decode_step_gdn_ex", "DN_GDN_BETA_2SIGMOID",
+           "dn_chunk_fwd_varlen", "dn_chunk_fwd_varlen_workspace_size", "dn_chunk_fwd_general", "dn_decode_step", "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated",
            "dn_device_status", "chunk_fwd", "decode_step", "ABI_SYMBOLS",
            "DN_OK", "DN_ERR_INVALID", "DN_ERR_UNSUPPORTED", "DN_ERR_CUDA", "DN_ERR_TIMEOUT"]
 
 DN_OK, DN_ERR_INVALID, DN_ERR_UNSUPPORTED, DN_ERR_CUDA, DN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+DN_GDN_BETA_2SIGMOID = 1
+DN_GDN_NORM_SIGMOID = 2
 _DTYPES = {"f32": 0, "bf16": 1}
 _GATES = {"none": 0, "scalar": 1, "per_key": 2}
 _PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_stall_test": 3}
 
 ABI_SYMBOLS = ("dn_chunk_fwd", "dn_chunk_fwd_ex", "dn_chunk_fwd_workspace_size", "dn_chunk_fwd_noalloc",
-               "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn",
-               "dn_decode_step", "dn_device_status", "dn_status_str", "dn_last_error", "dn_version",
-               "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated")
+               "dn_chunk_fwd_snapshots", "dn_chunk_fwd_gdn", "dn_decode_step_gdn", "dn_chunk_fwd_gva",
+               "dn_decode_step_gva", "dn_chunk_fwd_gdn_ex", "dn_decode_step_gdn_ex", "dn_chunk_fwd_varlen",
+               "dn_chunk_fwd_varlen_workspace_size", "dn_chunk_fwd_general", "dn_decode_step", "dn_device_status", "dn_status_str",
+               "dn_last_error", "dn_version", "dn_kernel_launches", "dn_causal_conv1d", "dn_rms_norm_gated")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -82,6 +93,21 @@ def load_library():
     lib.dn_chunk_fwd_gdn.restype = I
     lib.dn_decode_step_gdn.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, I, I, I, I, F, I, vp]
     lib.dn_decode_step_gdn.restype = I
+    lib.dn_chunk_fwd_gdn_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, I, vp,
+                                        fp, F, vp, Z, vp]
+    lib.dn_chunk_fwd_gdn_ex.restype = I
+    lib.dn_decode_step_gdn_ex.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp, fp, F, vp]
+    lib.dn_decode_step_gdn_ex.restype = I
+    lib.dn_chunk_fwd_gva.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, I, I, I, I, I, I, F, I, I, vp, Z, vp]
+    lib.dn_chunk_fwd_gva.restype = I
+    lib.dn_decode_step_gva.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, I, F, I, I, vp]
+    lib.dn_decode_step_gva.restype = I
+    lib.dn_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp, I, I, I, I, I, F, I, I, vp, Z, vp]
+    lib.dn_chunk_fwd_varlen.restype = I
+    lib.dn_chunk_fwd_varlen_workspace_size.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(Z)]
+    lib.dn_chunk_fwd_varlen_workspace_size.restype = I
+    lib.dn_chunk_fwd_general.argtypes = [vp, fp, vp, fp, vp, vp, fp, vp, fp, I, I, I, I, I, I, F, I, vp]
+    lib.dn_chunk_fwd_general.restype = I
     lib.dn_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I, ctypes.POINTER(Z)]
     lib.dn_chunk_fwd_workspace_size.restype = I
     lib.dn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, I, I, I, I, F, I, I, vp]
@@ -223,6 +249,52 @@ def dn_chunk_fwd_gdn(q, k, v, b, a, A_log, dt_bias, S0, o, S_T, *, scale: float 
     _check(lib, st)
 
 
+def dn_chunk_fwd_gdn_ex(q, k, v, b, a, A_log, dt_bias, S0, o, S_T, *, chunk: int = 64, scale: float = 1.0,
+                        path: str = "auto", allow_neg_eigval: bool = False, z=None, norm_weight=None,
+                        eps: float = 1e-6, norm_activation: str = "silu", workspace=None, stream=None) -> None:
+    """``dn_chunk_fwd_gdn`` on either kernel path (``dn_chunk_fwd_gdn_ex``): fp32 or
+    bf16 tokens, d in {64, 128}, chunk 1..64 on the CUDA-core path;
+    ``allow_neg_eigval`` takes beta = 2 sigmoid(b); with ``z`` [B, T, H, d_v] and
+    ``norm_weight`` [d_v], ``o`` [B, T, H, d_v] receives the gated RMSNorm of the
+    read-out (tensor-core path)."""
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    for t in (b, a, A_log, dt_bias, S0, S_T, norm_weight):
+        _f32(t)
+    if z is not None and (tuple(z.shape) != (B, T, H, dv) or z.dtype != q.dtype or tuple(o.shape) != (B, T, H, dv)):
+        raise ValueError("dn: z and o must be [B, T, H, d_v] in the token dtype")
+    flags = (DN_GDN_BETA_2SIGMOID if allow_neg_eigval else 0) | \
+        (DN_GDN_NORM_SIGMOID if z is not None and norm_activation == "sigmoid" else 0)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.dn_chunk_fwd_gdn_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias),
+                                 _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk), float(scale),
+                                 _dtype_code(q), _PATHS[path], flags, _ptr(z), _ptr(norm_weight), float(eps),
+                                 _ptr(workspace), ws_bytes, _stream(stream))
+    _check(lib, st)
+
+
+def dn_decode_step_gdn_ex(q, k, v, b, a, A_log, dt_bias, S, o, *, scale: float = 1.0,
+                          allow_neg_eigval: bool = False, z=None, norm_weight=None, eps: float = 1e-6,
+                          norm_activation: str = "silu", stream=None) -> None:
+    """``dn_decode_step_gdn`` with flags (``dn_decode_step_gdn_ex``):
+    ``allow_neg_eigval`` takes beta = 2 sigmoid(b); with ``z`` [B, H, d_v] and
+    ``norm_weight`` [d_v], ``o`` receives the gated RMSNorm of the read-out."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for t in (b, a, A_log, dt_bias, S, norm_weight):
+        _f32(t)
+    if z is not None and (tuple(z.shape) != (B, H, dv) or z.dtype != q.dtype):
+        raise ValueError("dn: z must be [B, H, d_v] in the token dtype")
+    flags = (DN_GDN_BETA_2SIGMOID if allow_neg_eigval else 0) | \
+        (DN_GDN_NORM_SIGMOID if z is not None and norm_activation == "sigmoid" else 0)
+    st = lib.dn_decode_step_gdn_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias),
+                                   _ptr(S), _ptr(o), B, H, dk, dv, float(scale), _dtype_code(q), flags, _ptr(z),
+                                   _ptr(norm_weight), float(eps), _stream(stream))
+    _check(lib, st)
+
+
 def dn_decode_step_gdn(q, k, v, b, a, A_log, dt_bias, S, o, *, scale: float = 1.0, stream=None) -> None:
     """One decode step with the Gated DeltaNet layer's prologue fused in, through
     ``dn_decode_step_gdn``: q and k [B, H, d] raw, b and a [B, H] raw, A_log and
@@ -234,6 +306,90 @@ def dn_decode_step_gdn(q, k, v, b, a, A_log, dt_bias, S, o, *, scale: float = 1.
         _f32(t)
     st = lib.dn_decode_step_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(b), _ptr(a), _ptr(A_log), _ptr(dt_bias), _ptr(S),
                                 _ptr(o), B, H, dk, dv, float(scale), _dtype_code(q), _stream(stream))
+    _check(lib, st)
+
+
+def dn_chunk_fwd_gva(q, k, v, beta, g, S0, o, S_T, *, scale: float = 1.0, gate: str | None = None,
+                     workspace=None, stream=None) -> None:
+    """Prefill with grouped value heads through ``dn_chunk_fwd_gva``: q and k
+    [B, H_k, T, d_k], v and o [B, H, T, d_v], beta and g [B, H, T], states
+    [B, H, d_k, d_v]; value head h reads key head h // (H // H_k)."""
+    lib = load_library()
+    B, Hk, T, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    if tuple(k.shape) != tuple(q.shape) or tuple(v.shape[:3]) != (B, H, T):
+        raise ValueError("dn: q, k must be [B, H_k, T, d_k] and v [B, H, T, d_v]")
+    for t in (beta, g, S0, S_T):
+        _f32(t)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.dn_chunk_fwd_gva(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T),
+                              B, T, Hk, H, dk, dv, float(scale), _dtype_code(q), _gate_code(gate, g, (B, H, T)),
+                              _ptr(workspace), ws_bytes, _stream(stream))
+    _check(lib, st)
+
+
+def dn_chunk_fwd_varlen_workspace_size(N: int, T: int, H: int, d_k: int, d_v: int, *, dtype: str = "bf16",
+                                       gate: str = "scalar") -> int:
+    """Bytes of workspace ``dn_chunk_fwd_varlen`` needs for N sequences of T tokens in all."""
+    lib = load_library()
+    out = ctypes.c_size_t(0)
+    _check(lib, lib.dn_chunk_fwd_varlen_workspace_size(N, T, H, d_k, d_v, _DTYPES[dtype], _GATES[gate],
+                                                       ctypes.byref(out)))
+    return out.value
+
+
+def dn_chunk_fwd_varlen(q, k, v, beta, g, S0, o, S_T, cu_seqlens, *, scale: float = 1.0, gate: str | None = None,
+                        workspace=None, stream=None) -> None:
+    """Prefill of N packed sequences through ``dn_chunk_fwd_varlen``: q, k, v, o
+    [1, H, T, d] (or [H, T, d]), beta and g [1, H, T] (or [H, T]), cu_seqlens a
+    CUDA int32 tensor [N + 1], states [N, H, d_k, d_v]."""
+    import torch
+    lib = load_library()
+    H, T, dk = q.shape[-3:]
+    dv = v.shape[-1]
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("dn: cu_seqlens must be int32")
+    N = cu_seqlens.numel() - 1
+    for t in (beta, g, S0, S_T):
+        _f32(t)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.dn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T),
+                                 _ptr(cu_seqlens), N, T, H, dk, dv, float(scale), _dtype_code(q),
+                                 _gate_code(gate, g, tuple(beta.shape)), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(lib, st)
+
+
+def dn_chunk_fwd_general(q, w_log, kappa, a, k, v, S0, o, S_T, *, chunk: int = 32, scale: float = 1.0,
+                         stream=None) -> None:
+    """The generalised delta rule of RWKV-7 through ``dn_chunk_fwd_general``:
+    q, kappa, k [B, H, T, d_k] and v [B, H, T, d_v] in the token dtype; w_log
+    (log of the per-channel decay) and a [B, H, T, d_k] fp32; states
+    [B, H, d_k, d_v] fp32."""
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    for t in (w_log, a, S0, S_T):
+        _f32(t)
+    st = lib.dn_chunk_fwd_general(_ptr(q), _ptr(w_log), _ptr(kappa), _ptr(a), _ptr(k), _ptr(v), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), B, T, H, dk, dv, int(chunk), float(scale), _dtype_code(q),
+                                  _stream(stream))
+    _check(lib, st)
+
+
+def dn_decode_step_gva(q, k, v, beta, g, S, o, *, scale: float = 1.0, gate: str | None = None,
+                       stream=None) -> None:
+    """One decode step with grouped value heads through ``dn_decode_step_gva``:
+    q and k [B, H_k, d_k], v and o [B, H, d_v], beta [B, H], S [B, H, d_k, d_v]."""
+    lib = load_library()
+    B, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
+    if tuple(k.shape) != tuple(q.shape) or tuple(v.shape[:2]) != (B, H):
+        raise ValueError("dn: q, k must be [B, H_k, d_k] and v [B, H, d_v]")
+    for t in (beta, g, S):
+        _f32(t)
+    st = lib.dn_decode_step_gva(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S), _ptr(o),
+                                B, Hk, H, dk, dv, float(scale), _dtype_code(q), _gate_code(gate, g, (B, H)),
+                                _stream(stream))
     _check(lib, st)
 
 

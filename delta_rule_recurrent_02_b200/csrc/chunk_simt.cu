@@ -56,13 +56,14 @@ struct SimtSmem {
 
 }  // namespace
 
-template <int DK, int GATE, typename Tin>
+template <int DK, int GATE, typename Tin, bool PRO = false>
 __global__ void __launch_bounds__(kNT)
 chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const float* __restrict__ beta,
                   const float* __restrict__ g, const float* S0,
                   Tin* __restrict__ o, float* S_T, int T, int DV, int chunk,
-                  float scale, float* snaps, int snap_every, int n_snap) {
+                  float scale, float* snaps, int snap_every, int n_snap,
+                  const float* A_log = nullptr, const float* dt_bias = nullptr, int H = 1, float bmul = 1.f) {
     using L = SimtSmem<DK, GATE>;
     constexpr int KS = L::KS;
     extern __shared__ float sm[];
@@ -151,10 +152,36 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
             }
         }
         if (tid < Cc) {
-            bs[tid] = pb;
-            if (GATE == kGateScalar) Gm[tid] = ps;
+            float bb = pb, aa = ps;
+            if (PRO) gdn_raw_gates(bb, aa, expf(A_log[bh % H]), dt_bias[bh % H], bmul);
+            bs[tid] = bb;
+            if (GATE == kGateScalar) Gm[tid] = aa;
         }
         __syncthreads();
+        if (PRO) {
+            // unit k and q rows, x / max(||x||, 1e-12), one warp per row (Qs holds scale q)
+            for (int i = warp; i < Cc; i += kNT / 32) {
+                float sk = 0.f, sq = 0.f;
+                for (int c = lane; c < DK; c += 32) {
+                    const float kv = Ks[i * KS + c], qv = Qs[i * KS + c];
+                    sk += kv * kv;
+                    sq += qv * qv;
+                }
+#pragma unroll
+                for (int o2 = 16; o2 > 0; o2 >>= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o2);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o2);
+                }
+                const float rk = 1.f / fmaxf(sqrtf(sk), 1e-12f);
+                const float as = fabsf(scale);
+                const float rq = as > 0.f ? 1.f / fmaxf(sqrtf(sq) / as, 1e-12f) : 0.f;
+                for (int c = lane; c < DK; c += 32) {
+                    Ks[i * KS + c] *= rk;
+                    Qs[i * KS + c] *= rq;
+                }
+            }
+            __syncthreads();
+        }
         if (c0 + chunk < T) prefetch(c0 + chunk);
         // ---- cumulative log-decay (inclusive) ---------------------------
         if (GATE == kGateScalar) {
@@ -319,17 +346,17 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     }
 }
 
-template <int DK, int GATE, typename Tin>
+template <int DK, int GATE, typename Tin, bool PRO = false>
 static cudaError_t launch_simt_t(const ChunkArgs& a, cudaStream_t st) {
     using L = SimtSmem<DK, GATE>;
-    auto kern = chunk_simt_kernel<DK, GATE, Tin>;
+    auto kern = chunk_simt_kernel<DK, GATE, Tin, PRO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (e != cudaSuccess) return e;
     const int64_t grid = a.B * a.H * (a.dv / kDVT);
     kern<<<(unsigned)grid, kNT, L::bytes, st>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         a.beta, a.g, a.S0, static_cast<Tin*>(a.o), a.S_T, (int)a.T, a.dv, a.chunk, a.scale, a.snaps, a.snap_every,
-        a.n_snap);
+        a.n_snap, a.A_log, a.dt_bias, (int)a.H, (float)a.prologue);
     return counted(cudaGetLastError());
 }
 
@@ -337,7 +364,9 @@ template <int DK, typename Tin>
 static cudaError_t launch_simt_gate(const ChunkArgs& a, cudaStream_t st) {
     switch (a.gate) {
         case kGateNone: return launch_simt_t<DK, kGateNone, Tin>(a, st);
-        case kGateScalar: return launch_simt_t<DK, kGateScalar, Tin>(a, st);
+        case kGateScalar:
+            return a.prologue ? launch_simt_t<DK, kGateScalar, Tin, true>(a, st)
+                              : launch_simt_t<DK, kGateScalar, Tin>(a, st);
         default: return launch_simt_t<DK, kGatePerKey, Tin>(a, st);
     }
 }

@@ -122,16 +122,103 @@ struct Args {
     const float* A_log;
     const float* dt_bias;
     int H;
+    int rep = 1;
+    // a packed batch of N sequences (null: B rows of T tokens): the chunk tables of
+    // varlen_table_kernel; `head` is then s H + h for sequence s and head h
+    const int* vl = nullptr;
+    int vl_N = 0;
+    // with the prologue: the layer's gated RMSNorm on the output rows (0 none, 1 SiLU(z),
+    // 2 sigmoid(z)); o then receives y = w * o / sqrt(mean(o^2) + eps) * act(z) token-major
+    // [B][T][H][d_v], the layout of z
+    int norm = 0;
+    const __nv_bfloat16* z = nullptr;
+    const float* norm_w = nullptr;
+    float eps = 0.f;
 };
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
 constexpr int G_KGAM = 0;
 
+// Output rows of chunk cp with the layer's gated RMSNorm, by the 128 output
+// threads (4 warps, thread j = value channel j = TMEM lane): per 8 positions,
+// each warp sums the squares of its 32 channels by a butterfly that leaves lane
+// l with position 4 bit4 + 2 bit3 + bit2 of l, the four warps' sums meet in the
+// gate slot's key-norm area (free in the state pass; two halves used in turn,
+// so one barrier per step suffices), and every thread forms
+// y = w_j o_ij / sqrt(mean_j o_ij^2 + eps) act(z_ij) for its channel, stored
+// token-major like z.  o_ij already carries 1 / ||q_i|| (the prologue).
+__device__ __forceinline__ void norm_rows(const Args& ar, uint32_t oc, float* gsp, int64_t bh, int cp, int Cc,
+                                          int j, int lane, int w4) {
+    const int64_t b = bh / ar.H, h = bh % ar.H;
+    const int64_t row0 = (b * ar.T + (int64_t)cp * kC) * ar.H + h;   // token-major row of position 0
+    const int64_t rstride = (int64_t)ar.H * kD;
+    const float wj = ar.norm_w[j];
+    const bool silu = ar.norm == 1;
+#pragma unroll 1
+    for (int it = 0; it < 8; ++it) {
+        float* red = gsp + G_RK + (it & 1) * 32;      // [8 positions][4 warps]
+        float zf[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = 8 * it + e;
+            zf[e] = i < Cc ? __bfloat162float(ar.z[row0 * kD + (int64_t)i * rstride + j]) : 0.f;
+        }
+        float v[8];
+        {
+            uint32_t u[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                           "=r"(u[7])
+                         : "r"(oc + 8 * it));
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(u[e]) * gsp[G_RQ + 8 * it + e];
+        }
+        float s4[4], s2[2], s1;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool hi = lane & 16;
+            const float keep = hi ? v[e + 4] * v[e + 4] : v[e] * v[e];
+            const float send = hi ? v[e] * v[e] : v[e + 4] * v[e + 4];
+            s4[e] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const bool hi = lane & 8;
+            const float keep = hi ? s4[e + 2] : s4[e];
+            const float send = hi ? s4[e] : s4[e + 2];
+            s2[e] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+        {
+            const bool hi = lane & 4;
+            const float keep = hi ? s2[1] : s2[0];
+            const float send = hi ? s2[0] : s2[1];
+            s1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        }
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        const int p = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+        if ((lane & 3) == 0) red[p * 4 + w4] = s1;
+        named_bar_sync(1, kSideThreads);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = 8 * it + e;
+            const float4 r4 = *reinterpret_cast<const float4*>(red + 4 * e);
+            const float ms = ((r4.x + r4.y) + (r4.z + r4.w)) * (1.f / (float)kD);
+            const float rs = 1.f / sqrtf(ms + ar.eps);
+            const float zz = zf[e];
+            const float gte = silu ? zz / (1.f + __expf(-zz)) : 1.f / (1.f + __expf(-zz));
+            if (i < Cc) ar.o[row0 * kD + (int64_t)i * rstride + j] = __float2bfloat16_rn(v[e] * rs * wj * gte);
+        }
+    }
+}
+
 // The state pass of head `head`, run by threads 0 .. kNT - 1 of a CTA whose
 // shared memory starts (1024-aligned) at sm.  HOSTED: the caller allocated the
 // TMEM (base tmem_given) and shares the SM with a WY group.
-// PRO: the layer's prologue (raw gates, unit q and k) is compiled in (scalar gate).
-template <int GATE, bool HOSTED, bool PRO = false>
+// PRO: the layer's prologue (raw gates, unit q and k) is compiled in (scalar gate),
+// 1 alone, 2 with the gated RMSNorm on the output rows.
+template <int GATE, bool HOSTED, int PRO = 0>
 __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head, uint32_t tmem_given) {
     using L = Layout<HOSTED>;
     constexpr int kStages = L::kStages;
@@ -160,7 +247,27 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t bh = head;
-    const int n = (T + kC - 1) / kC;
+    // the chain: its first row of q / k / v / o, its tokens, its tiles (tile0 + c tstep)
+    // and its key rows
+    int64_t row_base = bh * T, krow_base = key_head(bh, ar.H, ar.rep) * T, tile0;
+    int len = T, tstep = 1;
+    if (ar.vl) {
+        const VarlenTables vt{ar.vl, ar.vl_N};
+        const int s = (int)(head / ar.H), h = (int)(head % ar.H);
+        const int beg = vt.cu()[s];
+        len = vt.cu()[s + 1] - beg;
+        row_base = krow_base = (int64_t)h * T + beg;
+        tile0 = (int64_t)vt.coff()[s] * ar.H + h;
+        tstep = ar.H;
+    }
+    const int n = (len + kC - 1) / kC;
+    if (!ar.vl) tile0 = bh * n;
+    if (n == 0) {
+        // an empty sequence of a packed batch: its final state is its initial one
+        if (S_T)
+            for (int x = tid; x < kD * kD; x += kNT) S_T[bh * kD * kD + x] = S0 ? S0[bh * kD * kD + x] : 0.f;
+        return;
+    }
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i)
@@ -193,8 +300,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
         const float eA = PRO ? expf(ar.A_log[bh % ar.H]) : 0.f;
         const float dtb = PRO ? ar.dt_bias[bh % ar.H] : 0.f;
         auto fetch = [&](int cc) {
-            const int64_t t0 = bh * T + (int64_t)cc * kC;
-            const int Cn = min(kC, T - cc * kC);
+            const int64_t t0 = row_base + (int64_t)cc * kC;
+            const int Cn = min(kC, len - cc * kC);
             nb0 = lane < Cn ? beta[t0 + lane] : 0.f;
             nb1 = lane + 32 < Cn ? beta[t0 + lane + 32] : 0.f;
             if (GATE == kGateScalar) {
@@ -211,9 +318,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 if (PRO) {
                     // beta and g from the raw inputs, as the WY side computes them (here, one
                     // chunk after the loads were issued, so their latency stays hidden)
-                    const int Cn = min(kC, T - cc * kC);
-                    if (lane < Cn) gdn_raw_gates(b0, a0, eA, dtb);
-                    if (lane + 32 < Cn) gdn_raw_gates(b1, a1, eA, dtb);
+                    const int Cn = min(kC, len - cc * kC);
+                    if (lane < Cn) gdn_raw_gates(b0, a0, eA, dtb, (float)ar.prologue);
+                    if (lane + 32 < Cn) gdn_raw_gates(b1, a1, eA, dtb, (float)ar.prologue);
                 }
                 chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
                 __syncwarp();
@@ -226,23 +333,23 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             }
             if (!(test_flags & 1) && flags) {
                 // this chunk's workspace tiles are written (by another CTA, possibly right now)
-                bool ok = lane == 0 ? wait_flag(flags + bh * n + cc, abort_flag) : true;
+                bool ok = lane == 0 ? wait_flag(flags + tile0 + (int64_t)cc * tstep, abort_flag) : true;
                 if (!__shfl_sync(0xffffffffu, (int)ok, 0)) break;
             }
             if (KDA) {
                 // the chunk's decays per key channel, from the workspace, into slot cc % 4:
                 // its previous reader (chunk cc - 4) is done once chunk cc - 3's products are
                 const float4 gv = test_flags & 1 ? make_float4(1.f, 1.f, 1.f, 1.f)
-                                                 : reinterpret_cast<const float4*>(ar.gam + (bh * n + cc) * kD)[lane];
+                                                 : reinterpret_cast<const float4*>(ar.gam + (tile0 + (int64_t)cc * tstep) * kD)[lane];
                 reinterpret_cast<float4*>(gates + (cc & 3) * GATE_FLOATS + G_KGAM)[lane] = gv;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ctl.bar(B_GATE0 + (cc & 3)));
             }
             if (lane == 0 && !(test_flags & 1)) {
                 fence_async_global();
-                const int64_t tile = bh * n + cc;
+                const int64_t tile = tile0 + (int64_t)cc * tstep;
                 // q and k rows of the chunk; with the per-key gate, Qh and K~ rows of the tile
-                const int y = KDA ? (int)(tile * kC) : (int)(bh * T + (int64_t)cc * kC);
+                const int y = KDA ? (int)(tile * kC) : (int)(krow_base + (int64_t)cc * kC);
                 const uint32_t st = sb + s * SZ_STAGE;
                 const uint32_t fb = ctl.bar(B_FULL0 + s);
                 mbar_arrive_expect_tx(fb, STAGE_TX);
@@ -336,61 +443,70 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             if (c < n) {
                 // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
                 const int s = c % kStages;
-                const int Cc = min(kC, T - c * kC);
+                const int Cc = min(kC, len - c * kC);
                 float* gs = gates + (c & 3) * GATE_FLOATS;
                 const uint32_t st = sb + s * SZ_STAGE;
                 bool ok = ctl.wait(B_GATE0 + (c & 3), (uint32_t)(c >> 2) & 1u) &&
                           ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
-                if (PRO) {
-                    // 1 / ||q_i|| and 1 / ||k_i|| of the chunk from the stage's tiles, two
-                    // threads per row (read by the U epilogue after this chunk's READY)
-                    const int r = sid >> 1;
-                    const float rq = inv_row_norm(st + ST_B, r, sid & 1, 16384);
-                    const float rk = inv_row_norm(st + ST_K, r, sid & 1, 8192);
-                    if ((sid & 1) == 0) {
-                        gs[G_RQ + r] = rq;
-                        gs[G_RK + r] = rk;
-                    }
-                    named_bar_sync(1, kSideThreads);
-                }
+                float ssq[4] = {0.f, 0.f, 0.f, 0.f};
                 // (with the per-key gate the workspace holds Qh already)
 #pragma unroll
                 for (int u = 0; u < (GATE == kGatePerKey ? 0 : 8); ++u) {
                     const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
                     const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
                     const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
-                    const float f = i < Cc ? (PRO ? scale * gs[G_EG + i] * gs[G_RQ + i] : scale * gs[G_EG + i]) : 0.f;
+                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
                     const uint4 w = ld_shared_v4(a);
                     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
                     const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
                     const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+                    if (PRO)
+                        ssq[u & 3] += e0.x * e0.x + e0.y * e0.y + e1.x * e1.x + e1.y * e1.y +
+                                      e2.x * e2.x + e2.y * e2.y + e3.x * e3.x + e3.y * e3.y;
                     st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
                                  pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                 }
                 fence_async_smem();
                 mbar_arrive(ctl.bar(B_READY0 + s));
+                if (PRO) {
+                    // 1 / ||q_i|| of rows (sid / 8) + 16 u4 from the raw values just read, for the
+                    // output rows: 8 threads share a row (one 16-byte chunk of each d-block each)
+#pragma unroll
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        float s2 = ssq[u4];
+                        s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+                        s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+                        s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
+                        if ((sid & 7) == 0) gs[G_RQ + (sid >> 3) + 16 * u4] = 1.f / fmaxf(sqrtf(s2), 1e-12f);
+                    }
+                }
             }
             if (c >= 1) {
                 // ---- output rows of chunk c - 1 --------------------------------------------
                 const int cp = c - 1;
-                const int Cc = min(kC, T - cp * kC);
+                const int Cc = min(kC, len - cp * kC);
                 bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
                 tc_fence_after();
-                __nv_bfloat16* ob = o + (bh * T + (int64_t)cp * kC) * kD + j;
+                __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
                 const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
+                const float* gsp = gates + (cp & 3) * GATE_FLOATS;   // 1 / ||q_i|| with the prologue
+                if (PRO == 2) {
+                    norm_rows(ar, oc, gates + (cp & 3) * GATE_FLOATS, bh, cp, Cc, j, lane, warp - kSideWarp0);
+                } else {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float v[32];
-                    tmem_ld32(oc + hh * 32, v);
-                    tmem_wait_ld();
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float v[32];
+                        tmem_ld32(oc + hh * 32, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = hh * 32 + e;
-                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = hh * 32 + e;
+                            if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * gsp[G_RQ + i] : v[e]);
+                        }
                     }
                 }
                 tc_fence_before();
@@ -433,8 +549,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             const uint32_t st = sb + (c % kStages) * SZ_STAGE;
             // ---- U = u - W S -> bf16 pairs in TMEM, plain and decayed (U~), in two passes
             //      over positions 0-31 and 32-63 ------------------------------------------
-            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u) &&
-                 (!PRO || ctl.wait(B_READY0 + c % kStages, (uint32_t)(c / kStages) & 1u));
+            ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
             if (!ok) *abort_flag = 1;
             if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
             tc_fence_after();
@@ -466,11 +581,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
-                        if (PRO) {
-                            // times 1 / ||k_i||: K^T diag(1 / ||k||) U~ is K~^T U~ with unit keys
-                            const float4 rk = *reinterpret_cast<const float4*>(gsc + G_RK + i0 + 4 * q4);
-                            et.x *= rk.x; et.y *= rk.y; et.z *= rk.z; et.w *= rk.w;
-                        }
                         pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
                         pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
                     }

@@ -27,7 +27,7 @@ namespace dn {
 using namespace sm100;
 using namespace tc;
 
-template <int GATE, bool PRO>
+template <int GATE, int PRO>
 __global__ void __launch_bounds__(state::kNT, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
@@ -35,14 +35,72 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const float* __restrict__ beta, const float* __restrict__ g, const float* S0,
                    __nv_bfloat16* __restrict__ o, float* S_T, int T, float scale, unsigned int* status,
                    int test_flags, const float* __restrict__ gam, float* snaps, int snap_every, int n_snap,
-                   Prologue pro) {
+                   Prologue pro, const int* vl, int vl_N) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the __shared__ array itself so that
     // every access below compiles to a shared-memory (not generic) instruction
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
-                         gam, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H};
+                         gam, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, vl, vl_N,
+                         pro.norm, pro.z, pro.norm_w, pro.eps};
     state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
+}
+
+// The chunk tables of a packed batch (VarlenTables) from cu_seqlens [N + 1], by
+// one CTA: a checked copy of the offsets, each sequence's first global chunk
+// (an exclusive prefix sum of ceil(len / 64)) and each global chunk's sequence.
+// If cu_seqlens does not rise from 0 to T (non-decreasing), every length is
+// taken as zero (nothing runs, every S_T = S0) and bit 1 of the status word is
+// set, which dn_device_status reports as DN_ERR_INVALID.
+__global__ void __launch_bounds__(1024)
+varlen_table_kernel(const int* __restrict__ cu_in, int N, int T, int* tables, unsigned int* status) {
+    __shared__ int s_carry, s_bad;
+    __shared__ int s_warp[32];
+    const VarlenTables vt{tables, N};
+    int* cu = tables;
+    int* coff = tables + N + 1;
+    int* seq_of = tables + 2 * (N + 1);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) { s_carry = 0; s_bad = (cu_in[0] != 0 || cu_in[N] != T) ? 1 : 0; }
+    __syncthreads();
+    for (int s = tid; s < N; s += blockDim.x)
+        if (cu_in[s + 1] < cu_in[s]) s_bad = 1;
+    __syncthreads();
+    const bool bad = s_bad != 0;
+    for (int s = tid; s <= N; s += blockDim.x) cu[s] = bad ? 0 : cu_in[s];
+    if (bad && tid == 0) atomicOr(status, 2u);
+    // coff = exclusive prefix sum of the chunk counts, 1024 sequences per round
+    for (int s0 = 0; s0 <= N; s0 += blockDim.x) {
+        const int s = s0 + tid;
+        const int nch = (s < N && !bad) ? (cu_in[s + 1] - cu_in[s] + kC - 1) / kC : 0;
+        int x = nch;                                          // inclusive scan in the warp
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o2);
+            if (lane >= o2) x += y;
+        }
+        if (lane == 31) s_warp[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = s_warp[lane];
+#pragma unroll
+            for (int o2 = 1; o2 < 32; o2 <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o2);
+                if (lane >= o2) w += y;
+            }
+            s_warp[lane] = w;                                 // inclusive over warps
+        }
+        __syncthreads();
+        const int before = s_carry + (warp > 0 ? s_warp[warp - 1] : 0) + x - nch;
+        if (s <= N) coff[s] = before;
+        __syncthreads();
+        if (tid == blockDim.x - 1) s_carry = before + nch;
+        __syncthreads();
+    }
+    // seq_of: each sequence's chunks
+    for (int s = warp; s < N; s += blockDim.x / 32)
+        for (int c = coff[s] + lane; c < coff[s + 1]; c += 32) seq_of[c] = s;
+    (void)vt;
 }
 
 namespace {
@@ -58,7 +116,7 @@ static_assert(state::Layout<true>::kCols + wy::TM_COLS <= state::TM_COLS, "hoste
 constexpr uint32_t kHostBar = 6;                    // named barrier of the hosting CTA's state pass + WY group
 }  // namespace
 
-template <int GATE, bool HOSTED, bool PRO>
+template <int GATE, bool HOSTED, int PRO>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
@@ -75,10 +133,11 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // the later ones come from tickets, in order (chunk-major), to whichever group is free
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
-                      flags + tiles, BH, (int)G, pro.on, pro.A_log, pro.dt_bias, pro.H};
+                      flags + tiles, BH, (int)G, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep};
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H};
+                             test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H,
+                             pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps};
         if (!HOSTED) {
             // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
             if (warp >= state::kNT / 32) return;
@@ -110,7 +169,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int64_t pending = -1;
             for (int64_t t = (int64_t)(gridDim.x - BH) * 4 + blockIdx.x; ok && t < tiles;) {
                 const int c = (int)(t / BH);
-                ok = wy::wy_tile<GATE, PRO>(x, wa, c, t - (int64_t)c * BH, pending);
+                ok = wy::wy_tile<GATE, (PRO != 0)>(x, wa, c, t - (int64_t)c * BH, pending);
                 if (ok) t = G + (int64_t)wy::next_ticket(x);
             }
             if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
@@ -144,7 +203,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     int64_t pending = -1;
     for (int64_t t = (int64_t)(blockIdx.x - BH) * 4 + grp; ok && t < tiles;) {
         const int c = (int)(t / BH);
-        ok = wy::wy_tile<GATE, PRO>(x, wa, c, t - (int64_t)c * BH, pending);
+        ok = wy::wy_tile<GATE, (PRO != 0)>(x, wa, c, t - (int64_t)c * BH, pending);
         if (ok) t = G + (int64_t)wy::next_ticket(x);
     }
     if (ok && x.tid == wy::kStoreTid) wy::publish_pending(wa, pending);
@@ -182,7 +241,7 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_kt, &tm_qh, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags, gam, snaps, snap_every, n_snap, 0, nullptr, nullptr, 1};
-        state::state_pass<kGatePerKey, false>(sm, ar, blockIdx.x, 0u);
+        state::state_pass<kGatePerKey, false, 0>(sm, ar, blockIdx.x, 0u);
         return;
     }
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -231,21 +290,43 @@ bool fused_fits(int64_t BH, int num_sms) {
     return BH + 16 <= num_sms && BH * 4 <= (int64_t)num_sms * 3;
 }
 
-template <int GATE, bool PRO>
+template <int GATE, int PRO>
 cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     const uint64_t rows = (uint64_t)(a.B * a.H * a.T);
+    const uint64_t krows = rows / (uint64_t)a.rep;          // q and k: H / rep heads
     const int n = (int)((a.T + kC - 1) / kC);
-    const uint64_t tiles = (uint64_t)(a.B * a.H) * (uint64_t)n;
+    const bool packed = a.cu_seqlens != nullptr;
+    // a packed batch: tiles of H heads x the most chunks its tokens can make
+    const uint64_t tiles = (uint64_t)(a.B * a.H) * (uint64_t)(packed ? vl_chunks_max(a.T, a.N) : n);
     uint8_t* w_ws = static_cast<uint8_t*>(a.ws);
     uint8_t* u_ws = w_ws + tiles * kWsWBytes;
     uint8_t* p_ws = u_ws + tiles * kWsUBytes;
     TcMaps m;
-    if (!make_tmap(&m.q, a.q, kD, rows, 64) || !make_tmap(&m.k, a.k, kD, rows, 64) ||
+    if (!make_tmap(&m.q, a.q, kD, krows, 64) || !make_tmap(&m.k, a.k, kD, krows, 64) ||
         !make_tmap(&m.v, a.v, kD, rows, 64) || !make_tmap(&m.w, w_ws, kD, tiles * kC, 64) ||
         !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64))
         return cudaErrorInvalidValue;
     m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles));
+    if (packed) {
+        // the chunk tables, then all WY tiles, then one state pass per (sequence, head)
+        int* vl = reinterpret_cast<int*>(w_ws + ws_total_bytes(tiles));
+        m.vl = vl;
+        varlen_table_kernel<<<1, 1024, 0, st>>>(a.cu_seqlens, a.N, (int)a.T, vl, a.status);
+        cudaError_t e = counted(cudaGetLastError());
+        if (e != cudaSuccess) return e;
+        e = launch_chunk_wy(a, m, st);
+        if (e != cudaSuccess) return e;
+        auto kern = chunk_state_kernel<GATE, PRO>;
+        const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)(a.N * a.H), state::kNT, bytes, st>>>(
+            m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0, static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
+            a.scale, a.status, a.test_flags, nullptr, nullptr, 1, 0,
+            prologue_of(a), vl, a.N);
+        return counted(cudaGetLastError());
+    }
 
     int dev = 0, num_sms = 0, coop = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -276,7 +357,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             unsigned int* status = a.status;
             float* snaps = a.snaps;
             int snap_every = a.snap_every, n_snap = a.n_snap;
-            Prologue pro{a.prologue ? 1 : 0, a.A_log, a.dt_bias, (int)a.H};
+            Prologue pro = prologue_of(a);
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
                             &T_i, &n_i, &scale, &status, &test_flags, &snaps, &snap_every, &n_snap, &pro};
             // the flags are cleared on the same stream right before the launch
@@ -296,7 +377,8 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     kern<<<(unsigned)BH, state::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
                                                   a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap,
-                                                  Prologue{a.prologue ? 1 : 0, a.A_log, a.dt_bias, (int)a.H});
+                                                  prologue_of(a),
+                                                  nullptr, 0);
     return counted(cudaGetLastError());
 }
 
@@ -366,26 +448,31 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     }
     e = launch_chunk_wy_kda(a, m, st);
     if (e != cudaSuccess) return e;
-    auto kern = chunk_state_kernel<kGatePerKey, false>;
+    auto kern = chunk_state_kernel<kGatePerKey, 0>;
     const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(a.B * a.H), state::kNT, bytes, st>>>(m.kt, m.qh, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
                                                           a.scale, a.status, a.test_flags, m.gam_ws, a.snaps,
-                                                          a.snap_every, a.n_snap, Prologue{0, nullptr, nullptr, 1});
+                                                          a.snap_every, a.n_snap, Prologue{0, nullptr, nullptr, 1}, nullptr, 0);
     return counted(cudaGetLastError());
 }
 
 }  // namespace
 
 bool tc_supports(const ChunkArgs& a) {
-    const int64_t n = (a.T + kC - 1) / kC;
+    const int64_t n = a.cu_seqlens ? vl_chunks_max(a.T, a.N) : (a.T + kC - 1) / kC;
     return a.bf16 && a.chunk == kC && a.dk == kD && a.dv == kD &&
            a.B * a.H * a.T < (int64_t(1) << 31) && a.B * a.H * n * kD < (int64_t(1) << 31);
 }
 
 size_t tc_workspace_bytes(const ChunkArgs& a) {
+    if (a.cu_seqlens) {
+        // a packed batch: tiles for the most chunks its tokens can make, then its chunk tables
+        const int64_t nc = vl_chunks_max(a.T, a.N);
+        return ws_total_bytes((uint64_t)(a.H * nc)) + ((vl_table_ints(a.N, nc) * 4 + 255) / 256) * 256;
+    }
     const int64_t n = (a.T + kC - 1) / kC;
     return ws_total_bytes((uint64_t)(a.B * a.H * n), a.gate == kGatePerKey);
 }
@@ -393,8 +480,9 @@ size_t tc_workspace_bytes(const ChunkArgs& a) {
 cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
     if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
     if (a.gate == kGatePerKey) return launch_tc_kda(a, st);
-    if (a.prologue) return launch_tc_gate<kGateScalar, true>(a, st);   // the layer prologue: scalar gate
-    return a.gate == kGateScalar ? launch_tc_gate<kGateScalar, false>(a, st) : launch_tc_gate<kGateNone, false>(a, st);
+    // the layer prologue (scalar gate), with or without the gated RMSNorm on the output rows
+    if (a.prologue) return a.norm ? launch_tc_gate<kGateScalar, 2>(a, st) : launch_tc_gate<kGateScalar, 1>(a, st);
+    return a.gate == kGateScalar ? launch_tc_gate<kGateScalar, 0>(a, st) : launch_tc_gate<kGateNone, 0>(a, st);
 }
 
 }  // namespace dn

@@ -65,17 +65,58 @@ struct TcMaps {
     __nv_bfloat16* kt_ws;
     __nv_bfloat16* qh_ws;
     float* gam_ws;
+    // a packed batch only: the workspace's chunk tables (VarlenTables), else null
+    const int* vl = nullptr;
 };
 
 // The Gated DeltaNet layer's prologue, fused into the prefill kernels (scalar
 // gate): when `on`, the beta and g arrays hold the raw inputs b and a, and q
 // and k are normalised per row inside the kernels.
 struct Prologue {
-    int on;
+    int on;                  // 0: off; else beta = on * sigmoid(b) (1, or 2 for the gate in (0, 2))
     const float* A_log;      // [H]
     const float* dt_bias;    // [H]
     int H;                   // heads per batch row (head of bh: bh % H)
+    int rep = 1;             // value heads per key head (q and k have H / rep heads)
+    // the gated RMSNorm on the output rows (0 none, 1 SiLU(z), 2 sigmoid(z)): z and the
+    // output token-major [B][T][H][d_v]
+    int norm = 0;
+    const __nv_bfloat16* z = nullptr;
+    const float* norm_w = nullptr;
+    float eps = 0.f;
 };
+
+// Chunk tables of a packed batch of N sequences, built on the device from
+// cu_seqlens before the prefill kernels run (varlen_table_kernel), as ints:
+//   cu      [N + 1]   the sequences' token offsets (a checked copy: all zero if
+//                     cu_seqlens was not non-decreasing from 0 to the total)
+//   coff    [N + 1]   the first global chunk of each sequence; coff[N] = chunks in all
+//   seq_of  [nc_max]  the sequence of each global chunk
+struct VarlenTables {
+    const int* base;
+    int N;
+    __host__ __device__ const int* cu() const { return base; }
+    __host__ __device__ const int* coff() const { return base + N + 1; }
+    __host__ __device__ const int* seq_of() const { return base + 2 * (N + 1); }
+};
+// Global chunks of a packed batch of T tokens in N sequences: at most T / 64 + N.
+inline int64_t vl_chunks_max(int64_t T, int N) { return T / kC + N; }
+inline size_t vl_table_ints(int N, int64_t nc_max) { return 2 * (size_t)(N + 1) + (size_t)nc_max; }
+
+// The Prologue argument of the tensor-core kernels for a request.
+inline Prologue prologue_of(const ChunkArgs& a) {
+    Prologue p{a.prologue, a.A_log, a.dt_bias, (int)a.H, a.rep};
+    p.norm = a.norm;
+    p.z = static_cast<const __nv_bfloat16*>(a.z);
+    p.norm_w = a.norm_weight;
+    p.eps = a.eps;
+    return p;
+}
+
+// Row block of q and k for value head bh (b * H + h): key head h / rep of batch row b.
+__host__ __device__ __forceinline__ int64_t key_head(int64_t bh, int H, int rep) {
+    return rep == 1 ? bh : (bh / H) * (H / rep) + (bh % H) / rep;
+}
 
 // Gate slot of one chunk (floats).  G_RQ / G_RK: 1 / ||q_i|| and 1 / ||k_i||
 // when the layer's prologue normalises q and k inside the kernels, else 1.

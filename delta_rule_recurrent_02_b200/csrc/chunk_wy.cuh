@@ -182,6 +182,12 @@ struct Args {
     const float* A_log;
     const float* dt_bias;
     int H;
+    int rep = 1;
+    // a packed batch of sequences (null: B independent rows of T tokens): the chunk
+    // tables of varlen_tables(), with N sequences; c is then the batch's global chunk
+    // index and bh the head
+    const int* vl = nullptr;
+    int vl_N = 0;
 };
 
 // Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
@@ -192,11 +198,13 @@ __device__ __forceinline__ void prefetch_next(const Args& ar, unsigned int ticke
     const int64_t tn = (int64_t)ar.G + ticket;
     if (tn >= (int64_t)ar.BH * ar.n) return;
     const int cn = (int)(tn / ar.BH);
-    const int64_t y = (tn - (int64_t)cn * ar.BH) * ar.T + (int64_t)cn * kC;
-    tma_prefetch_2d(ar.tm_k, 0, (int)y);
-    tma_prefetch_2d(ar.tm_k, 64, (int)y);
-    tma_prefetch_2d(ar.tm_q, 0, (int)y);
-    tma_prefetch_2d(ar.tm_q, 64, (int)y);
+    const int64_t bhn = tn - (int64_t)cn * ar.BH;
+    const int64_t y = bhn * ar.T + (int64_t)cn * kC;
+    const int64_t yk = key_head(bhn, ar.H, ar.rep) * ar.T + (int64_t)cn * kC;
+    tma_prefetch_2d(ar.tm_k, 0, (int)yk);
+    tma_prefetch_2d(ar.tm_k, 64, (int)yk);
+    tma_prefetch_2d(ar.tm_q, 0, (int)yk);
+    tma_prefetch_2d(ar.tm_q, 64, (int)yk);
     tma_prefetch_2d(ar.tm_v, 0, (int)y);
     tma_prefetch_2d(ar.tm_v, 64, (int)y);
     if (ar.T - cn * kC >= kC) {
@@ -295,7 +303,8 @@ __device__ __forceinline__ void publish_pending(const Args& ar, int64_t& pending
     pending = -1;
 }
 
-// Chunk c of head bh.  `pending` (thread kStoreTid's copy counts) is the
+// Chunk c of head bh (of a packed batch: global chunk c of head bh, see
+// Args::vl).  `pending` (thread kStoreTid's copy counts) is the
 // group's tile whose flag is still to be raised, or -1; on return it is this
 // tile.  With a tile counter, thread kStoreTid also takes the group's next
 // ticket, prefetches that tile's inputs into L2, and hands the ticket on
@@ -322,9 +331,24 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     const CUtensorMap& tm_v = *ar.tm_v;
     const CUtensorMap& tm_w = *ar.tm_w;
     const CUtensorMap& tm_u = *ar.tm_u;
-    const int64_t tile = bh * n + c;
-    const int Cc = min(kC, T - c * kC);
-    const int64_t t0 = bh * T + (int64_t)c * kC;
+    int64_t tile, t0, t0k;
+    int Cc;
+    if (ar.vl) {
+        // chunk cs of sequence s: rows cu[s] + 64 cs .. of head bh in the packed [H][T][d] arrays
+        const VarlenTables vt{ar.vl, ar.vl_N};
+        const int s = vt.seq_of()[c];
+        const int cs = c - vt.coff()[s];
+        const int beg = vt.cu()[s], len = vt.cu()[s + 1] - beg;
+        tile = (int64_t)c * ar.H + bh;
+        Cc = min(kC, len - cs * kC);
+        t0 = bh * T + beg + (int64_t)cs * kC;
+        t0k = t0;
+    } else {
+        tile = bh * n + c;
+        Cc = min(kC, T - c * kC);
+        t0 = bh * T + (int64_t)c * kC;
+        t0k = key_head(bh, ar.H, ar.rep) * T + (int64_t)c * kC;   // q and k rows
+    }
     const bool load = !(ar.test_flags & 1);
     int loads = 0;                                   // load groups issued (thread 0)
     // the next ticket, taken now (by the thread that prefetches for it and hands it on)
@@ -333,7 +357,7 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
 
     if (tid == 0 && load) {
         const uint32_t fb = ctl.bar(B_FULL);
-        const int y = (int)t0;
+        const int y = (int)t0k;
         mbar_arrive_expect_tx(fb, 4 * 8192);
         tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, y, fb);
         tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, y, fb);
@@ -353,8 +377,9 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             // beta and g from the raw inputs (positions past the end stay identity steps)
             const int h = (int)(bh % ar.H);
             const float eA = expf(ar.A_log[h]), dtb = ar.dt_bias[h];
-            if (lane < Cc) gdn_raw_gates(b0, a0, eA, dtb);
-            if (lane + 32 < Cc) gdn_raw_gates(b1, a1, eA, dtb);
+            const float bm = (float)ar.prologue;
+            if (lane < Cc) gdn_raw_gates(b0, a0, eA, dtb, bm);
+            if (lane + 32 < Cc) gdn_raw_gates(b1, a1, eA, dtb, bm);
         }
         chunk_gates(gs, b0, b1, a0, a1, lane);
     }
@@ -377,9 +402,11 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         // 1 / ||k_i|| and 1 / ||q_i|| from the tiles (rows 0-63 K, 64-127 Q of each d-block),
         // two threads per row, while the gram runs
         if (ctl.wait(B_FULL, 0)) {
-            const int r = tid >> 1;
-            const float rn = inv_row_norm(sb + OFF_KV, r, tid & 1, 16384);
-            if ((tid & 1) == 0) gs[r < 64 ? G_RK + r : G_RQ + r - 64] = rn;
+            if (tid < 2 * kC) {
+                const int r = tid >> 1;
+                const float rn = inv_row_norm(sb + OFF_KV, r, tid & 1, 16384);
+                if ((tid & 1) == 0) gs[G_RK + r] = rn;
+            }
         } else {
             ok = false;
         }
@@ -452,8 +479,8 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
                 tmem_wait_ld();
-                const float si = i < Cc ? (PRO ? scale * gs[G_RQ + i] : scale) : 0.f;
-                const float* g2c = gs + (PRO ? G_ET : G_G2);   // column table (with the key norms folded in)
+                const float si = i < Cc ? scale : 0.f;
+                const float* g2c = gs + G_G2;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const float4 ga = *reinterpret_cast<const float4*>(g2c + j0 + 8 * q4);
@@ -489,8 +516,13 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         const int i = x >> 3, ch = x & 7;
         uint32_t w4[4] = {0u, 0u, 0u, 0u}, b4[4] = {0u, 0u, 0u, 0u};
         if ((ch >> 1) <= (i >> 4)) {
-            const float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
-            const float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
+            float4 t0v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch));
+            float4 t1v = *reinterpret_cast<const float4*>(Tm + fidx(i, 8 * ch + 4));
+            if (PRO) {
+                const float ri = gs[G_RK + i];
+                t0v.x *= ri; t0v.y *= ri; t0v.z *= ri; t0v.w *= ri;
+                t1v.x *= ri; t1v.y *= ri; t1v.z *= ri; t1v.w *= ri;
+            }
             // (with the prologue beta e^G / ||k||: W = T diag(beta e^G) K / ||k|| by rows of K)
             const float4 e0 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch);
             const float4 e1 = *reinterpret_cast<const float4*>(gs + G_BEG + 8 * ch + 4);
@@ -511,8 +543,8 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     if (tid == 0) {
         if (load) {
             const uint32_t fb = ctl.bar(B_FULL);     // the phase V opened
-            tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, (int)t0, fb);
-            tma_load_2d(sb + OFF_KV + 8192, &tm_k, 64, (int)t0, fb);
+            tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, (int)t0k, fb);
+            tma_load_2d(sb + OFF_KV + 8192, &tm_k, 64, (int)t0k, fb);
         }
         ok = ctl.wait(B_FULL, 1);
         if (ok) {

@@ -20,20 +20,27 @@
 namespace dn {
 
 // PRO: the Gated DeltaNet layer's prologue ("The full layer", steps 4 and 5):
-// q and k normalised per head, beta = sigmoid(b), g = -exp(A_log) softplus(a +
-// dt_bias), from the raw b and a in `beta` and `g` (scalar gate).
-template <int DK, int DV, typename Tin, int GATE, bool PRO = false>
+// q and k normalised per head, beta = bmul sigmoid(b) (bmul 1, or 2 for the
+// gate in (0, 2)), g = -exp(A_log) softplus(a + dt_bias), from the raw b and a
+// in `beta` and `g` (scalar gate).
+// NORM: the layer's gated RMSNorm ("The full layer", step 7) on the step's
+// output row: o <- weight * o / sqrt(mean(o^2) + eps) * act(z), act = SiLU
+// (NORM 1) or the logistic sigmoid (NORM 2); z [B, H, d_v], weight [d_v].
+template <int DK, int DV, typename Tin, int GATE, bool PRO = false, int NORM = 0>
 __global__ void __launch_bounds__(2 * DV)
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const float* __restrict__ beta,
                    const float* __restrict__ g, float* __restrict__ S,
                    Tin* __restrict__ o, float scale, const float* __restrict__ A_log = nullptr,
-                   const float* __restrict__ dt_bias = nullptr, int H = 1) {
+                   const float* __restrict__ dt_bias = nullptr, int H = 1, int rep = 1, float bmul = 1.f,
+                   const Tin* __restrict__ z = nullptr, const float* __restrict__ nw = nullptr,
+                   float eps = 0.f) {
     constexpr int NT = 2 * DV;     // threads
     constexpr int TPR = DV / 4;    // threads per state row
     constexpr int RS = NT / TPR;   // row sets (8)
     constexpr int RPT = DK / RS;   // rows per thread
     const int64_t head = blockIdx.x;
+    const int64_t khead = rep == 1 ? head : (head / H) * (H / rep) + (head % H) / rep;   // q and k row
     const int tid = threadIdx.x;
     const int cg = tid % TPR;
     const int rs = tid / TPR;
@@ -50,14 +57,14 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         s[m] = ld_stream_f4(Sh + (rs + RS * m) * DV + cg * 4);
 
     for (int i = tid; i < DK; i += NT) {
-        ks[i] = ld_elem(k + head * DK + i);
-        qs[i] = (PRO ? 1.f : scale) * ld_elem(q + head * DK + i);
+        ks[i] = ld_elem(k + khead * DK + i);
+        qs[i] = (PRO ? 1.f : scale) * ld_elem(q + khead * DK + i);
         if (GATE == kGatePerKey) as[i] = expf(g[head * DK + i]);
     }
     const float4 vv = ld4(v + head * DV + cg * 4);
     float b = beta[head];
     float a = (GATE == kGateScalar) ? g[head] : 0.f;
-    if (PRO) gdn_raw_gates(b, a, expf(A_log[head % H]), dt_bias[head % H]);
+    if (PRO) gdn_raw_gates(b, a, expf(A_log[head % H]), dt_bias[head % H], bmul);
     if (GATE == kGateScalar) a = expf(a);
     else a = 1.0f;
     __syncthreads();
@@ -132,6 +139,19 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         float4 ov;
         ov.x = qsum.x + qk * dl.x; ov.y = qsum.y + qk * dl.y;
         ov.z = qsum.z + qk * dl.z; ov.w = qsum.w + qk * dl.w;
+        if (NORM) {
+            // the row's mean square over the TPR threads of row set 0 (a warp, or half of one)
+            float ss = ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w;
+            constexpr unsigned kMask = TPR >= 32 ? 0xffffffffu : ((1u << TPR) - 1u);
+#pragma unroll
+            for (int off = TPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(kMask, ss, off);
+            const float r = 1.f / sqrtf(ss / (float)DV + eps);
+            const float4 zz = ld4(z + head * DV + cg * 4);
+            const float4 ww = *reinterpret_cast<const float4*>(nw + cg * 4);
+            auto act = [](float x) { return NORM == 1 ? x / (1.f + __expf(-x)) : 1.f / (1.f + __expf(-x)); };
+            ov.x = ov.x * r * ww.x * act(zz.x); ov.y = ov.y * r * ww.y * act(zz.y);
+            ov.z = ov.z * r * ww.z * act(zz.z); ov.w = ov.w * r * ww.w * act(zz.w);
+        }
         st4(o + head * DV + cg * 4, ov);
     }
 }
@@ -144,19 +164,32 @@ static cudaError_t launch_decode_gate(const DecodeArgs& a, cudaStream_t st) {
     const Tin* v = static_cast<const Tin*>(a.v);
     Tin* o = static_cast<Tin*>(a.o);
     if (a.prologue) {
-        decode_step_kernel<DK, DV, Tin, kGateScalar, true><<<grid, 2 * DV, 0, st>>>(
-            q, k, v, a.beta, a.g, a.S, o, a.scale, a.A_log, a.dt_bias, (int)a.H);
+        const Tin* z = static_cast<const Tin*>(a.z);
+        if (a.norm == 1)
+            decode_step_kernel<DK, DV, Tin, kGateScalar, true, 1><<<grid, 2 * DV, 0, st>>>(
+                q, k, v, a.beta, a.g, a.S, o, a.scale, a.A_log, a.dt_bias, (int)a.H, a.rep, (float)a.prologue, z,
+                a.norm_weight, a.eps);
+        else if (a.norm == 2)
+            decode_step_kernel<DK, DV, Tin, kGateScalar, true, 2><<<grid, 2 * DV, 0, st>>>(
+                q, k, v, a.beta, a.g, a.S, o, a.scale, a.A_log, a.dt_bias, (int)a.H, a.rep, (float)a.prologue, z,
+                a.norm_weight, a.eps);
+        else
+            decode_step_kernel<DK, DV, Tin, kGateScalar, true><<<grid, 2 * DV, 0, st>>>(
+                q, k, v, a.beta, a.g, a.S, o, a.scale, a.A_log, a.dt_bias, (int)a.H, a.rep, (float)a.prologue);
         return counted(cudaGetLastError());
     }
     switch (a.gate) {
         case kGateNone:
-            decode_step_kernel<DK, DV, Tin, kGateNone><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            decode_step_kernel<DK, DV, Tin, kGateNone><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale,
+                                                                          nullptr, nullptr, (int)a.H, a.rep);
             break;
         case kGateScalar:
-            decode_step_kernel<DK, DV, Tin, kGateScalar><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            decode_step_kernel<DK, DV, Tin, kGateScalar><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale,
+                                                                          nullptr, nullptr, (int)a.H, a.rep);
             break;
         default:
-            decode_step_kernel<DK, DV, Tin, kGatePerKey><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale);
+            decode_step_kernel<DK, DV, Tin, kGatePerKey><<<grid, 2 * DV, 0, st>>>(q, k, v, a.beta, a.g, a.S, o, a.scale,
+                                                                          nullptr, nullptr, (int)a.H, a.rep);
             break;
     }
     return counted(cudaGetLastError());

@@ -55,10 +55,12 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 // The Gated DeltaNet layer's gates from its raw per-token inputs ("Linear
 // attention and Gated DeltaNet", ch. 28, "The full layer", step 5): beta =
-// sigmoid(b), g = -exp(A_log) softplus(a + dt_bias), softplus(x) = log(1 + e^x)
-// (x above 20 taken as x).  eA = exp(A_log) of the head.
-__device__ __forceinline__ void gdn_raw_gates(float& b, float& a, float eA, float dt_bias) {
-    b = 1.f / (1.f + expf(-b));
+// bmul sigmoid(b), g = -exp(A_log) softplus(a + dt_bias), softplus(x) =
+// log(1 + e^x) (x above 20 taken as x).  eA = exp(A_log) of the head; bmul is 1,
+// or 2 for the gate 2 sigmoid(b) in (0, 2) that admits the negative eigenvalues
+// of D2L 12.5, "The reflection hiding in the delta rule".
+__device__ __forceinline__ void gdn_raw_gates(float& b, float& a, float eA, float dt_bias, float bmul) {
+    b = bmul / (1.f + expf(-b));
     const float x = a + dt_bias;
     a = -eA * (x > 20.f ? x : log1pf(expf(x)));
 }

@@ -21,11 +21,24 @@ struct ChunkArgs {
     void* ws;                 // tensor-core path: workspace of tc_workspace_bytes(), 256-byte aligned
     float* snaps;             // null, or [B, H, n_snap, d_k, d_v]: the state after every snap_every chunks
     int snap_every, n_snap;
-    // the layer's prologue inside the kernels (tensor-core path, scalar gate): beta and g
-    // hold the raw b and a; q and k are normalised per row
-    bool prologue;
+    // the layer's prologue inside the kernels (scalar gate): beta and g hold the raw b and
+    // a; q and k are normalised per row.  0: off; else beta = prologue * sigmoid(b)
+    // (1, or 2 for the gate in (0, 2))
+    int prologue;
     const float* A_log;       // [H]
     const float* dt_bias;     // [H]
+    int rep = 1;              // value heads per key head: q and k have H / rep heads
+    // a packed batch (tensor-core path): N sequences of the B = 1 row of T tokens,
+    // sequence s at tokens cu_seqlens[s] .. cu_seqlens[s + 1] - 1 (device int32 [N + 1]);
+    // S0 and S_T are then [N, H, d_k, d_v].  Null: B independent rows.
+    const int* cu_seqlens = nullptr;
+    int N = 0;
+    // with the prologue (tensor-core path): the layer's gated RMSNorm on the output rows
+    // (0 none, 1 SiLU(z), 2 sigmoid(z)); o then receives y token-major [B, T, H, d_v], as z
+    int norm = 0;
+    const void* z = nullptr;
+    const float* norm_weight = nullptr;
+    float eps = 0.f;
 };
 
 struct DecodeArgs {
@@ -38,13 +51,32 @@ struct DecodeArgs {
     bool bf16;
     int gate;
     // the layer's prologue (scalar gate): beta and g hold the raw b and a; q and k are
-    // normalised inside
-    bool prologue;
+    // normalised inside.  0: off; else beta = prologue * sigmoid(b)
+    int prologue;
     const float* A_log;       // [H]
     const float* dt_bias;     // [H]
+    int rep = 1;              // value heads per key head
+    // with the prologue: the gated RMSNorm on the output row (0 none, 1 SiLU(z), 2 sigmoid(z))
+    int norm = 0;
+    const void* z = nullptr;  // [B, H, d_v] dtype
+    const float* norm_weight = nullptr;   // [d_v]
+    float eps = 0.f;
 };
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t st);
+
+// The generalised delta rule of RWKV-7 in chunks, fp32 on CUDA cores (chunk_general.cu).
+struct GeneralArgs {
+    const void* q; const float* wlog; const void* kappa; const float* a; const void* k; const void* v;
+    const float* S0;
+    void* o; float* S_T;
+    int64_t B, T, H;
+    int dk, dv, chunk;
+    float scale;
+    bool bf16;
+};
+cudaError_t launch_chunk_general(const GeneralArgs& a, cudaStream_t st);
+int general_max_chunk();
 
 // The layer's causal conv over time (layer_ops.cu).
 struct ConvArgs {

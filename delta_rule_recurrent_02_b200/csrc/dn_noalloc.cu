@@ -12,10 +12,11 @@
 // The area is a file-scope __device__ array: the driver creates it once per
 // device when it loads this library's code there, and it stays until the
 // process exits.  Host code cannot use the array's name as a device address,
-// so the first call on each device looks the address up with
-// cudaGetSymbolAddress (with that device current) and keeps it.
+// so every call looks the address up with cudaGetSymbolAddress, with the
+// call's device current.  Nothing is cached: after a cudaDeviceReset or a
+// primary-context teardown the library's code is loaded again and the array
+// may move, and a kept address would then point at freed memory.
 #include <cuda_runtime.h>
-#include <mutex>
 #include <stdint.h>
 #include <stdio.h>
 
@@ -25,27 +26,15 @@
 namespace {
 
 constexpr size_t kScratchBytes = DN_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of this device's scratch area (looked up on first use).
+// Device address of the current device's scratch area, looked up afresh.
 cudaError_t scratch_for_current_device(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

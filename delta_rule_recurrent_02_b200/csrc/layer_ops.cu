@@ -119,34 +119,15 @@ causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __res
     using raw = typename VT::raw;
     constexpr int kCh = kConvThreads * V;       // channels of the block
     constexpr int kRow = kCh + 4;               // padded tap row: 16-byte aligned, banks shifted
+    constexpr int kPer = (kCh * K + kConvThreads - 1) / kConvThreads;   // filter values per thread
     __shared__ __align__(16) float ws[K][kRow];
     const int cb0 = blockIdx.x * kCh;
     const int nch = min(kCh, C - cb0);
-    for (int e = threadIdx.x; e < nch * K; e += kConvThreads) {
-        const int ch = e / K;
-        ws[e - ch * K][ch] = w[(int64_t)cb0 * K + e];
-    }
-    __syncthreads();
     const int cl = threadIdx.x * V;
     const int c0 = cb0 + cl;
-    if (c0 >= C) return;
+    const bool active = c0 < C;
     const int64_t b = blockIdx.z;
     const int t0 = blockIdx.y * kConvRows;
-
-    float wf[K][V];
-#pragma unroll
-    for (int j = 0; j < K; ++j) {
-        if constexpr (V % 4 == 0) {
-#pragma unroll
-            for (int v = 0; v < V; v += 4) {
-                const float4 f = *reinterpret_cast<const float4*>(&ws[j][cl + v]);
-                wf[j][v] = f.x; wf[j][v + 1] = f.y; wf[j][v + 2] = f.z; wf[j][v + 3] = f.w;
-            }
-        } else {
-#pragma unroll
-            for (int v = 0; v < V; ++v) wf[j][v] = ws[j][cl + v];
-        }
-    }
 
     // input row t of this thread's channels: x for t >= 0, the carried state before
     const Tin* xb = x + b * T * ld_x + c0;
@@ -162,16 +143,53 @@ causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __res
         }
     };
 
+    // the tile's rows first, so that their loads overlap the filter staging
     raw rows[K - 1 + kConvRows];
+    if (active) {
 #pragma unroll
-    for (int i = 0; i < K - 1 + kConvRows; ++i) {
-        const int t = t0 - (K - 1) + i;
-        if (t < 0) {
-            float f[V];
-            load_row(t, f);
-            rows[i] = VT::from_f(f);
-        } else if (t < T) {
-            rows[i] = *reinterpret_cast<const raw*>(xb + (int64_t)t * ld_x);
+        for (int i = 0; i < K - 1 + kConvRows; ++i) {
+            const int t = t0 - (K - 1) + i;
+            if (t < 0) {
+                float f[V];
+                load_row(t, f);
+                rows[i] = VT::from_f(f);
+            } else if (t < T) {
+                rows[i] = *reinterpret_cast<const raw*>(xb + (int64_t)t * ld_x);
+            }
+        }
+    }
+    // the block's filters, tap-major in shared memory: every load issued before any store
+    {
+        float wv[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int e = threadIdx.x + u * kConvThreads;
+            wv[u] = e < nch * K ? w[(int64_t)cb0 * K + e] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int e = threadIdx.x + u * kConvThreads;
+            if (e < nch * K) {
+                const int ch = e / K;
+                ws[e - ch * K][ch] = wv[u];
+            }
+        }
+    }
+    __syncthreads();
+    if (!active) return;
+
+    float wf[K][V];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if constexpr (V % 4 == 0) {
+#pragma unroll
+            for (int v = 0; v < V; v += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(&ws[j][cl + v]);
+                wf[j][v] = f.x; wf[j][v + 1] = f.y; wf[j][v + 2] = f.z; wf[j][v + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) wf[j][v] = ws[j][cl + v];
         }
     }
     // rows before token 0 were rounded back to Tin above; they are Tin values already
@@ -265,63 +283,57 @@ template <typename Tin, int D, bool SILU, bool X_HEAD_MAJOR>
 __global__ void __launch_bounds__(kNormWarps * 32)
 rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, const float* __restrict__ w,
                       Tin* __restrict__ y, int64_t rows, int T, int H, float eps) {
-    constexpr int E = D / 32;                                  // channels per lane
-    constexpr int VW = E < 16 / (int)sizeof(Tin) ? E : 16 / (int)sizeof(Tin);   // per access
-    constexpr int NV = E / VW;
-    static_assert(E * 32 == D && NV * VW == E, "D / 32 channels per lane in whole accesses");
-    using VT = Vec<Tin, VW>;
+    constexpr int VE = 16 / (int)sizeof(Tin);                   // channels per 16-byte access
+    constexpr int LPR = D / VE < 32 ? D / VE : 32;              // lanes per row
+    constexpr int NV = D / (VE * LPR);                          // accesses per lane
+    constexpr int RPW = 32 / LPR;                               // rows per warp
+    static_assert(NV * VE * LPR == D && RPW * LPR == 32, "row split");
+    using VT = Vec<Tin, VE>;
     using raw = typename VT::raw;
-    const int lane = threadIdx.x & 31;
-    const int64_t r0 = ((int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5)) * kNormRows;
-    if (r0 >= rows) return;
-    float wl[E];
+    const int lane = threadIdx.x & 31, l = lane % LPR;
+    const int64_t r0w = ((int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5)) * RPW;
+    if (r0w >= rows) return;
+    const int64_t r = r0w + lane / LPR;
+    const bool valid = r < rows;
+    int64_t xr = r;
+    if (X_HEAD_MAJOR && valid) {
+        const int64_t h = r % H, bt = r / H;
+        const int64_t t = bt % T, b = bt / T;
+        xr = (b * H + h) * T + t;
+    }
+    float xf[NV * VE], zf[NV * VE];
+    float ss = 0.f;
+    if (valid) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) wl[e] = w[lane * E + e];
-    float xf[kNormRows][E], zf[kNormRows][E];
-#pragma unroll
-    for (int u = 0; u < kNormRows; ++u) {
-        const int64_t r = r0 + u;                  // r = (b T + t) H + h
-        if (r < rows) {
-            int64_t xr = r;
-            if (X_HEAD_MAJOR) {
-                const int64_t h = r % H, bt = r / H;
-                const int64_t t = bt % T, b = bt / T;
-                xr = (b * H + h) * T + t;
-            }
-#pragma unroll
-            for (int a = 0; a < NV; ++a) {
-                VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + lane * E + a * VW), xf[u] + a * VW);
-                VT::to_f(*reinterpret_cast<const raw*>(z + r * D + lane * E + a * VW), zf[u] + a * VW);
-            }
+        for (int a = 0; a < NV; ++a) {
+            const int c = (a * LPR + l) * VE;
+            VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + c), xf + a * VE);
+            VT::to_f(*reinterpret_cast<const raw*>(z + r * D + c), zf + a * VE);
         }
+#pragma unroll
+        for (int e = 0; e < NV * VE; ++e) ss = fmaf(xf[e], xf[e], ss);
     }
 #pragma unroll
-    for (int u = 0; u < kNormRows; ++u) {
-        const int64_t r = r0 + u;
-        if (r < rows) {
-            float ss = 0.f;
+    for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (!valid) return;
+    const float inv = 1.f / sqrtf(ss / (float)D + eps);
 #pragma unroll
-            for (int e = 0; e < E; ++e) ss = fmaf(xf[u][e], xf[u][e], ss);
+    for (int a = 0; a < NV; ++a) {
+        const int c = (a * LPR + l) * VE;
+        float out[VE];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = 1.f / sqrtf(ss / (float)D + eps);
-            float out[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float gate = SILU ? silu(zf[u][e]) : sigmoid(zf[u][e]);
-                out[e] = wl[e] * (xf[u][e] * inv) * gate;
-            }
-#pragma unroll
-            for (int a = 0; a < NV; ++a)
-                *reinterpret_cast<raw*>(y + r * D + lane * E + a * VW) = VT::from_f(out + a * VW);
+        for (int e = 0; e < VE; ++e) {
+            const float gate = SILU ? silu(zf[a * VE + e]) : sigmoid(zf[a * VE + e]);
+            out[e] = w[c + e] * (xf[a * VE + e] * inv) * gate;
         }
+        *reinterpret_cast<raw*>(y + r * D + c) = VT::from_f(out);
     }
 }
 
 template <typename Tin, int D>
 cudaError_t launch_norm_d(const NormArgs& a, cudaStream_t st) {
     const int64_t rows = a.B * a.T * a.H;
-    const int64_t per_block = (int64_t)kNormWarps * kNormRows;
+    const int64_t per_block = (int64_t)kNormWarps * (32 / (D * (int)sizeof(Tin) / 16 < 32 ? D * (int)sizeof(Tin) / 16 : 32));
     const dim3 grid((unsigned)((rows + per_block - 1) / per_block));
     const Tin* x = static_cast<const Tin*>(a.x);
     const Tin* z = static_cast<const Tin*>(a.z);

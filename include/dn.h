@@ -198,6 +198,41 @@ DN_API int dn_chunk_fwd_gdn(const void* q, const void* k, const void* v, const f
                             int B, int T, int H, int d_k, int d_v, float scale,
                             void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/* Flags of the *_gdn_ex entry points. */
+enum {
+    /* beta = 2 sigmoid(b), in (0, 2): the write-strength gate of D2L 12.5, "The
+     * reflection hiding in the delta rule", whose transitions I - beta k k^T reach
+     * the eigenvalue 1 - beta < 0 (allow_neg_eigval) */
+    DN_GDN_BETA_2SIGMOID = 1,
+    /* the *_gdn_ex entry points with z: the gated RMSNorm's gate is sigmoid(z) instead of SiLU(z) */
+    DN_GDN_NORM_SIGMOID = 2
+};
+
+/*
+ * dn_chunk_fwd_gdn_ex -- dn_chunk_fwd_gdn on either kernel path, with flags.
+ * Same prologue and arguments as dn_chunk_fwd_gdn, plus
+ *   chunk, dtype, path   as dn_chunk_fwd_ex: the tensor-core kernels (bf16,
+ *         d_k = d_v = 128, chunk 64) or the fp32 CUDA-core kernel (fp32 or bf16
+ *         tokens, d in {64, 128}, chunk 1..64), which normalises q and k and
+ *         derives beta and g in the same way
+ *   flags DN_GDN_BETA_2SIGMOID: beta = 2 sigmoid(b); DN_GDN_NORM_SIGMOID: the
+ *         norm's gate is sigmoid(z), else SiLU(z); other bits return DN_ERR_INVALID
+ *   z, norm_weight, eps   NULL, NULL, 0: o is the rule's read-out [B,H,T,d_v].
+ *         Else the layer's gated RMSNorm (ch. 28, "The full layer", step 7) runs
+ *         on the output rows inside the kernels (tensor-core path only):
+ *         z [B,T,H,d_v] dtype (token-major, 16-byte aligned), norm_weight [d_v]
+ *         fp32 shared by every head, eps in (0, 1], and o receives
+ *         y = norm_weight * o / sqrt(mean(o^2) + eps) * act(z) token-major
+ *         [B,T,H,d_v], the layout of z (the mean over each head's d_v channels)
+ * The workspace is dn_chunk_fwd_workspace_size's for the scalar gate and the
+ * chosen path (zero on the CUDA-core path).
+ */
+DN_API int dn_chunk_fwd_gdn_ex(const void* q, const void* k, const void* v, const float* b, const float* a,
+                               const float* A_log, const float* dt_bias, const float* S0, void* o, float* S_T,
+                               int B, int T, int H, int d_k, int d_v, int chunk, float scale, dn_dtype dtype,
+                               dn_path path, int flags, const void* z, const float* norm_weight, float eps,
+                               void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 /*
  * dn_chunk_fwd_noalloc -- dn_chunk_fwd for callers that cannot allocate device
  * memory (a process that reserved the device's memory for its own pools, a
@@ -211,9 +246,13 @@ DN_API int dn_chunk_fwd_gdn(const void* q, const void* k, const void* v, const f
  * allocates or frees memory.
  *   - The area exists once per device, created when the library's code is
  *     loaded there, and is held until the process exits.
- *   - The first call on a device looks up the area's address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - Every call looks up the area's address (cudaGetSymbolAddress, with the
+ *     call's device current) and keeps nothing: after a cudaDeviceReset the
+ *     library's code is loaded again and the area may have moved.
+ *   - Capacity: a (b, h, chunk) tile takes 40,960 bytes with no gate or the
+ *     scalar gate (about 1638 tiles fit, e.g. B*H = 12 at T = 8192) and
+ *     74,240 bytes with the per-key gate (about 903 tiles, e.g. B*H = 7 at
+ *     T = 8192), plus 4 bytes of ready flag per tile.
  *   - A request needing more scratch than the area returns DN_ERR_UNSUPPORTED
  *     (dn_last_error() gives both sizes) before any device work.
  *   - Every call on a device shares the area and it keeps the last call's
@@ -222,13 +261,111 @@ DN_API int dn_chunk_fwd_gdn(const void* q, const void* k, const void* v, const f
  *     threads) race on it: order them on one stream, or use dn_chunk_fwd_ex
  *     with separate workspaces.
  */
-#define DN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)   /* 64 MiB: 1638 (b, h, chunk) tiles */
+#define DN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)   /* 64 MiB */
 
 DN_API int dn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                 const float* beta, const float* g, const float* S0,
                                 void* o, float* S_T,
                                 int B, int T, int H, int d_k, int d_v, int chunk, float scale,
                                 dn_dtype dtype, dn_gate gate, void* cuda_stream);
+
+/*
+ * dn_chunk_fwd_gva -- the chunked prefill with grouped value heads ("Linear
+ * attention and Gated DeltaNet", ch. 28, "The full layer", step 3: the
+ * layer projects fewer key heads than value heads, and each key head's q and
+ * k serve a group of value heads).
+ *
+ *   q, k      [B,H_k,T,d_k] dtype   H_k key heads
+ *   v, o      [B,H,T,d_v]   dtype   H value heads, H a multiple of H_k
+ *   beta      [B,H,T] fp32;  g NULL | [B,H,T] fp32 (per value head)
+ *   S0, S_T   [B,H,d_k,d_v] fp32 (per value head), as for dn_chunk_fwd
+ *   workspace as for dn_chunk_fwd_ex, dn_chunk_fwd_workspace_size(B, T, H, ...)
+ *             bytes (value heads); NULL allocates it stream-ordered
+ *
+ * Value head h of batch row b runs the rule of dn_chunk_fwd on q[b, h / R],
+ * k[b, h / R] with R = H / H_k, and its own v, beta, g and state.  The
+ * tensor-core kernels load each key head's tiles by its row, so no repeated
+ * copy of q and k is formed.  Tensor-core path only: bf16, d_k = d_v = 128,
+ * chunk 64, gate DN_GATE_NONE or DN_GATE_SCALAR; other requests return
+ * DN_ERR_UNSUPPORTED.  H % H_k != 0 returns DN_ERR_INVALID.
+ */
+DN_API int dn_chunk_fwd_gva(const void* q, const void* k, const void* v, const float* beta, const float* g,
+                            const float* S0, void* o, float* S_T, int B, int T, int H_k, int H, int d_k,
+                            int d_v, float scale, dn_dtype dtype, dn_gate gate, void* workspace,
+                            size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * dn_chunk_fwd_varlen -- the chunked prefill of a packed batch ("Linear
+ * attention and Gated DeltaNet", ch. 28, "The state a request carries": each
+ * request carries its own fixed-size state).  N sequences of different lengths
+ * share one time axis; sequence s holds tokens cu_seqlens[s] ..
+ * cu_seqlens[s + 1] - 1 and runs the rule of dn_chunk_fwd from its own S0[s]
+ * to its own S_T[s], chunked from its own first token.
+ *
+ *   q, k        [H,T,d_k] dtype;  v, o [H,T,d_v] dtype  (B = 1, T tokens in all)
+ *   beta        [H,T] fp32;  g NULL | [H,T] fp32 (DN_GATE_NONE or DN_GATE_SCALAR)
+ *   S0, S_T     NULL | [N,H,d_k,d_v] fp32, as for dn_chunk_fwd
+ *   cu_seqlens  DEVICE int32 [N + 1], non-decreasing from 0 to T; N >= 1;
+ *               empty sequences are allowed (their S_T is S0, or zeros)
+ *   workspace   dn_chunk_fwd_varlen_workspace_size bytes, 256-byte aligned, or
+ *               NULL (allocated stream-ordered on cuda_stream)
+ *
+ * Tensor-core path: bf16, d_k = d_v = 128 (chunk 64); else DN_ERR_UNSUPPORTED.
+ * The kernels read cu_seqlens on the device (no host synchronisation): one
+ * small kernel builds the chunk tables in the workspace, then the WY kernel
+ * covers every chunk and the state pass every (sequence, head).  If
+ * cu_seqlens does not rise from 0 to T, nothing is computed (o is left as it
+ * was, S_T = S0) and the next dn_device_status() returns DN_ERR_INVALID.
+ */
+DN_API int dn_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* beta, const float* g,
+                               const float* S0, void* o, float* S_T, const int* cu_seqlens, int N, int T,
+                               int H, int d_k, int d_v, float scale, dn_dtype dtype, dn_gate gate,
+                               void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Bytes of workspace dn_chunk_fwd_varlen needs for N sequences of T tokens in all
+ * (it depends on N and T only, not on the lengths). */
+DN_API int dn_chunk_fwd_varlen_workspace_size(int N, int T, int H, int d_k, int d_v, dn_dtype dtype,
+                                              dn_gate gate, size_t* bytes);
+
+/*
+ * dn_decode_step_gva -- dn_decode_step with grouped value heads (ch. 28,
+ * "The full layer", step 3).  q, k [B,H_k,d_k]; v, o [B,H,d_v]; beta [B,H];
+ * g NULL | [B,H] | [B,H,d_k]; S [B,H,d_k,d_v] in place.  Value head h reads
+ * q and k of key head h / (H / H_k).  Every gate, dtype and d of
+ * dn_decode_step.  H % H_k != 0 returns DN_ERR_INVALID.
+ */
+DN_API int dn_decode_step_gva(const void* q, const void* k, const void* v, const float* beta, const float* g,
+                              float* S, void* o, int B, int H_k, int H, int d_k, int d_v, float scale,
+                              dn_dtype dtype, dn_gate gate, void* cuda_stream);
+
+/*
+ * dn_chunk_fwd_general -- the generalised delta rule of RWKV-7 ("DeltaNet:
+ * Memory That Edits", D2L 12.5, "The generalized delta rule"), chunked:
+ *
+ *     S_t = (diag(w_t) - (a_t * kappa_t) kappa_t^T) S_{t-1} + k_t v_t^T
+ *     o_t = S_t^T (scale q_t)        (read after the write, as for dn_chunk_fwd)
+ *
+ * with w_t = exp(w_log_t) a per-key-channel decay, kappa_t the removal key, a_t
+ * a per-channel removal rate and k_t the write key (k_t need not equal
+ * kappa_t; w = 1, kappa = k', a = beta, k = beta k' is DeltaNet).
+ *
+ *   q, kappa, k  [B,H,T,d_k] dtype;  v [B,H,T,d_v] dtype
+ *   w_log, a     [B,H,T,d_k] fp32 (w_log <= 0 expected, not enforced; kappa is
+ *                used as given, not normalised)
+ *   S0, S_T      NULL | [B,H,d_k,d_v] fp32, as for dn_chunk_fwd
+ *   o            [B,H,T,d_v] dtype
+ *   d_k, d_v in {64, 128}; chunk 1..32 (the result does not depend on it
+ *   beyond rounding)
+ *
+ * fp32 arithmetic on the CUDA cores (fp32 or bf16 storage): the page gives the
+ * recurrence only, and its chunkwise form (pairwise per-channel decays inside
+ * the sums) runs here as derived from it.  Same aliasing and error rules as
+ * dn_chunk_fwd.
+ */
+DN_API int dn_chunk_fwd_general(const void* q, const float* w_log, const void* kappa, const float* a,
+                                const void* k, const void* v, const float* S0, void* o, float* S_T,
+                                int B, int T, int H, int d_k, int d_v, int chunk, float scale, dn_dtype dtype,
+                                void* cuda_stream);
 
 /*
  * dn_decode_step -- one recurrent step ("The recurrent form", ch. 28; KDA's
@@ -258,6 +395,25 @@ DN_API int dn_decode_step(const void* q, const void* k, const void* v,
 DN_API int dn_decode_step_gdn(const void* q, const void* k, const void* v, const float* b, const float* a,
                               const float* A_log, const float* dt_bias, float* S, void* o,
                               int B, int H, int d_k, int d_v, float scale, dn_dtype dtype, void* cuda_stream);
+
+/*
+ * dn_decode_step_gdn_ex -- dn_decode_step_gdn with flags and, optionally, the
+ * layer's gated RMSNorm fused into the step ("Linear attention and Gated
+ * DeltaNet", ch. 28, "The full layer", step 7, RMSNormGated):
+ *   flags        DN_GDN_BETA_2SIGMOID: beta = 2 sigmoid(b);
+ *                DN_GDN_NORM_SIGMOID: the norm's gate is sigmoid(z), else SiLU(z);
+ *                other bits return DN_ERR_INVALID
+ *   z            NULL (o is the rule's read-out) | [B,H,d_v] dtype: then
+ *                o = norm_weight * o / sqrt(mean(o^2) + eps) * act(z), the mean
+ *                over the d_v channels of each head's row
+ *   norm_weight  [d_v] fp32, shared by every head (required with z)
+ *   eps          in (0, 1] (required with z; the page uses 1e-6)
+ * z and norm_weight must be 16-byte aligned and must not overlap o or S.
+ */
+DN_API int dn_decode_step_gdn_ex(const void* q, const void* k, const void* v, const float* b, const float* a,
+                                 const float* A_log, const float* dt_bias, float* S, void* o,
+                                 int B, int H, int d_k, int d_v, float scale, dn_dtype dtype, int flags,
+                                 const void* z, const float* norm_weight, float eps, void* cuda_stream);
 
 /*
  * dn_causal_conv1d -- step 2 of the Gated DeltaNet layer ("Linear attention
@@ -327,7 +483,9 @@ DN_API const char* dn_last_error(void);
 
 /* ABI version, (major << 16) | minor.  2.2: the per-key gate on the tensor-core path;
  * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn; 2.5: dn_decode_step_gdn;
- * 2.6: dn_causal_conv1d, dn_rms_norm_gated. */
+ * 2.6: dn_causal_conv1d, dn_rms_norm_gated; 2.7: dn_chunk_fwd_gva, dn_decode_step_gva,
+ * dn_chunk_fwd_gdn_ex, dn_decode_step_gdn_ex (the CUDA-core prologue and the 2 sigmoid gate),
+ * dn_chunk_fwd_varlen, dn_chunk_fwd_varlen_workspace_size, dn_chunk_fwd_general. */
 DN_API int dn_version(void);
 
 /*

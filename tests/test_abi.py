@@ -333,3 +333,69 @@ def test_layer_op_bindings_check_shapes_before_any_device_call():
         dn.dn_rms_norm_gated(o, z, nw, yn)
     with pytest.raises(ValueError, match="CUDA"):
         dn.dn_rms_norm_gated(z, z, nw, yn, x_head_major=False)
+
+
+# ---- entry points added with grouped heads, packed batches and the 2 sigmoid gate ----
+
+def test_gva_rejects_before_device_work(lib):
+    # 8 value heads over 3 key heads: not a whole group per key head
+    st = lib.dn_chunk_fwd_gva(A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, None, A + 5 * STEP, None,
+                              1, 64, 3, 8, 128, 128, 1.0, 1, 1, None, 0, None)
+    assert st == dn.DN_ERR_INVALID
+    # fp32 tokens: grouped heads run on the tensor-core kernels only
+    st = lib.dn_chunk_fwd_gva(A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, None, A + 5 * STEP, None,
+                              1, 64, 2, 8, 128, 128, 1.0, 0, 1, None, 0, None)
+    assert st == dn.DN_ERR_UNSUPPORTED
+    st = lib.dn_decode_step_gva(A, A + STEP, A + 2 * STEP, A + 3 * STEP, None, A + 4 * STEP, A + 5 * STEP,
+                                2, 3, 8, 128, 128, 1.0, 1, 0, None)
+    assert st == dn.DN_ERR_INVALID
+
+
+def varlen_call(lib, **over):
+    args = dict(q=A, k=A + STEP, v=A + 2 * STEP, beta=A + 3 * STEP, g=A + 4 * STEP, S0=None, o=A + 5 * STEP,
+                S_T=A + 6 * STEP, cu=A + 7 * STEP, N=3, T=200, H=2, dk=128, dv=128, dtype=1, gate=1)
+    args.update(over)
+    return lib.dn_chunk_fwd_varlen(args["q"], args["k"], args["v"], args["beta"], args["g"], args["S0"], args["o"],
+                                   args["S_T"], args["cu"], args["N"], args["T"], args["H"], args["dk"], args["dv"],
+                                   1.0, args["dtype"], args["gate"], None, 0, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(cu=None), dn.DN_ERR_INVALID),
+    (dict(N=0), dn.DN_ERR_INVALID),
+    (dict(cu=A + 7 * STEP + 2), dn.DN_ERR_INVALID),          # not 4-byte aligned
+    (dict(o=A + 7 * STEP), dn.DN_ERR_INVALID),               # o overlaps cu_seqlens
+    (dict(gate=2), dn.DN_ERR_UNSUPPORTED),                   # per-key gate
+    (dict(dtype=0), dn.DN_ERR_UNSUPPORTED),                  # fp32 tokens
+    (dict(dk=64, dv=64), dn.DN_ERR_UNSUPPORTED),
+])
+def test_varlen_rejects_before_device_work(lib, over, code):
+    assert varlen_call(lib, **over) == code
+
+
+def test_varlen_workspace_size_depends_on_N_and_T(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.dn_chunk_fwd_varlen_workspace_size(3, 200, 2, 128, 128, 1, 1, ctypes.byref(out)) == dn.DN_OK
+    # at most 200 / 64 + 3 = 6 chunks per head: 12 tiles of 40 KiB, their flags, then the tables
+    tiles = 2 * (200 // 64 + 3)
+    assert out.value >= tiles * 40960 + 4 * (tiles + 1)
+    big = ctypes.c_size_t(0)
+    assert lib.dn_chunk_fwd_varlen_workspace_size(30, 200, 2, 128, 128, 1, 1, ctypes.byref(big)) == dn.DN_OK
+    assert big.value > out.value
+
+
+def test_gdn_ex_rejects_unknown_flags(lib):
+    st = lib.dn_chunk_fwd_gdn_ex(A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, A + 5 * STEP,
+                                 A + 5 * STEP + 256, None, A + 6 * STEP, None, 1, 8, 1, 128, 128, 64, 1.0, 1, 0, 4,
+                                 None, None, 0.0, None, 0, None)
+    assert st == dn.DN_ERR_INVALID
+    st = lib.dn_decode_step_gdn_ex(A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, A + 5 * STEP,
+                                   A + 5 * STEP + 256, A + 6 * STEP, A + 7 * STEP, 1, 1, 128, 128, 1.0, 1, 8, None,
+                                   None, 0.0, None)
+    assert st == dn.DN_ERR_INVALID
+    # the norm needs z and its weight, and a positive eps
+    base = (A, A + STEP, A + 2 * STEP, A + 3 * STEP, A + 4 * STEP, A + 5 * STEP, A + 5 * STEP + 256, A + 6 * STEP,
+            A + 7 * STEP, 1, 1, 128, 128, 1.0, 1)
+    assert lib.dn_decode_step_gdn_ex(*base, 2, None, None, 0.0, None) == dn.DN_ERR_INVALID
+    assert lib.dn_decode_step_gdn_ex(*base, 0, A + 8 * STEP, None, 1e-6, None) == dn.DN_ERR_INVALID
+    assert lib.dn_decode_step_gdn_ex(*base, 0, A + 8 * STEP, A + 9 * STEP, 0.0, None) == dn.DN_ERR_INVALID

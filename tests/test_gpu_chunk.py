@@ -254,25 +254,37 @@ def test_gated_deltanet_full(cuda_device, path):
     assert_close(S, rS, "bf16", "S_T")
 
 
-def _sampled(cfg, path, n_heads, seed):
-    inp = W.gen_prefill_config(cfg)
+_FULL_ORACLE = {}
+
+
+def _full_oracle(cfg):
+    """Inputs and the oracle's o, S_T on every head of a workload, computed once
+    per test session and shared by both kernel paths."""
+    if cfg.name not in _FULL_ORACLE:
+        inp = W.gen_prefill_config(cfg)
+        _FULL_ORACLE.clear()                # one workload's arrays at a time
+        _FULL_ORACLE[cfg.name] = (inp, oracle_prefill(inp, cfg.scale))
+    return _FULL_ORACLE[cfg.name]
+
+
+def _every_head(cfg, path):
+    # every (b, h) of the workload against the oracle: the kernels hand tiles to their
+    # groups from a shared counter, so a fault in that scheduling could hit any head
+    inp, (ro, rS) = _full_oracle(cfg)
     o, S = run(to_dev(inp), cfg.scale, chunk=cfg.chunk, path=path)
-    gen = torch.Generator().manual_seed(seed)
-    flat = torch.randperm(cfg.B * cfg.H, generator=gen)[:n_heads].tolist()
-    bh = [(f // cfg.H, f % cfg.H) for f in flat]
-    ro, rS = oracle_prefill(inp, cfg.scale, bh=bh)
-    assert_close(pick(o.cpu(), bh), ro, "bf16", "o (sampled heads)")
-    assert_close(pick(S.cpu(), bh), rS, "bf16", "S_T (sampled heads)")
+    dn.dn_device_status()
+    assert_close(o, ro, "bf16", "o (every head)")
+    assert_close(S, rS, "bf16", "S_T (every head)")
 
 
-@pytest.mark.parametrize("path", PATHS)
-def test_gated_deltanet_long_sampled(cuda_device, path):
-    _sampled(W.GDN_LONG, path, n_heads=4, seed=1)
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_gated_deltanet_long_full(cuda_device, path):
+    _every_head(W.GDN_LONG, path)
 
 
-@pytest.mark.parametrize("path", PATHS)
-def test_kda_sampled(cuda_device, path):
-    _sampled(W.KDA_PREFILL, path, n_heads=8, seed=2)
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_kda_full(cuda_device, path):
+    _every_head(W.KDA_PREFILL, path)
 
 
 @pytest.mark.parametrize("g_shift", [-1.0, 8.0])
@@ -375,13 +387,12 @@ def test_gdn_layer_prologue(cuda_device, B, H, T):
     S = torch.full((B, H, 128, 128), float("nan"), device="cuda")
     dn.dn_chunk_fwd_gdn(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], d["S0"], o, S, scale=sc)
     dn.dn_device_status()
-    bh = None if B * H <= 8 else [(0, 0), (B - 1, H - 1), (B // 2, 5)]
-    ro, rS = _gdn_oracle(raw, sc, bh=bh)
-    assert_close(o if bh is None else pick(o, bh), ro, "bf16", "o")
-    assert_close(S if bh is None else pick(S, bh), rS, "bf16", "S_T")
+    ro, rS = _gdn_oracle(raw, sc)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(S, rS, "bf16", "S_T")
 
 
-def test_gdn_layer_prologue_full_size_sampled(cuda_device):
+def test_gdn_layer_prologue_full_size(cuda_device):
     B, H, T = 4, 16, 4096
     raw = _gdn_raw(B, H, T, seed=9)
     d = to_dev(raw)
@@ -390,7 +401,68 @@ def test_gdn_layer_prologue_full_size_sampled(cuda_device):
     S = torch.empty((B, H, 128, 128), device="cuda")
     dn.dn_chunk_fwd_gdn(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], d["S0"], o, S, scale=sc)
     dn.dn_device_status()
-    bh = [(0, 0), (3, 15), (1, 7)]
-    ro, rS = _gdn_oracle(raw, sc, bh=bh)
-    assert_close(pick(o.cpu(), bh), ro, "bf16", "o (sampled heads)")
-    assert_close(pick(S.cpu(), bh), rS, "bf16", "S_T (sampled heads)")
+    # every head
+    ro, rS = _gdn_oracle(raw, sc)
+    assert_close(o, ro, "bf16", "o (every head)")
+    assert_close(S, rS, "bf16", "S_T (every head)")
+
+
+def _gdn_raw_d(B, H, T, d, dtype, seed):
+    """As _gdn_raw, at head size d and token dtype `dtype`."""
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, T, d, generator=gen) * (0.2 + 3 * torch.rand(B, H, T, 1, generator=gen))
+    k = torch.randn(B, H, T, d, generator=gen) * (0.2 + 3 * torch.rand(B, H, T, 1, generator=gen))
+    q[0, 0, 3] = 0.0
+    k[-1, -1, T // 2] = 0.0
+    v = torch.randn(B, H, T, d, generator=gen)
+    b = torch.randn(B, H, T, generator=gen)
+    a = torch.randn(B, H, T, generator=gen) - 1.0
+    A_log = torch.log(1 + 3 * torch.rand(H, generator=gen))
+    dt_bias = 0.5 * torch.randn(H, generator=gen)
+    S0 = 0.2 * torch.randn(B, H, d, d, generator=gen)
+    return {"q": q.to(dtype), "k": k.to(dtype), "v": v.to(dtype), "b": b, "a": a, "A_log": A_log,
+            "dt_bias": dt_bias, "S0": S0}
+
+
+@pytest.mark.parametrize("neg", [False, True])
+@pytest.mark.parametrize("path,dtype,d,chunk", [
+    ("tc", torch.bfloat16, 128, 64),
+    ("simt", torch.float32, 64, 64),
+    ("simt", torch.float32, 128, 16),
+    ("simt", torch.bfloat16, 128, 64),
+    ("simt", torch.bfloat16, 64, 5),
+])
+def test_gdn_prologue_ex_both_paths(cuda_device, neg, path, dtype, d, chunk):
+    # dn_chunk_fwd_gdn_ex: the layer's prologue on the tensor-core kernels and on the
+    # fp32 CUDA-core kernel; with allow_neg_eigval, beta = 2 sigmoid(b) ("DeltaNet:
+    # Memory That Edits", "The reflection hiding in the delta rule")
+    B, H, T = 2, 3, 150
+    raw = _gdn_raw_d(B, H, T, d, dtype, seed=1000 + d + chunk + 7 * neg)
+    dd = to_dev(raw)
+    sc = d ** -0.5
+    o = torch.full((B, H, T, d), float("nan"), dtype=dtype, device="cuda")
+    S = torch.full((B, H, d, d), float("nan"), device="cuda")
+    nb = dn.dn_chunk_fwd_workspace_size(B, T, H, d, d, chunk=chunk, dtype="bf16" if dtype == torch.bfloat16 else "f32",
+                                        gate="scalar", path=path)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+    dn.dn_chunk_fwd_gdn_ex(dd["q"], dd["k"], dd["v"], dd["b"], dd["a"], dd["A_log"], dd["dt_bias"], dd["S0"], o, S,
+                           chunk=chunk, scale=sc, path=path, allow_neg_eigval=neg, workspace=ws)
+    dn.dn_device_status()
+    qn, kn, beta, g = oracle.gdn_prologue(f64(raw["q"]), f64(raw["k"]), f64(raw["b"]), f64(raw["a"]),
+                                          f64(raw["A_log"]), f64(raw["dt_bias"]), allow_neg_eigval=neg)
+    ro, rS = oracle.delta_rule(qn, kn, f64(raw["v"]), beta, g, f64(raw["S0"]), scale=sc)
+    kind = "f32" if dtype == torch.float32 else "bf16"
+    assert_close(o, ro, kind, "o")
+    assert_close(S, rS, kind, "S_T")
+
+
+def test_gdn_prologue_ex_rejects_unknown_flags(cuda_device):
+    raw = _gdn_raw_d(1, 1, 8, 128, torch.bfloat16, seed=3)
+    dd = to_dev(raw)
+    o = torch.empty((1, 1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    lib = dn.load_library()
+    st = lib.dn_chunk_fwd_gdn_ex(dd["q"].data_ptr(), dd["k"].data_ptr(), dd["v"].data_ptr(), dd["b"].data_ptr(),
+                                 dd["a"].data_ptr(), dd["A_log"].data_ptr(), dd["dt_bias"].data_ptr(), None,
+                                 o.data_ptr(), None, 1, 8, 1, 128, 128, 64, 1.0, 1, 0, 4, None, None, 0.0, None, 0,
+                                 None)
+    assert st == dn.DN_ERR_INVALID

@@ -124,9 +124,10 @@ def test_decode_empty_and_errors(cuda_device):
     assert ei.value.status == dn.DN_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("neg", [False, True])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
-def test_decode_layer_prologue(cuda_device, dtype, dk, dv):
+def test_decode_layer_prologue(cuda_device, dtype, dk, dv, neg):
     # dn_decode_step_gdn: raw q and k (varied norms, one zero row), raw b and a with the
     # per-head A_log and dt_bias, against the oracle prologue then the oracle recurrence
     B, H, steps = 3, 5, 8
@@ -146,13 +147,56 @@ def test_decode_layer_prologue(cuda_device, dtype, dk, dv):
     outs = []
     for s in range(steps):
         o = torch.empty((B, H, dv), dtype=td, device="cuda")
-        dn.dn_decode_step_gdn(q[s].cuda(), k[s].cuda(), v[s].cuda(), b[s].cuda(), a[s].cuda(), A_log.cuda(),
-                              dt_bias.cuda(), S, o, scale=sc)
+        if neg:
+            # beta = 2 sigmoid(b) ("DeltaNet: Memory That Edits", "The reflection hiding in the delta rule")
+            dn.dn_decode_step_gdn_ex(q[s].cuda(), k[s].cuda(), v[s].cuda(), b[s].cuda(), a[s].cuda(), A_log.cuda(),
+                                     dt_bias.cuda(), S, o, scale=sc, allow_neg_eigval=True)
+        else:
+            dn.dn_decode_step_gdn(q[s].cuda(), k[s].cuda(), v[s].cuda(), b[s].cuda(), a[s].cuda(), A_log.cuda(),
+                                  dt_bias.cuda(), S, o, scale=sc)
         outs.append(o)
     dn.dn_device_status()
     # the prologue on [B,H,steps,...] (steps become the time axis)
     tr = lambda t: f64(t).transpose((1, 2, 0) + tuple(range(3, t.dim())))
-    qn, kn, beta, g = oracle.gdn_prologue(tr(q), tr(k), tr(b), tr(a), f64(A_log), f64(dt_bias))
+    qn, kn, beta, g = oracle.gdn_prologue(tr(q), tr(k), tr(b), tr(a), f64(A_log), f64(dt_bias), allow_neg_eigval=neg)
     ro, rS = oracle.delta_rule(qn, kn, tr(v), beta, g, f64(S0), scale=sc)
     assert_close(torch.stack(outs).permute(1, 2, 0, 3), ro, dtype, "o")
+    assert_close(S, rS, dtype, "S")
+
+
+@pytest.mark.parametrize("activation", ["silu", "sigmoid"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64)])
+def test_decode_prologue_and_gated_norm(cuda_device, activation, dtype, dk, dv):
+    # dn_decode_step_gdn_ex with z: the layer's prologue, the step and its gated RMSNorm
+    # ("The full layer", steps 4-7) in one kernel, against oracle.rms_norm_gated applied
+    # to the oracle recurrence's read-out
+    B, H, steps = 3, 4, 5
+    gen = torch.Generator().manual_seed(77 + dk + dv)
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    q = (torch.randn(steps, B, H, dk, generator=gen) * 2).to(td)
+    k = (torch.randn(steps, B, H, dk, generator=gen) * 2).to(td)
+    v = torch.randn(steps, B, H, dv, generator=gen).to(td)
+    z = (2 * torch.randn(steps, B, H, dv, generator=gen)).to(td)
+    b = torch.randn(steps, B, H, generator=gen)
+    a = torch.randn(steps, B, H, generator=gen)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen))
+    dt_bias = 0.5 * torch.randn(H, generator=gen)
+    w = 1 + 0.5 * torch.randn(dv, generator=gen)
+    S0 = 0.1 * torch.randn(B, H, dk, dv, generator=gen)
+    sc = dk ** -0.5
+    S = S0.cuda().clone()
+    outs = []
+    for s in range(steps):
+        o = torch.empty((B, H, dv), dtype=td, device="cuda")
+        dn.dn_decode_step_gdn_ex(q[s].cuda(), k[s].cuda(), v[s].cuda(), b[s].cuda(), a[s].cuda(), A_log.cuda(),
+                                 dt_bias.cuda(), S, o, scale=sc, z=z[s].cuda(), norm_weight=w.cuda(), eps=1e-6,
+                                 norm_activation=activation)
+        outs.append(o)
+    dn.dn_device_status()
+    tr = lambda t: f64(t).transpose((1, 2, 0) + tuple(range(3, t.dim())))
+    qn, kn, beta, g = oracle.gdn_prologue(tr(q), tr(k), tr(b), tr(a), f64(A_log), f64(dt_bias))
+    ro, rS = oracle.delta_rule(qn, kn, tr(v), beta, g, f64(S0), scale=sc)
+    ry = oracle.rms_norm_gated(ro, tr(z), f64(w), eps=1e-6, activation=activation)
+    assert_close(torch.stack(outs).permute(1, 2, 0, 3), ry, dtype, "y")
     assert_close(S, rS, dtype, "S")

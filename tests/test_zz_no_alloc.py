@@ -28,29 +28,70 @@ def ptr(t):
     return None if t is None else t.data_ptr()
 
 
+class DefaultPoolMeter:
+    """High-water mark of the device's default memory pool, the pool that
+    stream-ordered allocations (cudaMallocAsync) draw from when no other pool is
+    named, read through the driver API.  torch's caching allocator does not use
+    that pool, so between two reads it sees only the library's allocations."""
+
+    def __init__(self, device: int = 0):
+        from cuda.bindings import driver as cu
+        self.cu = cu
+        err, = cu.cuInit(0)
+        assert err == cu.CUresult.CUDA_SUCCESS, err
+        err, dev = cu.cuDeviceGet(device)
+        assert err == cu.CUresult.CUDA_SUCCESS, err
+        err, self.pool = cu.cuDeviceGetDefaultMemPool(dev)
+        assert err == cu.CUresult.CUDA_SUCCESS, err
+        self.attr = cu.CUmemPool_attribute.CU_MEMPOOL_ATTR_USED_MEM_HIGH
+
+    def reset(self):
+        err, = self.cu.cuMemPoolSetAttribute(self.pool, self.attr, self.cu.cuuint64_t(0))
+        assert err == self.cu.CUresult.CUDA_SUCCESS, err
+
+    def high(self) -> int:
+        err, v = self.cu.cuMemPoolGetAttribute(self.pool, self.attr)
+        assert err == self.cu.CUresult.CUDA_SUCCESS, err
+        return int(v)
+
+
 @pytest.mark.gpu
-def test_noalloc_matches_dn_chunk_fwd_on_two_calls(cuda_device):
+@pytest.mark.parametrize("gate", ["scalar", "per_key"])
+def test_noalloc_matches_dn_chunk_fwd_on_two_calls(cuda_device, gate):
     lib, f = noalloc_fn()
     stream = torch.cuda.current_stream()
+    meter = DefaultPoolMeter(torch.cuda.current_device())
     sc = 128 ** -0.5
+    gate_code = 1 if gate == "scalar" else 2
     # two different requests in a row: the second reuses the scratch area the
-    # first left behind
+    # first left behind (the per-key gate lays its tiles, gamma table and flags
+    # out differently, so both layouts run against the shared area)
     for B, H, T, seed in ((2, 4, 300, 71), (1, 3, 1000, 72)):
-        inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate="scalar", seed=seed, s0_std=0.2)
+        inp = W.gen_prefill(B, H, T, 128, 128, dtype="bf16", gate=gate, seed=seed, s0_std=0.2,
+                            g_shift=2.0 if gate == "scalar" else 3.0)
         d = to_dev(inp)
-        need = dn.dn_chunk_fwd_workspace_size(B, T, H, 128, 128)
+        need = dn.dn_chunk_fwd_workspace_size(B, T, H, 128, 128, gate=gate)
         assert 0 < need <= 64 << 20
         o = torch.full((B, H, T, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
         S = torch.full((B, H, 128, 128), float("nan"), device="cuda")
+        torch.cuda.synchronize()
+        meter.reset()
         st = f(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["beta"]), ptr(d["g"]), ptr(d["S0"]), ptr(o), ptr(S),
-               B, T, H, 128, 128, 64, sc, 1, 1, ctypes.c_void_p(stream.cuda_stream))
+               B, T, H, 128, 128, 64, sc, 1, gate_code, ctypes.c_void_p(stream.cuda_stream))
         assert st == dn.DN_OK, lib.dn_last_error()
+        torch.cuda.synchronize()
+        assert meter.high() == 0, "dn_chunk_fwd_noalloc drew memory from the default pool"
         o_ref = torch.empty_like(o)
         S_ref = torch.empty_like(S)
-        dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o_ref, S_ref, scale=sc)
+        # the allocating entry point (no workspace given) does move the meter: the
+        # check above can see a stream-ordered allocation
+        meter.reset()
+        dn.dn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o_ref, S_ref, scale=sc, gate=gate)
+        torch.cuda.synchronize()
+        assert meter.high() >= need
         dn.dn_device_status()
-        assert_close(o, o_ref.double().cpu().numpy(), "bf16", f"o (T={T})")
-        assert_close(S, S_ref.double().cpu().numpy(), "bf16", f"S_T (T={T})")
+        assert_close(o, o_ref.double().cpu().numpy(), "bf16", f"o (T={T}, {gate})")
+        assert_close(S, S_ref.double().cpu().numpy(), "bf16", f"S_T (T={T}, {gate})")
 
 
 def test_noalloc_rejects_requests_above_its_scratch_area():
