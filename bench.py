@@ -224,6 +224,31 @@ def oracle_sample_rate(prefill_heads=64, decode_heads=8192, seed_offset=0):
     return tokens / (full_p + full_d), full_p + full_d, desc, (tokens, full_p, full_d)
 
 
+def oracle_single_thread(prefill_heads=4):
+    """The fp64 oracle on one host thread for the small DeltaNet workload (whole)
+    and for the bench-size Gated DeltaNet prefill (a sample of heads, scaled to
+    all of them): {workload: {"s": seconds, "tokens_per_s": ..., "sample": ...}}."""
+    import oracle
+    from delta_rule_recurrent_02_b200 import workloads as W
+    f = lambda t: None if t is None else t.double().numpy()
+    out = {}
+    cfg = W.DELTANET_SMALL
+    inp = W.gen_prefill_config(cfg)
+    t0 = time.perf_counter()
+    oracle.delta_rule(*(f(inp[n]) for n in ("q", "k", "v", "beta", "g", "S0")), scale=cfg.scale, nthreads=1)
+    s = time.perf_counter() - t0
+    out[cfg.name] = {"s": s, "tokens_per_s": cfg.B * cfg.T / s, "sample": "whole workload"}
+    cfg = W.GDN_PREFILL
+    inp = W.gen_prefill(1, prefill_heads, cfg.T, cfg.dk, cfg.dv, dtype=cfg.dtype, gate=cfg.gate, seed=cfg.seed,
+                        q_norm=True, g_shift=cfg.g_shift)
+    t0 = time.perf_counter()
+    oracle.delta_rule(*(f(inp[n]) for n in ("q", "k", "v", "beta", "g")), None, scale=cfg.scale, nthreads=1)
+    s = (time.perf_counter() - t0) * (cfg.B * cfg.H) / prefill_heads
+    out[cfg.name] = {"s": s, "tokens_per_s": cfg.B * cfg.T / s,
+                     "sample": f"{prefill_heads} of {cfg.B * cfg.H} heads, scaled by head count"}
+    return out
+
+
 def run_reference(args):
     """The reference arm: the fp64 oracle timed as it stands on the host cores."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -244,7 +269,7 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
-                             "kind": "oracle", "sample": desc},
+                             "nproc": os.cpu_count(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -572,8 +597,9 @@ def main():
         reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]
         v = statistics.median(r[0] for r in reps)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": oracle.max_threads(),
-                                "kind": "oracle",
-                                "sample": f"median of {len(reps)} repetitions; each: " + reps[0][2]}
+                                "nproc": os.cpu_count(), "kind": "oracle",
+                                "sample": f"median of {len(reps)} repetitions; each: " + reps[0][2],
+                                "single_thread": oracle_single_thread()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -466,3 +466,39 @@ def test_gdn_prologue_ex_rejects_unknown_flags(cuda_device):
                                  o.data_ptr(), None, 1, 8, 1, 128, 128, 64, 1.0, 1, 0, 4, None, None, 0.0, None, 0,
                                  None)
     assert st == dn.DN_ERR_INVALID
+
+
+@pytest.mark.parametrize("activation", ["silu", "sigmoid"])
+@pytest.mark.parametrize("B,H,T", [(2, 3, 150), (1, 2, 64), (3, 32, 100), (4, 16, 1024)])
+def test_gdn_prologue_and_gated_norm(cuda_device, activation, B, H, T):
+    # dn_chunk_fwd_gdn_ex with z: the layer's prologue, the rule and the gated RMSNorm
+    # ("The full layer", steps 4-7) in the tensor-core kernels, against
+    # oracle.rms_norm_gated on the oracle recurrence's read-out (token-major y);
+    # 6 and 2 heads: the single launch; 96 heads: hosted WY groups; 64 heads, long
+    raw = _gdn_raw(B, H, T, seed=B * 7 + H + T, zero_rows=True)
+    gen = torch.Generator().manual_seed(T + H)
+    z = (2 * torch.randn(B, T, H, 128, generator=gen)).to(torch.bfloat16)
+    w = 1 + 0.5 * torch.randn(128, generator=gen)
+    d = to_dev(raw)
+    sc = 128 ** -0.5
+    y = torch.full((B, T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    S = torch.full((B, H, 128, 128), float("nan"), device="cuda")
+    dn.dn_chunk_fwd_gdn_ex(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], d["S0"], y, S,
+                           scale=sc, path="tc", z=z.cuda(), norm_weight=w.cuda(), eps=1e-6,
+                           norm_activation=activation)
+    dn.dn_device_status()
+    ro, rS = _gdn_oracle(raw, sc)
+    ry = oracle.rms_norm_gated(ro.transpose(0, 2, 1, 3), f64(z), f64(w), eps=1e-6, activation=activation)
+    assert_close(y.permute(0, 2, 1, 3), ry.transpose(0, 2, 1, 3), "bf16", "y")
+    assert_close(S, rS, "bf16", "S_T")
+
+
+def test_gdn_norm_needs_tensor_cores(cuda_device):
+    raw = _gdn_raw_d(1, 1, 8, 64, torch.float32, seed=2)
+    d = to_dev(raw)
+    y = torch.empty((1, 8, 1, 64), device="cuda")
+    with pytest.raises(dn.DNError) as ei:
+        dn.dn_chunk_fwd_gdn_ex(d["q"], d["k"], d["v"], d["b"], d["a"], d["A_log"], d["dt_bias"], None, y, None,
+                               path="simt", z=torch.zeros(1, 8, 1, 64, device="cuda"),
+                               norm_weight=torch.ones(64, device="cuda"))
+    assert ei.value.status == dn.DN_ERR_UNSUPPORTED
