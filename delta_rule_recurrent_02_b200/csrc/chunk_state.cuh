@@ -46,14 +46,23 @@ namespace state {
 using namespace sm100;
 using namespace tc;
 
-constexpr int kNT = 512;          // 16 warps
 constexpr int kSideWarp0 = 4;     // Qh / output warps 4..7
 constexpr int kSideThreads = 128;
-constexpr int kChainWarp0 = 8;    // state warps 8..15
-constexpr int kChainThreads = 256;
-static_assert(kSideThreads == (kChainWarp0 - kSideWarp0) * 32 && kChainThreads == kNT - kChainWarp0 * 32,
-              "named-barrier thread counts must match the warps of each role");
-// named barriers: 1 Qh / output warps, 2 state warps, kCtaBar all kNT threads
+constexpr int kChainWarp0 = 8;    // state warps 8 ..
+// Warps of the state pass: 8 warps of producer, MMA issue and Qh / output rows, then the
+// U and state epilogue warps, kNQ per TMEM lane quarter (each takes 1 / kNQ of a pass's
+// columns).  With the per-key gate the pass shares its CTA shape with the KDA WY groups
+// (16 warps), else it has 24.
+template <int GATE>
+struct Roles {
+    static constexpr int kChainWarps = GATE == kGatePerKey ? 8 : 16;
+    static constexpr int kNT = (kChainWarp0 + kChainWarps) * 32;
+    static constexpr int kChainThreads = kChainWarps * 32;
+    static constexpr int kNQ = kChainWarps / 4;
+};
+static_assert(kSideThreads == (kChainWarp0 - kSideWarp0) * 32, "named-barrier thread count of the side warps");
+constexpr int kMaxNT = Roles<kGateScalar>::kNT;
+// named barriers: 1 Qh / output warps, 2 state warps, kCtaBar all the pass's threads
 constexpr uint32_t kCtaBar = 3;
 
 // TMEM columns (32-bit, 128 lanes)
@@ -77,8 +86,7 @@ struct Layout {
     static constexpr int kOuBufs = HOSTED ? 1 : 2;
     static constexpr uint32_t TM_ST = TM_OU + 128 * kOuBufs;   // S^T bf16 pairs [dv][dk/2]
     static constexpr uint32_t TM_UT = TM_ST + 64;               // U^T bf16 pairs [dv][C/2]
-    static constexpr uint32_t TM_UK = TM_UT + 32;               // U~^T bf16 pairs [dv][C/2]
-    static constexpr uint32_t kCols = TM_UK + 32;
+    static constexpr uint32_t kCols = TM_UT + 32;
     static constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
     static constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
     static constexpr uint32_t STATE_BYTES = OFF_BAR + 256;
@@ -93,6 +101,7 @@ enum {
     B_WS = 10, B_KU, B_PU0, B_PU1,                       // MMA completions
     B_READY0, B_READY1, B_READY2, B_OFREE0, B_OFREE1,    // Qh / output warps -> MMA (Qh per stage)
     B_UTA, B_UTB, B_STA, B_STB,                          // state warps -> MMA (first / second half)
+    B_SC,                                                // state warps -> MMA: fp32 state rescaled
     B_COUNT
 };
 static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
@@ -138,6 +147,28 @@ struct Args {
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
 constexpr int G_KGAM = 0;
+
+// TMEM loads and stores of N consecutive 32-bit columns of the thread's lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&r)[N]) {
+    static_assert(N == 8 || N == 16 || N == 32, "column count");
+    if constexpr (N == 8) tmem_ld8(taddr, r);
+    else if constexpr (N == 16) tmem_ld16(taddr, r);
+    else tmem_ld32(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&u)[N]) {
+    static_assert(N == 4 || N == 8 || N == 16, "column count");
+    if constexpr (N == 4) tmem_st4(taddr, u);
+    else if constexpr (N == 8) tmem_st8(taddr, u);
+    else tmem_st16(taddr, u);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_f32(uint32_t taddr, const float (&v)[N]) {
+    static_assert(N == 16 || N == 32, "column count");
+    if constexpr (N == 16) tmem_st16(taddr, reinterpret_cast<const uint32_t(&)[16]>(v));
+    else tmem_st32(taddr, v);
+}
 
 // Output rows of chunk cp with the layer's gated RMSNorm, by the 128 output
 // threads (4 warps, thread j = value channel j = TMEM lane): per 8 positions,
@@ -223,7 +254,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
     using L = Layout<HOSTED>;
     constexpr int kStages = L::kStages;
     constexpr uint32_t OFF_GATE = L::OFF_GATE, OFF_BAR = L::OFF_BAR;
-    constexpr uint32_t TM_ST = L::TM_ST, TM_UT = L::TM_UT, TM_UK = L::TM_UK;
+    constexpr uint32_t TM_ST = L::TM_ST, TM_UT = L::TM_UT;
+    using R = Roles<GATE>;
+    constexpr int kNT = R::kNT, kChainThreads = R::kChainThreads, kNQ = R::kNQ;
     const CUtensorMap& tm_k = *ar.tm_k;
     const CUtensorMap& tm_q = *ar.tm_q;
     const CUtensorMap& tm_w = *ar.tm_w;
@@ -375,8 +408,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             const uint32_t I_SW = idesc_bf16(128, 128, 0, 0);       // [O|U] = S^T [Qh;-W]^T
             const uint32_t I_KU = idesc_bf16(128, 128, 0, 1);       // B MN-major
             const uint32_t I_PU = idesc_bf16(128, 64, 0, 0);
-            // A operand of KU: U~^T, or U^T itself with the per-key gate (K~ carries the decay)
-            const uint32_t TM_KU_A = GATE == kGatePerKey ? TM_UT : TM_UK;
             bool ok = true;
             for (int c = 0; ok && c < n; ++c) {
                 const uint32_t par = (uint32_t)c & 1u;
@@ -409,25 +440,23 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 for (int kk = 4; kk < 8; ++kk)
                     mma_bf16_ts(ou, tmem + TM_ST + kk * 8, dB + (uint64_t)(16384 / 16 + 2 * (kk & 3)), I_SW, 1);
                 mma_commit(ctl.bar(B_WS));
-                // S^T += U~^T K and O^T += U^T P^T, positions 0-31 then 32-63
-                ok = ctl.wait(B_UTA, par);
+                // S^T += U^T K~ (the decayed keys), positions 0-31 then 32-63, once the fp32
+                // state has been rescaled for this chunk; then O^T += U^T P^T, off the chain
+                ok = ctl.wait(B_UTA, par) && ctl.wait(B_SC, par);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_KU_A + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk)
-                    mma_bf16_ts(ou, tmem + TM_UT + kk * 8, dP + (uint64_t)(2 * kk), I_PU, 1);
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UT + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
                 ok = ctl.wait(B_UTB, par);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 2; kk < 4; ++kk)
-                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_KU_A + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
+                    mma_bf16_ts(tmem + TM_SACC, tmem + TM_UT + kk * 8, dK + (uint64_t)(128 * kk), I_KU, 1);
                 mma_commit(ctl.bar(B_KU));
 #pragma unroll
-                for (int kk = 2; kk < 4; ++kk)
+                for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(ou, tmem + TM_UT + kk * 8, dP + (uint64_t)(2 * kk), I_PU, 1);
                 mma_commit(ctl.bar(B_PU0 + (c & 1)));
                 mma_commit(ctl.bar(B_FREE0 + s));        // the stage's last reader is done
@@ -465,6 +494,22 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                     if (PRO)
                         ssq[u & 3] += e0.x * e0.x + e0.y * e0.y + e1.x * e1.x + e1.y * e1.y +
                                       e2.x * e2.x + e2.y * e2.y + e3.x * e3.x + e3.y * e3.y;
+                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                }
+                // ---- K~ = K (.) e^(G_last - G) in place over the k tile: each position's decay to
+                //      the chunk's end folded into its key, so that the KU product reads U itself
+                //      (no gate: the factor is 1; per-key gate: the workspace holds K~)
+#pragma unroll
+                for (int u = 0; u < (GATE == kGateScalar ? 8 : 0); ++u) {
+                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
+                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                    const uint32_t a = st + ST_K + blk * 8192 + sw128_off(i, ch);
+                    const float f = gs[G_ET + i];
+                    const uint4 w = ld_shared_v4(a);
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
                     st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
                                  pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                 }
@@ -514,54 +559,56 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             }
         }
     } else if (warp >= kChainWarp0) {
-        // ================= U and the state (256 threads) ===========================
+        // ================= U and the state (kChainThreads threads) =================
+        // kNQ warps per TMEM lane quarter; each pass splits its columns among them
+        constexpr int SCOLS = 64 / kNQ;              // d_k columns of a state pass, per thread
+        constexpr int UPOS = 32 / kNQ;               // positions of a U pass, per thread
         const int q = warp & 3;
-        const int hc = (warp - kChainWarp0) >> 2;    // which half of each pass
+        const int hc = (warp - kChainWarp0) >> 2;    // which part of each pass
         const int j = (q << 5) + lane;               // value channel = TMEM lane
         const uint32_t lane_off = (uint32_t)(q << 5) << 16;
         bool ok = ctl.wait(B_GATE0, 0);
-        if (!ok) *abort_flag = 1;
-        ok = !named_bar_any(2, kChainThreads, !ok);
         if (ok) {
-            // S0 -> TMEM: fp32 pre-scaled by chunk 0's decay, and its bf16 copy
+            // S0 -> TMEM: its bf16 copy (which the first products read; signalled at once),
+            // then the fp32 accumulator pre-scaled by chunk 0's decay
             const float gamma0 = GATE == kGatePerKey ? 0.f : gates[G_GAMMA];
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
-                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
-                float v[32];
+                const int c0 = 64 * p + SCOLS * hc;      // d_k columns c0 .. c0 + SCOLS - 1
+                float v[SCOLS];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = S0 ? S0[(bh * kD + pc * 32 + e) * kD + j] : 0.f;
-                uint32_t pk[16];
+                for (int e = 0; e < SCOLS; ++e) v[e] = S0 ? S0[(bh * kD + c0 + e) * kD + j] : 0.f;
+                uint32_t pk[SCOLS / 2];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    v[e] *= GATE == kGatePerKey ? gates[G_KGAM + pc * 32 + e] : gamma0;
-                tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+                for (int e = 0; e < SCOLS / 2; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st_cols(tmem + lane_off + TM_ST + c0 / 2, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
+#pragma unroll
+                for (int e = 0; e < SCOLS; ++e) v[e] *= GATE == kGatePerKey ? gates[G_KGAM + c0 + e] : gamma0;
+                tmem_st_f32(tmem + lane_off + TM_SACC + c0, v);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_SC));
         }
         for (int c = 0; ok && c < n; ++c) {
             const uint32_t par = (uint32_t)c & 1u;
             const uint32_t st = sb + (c % kStages) * SZ_STAGE;
-            // ---- U = u - W S -> bf16 pairs in TMEM, plain and decayed (U~), in two passes
-            //      over positions 0-31 and 32-63 ------------------------------------------
+            // ---- U = u - W S -> bf16 pairs in TMEM, in two passes over positions 0-31 and
+            //      32-63 (the KU product reads U itself: the decays are in K~) -------------
             ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            if (!ok) break;
             tc_fence_after();
-            const float* gsc = gates + (c & 3) * GATE_FLOATS;
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
-                const int i0 = 32 * p + 16 * hc;         // positions i0 .. i0 + 15
-                float v[16];
-                tmem_ld16(tmem + lane_off + TM_OU + (c % L::kOuBufs) * 128 + 64 + i0, v);
+                const int i0 = 32 * p + UPOS * hc;       // positions i0 .. i0 + UPOS - 1
+                float v[UPOS];
+                tmem_ld_cols(tmem + lane_off + TM_OU + (c % L::kOuBufs) * 128 + 64 + i0, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
+                for (int ch = 0; ch < UPOS / 8; ++ch) {
                     const uint4 w = ld_shared_v4(st + ST_UT + sw128_off(j, (i0 >> 3) + ch));
                     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
@@ -571,30 +618,20 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                         v[8 * ch + 2 * e + 1] += f.y;
                     }
                 }
-                uint32_t pk[8];
+                uint32_t pk[UPOS / 2];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                tmem_st8(tmem + lane_off + TM_UT + (i0 >> 1), pk);
-                if (GATE != kGatePerKey) {
-                    // U~ = U (.) e^(G_last - G) by rows; with the per-key gate K~ carries the
-                    // decay and the KU product reads U^T itself
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        float4 et = *reinterpret_cast<const float4*>(gsc + G_ET + i0 + 4 * q4);
-                        pk[2 * q4] = pack_bf16x2(v[4 * q4 + 0] * et.x, v[4 * q4 + 1] * et.y);
-                        pk[2 * q4 + 1] = pack_bf16x2(v[4 * q4 + 2] * et.z, v[4 * q4 + 3] * et.w);
-                    }
-                    tmem_st8(tmem + lane_off + TM_UK + (i0 >> 1), pk);
-                }
+                for (int e = 0; e < UPOS / 2; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                tmem_st_cols(tmem + lane_off + TM_UT + (i0 >> 1), pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
             }
             // ---- state: S_{c+1} = gamma_c S_c + dS (already summed in TMEM), in two passes
-            //      over d_k 0-63 and 64-127 ---------------------------------------------------
+            //      over d_k 0-63 and 64-127: the bf16 copy first (the next chunk's first
+            //      products wait for it), then the fp32 accumulator pre-scaled by the next
+            //      chunk's decay (the next KU product waits for that) ---------------------
             ok = ctl.wait(B_KU, par) && (c + 1 >= n || ctl.wait(B_GATE0 + ((c + 1) & 3), (uint32_t)((c + 1) >> 2) & 1u));
-            if (!ok) *abort_flag = 1;
-            if (named_bar_any(2, kChainThreads, !ok)) { ok = false; break; }
+            if (!ok) break;
             tc_fence_after();
             const bool last = c + 1 == n;
             const float* gsn = gates + ((c + 1) & 3) * GATE_FLOATS;
@@ -605,32 +642,37 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             const float gnext = last || GATE == kGatePerKey ? 1.f : gsn[G_GAMMA];
 #pragma unroll 1
             for (int p = 0; p < 2; ++p) {
-                const int pc = 2 * p + hc;               // d_k columns 32 pc .. 32 pc + 31
-                float v[32];
-                tmem_ld32(tmem + lane_off + TM_SACC + pc * 32, v);
+                const int c0 = 64 * p + SCOLS * hc;      // d_k columns c0 .. c0 + SCOLS - 1
+                float v[SCOLS];
+                tmem_ld_cols(tmem + lane_off + TM_SACC + c0, v);
                 tmem_wait_ld();
                 if (snap) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) snap_out[(pc * 32 + e) * kD] = v[e];
+                    for (int e = 0; e < SCOLS; ++e) snap_out[(c0 + e) * kD] = v[e];
                 }
                 if (last) {
                     if (S_T) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) S_T[(bh * kD + pc * 32 + e) * kD + j] = v[e];
+                        for (int e = 0; e < SCOLS; ++e) S_T[(bh * kD + c0 + e) * kD + j] = v[e];
                     }
                 } else {
-                    uint32_t pk[16];
+                    uint32_t pk[SCOLS / 2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                    tmem_st16(tmem + lane_off + TM_ST + pc * 16, pk);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= GATE == kGatePerKey ? gsn[G_KGAM + pc * 32 + e] : gnext;
-                    tmem_st32(tmem + lane_off + TM_SACC + pc * 32, v);
+                    for (int e = 0; e < SCOLS / 2; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+                    tmem_st_cols(tmem + lane_off + TM_ST + c0 / 2, pk);
                     tmem_wait_st();
                 }
                 tc_fence_before();
                 mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
+                if (!last) {
+#pragma unroll
+                    for (int e = 0; e < SCOLS; ++e) v[e] *= GATE == kGatePerKey ? gsn[G_KGAM + c0 + e] : gnext;
+                    tmem_st_f32(tmem + lane_off + TM_SACC + c0, v);
+                }
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_SC));
         }
         if (!ok) *abort_flag = 1;
     }
