@@ -377,6 +377,141 @@ def measure_gdn_prologue(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
             "traffic": None, "timing": f"median of {calls} calls after {warm}, CUDA events"}
 
 
+def _time_calls(torch, call, stream, calls, warm):
+    for _ in range(warm):
+        call()
+    ts = []
+    for _ in range(calls):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def measure_next_rows(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
+    """The entry points beyond the bench step, each on a synthetic workload of
+    the layer's shapes, CUDA-event timed (median of `calls` after `warm`):
+    grouped value heads (16 key : 48 value heads), a packed batch of ragged
+    sequences, the layer with its prologue and gated RMSNorm fused into the
+    prefill and into the decode step, and the generalised (RWKV-7) rule."""
+    out = {}
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    gen = torch.Generator().manual_seed(11)
+    unit = lambda x: x / x.norm(dim=-1, keepdim=True)
+    d, T, sc = 128, 4096, 128 ** -0.5
+
+    def entry(name, ms, tokens, fl, by, path, bound="hbm"):
+        e = {"ms_per_call": ms, "tokens_per_s": tokens / (ms * 1e-3), "path": path, "algorithmic_bytes": by,
+             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac": by / (ms * 1e-3) / 1e9 / hbm, "bound": bound,
+             "timing": f"median of {calls} calls after {warm}, CUDA events"}
+        if fl:
+            e.update({"counted_flops": fl, "tensor_tflops": fl / (ms * 1e-3) / 1e12,
+                      "tensor_frac": fl / (ms * 1e-3) / 1e12 / tc})
+        out[name] = e
+
+    # grouped value heads: 16 key heads serve 48 value heads
+    Hk, Hv = 16, 48
+    q = unit(torch.randn(1, Hk, T, d, generator=gen)).to(torch.bfloat16).to(dev)
+    k = unit(torch.randn(1, Hk, T, d, generator=gen)).to(torch.bfloat16).to(dev)
+    v = torch.randn(1, Hv, T, d, generator=gen).to(torch.bfloat16).to(dev)
+    beta = torch.sigmoid(torch.randn(1, Hv, T, generator=gen)).to(dev)
+    g = (-torch.nn.functional.softplus(torch.randn(1, Hv, T, generator=gen) + 2)).to(dev)
+    o = torch.empty((1, Hv, T, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((1, Hv, d, d), device=dev)
+    ws = torch.empty(dn.dn_chunk_fwd_workspace_size(1, T, Hv, d, d), dtype=torch.uint8, device=dev)
+    ms = _time_calls(torch, lambda: dn.dn_chunk_fwd_gva(q, k, v, beta, g, None, o, S, scale=sc, workspace=ws,
+                                                        stream=stream), stream, calls, warm)
+    by = Hk * T * d * 2 * 2 + Hv * T * (d * 2 * 2 + 8) + Hv * d * d * 4
+    entry("gva_bf16_B1_Hk16_Hv48_T4096_d128", ms, T, prefill_flops(1, Hv, T, d, d), by,
+          "tensor cores, q and k read once per key head")
+    del q, k, v, beta, g, o, S, ws
+
+    # a packed batch: 8 ragged sequences, 16384 tokens in all, 16 heads
+    lens = [4096, 1000, 3000, 64, 1, 4095, 2048, 2080]
+    Tt, H, N = sum(lens), 16, len(lens)
+    q = unit(torch.randn(1, H, Tt, d, generator=gen)).to(torch.bfloat16).to(dev)
+    k = unit(torch.randn(1, H, Tt, d, generator=gen)).to(torch.bfloat16).to(dev)
+    v = torch.randn(1, H, Tt, d, generator=gen).to(torch.bfloat16).to(dev)
+    beta = torch.sigmoid(torch.randn(1, H, Tt, generator=gen)).to(dev)
+    g = (-torch.nn.functional.softplus(torch.randn(1, H, Tt, generator=gen) + 2)).to(dev)
+    cu = torch.tensor([0] + [sum(lens[:i + 1]) for i in range(N)], dtype=torch.int32, device=dev)
+    o = torch.empty((1, H, Tt, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((N, H, d, d), device=dev)
+    ws = torch.empty(dn.dn_chunk_fwd_varlen_workspace_size(N, Tt, H, d, d), dtype=torch.uint8, device=dev)
+    ms = _time_calls(torch, lambda: dn.dn_chunk_fwd_varlen(q, k, v, beta, g, None, o, S, cu, scale=sc, workspace=ws,
+                                                           stream=stream), stream, calls, warm)
+    fl = sum(prefill_flops(1, H, L, d, d) for L in lens if L)
+    by = prefill_bytes(1, H, Tt, d, d, st=False) + N * H * d * d * 4 + (N + 1) * 4
+    entry("varlen_bf16_N8_T16384_H16_d128", ms, Tt, fl, by, "tensor cores: chunk tables, WY kernel, state pass")
+    del q, k, v, beta, g, o, S, ws, cu
+
+    # the layer's prologue, the rule and the gated RMSNorm in one prefill (bench prefill shape)
+    pc = W.GDN_PREFILL
+    B, H = pc.B, pc.H
+    q = (torch.randn(B, H, T, d, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    k = (torch.randn(B, H, T, d, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, H, T, d, generator=gen).to(torch.bfloat16).to(dev)
+    b = torch.randn(B, H, T, generator=gen).to(dev)
+    a = torch.randn(B, H, T, generator=gen).to(dev)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen)).to(dev)
+    dt_bias = torch.randn(H, generator=gen).to(dev)
+    z = torch.randn(B, T, H, d, generator=gen).to(torch.bfloat16).to(dev)
+    nw = torch.ones(d, device=dev)
+    y = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, H, d, d), device=dev)
+    ws = torch.empty(dn.dn_chunk_fwd_workspace_size(B, T, H, d, d, path="tc"), dtype=torch.uint8, device=dev)
+    ms = _time_calls(torch, lambda: dn.dn_chunk_fwd_gdn_ex(q, k, v, b, a, A_log, dt_bias, None, y, S, scale=sc,
+                                                           path="tc", z=z, norm_weight=nw, workspace=ws,
+                                                           stream=stream), stream, calls, warm)
+    by = prefill_bytes(B, H, T, d, d) + B * H * T * d * 2 + d * 4 + 2 * H * 4
+    entry("gdn_layer_prologue_norm_bf16_B4_H16_T4096_d128", ms, B * T, prefill_flops(B, H, T, d, d), by,
+          "tensor cores, prologue and gated RMSNorm fused")
+    del q, k, v, b, a, z, y, S, ws
+
+    # the decode step with the prologue and the gated RMSNorm (decode workload shape)
+    dc = W.DECODE
+    B, H = dc.B, dc.H
+    q = (torch.randn(B, H, d, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    k = (torch.randn(B, H, d, generator=gen) * 2).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, H, d, generator=gen).to(torch.bfloat16).to(dev)
+    b = torch.randn(B, H, generator=gen).to(dev)
+    a = torch.randn(B, H, generator=gen).to(dev)
+    A_log = torch.log(1 + 15 * torch.rand(H, generator=gen)).to(dev)
+    dt_bias = torch.randn(H, generator=gen).to(dev)
+    z = torch.randn(B, H, d, generator=gen).to(torch.bfloat16).to(dev)
+    Sd = (0.1 * torch.randn(B, H, d, d, generator=gen)).to(dev)
+    y = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+    ms = _time_calls(torch, lambda: dn.dn_decode_step_gdn_ex(q, k, v, b, a, A_log, dt_bias, Sd, y, scale=sc, z=z,
+                                                             norm_weight=nw, stream=stream), stream, calls, warm)
+    by = decode_bytes(B, H, d, d) + B * H * d * 2 + d * 4
+    entry("decode_step_prologue_norm_bf16_B256_H32_d128", ms, B, None, by,
+          "one CTA per head; prologue and gated RMSNorm fused")
+    del q, k, v, b, a, z, Sd, y
+
+    # the generalised (RWKV-7) rule: fp32 arithmetic on CUDA cores
+    B, H, Tg = 1, 8, 2048
+    q = torch.randn(B, H, Tg, d, generator=gen).to(torch.bfloat16).to(dev)
+    wl = (-torch.exp(torch.randn(B, H, Tg, d, generator=gen) - 2)).to(dev)
+    kp = unit(torch.randn(B, H, Tg, d, generator=gen)).to(torch.bfloat16).to(dev)
+    ar = torch.sigmoid(torch.randn(B, H, Tg, d, generator=gen)).to(dev)
+    kw = (torch.randn(B, H, Tg, d, generator=gen) / d ** 0.5).to(torch.bfloat16).to(dev)
+    v = torch.randn(B, H, Tg, d, generator=gen).to(torch.bfloat16).to(dev)
+    o = torch.empty((B, H, Tg, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, H, d, d), device=dev)
+    ms = _time_calls(torch, lambda: dn.dn_chunk_fwd_general(q, wl, kp, ar, kw, v, None, o, S, chunk=32, scale=sc,
+                                                            stream=stream), stream, 3, 1)
+    by = B * H * Tg * (d * 2 * 4 + d * 4 * 2) + B * H * d * d * 4
+    entry("general_rule_bf16_B1_H8_T2048_d128", ms, B * Tg, None, by,
+          "fp32 on CUDA cores, chunk 32 (per-channel decays exact per pair)", bound="alu")
+    del q, wl, kp, ar, kw, v, o, S
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_layer_ops(dn, torch, W, peaks, dev, stream, calls=5, warm=2):
     """The layer steps on either side of the rule at the bench prefill's shape
     (B=4, T=4096, 16 heads of 128), bf16, each against the HBM roofline:
@@ -467,7 +602,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip timing the other prefill workloads (small DeltaNet, long GDN, KDA)")
-    ap.add_argument("--profile-case", choices=["prefill", "decode", "kda"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "kda", "layer_ops"], default=None,
                     help="launch one kernel of the step a few times without timing (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -592,6 +727,7 @@ def main():
     if world == 1 and not args.no_configs:
         line["other_prefill_workloads"] = measure_prefill_configs(dn, torch, W, peaks, dev, stream)
         line["layer_ops"] = measure_layer_ops(dn, torch, W, peaks, dev, stream)
+        line["next_rows"] = measure_next_rows(dn, torch, W, peaks, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         reps = [oracle_sample_rate(seed_offset=r) for r in range(4)]
@@ -626,6 +762,29 @@ def run_profile_case(args):
         for _ in range(args.warmup + args.steps):
             dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o, S_T, chunk=pc.chunk,
                             scale=pc.scale, path=args.path, workspace=ws)
+    elif args.profile_case == "layer_ops":
+        # the layer's conv (q, k, v slices of one projection row) and gated norm at the
+        # bench prefill's shape: 3 conv launches and 1 norm launch per repetition
+        pc = W.GDN_PREFILL
+        B, H, T, d, K = pc.B, pc.H, pc.T, pc.dk, 4
+        C3 = 3 * H * d
+        gen = torch.Generator().manual_seed(pc.seed + 1)
+        proj = torch.randn(B, T, C3, generator=gen).to(torch.bfloat16).to(dev)
+        w = (torch.randn(C3, K, generator=gen) * 0.5).to(dev)
+        w_parts = [w[i * H * d:(i + 1) * H * d].contiguous() for i in range(3)]
+        s_in = torch.randn(B, K - 1, C3, generator=gen).to(torch.bfloat16).to(dev)
+        s_parts = [s_in[:, :, i * H * d:(i + 1) * H * d].contiguous() for i in range(3)]
+        s_outs = [torch.empty_like(sp) for sp in s_parts]
+        ys = [torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        o = torch.randn(B, H, T, d, generator=gen).to(torch.bfloat16).to(dev)
+        z = torch.randn(B, T, H, d, generator=gen).to(torch.bfloat16).to(dev)
+        nw = torch.ones(d, device=dev)
+        y = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+        for _ in range(args.warmup + args.steps):
+            for i in range(3):
+                dn.dn_causal_conv1d(proj[:, :, i * H * d:(i + 1) * H * d], w_parts[i], ys[i], s_parts[i],
+                                    s_outs[i], head_dim=d)
+            dn.dn_rms_norm_gated(o, z, nw, y)
     else:
         dc = W.DECODE
         D = {k: (None if v is None else v.to(dev)) for k, v in W.gen_decode(dc).items()}

@@ -53,16 +53,20 @@ constexpr int kChainWarp0 = 8;    // state warps 8 ..
 // U and state epilogue warps, kNQ per TMEM lane quarter (each takes 1 / kNQ of a pass's
 // columns).  With the per-key gate the pass shares its CTA shape with the KDA WY groups
 // (16 warps), else it has 24.
-template <int GATE>
+// On the plain path (no prologue) of a state pass alone on its SM, four more warps
+// write the output rows, so that the side warps only transform stages and run ahead.
+template <int GATE, bool HOSTED = false, int PRO = 0>
 struct Roles {
     static constexpr int kChainWarps = GATE == kGatePerKey ? 8 : 16;
-    static constexpr int kNT = (kChainWarp0 + kChainWarps) * 32;
+    static constexpr bool kSplitOut = !HOSTED && PRO == 0 && GATE != kGatePerKey;
+    static constexpr int kOutWarp0 = kChainWarp0 + kChainWarps;     // output warps (kSplitOut)
+    static constexpr int kNT = (kChainWarp0 + kChainWarps + (kSplitOut ? 4 : 0)) * 32;
     static constexpr int kChainThreads = kChainWarps * 32;
     static constexpr int kNQ = kChainWarps / 4;
 };
 static_assert(kSideThreads == (kChainWarp0 - kSideWarp0) * 32, "named-barrier thread count of the side warps");
-constexpr int kMaxNT = Roles<kGateScalar>::kNT;
-// named barriers: 1 Qh / output warps, 2 state warps, kCtaBar all the pass's threads
+constexpr int kHostedNT = Roles<kGateScalar, true>::kNT;   // 24 warps: with a hosted WY group, 32
+// named barriers: 1 Qh / output warps, 5 output warps (split), kCtaBar all the pass's threads
 constexpr uint32_t kCtaBar = 3;
 
 // TMEM columns (32-bit, 128 lanes)
@@ -185,14 +189,22 @@ __device__ __forceinline__ void norm_rows(const Args& ar, uint32_t oc, float* gs
     const int64_t rstride = (int64_t)ar.H * kD;
     const float wj = ar.norm_w[j];
     const bool silu = ar.norm == 1;
+    // z of the first 8 positions; each step then requests the next step's z before its own work
+    __nv_bfloat16 zn[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zn[e] = e < Cc ? ar.z[row0 * kD + (int64_t)e * rstride + j] : __float2bfloat16(0.f);
 #pragma unroll 1
     for (int it = 0; it < 8; ++it) {
         float* red = gsp + G_RK + (it & 1) * 32;      // [8 positions][4 warps]
         float zf[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * it + e;
-            zf[e] = i < Cc ? __bfloat162float(ar.z[row0 * kD + (int64_t)i * rstride + j]) : 0.f;
+        for (int e = 0; e < 8; ++e) zf[e] = __bfloat162float(zn[e]);
+        if (it + 1 < 8) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i = 8 * (it + 1) + e;
+                zn[e] = i < Cc ? ar.z[row0 * kD + (int64_t)i * rstride + j] : __float2bfloat16(0.f);
+            }
         }
         float v[8];
         {
@@ -255,8 +267,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
     constexpr int kStages = L::kStages;
     constexpr uint32_t OFF_GATE = L::OFF_GATE, OFF_BAR = L::OFF_BAR;
     constexpr uint32_t TM_ST = L::TM_ST, TM_UT = L::TM_UT;
-    using R = Roles<GATE>;
+    using R = Roles<GATE, HOSTED, PRO>;
     constexpr int kNT = R::kNT, kChainThreads = R::kChainThreads, kNQ = R::kNQ;
+    constexpr bool kSplitOut = R::kSplitOut;
     const CUtensorMap& tm_k = *ar.tm_k;
     const CUtensorMap& tm_q = *ar.tm_q;
     const CUtensorMap& tm_w = *ar.tm_w;
@@ -395,6 +408,14 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
                 tma_load_2d(st + ST_P, &tm_p, 0, (int)(tile * kC), fb);
             }
+            if (PRO == 2 && !(test_flags & 1)) {
+                // the gated norm's z rows of this chunk into L2 (64 rows of 256 bytes, H d_v
+                // elements apart), so that the output warps' loads of them hit L2
+                const int64_t b = bh / ar.H, h = bh % ar.H;
+                const int Cn = min(kC, len - cc * kC);
+                for (int i = lane; i < Cn; i += 32)
+                    bulk_prefetch_l2(ar.z + (((b * T + (int64_t)cc * kC + i) * ar.H + h) * kD), kD * 2);
+            }
             if (!(test_flags & 1)) issued = cc + 1;
         }
         if (*abort_flag && lane == 0) {
@@ -528,7 +549,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                     }
                 }
             }
-            if (c >= 1) {
+            if (!kSplitOut && c >= 1) {
                 // ---- output rows of chunk c - 1 --------------------------------------------
                 const int cp = c - 1;
                 const int Cc = min(kC, len - cp * kC);
@@ -557,6 +578,32 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tc_fence_before();
                 mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
             }
+        }
+    } else if (kSplitOut && warp >= R::kOutWarp0) {
+        // ================= output rows of each chunk (128 threads, plain path) ==========
+        const int q = warp & 3;                    // TMEM lane quarter
+        const int j = (q << 5) + lane;             // value channel = TMEM lane
+        for (int cp = 0; cp < n; ++cp) {
+            const int Cc = min(kC, len - cp * kC);
+            bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
+            if (!ok) *abort_flag = 1;
+            if (named_bar_any(5, kSideThreads, !ok)) break;
+            tc_fence_after();
+            __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
+            const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                tmem_ld32(oc + hh * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = hh * 32 + e;
+                    if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
         }
     } else if (warp >= kChainWarp0) {
         // ================= U and the state (kChainThreads threads) =================
@@ -601,30 +648,35 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             ok = ctl.wait(B_WS, par) && ctl.wait(B_FULL0 + c % kStages, (uint32_t)(c / kStages) & 1u);
             if (!ok) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const int i0 = 32 * p + UPOS * hc;       // positions i0 .. i0 + UPOS - 1
-                float v[UPOS];
-                tmem_ld_cols(tmem + lane_off + TM_OU + (c % L::kOuBufs) * 128 + 64 + i0, v);
+            {
+                // both halves' columns requested at once: the second half waits no second latency
+                float v[2][UPOS];
+                const uint32_t ub = tmem + lane_off + TM_OU + (c % L::kOuBufs) * 128 + 64 + UPOS * hc;
+                tmem_ld_cols(ub, v[0]);
+                tmem_ld_cols(ub + 32, v[1]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int ch = 0; ch < UPOS / 8; ++ch) {
-                    const uint4 w = ld_shared_v4(st + ST_UT + sw128_off(j, (i0 >> 3) + ch));
-                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+                for (int p = 0; p < 2; ++p) {
+                    const int i0 = 32 * p + UPOS * hc;   // positions i0 .. i0 + UPOS - 1
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(h2[e]);
-                        v[8 * ch + 2 * e] += f.x;
-                        v[8 * ch + 2 * e + 1] += f.y;
+                    for (int ch = 0; ch < UPOS / 8; ++ch) {
+                        const uint4 w = ld_shared_v4(st + ST_UT + sw128_off(j, (i0 >> 3) + ch));
+                        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h2[e]);
+                            v[p][8 * ch + 2 * e] += f.x;
+                            v[p][8 * ch + 2 * e + 1] += f.y;
+                        }
                     }
-                }
-                uint32_t pk[UPOS / 2];
+                    uint32_t pk[UPOS / 2];
 #pragma unroll
-                for (int e = 0; e < UPOS / 2; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                tmem_st_cols(tmem + lane_off + TM_UT + (i0 >> 1), pk);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
+                    for (int e = 0; e < UPOS / 2; ++e) pk[e] = pack_bf16x2(v[p][2 * e], v[p][2 * e + 1]);
+                    tmem_st_cols(tmem + lane_off + TM_UT + (i0 >> 1), pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(ctl.bar(p == 0 ? B_UTA : B_UTB));
+                }
             }
             // ---- state: S_{c+1} = gamma_c S_c + dS (already summed in TMEM), in two passes
             //      over d_k 0-63 and 64-127: the bf16 copy first (the next chunk's first
@@ -640,34 +692,45 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             float* snap_out = snap ? ar.snaps + ((bh * ar.n_snap + (c + 1) / ar.snap_every - 1) * kD) * kD + j
                                    : nullptr;
             const float gnext = last || GATE == kGatePerKey ? 1.f : gsn[G_GAMMA];
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                const int c0 = 64 * p + SCOLS * hc;      // d_k columns c0 .. c0 + SCOLS - 1
-                float v[SCOLS];
-                tmem_ld_cols(tmem + lane_off + TM_SACC + c0, v);
+            {
+                // both halves' columns requested at once; the bf16 copies first (each half
+                // signalled as soon as it is stored), the fp32 rescale after both
+                float v[2][SCOLS];
+                const uint32_t sa = tmem + lane_off + TM_SACC + SCOLS * hc;
+                tmem_ld_cols(sa, v[0]);
+                tmem_ld_cols(sa + 64, v[1]);
                 tmem_wait_ld();
-                if (snap) {
 #pragma unroll
-                    for (int e = 0; e < SCOLS; ++e) snap_out[(c0 + e) * kD] = v[e];
-                }
-                if (last) {
-                    if (S_T) {
+                for (int p = 0; p < 2; ++p) {
+                    const int c0 = 64 * p + SCOLS * hc;  // d_k columns c0 .. c0 + SCOLS - 1
+                    if (snap) {
 #pragma unroll
-                        for (int e = 0; e < SCOLS; ++e) S_T[(bh * kD + c0 + e) * kD + j] = v[e];
+                        for (int e = 0; e < SCOLS; ++e) snap_out[(c0 + e) * kD] = v[p][e];
                     }
-                } else {
-                    uint32_t pk[SCOLS / 2];
+                    if (last) {
+                        if (S_T) {
 #pragma unroll
-                    for (int e = 0; e < SCOLS / 2; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-                    tmem_st_cols(tmem + lane_off + TM_ST + c0 / 2, pk);
-                    tmem_wait_st();
+                            for (int e = 0; e < SCOLS; ++e) S_T[(bh * kD + c0 + e) * kD + j] = v[p][e];
+                        }
+                    } else {
+                        uint32_t pk[SCOLS / 2];
+#pragma unroll
+                        for (int e = 0; e < SCOLS / 2; ++e) pk[e] = pack_bf16x2(v[p][2 * e], v[p][2 * e + 1]);
+                        tmem_st_cols(tmem + lane_off + TM_ST + c0 / 2, pk);
+                        tmem_wait_st();
+                    }
+                    tc_fence_before();
+                    mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
                 }
-                tc_fence_before();
-                mbar_arrive(ctl.bar(p == 0 ? B_STA : B_STB));
                 if (!last) {
 #pragma unroll
-                    for (int e = 0; e < SCOLS; ++e) v[e] *= GATE == kGatePerKey ? gsn[G_KGAM + c0 + e] : gnext;
-                    tmem_st_f32(tmem + lane_off + TM_SACC + c0, v);
+                    for (int p = 0; p < 2; ++p) {
+                        const int c0 = 64 * p + SCOLS * hc;
+#pragma unroll
+                        for (int e = 0; e < SCOLS; ++e)
+                            v[p][e] *= GATE == kGatePerKey ? gsn[G_KGAM + c0 + e] : gnext;
+                        tmem_st_f32(sa + 64 * p, v[p]);
+                    }
                 }
             }
             tmem_wait_st();

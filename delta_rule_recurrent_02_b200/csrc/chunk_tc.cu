@@ -28,7 +28,7 @@ using namespace sm100;
 using namespace tc;
 
 template <int GATE, int PRO>
-__global__ void __launch_bounds__(state::Roles<GATE>::kNT, 1)
+__global__ void __launch_bounds__(state::Roles<GATE, false, PRO>::kNT, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
                    const __grid_constant__ CUtensorMap tm_p, const unsigned int* __restrict__ flags,
@@ -105,7 +105,8 @@ varlen_table_kernel(const int* __restrict__ cu_in, int N, int T, int* tables, un
 
 namespace {
 constexpr int kFusedThreads = 4 * wy::kNT;          // 32 warps: 4 WY groups, or the state pass + up to 16 more
-static_assert(state::kMaxNT + wy::kNT <= kFusedThreads, "fused CTA size");
+static_assert(state::kHostedNT + wy::kNT <= kFusedThreads && state::Roles<kGateScalar>::kNT <= kFusedThreads,
+              "fused CTA size");
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 // a hosted WY group's shared memory starts past the hosted state pass's
 constexpr uint32_t kHostedWyOff = align1k(state::Layout<true>::STATE_BYTES);
@@ -140,12 +141,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                              pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps};
         if (!HOSTED) {
             // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
-            if (warp >= state::Roles<GATE>::kNT / 32) return;
+            if (warp >= state::Roles<GATE, false, PRO>::kNT / 32) return;
             state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
             return;
         }
         // ---- state pass (warps 0-15) and one WY group (warps 16-23) ------------------------
-        constexpr int kStateNT = state::Roles<GATE>::kNT;
+        constexpr int kStateNT = state::Roles<GATE, true, PRO>::kNT;
         constexpr int kHostThreads = kStateNT + wy::kNT;
         if (tid >= kHostThreads) return;
         uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kHostedWyOff + wy::GROUP_BYTES - 16);
@@ -322,7 +323,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         const uint32_t bytes = state::Layout<false>::STATE_BYTES + 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return e;
-        kern<<<(unsigned)(a.N * a.H), state::Roles<GATE>::kNT, bytes, st>>>(
+        kern<<<(unsigned)(a.N * a.H), state::Roles<GATE, false, PRO>::kNT, bytes, st>>>(
             m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0, static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
             a.scale, a.status, a.test_flags, nullptr, nullptr, 1, 0,
             prologue_of(a), vl, a.N);
@@ -375,7 +376,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     // the WY kernel has finished before this launch starts: no flags to wait for
-    kern<<<(unsigned)BH, state::Roles<GATE>::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
+    kern<<<(unsigned)BH, state::Roles<GATE, false, PRO>::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
                                                   a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap,
                                                   prologue_of(a),
