@@ -53,14 +53,17 @@ constexpr int kChainWarp0 = 8;    // state warps 8 ..
 // U and state epilogue warps, kNQ per TMEM lane quarter (each takes 1 / kNQ of a pass's
 // columns).  With the per-key gate the pass shares its CTA shape with the KDA WY groups
 // (16 warps), else it has 24.
-// On the plain path (no prologue) of a state pass alone on its SM, four more warps
-// write the output rows, so that the side warps only transform stages and run ahead.
+// Alone on its SM (and without the per-key gate) a state pass has warps of its own that
+// write the output rows (four; eight with the gated norm), so that the side warps only
+// transform stages and run ahead.
 template <int GATE, bool HOSTED = false, int PRO = 0>
 struct Roles {
     static constexpr int kChainWarps = GATE == kGatePerKey ? 8 : 16;
-    static constexpr bool kSplitOut = !HOSTED && PRO == 0 && GATE != kGatePerKey;
+    static constexpr bool kSplitOut = !HOSTED && GATE != kGatePerKey;
     static constexpr int kOutWarp0 = kChainWarp0 + kChainWarps;     // output warps (kSplitOut)
-    static constexpr int kNT = (kChainWarp0 + kChainWarps + (kSplitOut ? 4 : 0)) * 32;
+    static constexpr int kOutWarps = kSplitOut ? (PRO == 2 ? 8 : 4) : 0;
+    static constexpr int kOutThreads = kSplitOut ? kOutWarps * 32 : kSideThreads;   // who writes the rows
+    static constexpr int kNT = (kChainWarp0 + kChainWarps + kOutWarps) * 32;
     static constexpr int kChainThreads = kChainWarps * 32;
     static constexpr int kNQ = kChainWarps / 4;
 };
@@ -83,15 +86,21 @@ constexpr uint32_t ST_P = 65536;        //   P [64 rows (i)][128 B (j)]         
 
 // Two layouts: alone on its SM (three stages, two [O|U] buffers, all 512 TMEM
 // columns), or hosting a WY group (two stages, one [O|U] buffer, 384 columns;
-// the group gets the other 128 and the shared memory past STATE_BYTES).
-template <bool HOSTED>
+// the group gets the other 128 and the shared memory past STATE_BYTES).  ZB
+// (the gated norm on the output rows, alone on its SM): two stages, and in the
+// room of the third z of two chunks and one chunk's output rows in fp32.
+template <bool HOSTED, bool ZB = false>
 struct Layout {
-    static constexpr int kStages = HOSTED ? 2 : 3;
+    static_assert(!(HOSTED && ZB), "the gated norm runs on a state pass alone on its SM");
+    static constexpr int kStages = HOSTED || ZB ? 2 : 3;
     static constexpr int kOuBufs = HOSTED ? 1 : 2;
     static constexpr uint32_t TM_ST = TM_OU + 128 * kOuBufs;   // S^T bf16 pairs [dv][dk/2]
     static constexpr uint32_t TM_UT = TM_ST + 64;               // U^T bf16 pairs [dv][C/2]
     static constexpr uint32_t kCols = TM_UT + 32;
-    static constexpr uint32_t OFF_GATE = kStages * SZ_STAGE;   // 4 gate slots
+    static constexpr uint32_t SZ_Z = kC * kD * 2;               // z of one chunk [64 rows][d_v] bf16
+    static constexpr uint32_t OFF_Z = kStages * SZ_STAGE;       // ZB: two of them
+    static constexpr uint32_t OFF_OB = OFF_Z + 2 * SZ_Z;        // ZB: output rows [64][d_v] fp32
+    static constexpr uint32_t OFF_GATE = ZB ? OFF_OB + kC * kD * 4 : OFF_Z;   // 4 gate slots
     static constexpr uint32_t OFF_BAR = OFF_GATE + 4 * GATE_FLOATS * 4;   // mbarriers, TMEM slot, flag
     static constexpr uint32_t STATE_BYTES = OFF_BAR + 256;
 };
@@ -174,85 +183,83 @@ __device__ __forceinline__ void tmem_st_f32(uint32_t taddr, const float (&v)[N])
     else tmem_st32(taddr, v);
 }
 
-// Output rows of chunk cp with the layer's gated RMSNorm, by the 128 output
-// threads (4 warps, thread j = value channel j = TMEM lane): per 8 positions,
-// each warp sums the squares of its 32 channels by a butterfly that leaves lane
-// l with position 4 bit4 + 2 bit3 + bit2 of l, the four warps' sums meet in the
-// gate slot's key-norm area (free in the state pass; two halves used in turn,
-// so one barrier per step suffices), and every thread forms
-// y = w_j o_ij / sqrt(mean_j o_ij^2 + eps) act(z_ij) for its channel, stored
-// token-major like z.  o_ij already carries 1 / ||q_i|| (the prologue).
-__device__ __forceinline__ void norm_rows(const Args& ar, uint32_t oc, float* gsp, int64_t bh, int cp, int Cc,
-                                          int j, int lane, int w4) {
+// 1 / ||q_i|| of chunk c (with the prologue) sits in the chunk's gate slot, in
+// one of two fields by (c / 4) mod 2: the side warps write it up to four chunks
+// ahead of the output rows that read it, which then never share a field.
+__device__ __forceinline__ int rq_field(int c) { return (c >> 2) & 1 ? G_RK : G_RQ; }
+
+// z of chunk c (64 token-major rows of d_v, H d_v elements apart) into the shared
+// buffer zb by the NTHR output threads, 16 bytes a copy; rows past the chunk's
+// end are zero-filled and not read.
+template <int NTHR>
+__device__ __forceinline__ void z_load(const Args& ar, uint32_t zb, int64_t bh, int c, int Cc, int oid) {
+    const int64_t b = bh / ar.H, h = bh % ar.H;
+    const __nv_bfloat16* z0 = ar.z + ((b * ar.T + (int64_t)c * kC) * ar.H + h) * kD;
+#pragma unroll
+    for (int u = 0; u < 1024 / NTHR; ++u) {
+        const int x = oid + NTHR * u;              // 0..1023: (row, 16-byte chunk)
+        const int i = x >> 4, ch = x & 15;
+        const bool in = i < Cc;
+        cp_async16(zb + (uint32_t)(i * kD * 2 + ch * 16), z0 + (in ? (int64_t)i * ar.H * kD + ch * 8 : 0),
+                   in ? 16u : 0u);
+    }
+    cp_async_commit();
+}
+
+// Output rows of chunk cp with the layer's gated RMSNorm, in two steps by the
+// 256 output threads (8 warps).  First each thread copies 32 positions of its
+// value channel j (= TMEM lane) of the chunk's o' (fp32, TMEM) into the
+// row-major buffer ob (warps 0-3 positions 0-31, warps 4-7 positions 32-63);
+// then, after a barrier, thread t takes channels 8 (t mod 16) .. + 7 of rows
+// t / 16 + 16 u: the 16 threads of a row sum its squares by shuffles, and each
+// forms y_ij = w_j o_ij / sqrt(mean_j o_ij^2 + eps) act(z_ij) for its eight
+// channels (16-byte loads of o' and z, a 16-byte store of y, token-major like
+// z).  With the prologue o_ij = r_i o'_ij (r_i = 1 / ||q_i||), so row i's
+// factor is r_i / sqrt(r_i^2 mean_j o'_ij^2 + eps).
+__device__ __forceinline__ void norm_stage(uint32_t oc, float* __restrict__ ob, int j, int hh) {
+    float v[32];
+    tmem_ld32(oc + hh * 32, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ob[(hh * 32 + e) * kD + j] = v[e];
+}
+__device__ __forceinline__ void norm_rows(const Args& ar, const float* __restrict__ ob,
+                                          const __nv_bfloat16* __restrict__ zb, const float* rq, int64_t bh,
+                                          int cp, int Cc, int oid) {
     const int64_t b = bh / ar.H, h = bh % ar.H;
     const int64_t row0 = (b * ar.T + (int64_t)cp * kC) * ar.H + h;   // token-major row of position 0
-    const int64_t rstride = (int64_t)ar.H * kD;
-    const float wj = ar.norm_w[j];
+    const int c8 = (oid & 15) * 8;                                   // first channel of the thread
     const bool silu = ar.norm == 1;
-    // z of the first 8 positions; each step then requests the next step's z before its own work
-    __nv_bfloat16 zn[8];
+    float w[8];
+    *reinterpret_cast<float4*>(w) = *reinterpret_cast<const float4*>(ar.norm_w + c8);
+    *reinterpret_cast<float4*>(w + 4) = *reinterpret_cast<const float4*>(ar.norm_w + c8 + 4);
+#pragma unroll 2
+    for (int u = 0; u < 4; ++u) {
+        const int i = (oid >> 4) + 16 * u;
+        float x[8];
+        *reinterpret_cast<float4*>(x) = *reinterpret_cast<const float4*>(ob + i * kD + c8);
+        *reinterpret_cast<float4*>(x + 4) = *reinterpret_cast<const float4*>(ob + i * kD + c8 + 4);
+        const uint4 zv = *reinterpret_cast<const uint4*>(zb + i * kD + c8);
+        float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zn[e] = e < Cc ? ar.z[row0 * kD + (int64_t)e * rstride + j] : __float2bfloat16(0.f);
-#pragma unroll 1
-    for (int it = 0; it < 8; ++it) {
-        float* red = gsp + G_RK + (it & 1) * 32;      // [8 positions][4 warps]
-        float zf[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) zf[e] = __bfloat162float(zn[e]);
-        if (it + 1 < 8) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int i = 8 * (it + 1) + e;
-                zn[e] = i < Cc ? ar.z[row0 * kD + (int64_t)i * rstride + j] : __float2bfloat16(0.f);
-            }
-        }
-        float v[8];
-        {
-            uint32_t u[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-                           "=r"(u[7])
-                         : "r"(oc + 8 * it));
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(u[e]) * gsp[G_RQ + 8 * it + e];
-        }
-        float s4[4], s2[2], s1;
+        for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+        const float r = rq[i];
+        const float f = r * rsqrtf(r * r * ss * (1.f / (float)kD) + ar.eps);
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
+        uint32_t y[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const bool hi = lane & 16;
-            const float keep = hi ? v[e + 4] * v[e + 4] : v[e] * v[e];
-            const float send = hi ? v[e] * v[e] : v[e + 4] * v[e + 4];
-            s4[e] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            const float2 zz = __bfloat1622float2(z2[e]);
+            const float s0 = __fdividef(1.f, 1.f + __expf(-zz.x)), s1 = __fdividef(1.f, 1.f + __expf(-zz.y));
+            const float g0 = silu ? zz.x * s0 : s0, g1 = silu ? zz.y * s1 : s1;
+            y[e] = pack_bf16x2(x[2 * e] * f * w[2 * e] * g0, x[2 * e + 1] * f * w[2 * e + 1] * g1);
         }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const bool hi = lane & 8;
-            const float keep = hi ? s4[e + 2] : s4[e];
-            const float send = hi ? s4[e] : s4[e + 2];
-            s2[e] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        {
-            const bool hi = lane & 4;
-            const float keep = hi ? s2[1] : s2[0];
-            const float send = hi ? s2[0] : s2[1];
-            s1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-        const int p = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-        if ((lane & 3) == 0) red[p * 4 + w4] = s1;
-        named_bar_sync(1, kSideThreads);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * it + e;
-            const float4 r4 = *reinterpret_cast<const float4*>(red + 4 * e);
-            const float ms = ((r4.x + r4.y) + (r4.z + r4.w)) * (1.f / (float)kD);
-            const float rs = 1.f / sqrtf(ms + ar.eps);
-            const float zz = zf[e];
-            const float gte = silu ? zz / (1.f + __expf(-zz)) : 1.f / (1.f + __expf(-zz));
-            if (i < Cc) ar.o[row0 * kD + (int64_t)i * rstride + j] = __float2bfloat16_rn(v[e] * rs * wj * gte);
-        }
+        if (i < Cc)
+            *reinterpret_cast<uint4*>(ar.o + (row0 + (int64_t)i * ar.H) * kD + c8) = make_uint4(y[0], y[1], y[2], y[3]);
     }
 }
 
@@ -263,7 +270,7 @@ __device__ __forceinline__ void norm_rows(const Args& ar, uint32_t oc, float* gs
 // 1 alone, 2 with the gated RMSNorm on the output rows.
 template <int GATE, bool HOSTED, int PRO = 0>
 __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t head, uint32_t tmem_given) {
-    using L = Layout<HOSTED>;
+    using L = Layout<HOSTED, PRO == 2>;
     constexpr int kStages = L::kStages;
     constexpr uint32_t OFF_GATE = L::OFF_GATE, OFF_BAR = L::OFF_BAR;
     constexpr uint32_t TM_ST = L::TM_ST, TM_UT = L::TM_UT;
@@ -317,7 +324,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i)
-            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads : i >= B_READY0 ? kSideThreads : 1);
+            mbar_init(ctl.bar(i), i >= B_UTA ? kChainThreads
+                                  : i == B_OFREE0 || i == B_OFREE1 ? R::kOutThreads
+                                  : i >= B_READY0 ? kSideThreads : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -407,14 +416,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tma_load_2d(st + ST_B + 24576, &tm_w, 64, (int)(tile * kC), fb);
                 tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
                 tma_load_2d(st + ST_P, &tm_p, 0, (int)(tile * kC), fb);
-            }
-            if (PRO == 2 && !(test_flags & 1)) {
-                // the gated norm's z rows of this chunk into L2 (64 rows of 256 bytes, H d_v
-                // elements apart), so that the output warps' loads of them hit L2
-                const int64_t b = bh / ar.H, h = bh % ar.H;
-                const int Cn = min(kC, len - cc * kC);
-                for (int i = lane; i < Cn; i += 32)
-                    bulk_prefetch_l2(ar.z + (((b * T + (int64_t)cc * kC + i) * ar.H + h) * kD), kD * 2);
             }
             if (!(test_flags & 1)) issued = cc + 1;
         }
@@ -545,7 +546,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
-                        if ((sid & 7) == 0) gs[G_RQ + (sid >> 3) + 16 * u4] = 1.f / fmaxf(sqrtf(s2), 1e-12f);
+                        if ((sid & 7) == 0) gs[rq_field(c) + (sid >> 3) + 16 * u4] = 1.f / fmaxf(sqrtf(s2), 1e-12f);
                     }
                 }
             }
@@ -559,20 +560,16 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tc_fence_after();
                 __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
                 const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
-                const float* gsp = gates + (cp & 3) * GATE_FLOATS;   // 1 / ||q_i|| with the prologue
-                if (PRO == 2) {
-                    norm_rows(ar, oc, gates + (cp & 3) * GATE_FLOATS, bh, cp, Cc, j, lane, warp - kSideWarp0);
-                } else {
+                const float* rq = gates + (cp & 3) * GATE_FLOATS + rq_field(cp);   // 1 / ||q_i||
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float v[32];
-                        tmem_ld32(oc + hh * 32, v);
-                        tmem_wait_ld();
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tmem_ld32(oc + hh * 32, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = hh * 32 + e;
-                            if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * gsp[G_RQ + i] : v[e]);
-                        }
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = hh * 32 + e;
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * rq[i] : v[e]);
                     }
                 }
                 tc_fence_before();
@@ -580,31 +577,53 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
             }
         }
     } else if (kSplitOut && warp >= R::kOutWarp0) {
-        // ================= output rows of each chunk (128 threads, plain path) ==========
+        // ================= output rows of each chunk (128 threads) =======================
         const int q = warp & 3;                    // TMEM lane quarter
         const int j = (q << 5) + lane;             // value channel = TMEM lane
+        constexpr int kOT = R::kOutThreads;
+        const int oid = tid - R::kOutWarp0 * 32;   // 0 .. kOT - 1
+        // with the gated norm, z of each chunk is copied in one chunk ahead
+        const uint32_t zbuf = sb + L::OFF_Z;
+        if (PRO == 2) z_load<kOT>(ar, zbuf, bh, 0, min(kC, len), oid);
         for (int cp = 0; cp < n; ++cp) {
             const int Cc = min(kC, len - cp * kC);
             bool ok = ctl.wait(B_PU0 + (cp & 1), (uint32_t)(cp >> 1) & 1u);
             if (!ok) *abort_flag = 1;
-            if (named_bar_any(5, kSideThreads, !ok)) break;
+            if (PRO == 2) cp_async_wait_all();
+            if (named_bar_any(5, kOT, !ok)) break;
+            // every thread is past chunk cp - 1, whose z buffer now takes chunk cp + 1
+            if (PRO == 2 && cp + 1 < n)
+                z_load<kOT>(ar, zbuf + ((cp + 1) & 1) * L::SZ_Z, bh, cp + 1, min(kC, len - (cp + 1) * kC), oid);
             tc_fence_after();
-            __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
             const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
+            const float* rq = gates + (cp & 3) * GATE_FLOATS + rq_field(cp);   // 1 / ||q_i||
+            if constexpr (PRO == 2) {
+                float* ob = reinterpret_cast<float*>(sm + L::OFF_OB);
+                norm_stage(oc, ob, j, oid >> 7);
+                tc_fence_before();
+                mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));        // the TMEM buffer is read
+                named_bar_sync(5, kOT);
+                norm_rows(ar, ob, reinterpret_cast<const __nv_bfloat16*>(sm + L::OFF_Z + (cp & 1) * L::SZ_Z), rq,
+                          bh, cp, Cc, oid);
+            } else {
+                __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[32];
-                tmem_ld32(oc + hh * 32, v);
-                tmem_wait_ld();
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tmem_ld32(oc + hh * 32, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = hh * 32 + e;
-                    if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = hh * 32 + e;
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * rq[i] : v[e]);
+                    }
                 }
+                tc_fence_before();
+                mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
             }
-            tc_fence_before();
-            mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));
         }
+        // no copy of this thread is still in flight when the shared memory is released
+        if (PRO == 2) cp_async_wait_all();
     } else if (warp >= kChainWarp0) {
         // ================= U and the state (kChainThreads threads) =================
         // kNQ warps per TMEM lane quarter; each pass splits its columns among them

@@ -105,7 +105,7 @@ varlen_table_kernel(const int* __restrict__ cu_in, int N, int T, int* tables, un
 
 namespace {
 constexpr int kFusedThreads = 4 * wy::kNT;          // 32 warps: 4 WY groups, or the state pass + up to 16 more
-static_assert(state::kHostedNT + wy::kNT <= kFusedThreads && state::Roles<kGateScalar>::kNT <= kFusedThreads,
+static_assert(state::kHostedNT + wy::kNT <= kFusedThreads && state::Roles<kGateScalar, false, 2>::kNT <= kFusedThreads,
               "fused CTA size");
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 // a hosted WY group's shared memory starts past the hosted state pass's
@@ -139,13 +139,13 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H,
                              pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps};
-        if (!HOSTED) {
-            // ---- state pass of head blockIdx.x (warps 0-15) ------------------------------
+        if constexpr (!HOSTED) {
+            // ---- state pass of head blockIdx.x --------------------------------------------
             if (warp >= state::Roles<GATE, false, PRO>::kNT / 32) return;
             state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
             return;
-        }
-        // ---- state pass (warps 0-15) and one WY group (warps 16-23) ------------------------
+        } else {
+        // ---- state pass (warps 0-23) and one WY group (warps 24-31) ------------------------
         constexpr int kStateNT = state::Roles<GATE, true, PRO>::kNT;
         constexpr int kHostThreads = kStateNT + wy::kNT;
         if (tid >= kHostThreads) return;
@@ -184,6 +184,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tmem_dealloc(tbase, state::TM_COLS);
         }
         return;
+        }
     }
     // ---- four WY groups, each taking every G-th tile in chunk-major order -----------------
     const int grp = warp >> 3;                       // 0..3
@@ -338,8 +339,11 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     const int64_t BH = a.B * a.H;
     if (coop && fused_fits(BH, num_sms)) {
         // with many heads the dedicated WY groups get scarce: the state-pass CTAs
-        // host one each (measured: at 64 heads of 148 SMs hosting is not yet a gain)
-        auto kern = BH * 2 > (int64_t)num_sms + 12 ? chunk_fused_kernel<GATE, true, PRO> : chunk_fused_kernel<GATE, false, PRO>;
+        // host one each (measured: at 64 heads of 148 SMs hosting is not yet a gain);
+        // the gated norm's state pass needs its SM's shared memory alone
+        auto kern = chunk_fused_kernel<GATE, false, PRO>;
+        if constexpr (PRO != 2)
+            if (BH * 2 > (int64_t)num_sms + 12) kern = chunk_fused_kernel<GATE, true, PRO>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedBytes);
         if (e != cudaSuccess) return e;
         int per_sm = 0;

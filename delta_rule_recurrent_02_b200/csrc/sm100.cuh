@@ -88,6 +88,16 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) 
                  : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (through L2 only); the bytes past
+// src_bytes (0 or 16) are zero-filled and not read.  Both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// every cp.async of this thread has landed (visible to the thread; a barrier publishes it)
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Tile store shared -> global through a tensor map (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uint32_t src) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
