@@ -466,12 +466,16 @@ int dn_causal_conv1d(const void* x, int ld_x, const float* weight, const void* s
         return fail(DN_ERR_INVALID, "state_out may be state_in itself only when T <= 16; otherwise it must not overlap it");
     const int V = (int)(8 / esz);     // channels per 8-byte access
     bool vec = C % V == 0 && ld_x % V == 0 && head_dim % V == 0;
-    for (const void* p : pe)
+    bool vec16 = C % (2 * V) == 0 && ld_x % (2 * V) == 0 && head_dim % (2 * V) == 0;
+    for (const void* p : pe) {
         if (p && !aligned(p, 8)) vec = false;
+        if (p && !aligned(p, 16)) vec16 = false;
+    }
+    if (!aligned(weight, 16)) vec16 = false;
     dn::ConvArgs a;
     a.x = x; a.ld_x = ld_x; a.weight = weight; a.state_in = state_in; a.y = y; a.state_out = state_out;
     a.B = B; a.T = T; a.C = C; a.K = K; a.head_dim = head_dim;
-    a.activation = activation == 1; a.bf16 = dtype == DN_BF16; a.vec = vec;
+    a.activation = activation == 1; a.bf16 = dtype == DN_BF16; a.vec = vec; a.vec16 = vec16;
     if (T == 0 && (!state_out || K == 1)) return ok();
     cudaError_t e = dn::launch_causal_conv1d(a, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "causal conv kernel");

@@ -91,6 +91,7 @@ struct ConvArgs {
     bool activation;          // SiLU
     bool bf16;
     bool vec;                 // 8-byte accesses (alignment checked by the caller)
+    bool vec16 = false;       // 16-byte accesses (likewise)
 };
 cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st);
 

@@ -11,6 +11,7 @@
 #include <stdint.h>
 
 #include "dn_kernels.h"
+#include "sm100.cuh"
 
 namespace dn {
 namespace {
@@ -94,9 +95,10 @@ struct Vec<float, 2> {
     __device__ static raw from_f(const float* f) { return make_float2(f[0], f[1]); }
 };
 
-// SiLU and the logistic sigmoid through the fast exp and a correctly rounded reciprocal:
-// for very negative x the exp overflows to inf and the reciprocal gives 0, the right limit
-__device__ __forceinline__ float sigmoid(float x) { return __frcp_rn(1.f + __expf(-x)); }
+// SiLU and the logistic sigmoid through the fast exp and the approximate reciprocal
+// (a few ulp, far inside a bf16 rounding): for very negative x the exp overflows to
+// inf and 1 / inf gives 0, the right limit
+__device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 __device__ __forceinline__ float silu(float x) { return x * sigmoid(x); }
 
 // ---- causal conv ----------------------------------------------------------------------
@@ -239,6 +241,176 @@ causal_conv1d_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __res
     }
 }
 
+// Tiled form for layouts that allow 16-byte accesses.  A block owns 32 vectors of
+// V = 16 / sizeof(Tin) channels of one sequence (their filters stay in registers)
+// and a run of 32-token tiles of it.  Each tile and the K-1 rows before it (x, or
+// the carried state before token 0, or zeros) are copied into shared memory by
+// cp.async, the next tile while the current one is computed (two buffers); each
+// thread slides its channels' filter over 8 consecutive rows from there and
+// stores 16 bytes a row.  The block of the last tile also writes the new state
+// from the same rows.
+constexpr int kTileRows = 32;
+constexpr int kConvStages = 2;                           // tiles in flight per block
+constexpr int kConvWarps = 4;                            // each thread: 32 / kConvWarps rows of a tile
+
+template <typename Tin, int K>
+struct ConvTile {
+    static constexpr int V = 16 / (int)sizeof(Tin);
+    static constexpr int kCh = 32 * V;                   // channels of a block
+    static constexpr int kRowsIn = kTileRows + K - 1;
+    Tin rows[kConvStages][kRowsIn][kCh];
+};
+
+template <typename Tin, int K, bool ACT>
+__global__ void __launch_bounds__(kConvWarps * 32)
+causal_conv1d_tile_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* __restrict__ w, const Tin* s_in,
+                          Tin* __restrict__ y, Tin* s_out, int T, int C, int hd, int run) {
+    using CT = ConvTile<Tin, K>;
+    constexpr int V = CT::V, kCh = CT::kCh, kRowsIn = CT::kRowsIn;
+    constexpr int kNT = kConvWarps * 32, kRPT = kTileRows / kConvWarps;   // threads; rows per thread
+    using VT = Vec<Tin, V>;
+    using raw = typename VT::raw;
+    extern __shared__ __align__(16) unsigned char conv_smem[];
+    CT& sm = *reinterpret_cast<CT*>(conv_smem);
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int cb0 = blockIdx.x * kCh;
+    const int64_t b = blockIdx.z;
+    const int n_tiles = T > 0 ? (T + kTileRows - 1) / kTileRows : 1;
+    const int tile_beg = blockIdx.y * run, tile_end = min(n_tiles, tile_beg + run);
+    if (tile_beg >= tile_end) return;
+    // rows t0 - (K-1) .. t0 + 31 of the block's channels into buffer buf; zero past
+    // the sequence or C
+    auto fetch = [&](int tile, int buf) {
+        const int t0 = tile * kTileRows;
+        for (int idx = threadIdx.x; idx < kRowsIn * 32; idx += kNT) {
+            const int r = idx >> 5, cv = idx & 31;
+            const int t = t0 - (K - 1) + r, c = cb0 + cv * V;
+            const Tin* src = nullptr;
+            if (c < C) {
+                if (t >= 0 && t < T) src = x + (b * T + t) * ld_x + c;
+                else if (t < 0 && s_in) src = s_in + (b * (K - 1) + (t + K - 1)) * (int64_t)C + c;
+            }
+            if (src) sm100::cp_async16(sm100::smem_u32(&sm.rows[buf][r][cv * V]), src, 16);
+            else *reinterpret_cast<uint4*>(&sm.rows[buf][r][cv * V]) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        sm100::cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kConvStages - 1; ++s)
+        if (tile_beg + s < tile_end) fetch(tile_beg + s, s);
+    // the thread's filters while the rows land: channels c0 .. c0 + V - 1, K taps each,
+    // V K consecutive floats of w
+    const int c0 = cb0 + tx * V;
+    const bool active = c0 < C;
+    float wf[K][V];
+    {
+        float wl[V * K];
+#pragma unroll
+        for (int u = 0; u < V * K / 4; ++u) {
+            const float4 f = active ? reinterpret_cast<const float4*>(w + (int64_t)c0 * K)[u]
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            wl[4 * u] = f.x; wl[4 * u + 1] = f.y; wl[4 * u + 2] = f.z; wl[4 * u + 3] = f.w;
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int j = 0; j < K; ++j) wf[j][v] = wl[v * K + j];
+    }
+    const int nh = C / hd;
+    const int head = c0 / hd, jj = c0 - head * hd;
+    Tin* yb = y + ((b * nh + (active ? head : 0)) * (int64_t)T) * hd + jj;
+    const int r0 = ty * kRPT;                             // the thread's first output row of a tile
+    for (int tile = tile_beg; tile < tile_end; ++tile) {
+        const int buf = (tile - tile_beg) % kConvStages;
+        // the tile kConvStages - 1 ahead into the buffer read one tile ago (the barrier at
+        // the end of that tile is behind every thread), then wait for this tile's rows
+        const int ahead = tile + kConvStages - 1;
+        if (ahead < tile_end) fetch(ahead, (ahead - tile_beg) % kConvStages);
+        const int later = min(tile_end - 1, ahead) - tile;     // groups committed after this tile's
+        if (later >= 2) sm100::cp_async_wait_group<2>();
+        else if (later == 1) sm100::cp_async_wait_group<1>();
+        else sm100::cp_async_wait_group<0>();
+        __syncthreads();
+        const int t0 = tile * kTileRows;
+        if (active) {
+            float win[K][V];
+#pragma unroll
+            for (int j = 0; j < K - 1; ++j) VT::to_f(*reinterpret_cast<const raw*>(&sm.rows[buf][r0 + j][tx * V]), win[j]);
+#pragma unroll
+            for (int i = 0; i < kRPT; ++i) {
+                const int t = t0 + r0 + i;
+                VT::to_f(*reinterpret_cast<const raw*>(&sm.rows[buf][r0 + i + K - 1][tx * V]), win[K - 1]);
+                float acc[V];
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int j = 0; j < K; ++j) a = fmaf(wf[j][v], win[j][v], a);
+                    acc[v] = ACT ? silu(a) : a;
+                }
+                if (t < T) *reinterpret_cast<raw*>(yb + (int64_t)t * hd) = VT::from_f(acc);
+#pragma unroll
+                for (int j = 0; j < K - 1; ++j)
+#pragma unroll
+                    for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
+            }
+            if (s_out && K > 1 && ty == 0 && t0 + kTileRows >= T) {
+                // new state row j = input row T - K + 1 + j, local row T - t0 + j (all read
+                // into shared memory above, so s_out may be s_in itself when this is the
+                // only tile)
+#pragma unroll
+                for (int j = 0; j < K - 1; ++j)
+                    *reinterpret_cast<uint4*>(s_out + (b * (K - 1) + j) * (int64_t)C + c0) =
+                        *reinterpret_cast<const uint4*>(&sm.rows[buf][T - t0 + j][tx * V]);
+            }
+        }
+        __syncthreads();                                   // buf is refilled from the next tile on
+    }
+}
+
+template <typename Tin, int K>
+cudaError_t launch_conv_tile_k(const ConvArgs& a, cudaStream_t st) {
+    constexpr int kCh = ConvTile<Tin, K>::kCh;
+    const int n_tiles = a.T > 0 ? (a.T + kTileRows - 1) / kTileRows : 1;
+    const int n_cb = (a.C + kCh - 1) / kCh;
+    // about four blocks per SM, each a run of consecutive tiles of one (sequence, channel block)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    constexpr int kBytes = (int)sizeof(ConvTile<Tin, K>);
+    if (kBytes > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(a.activation ? causal_conv1d_tile_kernel<Tin, K, true>
+                                                                : causal_conv1d_tile_kernel<Tin, K, false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t pairs = (int64_t)n_cb * a.B;
+    const int64_t want = (4 * (int64_t)sms + pairs - 1) / pairs;
+    const int splits = (int)(want < 1 ? 1 : want > n_tiles ? n_tiles : want);
+    const int run = (n_tiles + splits - 1) / splits;
+    const dim3 grid((unsigned)n_cb, (unsigned)((n_tiles + run - 1) / run), (unsigned)a.B);
+    const Tin* x = static_cast<const Tin*>(a.x);
+    const Tin* s_in = static_cast<const Tin*>(a.state_in);
+    Tin* y = static_cast<Tin*>(a.y);
+    Tin* s_out = static_cast<Tin*>(a.state_out);
+    if (a.activation)
+        causal_conv1d_tile_kernel<Tin, K, true><<<grid, kConvWarps * 32, kBytes, st>>>(
+            x, a.ld_x, a.weight, s_in, y, s_out, a.T, a.C, a.head_dim, run);
+    else
+        causal_conv1d_tile_kernel<Tin, K, false><<<grid, kConvWarps * 32, kBytes, st>>>(
+            x, a.ld_x, a.weight, s_in, y, s_out, a.T, a.C, a.head_dim, run);
+    return counted(cudaGetLastError());
+}
+
+template <typename Tin>
+cudaError_t launch_conv_tile(const ConvArgs& a, cudaStream_t st) {
+    switch (a.K) {
+        case 1: return launch_conv_tile_k<Tin, 1>(a, st);
+        case 2: return launch_conv_tile_k<Tin, 2>(a, st);
+        case 3: return launch_conv_tile_k<Tin, 3>(a, st);
+        default: return launch_conv_tile_k<Tin, 4>(a, st);
+    }
+}
+
 template <typename Tin, int V, int K>
 cudaError_t launch_conv_k(const ConvArgs& a, cudaStream_t st) {
     const int n_cv = a.C / V;
@@ -316,7 +488,7 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
 #pragma unroll
     for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (!valid) return;
-    const float inv = 1.f / sqrtf(ss / (float)D + eps);
+    const float inv = rsqrtf(ss / (float)D + eps);
 #pragma unroll
     for (int a = 0; a < NV; ++a) {
         const int c = (a * LPR + l) * VE;
@@ -364,8 +536,10 @@ cudaError_t launch_norm_t(const NormArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-// 8-byte accesses where the layout allows (a.vec): 4 bf16 or 2 fp32 channels per thread
+// The tiled kernel where the layout allows 16-byte accesses (a.vec16); else 8-byte
+// accesses where it allows those (a.vec): 4 bf16 or 2 fp32 channels per thread
 cudaError_t launch_causal_conv1d(const ConvArgs& a, cudaStream_t st) {
+    if (a.vec16) return a.bf16 ? launch_conv_tile<__nv_bfloat16>(a, st) : launch_conv_tile<float>(a, st);
     if (a.bf16) return a.vec ? launch_conv_v<__nv_bfloat16, 4>(a, st) : launch_conv_v<__nv_bfloat16, 1>(a, st);
     return a.vec ? launch_conv_v<float, 2>(a, st) : launch_conv_v<float, 1>(a, st);
 }

@@ -97,6 +97,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // every cp.async of this thread has landed (visible to the thread; a barrier publishes it)
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// all but this thread's N most recent committed groups have landed
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
 // Tile store shared -> global through a tensor map (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uint32_t src) {

@@ -57,6 +57,7 @@ def head_major(y, B, T, C, hd):
     (2, 21, 64, 1, 64, None, True, True),       # K = 1: no history
     (2, 19, 96, 4, 96, None, True, False),      # no carried state: zeros
     (1, 2, 64, 4, 64, None, True, True),        # T < K - 1: the new state keeps old rows
+    (2, 70, 320, 4, 64, 448, True, True),       # several channel blocks (the last partial), 3 row tiles
 ])
 def test_causal_conv1d_matches_oracle(cuda_device, dtype, B, T, C, K, hd, ld, act, state):
     wide, x, w, s = conv_inputs(B, T, C, K, dtype, seed=B * 1000 + T + C + K, with_state=state, ld=ld)
