@@ -503,37 +503,56 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 if (named_bar_any(1, kSideThreads, !ok)) break;
                 float ssq[4] = {0.f, 0.f, 0.f, 0.f};
                 // (with the per-key gate the workspace holds Qh already)
+                // (loads four at a time: the ld / st helpers keep their order, so one load per
+                // iteration would wait out each load's latency in turn)
 #pragma unroll
-                for (int u = 0; u < (GATE == kGatePerKey ? 0 : 8); ++u) {
-                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
-                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
-                    const uint32_t a = st + ST_B + blk * 16384 + sw128_off(i, ch);
-                    const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
-                    const uint4 w = ld_shared_v4(a);
-                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                    if (PRO)
-                        ssq[u & 3] += e0.x * e0.x + e0.y * e0.y + e1.x * e1.x + e1.y * e1.y +
-                                      e2.x * e2.x + e2.y * e2.y + e3.x * e3.x + e3.y * e3.y;
-                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                for (int u0 = 0; u0 < (GATE == kGatePerKey ? 0 : 8); u0 += 4) {
+                    uint4 w[4];
+                    uint32_t a[4];
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        const int x = sid + (u0 + uu) * kSideThreads;   // (d-block, row, 16-byte chunk)
+                        const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                        a[uu] = st + ST_B + blk * 16384 + sw128_off(i, ch);
+                        w[uu] = ld_shared_v4(a[uu]);
+                    }
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        const int i = ((sid + (u0 + uu) * kSideThreads) >> 3) & 63;
+                        const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
+                        const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+                        const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+                        if (PRO)
+                            ssq[uu] += (e0.x * e0.x + e0.y * e0.y + e1.x * e1.x + e1.y * e1.y) +
+                                       (e2.x * e2.x + e2.y * e2.y + e3.x * e3.x + e3.y * e3.y);
+                        st_shared_v4(a[uu], pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                                     pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                    }
                 }
                 // ---- K~ = K (.) e^(G_last - G) in place over the k tile: each position's decay to
                 //      the chunk's end folded into its key, so that the KU product reads U itself
                 //      (no gate: the factor is 1; per-key gate: the workspace holds K~)
 #pragma unroll
-                for (int u = 0; u < (GATE == kGateScalar ? 8 : 0); ++u) {
-                    const int x = sid + u * kSideThreads;     // 0..1023: (d-block, row, 16-byte chunk)
-                    const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
-                    const uint32_t a = st + ST_K + blk * 8192 + sw128_off(i, ch);
-                    const float f = gs[G_ET + i];
-                    const uint4 w = ld_shared_v4(a);
-                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-                    const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-                    const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                    st_shared_v4(a, pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                                 pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                for (int u0 = 0; u0 < (GATE == kGateScalar ? 8 : 0); u0 += 4) {
+                    uint4 w[4];
+                    uint32_t a[4];
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        const int x = sid + (u0 + uu) * kSideThreads;   // (d-block, row, 16-byte chunk)
+                        const int blk = x >> 9, i = (x >> 3) & 63, ch = x & 7;
+                        a[uu] = st + ST_K + blk * 8192 + sw128_off(i, ch);
+                        w[uu] = ld_shared_v4(a[uu]);
+                    }
+#pragma unroll
+                    for (int uu = 0; uu < 4; ++uu) {
+                        const float f = gs[G_ET + (((sid + (u0 + uu) * kSideThreads) >> 3) & 63)];
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
+                        const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
+                        const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
+                        st_shared_v4(a[uu], pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
+                                     pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                    }
                 }
                 fence_async_smem();
                 mbar_arrive(ctl.bar(B_READY0 + s));
@@ -546,7 +565,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
                         s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
-                        if ((sid & 7) == 0) gs[rq_field(c) + (sid >> 3) + 16 * u4] = 1.f / fmaxf(sqrtf(s2), 1e-12f);
+                        if ((sid & 7) == 0) gs[rq_field(c) + (sid >> 3) + 16 * u4] = fminf(rsqrtf(s2), 1e12f);
                     }
                 }
             }

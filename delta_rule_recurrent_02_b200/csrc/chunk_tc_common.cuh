@@ -128,19 +128,22 @@ constexpr uint32_t GATE_FLOATS = 512;
 // summed by two threads: this one takes the 64 columns of block `half`; the
 // partner (lane ^ 1) the other.
 __device__ __forceinline__ float inv_row_norm(uint32_t tile, int row, int half, uint32_t block_bytes) {
-    float ss = 0.f;
+    uint4 w[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) w[ch] = ld_shared_v4(tile + (uint32_t)half * block_bytes + sw128_off(row, ch));
+    float ss[4] = {0.f, 0.f, 0.f, 0.f};                  // four partial sums: short dependency chains
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
-        const uint4 w = ld_shared_v4(tile + (uint32_t)half * block_bytes + sw128_off(row, ch));
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[ch]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(h[e]);
-            ss += f.x * f.x + f.y * f.y;
+            ss[e] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[e]));
         }
     }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    return 1.f / fmaxf(sqrtf(ss), 1e-12f);
+    float t = (ss[0] + ss[1]) + (ss[2] + ss[3]);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    return fminf(rsqrtf(t), 1e12f);                      // 1 / max(||x||, 1e-12)
 }
 
 // Gates of one chunk from beta and g at positions lane and lane + 32 (zero past

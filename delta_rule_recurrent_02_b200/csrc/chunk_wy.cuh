@@ -33,7 +33,9 @@
 // which raises the flag during the group's next tile, while warps 0-5 form the
 // M blocks and warp 6 has nothing else to do (after the group's last tile, the
 // caller raises it with publish_pending()).  The gpu-scope release costs about
-// 1.5k cycles under load; there it is off the group's critical path.
+// 1.5k cycles under load; there it is off the group's critical path.  Tiles of
+// the first two chunks are the exception: every state pass starts by waiting
+// for them, so their flags go up as soon as their stores are complete.
 //
 // A partial last chunk has beta = 0 and g = 0 past its end: those rows of A
 // and P, and those columns of W^T and u^T, are zero (equal to zero padding).
@@ -603,6 +605,9 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         // the flag waits until the stores are complete
         bulk_wait_read_all();
         pending = tile;
+        // the first two chunk columns gate the start of every state pass: their flags go up
+        // as soon as the stores are complete, not during the group's next tile
+        if (c < 2) publish_pending(ar, pending);
     }
     if (tid == kStoreTid) *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 24) = ticket;
     tc_fence_before();
