@@ -32,11 +32,13 @@ constexpr int kNT = 256;     // threads per CTA
 constexpr int kDVT = 32;     // value columns per CTA
 constexpr int kCmax = 64;    // largest chunk
 constexpr int kVS = kDVT + 1;
-constexpr int kCS = kCmax + 1;
+constexpr int kCS = kCmax + 4;   // A, P rows: 16-byte aligned (read as float4 along a row)
 
+// Row strides are multiples of 4 floats, and so every region's offset: rows of K, Q
+// and P are read as float4, broadcast to a warp, along the contraction.
 template <int DK, int GATE>
 struct SimtSmem {
-    static constexpr int KS = DK + 1;
+    static constexpr int KS = DK + 4;
     static constexpr int kK = 0;                              // K      [Cmax][KS]
     static constexpr int kQ = kK + kCmax * KS;                // Q      [Cmax][KS]
     static constexpr int kG = kQ + kCmax * KS;                // Gamma  [Cmax][KS] or [Cmax]
@@ -50,7 +52,8 @@ struct SimtSmem {
     static constexpr int kB = kS + DK * kVS;                  // beta   [Cmax]
     static constexpr int kE = kB + kCmax;                     // e^G_i  [Cmax]
     static constexpr int kT = kE + kCmax;                     // e^(G_last - G_i) [Cmax]
-    static constexpr int kTotal = kT + kCmax;
+    static constexpr int kD = kT + kCmax;                     // (I + A_bb)^-1 [4 blocks][16][17]
+    static constexpr int kTotal = kD + 4 * 16 * 17;
     static constexpr size_t bytes = sizeof(float) * kTotal;
 };
 
@@ -78,6 +81,7 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     float* bs = sm + L::kB;
     float* eG = sm + L::kE;
     float* eT = sm + L::kT;
+    float* Dm = sm + L::kD;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -151,6 +155,8 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 vd[0] = pv[u].x; vd[1] = pv[u].y; vd[2] = pv[u].z; vd[3] = pv[u].w;
             }
         }
+        // rows of V past a short chunk's end are zero: the blocked products read whole rows
+        for (int x = Cc * kDVT + tid; x < kCmax * kDVT; x += kNT) Vs[(x / kDVT) * kVS + x % kDVT] = 0.f;
         if (tid < Cc) {
             float bb = pb, aa = ps;
             if (PRO) gdn_raw_gates(bb, aa, expf(A_log[bh % H]), dt_bias[bh % H], bmul);
@@ -217,14 +223,48 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         }
         __syncthreads();
         // ---- pairwise decayed products: A (strict lower) and P (lower) ---
-        for (int p = tid; p < Cc * Cc; p += kNT) {
-            const int i = p / Cc, j = p % Cc;
-            float kd = 0.f, qd = 0.f;
-            if (j <= i) {
-                const float* ki = Ks + i * KS;
-                const float* qi = Qs + i * KS;
-                const float* kj = Ks + j * KS;
-                if (GATE == kGatePerKey) {
+        if (GATE != kGatePerKey) {
+            // warp w: rows 8w .. 8w + 7 (K and Q rows read as broadcast float4 along c);
+            // lane: columns lane and lane + 32.  Whole 64 x 64 tiles are written (zero
+            // outside the chunk), so the later products need no bounds
+            const int i0 = warp * 8;
+            float ka[8][2], qa[8][2];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) ka[r][0] = ka[r][1] = qa[r][0] = qa[r][1] = 0.f;
+#pragma unroll 2
+            for (int c = 0; c < DK; c += 4) {
+                const float4 kj0 = *reinterpret_cast<const float4*>(Ks + lane * KS + c);
+                const float4 kj1 = *reinterpret_cast<const float4*>(Ks + (lane + 32) * KS + c);
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float4 ki = *reinterpret_cast<const float4*>(Ks + (i0 + r) * KS + c);
+                    const float4 qi = *reinterpret_cast<const float4*>(Qs + (i0 + r) * KS + c);
+                    ka[r][0] = fmaf(ki.x, kj0.x, fmaf(ki.y, kj0.y, fmaf(ki.z, kj0.z, fmaf(ki.w, kj0.w, ka[r][0]))));
+                    ka[r][1] = fmaf(ki.x, kj1.x, fmaf(ki.y, kj1.y, fmaf(ki.z, kj1.z, fmaf(ki.w, kj1.w, ka[r][1]))));
+                    qa[r][0] = fmaf(qi.x, kj0.x, fmaf(qi.y, kj0.y, fmaf(qi.z, kj0.z, fmaf(qi.w, kj0.w, qa[r][0]))));
+                    qa[r][1] = fmaf(qi.x, kj1.x, fmaf(qi.y, kj1.y, fmaf(qi.z, kj1.z, fmaf(qi.w, kj1.w, qa[r][1]))));
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int i = i0 + r;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = lane + 32 * h;
+                    const bool in = i < Cc && j <= i;
+                    const float d = (GATE == kGateScalar && in) ? expf(Gm[i] - Gm[j]) : 1.f;
+                    Am[i * kCS + j] = (in && j < i) ? bs[i] * ka[r][h] * d : 0.f;
+                    Pm[i * kCS + j] = in ? qa[r][h] * d : 0.f;
+                }
+            }
+        } else {
+            for (int p = tid; p < kCmax * kCmax; p += kNT) {
+                const int i = p / kCmax, j = p % kCmax;
+                float kd = 0.f, qd = 0.f;
+                if (j <= i && i < Cc) {
+                    const float* ki = Ks + i * KS;
+                    const float* qi = Qs + i * KS;
+                    const float* kj = Ks + j * KS;
                     const float* gi = Gm + i * KS;
                     const float* gj = Gm + j * KS;
 #pragma unroll 4
@@ -233,21 +273,10 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                         kd += ki[c] * w;
                         qd += qi[c] * w;
                     }
-                } else {
-#pragma unroll 8
-                    for (int c = 0; c < DK; ++c) {
-                        kd += ki[c] * kj[c];
-                        qd += qi[c] * kj[c];
-                    }
-                    if (GATE == kGateScalar) {
-                        const float d = expf(Gm[i] - Gm[j]);
-                        kd *= d;
-                        qd *= d;
-                    }
                 }
+                Am[i * kCS + j] = (j < i && i < Cc) ? bs[i] * kd : 0.f;
+                Pm[i * kCS + j] = (j <= i && i < Cc) ? qd : 0.f;
             }
-            Am[i * kCS + j] = (j < i) ? bs[i] * kd : 0.f;
-            Pm[i * kCS + j] = qd;
         }
         if (GATE == kGatePerKey) {
             __syncthreads();   // P used the raw q; now Q <- Q * e^Gamma, Kx <- K * e^Gamma
@@ -260,45 +289,140 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         }
         __syncthreads();
         // ---- right-hand side: beta * (V - (K * e^Gamma) S) ---------------
+        //      warp w: rows 8w .. 8w + 7 (K rows as broadcast float4 along c); lane: column
         {
-            const int j = lane;
-            for (int i = warp; i < Cc; i += kNT / 32) {
-                const float* kr = (GATE == kGatePerKey) ? (Kx + i * KS) : (Ks + i * KS);
-                float acc = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) acc += kr[c] * Ss[c * kVS + j];
-                if (GATE != kGatePerKey) acc *= eG[i];
-                Vs[i * kVS + j] = bs[i] * (Vs[i * kVS + j] - acc);
+            const int j = lane, i0 = warp * 8;
+            if (i0 < Cc) {
+                const float* kb = (GATE == kGatePerKey) ? Kx : Ks;
+                float acc[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+#pragma unroll 2
+                for (int c = 0; c < DK; c += 4) {
+                    const float s0 = Ss[c * kVS + j], s1 = Ss[(c + 1) * kVS + j];
+                    const float s2 = Ss[(c + 2) * kVS + j], s3 = Ss[(c + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float4 kv = *reinterpret_cast<const float4*>(kb + (i0 + r) * KS + c);
+                        acc[r] = fmaf(kv.x, s0, fmaf(kv.y, s1, fmaf(kv.z, s2, fmaf(kv.w, s3, acc[r]))));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int i = i0 + r;
+                    if (i < Cc) {
+                        const float a = (GATE != kGatePerKey) ? acc[r] * eG[i] : acc[r];
+                        Vs[i * kVS + j] = bs[i] * (Vs[i * kVS + j] - a);
+                    }
+                }
             }
         }
         __syncthreads();
-        // ---- forward substitution (I + A) U = rhs, 4 columns per warp ----
+        // ---- (I + A) U = rhs by 16-row blocks: the diagonal inverses D_b = (I + A_bb)^-1 of
+        //      every block at once (forward substitution, one warp per block, lane = column),
+        //      then U_b = D_b (rhs_b - sum_{m < 16 b} A_bm U_m) block after block.  Rows and
+        //      columns past Cc are identity / zero (never read by the later steps) ----------
         {
-            const int j = warp * 4 + (lane >> 3);
-            const int part = lane & 7;
-            for (int i = 1; i < Cc; ++i) {
-                float acc = 0.f;
-                for (int m = part; m < i; m += 8) acc += Am[i * kCS + m] * Vs[m * kVS + j];
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (part == 0) Vs[i * kVS + j] -= acc;
-                __syncwarp();
+            const int nb = (Cc + 15) >> 4;
+            if (warp < nb && lane < 16) {
+                const int k0 = warp * 16, jj = lane;
+                float x[16];
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) {
+                    float p0 = ii == jj ? 1.f : 0.f, p1 = 0.f;
+                    if (k0 + ii < Cc) {
+#pragma unroll
+                        for (int m = 0; m < ii; m += 2) {
+                            p0 -= Am[(k0 + ii) * kCS + k0 + m] * x[m];
+                            if (m + 1 < ii) p1 -= Am[(k0 + ii) * kCS + k0 + m + 1] * x[m + 1];
+                        }
+                    }
+                    x[ii] = p0 + p1;
+                }
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) Dm[(warp * 16 + ii) * 17 + jj] = x[ii];
+            }
+            __syncthreads();
+            for (int b = 0; b < nb; ++b) {
+                const int r0 = 16 * b;
+                // rhs_b -= A_b,<b U_<b : 16 x kDVT outputs, two per thread
+                if (b > 0) {
+                    for (int x = tid; x < 16 * kDVT; x += kNT) {
+                        const int i = r0 + x / kDVT, j = x % kDVT;
+                        if (i < Cc) {
+                            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                            for (int m = 0; m < r0; m += 4) {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    a4[u] = fmaf(Am[i * kCS + m + u], Vs[(m + u) * kVS + j], a4[u]);
+                            }
+                            Vs[i * kVS + j] -= (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                        }
+                    }
+                    __syncthreads();
+                }
+                // U_b = D_b rhs_b (all reads before any write)
+                float val[16 * kDVT / kNT];
+#pragma unroll
+                for (int u = 0; u < 16 * kDVT / kNT; ++u) {
+                    const int x = tid + u * kNT;
+                    const int ii = x / kDVT, j = x % kDVT;
+                    const float* drow = Dm + (b * 16 + ii) * 17;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int t = 0; t < 16; t += 2) {
+                        if (t <= ii) a0 = fmaf(drow[t], Vs[(r0 + t) * kVS + j], a0);
+                        if (t + 1 <= ii) a1 = fmaf(drow[t + 1], Vs[(r0 + t + 1) * kVS + j], a1);
+                    }
+                    val[u] = a0 + a1;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int u = 0; u < 16 * kDVT / kNT; ++u) {
+                    const int x = tid + u * kNT;
+                    const int ii = x / kDVT, j = x % kDVT;
+                    if (r0 + ii < Cc) Vs[(r0 + ii) * kVS + j] = val[u];
+                }
+                __syncthreads();
             }
         }
-        __syncthreads();
         // ---- output: O = (Q * e^Gamma) S + P U ---------------------------
+        //      warp w: rows 8w .. 8w + 7 (Q and P rows as broadcast float4); lane: column
         {
-            const int j = lane;
-            for (int i = warp; i < Cc; i += kNT / 32) {
-                const float* qr = Qs + i * KS;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) acc += qr[c] * Ss[c * kVS + j];
-                if (GATE != kGatePerKey) acc *= eG[i];
-                const float* pr = Pm + i * kCS;
-                for (int m = 0; m <= i; ++m) acc += pr[m] * Vs[m * kVS + j];
-                st_elem(o + (tok0 + c0 + i) * DV + col0 + j, acc);
+            const int j = lane, i0 = warp * 8;
+            if (i0 < Cc) {
+                float acc[8], pu[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) acc[r] = pu[r] = 0.f;
+#pragma unroll 2
+                for (int c = 0; c < DK; c += 4) {
+                    const float s0 = Ss[c * kVS + j], s1 = Ss[(c + 1) * kVS + j];
+                    const float s2 = Ss[(c + 2) * kVS + j], s3 = Ss[(c + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float4 qv = *reinterpret_cast<const float4*>(Qs + (i0 + r) * KS + c);
+                        acc[r] = fmaf(qv.x, s0, fmaf(qv.y, s1, fmaf(qv.z, s2, fmaf(qv.w, s3, acc[r]))));
+                    }
+                }
+                // P U over positions 0 .. i0 + 7 (P is zero above the diagonal and past Cc,
+                // and so are the rows of U past Cc)
+                for (int m = 0; m < i0 + 8; m += 4) {
+                    const float u0 = Vs[m * kVS + j], u1 = Vs[(m + 1) * kVS + j];
+                    const float u2 = Vs[(m + 2) * kVS + j], u3 = Vs[(m + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float4 pv = *reinterpret_cast<const float4*>(Pm + (i0 + r) * kCS + m);
+                        pu[r] = fmaf(pv.x, u0, fmaf(pv.y, u1, fmaf(pv.z, u2, fmaf(pv.w, u3, pu[r]))));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int i = i0 + r;
+                    if (i < Cc) {
+                        const float a = (GATE != kGatePerKey) ? acc[r] * eG[i] : acc[r];
+                        st_elem(o + (tok0 + c0 + i) * DV + col0 + j, a + pu[r]);
+                    }
+                }
             }
         }
         if (GATE == kGatePerKey) {
@@ -310,17 +434,29 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         }
         __syncthreads();
         // ---- state: S <- Diag(e^Gamma_last) S + (K * e^(Gamma_last - Gamma))^T U
+        //      warp w: key channels 8w .. 8w + 7 (+ 64) (K rows as broadcast float4); lane: column
         {
             const int j = lane;
-            for (int c = warp; c < DK; c += kNT / 32) {
-                float acc = 0.f;
-                if (GATE == kGatePerKey) {
-                    for (int i = 0; i < Cc; ++i) acc += Kx[i * KS + c] * Vs[i * kVS + j];
-                    Ss[c * kVS + j] = expf(Gm[(Cc - 1) * KS + c]) * Ss[c * kVS + j] + acc;
-                } else {
-                    for (int i = 0; i < Cc; ++i) acc += Ks[i * KS + c] * eT[i] * Vs[i * kVS + j];
-                    const float dec = (GATE == kGateScalar) ? expf(Gm[Cc - 1]) : 1.f;
-                    Ss[c * kVS + j] = dec * Ss[c * kVS + j] + acc;
+            for (int cb = warp * 8; cb < DK; cb += 8 * (kNT / 32)) {
+                float acc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                const float* kb = (GATE == kGatePerKey) ? Kx : Ks;
+                for (int i = 0; i < Cc; ++i) {
+                    const float u = (GATE == kGatePerKey) ? Vs[i * kVS + j] : Vs[i * kVS + j] * eT[i];
+                    const float4 k0 = *reinterpret_cast<const float4*>(kb + i * KS + cb);
+                    const float4 k1 = *reinterpret_cast<const float4*>(kb + i * KS + cb + 4);
+                    acc[0] = fmaf(k0.x, u, acc[0]); acc[1] = fmaf(k0.y, u, acc[1]);
+                    acc[2] = fmaf(k0.z, u, acc[2]); acc[3] = fmaf(k0.w, u, acc[3]);
+                    acc[4] = fmaf(k1.x, u, acc[4]); acc[5] = fmaf(k1.y, u, acc[5]);
+                    acc[6] = fmaf(k1.z, u, acc[6]); acc[7] = fmaf(k1.w, u, acc[7]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = cb + e;
+                    const float dec = (GATE == kGatePerKey) ? expf(Gm[(Cc - 1) * KS + c])
+                                      : (GATE == kGateScalar) ? expf(Gm[Cc - 1]) : 1.f;
+                    Ss[c * kVS + j] = dec * Ss[c * kVS + j] + acc[e];
                 }
             }
         }
