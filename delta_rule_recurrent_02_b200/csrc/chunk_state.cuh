@@ -156,6 +156,8 @@ struct Args {
     const __nv_bfloat16* z = nullptr;
     const float* norm_w = nullptr;
     float eps = 0.f;
+    // with the prologue: the workspace's 1 / ||q_i|| rows, written by the WY tiles
+    const float* rq = nullptr;
 };
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
@@ -501,7 +503,12 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                           ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
-                float ssq[4] = {0.f, 0.f, 0.f, 0.f};
+                // with the prologue: the WY tile's 1 / ||q_i|| of this chunk's rows (published with
+                // the tile, whose flag the producer acquired before these tiles were loaded),
+                // requested now and stored into the gate slot before READY
+                float4 rq4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (PRO && sid < kC / 4)
+                    rq4 = reinterpret_cast<const float4*>(ar.rq + (tile0 + (int64_t)c * tstep) * kC)[sid];
                 // (with the per-key gate the workspace holds Qh already)
                 // (loads four at a time: the ld / st helpers keep their order, so one load per
                 // iteration would wait out each load's latency in turn)
@@ -523,9 +530,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
                         const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
                         const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                        if (PRO)
-                            ssq[uu] += (e0.x * e0.x + e0.y * e0.y + e1.x * e1.x + e1.y * e1.y) +
-                                       (e2.x * e2.x + e2.y * e2.y + e3.x * e3.x + e3.y * e3.y);
                         st_shared_v4(a[uu], pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
                                      pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                     }
@@ -554,20 +558,11 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                                      pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                     }
                 }
+                // 1 / ||q_i|| for the output rows, ordered before READY (and so before the
+                // products whose completion the output rows wait for)
+                if (PRO && sid < kC / 4) reinterpret_cast<float4*>(gs + rq_field(c))[sid] = rq4;
                 fence_async_smem();
                 mbar_arrive(ctl.bar(B_READY0 + s));
-                if (PRO) {
-                    // 1 / ||q_i|| of rows (sid / 8) + 16 u4 from the raw values just read, for the
-                    // output rows: 8 threads share a row (one 16-byte chunk of each d-block each)
-#pragma unroll
-                    for (int u4 = 0; u4 < 4; ++u4) {
-                        float s2 = ssq[u4];
-                        s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
-                        s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
-                        s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
-                        if ((sid & 7) == 0) gs[rq_field(c) + (sid >> 3) + 16 * u4] = fminf(rsqrtf(s2), 1e12f);
-                    }
-                }
             }
             if (!kSplitOut && c >= 1) {
                 // ---- output rows of chunk c - 1 --------------------------------------------

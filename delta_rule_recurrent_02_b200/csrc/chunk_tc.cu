@@ -42,7 +42,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
                          gam, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, vl, vl_N,
-                         pro.norm, pro.z, pro.norm_w, pro.eps};
+                         pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq};
     state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
 }
 
@@ -134,11 +134,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // the later ones come from tickets, in order (chunk-major), to whichever group is free
     const int64_t G = (int64_t)(gridDim.x - BH) * 4 + (HOSTED ? BH : 0);   // WY groups in the grid
     const wy::Args wa{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags,
-                      flags + tiles, BH, (int)G, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep};
+                      flags + tiles, BH, (int)G, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, nullptr, 0,
+                      pro.rq};
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H,
-                             pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps};
+                             pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq};
         if constexpr (!HOSTED) {
             // ---- state pass of head blockIdx.x --------------------------------------------
             if (warp >= state::Roles<GATE, false, PRO>::kNT / 32) return;
@@ -310,6 +311,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         !make_tmap(&m.u, u_ws, kC, tiles * kD, 128) || !make_tmap(&m.p, p_ws, kC, tiles * kC, 64))
         return cudaErrorInvalidValue;
     m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
+    m.rq_ws = reinterpret_cast<float*>(p_ws + tiles * kWsPBytes);
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles));
     if (packed) {
         // the chunk tables, then all WY tiles, then one state pass per (sequence, head)
@@ -327,7 +329,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         kern<<<(unsigned)(a.N * a.H), state::Roles<GATE, false, PRO>::kNT, bytes, st>>>(
             m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0, static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
             a.scale, a.status, a.test_flags, nullptr, nullptr, 1, 0,
-            prologue_of(a), vl, a.N);
+            prologue_of(a, m), vl, a.N);
         return counted(cudaGetLastError());
     }
 
@@ -363,7 +365,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
             unsigned int* status = a.status;
             float* snaps = a.snaps;
             int snap_every = a.snap_every, n_snap = a.n_snap;
-            Prologue pro = prologue_of(a);
+            Prologue pro = prologue_of(a, m);
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &p_out, &flags, &bh_i, &beta, &g, &S0, &o, &S_T,
                             &T_i, &n_i, &scale, &status, &test_flags, &snaps, &snap_every, &n_snap, &pro};
             // the flags are cleared on the same stream right before the launch
@@ -383,7 +385,7 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
     kern<<<(unsigned)BH, state::Roles<GATE, false, PRO>::kNT, bytes, st>>>(m.k, m.q, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                   static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T, a.scale,
                                                   a.status, a.test_flags, nullptr, a.snaps, a.snap_every, a.n_snap,
-                                                  prologue_of(a),
+                                                  prologue_of(a, m),
                                                   nullptr, 0);
     return counted(cudaGetLastError());
 }
@@ -397,7 +399,7 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     uint8_t* w_ws = static_cast<uint8_t*>(a.ws);
     uint8_t* u_ws = w_ws + tiles * kWsWBytes;
     uint8_t* p_ws = u_ws + tiles * kWsUBytes;
-    uint8_t* kt_ws = p_ws + tiles * kWsPBytes;
+    uint8_t* kt_ws = p_ws + tiles * (kWsPBytes + kWsRqBytes);
     uint8_t* qh_ws = kt_ws + tiles * kWsKtBytes;
     uint8_t* gam_ws = qh_ws + tiles * kWsQhBytes;
     TcMaps m;

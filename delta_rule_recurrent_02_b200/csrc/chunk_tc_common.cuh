@@ -25,10 +25,13 @@ constexpr uint64_t kWaitNs = 1000000000ull; // every mbarrier wait gives up afte
 //   -W   [tiles * 64 rows (position)][128 (d_k)]
 //   u^T  [tiles * 128 rows (d_v)][64 (position)]
 //   P    [tiles * 64 rows (i)][64 (j)]
+//   rq   [tiles][64]  1 / max(||q_i||, 1e-12) of the tile's rows (fp32; written
+//        only with the layer's prologue, for the state pass's output rows)
 constexpr size_t kWsWBytes = (size_t)kC * kD * 2;
 constexpr size_t kWsUBytes = (size_t)kD * kC * 2;
 constexpr size_t kWsPBytes = (size_t)kC * kC * 2;
-constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes;
+constexpr size_t kWsRqBytes = (size_t)kC * 4;
+constexpr size_t kWsTileBytes = kWsWBytes + kWsUBytes + kWsPBytes + kWsRqBytes;
 // With the per-key gate (KDA) three more arrays follow, which the state pass
 // reads in place of q and k and of the scalar decays:
 //   K~   [tiles * 64 rows][128]  k (.) e^(Gamma_last - Gamma)      (bf16)
@@ -67,6 +70,7 @@ struct TcMaps {
     float* gam_ws;
     // a packed batch only: the workspace's chunk tables (VarlenTables), else null
     const int* vl = nullptr;
+    float* rq_ws = nullptr;  // the workspace's rq array
 };
 
 // The Gated DeltaNet layer's prologue, fused into the prefill kernels (scalar
@@ -84,6 +88,7 @@ struct Prologue {
     const __nv_bfloat16* z = nullptr;
     const float* norm_w = nullptr;
     float eps = 0.f;
+    float* rq = nullptr;     // the workspace's 1 / ||q_i|| per tile row (with the prologue)
 };
 
 // Chunk tables of a packed batch of N sequences, built on the device from
@@ -104,12 +109,13 @@ inline int64_t vl_chunks_max(int64_t T, int N) { return T / kC + N; }
 inline size_t vl_table_ints(int N, int64_t nc_max) { return 2 * (size_t)(N + 1) + (size_t)nc_max; }
 
 // The Prologue argument of the tensor-core kernels for a request.
-inline Prologue prologue_of(const ChunkArgs& a) {
+inline Prologue prologue_of(const ChunkArgs& a, const TcMaps& m) {
     Prologue p{a.prologue, a.A_log, a.dt_bias, (int)a.H, a.rep};
     p.norm = a.norm;
     p.z = static_cast<const __nv_bfloat16*>(a.z);
     p.norm_w = a.norm_weight;
     p.eps = a.eps;
+    if (a.prologue) p.rq = m.rq_ws;
     return p;
 }
 

@@ -42,7 +42,7 @@ chunk_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     x.tmem = *tmem_slot;
     const Args ar{&tm_q, &tm_k, &tm_v, &tm_w, &tm_u, p_out, flags, beta, g, T, n, scale, test_flags, nullptr,
-                  BH, 0, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, vl, vl_N};
+                  BH, 0, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, vl, vl_N, pro.rq};
     // chunk-major order: chunk 0 of every head first
     const int c = (int)(blockIdx.x / (unsigned)BH);
     const int64_t bh = blockIdx.x - (int64_t)c * BH;
@@ -74,7 +74,7 @@ cudaError_t launch_wy_gate(const ChunkArgs& a, const TcMaps& m, int n, cudaStrea
     const int64_t chunks = a.cu_seqlens ? vl_chunks_max(a.T, a.N) : n;
     kern<<<(unsigned)(a.B * a.H * chunks), kNT, SMEM_BYTES, st>>>(
         m.q, m.k, m.v, m.w, m.u, m.p_ws, m.flags, (int)(a.B * a.H), a.beta, a.g, (int)a.T, n, a.scale, a.status,
-        a.test_flags, prologue_of(a), m.vl, a.N);
+        a.test_flags, prologue_of(a, m), m.vl, a.N);
     return counted(cudaGetLastError());
 }
 

@@ -190,6 +190,7 @@ struct Args {
     // index and bh the head
     const int* vl = nullptr;
     int vl_N = 0;
+    float* rq = nullptr;     // with the prologue: the workspace's 1 / ||q_i|| rows
 };
 
 // Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
@@ -401,13 +402,15 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         }
     }
     if (PRO) {
-        // 1 / ||k_i|| and 1 / ||q_i|| from the tiles (rows 0-63 K, 64-127 Q of each d-block),
-        // two threads per row, while the gram runs
+        // 1 / ||k_i|| (threads 0-127) and 1 / ||q_i|| (128-255) from the [K0 | Q0 | K1 | Q1]
+        // tiles, two threads per row, while the gram runs; r_k stays in the gate slot, r_q
+        // goes to the workspace (published with the tile) for the state pass's output rows
         if (ctl.wait(B_FULL, 0)) {
-            if (tid < 2 * kC) {
-                const int r = tid >> 1;
-                const float rn = inv_row_norm(sb + OFF_KV, r, tid & 1, 16384);
-                if ((tid & 1) == 0) gs[G_RK + r] = rn;
+            const int r = (tid & 127) >> 1, which = tid >> 7;
+            const float rn = inv_row_norm(sb + OFF_KV + (uint32_t)which * 8192u, r, tid & 1, 16384);
+            if ((tid & 1) == 0) {
+                if (which == 0) gs[G_RK + r] = rn;
+                else if (ar.rq) ar.rq[tile * kC + r] = rn;
             }
         } else {
             ok = false;

@@ -122,13 +122,14 @@ DN_API int dn_chunk_fwd(const void* q, const void* k, const void* v,
  * tensor-core path computes W = T diag(beta e^G) K, u = T diag(beta) V and the
  * intra-chunk attention P of every chunk ("Training it: the WY trick", D2L
  * 12.5; "The chunked form", ch. 28) in a kernel that runs over all chunks at
- * once, then streams them into the sequential state pass: 40 KiB and a 4-byte
+ * once, then streams them into the sequential state pass: 40.25 KiB (W, u, P and,
+ * for the layer prologue's output rows, 1 / ||q|| of each position) and a 4-byte
  * ready flag per (b, h, chunk), and a 4-byte tile counter, i.e. with
- * n = B * H * ceil(T / 64) chunks, n * 40960 + (4 (n + 1) rounded up to a
+ * n = B * H * ceil(T / 64) chunks, n * 41216 + (4 (n + 1) rounded up to a
  * multiple of 256) bytes.  With the per-key
  * gate (KDA: "A walk through of the DeltaNet family of linear attention
  * variants") each chunk also keeps q and k with their decays applied and the
- * chunk's decay per key channel: 72.5 KiB per chunk, n * 74240 + (4 (n + 1)
+ * chunk's decay per key channel: 72.75 KiB per chunk, n * 74496 + (4 (n + 1)
  * rounded up to a multiple of 256) bytes.  Its gram splits the decays around one
  * reference position per 16-token block, so the tensor-core result is exact up
  * to rounding while no key channel decays by more than e^-80 over 8
@@ -485,7 +486,8 @@ DN_API const char* dn_last_error(void);
  * 2.3: dn_chunk_fwd_snapshots; 2.4: dn_chunk_fwd_gdn; 2.5: dn_decode_step_gdn;
  * 2.6: dn_causal_conv1d, dn_rms_norm_gated; 2.7: dn_chunk_fwd_gva, dn_decode_step_gva,
  * dn_chunk_fwd_gdn_ex, dn_decode_step_gdn_ex (the CUDA-core prologue and the 2 sigmoid gate),
- * dn_chunk_fwd_varlen, dn_chunk_fwd_varlen_workspace_size, dn_chunk_fwd_general. */
+ * dn_chunk_fwd_varlen, dn_chunk_fwd_varlen_workspace_size, dn_chunk_fwd_general; 2.8: 256 more
+ * workspace bytes per tensor-core chunk (1 / ||q|| of its positions, for the layer prologue). */
 DN_API int dn_version(void);
 
 /*

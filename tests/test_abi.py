@@ -84,7 +84,7 @@ WS = A + 8 * STEP
     (dict(dv=256), dn.DN_ERR_UNSUPPORTED),
     (dict(path=2), dn.DN_ERR_UNSUPPORTED),                    # tensor-core path needs bf16, d = 128
     (dict(path=3), dn.DN_ERR_UNSUPPORTED),                    # so does its self-test
-    (dict(TC, ws=WS, ws_bytes=40960 + 255), dn.DN_ERR_INVALID),     # workspace smaller than one chunk's tiles
+    (dict(TC, ws=WS, ws_bytes=41216 + 255), dn.DN_ERR_INVALID),     # workspace smaller than one chunk's tiles
     (dict(TC, ws=WS + 128, ws_bytes=1 << 20), dn.DN_ERR_INVALID),   # not 256-byte aligned
     (dict(TC, ws=A + 256, ws_bytes=1 << 20), dn.DN_ERR_INVALID),    # overlaps q
     (dict(TC, ws=A + 6 * STEP, ws_bytes=1 << 20), dn.DN_ERR_INVALID),  # overlaps S_T
@@ -104,13 +104,13 @@ def ws_size(lib, B=2, T=130, H=3, dk=128, dv=128, chunk=64, dtype=1, gate=1, pat
 
 def test_workspace_size():
     lib = dn.load_library()
-    # -W and u^T (bf16, 64 x 128 each) and P (bf16, 64 x 64) per (b, h, chunk), then
+    # -W and u^T (bf16, 64 x 128 each), P (bf16, 64 x 64) and 1 / ||q|| (fp32, 64) per (b, h, chunk), then
     # a 4-byte ready flag per chunk rounded up to 256 bytes: ceil(130 / 64) = 3 chunks
     tiles = 2 * 3 * 3
-    assert ws_size(lib) == (dn.DN_OK, tiles * (2 * 64 * 128 + 64 * 64) * 2 + 256)
-    assert ws_size(lib, path=2) == (dn.DN_OK, tiles * 40960 + 256)
+    assert ws_size(lib) == (dn.DN_OK, tiles * ((2 * 64 * 128 + 64 * 64) * 2 + 64 * 4) + 256)
+    assert ws_size(lib, path=2) == (dn.DN_OK, tiles * 41216 + 256)
     # per-key gate: also K~ and Qh (bf16, 64 x 128 each) and e^Gamma_last (fp32, 128) per chunk
-    assert ws_size(lib, gate=2, path=2) == (dn.DN_OK, tiles * (40960 + 2 * 16384 + 512) + 256)
+    assert ws_size(lib, gate=2, path=2) == (dn.DN_OK, tiles * (41216 + 2 * 16384 + 512) + 256)
     assert ws_size(lib, gate=2, path=1) == (dn.DN_OK, 0)
     assert ws_size(lib, T=0) == (dn.DN_OK, 0)
     assert ws_size(lib, path=1) == (dn.DN_OK, 0)             # SIMT needs none
@@ -119,7 +119,7 @@ def test_workspace_size():
     assert ws_size(lib, dtype=0, path=2)[0] == dn.DN_ERR_UNSUPPORTED
     assert ws_size(lib, B=-1) == (dn.DN_ERR_INVALID, 12345)  # not written on failure
     assert lib.dn_chunk_fwd_workspace_size(1, 8, 1, 128, 128, 64, 1, 1, 0, None) == dn.DN_ERR_INVALID
-    assert dn.dn_chunk_fwd_workspace_size(1, 64, 1, 128, 128) == 40960 + 256
+    assert dn.dn_chunk_fwd_workspace_size(1, 64, 1, 128, 128) == 41216 + 256
 
 
 def test_chunk_fwd_empty_batch_is_ok_without_device(lib):
@@ -376,9 +376,9 @@ def test_varlen_rejects_before_device_work(lib, over, code):
 def test_varlen_workspace_size_depends_on_N_and_T(lib):
     out = ctypes.c_size_t(0)
     assert lib.dn_chunk_fwd_varlen_workspace_size(3, 200, 2, 128, 128, 1, 1, ctypes.byref(out)) == dn.DN_OK
-    # at most 200 / 64 + 3 = 6 chunks per head: 12 tiles of 40 KiB, their flags, then the tables
+    # at most 200 / 64 + 3 = 6 chunks per head: 12 tiles of 40.25 KiB, their flags, then the tables
     tiles = 2 * (200 // 64 + 3)
-    assert out.value >= tiles * 40960 + 4 * (tiles + 1)
+    assert out.value >= tiles * 41216 + 4 * (tiles + 1)
     big = ctypes.c_size_t(0)
     assert lib.dn_chunk_fwd_varlen_workspace_size(30, 200, 2, 128, 128, 1, 1, ctypes.byref(big)) == dn.DN_OK
     assert big.value > out.value

@@ -152,7 +152,7 @@ def test_tc_workspace_caller_internal_and_poisoned(cuda_device):
     d = to_dev(inp)
     sc = 128 ** -0.5
     nbytes = dn.dn_chunk_fwd_workspace_size(2, 200, 3, 128, 128, path="tc")
-    assert nbytes == 2 * 3 * 4 * 40960 + 256
+    assert nbytes == 2 * 3 * 4 * 41216 + 256
     ws = torch.full((nbytes // 2,), float("nan"), dtype=torch.bfloat16, device="cuda")
     outs = []
     for w in (ws, None):

@@ -95,7 +95,7 @@ def test_noalloc_matches_dn_chunk_fwd_on_two_calls(cuda_device, gate):
 
 
 def test_noalloc_rejects_requests_above_its_scratch_area():
-    # 32 heads x 1024 chunks x 40 KiB, plus a 4-byte flag per chunk and a tile counter, is
+    # 32 heads x 1024 chunks x 40.25 KiB, plus a 4-byte flag per chunk and a tile counter, is
     # 1.25 GiB of scratch, above the fixed 64 MiB: refused before any device work (the fake
     # addresses are never used)
     lib, f = noalloc_fn()
@@ -105,5 +105,5 @@ def test_noalloc_rejects_requests_above_its_scratch_area():
     assert st == dn.DN_ERR_UNSUPPORTED
     msg = lib.dn_last_error().decode()
     n = 32 * 1024
-    need = n * 40960 + (4 * (n + 1) + 255) // 256 * 256
+    need = n * 41216 + (4 * (n + 1) + 255) // 256 * 256
     assert str(need) in msg and str(64 << 20) in msg
