@@ -28,6 +28,13 @@
 // of S evolve independently); the state slice stays in shared memory for the
 // whole sequence.  Chunks of 1..32 tokens (the five key-side tiles of a chunk
 // are kept in shared memory).  A partial last chunk just has fewer rows.
+//
+// Once the pairwise sums are formed, the key-side tiles are replaced in place by
+// their decayed forms (q e^G, kappa e^Gp, k e^(G_C - G), l e^(G_C - G)), so that
+// the right-hand side, the output rows and the state update are plain sums of
+// products; those read 4 rows a warp as float4 broadcasts (rows padded to a
+// multiple of 4 floats), one value column per lane.  The system is solved by
+// 16-row blocks: the diagonal inverses at once, then block after block.
 #include "dn_common.cuh"
 #include "dn_kernels.h"
 
@@ -39,11 +46,11 @@ constexpr int kNT = 256;     // threads per CTA
 constexpr int kDVT = 32;     // value columns per CTA
 constexpr int kCmax = 32;    // largest chunk
 constexpr int kVS = kDVT + 1;
-constexpr int kCS = kCmax + 1;
+constexpr int kCS = kCmax + 4;   // rows of M, N, Pk, Pl: 16-byte aligned
 
 template <int DK>
 struct GenSmem {
-    static constexpr int KS = DK + 1;
+    static constexpr int KS = DK + 4;
     static constexpr int kQ = 0;                           // q        [Cmax][KS]
     static constexpr int kR = kQ + kCmax * KS;             // kappa    [Cmax][KS]
     static constexpr int kL = kR + kCmax * KS;             // a*kappa  [Cmax][KS]
@@ -56,7 +63,8 @@ struct GenSmem {
     static constexpr int kPk = kN + kCmax * kCS;           // Pk       [Cmax][CS]
     static constexpr int kPl = kPk + kCmax * kCS;          // Pl       [Cmax][CS]
     static constexpr int kS = kPl + kCmax * kCS;           // S slice  [DK][VS]
-    static constexpr int kTotal = kS + DK * kVS;
+    static constexpr int kD = kS + DK * kVS;               // (I + M_bb)^-1 [2 blocks][16][17]
+    static constexpr int kTotal = kD + 2 * 16 * 17;
     static constexpr size_t bytes = sizeof(float) * kTotal;
 };
 
@@ -80,6 +88,7 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
     float* Pk = sm + L::kPk;
     float* Pl = sm + L::kPl;
     float* Ss = sm + L::kS;
+    float* Dm = sm + L::kD;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -107,9 +116,9 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
             Ws[i * KS + c] = ld_elem(kw + off);
             Gm[i * KS + c] = wlog[off];
         }
-        for (int x = tid; x < Cc * kDVT; x += kNT) {
+        for (int x = tid; x < kCmax * kDVT; x += kNT) {
             const int i = x / kDVT, j = x % kDVT;
-            Vs[i * kVS + j] = ld_elem(v + (tok0 + c0 + i) * DV + col0 + j);
+            Vs[i * kVS + j] = i < Cc ? ld_elem(v + (tok0 + c0 + i) * DV + col0 + j) : 0.f;
         }
         __syncthreads();
         // ---- G: inclusive prefix sum of the log-decays over the chunk, per channel -----
@@ -122,10 +131,10 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
         }
         __syncthreads();
         // ---- pairwise sums over channels: M, N (j < i), Pk, Pl (j <= i) ---------------
-        for (int p = tid; p < Cc * Cc; p += kNT) {
-            const int i = p / Cc, j = p % Cc;
+        for (int p = tid; p < kCmax * kCmax; p += kNT) {
+            const int i = p / kCmax, j = p % kCmax;
             float m = 0.f, nn = 0.f, pk = 0.f, pl = 0.f;
-            if (j <= i) {
+            if (j <= i && i < Cc) {
                 const float* gi = Gm + i * KS;
                 const float* gj = Gm + j * KS;
                 const float* gp = i > 0 ? Gm + (i - 1) * KS : nullptr;   // Gp_i = G_{i-1}
@@ -135,11 +144,11 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
                 const float* wj = Ws + j * KS;
 #pragma unroll 4
                 for (int c = 0; c < DK; ++c) {
-                    const float e2 = expf(gi[c] - gj[c]);
+                    const float e2 = __expf(gi[c] - gj[c]);
                     pk += qi[c] * e2 * wj[c];
                     pl += qi[c] * e2 * lj[c];
                     if (j < i) {
-                        const float e1 = expf(gp[c] - gj[c]);
+                        const float e1 = __expf(gp[c] - gj[c]);
                         m += ri[c] * e1 * lj[c];
                         nn += ri[c] * e1 * wj[c];
                     }
@@ -151,66 +160,179 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
             Pl[i * kCS + j] = scale * pl;
         }
         __syncthreads();
-        // ---- right-hand side: (kappa * e^Gp) S_0 + N V ---------------------------------
+        // ---- the decayed tiles, in place (the raw ones are read for the last time above):
+        //      q e^G (output), kappa e^Gp (right-hand side), k and l times e^(G_C - G) (state)
+        for (int x = tid; x < Cc * DK; x += kNT) {
+            const int i = x / DK, c = x % DK;
+            const float gi = Gm[i * KS + c], gc = Gm[(Cc - 1) * KS + c];
+            const float gp = i > 0 ? Gm[(i - 1) * KS + c] : 0.f;
+            const float ed = __expf(gc - gi);
+            Qs[i * KS + c] *= __expf(gi);
+            Rs[i * KS + c] *= __expf(gp);
+            Ws[i * KS + c] *= ed;
+            Ls[i * KS + c] *= ed;
+        }
+        __syncthreads();
+        // e^(G_C) per channel, for the state's decay (row 0 of G is free now)
+        for (int c = tid; c < DK; c += kNT) Gm[c] = __expf(Gm[(Cc - 1) * KS + c]);
+        // ---- right-hand side: (kappa e^Gp) S_0 + N V; warp w: rows 4w .. 4w + 3, lane: column
         {
-            const int j = lane;
-            for (int i = warp; i < Cc; i += kNT / 32) {
-                const float* ri = Rs + i * KS;
-                float acc = 0.f;
-                if (i > 0) {
-                    const float* gp = Gm + (i - 1) * KS;
-#pragma unroll 8
-                    for (int c = 0; c < DK; ++c) acc += ri[c] * expf(gp[c]) * Ss[c * kVS + j];
-                } else {
-#pragma unroll 8
-                    for (int c = 0; c < DK; ++c) acc += ri[c] * Ss[c * kVS + j];
+            const int j = lane, i0 = warp * 4;
+            if (i0 < Cc) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+                for (int c = 0; c < DK; c += 4) {
+                    const float s0 = Ss[c * kVS + j], s1 = Ss[(c + 1) * kVS + j];
+                    const float s2 = Ss[(c + 2) * kVS + j], s3 = Ss[(c + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float4 rv = *reinterpret_cast<const float4*>(Rs + (i0 + r) * KS + c);
+                        acc[r] = fmaf(rv.x, s0, fmaf(rv.y, s1, fmaf(rv.z, s2, fmaf(rv.w, s3, acc[r]))));
+                    }
                 }
-                for (int m = 0; m < i; ++m) acc += Nm[i * kCS + m] * Vs[m * kVS + j];
-                Us[i * kVS + j] = acc;
-            }
-        }
-        __syncthreads();
-        // ---- forward substitution (I + M) U = rhs, 4 columns per warp ----------------
-        {
-            const int j = warp * 4 + (lane >> 3);
-            const int part = lane & 7;
-            for (int i = 1; i < Cc; ++i) {
-                float acc = 0.f;
-                for (int m = part; m < i; m += 8) acc += Mm[i * kCS + m] * Us[m * kVS + j];
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (part == 0) Us[i * kVS + j] -= acc;
-                __syncwarp();
-            }
-        }
-        __syncthreads();
-        // ---- output: scale (q * e^G) S_0 + Pk V - Pl U --------------------------------
-        {
-            const int j = lane;
-            for (int i = warp; i < Cc; i += kNT / 32) {
-                const float* qi = Qs + i * KS;
-                const float* gi = Gm + i * KS;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) acc += qi[c] * expf(gi[c]) * Ss[c * kVS + j];
-                acc *= scale;
-                for (int m = 0; m <= i; ++m) acc += Pk[i * kCS + m] * Vs[m * kVS + j] - Pl[i * kCS + m] * Us[m * kVS + j];
-                st_elem(o + (tok0 + c0 + i) * DV + col0 + j, acc);
-            }
-        }
-        __syncthreads();
-        // ---- state: e^(G_C) * S_0 + sum_s (e^(G_C - G_s) * k_s) v_s^T - (e^(G_C - G_s) * l_s) U_s
-        {
-            const int j = lane;
-            const float* gl = Gm + (Cc - 1) * KS;
-            for (int c = warp; c < DK; c += kNT / 32) {
-                float acc = 0.f;
-                for (int s = 0; s < Cc; ++s) {
-                    const float e = expf(gl[c] - Gm[s * KS + c]);
-                    acc += e * (Ws[s * KS + c] * Vs[s * kVS + j] - Ls[s * KS + c] * Us[s * kVS + j]);
+                // N V over positions < i0 + 4 (N is zero on and above the diagonal and past Cc)
+                for (int m = 0; m < i0 + 4; m += 4) {
+                    const float v0 = Vs[m * kVS + j], v1 = Vs[(m + 1) * kVS + j];
+                    const float v2 = Vs[(m + 2) * kVS + j], v3 = Vs[(m + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float4 nv = *reinterpret_cast<const float4*>(Nm + (i0 + r) * kCS + m);
+                        acc[r] = fmaf(nv.x, v0, fmaf(nv.y, v1, fmaf(nv.z, v2, fmaf(nv.w, v3, acc[r]))));
+                    }
                 }
-                Ss[c * kVS + j] = expf(gl[c]) * Ss[c * kVS + j] + acc;
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (i0 + r < Cc) Us[(i0 + r) * kVS + j] = acc[r];
+            }
+        }
+        __syncthreads();
+        // ---- (I + M) U = rhs by 16-row blocks: both diagonal inverses at once (one warp a
+        //      block, lane = column), then U_b = D_b (rhs_b - M_b,<b U_<b) -----------------
+        {
+            const int nb = (Cc + 15) >> 4;
+            if (warp < nb && lane < 16) {
+                const int k0 = warp * 16, jj = lane;
+                float xr[16];
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) {
+                    float p0 = ii == jj ? 1.f : 0.f, p1 = 0.f;
+                    if (k0 + ii < Cc) {
+#pragma unroll
+                        for (int m = 0; m < ii; m += 2) {
+                            p0 -= Mm[(k0 + ii) * kCS + k0 + m] * xr[m];
+                            if (m + 1 < ii) p1 -= Mm[(k0 + ii) * kCS + k0 + m + 1] * xr[m + 1];
+                        }
+                    }
+                    xr[ii] = p0 + p1;
+                }
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) Dm[(warp * 16 + ii) * 17 + jj] = xr[ii];
+            }
+            __syncthreads();
+            for (int bb = 0; bb < nb; ++bb) {
+                const int r0 = 16 * bb;
+                if (bb > 0) {
+                    for (int x = tid; x < 16 * kDVT; x += kNT) {
+                        const int i = r0 + x / kDVT, j = x % kDVT;
+                        if (i < Cc) {
+                            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                            for (int m = 0; m < r0; m += 4) {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    a4[u] = fmaf(Mm[i * kCS + m + u], Us[(m + u) * kVS + j], a4[u]);
+                            }
+                            Us[i * kVS + j] -= (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                        }
+                    }
+                    __syncthreads();
+                }
+                float val[16 * kDVT / kNT];
+#pragma unroll
+                for (int u = 0; u < 16 * kDVT / kNT; ++u) {
+                    const int x = tid + u * kNT;
+                    const int ii = x / kDVT, j = x % kDVT;
+                    const float* drow = Dm + (bb * 16 + ii) * 17;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int t = 0; t < 16; t += 2) {
+                        if (t <= ii && r0 + t < Cc) a0 = fmaf(drow[t], Us[(r0 + t) * kVS + j], a0);
+                        if (t + 1 <= ii && r0 + t + 1 < Cc) a1 = fmaf(drow[t + 1], Us[(r0 + t + 1) * kVS + j], a1);
+                    }
+                    val[u] = a0 + a1;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int u = 0; u < 16 * kDVT / kNT; ++u) {
+                    const int x = tid + u * kNT;
+                    const int ii = x / kDVT, j = x % kDVT;
+                    if (r0 + ii < Cc) Us[(r0 + ii) * kVS + j] = val[u];
+                }
+                __syncthreads();
+            }
+            // rows of U past a short chunk are zero for the products below
+            for (int x = Cc * kDVT + tid; x < kCmax * kDVT; x += kNT) Us[(x / kDVT) * kVS + x % kDVT] = 0.f;
+            __syncthreads();
+        }
+        // ---- output: scale (q e^G) S_0 + Pk V - Pl U (Pk, Pl carry the scale); warp w: rows
+        //      4w .. 4w + 3, lane: column --------------------------------------------------
+        {
+            const int j = lane, i0 = warp * 4;
+            if (i0 < Cc) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f}, pv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+                for (int c = 0; c < DK; c += 4) {
+                    const float s0 = Ss[c * kVS + j], s1 = Ss[(c + 1) * kVS + j];
+                    const float s2 = Ss[(c + 2) * kVS + j], s3 = Ss[(c + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float4 qv = *reinterpret_cast<const float4*>(Qs + (i0 + r) * KS + c);
+                        acc[r] = fmaf(qv.x, s0, fmaf(qv.y, s1, fmaf(qv.z, s2, fmaf(qv.w, s3, acc[r]))));
+                    }
+                }
+                for (int m = 0; m < i0 + 4; m += 4) {
+                    const float v0 = Vs[m * kVS + j], v1 = Vs[(m + 1) * kVS + j];
+                    const float v2 = Vs[(m + 2) * kVS + j], v3 = Vs[(m + 3) * kVS + j];
+                    const float u0 = Us[m * kVS + j], u1 = Us[(m + 1) * kVS + j];
+                    const float u2 = Us[(m + 2) * kVS + j], u3 = Us[(m + 3) * kVS + j];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float4 kv = *reinterpret_cast<const float4*>(Pk + (i0 + r) * kCS + m);
+                        const float4 lv = *reinterpret_cast<const float4*>(Pl + (i0 + r) * kCS + m);
+                        pv[r] = fmaf(kv.x, v0, fmaf(kv.y, v1, fmaf(kv.z, v2, fmaf(kv.w, v3, pv[r]))));
+                        pv[r] = fmaf(-lv.x, u0, fmaf(-lv.y, u1, fmaf(-lv.z, u2, fmaf(-lv.w, u3, pv[r]))));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (i0 + r < Cc) st_elem(o + (tok0 + c0 + i0 + r) * DV + col0 + j, scale * acc[r] + pv[r]);
+            }
+        }
+        __syncthreads();
+        // ---- state: e^(G_C) * S_0 + sum_s (k e^(G_C - G))_s v_s^T - (l e^(G_C - G))_s U_s;
+        //      warp w: key channels 16w .. 16w + 15 (+ 128), lane: column ----------------
+        {
+            const int j = lane;
+            for (int cb = warp * 16; cb < DK; cb += 16 * (kNT / 32)) {
+                float acc[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+                for (int s2 = 0; s2 < Cc; ++s2) {
+                    const float vv = Vs[s2 * kVS + j], uu = Us[s2 * kVS + j];
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 kw4 = *reinterpret_cast<const float4*>(Ws + s2 * KS + cb + 4 * e4);
+                        const float4 l4 = *reinterpret_cast<const float4*>(Ls + s2 * KS + cb + 4 * e4);
+                        acc[4 * e4 + 0] = fmaf(kw4.x, vv, fmaf(-l4.x, uu, acc[4 * e4 + 0]));
+                        acc[4 * e4 + 1] = fmaf(kw4.y, vv, fmaf(-l4.y, uu, acc[4 * e4 + 1]));
+                        acc[4 * e4 + 2] = fmaf(kw4.z, vv, fmaf(-l4.z, uu, acc[4 * e4 + 2]));
+                        acc[4 * e4 + 3] = fmaf(kw4.w, vv, fmaf(-l4.w, uu, acc[4 * e4 + 3]));
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int c = cb + e;
+                    Ss[c * kVS + j] = Gm[c] * Ss[c * kVS + j] + acc[e];
+                }
             }
         }
     }
