@@ -250,9 +250,9 @@ DN_API int dn_chunk_fwd_gdn_ex(const void* q, const void* k, const void* v, cons
  *   - Every call looks up the area's address (cudaGetSymbolAddress, with the
  *     call's device current) and keeps nothing: after a cudaDeviceReset the
  *     library's code is loaded again and the area may have moved.
- *   - Capacity: a (b, h, chunk) tile takes 40,960 bytes with no gate or the
- *     scalar gate (about 1638 tiles fit, e.g. B*H = 12 at T = 8192) and
- *     74,240 bytes with the per-key gate (about 903 tiles, e.g. B*H = 7 at
+ *   - Capacity: a (b, h, chunk) tile takes 41,216 bytes with no gate or the
+ *     scalar gate (about 1628 tiles fit, e.g. B*H = 12 at T = 8192) and
+ *     74,496 bytes with the per-key gate (about 900 tiles, e.g. B*H = 7 at
  *     T = 8192), plus 4 bytes of ready flag per tile.
  *   - A request needing more scratch than the area returns DN_ERR_UNSUPPORTED
  *     (dn_last_error() gives both sizes) before any device work.
