@@ -469,7 +469,7 @@ def test_gdn_prologue_ex_rejects_unknown_flags(cuda_device):
 
 
 @pytest.mark.parametrize("activation", ["silu", "sigmoid"])
-@pytest.mark.parametrize("B,H,T", [(2, 3, 150), (1, 2, 64), (3, 32, 100), (4, 16, 1024)])
+@pytest.mark.parametrize("B,H,T", [(2, 3, 150), (1, 2, 64), (3, 32, 100), (4, 16, 1024), (4, 32, 130)])
 def test_gdn_prologue_and_gated_norm(cuda_device, activation, B, H, T):
     # dn_chunk_fwd_gdn_ex with z: the layer's prologue, the rule and the gated RMSNorm
     # ("The full layer", steps 4-7) in the tensor-core kernels, against
