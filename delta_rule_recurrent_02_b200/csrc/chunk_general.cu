@@ -130,27 +130,52 @@ chunk_general_kernel(const Tin* __restrict__ q, const float* __restrict__ wlog, 
             }
         }
         __syncthreads();
-        // ---- pairwise sums over channels: M, N (j < i), Pk, Pl (j <= i) ---------------
+        // ---- pairwise sums over channels: M, N (j < i), Pk, Pl (j <= i), read as float4 along
+        //      the channels (row j per lane: distinct bank groups; row i broadcast) -----------
         for (int p = tid; p < kCmax * kCmax; p += kNT) {
             const int i = p / kCmax, j = p % kCmax;
             float m = 0.f, nn = 0.f, pk = 0.f, pl = 0.f;
             if (j <= i && i < Cc) {
                 const float* gi = Gm + i * KS;
                 const float* gj = Gm + j * KS;
-                const float* gp = i > 0 ? Gm + (i - 1) * KS : nullptr;   // Gp_i = G_{i-1}
-                const float* ri = Rs + i * KS;
                 const float* qi = Qs + i * KS;
                 const float* lj = Ls + j * KS;
                 const float* wj = Ws + j * KS;
-#pragma unroll 4
-                for (int c = 0; c < DK; ++c) {
-                    const float e2 = __expf(gi[c] - gj[c]);
-                    pk += qi[c] * e2 * wj[c];
-                    pl += qi[c] * e2 * lj[c];
-                    if (j < i) {
-                        const float e1 = __expf(gp[c] - gj[c]);
-                        m += ri[c] * e1 * lj[c];
-                        nn += ri[c] * e1 * wj[c];
+                if (j < i) {
+                    const float* gp = Gm + (i - 1) * KS;   // Gp_i = G_{i-1}
+                    const float* ri = Rs + i * KS;
+#pragma unroll 2
+                    for (int c = 0; c < DK; c += 4) {
+                        const float4 gi4 = *reinterpret_cast<const float4*>(gi + c);
+                        const float4 gj4 = *reinterpret_cast<const float4*>(gj + c);
+                        const float4 gp4 = *reinterpret_cast<const float4*>(gp + c);
+                        const float4 qi4 = *reinterpret_cast<const float4*>(qi + c);
+                        const float4 ri4 = *reinterpret_cast<const float4*>(ri + c);
+                        const float4 lj4 = *reinterpret_cast<const float4*>(lj + c);
+                        const float4 wj4 = *reinterpret_cast<const float4*>(wj + c);
+                        const float g_i[4] = {gi4.x, gi4.y, gi4.z, gi4.w}, g_j[4] = {gj4.x, gj4.y, gj4.z, gj4.w};
+                        const float g_p[4] = {gp4.x, gp4.y, gp4.z, gp4.w}, q_i[4] = {qi4.x, qi4.y, qi4.z, qi4.w};
+                        const float r_i[4] = {ri4.x, ri4.y, ri4.z, ri4.w}, l_j[4] = {lj4.x, lj4.y, lj4.z, lj4.w};
+                        const float w_j[4] = {wj4.x, wj4.y, wj4.z, wj4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float e2 = __expf(g_i[e] - g_j[e]) * q_i[e];
+                            const float e1 = __expf(g_p[e] - g_j[e]) * r_i[e];
+                            pk = fmaf(e2, w_j[e], pk);
+                            pl = fmaf(e2, l_j[e], pl);
+                            m = fmaf(e1, l_j[e], m);
+                            nn = fmaf(e1, w_j[e], nn);
+                        }
+                    }
+                } else {
+                    // the diagonal: e^(G_i - G_i) = 1
+#pragma unroll 2
+                    for (int c = 0; c < DK; c += 4) {
+                        const float4 qi4 = *reinterpret_cast<const float4*>(qi + c);
+                        const float4 lj4 = *reinterpret_cast<const float4*>(lj + c);
+                        const float4 wj4 = *reinterpret_cast<const float4*>(wj + c);
+                        pk = fmaf(qi4.x, wj4.x, fmaf(qi4.y, wj4.y, fmaf(qi4.z, wj4.z, fmaf(qi4.w, wj4.w, pk))));
+                        pl = fmaf(qi4.x, lj4.x, fmaf(qi4.y, lj4.y, fmaf(qi4.z, lj4.z, fmaf(qi4.w, lj4.w, pl))));
                     }
                 }
             }
