@@ -262,16 +262,23 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 const int i = p / kCmax, j = p % kCmax;
                 float kd = 0.f, qd = 0.f;
                 if (j <= i && i < Cc) {
+                    // float4 along the channels: row j per lane lands in distinct bank groups
                     const float* ki = Ks + i * KS;
                     const float* qi = Qs + i * KS;
                     const float* kj = Ks + j * KS;
                     const float* gi = Gm + i * KS;
                     const float* gj = Gm + j * KS;
-#pragma unroll 4
-                    for (int c = 0; c < DK; ++c) {
-                        const float w = kj[c] * expf(gi[c] - gj[c]);
-                        kd += ki[c] * w;
-                        qd += qi[c] * w;
+#pragma unroll 2
+                    for (int c = 0; c < DK; c += 4) {
+                        const float4 ki4 = *reinterpret_cast<const float4*>(ki + c);
+                        const float4 qi4 = *reinterpret_cast<const float4*>(qi + c);
+                        const float4 kj4 = *reinterpret_cast<const float4*>(kj + c);
+                        const float4 gi4 = *reinterpret_cast<const float4*>(gi + c);
+                        const float4 gj4 = *reinterpret_cast<const float4*>(gj + c);
+                        const float w0 = kj4.x * __expf(gi4.x - gj4.x), w1 = kj4.y * __expf(gi4.y - gj4.y);
+                        const float w2 = kj4.z * __expf(gi4.z - gj4.z), w3 = kj4.w * __expf(gi4.w - gj4.w);
+                        kd = fmaf(ki4.x, w0, fmaf(ki4.y, w1, fmaf(ki4.z, w2, fmaf(ki4.w, w3, kd))));
+                        qd = fmaf(qi4.x, w0, fmaf(qi4.y, w1, fmaf(qi4.z, w2, fmaf(qi4.w, w3, qd))));
                     }
                 }
                 Am[i * kCS + j] = (j < i && i < Cc) ? bs[i] * kd : 0.f;
