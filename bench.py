@@ -818,52 +818,125 @@ def run_e2e(dn, torch, W, pin, din, pc, dc, args, stream, dev, world, tokens_ste
     """Same step through the C ABI with pinned HOST buffers: per step, copy the
     prefill inputs and the decode token set host->device, run both calls, copy
     o, S_T and the decode output device->host.  The decode state stays
-    resident (it is the layer's memory, like weights)."""
+    resident (it is the layer's memory, like weights).
+
+    Steps are double-buffered over three streams, as a server streaming
+    requests would run them: step s's uploads (copy stream) overlap step s-1's
+    kernels (the caller's stream) and step s-2's downloads (a third stream),
+    so the PCIe link's two directions and the GPU work at once.  Every step
+    still moves all of its own inputs and results.  The same step run serially
+    on one stream is reported beside it (serial_ms_per_step)."""
     hp = {k: (None if v is None else v.pin_memory()) for k, v in pin.items()}
     hd = {k: (None if v is None else v.pin_memory()) for k, v in din.items() if k != "S"}
-    P = {k: torch.empty_like(v, device=dev) for k, v in hp.items() if v is not None}
-    Dt = {k: torch.empty_like(v[0], device=dev) for k, v in hd.items() if v is not None}
     S_dec = din["S"].to(dev)
-    o_p = torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev)
-    S_T = torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev)
-    o_d = torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev)
     ws = prefill_workspace(dn, torch, pc, args.path, dev)
-    h_o = torch.empty(o_p.shape, dtype=o_p.dtype).pin_memory()
-    h_S = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
-    h_od = torch.empty(o_d.shape, dtype=o_d.dtype).pin_memory()
+
+    def buffers():
+        return dict(P={k: torch.empty_like(v, device=dev) for k, v in hp.items() if v is not None},
+                    Dt={k: torch.empty_like(v[0], device=dev) for k, v in hd.items() if v is not None},
+                    o_p=torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16, device=dev),
+                    S_T=torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32, device=dev),
+                    o_d=torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16, device=dev),
+                    h_o=torch.empty((pc.B, pc.H, pc.T, pc.dv), dtype=torch.bfloat16).pin_memory(),
+                    h_S=torch.empty((pc.B, pc.H, pc.dk, pc.dv), dtype=torch.float32).pin_memory(),
+                    h_od=torch.empty((dc.B, dc.H, dc.dv), dtype=torch.bfloat16).pin_memory())
+
+    bufs = [buffers(), buffers()]
     h2d = sum(v.numel() * v.element_size() for v in hp.values() if v is not None) + \
         sum(v[0].numel() * v.element_size() for v in hd.values() if v is not None)
-    d2h = sum(t.numel() * t.element_size() for t in (h_o, h_S, h_od))
+    d2h = sum(bufs[0][k].numel() * bufs[0][k].element_size() for k in ("h_o", "h_S", "h_od"))
 
-    def step(s):
+    def upload(bf, s):
         for k, v in hp.items():
             if v is not None:
-                P[k].copy_(v, non_blocking=True)
+                bf["P"][k].copy_(v, non_blocking=True)
         j = s % dc.bank
         for k, v in hd.items():
             if v is not None:
-                Dt[k].copy_(v[j], non_blocking=True)
-        dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, o_p, S_T, chunk=pc.chunk,
-                        scale=pc.scale, path=args.path, workspace=ws, stream=stream)
-        dn.dn_decode_step(Dt["q"], Dt["k"], Dt["v"], Dt["beta"], Dt["g"], S_dec, o_d, scale=dc.scale,
-                          stream=stream)
-        h_o.copy_(o_p, non_blocking=True)
-        h_S.copy_(S_T, non_blocking=True)
-        h_od.copy_(o_d, non_blocking=True)
+                bf["Dt"][k].copy_(v[j], non_blocking=True)
+
+    def compute(bf, st):
+        P, Dt = bf["P"], bf["Dt"]
+        dn.dn_chunk_fwd(P["q"], P["k"], P["v"], P["beta"], P["g"], None, bf["o_p"], bf["S_T"], chunk=pc.chunk,
+                        scale=pc.scale, path=args.path, workspace=ws, stream=st)
+        dn.dn_decode_step(Dt["q"], Dt["k"], Dt["v"], Dt["beta"], Dt["g"], S_dec, bf["o_d"], scale=dc.scale,
+                          stream=st)
+
+    def download(bf):
+        bf["h_o"].copy_(bf["o_p"], non_blocking=True)
+        bf["h_S"].copy_(bf["S_T"], non_blocking=True)
+        bf["h_od"].copy_(bf["o_d"], non_blocking=True)
+
+    # ---- serial: one stream, a few steps -----------------------------------------
+    def serial_step(s):
+        with torch.cuda.stream(stream):
+            upload(bufs[0], s)
+            compute(bufs[0], stream)
+            download(bufs[0])
 
     for s in range(args.warmup):
-        step(s)
+        serial_step(s)
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    n_serial = max(1, min(args.steps, 5))
+    a.record(stream)
+    for s in range(n_serial):
+        serial_step(s)
+    b.record(stream)
+    b.synchronize()
+    serial_ms = max_over_ranks(a.elapsed_time(b), world) / n_serial
+
+    # ---- double-buffered over three streams --------------------------------------
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
+    uploaded = [ev() for _ in range(2)]
+    computed = [ev() for _ in range(2)]
+    downloaded = [ev() for _ in range(2)]
+    used = [False, False]
+
+    def pipelined_step(s):
+        x = s & 1
+        bf = bufs[x]
+        with torch.cuda.stream(s_in):
+            if used[x]:
+                s_in.wait_event(computed[x])      # step s - 2 has read these inputs
+            upload(bf, s)
+            uploaded[x].record(s_in)
+        stream.wait_event(uploaded[x])
+        if used[x]:
+            stream.wait_event(downloaded[x])      # step s - 2's results are copied out
+        compute(bf, stream)
+        computed[x].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[x])
+            download(bf)
+            downloaded[x].record(s_out)
+        used[x] = True
+
+    for s in range(args.warmup):
+        pipelined_step(s)
+    torch.cuda.synchronize()
     barrier(world)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(s_in)
     for s in range(args.steps):
-        step(s)
-    b.record(stream)
+        pipelined_step(s)
+    s_out.wait_stream(stream)
+    s_out.wait_stream(s_in)
+    b.record(s_out)
+    b.synchronize()
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
     return {"value": world * tokens_step / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "schedule": "double-buffered over three streams: step s's uploads overlap step s-1's kernels "
+                        "and step s-2's downloads",
+            "serial_ms_per_step": serial_ms,
+            "serial_tokens_per_s": world * tokens_step / (serial_ms * 1e-3)}
 
 
 if __name__ == "__main__":
