@@ -185,11 +185,6 @@ __device__ __forceinline__ void tmem_st_f32(uint32_t taddr, const float (&v)[N])
     else tmem_st32(taddr, v);
 }
 
-// 1 / ||q_i|| of chunk c (with the prologue) sits in the chunk's gate slot, in
-// one of two fields by (c / 4) mod 2: the side warps write it up to four chunks
-// ahead of the output rows that read it, which then never share a field.
-__device__ __forceinline__ int rq_field(int c) { return (c >> 2) & 1 ? G_RK : G_RQ; }
-
 // z of chunk c (64 token-major rows of d_v, H d_v elements apart) into the shared
 // buffer zb by the NTHR output threads, 16 bytes a copy; rows past the chunk's
 // end are zero-filled and not read.
@@ -210,14 +205,13 @@ __device__ __forceinline__ void z_load(const Args& ar, uint32_t zb, int64_t bh, 
 
 // Output rows of chunk cp with the layer's gated RMSNorm, in two steps by the
 // 256 output threads (8 warps).  First each thread copies 32 positions of its
-// value channel j (= TMEM lane) of the chunk's o' (fp32, TMEM) into the
+// value channel j (= TMEM lane) of the chunk's o (fp32, TMEM) into the
 // row-major buffer ob (warps 0-3 positions 0-31, warps 4-7 positions 32-63);
 // then, after a barrier, thread t takes channels 8 (t mod 16) .. + 7 of rows
 // t / 16 + 16 u: the 16 threads of a row sum its squares by shuffles, and each
 // forms y_ij = w_j o_ij / sqrt(mean_j o_ij^2 + eps) act(z_ij) for its eight
-// channels (16-byte loads of o' and z, a 16-byte store of y, token-major like
-// z).  With the prologue o_ij = r_i o'_ij (r_i = 1 / ||q_i||), so row i's
-// factor is r_i / sqrt(r_i^2 mean_j o'_ij^2 + eps).
+// channels (16-byte loads of o and z, a 16-byte store of y, token-major like
+// z).  (The prologue's 1 / ||q_i|| is already in o: Qh and P carry it.)
 __device__ __forceinline__ void norm_stage(uint32_t oc, float* __restrict__ ob, int j, int hh) {
     float v[32];
     tmem_ld32(oc + hh * 32, v);
@@ -226,8 +220,8 @@ __device__ __forceinline__ void norm_stage(uint32_t oc, float* __restrict__ ob, 
     for (int e = 0; e < 32; ++e) ob[(hh * 32 + e) * kD + j] = v[e];
 }
 __device__ __forceinline__ void norm_rows(const Args& ar, const float* __restrict__ ob,
-                                          const __nv_bfloat16* __restrict__ zb, const float* rq, int64_t bh,
-                                          int cp, int Cc, int oid) {
+                                          const __nv_bfloat16* __restrict__ zb, int64_t bh, int cp, int Cc,
+                                          int oid) {
     const int64_t b = bh / ar.H, h = bh % ar.H;
     const int64_t row0 = (b * ar.T + (int64_t)cp * kC) * ar.H + h;   // token-major row of position 0
     const int c8 = (oid & 15) * 8;                                   // first channel of the thread
@@ -249,8 +243,7 @@ __device__ __forceinline__ void norm_rows(const Args& ar, const float* __restric
         ss += __shfl_xor_sync(0xffffffffu, ss, 2);
         ss += __shfl_xor_sync(0xffffffffu, ss, 4);
         ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-        const float r = rq[i];
-        const float f = r * rsqrtf(r * r * ss * (1.f / (float)kD) + ar.eps);
+        const float f = rsqrtf(ss * (1.f / (float)kD) + ar.eps);
         const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
         uint32_t y[4];
 #pragma unroll
@@ -376,8 +369,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                     // beta and g from the raw inputs, as the WY side computes them (here, one
                     // chunk after the loads were issued, so their latency stays hidden)
                     const int Cn = min(kC, len - cc * kC);
-                    if (lane < Cn) gdn_raw_gates(b0, a0, eA, dtb, (float)ar.prologue);
-                    if (lane + 32 < Cn) gdn_raw_gates(b1, a1, eA, dtb, (float)ar.prologue);
+                    if (lane < Cn) gdn_raw_gates_fast(b0, a0, eA, dtb, (float)ar.prologue);
+                    if (lane + 32 < Cn) gdn_raw_gates_fast(b1, a1, eA, dtb, (float)ar.prologue);
                 }
                 chunk_gates(gates + (cc & 3) * GATE_FLOATS, b0, b1, a0, a1, lane);
                 __syncwarp();
@@ -409,7 +402,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 const int y = KDA ? (int)(tile * kC) : (int)(krow_base + (int64_t)cc * kC);
                 const uint32_t st = sb + s * SZ_STAGE;
                 const uint32_t fb = ctl.bar(B_FULL0 + s);
-                mbar_arrive_expect_tx(fb, STAGE_TX);
+                mbar_arrive_expect_tx(fb, PRO ? STAGE_TX + kC * 4 : STAGE_TX);
                 tma_load_2d(st + ST_K + 0, &tm_k, 0, y, fb);
                 tma_load_2d(st + ST_K + 8192, &tm_k, 64, y, fb);
                 tma_load_2d(st + ST_B + 0, &tm_q, 0, y, fb);
@@ -418,6 +411,10 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tma_load_2d(st + ST_B + 24576, &tm_w, 64, (int)(tile * kC), fb);
                 tma_load_2d(st + ST_UT, &tm_u, 0, (int)(tile * kD), fb);
                 tma_load_2d(st + ST_P, &tm_p, 0, (int)(tile * kC), fb);
+                // with the prologue: the WY tile's 1 / ||q_i|| row (published with the tile)
+                // into the chunk's gate slot, for Qh; its previous reader, chunk cc - 4's
+                // side warps, finished before chunk cc - 3's products, which freed this stage
+                if (PRO) bulk_load(smem_u32(gates + (cc & 3) * GATE_FLOATS + G_RQ), ar.rq + tile * kC, kC * 4, fb);
             }
             if (!(test_flags & 1)) issued = cc + 1;
         }
@@ -494,7 +491,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
         const int j = (q << 5) + lane;             // value channel = TMEM lane
         for (int c = 0; c <= n; ++c) {
             if (c < n) {
-                // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block)
+                // ---- Qh = scale e^G Q in place over the q tile (rows 0-63 of each d-block);
+                //      with the prologue, Q's rows also normalised
                 const int s = c % kStages;
                 const int Cc = min(kC, len - c * kC);
                 float* gs = gates + (c & 3) * GATE_FLOATS;
@@ -503,12 +501,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                           ctl.wait(B_FULL0 + s, (uint32_t)(c / kStages) & 1u);
                 if (!ok) *abort_flag = 1;
                 if (named_bar_any(1, kSideThreads, !ok)) break;
-                // with the prologue: the WY tile's 1 / ||q_i|| of this chunk's rows (published with
-                // the tile, whose flag the producer acquired before these tiles were loaded),
-                // requested now and stored into the gate slot before READY
-                float4 rq4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (PRO && sid < kC / 4)
-                    rq4 = reinterpret_cast<const float4*>(ar.rq + (tile0 + (int64_t)c * tstep) * kC)[sid];
                 // (with the per-key gate the workspace holds Qh already)
                 // (loads four at a time: the ld / st helpers keep their order, so one load per
                 // iteration would wait out each load's latency in turn)
@@ -526,7 +518,8 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int uu = 0; uu < 4; ++uu) {
                         const int i = ((sid + (u0 + uu) * kSideThreads) >> 3) & 63;
-                        const float f = i < Cc ? scale * gs[G_EG + i] : 0.f;
+                        // (with the prologue Qh also takes 1 / ||q_i||, which landed with the stage)
+                        const float f = i < Cc ? (PRO ? scale * gs[G_EG + i] * gs[G_RQ + i] : scale * gs[G_EG + i]) : 0.f;
                         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
                         const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
                         const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
@@ -558,9 +551,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                                      pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
                     }
                 }
-                // 1 / ||q_i|| for the output rows, ordered before READY (and so before the
-                // products whose completion the output rows wait for)
-                if (PRO && sid < kC / 4) reinterpret_cast<float4*>(gs + rq_field(c))[sid] = rq4;
                 fence_async_smem();
                 mbar_arrive(ctl.bar(B_READY0 + s));
             }
@@ -574,7 +564,6 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 tc_fence_after();
                 __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
                 const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
-                const float* rq = gates + (cp & 3) * GATE_FLOATS + rq_field(cp);   // 1 / ||q_i||
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -583,7 +572,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int i = hh * 32 + e;
-                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * rq[i] : v[e]);
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
                     }
                 }
                 tc_fence_before();
@@ -610,15 +599,14 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 z_load<kOT>(ar, zbuf + ((cp + 1) & 1) * L::SZ_Z, bh, cp + 1, min(kC, len - (cp + 1) * kC), oid);
             tc_fence_after();
             const uint32_t oc = tmem + ((uint32_t)(q << 5) << 16) + TM_OU + (cp % L::kOuBufs) * 128;
-            const float* rq = gates + (cp & 3) * GATE_FLOATS + rq_field(cp);   // 1 / ||q_i||
             if constexpr (PRO == 2) {
                 float* ob = reinterpret_cast<float*>(sm + L::OFF_OB);
                 norm_stage(oc, ob, j, oid >> 7);
                 tc_fence_before();
                 mbar_arrive(ctl.bar(B_OFREE0 + (cp & 1)));        // the TMEM buffer is read
                 named_bar_sync(5, kOT);
-                norm_rows(ar, ob, reinterpret_cast<const __nv_bfloat16*>(sm + L::OFF_Z + (cp & 1) * L::SZ_Z), rq,
-                          bh, cp, Cc, oid);
+                norm_rows(ar, ob, reinterpret_cast<const __nv_bfloat16*>(sm + L::OFF_Z + (cp & 1) * L::SZ_Z), bh, cp,
+                          Cc, oid);
             } else {
                 __nv_bfloat16* ob = o + (row_base + (int64_t)cp * kC) * kD + j;
 #pragma unroll
@@ -629,7 +617,7 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int i = hh * 32 + e;
-                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(PRO ? v[e] * rq[i] : v[e]);
+                        if (i < Cc) ob[(int64_t)i * kD] = __float2bfloat16_rn(v[e]);
                     }
                 }
                 tc_fence_before();

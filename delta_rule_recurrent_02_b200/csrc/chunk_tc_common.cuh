@@ -129,27 +129,20 @@ __host__ __device__ __forceinline__ int64_t key_head(int64_t bh, int H, int rep)
 constexpr int G_BETA = 0, G_G2 = 64, G_EG = 128, G_ET = 192, G_BEG = 256, G_GAMMA = 320, G_RQ = 384, G_RK = 448;
 constexpr uint32_t GATE_FLOATS = 512;
 
-// 1 / max(||x||, 1e-12) for a row of d_k = 128 bf16 values in a [rows][128 B]
-// tile pair with 128-byte swizzle (blocks of 64 columns `block_bytes` apart),
-// summed by two threads: this one takes the 64 columns of block `half`; the
-// partner (lane ^ 1) the other.
-__device__ __forceinline__ float inv_row_norm(uint32_t tile, int row, int half, uint32_t block_bytes) {
-    uint4 w[8];
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) w[ch] = ld_shared_v4(tile + (uint32_t)half * block_bytes + sw128_off(row, ch));
-    float ss[4] = {0.f, 0.f, 0.f, 0.f};                  // four partial sums: short dependency chains
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[ch]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h[e]);
-            ss[e] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[e]));
-        }
-    }
-    float t = (ss[0] + ss[1]) + (ss[2] + ss[3]);
-    t += __shfl_xor_sync(0xffffffffu, t, 1);
-    return fminf(rsqrtf(t), 1e12f);                      // 1 / max(||x||, 1e-12)
+// The layer's raw gates as gdn_raw_gates computes them, with the fast exponential,
+// logarithm and division, for the tensor-core kernels (the WY tile and the state
+// pass both use this one, so they see the same beta and g).  softplus(x) =
+// log(1 + y), y = e^x: x above 20, the series y - y^2/2 + y^3/3 - y^4/4 for
+// y < 1/16 (truncated after y^4: under 3.1e-6 of the value), else log(1 + y)
+// (the rounding of 1 + y and the fast logarithm: under about 7e-6 of the value).
+__device__ __forceinline__ void gdn_raw_gates_fast(float& b, float& a, float eA, float dt_bias, float bmul) {
+    b = __fdividef(bmul, 1.f + __expf(-b));
+    const float x = a + dt_bias;
+    const float y = __expf(x);
+    const float sp = x > 20.f ? x
+                   : y < 0.0625f ? y * (1.f - y * (0.5f - y * (1.f / 3.f - 0.25f * y)))
+                                 : __logf(1.f + y);
+    a = -eA * sp;
 }
 
 // Gates of one chunk from beta and g at positions lane and lane + 32 (zero past

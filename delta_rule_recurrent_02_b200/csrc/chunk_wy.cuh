@@ -381,18 +381,19 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             const int h = (int)(bh % ar.H);
             const float eA = expf(ar.A_log[h]), dtb = ar.dt_bias[h];
             const float bm = (float)ar.prologue;
-            if (lane < Cc) gdn_raw_gates(b0, a0, eA, dtb, bm);
-            if (lane + 32 < Cc) gdn_raw_gates(b1, a1, eA, dtb, bm);
+            if (lane < Cc) gdn_raw_gates_fast(b0, a0, eA, dtb, bm);
+            if (lane + 32 < Cc) gdn_raw_gates_fast(b1, a1, eA, dtb, bm);
         }
         chunk_gates(gs, b0, b1, a0, a1, lane);
     }
     bool ok = true;
     if (tid == 0) {
-        // [K;Q] K^T once the tiles have landed
+        // [K;Q] K^T once the tiles have landed; with the prologue [K;Q][K;Q]^T (the same
+        // cost for N = 128 as for 64), whose diagonal holds ||k_i||^2 and ||q_i||^2
         ok = ctl.wait(B_FULL, 0);
         if (ok) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, 64, 0, 0);
+            const uint32_t idesc = idesc_bf16(128, PRO ? 128 : 64, 0, 0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t a = sb + OFF_KV + (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -401,31 +402,7 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             mma_commit(ctl.bar(B_MMA));
         }
     }
-    if (PRO) {
-        // 1 / ||k_i|| (threads 0-127) and 1 / ||q_i|| (128-255) from the [K0 | Q0 | K1 | Q1]
-        // tiles, two threads per row, while the gram runs; r_k stays in the gate slot, r_q
-        // goes to the workspace (published with the tile) for the state pass's output rows
-        if (ctl.wait(B_FULL, 0)) {
-            const int r = (tid & 127) >> 1, which = tid >> 7;
-            const float rn = inv_row_norm(sb + OFF_KV + (uint32_t)which * 8192u, r, tid & 1, 16384);
-            if ((tid & 1) == 0) {
-                if (which == 0) gs[G_RK + r] = rn;
-                else if (ar.rq) ar.rq[tile * kC + r] = rn;
-            }
-        } else {
-            ok = false;
-        }
-    }
     named_bar_sync(x.bar, kNT);                       // gates visible
-    if (PRO && tid < kC) {
-        // the key norms enter the gram as a column factor folded into the decay,
-        // rk_j 2^(G2_i - G2_j) = 2^(G2_i - (G2_j - log2 rk_j)): the shifted column
-        // table goes where e^(G_last - G) was (the state pass's, unused here), and
-        // T diag(beta e^G) takes rk_j by scaling beta e^G
-        const float rk = gs[G_RK + tid];
-        gs[G_ET + tid] = gs[G_G2 + tid] - log2f(rk);
-        gs[G_BEG + tid] *= rk;
-    }
     ok = ok && ctl.wait(B_MMA, 0);
     if (named_bar_any(x.bar, kNT, !ok)) goto done;
     tc_fence_after();
@@ -447,6 +424,33 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         const int i = ((q & 1) << 5) + lane;
         const int j0 = (warp >> 2) << 5;
         const float g2i = gs[G_G2 + i];
+        float rq_i = 0.f;
+        if constexpr (PRO) {
+            // 1 / max(||x_i||, 1e-12) from the gram's diagonal, before A and P: the key
+            // norms by warps 0 and 5 (whose A columns hold the diagonal) into the gate
+            // slot, with T diag(beta e^G) taking r_kj by scaling beta e^G; the query norms
+            // by the P warps 2, 3 and 7 for their own rows (warps 2 and 3 also write them
+            // to the workspace, published with the tile, for the state pass's Qh)
+            const bool kdiag = q < 2 && j0 == (q << 5);
+            const bool qdiag = q >= 2 && !(q == 2 && j0 == 32);
+            if (kdiag || qdiag) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + (kdiag ? j0 : 64 + ((q - 2) << 5)), v);
+                tmem_wait_ld();
+                float dsq = v[0];
+#pragma unroll
+                for (int e = 1; e < 32; ++e) dsq = lane == e ? v[e] : dsq;
+                const float rn = fminf(rsqrtf(dsq), 1e12f);
+                if (kdiag) {
+                    gs[G_RK + i] = rn;
+                    gs[G_BEG + i] *= rn;
+                } else {
+                    rq_i = rn;
+                    if (j0 == 0 && ar.rq) ar.rq[tile * kC + i] = rn;
+                }
+            }
+            named_bar_sync(x.bar, kNT);
+        }
         if (q == 0 && j0 == 32) {
             // A rows 0-31 x columns 32-63 lie above the diagonal: never read
         } else if (q < 2) {
@@ -454,16 +458,21 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
             tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
             tmem_wait_ld();
             const float bi = PRO ? gs[G_BETA + i] * gs[G_RK + i] : gs[G_BETA + i];   // zero past the chunk's end
-            const float* g2c = gs + (PRO ? G_ET : G_G2);   // column table (with the key norms folded in)
+            const float* g2c = gs + G_G2;
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
                 const float4 gj = *reinterpret_cast<const float4*>(g2c + j0 + 4 * q4);
                 const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+                // with the prologue, column j also takes r_kj
+                const float4 rk = PRO ? *reinterpret_cast<const float4*>(gs + G_RK + j0 + 4 * q4)
+                                      : make_float4(1.f, 1.f, 1.f, 1.f);
+                const float rkv[4] = {rk.x, rk.y, rk.z, rk.w};
                 float a[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j0 + 4 * q4 + e;
-                    a[e] = j < i ? bi * v[4 * q4 + e] * decay2(g2i, gjv[e]) : 0.f;
+                    a[e] = j < i ? bi * v[4 * q4 + e] * (PRO ? decay2(g2i, gjv[e]) * rkv[e] : decay2(g2i, gjv[e]))
+                                 : 0.f;
                 }
                 *reinterpret_cast<float4*>(Am + fidx(i, j0 + 4 * q4)) = make_float4(a[0], a[1], a[2], a[3]);
             }
@@ -484,7 +493,9 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(q << 5) << 16) + TM_G + j0, v);
                 tmem_wait_ld();
-                const float si = i < Cc ? scale : 0.f;
+                // (with the prologue, row i also takes 1 / ||q_i||, so that the state pass's
+                // output rows come out normalised)
+                const float si = i < Cc ? (PRO ? scale * rq_i : scale) : 0.f;
                 const float* g2c = gs + G_G2;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {

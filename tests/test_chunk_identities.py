@@ -8,13 +8,14 @@ check two placements of those factors against the sequential recurrence (the
 oracle) run on the normalised inputs, over several chunks with a carried
 state:
 
-- the kernels' placement:
+- the plain placement:
   - A_ij carries r_ki r_kj, and P_ij carries r_qi r_kj;
   - W = T diag(beta e^G r_k) K;
   - Q-hat rows carry r_q, and the rows of U~ carry r_k;
-- a fold that keeps r_k out of the state pass: u' = diag(r_k) u,
-  W' = diag(r_k) W and P' = P diag(1/r_k), so that U' = u' - W'S = diag(r_k) U,
-  K^T U~' = K-hat^T U~ and P'U' = PU;
+- the kernels' placement, a fold that keeps r_k out of the state pass:
+  u' = diag(r_k) u, W' = diag(r_k) W and P' = P diag(1/r_k) (rows still
+  carrying r_q), so that U' = u' - W'S = diag(r_k) U, K^T U~' = K-hat^T U~
+  and P'U' = PU; Q-hat keeps its r_q, and the output rows need no factor;
 - the full fold, which also moves r_q to the output rows: P'' = scale tril(QK^T * D),
   with no norm factor at all, Q-hat without r_q, and O = diag(r_q)(Q-hat S + P''U').
 
@@ -102,7 +103,8 @@ def test_factor_placement_catches_a_dropped_factor():
     assert np.abs(o - o_ref[0, 0]).max() > 1e-3 * np.abs(o_ref).max()
 
 
-def test_full_fold_with_zero_rows():
+@pytest.mark.parametrize("fold", [True, "all"])
+def test_fold_with_zero_rows(fold):
     """A zero key row gets r_k = 1e12 and a zero query row r_q = 1e12 (the
     max(||x||, 1e-12) clamp).  The fold then scales u and W rows by 1e12, and
     still matches the recurrence, whose unit key and query are zero there."""
@@ -113,7 +115,7 @@ def test_full_fold_with_zero_rows():
     scale = q.shape[1] ** -0.5
     o_ref, S_ref = oracle.delta_rule(qn, kn, v[None, None], beta[None, None], g[None, None], S0[None, None],
                                      scale=scale)
-    o, S = chunk_pass(q, k, v, beta, g, S0, scale, 8, "all")
+    o, S = chunk_pass(q, k, v, beta, g, S0, scale, 8, fold)
     assert np.isfinite(o).all() and np.isfinite(S).all()
     assert np.allclose(o, o_ref[0, 0], rtol=0, atol=1e-9 * np.abs(o_ref).max())
     assert np.allclose(S, S_ref[0, 0], rtol=0, atol=1e-9 * np.abs(S_ref).max())
