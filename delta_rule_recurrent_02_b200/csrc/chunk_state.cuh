@@ -518,13 +518,14 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int uu = 0; uu < 4; ++uu) {
                         const int i = ((sid + (u0 + uu) * kSideThreads) >> 3) & 63;
-                        // (with the prologue Qh also takes 1 / ||q_i||, which landed with the stage)
+                        // (with the prologue Qh also takes 1 / ||q_i||, which landed with the stage).
+                        // The row's factor is rounded to bf16 and applied by packed bf16 multiplies:
+                        // the side warps share the SM's issue slots with the chain's epilogues, and
+                        // their instruction count, not this one rounding, showed in the chain
                         const float f = i < Cc ? (PRO ? scale * gs[G_EG + i] * gs[G_RQ + i] : scale * gs[G_EG + i]) : 0.f;
-                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
-                        const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-                        const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                        st_shared_v4(a[uu], pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                                     pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                        const uint32_t f2 = pack_bf16x2(f, f);
+                        st_shared_v4(a[uu], mul_bf16x2(w[uu].x, f2), mul_bf16x2(w[uu].y, f2), mul_bf16x2(w[uu].z, f2),
+                                     mul_bf16x2(w[uu].w, f2));
                     }
                 }
                 // ---- K~ = K (.) e^(G_last - G) in place over the k tile: each position's decay to
@@ -544,11 +545,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 #pragma unroll
                     for (int uu = 0; uu < 4; ++uu) {
                         const float f = gs[G_ET + (((sid + (u0 + uu) * kSideThreads) >> 3) & 63)];
-                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w[uu]);
-                        const float2 e0 = __bfloat1622float2(h[0]), e1 = __bfloat1622float2(h[1]);
-                        const float2 e2 = __bfloat1622float2(h[2]), e3 = __bfloat1622float2(h[3]);
-                        st_shared_v4(a[uu], pack_bf16x2(f * e0.x, f * e0.y), pack_bf16x2(f * e1.x, f * e1.y),
-                                     pack_bf16x2(f * e2.x, f * e2.y), pack_bf16x2(f * e3.x, f * e3.y));
+                        const uint32_t f2 = pack_bf16x2(f, f);
+                        st_shared_v4(a[uu], mul_bf16x2(w[uu].x, f2), mul_bf16x2(w[uu].y, f2), mul_bf16x2(w[uu].z, f2),
+                                     mul_bf16x2(w[uu].w, f2));
                     }
                 }
                 fence_async_smem();
