@@ -320,6 +320,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(a), "f"(b));
     return r;
 }
+// d0 += x a0, d1 += x a1 as one packed fp32 FMA (each half rounded like fmaf).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float x, float a0, float a1) {
+    uint64_t d, a, b, c;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(x));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(d0), "f"(d1));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
 // Two bf16 products, each rounded to nearest: one instruction for what unpacking,
 // two fp32 multiplies and a repack take five.
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
