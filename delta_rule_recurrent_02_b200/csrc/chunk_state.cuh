@@ -158,7 +158,41 @@ struct Args {
     float eps = 0.f;
     // with the prologue: the workspace's 1 / ||q_i|| rows, written by the WY tiles
     const float* rq = nullptr;
+    // the workspace (128-byte aligned) and its tile count: each tile's lines are dropped
+    // from L2 once its loads have landed (null: kept)
+    uint8_t* scratch = nullptr;
+    long long scratch_tiles = 0;
 };
+
+// Drop tile t's workspace lines from L2 (one warp): -W, u^T, P, the 1 / ||q_i|| row
+// with the prologue, and K~, Qh and e^Gamma_last with the per-key gate.  The tile's
+// loads have landed in shared memory and nothing reads it again in this call, so the
+// lines need never be written back to memory.
+template <int GATE, int PRO>
+__device__ __forceinline__ void drop_tile(const Args& ar, int64_t t, int lane) {
+    const int64_t nt = ar.scratch_tiles;
+    uint8_t* const base = ar.scratch;
+    uint8_t* const w = base + t * (int64_t)kWsWBytes;
+    uint8_t* const u = base + nt * (int64_t)kWsWBytes + t * (int64_t)kWsUBytes;
+    uint8_t* const p = base + nt * (int64_t)(kWsWBytes + kWsUBytes) + t * (int64_t)kWsPBytes;
+    for (int l = lane; l < (int)(kWsWBytes / 128); l += 32) {
+        discard_l2(w + 128 * l);
+        discard_l2(u + 128 * l);
+    }
+    for (int l = lane; l < (int)(kWsPBytes / 128); l += 32) discard_l2(p + 128 * l);
+    constexpr int64_t kBeforeRq = (int64_t)(kWsWBytes + kWsUBytes + kWsPBytes);
+    if (PRO && lane < (int)(kWsRqBytes / 128)) discard_l2(base + nt * kBeforeRq + t * (int64_t)kWsRqBytes + 128 * lane);
+    if constexpr (GATE == kGatePerKey) {
+        uint8_t* const kt = base + nt * (int64_t)kWsTileBytes + t * (int64_t)kWsKtBytes;
+        uint8_t* const qh = base + nt * (int64_t)(kWsTileBytes + kWsKtBytes) + t * (int64_t)kWsQhBytes;
+        uint8_t* const gm = base + nt * (int64_t)(kWsTileBytes + kWsKtBytes + kWsQhBytes) + t * (int64_t)kWsGamBytes;
+        for (int l = lane; l < (int)(kWsKtBytes / 128); l += 32) {
+            discard_l2(kt + 128 * l);
+            discard_l2(qh + 128 * l);
+        }
+        if (lane < (int)(kWsGamBytes / 128)) discard_l2(gm + 128 * lane);
+    }
+}
 
 // Gate slot with the per-key gate: e^Gamma_last of each key channel.
 constexpr int G_KGAM = 0;
@@ -417,6 +451,10 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
                 if (PRO) bulk_load(smem_u32(gates + (cc & 3) * GATE_FLOATS + G_RQ), ar.rq + tile * kC, kC * 4, fb);
             }
             if (!(test_flags & 1)) issued = cc + 1;
+            // chunk cc - 3's workspace tile (its loads landed before the stage was freed) is
+            // dropped from L2, after this chunk's loads are under way
+            if (cc >= kStages && ar.scratch && !(test_flags & 1))
+                drop_tile<GATE, PRO>(ar, tile0 + (int64_t)(cc - kStages) * tstep, lane);
         }
         if (*abort_flag && lane == 0) {
             // let every load this CTA issued land before its shared memory is released
@@ -762,6 +800,9 @@ __device__ __forceinline__ void state_pass(uint8_t* sm, const Args& ar, int64_t 
 
     named_bar_sync(kCtaBar, kNT);
     if (*abort_flag && tid == 0) atomicOr(status, 1u);
+    // the last chunks' tiles (every product is done)
+    if (warp == 0 && ar.scratch && !(test_flags & 1) && !*abort_flag)
+        for (int cd = max(0, n - kStages); cd < n; ++cd) drop_tile<GATE, PRO>(ar, tile0 + (int64_t)cd * tstep, lane);
     if (!HOSTED && warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);

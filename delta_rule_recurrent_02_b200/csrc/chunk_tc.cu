@@ -42,7 +42,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status, test_flags,
                          gam, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H, pro.rep, vl, vl_N,
-                         pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq};
+                         pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq, pro.scratch, pro.scratch_tiles};
     state::state_pass<GATE, false, PRO>(sm, ar, blockIdx.x, 0u);
 }
 
@@ -139,7 +139,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_k, &tm_q, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
                              test_flags, nullptr, snaps, snap_every, n_snap, pro.on, pro.A_log, pro.dt_bias, pro.H,
-                             pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq};
+                             pro.rep, nullptr, 0, pro.norm, pro.z, pro.norm_w, pro.eps, pro.rq, pro.scratch, pro.scratch_tiles};
         if constexpr (!HOSTED) {
             // ---- state pass of head blockIdx.x --------------------------------------------
             if (warp >= state::Roles<GATE, false, PRO>::kNT / 32) return;
@@ -239,12 +239,14 @@ chunk_fused_kda_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        __nv_bfloat16* p_out, __nv_bfloat16* kt_out, __nv_bfloat16* qh_out, float* gam,
                        unsigned int* flags, int BH, const float* __restrict__ beta, const float* __restrict__ g,
                        const float* S0, __nv_bfloat16* __restrict__ o, float* S_T, int T, int n, float scale,
-                       unsigned int* status, int test_flags, float* snaps, int snap_every, int n_snap) {
+                       unsigned int* status, int test_flags, float* snaps, int snap_every, int n_snap,
+                       uint8_t* scratch, long long scratch_tiles) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     if ((int)blockIdx.x < BH) {
         const state::Args ar{&tm_kt, &tm_qh, &tm_w, &tm_u, &tm_p, flags, beta, g, S0, o, S_T, T, scale, status,
-                             test_flags, gam, snaps, snap_every, n_snap, 0, nullptr, nullptr, 1};
+                             test_flags, gam, snaps, snap_every, n_snap, 0, nullptr, nullptr, 1, 1, nullptr, 0, 0,
+                             nullptr, nullptr, 0.f, nullptr, scratch, scratch_tiles};
         state::state_pass<kGatePerKey, false, 0>(sm, ar, blockIdx.x, 0u);
         return;
     }
@@ -312,6 +314,8 @@ cudaError_t launch_tc_gate(const ChunkArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     m.p_ws = reinterpret_cast<__nv_bfloat16*>(p_ws);
     m.rq_ws = reinterpret_cast<float*>(p_ws + tiles * kWsPBytes);
+    m.scratch = drop_scratch(w_ws, tiles * kWsTileBytes);
+    m.tiles = tiles;
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles));
     if (packed) {
         // the chunk tables, then all WY tiles, then one state pass per (sequence, head)
@@ -413,6 +417,8 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     m.qh_ws = reinterpret_cast<__nv_bfloat16*>(qh_ws);
     m.gam_ws = reinterpret_cast<float*>(gam_ws);
     m.flags = reinterpret_cast<unsigned int*>(w_ws + ws_flags_offset(tiles, true));
+    m.scratch = drop_scratch(w_ws, tiles * kWsKdaTileBytes);
+    m.tiles = tiles;
 
     int dev = 0, num_sms = 0, coop = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -444,9 +450,11 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
             unsigned int* status = a.status;
             float* snaps = a.snaps;
             int snap_every = a.snap_every, n_snap = a.n_snap;
+            uint8_t* scratch = m.scratch;
+            long long scratch_tiles = (long long)m.tiles;
             void* args[] = {&m.q, &m.k, &m.v, &m.w, &m.u, &m.p, &m.kt, &m.qh, &p_out, &kt_out, &qh_out, &gam,
                             &flags, &bh_i, &beta, &g, &S0, &o, &S_T, &T_i, &n_i, &scale, &status, &test_flags,
-                            &snaps, &snap_every, &n_snap};
+                            &snaps, &snap_every, &n_snap, &scratch, &scratch_tiles};
             // the flags are cleared on the same stream right before the launch
             e = cudaMemsetAsync(m.flags, 0, ws_flag_words(tiles) * 4, st);
             if (e != cudaSuccess) return e;
@@ -463,7 +471,7 @@ cudaError_t launch_tc_kda(const ChunkArgs& a, cudaStream_t st) {
     kern<<<(unsigned)(a.B * a.H), state::Roles<kGatePerKey>::kNT, bytes, st>>>(m.kt, m.qh, m.w, m.u, m.p, nullptr, a.beta, a.g, a.S0,
                                                           static_cast<__nv_bfloat16*>(a.o), a.S_T, (int)a.T,
                                                           a.scale, a.status, a.test_flags, m.gam_ws, a.snaps,
-                                                          a.snap_every, a.n_snap, Prologue{0, nullptr, nullptr, 1}, nullptr, 0);
+                                                          a.snap_every, a.n_snap, prologue_of(a, m), nullptr, 0);
     return counted(cudaGetLastError());
 }
 

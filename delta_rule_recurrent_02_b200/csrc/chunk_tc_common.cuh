@@ -71,6 +71,9 @@ struct TcMaps {
     // a packed batch only: the workspace's chunk tables (VarlenTables), else null
     const int* vl = nullptr;
     float* rq_ws = nullptr;  // the workspace's rq array
+    // the workspace itself (null unless 128-byte aligned) and its tile count
+    uint8_t* scratch = nullptr;
+    uint64_t tiles = 0;
 };
 
 // The Gated DeltaNet layer's prologue, fused into the prefill kernels (scalar
@@ -89,6 +92,10 @@ struct Prologue {
     const float* norm_w = nullptr;
     float eps = 0.f;
     float* rq = nullptr;     // the workspace's 1 / ||q_i|| per tile row (with the prologue)
+    // the workspace and its tile count: the state pass drops each tile's lines from L2
+    // once its loads have landed, so that they are never written back (null: kept)
+    uint8_t* scratch = nullptr;
+    long long scratch_tiles = 0;
 };
 
 // Chunk tables of a packed batch of N sequences, built on the device from
@@ -108,6 +115,19 @@ struct VarlenTables {
 inline int64_t vl_chunks_max(int64_t T, int N) { return T / kC + N; }
 inline size_t vl_table_ints(int N, int64_t nc_max) { return 2 * (size_t)(N + 1) + (size_t)nc_max; }
 
+// The workspace whose consumed tiles the state passes drop from L2 (null: none).
+// Dropping pays when a tile is consumed soon after it is written, while its
+// lines are still in L2 (126 MB): then they are never written back to memory
+// (measured at 4096 tiles, 169 MB: 196 -> 87 MB of DRAM writes per launch, no
+// time cost).  Where the WY side runs far ahead of the chains (long sequences
+// on few heads, workspaces of a GB and more) the lines have been written back
+// long before; dropping saves nothing there and costs about 1%, so it is done
+// only up to 512 MB of tiles.  The discards need 128-byte aligned lines.
+inline uint8_t* drop_scratch(uint8_t* ws, uint64_t tile_bytes) {
+    constexpr uint64_t kDropMaxBytes = 512ull << 20;
+    return (reinterpret_cast<uintptr_t>(ws) & 127u) == 0 && tile_bytes <= kDropMaxBytes ? ws : nullptr;
+}
+
 // The Prologue argument of the tensor-core kernels for a request.
 inline Prologue prologue_of(const ChunkArgs& a, const TcMaps& m) {
     Prologue p{a.prologue, a.A_log, a.dt_bias, (int)a.H, a.rep};
@@ -116,6 +136,8 @@ inline Prologue prologue_of(const ChunkArgs& a, const TcMaps& m) {
     p.norm_w = a.norm_weight;
     p.eps = a.eps;
     if (a.prologue) p.rq = m.rq_ws;
+    p.scratch = m.scratch;
+    p.scratch_tiles = (long long)m.tiles;
     return p;
 }
 

@@ -70,6 +70,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         :: "r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
+// Drop the 128-byte line at p (128-byte aligned) from L2 without writing it back to
+// memory; its contents become undefined.  For scratch data that nothing reads again.
+__device__ __forceinline__ void discard_l2(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" :: "l"(reinterpret_cast<uint64_t>(p)) : "memory");
+}
+
 // Contiguous copy global -> shared of `bytes` (a multiple of 16; both addresses
 // 16-byte aligned), completing on the mbarrier bar like a tensor load.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
