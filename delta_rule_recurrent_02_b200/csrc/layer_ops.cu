@@ -95,6 +95,50 @@ struct Vec<float, 2> {
     __device__ static raw from_f(const float* f) { return make_float2(f[0], f[1]); }
 };
 
+// ---- packed fp32 pairs: two IEEE-rounded operations in one instruction, the same
+//      results as the scalar ones in half the issue slots -----------------------------
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {   // a * b + c
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// The hardware's approximate reciprocal (about 1 ulp; 1 / inf = 0).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+// The logistic sigmoid 1 / (1 + e^-x) of a pair, with e^-x = 2^(-x log2 e) on the
+// hardware's approximate exp2 and reciprocal (a few ulp, far inside a bf16
+// rounding); for very negative x the exp2 overflows to inf and the reciprocal gives 0,
+// the right limit.  silu2 is x sigmoid(x).
+__device__ __forceinline__ float2 sigmoid2(float2 x) {
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 t = mul2(x, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = add2(make_float2(sm100::ex2_approx(t.x), sm100::ex2_approx(t.y)), make_float2(1.f, 1.f));
+    return make_float2(rcp_approx(d.x), rcp_approx(d.y));
+}
+__device__ __forceinline__ float2 silu2(float2 x) { return mul2(x, sigmoid2(x)); }
+
 // SiLU and the logistic sigmoid through the fast exp and the approximate reciprocal
 // (a few ulp, far inside a bf16 rounding): for very negative x the exp overflows to
 // inf and 1 / inf gives 0, the right limit
@@ -341,12 +385,26 @@ causal_conv1d_tile_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* 
                 const int t = t0 + r0 + i;
                 VT::to_f(*reinterpret_cast<const raw*>(&sm.rows[buf][r0 + i + K - 1][tx * V]), win[K - 1]);
                 float acc[V];
+                if constexpr (V % 2 == 0) {
+                    // channel pairs through packed fp32 (the kernel is bound by instruction issue)
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    float a = 0.f;
+                    for (int v = 0; v < V; v += 2) {
+                        float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int j = 0; j < K; ++j) a = fmaf(wf[j][v], win[j][v], a);
-                    acc[v] = ACT ? silu(a) : a;
+                        for (int j = 0; j < K; ++j)
+                            a = fma2(make_float2(wf[j][v], wf[j][v + 1]), make_float2(win[j][v], win[j][v + 1]), a);
+                        if (ACT) a = silu2(a);
+                        acc[v] = a.x;
+                        acc[v + 1] = a.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int j = 0; j < K; ++j) a = fmaf(wf[j][v], win[j][v], a);
+                        acc[v] = ACT ? silu(a) : a;
+                    }
                 }
                 if (t < T) *reinterpret_cast<raw*>(yb + (int64_t)t * hd) = VT::from_f(acc);
 #pragma unroll
@@ -463,6 +521,11 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
     using VT = Vec<Tin, VE>;
     using raw = typename VT::raw;
     const int lane = threadIdx.x & 31, l = lane % LPR;
+    // the weight, shared by every row, into shared memory (16-byte aligned there; the
+    // caller's array need only be 4-byte aligned)
+    __shared__ __align__(16) float ws[D];
+    for (int c = threadIdx.x; c < D; c += kNormWarps * 32) ws[c] = w[c];
+    __syncthreads();
     const int64_t r0w = ((int64_t)blockIdx.x * kNormWarps + (threadIdx.x >> 5)) * RPW;
     if (r0w >= rows) return;
     const int64_t r = r0w + lane / LPR;
@@ -482,8 +545,13 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
             VT::to_f(*reinterpret_cast<const raw*>(x + xr * D + c), xf + a * VE);
             VT::to_f(*reinterpret_cast<const raw*>(z + r * D + c), zf + a * VE);
         }
+        float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < NV * VE; ++e) ss = fmaf(xf[e], xf[e], ss);
+        for (int e = 0; e < NV * VE; e += 2) {
+            const float2 xv = make_float2(xf[e], xf[e + 1]);
+            s2 = fma2(xv, xv, s2);
+        }
+        ss = s2.x + s2.y;
     }
 #pragma unroll
     for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -493,10 +561,15 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
     for (int a = 0; a < NV; ++a) {
         const int c = (a * LPR + l) * VE;
         float out[VE];
+        // channel pairs through packed fp32 (the kernel is bound by instruction issue)
 #pragma unroll
-        for (int e = 0; e < VE; ++e) {
-            const float gate = SILU ? silu(zf[a * VE + e]) : sigmoid(zf[a * VE + e]);
-            out[e] = w[c + e] * (xf[a * VE + e] * inv) * gate;
+        for (int e = 0; e < VE; e += 2) {
+            const float2 zv = make_float2(zf[a * VE + e], zf[a * VE + e + 1]);
+            const float2 gate = SILU ? silu2(zv) : sigmoid2(zv);
+            const float2 xn = mul2(make_float2(xf[a * VE + e], xf[a * VE + e + 1]), make_float2(inv, inv));
+            const float2 o2 = mul2(mul2(*reinterpret_cast<const float2*>(ws + c + e), xn), gate);
+            out[e] = o2.x;
+            out[e + 1] = o2.y;
         }
         *reinterpret_cast<raw*>(y + r * D + c) = VT::from_f(out);
     }
