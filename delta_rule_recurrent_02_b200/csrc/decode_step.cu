@@ -68,35 +68,31 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     if (GATE == kGateScalar) a = expf(a);
     else a = 1.0f;
     __syncthreads();
-    if (PRO) {
-        // k / max(||k||, 1e-12) and scale q / max(||q||, 1e-12)
-        if (tid < 32) {
-            float sk = 0.f, sq = 0.f;
-            for (int i = tid; i < DK; i += 32) {
+    // q . k; with the prologue also ||k||^2 and ||q||^2 of the raw rows: k and q enter
+    // every product linearly, so their factors rk = 1 / max(||k||, 1e-12) and
+    // rq = scale / max(||q||, 1e-12) are applied to the reduced sums below instead of
+    // to the rows (no pass over the rows, no barrier of its own)
+    if (tid < 32) {
+        float x = 0.f, sk = 0.f, sq = 0.f;
+        for (int i = tid; i < DK; i += 32) {
+            x += qs[i] * ks[i];
+            if (PRO) {
                 sk += ks[i] * ks[i];
                 sq += qs[i] * qs[i];
             }
+        }
+        x = warp_sum(x);
+        if (PRO) {
             sk = warp_sum(sk);
             sq = warp_sum(sq);
-            if (tid == 0) {
-                rn_s[0] = 1.f / fmaxf(sqrtf(sk), 1e-12f);
-                rn_s[1] = scale / fmaxf(sqrtf(sq), 1e-12f);
+        }
+        if (tid == 0) {
+            qk_s = x;
+            if (PRO) {
+                rn_s[0] = fminf(rsqrtf(sk), 1e12f);
+                rn_s[1] = scale * fminf(rsqrtf(sq), 1e12f);
             }
         }
-        __syncthreads();
-        const float rk = rn_s[0], rq = rn_s[1];
-        for (int i = tid; i < DK; i += NT) {
-            ks[i] *= rk;
-            qs[i] *= rq;
-        }
-        __syncthreads();
-    }
-
-    if (tid < 32) {
-        float x = 0.f;
-        for (int i = tid; i < DK; i += 32) x += qs[i] * ks[i];
-        x = warp_sum(x);
-        if (tid == 0) qk_s = x;
     }
 
     float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), q4 = p4;
@@ -122,20 +118,29 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         pred.x += x.x; pred.y += x.y; pred.z += x.z; pred.w += x.w;
         qsum.x += y.x; qsum.y += y.y; qsum.z += y.z; qsum.w += y.w;
     }
+    // with the prologue: the unit k's and the scaled unit q's sums (rk, rq are visible
+    // after the barrier above)
+    const float rk = PRO ? rn_s[0] : 1.f, rq = PRO ? rn_s[1] : 1.f;
+    if (PRO) {
+        pred.x *= rk; pred.y *= rk; pred.z *= rk; pred.w *= rk;
+        qsum.x *= rq; qsum.y *= rq; qsum.z *= rq; qsum.w *= rq;
+    }
     float4 dl;
     dl.x = b * (vv.x - pred.x); dl.y = b * (vv.y - pred.y);
     dl.z = b * (vv.z - pred.z); dl.w = b * (vv.w - pred.w);
+    // the state takes (rk k_raw) dl^T: rk rides on dl
+    const float4 dk = PRO ? make_float4(rk * dl.x, rk * dl.y, rk * dl.z, rk * dl.w) : dl;
 
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
         const int r = rs + RS * m;
         const float kr = ks[r];
         float4 x = s[m];
-        x.x += kr * dl.x; x.y += kr * dl.y; x.z += kr * dl.z; x.w += kr * dl.w;
+        x.x += kr * dk.x; x.y += kr * dk.y; x.z += kr * dk.z; x.w += kr * dk.w;
         st_stream_f4(Sh + r * DV + cg * 4, x);
     }
     if (rs == 0) {
-        const float qk = qk_s;
+        const float qk = PRO ? rq * rk * qk_s : qk_s;
         float4 ov;
         ov.x = qsum.x + qk * dl.x; ov.y = qsum.y + qk * dl.y;
         ov.z = qsum.z + qk * dl.z; ov.w = qsum.w + qk * dl.w;
