@@ -95,50 +95,6 @@ struct Vec<float, 2> {
     __device__ static raw from_f(const float* f) { return make_float2(f[0], f[1]); }
 };
 
-// ---- packed fp32 pairs: two IEEE-rounded operations in one instruction, the same
-//      results as the scalar ones in half the issue slots -----------------------------
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {   // a * b + c
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-// The hardware's approximate reciprocal (about 1 ulp; 1 / inf = 0).
-__device__ __forceinline__ float rcp_approx(float x) {
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-// The logistic sigmoid 1 / (1 + e^-x) of a pair, with e^-x = 2^(-x log2 e) on the
-// hardware's approximate exp2 and reciprocal (a few ulp, far inside a bf16
-// rounding); for very negative x the exp2 overflows to inf and the reciprocal gives 0,
-// the right limit.  silu2 is x sigmoid(x).
-__device__ __forceinline__ float2 sigmoid2(float2 x) {
-    constexpr float kNegLog2e = -1.4426950408889634f;
-    const float2 t = mul2(x, make_float2(kNegLog2e, kNegLog2e));
-    const float2 d = add2(make_float2(sm100::ex2_approx(t.x), sm100::ex2_approx(t.y)), make_float2(1.f, 1.f));
-    return make_float2(rcp_approx(d.x), rcp_approx(d.y));
-}
-__device__ __forceinline__ float2 silu2(float2 x) { return mul2(x, sigmoid2(x)); }
-
 // SiLU and the logistic sigmoid through the fast exp and the approximate reciprocal
 // (a few ulp, far inside a bf16 rounding): for very negative x the exp overflows to
 // inf and 1 / inf gives 0, the right limit
@@ -392,8 +348,8 @@ causal_conv1d_tile_kernel(const Tin* __restrict__ x, int64_t ld_x, const float* 
                         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int j = 0; j < K; ++j)
-                            a = fma2(make_float2(wf[j][v], wf[j][v + 1]), make_float2(win[j][v], win[j][v + 1]), a);
-                        if (ACT) a = silu2(a);
+                            a = sm100::fma2(make_float2(wf[j][v], wf[j][v + 1]), make_float2(win[j][v], win[j][v + 1]), a);
+                        if (ACT) a = sm100::silu2(a);
                         acc[v] = a.x;
                         acc[v + 1] = a.y;
                     }
@@ -549,7 +505,7 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
 #pragma unroll
         for (int e = 0; e < NV * VE; e += 2) {
             const float2 xv = make_float2(xf[e], xf[e + 1]);
-            s2 = fma2(xv, xv, s2);
+            s2 = sm100::fma2(xv, xv, s2);
         }
         ss = s2.x + s2.y;
     }
@@ -565,9 +521,9 @@ rms_norm_gated_kernel(const Tin* __restrict__ x, const Tin* __restrict__ z, cons
 #pragma unroll
         for (int e = 0; e < VE; e += 2) {
             const float2 zv = make_float2(zf[a * VE + e], zf[a * VE + e + 1]);
-            const float2 gate = SILU ? silu2(zv) : sigmoid2(zv);
-            const float2 xn = mul2(make_float2(xf[a * VE + e], xf[a * VE + e + 1]), make_float2(inv, inv));
-            const float2 o2 = mul2(mul2(*reinterpret_cast<const float2*>(ws + c + e), xn), gate);
+            const float2 gate = SILU ? sm100::silu2(zv) : sm100::sigmoid2(zv);
+            const float2 xn = sm100::mul2(make_float2(xf[a * VE + e], xf[a * VE + e + 1]), make_float2(inv, inv));
+            const float2 o2 = sm100::mul2(sm100::mul2(*reinterpret_cast<const float2*>(ws + c + e), xn), gate);
             out[e] = o2.x;
             out[e + 1] = o2.y;
         }

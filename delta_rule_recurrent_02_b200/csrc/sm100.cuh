@@ -326,6 +326,58 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(a), "f"(b));
     return r;
 }
+// ---- packed fp32 pairs: two IEEE-rounded operations in one instruction, the same
+//      results as the scalar ones in half the issue slots -----------------------------
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {   // a * b + c
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// The hardware's approximate reciprocal (about 1 ulp; 1 / inf = 0).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+// The logistic sigmoid 1 / (1 + e^-x) of a pair, with e^-x = 2^(-x log2 e) on the
+// hardware's approximate exp2 and reciprocal (a few ulp, far inside a bf16
+// rounding); for very negative x the exp2 overflows to inf and the reciprocal gives 0,
+// the right limit.  silu2 is x sigmoid(x).
+__device__ __forceinline__ float2 sigmoid2(float2 x) {
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 t = mul2(x, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = add2(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.f, 1.f));
+    return make_float2(rcp_approx(d.x), rcp_approx(d.y));
+}
+__device__ __forceinline__ float2 silu2(float2 x) { return mul2(x, sigmoid2(x)); }
+
 // d0 += x a0, d1 += x a1 as one packed fp32 FMA (each half rounded like fmaf).
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float x, float a0, float a1) {
     uint64_t d, a, b, c;
