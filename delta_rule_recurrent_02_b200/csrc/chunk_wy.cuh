@@ -165,7 +165,9 @@ __device__ __forceinline__ void init_group(const Group& x) {
     mbar_init(x.ctl.bar(B_FULL), 1);
     mbar_init(x.ctl.bar(B_MMA), 1);
     *x.ctl.abort = 0;
+    *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 28) = 0u;   // no tile's K, Q preloaded
 }
+
 
 struct Args {
     const CUtensorMap* tm_q;
@@ -196,6 +198,26 @@ struct Args {
     int vl_N = 0;
     float* rq = nullptr;     // with the prologue: the workspace's 1 / ||q_i|| rows
 };
+
+// Thread kStoreTid, at the end of a tile whose stores have read their staging space:
+// the K and Q tiles of the tile that `ticket` names (the group's next) into that
+// space, on B_FULL's next phase, so that they land during this tile's tail.  Returns
+// whether it did (not for the last tile, a packed batch or without a tile counter).
+__device__ __forceinline__ bool preload_next(const Args& ar, const Ctl& ctl, uint32_t sb, unsigned int ticket) {
+    if (!ar.counter || ar.vl || (ar.test_flags & 1)) return false;
+    const int64_t tn = (int64_t)ar.G + ticket;
+    if (tn >= (int64_t)ar.BH * ar.n) return false;
+    const int cn = (int)(tn / ar.BH);
+    const int64_t bhn = tn - (int64_t)cn * ar.BH;
+    const int yk = (int)(key_head(bhn, ar.H, ar.rep) * ar.T + (int64_t)cn * kC);
+    const uint32_t fb = ctl.bar(B_FULL);
+    mbar_arrive_expect_tx(fb, 4 * 8192);
+    tma_load_2d(sb + OFF_KV + 0, ar.tm_k, 0, yk, fb);
+    tma_load_2d(sb + OFF_KV + 16384, ar.tm_k, 64, yk, fb);
+    tma_load_2d(sb + OFF_KV + 8192, ar.tm_q, 0, yk, fb);
+    tma_load_2d(sb + OFF_KV + 24576, ar.tm_q, 64, yk, fb);
+    return true;
+}
 
 // Thread kStoreTid, during a tile: the inputs of the tile that `ticket` names
 // (if any) into L2, so that its loads at the group's next tile hit L2: K, Q
@@ -363,13 +385,16 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
     const unsigned int ticket = tid == kStoreTid && ar.counter ? atomicAdd(ar.counter, 1u) : 0u;
 
     if (tid == 0 && load) {
-        const uint32_t fb = ctl.bar(B_FULL);
-        const int y = (int)t0k;
-        mbar_arrive_expect_tx(fb, 4 * 8192);
-        tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, y, fb);
-        tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, y, fb);
-        tma_load_2d(sb + OFF_KV + 8192, &tm_q, 0, y, fb);
-        tma_load_2d(sb + OFF_KV + 24576, &tm_q, 64, y, fb);
+        // (unless the group's previous tile issued them at its end)
+        if (*reinterpret_cast<volatile const unsigned int*>(x.sm + OFF_BAR + 28) == 0u) {
+            const uint32_t fb = ctl.bar(B_FULL);
+            const int y = (int)t0k;
+            mbar_arrive_expect_tx(fb, 4 * 8192);
+            tma_load_2d(sb + OFF_KV + 0, &tm_k, 0, y, fb);
+            tma_load_2d(sb + OFF_KV + 16384, &tm_k, 64, y, fb);
+            tma_load_2d(sb + OFF_KV + 8192, &tm_q, 0, y, fb);
+            tma_load_2d(sb + OFF_KV + 24576, &tm_q, 64, y, fb);
+        }
         loads = 1;
     }
     if (warp == 2) {
@@ -619,9 +644,10 @@ __device__ __forceinline__ bool wy_tile(const Group& x, const Args& ar, int c, i
         tma_store_2d(&tm_w, 64, (int)(tile * kC), sb + OFF_KV + 8192);
         tma_store_2d(&tm_u, 0, (int)(tile * kD), sb + OFF_KV + 16384);
         bulk_commit_group();
-        // the staging tiles are read: the space is free for the next tile's loads;
+        // the staging tiles are read: the space takes the next tile's K and Q at once;
         // the flag waits until the stores are complete
         bulk_wait_read_all();
+        *reinterpret_cast<volatile unsigned int*>(x.sm + OFF_BAR + 28) = preload_next(ar, ctl, sb, ticket) ? 1u : 0u;
         pending = tile;
         // the first two chunk columns gate the start of every state pass: their flags go up
         // as soon as the stores are complete, not during the group's next tile
